@@ -1,0 +1,217 @@
+"""Plain fp64 oracle of one Switch Transformer layer, forward pass.
+
+TEST INFRASTRUCTURE.  Imported only by the tests, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``; never by the product path.
+
+Sources (web pages on the Switch Transformer; cited by page title and section):
+
+* [ST-note]  "Switch Transformer" reading note (eightmm.github.io), sections
+  "Router", "Expert FFN Layer", "Dense FFN Baseline", "Capacity Factor",
+  "Load-Balancing Loss", "Batch and Sequence Shape".
+* [ST-paper] "Switch Transformers: Scaling to Trillion Parameter Models with
+  Simple and Efficient Sparsity" (paper-graph summary of arXiv 2101.03961),
+  section 3.4: "The mathematics of routing", "The loss formulation", the
+  expert-capacity formula, "The routing mechanics in detail", "The selective
+  precision solution".
+* [ST-explained] "Switch Transformer, explained." (vibeengines), recipe steps 2-5.
+* [LB-card] "Chapter 8 - Attention and Transformers" companion, card 08
+  "Penalize uneven expert traffic".
+
+Every floating-point step runs in float64 on inputs upcast exactly from their
+stored fp32 / bf16 values.  Matrices act on column vectors as [ST-note] writes
+them: z_t = W_r x_t, W_1 in R^{d_ff x d}, W_2 in R^{d x d_ff}; stored row-major
+as W_r [N, d], W1 [N, d_ff, d], W2 [N, d, d_ff].
+
+Readings where the pages are silent or disagree (each also listed in the design doc):
+
+* capacity: C = ceil(capacity_factor * T / N) with the exact rational value of
+  the given double ([ST-note] "Capacity Factor"; [ST-paper] prints a floor
+  variant, [ST-explained] no rounding -- all agree when cf*T/N is an integer).
+* argmax ties go to the lowest expert index (pages silent).
+* positions are 0-based ranks in token order; a token is dropped iff its
+  position >= C ([ST-paper] routing mechanics: cumsum over each expert's column
+  in token order, overflow masked).
+* f_i counts the argmax choices before the capacity cut ([ST-paper] loss
+  formulation, indicator on argmax); aux is returned without the alpha factor.
+* dropped tokens get a zero layer output; no residual is added here.
+* b_2 sits inside the gate: y = g * (W_2 relu(W_1 x + b_1) + b_2)
+  ([ST-note] "Expert FFN Layer" and "Router": y_t = g_t E_{e_t}(x_t)).
+* an empty batch (T = 0) gives no outputs and aux = 0.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+from typing import Callable, Dict, Iterable, Optional
+
+import numpy as np
+
+
+def _f64(a) -> np.ndarray:
+    """Exact upcast of an fp32/bf16 array (numpy or torch, any device) to float64."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# capacity  ([ST-note] "Capacity Factor": C = ceil(T/N * alpha))
+# ---------------------------------------------------------------------------
+def capacity(T: int, N: int, capacity_factor: float) -> int:
+    """Expert capacity ceil(cf * T / N), evaluated exactly on the double cf."""
+    if N <= 0 or T < 0 or not math.isfinite(capacity_factor) or capacity_factor <= 0:
+        raise ValueError("invalid capacity arguments")
+    return math.ceil(Fraction(capacity_factor) * T / N)
+
+
+# ---------------------------------------------------------------------------
+# router  ([ST-paper] 3.4 "The mathematics of routing"; [ST-note] "Router")
+# ---------------------------------------------------------------------------
+def router_logits(x, W_r, b_r=None) -> np.ndarray:
+    """h(x_t) = W_r x_t (+ b_r): logits [T, N] in float64."""
+    z = _f64(x) @ _f64(W_r).T
+    if b_r is not None:
+        z = z + _f64(b_r)[None, :]
+    return z
+
+
+def router_probs(z: np.ndarray) -> np.ndarray:
+    """p_i = exp(h_i) / sum_j exp(h_j) over the N experts (max-shifted)."""
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def top1(p: np.ndarray):
+    """e_t = argmax_i p_{t,i} (lowest index on ties) and gate g_t = p_{t,e_t}."""
+    e = np.argmax(p, axis=1)          # numpy returns the first maximal index
+    g = p[np.arange(p.shape[0]), e]
+    return e.astype(np.int64), g
+
+
+def logit_gap(z: np.ndarray) -> np.ndarray:
+    """Top-1 minus top-2 logit per token (inf when N == 1)."""
+    if z.shape[1] < 2:
+        return np.full(z.shape[0], np.inf)
+    s = np.sort(z, axis=1)
+    return s[:, -1] - s[:, -2]
+
+
+# ---------------------------------------------------------------------------
+# positions and drops ([ST-paper] "The routing mechanics in detail")
+# ---------------------------------------------------------------------------
+def positions(expert_idx: Iterable[int], N: int) -> np.ndarray:
+    """pos_t = number of earlier tokens (in token order) routed to e_t."""
+    seen = [0] * N
+    out = []
+    for e in expert_idx:
+        out.append(seen[int(e)])
+        seen[int(e)] += 1
+    return np.asarray(out, dtype=np.int64)
+
+
+# ---------------------------------------------------------------------------
+# expert FFN ([ST-note] "Expert FFN Layer": E_i(x) = W_2i relu(W_1i x + b_1i) + b_2i)
+# ---------------------------------------------------------------------------
+def expert_ffn(x_rows, W1e, b1e, W2e, b2e) -> np.ndarray:
+    """E(x) for rows of x: relu(x W1^T + b1) W2^T + b2, float64."""
+    h = _f64(x_rows) @ _f64(W1e).T + _f64(b1e)[None, :]
+    h = np.maximum(h, 0.0)
+    return h @ _f64(W2e).T + _f64(b2e)[None, :]
+
+
+# ---------------------------------------------------------------------------
+# load-balancing loss ([ST-paper] "The loss formulation"; [LB-card])
+# ---------------------------------------------------------------------------
+def load_balance_stats(expert_idx: np.ndarray, p: np.ndarray):
+    """f_i = fraction of tokens whose argmax is i; P_i = mean router prob of i."""
+    T, N = p.shape
+    if T == 0:
+        return np.zeros(N), np.zeros(N)
+    counts = np.bincount(expert_idx, minlength=N).astype(np.float64)
+    return counts / T, p.sum(axis=0) / T
+
+
+def aux_loss(f: np.ndarray, P: np.ndarray) -> float:
+    """N * sum_i f_i P_i (the alpha factor is left to the caller)."""
+    f = np.asarray(f, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    return float(len(f) * np.sum(f * P))
+
+
+# ---------------------------------------------------------------------------
+# the whole layer
+# ---------------------------------------------------------------------------
+def switch_forward(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None) -> Dict:
+    """Full forward pass in float64.
+
+    Returns out [T, d] (float64; zero rows for dropped tokens), expert_idx,
+    gate, pos_in_expert, kept, capacity, f, P, aux, probs, logits."""
+    xs = _f64(x)
+    T = xs.shape[0]
+    N = _f64(W_r).shape[0]
+    z = router_logits(xs, W_r, b_r)
+    p = router_probs(z) if T else np.zeros((0, N))
+    e, g = top1(p) if T else (np.zeros(0, np.int64), np.zeros(0))
+    C = capacity(T, N, capacity_factor)
+    pos = positions(e, N)
+    kept = pos < C
+    out = np.zeros((T, xs.shape[1]))
+    for i in range(N):
+        rows = np.nonzero((e == i) & kept)[0]
+        if rows.size == 0:
+            continue
+        u = expert_ffn(xs[rows], W1[i], b1[i], W2[i], b2[i])
+        out[rows] = g[rows, None] * u
+    f, P = load_balance_stats(e, p)
+    aux = aux_loss(f, P) if T else 0.0
+    return {"out": out, "expert_idx": e, "gate": g, "pos_in_expert": pos, "kept": kept,
+            "capacity": C, "f": f, "P": P, "aux": aux, "probs": p, "logits": z}
+
+
+def switch_forward_sampled(x, W_r, capacity_factor: float, sample_tokens,
+                           expert_weights: Callable[[int], Dict], b_r=None,
+                           chunk: int = 4096) -> Dict:
+    """Routing for every token, expert outputs only for ``sample_tokens``.
+
+    ``expert_weights(e)`` returns {"W1","b1","W2","b2"} of expert e, so large
+    layers never hold all expert weights at once.  The router runs over token
+    chunks (rows are independent); positions need every token's choice."""
+    xs = x
+    T = xs.shape[0]
+    N = W_r.shape[0]
+    e_all = np.empty(T, dtype=np.int64)
+    g_all = np.empty(T)
+    psum = np.zeros(N)
+    for s in range(0, T, chunk):
+        z = router_logits(xs[s:s + chunk], W_r, b_r)
+        p = router_probs(z)
+        e, g = top1(p)
+        e_all[s:s + chunk] = e
+        g_all[s:s + chunk] = g
+        psum += p.sum(axis=0)
+    C = capacity(T, N, capacity_factor)
+    pos = positions(e_all, N)
+    kept = pos < C
+    counts = np.bincount(e_all, minlength=N).astype(np.float64)
+    f, P = counts / T, psum / T
+    sample_tokens = np.asarray(sorted(set(int(t) for t in sample_tokens)), dtype=np.int64)
+    out = {}
+    by_expert: Dict[int, list] = {}
+    for t in sample_tokens:
+        if kept[t]:
+            by_expert.setdefault(int(e_all[t]), []).append(int(t))
+        else:
+            out[int(t)] = np.zeros(xs.shape[1])
+    for i, toks in sorted(by_expert.items()):
+        w = expert_weights(i)
+        u = expert_ffn(_f64(xs[toks]), w["W1"], w["b1"], w["W2"], w["b2"])
+        for j, t in enumerate(toks):
+            out[t] = g_all[t] * u[j]
+    return {"out_rows": out, "expert_idx": e_all, "gate": g_all, "pos_in_expert": pos,
+            "kept": kept, "capacity": C, "f": f, "P": P, "aux": aux_loss(f, P)}
+

@@ -1,0 +1,289 @@
+"""Checks that pin the fp64 oracle to facts fixed by the pages and by mathematics.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees.  They
+are run as tests in ``test_oracle_pins.py`` and, with mistakes planted in the
+oracle, in ``test_oracle_mutations.py`` (each planted mistake must trip a pin).
+
+None of the checks retypes the oracle's own formula: they use the pages'
+printed worked example, closed forms, invariants, brute force, or special cases
+that reduce to a library routine (torch float64 linear / relu / softmax / sigmoid).
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import oracle.switch_layer as S
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand_ffn(rng, N, d, d_ff, scale=0.5):
+    W1 = rng.normal(size=(N, d_ff, d)) * scale
+    b1 = rng.normal(size=(N, d_ff)) * 0.1
+    W2 = rng.normal(size=(N, d, d_ff)) * scale
+    b2 = rng.normal(size=(N, d)) * 0.1
+    return W1, b1, W2, b2
+
+
+# ---------------------------------------------------------------------------
+# load-balancing loss: the worked example printed on the "Penalize uneven
+# expert traffic" card (N=4, T=8) and its "check your understanding" case.
+# ---------------------------------------------------------------------------
+def pin_lb_worked_example():
+    g = _gold("lb_card_worked_example.json")
+    bb = g["book_batch"]
+    assert abs(S.aux_loss(bb["f"], bb["P"]) - bb["loss"]) < 1e-12
+    assert abs(S.aux_loss(bb["f"], bb["P"]) / bb["N"] - bb["inner_sum"]) < 1e-12
+    ev = g["even_router_weights"]
+    assert abs(S.aux_loss(ev["f"], ev["P"]) - ev["loss"]) < 1e-12
+
+    # The same batch end to end through router -> softmax -> argmax -> stats.
+    # Eight tokens whose router probabilities have argmax counts (3,2,1,2) and
+    # column means P; with W_r = I and x_t = log p_t, softmax(W_r x_t) = p_t.
+    rows = ([[.60, .20, .05, .15]] * 3 + [[.30, .50, .05, .15]] * 2 +
+            [[.30, .10, .45, .15]] + [[.25, .15, .05, .55]] * 2)
+    order = [5, 0, 7, 2, 6, 1, 4, 3]          # token order must not matter
+    p_rows = np.array(rows)[order]
+    x = np.log(p_rows)
+    rng = np.random.default_rng(1)
+    W1, b1, W2, b2 = _rand_ffn(rng, 4, 4, 3)
+    r = S.switch_forward(x, np.eye(4), W1, b1, W2, b2, capacity_factor=1.0)
+    assert np.allclose(r["probs"], p_rows, rtol=0, atol=1e-15)
+    assert np.array_equal(np.sort(np.bincount(r["expert_idx"], minlength=4)), [1, 2, 2, 3])
+    assert np.allclose(r["f"], bb["f"], rtol=0, atol=0)
+    assert np.allclose(r["P"], bb["P"], rtol=0, atol=1e-15)
+    assert abs(r["aux"] - bb["loss"]) < 1e-12
+
+
+def pin_even_routing_is_one():
+    """Uniform router (W_r = 0): every p_i = 1/N and the loss is exactly 1,
+    whatever the traffic split (card 08: 1 whenever p is uniform)."""
+    g = _gold("lb_card_worked_example.json")
+    rng = np.random.default_rng(2)
+    for N in (1, 2, 3, 7):
+        T, d = 11, 5
+        x = rng.normal(size=(T, d))
+        W1, b1, W2, b2 = _rand_ffn(rng, N, d, 4)
+        r = S.switch_forward(x, np.zeros((N, d)), W1, b1, W2, b2, capacity_factor=1.0)
+        assert abs(r["aux"] - g["even_routing_loss"]) < 1e-12
+        assert np.allclose(r["gate"], 1.0 / N, rtol=0, atol=1e-15)
+        # all logits tie, so the lowest index wins every token
+        assert np.all(r["expert_idx"] == 0)
+
+
+def pin_collapse_tends_to_N():
+    """One expert takes every token with probability -> 1: loss -> N
+    (Switch Transformer, explained: 'climbs toward N').  Logits of 1e3 also
+    need the max-shifted softmax to stay finite."""
+    rng = np.random.default_rng(3)
+    for N in (2, 4, 9):
+        T, d = 13, 6
+        x = rng.normal(size=(T, d))
+        b_r = np.zeros(N)
+        b_r[N - 1] = 1000.0
+        W1, b1, W2, b2 = _rand_ffn(rng, N, d, 3)
+        r = S.switch_forward(x, rng.normal(size=(N, d)), W1, b1, W2, b2,
+                             capacity_factor=float(N), b_r=b_r)
+        assert np.all(r["expert_idx"] == N - 1)
+        assert abs(r["aux"] - N) < 1e-9
+
+
+def pin_not_a_lower_bound():
+    """Card 08: for unrelated f and p the value 1 is not a lower bound.
+    N=3, p rows (.34,.33,.33) and (.01,.50,.49): f=(1/2,1/2,0),
+    P=(.175,.415,.41), loss = 3*(.0875+.2075) = 0.885."""
+    p_rows = np.array([[.34, .33, .33], [.01, .50, .49]])
+    rng = np.random.default_rng(4)
+    W1, b1, W2, b2 = _rand_ffn(rng, 3, 3, 2)
+    r = S.switch_forward(np.log(p_rows), np.eye(3), W1, b1, W2, b2, capacity_factor=1.0)
+    assert list(r["expert_idx"]) == [0, 1]
+    assert abs(r["aux"] - 0.885) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# softmax and argmax
+# ---------------------------------------------------------------------------
+def pin_softmax_rows_and_closed_form():
+    rng = np.random.default_rng(5)
+    z = rng.normal(size=(50, 17)) * 30
+    p = S.router_probs(z)
+    assert np.all(np.abs(p.sum(axis=1) - 1) < 1e-12)
+    assert np.all(p >= 0)
+    # N = 2: p_0 = 1 / (1 + exp(z_1 - z_0)) = sigmoid(z_0 - z_1)
+    x = rng.normal(size=(40, 6))
+    Wr = rng.normal(size=(2, 6)) * 3
+    b_r = np.array([0.3, -0.2])
+    z2 = S.router_logits(x, Wr, b_r)
+    p2 = S.router_probs(z2)
+    lib = torch.sigmoid(torch.from_numpy(x @ Wr[0] - x @ Wr[1] + (b_r[0] - b_r[1]))).numpy()
+    assert np.allclose(p2[:, 0], lib, rtol=0, atol=1e-12)
+    assert np.allclose(p2[:, 1], 1.0 - lib, rtol=0, atol=1e-12)
+
+
+def pin_ties_lowest_index():
+    rng = np.random.default_rng(6)
+    d, N = 5, 4
+    Wr = np.zeros((N, d))
+    Wr[0, 0], Wr[1, 1], Wr[2, 1], Wr[3, 3] = 1.0, 1.0, 1.0, 1.0   # experts 1, 2 equal
+    x = rng.normal(size=(9, d))
+    x[:, 1] = np.abs(x).max() + 1.0        # experts 1 and 2 tie and beat 0 and 3
+    z = S.router_logits(x, Wr)
+    e, g = S.top1(S.router_probs(z))
+    assert np.all(z[:, 1] == z[:, 2]) and np.all(z[:, 1] > z[:, 0]) and np.all(z[:, 1] > z[:, 3])
+    assert np.all(e == 1)
+    # the top-1 choice is the largest logit otherwise
+    x = rng.normal(size=(200, d))
+    z = S.router_logits(x, rng.normal(size=(N, d)))
+    e, g = S.top1(S.router_probs(z))
+    assert np.array_equal(e, torch.from_numpy(z).argmax(dim=1).numpy())
+    assert np.allclose(g, torch.softmax(torch.from_numpy(z), dim=1).max(dim=1).values.numpy(),
+                       rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# capacity, positions, drops
+# ---------------------------------------------------------------------------
+def _smallest_integer_at_least(q: Fraction) -> int:
+    c = 0
+    while c < q:
+        c += 1
+    return c
+
+
+def pin_capacity():
+    # exact search for the smallest integer >= cf*T/N (positive cf)
+    for T in (0, 1, 5, 10, 64, 97):
+        for N in (1, 3, 4, 8):
+            for cf in (0.25, 0.5, 1.0, 1.1, 1.25, 2.0, 3.75):
+                want = _smallest_integer_at_least(Fraction(cf) * T / N)
+                assert S.capacity(T, N, cf) == want, (T, N, cf)
+    assert S.capacity(10, 4, 1.0) == 3       # ceil(2.5): the ceil reading
+    # The five workloads: ceil, floor(T/N)*cf and (T/N)*cf readings coincide,
+    # and the tiny / many-expert descriptions print C=16 and C=32.
+    table = {(64, 4, 1.0): 16, (4096, 64, 1.25): 80, (16384, 128, 1.0): 128,
+             (32768, 64, 2.0): 1024, (65536, 2048, 1.0): 32}
+    for (T, N, cf), C in table.items():
+        assert S.capacity(T, N, cf) == C
+        assert (T // N) * cf == C and T / N * cf == C
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        try:
+            S.capacity(10, 2, bad)
+        except ValueError:
+            continue
+        raise AssertionError("capacity accepted cf=%r" % bad)
+
+
+def pin_positions_bruteforce():
+    """All N**T assignments for T <= 6, N <= 3: the kept tokens of each expert
+    are exactly its first min(count, C) tokens in index order, and positions
+    count up 0,1,2,... along each expert's tokens."""
+    for T in range(0, 7):
+        for N in range(1, 4):
+            for assign in itertools.product(range(N), repeat=T):
+                pos = S.positions(list(assign), N)
+                for i in range(N):
+                    toks = [t for t in range(T) if assign[t] == i]
+                    assert sorted(pos[toks].tolist()) == list(range(len(toks)))
+                    assert all(pos[a] < pos[b] for a, b in zip(toks, toks[1:]))
+                    for C in range(0, T + 2):
+                        kept = [t for t in toks if pos[t] < C]
+                        assert kept == toks[:min(len(toks), C)]
+
+
+def pin_drops():
+    """A capacity cut only removes tokens: dropped rows are exactly zero and
+    kept rows equal the uncut layer's rows.  Large cf (C >= T) drops nothing."""
+    rng = np.random.default_rng(7)
+    T, d, d_ff, N = 40, 6, 5, 3
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(N, d))
+    Wr[0] *= 3
+    W1, b1, W2, b2 = _rand_ffn(rng, N, d, d_ff)
+    full = S.switch_forward(x, Wr, W1, b1, W2, b2, capacity_factor=float(N))
+    assert full["kept"].all() and full["capacity"] >= T
+    cut = S.switch_forward(x, Wr, W1, b1, W2, b2, capacity_factor=0.5)
+    assert (~cut["kept"]).any()
+    assert np.all(cut["out"][~cut["kept"]] == 0.0)
+    assert np.array_equal(cut["out"][cut["kept"]], full["out"][cut["kept"]])
+    assert np.array_equal(cut["expert_idx"], full["expert_idx"])
+    # f counts argmax choices before the cut: it still sums to one
+    assert abs(cut["f"].sum() - 1.0) < 1e-15
+    assert np.array_equal(cut["f"], full["f"]) and np.array_equal(cut["P"], full["P"])
+
+
+# ---------------------------------------------------------------------------
+# expert FFN and gate, via special cases that reduce to library routines
+# ---------------------------------------------------------------------------
+def _torch_ffn(x, W1, b1, W2, b2):
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    return F.linear(F.relu(F.linear(t(x), t(W1), t(b1))), t(W2), t(b2)).numpy()
+
+
+def pin_single_expert_is_dense_ffn():
+    """N = 1: p = 1, C = ceil(cf*T) >= T for cf >= 1: the layer is the dense FFN
+    W_2 relu(W_1 x + b_1) + b_2 of the "Dense FFN Baseline" section."""
+    rng = np.random.default_rng(8)
+    for T, d, d_ff in ((23, 7, 9), (17, 8, 8)):      # square case: W_2 vs W_2^T
+        x = rng.normal(size=(T, d))
+        W1, b1, W2, b2 = _rand_ffn(rng, 1, d, d_ff)
+        r = S.switch_forward(x, rng.normal(size=(1, d)), W1, b1, W2, b2, capacity_factor=1.0)
+        ref = _torch_ffn(x, W1[0], b1[0], W2[0], b2[0])
+        assert np.all(r["gate"] == 1.0) and r["kept"].all()
+        assert np.allclose(r["out"], ref, rtol=1e-13, atol=1e-13)
+
+
+def pin_identical_experts_scale_by_gate():
+    """All experts equal to one FFN and no drops: y_t = max_i softmax(z_t)_i * FFN(x_t)
+    (y_t = g_t E_{e_t}(x_t) with b_2 inside E)."""
+    rng = np.random.default_rng(9)
+    T, d, d_ff, N = 31, 6, 8, 5
+    x = rng.normal(size=(T, d))
+    W1, b1, W2, b2 = _rand_ffn(rng, 1, d, d_ff)
+    rep = lambda a: np.repeat(a, N, axis=0)
+    Wr = rng.normal(size=(N, d))
+    b_r = rng.normal(size=N)
+    r = S.switch_forward(x, Wr, rep(W1), rep(b1), rep(W2), rep(b2),
+                         capacity_factor=float(N), b_r=b_r)
+    z = torch.from_numpy(x) @ torch.from_numpy(Wr).T + torch.from_numpy(b_r)
+    g = torch.softmax(z, dim=1).max(dim=1).values.numpy()
+    ref = g[:, None] * _torch_ffn(x, W1[0], b1[0], W2[0], b2[0])
+    assert np.allclose(r["out"], ref, rtol=1e-13, atol=1e-13)
+
+
+def pin_sampled_matches_full():
+    rng = np.random.default_rng(10)
+    T, d, d_ff, N = 300, 8, 6, 7
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(N, d))
+    W1, b1, W2, b2 = _rand_ffn(rng, N, d, d_ff)
+    full = S.switch_forward(x, Wr, W1, b1, W2, b2, capacity_factor=1.0)
+    samp = rng.choice(T, size=60, replace=False)
+    part = S.switch_forward_sampled(
+        x, Wr, 1.0, samp, lambda e: {"W1": W1[e], "b1": b1[e], "W2": W2[e], "b2": b2[e]},
+        chunk=64)
+    for k in ("expert_idx", "pos_in_expert", "kept"):
+        assert np.array_equal(full[k], part[k])
+    assert np.allclose(full["gate"], part["gate"], rtol=0, atol=1e-15)
+    assert abs(full["aux"] - part["aux"]) < 1e-12
+    for t in samp:
+        assert np.allclose(part["out_rows"][int(t)], full["out"][t], rtol=1e-13, atol=1e-13)
+
+
+ALL_PINS = [
+    pin_lb_worked_example, pin_even_routing_is_one, pin_collapse_tends_to_N,
+    pin_not_a_lower_bound, pin_softmax_rows_and_closed_form, pin_ties_lowest_index,
+    pin_capacity, pin_positions_bruteforce, pin_drops, pin_single_expert_is_dense_ffn,
+    pin_identical_experts_scale_by_gate, pin_sampled_matches_full,
+]

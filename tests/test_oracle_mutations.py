@@ -1,0 +1,109 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins
+catch every one of them.  A pin set that lets a planted mistake through would
+not be evidence that the oracle is right."""
+import numpy as np
+import pytest
+
+import oracle.switch_layer as S
+import oracle_pins as P
+
+
+def _top1_highest_tie(p):
+    e = p.shape[1] - 1 - np.argmax(p[:, ::-1], axis=1)
+    return e.astype(np.int64), p[np.arange(p.shape[0]), e]
+
+
+def _positions_one_based(expert_idx, N):
+    return _orig_positions(expert_idx, N) + 1
+
+
+def _ffn_no_relu(x_rows, W1e, b1e, W2e, b2e):
+    h = S._f64(x_rows) @ S._f64(W1e).T + S._f64(b1e)[None, :]
+    return h @ S._f64(W2e).T + S._f64(b2e)[None, :]
+
+
+def _ffn_transposed_w2(x_rows, W1e, b1e, W2e, b2e):
+    h = np.maximum(S._f64(x_rows) @ S._f64(W1e).T + S._f64(b1e)[None, :], 0.0)
+    W2 = S._f64(W2e)
+    W2 = W2.T if W2.shape[0] == W2.shape[1] else W2
+    return h @ W2.T + S._f64(b2e)[None, :]
+
+
+def _ffn_no_b2(x_rows, W1e, b1e, W2e, b2e):
+    h = np.maximum(S._f64(x_rows) @ S._f64(W1e).T + S._f64(b1e)[None, :], 0.0)
+    return h @ S._f64(W2e).T
+
+
+def _aux_no_N(f, P_):
+    return float(np.sum(np.asarray(f) * np.asarray(P_)))
+
+
+def _probs_no_shift(z):
+    with np.errstate(over="ignore", invalid="ignore"):
+        e = np.exp(z)
+        return e / e.sum(axis=1, keepdims=True)
+
+
+def _capacity_floor(T, N, cf):
+    import math
+    from fractions import Fraction
+    if N <= 0 or T < 0 or not math.isfinite(cf) or cf <= 0:
+        raise ValueError
+    return math.floor(Fraction(cf) * T / N)
+
+
+def _stats_after_cut(expert_idx, p):
+    T, N = p.shape
+    # mistake: counts only the first T//2 tokens (as if capacity applied to f)
+    counts = np.bincount(expert_idx[: max(1, T // 2)], minlength=N).astype(np.float64)
+    return counts / T, p.sum(axis=0) / T
+
+
+def _logits_sign(x, W_r, b_r=None):
+    z = -(S._f64(x) @ S._f64(W_r).T)
+    if b_r is not None:
+        z = z + S._f64(b_r)[None, :]
+    return z
+
+
+def _gate_is_one(p):
+    e = np.argmax(p, axis=1)
+    return e.astype(np.int64), np.ones(p.shape[0])
+
+
+MUTATIONS = {
+    "ties_to_highest": ("top1", _top1_highest_tie),
+    "positions_one_based": ("positions", _positions_one_based),
+    "no_relu": ("expert_ffn", _ffn_no_relu),
+    "w2_transposed": ("expert_ffn", _ffn_transposed_w2),
+    "no_b2": ("expert_ffn", _ffn_no_b2),
+    "aux_without_N": ("aux_loss", _aux_no_N),
+    "softmax_unshifted": ("router_probs", _probs_no_shift),
+    "capacity_floor": ("capacity", _capacity_floor),
+    "f_after_cut": ("load_balance_stats", _stats_after_cut),
+    "logit_sign": ("router_logits", _logits_sign),
+    "gate_one": ("top1", _gate_is_one),
+}
+
+
+def _orig_positions(expert_idx, N):
+    seen = [0] * N
+    out = []
+    for e in expert_idx:
+        out.append(seen[int(e)])
+        seen[int(e)] += 1
+    return np.asarray(out, dtype=np.int64)
+
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(S, attr, fn)
+    failed = []
+    for pin in P.ALL_PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError, FloatingPointError):
+            failed.append(pin.__name__)
+    assert failed, "planted mistake %r passed every pin" % name
