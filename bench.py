@@ -1,0 +1,423 @@
+"""Benchmark: Switch-layer forward tokens/s on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one full forward pass of the layer (router logits, softmax/argmax,
+dispatch scan + aux loss, gather, expert GEMM1, expert GEMM2 + combine) over
+one batch of seeded synthetic tokens already resident in HBM.  Default
+workload: the Switch-Base-like layer (T=4096 tokens, d=768, d_ff=3072, N=64
+experts, capacity factor 1.25, bf16 with an fp32 router).
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the layer on its own
+batch (independent problems, weak scaling, no collective on the data path);
+the timed region is bracketed by barriers and the max over ranks is reported.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), each step
+a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "base_T4096_d768_N64"
+METRIC = "Switch-layer fwd tokens/sec on 1 B200; expert-GEMM % of bf16 tensor peak"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(ws, v: float) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _traffic_entry(kernel: str, workload: str):
+    """Per-launch DRAM bytes of ``kernel`` from a committed ncu capture, or None
+    if absent or if the kernel's source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel, {}).get(workload)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if h != ent.get("source_sha256"):
+        return None
+    return float(ent["dram_bytes_per_launch"])
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import sparse_mixture_experts_argmax_b200 as swl
+
+    ws_n, rank, local = _dist_init()
+    dev = torch.device("cuda", local)
+    spec = synth.WORKLOADS[args.workload]
+    T, d, d_ff, N, cf = spec.T, spec.d, spec.d_ff, spec.N, spec.cf
+    redraws = synth.load_gap_redraws(spec.name) if rank == 0 else {}
+    inputs = synth.make_layer_inputs(spec, seed=rank, device=dev, redraws=redraws)
+    act = inputs["x"].dtype
+    work = swl.alloc_workspace(T, d, d_ff, N, act, cf, device=dev)
+    outs = swl.alloc_outputs(T, d, act, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    S = swl.SWL_NUM_STAGES
+
+    def step(events=None):
+        swl.switch_layer_forward(inputs["x"], inputs["W_r"], inputs["W1"], inputs["b1"],
+                                 inputs["W2"], inputs["b2"], cf, outs["out"],
+                                 outs["expert_idx"], outs["gate"], outs["pos_in_expert"],
+                                 outs["aux_loss"], b_r=inputs["b_r"], workspace=work,
+                                 stream=stream, stage_events=events)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if swl.switch_layer_device_status(work, stream) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    # ---- timed region: K steps, L2 flushed between steps (outside the events)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)]
+          for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)        # create the CUDA events before timing
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    _barrier(ws_n)
+    torch.cuda.synchronize()
+    launches0 = swl.switch_layer_launch_count()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        step(ev[k])
+    torch.cuda.synchronize()
+    launches = swl.switch_layer_launch_count() - launches0
+    _barrier(ws_n)
+    clk = clocks.stop()
+    stage_ms = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(S)]
+                         for k in range(args.steps)])
+    step_ms = stage_ms.sum(axis=1)
+    total_ms = _max_over_ranks(ws_n, float(step_ms.sum()))
+    ms_per_step = total_ms / args.steps
+    value = ws_n * T * args.steps / (total_ms / 1e3)
+    if swl.switch_layer_device_status(work, stream) != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+
+    # ---- end to end through the host-I/O entry point (pinned host x and outputs)
+    work_h = swl.alloc_workspace(T, d, d_ff, N, act, cf, host_io=True, device=dev)
+    xh = inputs["x"].cpu().pin_memory()
+    oh = [torch.empty((T, d), dtype=act).pin_memory(),
+          torch.empty(T, dtype=torch.int32).pin_memory(),
+          torch.empty(T, dtype=torch.float32).pin_memory(),
+          torch.empty(T, dtype=torch.int32).pin_memory(),
+          torch.empty(1, dtype=torch.float32).pin_memory()]
+
+    def step_e2e():
+        swl.switch_layer_forward_host_io(xh, inputs["W_r"], inputs["W1"], inputs["b1"],
+                                         inputs["W2"], inputs["b2"], cf, *oh,
+                                         b_r=inputs["b_r"], workspace=work_h, stream=stream)
+
+    for _ in range(args.warmup):
+        step_e2e()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    _barrier(ws_n)
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step_e2e()
+        b.record(stream)
+        b.synchronize()             # the step's result is on the host
+        e2e_ms.append(a.elapsed_time(b))
+    _barrier(ws_n)
+    e2e_total = _max_over_ranks(ws_n, float(sum(e2e_ms)))
+    e2e_value = ws_n * T * args.steps / (e2e_total / 1e3)
+    elem = 2 if act == torch.bfloat16 else 4
+    h2d = T * d * elem
+    d2h = T * d * elem + 3 * 4 * T + 4
+
+    # ---- roofline of the dominant kernel (algorithmic bytes / launch duration)
+    e_idx = outs["expert_idx"].long()
+    kept = outs["pos_in_expert"].long() < swl.switch_layer_capacity(T, N, cf)
+    counts = torch.bincount(e_idx, minlength=N)
+    touched = int((counts > 0).sum())
+    K_kept = int(kept.sum())
+    avg_stage = stage_ms.mean(axis=0)
+    names = [swl.switch_layer_stage_name(i) for i in range(S)]
+    # algorithmic bytes per launch of each expert GEMM (bf16)
+    w_bytes = touched * (d * d_ff * elem)
+    gemm_bytes = {
+        "expert_gemm1": w_bytes + touched * d_ff * elem + K_kept * (d + d_ff) * elem,
+        "expert_gemm2": w_bytes + touched * d * elem + K_kept * (d_ff + d) * elem + K_kept * 8,
+    }
+    dom = max(("expert_gemm1", "expert_gemm2"), key=lambda n: avg_stage[names.index(n)])
+    dom_s = avg_stage[names.index(dom)] / 1e3
+    peaks = _peaks()
+    achieved = gemm_bytes[dom] / dom_s / 1e9
+    traffic = _traffic_entry(dom, spec.name)
+    gemm_s = (avg_stage[names.index("expert_gemm1")] + avg_stage[names.index("expert_gemm2")]) / 1e3
+    gemm_flops = 4.0 * K_kept * d * d_ff
+    tensor_frac = gemm_flops / gemm_s / (peaks["bf16_tflops"] * 1e12)
+
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": ws_n,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if act == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded; x ~ N(0,1), T5 truncated-normal init s=0.1)",
+        "config": {
+            "workload": spec.name, "T": T, "d": d, "d_ff": d_ff, "N": N,
+            "capacity_factor": cf, "capacity": swl.switch_layer_capacity(T, N, cf),
+            "router": "fp32", "parallelism": "dp%d (independent batches)" % ws_n,
+            "l2": "flushed between timed steps (256 MiB write, outside the step events); "
+                  "expert weights %.0f MB > 126 MB L2" % (2 * N * d * d_ff * elem / 1e6),
+        },
+        "stages_us": {n: round(float(v) * 1e3, 2) for n, v in zip(names, avg_stage)},
+        "roofline": {
+            "kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "algorithmic_bytes": gemm_bytes[dom], "peak_source": peaks["source"] + " (burst copy)",
+        },
+        "expert_gemm_tensor_frac": {
+            "value": tensor_frac, "flops_per_step": gemm_flops,
+            "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"],
+            "note": "GEMM1+GEMM2 kept-token FLOPs / their time / dense bf16 peak; the stage is "
+                    "bound by streaming expert weights, see roofline",
+        },
+        "routing": {"experts_touched": touched, "kept_tokens": K_kept,
+                    "dropped_tokens": T - K_kept, "max_load": int(counts.max()),
+                    "aux_loss": float(outs["aux_loss"][0])},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_step(spec, inputs, n_tok: int):
+    import oracle
+    x = inputs["x"][:n_tok]
+    oracle.switch_forward(x, inputs["W_r"], inputs["W1"], inputs["b1"], inputs["W2"],
+                          inputs["b2"], spec.cf, b_r=inputs["b_r"])
+
+
+def cpu_baseline(spec, budget_s: float = 20.0, steps: int = None):
+    """The fp64 oracle on the host cores: full-batch forwards until ~budget_s."""
+    inputs = synth.make_layer_inputs(spec, 0, device="cpu",
+                                     redraws=synth.load_gap_redraws(spec.name))
+    t0 = time.perf_counter()
+    _oracle_step(spec, inputs, spec.T)
+    dt = [time.perf_counter() - t0]
+    while sum(dt) < budget_s * 0.5 and len(dt) < 50:
+        t0 = time.perf_counter()
+        _oracle_step(spec, inputs, spec.T)
+        dt.append(time.perf_counter() - t0)
+    return {"value": spec.T * len(dt) / sum(dt), "unit": "tokens/s", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": "%d full-batch fp64 oracle forwards of %s (T=%d), %.1f s wall" % (
+                len(dt), spec.name, spec.T, sum(dt))}
+
+
+def run_reference(args):
+    ws_n = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    spec = synth.WORKLOADS[args.workload]
+    inputs = synth.make_layer_inputs(spec, 0, device="cpu",
+                                     redraws=synth.load_gap_redraws(spec.name))
+    # calibrate a token sample so warm-up + timed steps stay within ~budget seconds
+    budget = args.cpu_budget * 6
+    t0 = time.perf_counter()
+    _oracle_step(spec, inputs, spec.T)
+    t_full = time.perf_counter() - t0
+    frac = min(1.0, budget / max(1e-9, (args.steps + args.warmup) * t_full))
+    n_tok = max(128, int(spec.T * frac) // 128 * 128)
+    for _ in range(args.warmup):
+        _oracle_step(spec, inputs, n_tok)
+    dts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_step(spec, inputs, n_tok)
+        dts.append(time.perf_counter() - t0)
+    total = sum(dts)
+    v = n_tok * args.steps / total
+    cores = _blas_threads()
+    sample = ("each step: fp64 oracle forward on the first %d of %d tokens of %s "
+              "(same weights, capacity from the formula)" % (n_tok, spec.T, spec.name))
+    res = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": spec.name, "T": spec.T, "d": spec.d, "d_ff": spec.d_ff,
+                   "N": spec.N, "capacity_factor": spec.cf},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * switch_layer.h -- C ABI of a B200 (sm_100a) implementation of the forward
+ * pass of one Switch Transformer expert layer.
+ *
+ * The layer (sources: "Switch Transformer" reading note, eightmm.github.io,
+ * sections "Router", "Expert FFN Layer", "Capacity Factor", "Load-Balancing
+ * Loss"; paper-graph summary of arXiv 2101.03961 "Switch Transformers: Scaling
+ * to Trillion Parameter Models with Simple and Efficient Sparsity", section 3.4:
+ * "The mathematics of routing", "The loss formulation", the expert-capacity
+ * formula, "The routing mechanics in detail", "The selective precision
+ * solution"; "Switch Transformer, explained." recipe steps 2-5):
+ *
+ *   z_t   = W_r x_t + b_r                     router logits, fp32
+ *   p_t   = softmax(z_t)                      fp32
+ *   e_t   = argmax_i p_t,i                    lowest index on ties
+ *   g_t   = p_t,e_t                           gate
+ *   C     = ceil(capacity_factor * T / N)     expert capacity
+ *   pos_t = #{ s < t : e_s = e_t }            0-based position in token order
+ *   kept  = pos_t < C                         overflow tokens are dropped
+ *   out_t = kept ? g_t * (W2[e] relu(W1[e] x_t + b1[e]) + b2[e]) : 0
+ *   aux   = N * sum_i f_i * P_i,  f_i = #{t : e_t = i} / T,  P_i = mean_t p_t,i
+ *
+ * No residual is added (a dropped token's layer output is zero; the caller's
+ * residual connection carries it).  aux is returned without the alpha factor.
+ *
+ * Conventions for every entry point:
+ *  - Memory: every tensor pointer is a DEVICE pointer owned by the caller
+ *    (except the *_host arguments of switch_layer_forward_host_io, which are
+ *    host pointers, ideally pinned).  The library allocates nothing and keeps no
+ *    state between calls besides a launch counter.
+ *  - Layouts: contiguous row-major.  x [T,d]; W_r [N,d] fp32; b_r [N] fp32;
+ *    W1 [N,d_ff,d]; b1 [N,d_ff]; W2 [N,d,d_ff]; b2 [N,d]; out [T,d];
+ *    expert_idx, pos_in_expert [T] int32; gate [T] fp32; aux_loss [1] fp32.
+ *    x, W1, b1, W2, b2 and out share the activation dtype (SWL_F32 or SWL_BF16).
+ *  - Asynchrony: calls enqueue work on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and return; outputs are valid once the stream has
+ *    executed the work.  Device-side failures are read with
+ *    switch_layer_device_status.
+ *  - Errors: arguments are validated on the host before anything is enqueued;
+ *    an invalid call returns a non-zero swl_status and enqueues nothing.
+ *    Nothing traps or aborts.
+ *  - Thread safety: calls may be made from several host threads; two calls that
+ *    share a workspace must not overlap on the GPU.
+ */
+#ifndef SWITCH_LAYER_H
+#define SWITCH_LAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SWL_ABI_VERSION 1
+
+typedef enum swl_status {
+  SWL_OK = 0,
+  SWL_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad dtype or capacity factor */
+  SWL_ERR_UNSUPPORTED = 2,  /* valid but not handled: bf16 with d or d_ff not a multiple of 8,
+                               misaligned pointer, sizes beyond int32 indexing */
+  SWL_ERR_WORKSPACE = 3,    /* workspace smaller than switch_layer_workspace_size() */
+  SWL_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, event) */
+  SWL_ERR_DEVICE = 5        /* a kernel reported a failure (see switch_layer_device_status) */
+} swl_status;
+
+typedef enum swl_dtype { SWL_F32 = 0, SWL_BF16 = 1 } swl_dtype;
+
+/* Workspace flag: also reserve device staging buffers for switch_layer_forward_host_io. */
+#define SWL_WS_HOST_IO 1
+
+/* Number of timed stages and their order (see switch_layer_forward_timed):
+ * 0 router logits, 1 router softmax/argmax/rank, 2 dispatch scan + aux loss,
+ * 3 dispatch gather, 4 expert GEMM1 (+bias, ReLU), 5 expert GEMM2 (+bias, gate, combine). */
+#define SWL_NUM_STAGES 6
+
+/* Expert capacity C = ceil(capacity_factor * T / N) ("Capacity Factor" section
+ * of the reading note), evaluated exactly on the binary value of the double
+ * capacity_factor.  Returns -1 for T < 0, N <= 0 or a capacity factor that is
+ * not finite and positive; saturates at INT64_MAX. */
+int64_t switch_layer_capacity(int64_t T, int64_t N, double capacity_factor);
+
+/* Device workspace bytes needed by a forward call of this shape (flags: 0 or
+ * SWL_WS_HOST_IO).  The workspace must be 256-byte aligned; its contents need
+ * no initialisation.  Returns SWL_ERR_INVALID_ARG / SWL_ERR_UNSUPPORTED for
+ * shapes the forward call would reject. */
+swl_status switch_layer_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                       double capacity_factor, int flags, size_t* bytes);
+
+/* Forward pass of the Switch layer (formulas above).
+ *   T, d, d_ff, N   tokens, model width, expert FFN width, experts (T = 0 is an
+ *                   empty batch: nothing is written except *aux_loss = 0)
+ *   dtype           SWL_F32 or SWL_BF16: dtype of x, W1, b1, W2, b2, out
+ *   x ... b2        inputs (layouts above); W_r and b_r are always fp32
+ *   capacity_factor > 0, finite
+ *   out             [T,d] layer output (zero rows for dropped tokens)
+ *   expert_idx      [T] e_t
+ *   gate            [T] g_t = p_t,e_t (fp32)
+ *   pos_in_expert   [T] pos_t; the token was dropped iff pos_t >= C
+ *   aux_loss        [1] N * sum_i f_i P_i (f before the capacity cut)
+ *   b_r             [N] router-logit bias or NULL for none
+ *   workspace       device scratch of workspace_bytes >= switch_layer_workspace_size()
+ *   stream          cudaStream_t to enqueue on
+ * bf16 additionally requires d % 8 == 0, d_ff % 8 == 0 and 16-byte aligned x,
+ * W1, W2 and out (TMA rows). */
+swl_status switch_layer_forward(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                const void* x, const float* W_r, const void* W1, const void* b1,
+                                const void* W2, const void* b2, double capacity_factor,
+                                void* out, int32_t* expert_idx, float* gate,
+                                int32_t* pos_in_expert, float* aux_loss, const float* b_r,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* As switch_layer_forward, and records cudaEvent_t stage_events[k] on `stream`
+ * before stage 0 (k = 0) and after stage k-1 (k = 1..SWL_NUM_STAGES): an array
+ * of SWL_NUM_STAGES + 1 events created by the caller (timing enabled). */
+swl_status switch_layer_forward_timed(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                      const void* x, const float* W_r, const void* W1,
+                                      const void* b1, const void* W2, const void* b2,
+                                      double capacity_factor, void* out, int32_t* expert_idx,
+                                      float* gate, int32_t* pos_in_expert, float* aux_loss,
+                                      const float* b_r, void* workspace, size_t workspace_bytes,
+                                      void* stream, void* const* stage_events);
+
+/* End-to-end variant with HOST input and outputs: copies x_host to the device,
+ * runs the forward pass, and copies out, expert_idx, gate, pos_in_expert and
+ * aux_loss back into the *_host buffers, all enqueued on `stream` (the caller
+ * synchronises the stream before reading them).  Weights stay device pointers.
+ * The workspace must be sized with SWL_WS_HOST_IO; it holds the device copies. */
+swl_status switch_layer_forward_host_io(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                        const void* x_host, const float* W_r, const void* W1,
+                                        const void* b1, const void* W2, const void* b2,
+                                        double capacity_factor, void* out_host,
+                                        int32_t* expert_idx_host, float* gate_host,
+                                        int32_t* pos_in_expert_host, float* aux_loss_host,
+                                        const float* b_r, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device status of the last forward call
+ * that used `workspace`: SWL_OK, or SWL_ERR_DEVICE if a kernel reported a
+ * failure (a bounded pipeline wait expired, or non-finite router logits).
+ * SWL_ERR_CUDA if the synchronisation itself failed. */
+swl_status switch_layer_device_status(const void* workspace, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* switch_layer_status_string(swl_status status);
+
+/* Name of timed stage k (0 <= k < SWL_NUM_STAGES), or NULL. */
+const char* switch_layer_stage_name(int k);
+
+/* Number of kernel launches this library has issued since it was loaded. */
+uint64_t switch_layer_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWITCH_LAYER_H */

@@ -1,0 +1,266 @@
+"""Python binding of libswitchlayer.so, the sm_100a Switch-layer forward pass.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory (tensors) and the current stream.
+There is no fallback: if the shared library is missing or cannot be loaded,
+every call raises.
+
+The C entry points are exposed under their C names (``switch_layer_forward``,
+``switch_layer_capacity`` ...); ``forward`` is a convenience wrapper that
+allocates the outputs and the workspace with torch and calls
+``switch_layer_forward``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libswitchlayer.so")
+
+SWL_F32, SWL_BF16 = 0, 1
+SWL_WS_HOST_IO = 1
+SWL_NUM_STAGES = 6
+STATUS = {0: "SWL_OK", 1: "SWL_ERR_INVALID_ARG", 2: "SWL_ERR_UNSUPPORTED",
+          3: "SWL_ERR_WORKSPACE", 4: "SWL_ERR_CUDA", 5: "SWL_ERR_DEVICE"}
+
+# Every symbol declared in include/switch_layer.h.
+EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer_forward",
+           "switch_layer_forward_timed", "switch_layer_forward_host_io",
+           "switch_layer_device_status", "switch_layer_status_string",
+           "switch_layer_stage_name", "switch_layer_launch_count")
+
+
+class SwitchLayerError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__("%s (%s)%s" % (STATUS.get(status, "status %d" % status),
+                                        _status_string(status),
+                                        (": " + what) if what else ""))
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_i64, _i32, _dbl, _vp, _sz = (ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
+                              ctypes.c_size_t)
+_FWD_ARGS = [_i64, _i64, _i64, _i64, _i32,            # T, d, d_ff, N, dtype
+             _vp, _vp, _vp, _vp, _vp, _vp, _dbl,       # x, W_r, W1, b1, W2, b2, cf
+             _vp, _vp, _vp, _vp, _vp,                  # out, expert_idx, gate, pos, aux
+             _vp, _vp, _sz, _vp]                       # b_r, workspace, bytes, stream
+
+
+def lib() -> ctypes.CDLL:
+    """Load libswitchlayer.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libswitchlayer.so is missing: build it with "
+                           "`python -m sparse_mixture_experts_argmax_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.switch_layer_capacity.restype = _i64
+    L.switch_layer_capacity.argtypes = [_i64, _i64, _dbl]
+    L.switch_layer_workspace_size.restype = _i32
+    L.switch_layer_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i32, _dbl, _i32,
+                                              ctypes.POINTER(_sz)]
+    L.switch_layer_forward.restype = _i32
+    L.switch_layer_forward.argtypes = _FWD_ARGS
+    L.switch_layer_forward_timed.restype = _i32
+    L.switch_layer_forward_timed.argtypes = _FWD_ARGS + [ctypes.POINTER(_vp)]
+    L.switch_layer_forward_host_io.restype = _i32
+    L.switch_layer_forward_host_io.argtypes = _FWD_ARGS
+    L.switch_layer_device_status.restype = _i32
+    L.switch_layer_device_status.argtypes = [_vp, _vp]
+    L.switch_layer_status_string.restype = ctypes.c_char_p
+    L.switch_layer_status_string.argtypes = [_i32]
+    L.switch_layer_stage_name.restype = ctypes.c_char_p
+    L.switch_layer_stage_name.argtypes = [_i32]
+    L.switch_layer_launch_count.restype = ctypes.c_uint64
+    L.switch_layer_launch_count.argtypes = []
+    _lib = L
+    return L
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().switch_layer_status_string(status).decode()
+    except Exception:  # pragma: no cover - only while reporting another failure
+        return "?"
+
+
+def _check(status: int, what: str = "") -> None:
+    if status != 0:
+        raise SwitchLayerError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return SWL_F32
+    if dt == torch.bfloat16:
+        return SWL_BF16
+    raise TypeError("activation dtype must be float32 or bfloat16, got %s" % dt)
+
+
+# ---------------------------------------------------------------------------
+# C entry points, same names
+# ---------------------------------------------------------------------------
+def switch_layer_capacity(T: int, N: int, capacity_factor: float) -> int:
+    return int(lib().switch_layer_capacity(T, N, capacity_factor))
+
+
+def switch_layer_workspace_size(T, d, d_ff, N, dtype: int, capacity_factor: float,
+                                flags: int = 0) -> int:
+    n = _sz(0)
+    _check(lib().switch_layer_workspace_size(T, d, d_ff, N, dtype, capacity_factor, flags,
+                                             ctypes.byref(n)), "workspace_size")
+    return int(n.value)
+
+
+def _shape_of(x, W1, W_r):
+    T, d = x.shape
+    N, d_ff, d2 = W1.shape
+    if d2 != d or tuple(W_r.shape) != (N, d):
+        raise ValueError("shape mismatch: x %s, W_r %s, W1 %s" % (tuple(x.shape),
+                                                                  tuple(W_r.shape),
+                                                                  tuple(W1.shape)))
+    return T, d, d_ff, N
+
+
+def _require(t: torch.Tensor, name: str, dtype=None, device="cuda"):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if device == "cuda" and not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if device == "cpu" and t.is_cuda:
+        raise ValueError("%s must be a host tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def switch_layer_forward(x, W_r, W1, b1, W2, b2, capacity_factor, out, expert_idx, gate,
+                         pos_in_expert, aux_loss, b_r=None, workspace=None, stream=None,
+                         stage_events: Optional[Sequence] = None) -> None:
+    """Enqueue one forward pass (all tensors on the GPU; see include/switch_layer.h)."""
+    T, d, d_ff, N = _shape_of(x, W1, W_r)
+    act = x.dtype
+    for t, n in ((x, "x"), (W1, "W1"), (b1, "b1"), (W2, "W2"), (b2, "b2"), (out, "out")):
+        _require(t, n, act)
+    _require(W_r, "W_r", torch.float32)
+    if b_r is not None:
+        _require(b_r, "b_r", torch.float32)
+    _require(expert_idx, "expert_idx", torch.int32)
+    _require(pos_in_expert, "pos_in_expert", torch.int32)
+    _require(gate, "gate", torch.float32)
+    _require(aux_loss, "aux_loss", torch.float32)
+    _require(workspace, "workspace", torch.uint8)
+    args = (T, d, d_ff, N, dtype_code(act), _ptr(x), _ptr(W_r), _ptr(W1), _ptr(b1), _ptr(W2),
+            _ptr(b2), float(capacity_factor), _ptr(out), _ptr(expert_idx), _ptr(gate),
+            _ptr(pos_in_expert), _ptr(aux_loss), _ptr(b_r), _ptr(workspace),
+            workspace.numel(), _stream_handle(stream))
+    if stage_events is None:
+        _check(lib().switch_layer_forward(*args), "forward")
+    else:
+        if len(stage_events) != SWL_NUM_STAGES + 1:
+            raise ValueError("need %d stage events" % (SWL_NUM_STAGES + 1))
+        for e in stage_events:          # torch creates the CUDA event on first record
+            if not e.cuda_event:
+                e.record()
+        evs = (_vp * (SWL_NUM_STAGES + 1))(*[ctypes.c_void_p(int(e.cuda_event))
+                                             for e in stage_events])
+        _check(lib().switch_layer_forward_timed(*args, evs), "forward_timed")
+
+
+def switch_layer_forward_host_io(x_host, W_r, W1, b1, W2, b2, capacity_factor, out_host,
+                                 expert_idx_host, gate_host, pos_host, aux_host, b_r=None,
+                                 workspace=None, stream=None) -> None:
+    """Enqueue H2D(x) -> forward -> D2H(outputs); host tensors should be pinned."""
+    T, d, d_ff, N = _shape_of(x_host, W1, W_r)
+    act = x_host.dtype
+    _require(x_host, "x_host", act, device="cpu")
+    _require(out_host, "out_host", act, device="cpu")
+    for t, n in ((W1, "W1"), (b1, "b1"), (W2, "W2"), (b2, "b2")):
+        _require(t, n, act)
+    _require(W_r, "W_r", torch.float32)
+    _require(expert_idx_host, "expert_idx_host", torch.int32, device="cpu")
+    _require(pos_host, "pos_host", torch.int32, device="cpu")
+    _require(gate_host, "gate_host", torch.float32, device="cpu")
+    _require(aux_host, "aux_host", torch.float32, device="cpu")
+    _require(workspace, "workspace", torch.uint8)
+    _check(lib().switch_layer_forward_host_io(
+        T, d, d_ff, N, dtype_code(act), _ptr(x_host), _ptr(W_r), _ptr(W1), _ptr(b1), _ptr(W2),
+        _ptr(b2), float(capacity_factor), _ptr(out_host), _ptr(expert_idx_host),
+        _ptr(gate_host), _ptr(pos_host), _ptr(aux_host), _ptr(b_r), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)), "forward_host_io")
+
+
+def switch_layer_device_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(lib().switch_layer_device_status(_ptr(workspace), _stream_handle(stream)))
+
+
+def switch_layer_status_string(status: int) -> str:
+    return _status_string(status)
+
+
+def switch_layer_stage_name(k: int) -> Optional[str]:
+    r = lib().switch_layer_stage_name(k)
+    return None if r is None else r.decode()
+
+
+def switch_layer_launch_count() -> int:
+    return int(lib().switch_layer_launch_count())
+
+
+# ---------------------------------------------------------------------------
+# convenience: allocate outputs + workspace with torch and run
+# ---------------------------------------------------------------------------
+def alloc_workspace(T, d, d_ff, N, act_dtype: torch.dtype, capacity_factor: float,
+                    host_io: bool = False, device="cuda") -> torch.Tensor:
+    n = switch_layer_workspace_size(T, d, d_ff, N, dtype_code(act_dtype), capacity_factor,
+                                    SWL_WS_HOST_IO if host_io else 0)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def alloc_outputs(T, d, act_dtype, device="cuda") -> dict:
+    return {
+        "out": torch.empty((T, d), dtype=act_dtype, device=device),
+        "expert_idx": torch.empty(T, dtype=torch.int32, device=device),
+        "gate": torch.empty(T, dtype=torch.float32, device=device),
+        "pos_in_expert": torch.empty(T, dtype=torch.int32, device=device),
+        "aux_loss": torch.empty(1, dtype=torch.float32, device=device),
+    }
+
+
+def forward(inputs: dict, capacity_factor: float, workspace: Optional[torch.Tensor] = None,
+            outputs: Optional[dict] = None, stream=None, check: bool = True) -> dict:
+    """Run the layer on ``inputs`` (keys x, W_r, b_r, W1, b1, W2, b2; CUDA tensors)."""
+    x, W1 = inputs["x"], inputs["W1"]
+    T, d = x.shape
+    N, d_ff, _ = W1.shape
+    if workspace is None:
+        workspace = alloc_workspace(T, d, d_ff, N, x.dtype, capacity_factor, device=x.device)
+    if outputs is None:
+        outputs = alloc_outputs(T, d, x.dtype, device=x.device)
+    switch_layer_forward(x, inputs["W_r"], W1, inputs["b1"], inputs["W2"], inputs["b2"],
+                         capacity_factor, outputs["out"], outputs["expert_idx"], outputs["gate"],
+                         outputs["pos_in_expert"], outputs["aux_loss"], b_r=inputs.get("b_r"),
+                         workspace=workspace, stream=stream)
+    if check:
+        _check(switch_layer_device_status(workspace, stream), "device status")
+    return outputs

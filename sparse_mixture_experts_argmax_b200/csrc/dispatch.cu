@@ -1,0 +1,214 @@
+// Dispatch of the Switch layer: capacity, positions, drops and the gather into
+// per-expert buffers, plus the load-balancing loss.
+//
+// Positions follow the cumulative sum over each expert's column of the dispatch
+// mask in token order; a token whose position reaches the expert capacity
+// overflows and is dropped (paper-graph summary of arXiv 2101.03961, section
+// 3.4, "The routing mechanics in detail"; capacity C = ceil(cf * T / N) from
+// the "Capacity Factor" section of the Switch Transformer reading note).
+// Dropped tokens get a zero layer output (Switch Transformer, explained: they
+// skip the expert and continue on the residual path, which is outside this layer).
+//
+// Aux loss = N * sum_i f_i P_i with f_i the fraction of tokens whose argmax is i
+// and P_i the mean router probability of i ("The loss formulation"), returned
+// without the alpha factor.
+//
+// dispatch_scan_kernel:   per expert, exclusive scan of the per-block counts over
+//                         token blocks (token order); expert totals; fp64 sums of
+//                         p.  The last CTA to finish scans over experts (packed
+//                         row bases, GEMM tile prefix) and writes the aux loss.
+// dispatch_gather_kernel: pos = block offset + in-block rank; kept tokens are
+//                         copied into their packed row of the expert buffer with
+//                         16-byte vector moves, dropped tokens' output rows zeroed.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <type_traits>
+
+#include "kernels.h"
+
+namespace swl {
+namespace {
+
+constexpr int kScanThreads = 256;
+constexpr int kScanWarps = kScanThreads / 32;
+
+__global__ void __launch_bounds__(kScanThreads)
+dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict__ blk_psum,
+                     int* __restrict__ blk_off, int* __restrict__ exp_count,
+                     double* __restrict__ psum64, int* __restrict__ exp_rows,
+                     int* __restrict__ exp_base, int* __restrict__ tile_prefix,
+                     float* __restrict__ aux_loss, WsHeader* hdr, int nblk, int N, int T,
+                     int C_eff, int tile_rows) {
+  __shared__ int wc[kScanWarps][32];
+  __shared__ double wp[kScanWarps][32];
+  __shared__ int is_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + lane;
+  const int per = (nblk + kScanWarps - 1) / kScanWarps;
+  const int b0 = warp * per, b1 = min(nblk, b0 + per);
+
+  // pass 1: this warp's share of blocks, per expert (lane)
+  int csum = 0;
+  double psum = 0.0;
+  if (e < N) {
+    for (int b = b0; b < b1; ++b) {
+      csum += blk_count[(size_t)b * N + e];
+      psum += (double)blk_psum[(size_t)b * N + e];
+    }
+  }
+  wc[warp][lane] = csum;
+  wp[warp][lane] = psum;
+  __syncthreads();
+  // pass 2: exclusive offsets in token order
+  if (e < N) {
+    int off = 0;
+    for (int w = 0; w < warp; ++w) off += wc[w][lane];
+    for (int b = b0; b < b1; ++b) {
+      const size_t i = (size_t)b * N + e;
+      const int c = blk_count[i];
+      blk_off[i] = off;
+      off += c;
+    }
+    if (warp == 0) {
+      int tot = 0;
+      double ps = 0.0;
+      for (int w = 0; w < kScanWarps; ++w) { tot += wc[w][lane]; ps += wp[w][lane]; }
+      exp_count[e] = tot;
+      psum64[e] = ps;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int ticket = atomicAdd(&hdr->done, 1u);
+    is_last = (ticket == gridDim.x - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  // ---- last CTA: scan over experts, tile prefix, aux loss
+  __shared__ int s_rows[kScanThreads];
+  __shared__ int s_tiles[kScanThreads];
+  __shared__ double s_aux[kScanThreads];
+  const int chunk = (N + kScanThreads - 1) / kScanThreads;
+  const int e0 = threadIdx.x * chunk, e1 = min(N, e0 + chunk);
+  int rows = 0, tiles = 0;
+  double aux = 0.0;
+  for (int i = e0; i < e1; ++i) {
+    const int c = __ldcg(exp_count + i);
+    const int m = min(c, C_eff);
+    rows += m;
+    tiles += (m + tile_rows - 1) / tile_rows;
+    aux += (double)c * __ldcg(psum64 + i);
+  }
+  s_rows[threadIdx.x] = rows;
+  s_tiles[threadIdx.x] = tiles;
+  s_aux[threadIdx.x] = aux;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // serial exclusive scan over the 256 partials (fixed order, deterministic)
+    int r = 0, t = 0;
+    double a = 0.0;
+    for (int i = 0; i < kScanThreads; ++i) {
+      const int rr = s_rows[i], tt = s_tiles[i];
+      s_rows[i] = r;
+      s_tiles[i] = t;
+      r += rr;
+      t += tt;
+      a += s_aux[i];
+    }
+    tile_prefix[N] = t;
+    // aux = N * sum_i (count_i / T) * (psum_i / T)
+    *aux_loss = (float)((double)N * a / ((double)T * (double)T));
+    hdr->done = 0u;   // ready for the next call
+  }
+  __syncthreads();
+  rows = s_rows[threadIdx.x];
+  tiles = s_tiles[threadIdx.x];
+  for (int i = e0; i < e1; ++i) {
+    const int m = min(__ldcg(exp_count + i), C_eff);
+    exp_rows[i] = m;
+    exp_base[i] = rows;
+    tile_prefix[i] = tiles;
+    rows += m;
+    tiles += (m + tile_rows - 1) / tile_rows;
+  }
+}
+
+constexpr int kGatherThreads = 256;
+constexpr int kGatherWarps = kGatherThreads / 32;
+
+// One warp per token.  VEC = bytes per vector move (16 for bf16 rows, 4 for fp32).
+template <int VEC>
+__global__ void __launch_bounds__(kGatherThreads)
+dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ expert_idx,
+                       int* __restrict__ pos_in_expert, const int* __restrict__ blk_off,
+                       const int* __restrict__ exp_base, int* __restrict__ slot_token,
+                       uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out, int T, int N,
+                       int C_eff, int row_bytes, WsHeader* hdr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kGatherWarps + warp;
+  if (t >= T) return;
+  const int e = expert_idx[t];
+  if (e < 0 || e >= N) {          // cannot happen: the router clamps its choice
+    if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
+    return;
+  }
+  const int b = t / kTokensPerBlock;
+  const int pos = blk_off[(size_t)b * N + e] + pos_in_expert[t];   // holds the in-block rank
+  __syncwarp();
+  if (lane == 0) pos_in_expert[t] = pos;
+  using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
+  const int nv = row_bytes / VEC;
+  if (pos < C_eff) {
+    const int row = exp_base[e] + pos;
+    if (lane == 0) slot_token[row] = t;
+    const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
+    V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
+    for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+  } else {
+    V* dst = reinterpret_cast<V*>(out + (size_t)t * row_bytes);
+    V z;
+    memset(&z, 0, sizeof(V));
+    for (int i = lane; i < nv; i += 32) dst[i] = z;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
+                                 cudaStream_t stream) {
+  const int grid = (int)((s.N + 31) / 32);
+  dispatch_scan_kernel<<<grid, kScanThreads, 0, stream>>>(
+      ws.blk_count, ws.blk_psum, ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base,
+      ws.tile_prefix, aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
+                                   const int* expert_idx, int* pos_in_expert, void* out,
+                                   cudaStream_t stream) {
+  const int grid = (int)((s.T + kGatherWarps - 1) / kGatherWarps);
+  const int elem = s.dtype == 1 ? 2 : 4;
+  const int row_bytes = (int)(s.d * elem);
+  const bool vec16 = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(out) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ws.xbuf) & 15) == 0);
+  if (vec16)
+    dispatch_gather_kernel<16><<<grid, kGatherThreads, 0, stream>>>(
+        static_cast<const uint8_t*>(x), expert_idx, pos_in_expert, ws.blk_off, ws.exp_base,
+        ws.slot_token, static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
+        (int)s.N, (int)s.C_eff, row_bytes, ws.hdr);
+  else
+    dispatch_gather_kernel<4><<<grid, kGatherThreads, 0, stream>>>(
+        static_cast<const uint8_t*>(x), expert_idx, pos_in_expert, ws.blk_off, ws.exp_base,
+        ws.slot_token, static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
+        (int)s.N, (int)s.C_eff, row_bytes, ws.hdr);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace swl

@@ -1,0 +1,97 @@
+// fp32 expert FFN GEMMs (CUDA cores, FFMA) for layers whose activations and
+// expert weights are fp32.  Same packed-row layout and fused epilogues as the
+// bf16 tensor-core path:
+//   GEMM1: hbuf[r, :]  = relu(W1[e] xbuf[r, :] + b1[e])
+//   GEMM2: out[tok, :] = g_tok * (W2[e] hbuf[r, :] + b2[e]),  tok = slot_token[r]
+// (Switch Transformer reading note, "Expert FFN Layer" and "Router").
+// Tensor cores are not used here: tf32 would not meet a 1e-4 tolerance.
+//
+// CTA = 32 output features x 32 packed rows of one expert; 256 threads, 4
+// outputs each; K staged through shared memory in chunks of 32.  grid.x walks
+// the per-expert row tiles through the device tile prefix (tile rows = 32),
+// grid.y the 32-feature blocks.
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+
+namespace swl {
+namespace {
+
+constexpr int kTile = kF32TileRows;   // 32
+
+__global__ void __launch_bounds__(256)
+expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ W,
+                       const float* __restrict__ bias, const int* __restrict__ tile_prefix,
+                       const int* __restrict__ exp_rows, const int* __restrict__ exp_base,
+                       const int* __restrict__ slot_token, const float* __restrict__ gate,
+                       float* __restrict__ out, int num_experts, int M, int K, int mode) {
+  __shared__ float As[kTile][kTile + 1];   // [row][k]
+  __shared__ float Ws[kTile][kTile + 1];   // [feature][k]
+  const int g = blockIdx.x;
+  if (g >= tile_prefix[num_experts]) return;
+  int lo = 0, hi = num_experts;            // last e with prefix[e] <= g
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_prefix[mid] <= g) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  const int nt = g - tile_prefix[e];
+  const int r0 = exp_base[e] + nt * kTile;
+  const int nrows = min(kTile, exp_rows[e] - nt * kTile);
+  const int m0 = blockIdx.y * kTile;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // feature, row group
+  const float* We = W + (size_t)e * M * K;
+
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < K; k0 += kTile) {
+    for (int i = threadIdx.x; i < kTile * kTile; i += 256) {
+      const int rr = i / kTile, kk = i % kTile;
+      As[rr][kk] = (rr < nrows && k0 + kk < K) ? act[(size_t)(r0 + rr) * K + k0 + kk] : 0.f;
+      Ws[rr][kk] = (m0 + rr < M && k0 + kk < K) ? We[(size_t)(m0 + rr) * K + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kTile; ++kk) {
+      const float w = Ws[tx][kk];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(As[ty * 4 + i][kk], w, acc[i]);
+    }
+    __syncthreads();
+  }
+  const int m = m0 + tx;
+  if (m >= M) return;
+  const float bm = bias[(size_t)e * M + m];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = ty * 4 + i;
+    if (rr >= nrows) continue;
+    const float v = acc[i] + bm;
+    if (mode == 0) {
+      out[(size_t)(r0 + rr) * M + m] = fmaxf(v, 0.f);
+    } else {
+      const int tok = slot_token[r0 + rr];
+      out[(size_t)tok * M + m] = gate[tok] * v;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int which, const void* W,
+                                   const void* bias, const float* gate, void* out,
+                                   cudaStream_t stream) {
+  const int M = static_cast<int>(which == 0 ? s.d_ff : s.d);
+  const int K = static_cast<int>(which == 0 ? s.d : s.d_ff);
+  const float* act = static_cast<const float*>(which == 0 ? ws.xbuf : ws.hbuf);
+  // upper bound on row tiles: sum_e ceil(m_e / 32) <= T / 32 + N
+  const int64_t max_tiles = (s.T + kTile - 1) / kTile + s.N;
+  dim3 grid(static_cast<unsigned>(max_tiles), (M + kTile - 1) / kTile);
+  expert_gemm_f32_kernel<<<grid, 256, 0, stream>>>(
+      act, static_cast<const float*>(W), static_cast<const float*>(bias), ws.tile_prefix,
+      ws.exp_rows, ws.exp_base, ws.slot_token, gate, static_cast<float*>(out),
+      static_cast<int>(s.N), M, K, which);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace swl

@@ -1,0 +1,340 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM),
+// bf16 inputs with fp32 accumulation.
+//
+// Each expert is an FFN, E_i(x) = W_2,i relu(W_1,i x + b_1,i) + b_2,i, and a
+// kept token's layer output is y_t = g_t E_{e_t}(x_t) (Switch Transformer
+// reading note, sections "Expert FFN Layer" and "Router").  The expert
+// computation is a batched matrix multiplication over the tokens each expert
+// received (paper-graph summary of arXiv 2101.03961, "The routing mechanics in
+// detail": expert computation).
+//
+//   GEMM1 (which = 0): hbuf[r, :]  = relu(W1[e] xbuf[r, :] + b1[e])        (bf16)
+//   GEMM2 (which = 1): out[tok, :] = g_tok * (W2[e] hbuf[r, :] + b2[e])     (bf16)
+//                      with tok = slot_token[r]: the scatter back to token order
+//                      (the combine) happens in this epilogue.
+//
+// Formulation ("swap AB"): the weight matrix is the UMMA A operand (M = 128
+// output features per tile, K-major), the packed token rows of one expert are
+// the B operand (N = up to 256 tokens, K-major), so every weight byte is
+// streamed from HBM once per token tile no matter how few tokens an expert has.
+// D[feature, token] accumulates in TMEM.
+//
+// Persistent kernel, one CTA per SM, 256 threads:
+//   warp 0      TMA producer (one thread): A and B k-blocks of 64 elements into a
+//               ring of shared-memory stages (128-byte swizzle)
+//   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
+//   warp 2      TMEM allocator (512 columns: two 256-column accumulators)
+//   warps 4..7  epilogue: tcgen05.ld, bias / ReLU / gate in fp32, bf16 pack,
+//               transpose through shared memory, 16-byte stores
+// Tiles (expert, 128-feature block, token block) are numbered expert-major and
+// handed out round-robin; the token-block count of each expert comes from the
+// device tile prefix written by the dispatch scan.  Every wait is bounded; a
+// stuck pipeline sets the device error word and the CTA drains and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace swl {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBM = 128;              // UMMA M: output features per tile
+constexpr int kBK = 64;               // K elements per stage (one 128-byte swizzle row)
+constexpr int kUmmaK = 16;            // K per tcgen05.mma (bf16)
+constexpr int kMaxStages = 12;
+constexpr int kAccCols = 256;         // TMEM columns per accumulator buffer
+constexpr int kTmemCols = 512;
+constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KiB
+constexpr int kEpiStageBytes = 4 * 32 * 32 * 2;   // per-warp 32x32 bf16 transpose tiles
+
+struct GemmArgs {
+  const int* tile_prefix;      // [N+1]
+  const int* exp_rows;         // [N]
+  const int* exp_base;         // [N]
+  const __nv_bfloat16* bias;   // [N, M]
+  const float* gate;           // [T]       (GEMM2)
+  const int* slot_token;       // [T]       (GEMM2)
+  __nv_bfloat16* out;          // GEMM1: hbuf [T, M] (packed rows); GEMM2: out [T, M]
+  int* err;
+  int num_experts;
+  int M;          // output features per expert
+  int m_tiles;    // ceil(M / 128)
+  int k_blocks;   // ceil(K / 64)
+  int bn;         // token rows per tile (multiple of 16, <= 256)
+  int stages;
+  int mode;       // 0: bias + ReLU, packed rows; 1: bias, gate, scatter to token rows
+};
+
+struct TileCoord {
+  int e, mt, nt;
+};
+
+// Tile t of expert e occupies [P[e]*m_tiles, P[e+1]*m_tiles) with P the tile
+// prefix; inside, token blocks vary fastest so concurrent CTAs share weights.
+__device__ __forceinline__ TileCoord decode_tile(int tile, const GemmArgs& a) {
+  const int q = tile / a.m_tiles;
+  int lo = 0, hi = a.num_experts;     // find last e with P[e] <= q  (P[N] > q)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a.tile_prefix + mid) <= q) lo = mid; else hi = mid;
+  }
+  const int p0 = __ldg(a.tile_prefix + lo);
+  const int nts = __ldg(a.tile_prefix + lo + 1) - p0;
+  const int local = tile - p0 * a.m_tiles;
+  TileCoord c;
+  c.e = lo;
+  c.mt = local / nts;
+  c.nt = local - c.mt * nts;
+  return c;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int stages = args.stages;
+  const uint32_t b_bytes = static_cast<uint32_t>(args.bn) * kBK * 2;
+  uint8_t* smem_a = smem;
+  uint8_t* smem_b = smem_a + stages * kABytes;
+  __nv_bfloat16* epi = reinterpret_cast<__nv_bfloat16*>(smem_b + stages * b_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(epi) + kEpiStageBytes);
+  uint64_t* full_bar = bars;                    // [kMaxStages]
+  uint64_t* empty_bar = bars + kMaxStages;      // [kMaxStages]
+  uint64_t* tfull_bar = bars + 2 * kMaxStages;  // [2]
+  uint64_t* tempty_bar = tfull_bar + 2;         // [2]
+  uint64_t* drain_bar = tempty_bar + 2;         // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = __ldg(args.tile_prefix + args.num_experts) * args.m_tiles;
+  if (static_cast<int>(blockIdx.x) >= total) return;   // uniform per CTA: nothing to do
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(&full_bar[s], 1);
+      ptx::mbar_init(&empty_bar[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&tfull_bar[i], 1);
+      ptx::mbar_init(&tempty_bar[i], 4);      // one arrive per epilogue warp
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicExch(args.err, kDevPipelineTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = ptx::l2_policy_evict_first();
+      const uint64_t pol_x = ptx::l2_policy_evict_last();
+      uint32_t issued = 0u;           // stages that received at least one load
+      uint32_t last_par = 0u;         // parity of each stage's latest load
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord c = decode_tile(tile, args);
+        const int arow = c.e * args.M + c.mt * kBM;
+        const int brow = __ldg(args.exp_base + c.e) + c.nt * args.bn;
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag)) { fail(); ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
+          ptx::tma_load_2d(smem_a + stage * kABytes, &tmA, &full_bar[stage], kb * kBK, arow, pol_w);
+          ptx::tma_load_2d(smem_b + stage * b_bytes, &tmB, &full_bar[stage], kb * kBK, brow, pol_x);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (ph << stage);
+          if (++stage == stages) { stage = 0; ph ^= 1u; }
+        }
+      }
+      // drain: every issued load must land before the CTA may exit
+      for (int s = 0; s < stages; ++s) {
+        if (issued & (1u << s)) {
+          volatile int never = 0;
+          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never)) {
+            atomicExch(args.err, kDevPipelineTimeout);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord c = decode_tile(tile, args);
+        const int rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
+        const uint32_t n_mma = static_cast<uint32_t>((rows + 15) & ~15);
+        const uint32_t idesc = ptx::umma_idesc_bf16_f32(n_mma);
+        if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { fail(); break; }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag)) { fail(); ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_u32(smem_a + stage * kABytes);
+          const uint32_t b_addr = ptx::smem_u32(smem_b + stage * b_bytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + k * kUmmaK * 2);
+            const uint64_t bd = ptx::umma_desc_sw128_kmajor(b_addr + k * kUmmaK * 2);
+            ptx::umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          ptx::umma_commit(&empty_bar[stage]);      // frees the stage when these MMAs finish
+          if (++stage == stages) { stage = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        ptx::umma_commit(&tfull_bar[acc]);          // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      // drain: all MMAs issued by this thread complete before TMEM is released
+      ptx::umma_commit(drain_bar);
+      volatile int never = 0;
+      if (!ptx::mbar_wait(drain_bar, 0u, &never)) atomicExch(args.err, kDevPipelineTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                        // TMEM lane quarter of this warp
+    __nv_bfloat16* st = epi + q * 32 * 32;         // [32 tokens][32 features]
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileCoord c = decode_tile(tile, args);
+      const int rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
+      const int row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
+      if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
+      ptx::tc_fence_after();
+      const int feat0 = c.mt * kBM + q * 32;       // first feature of this warp
+      const int f = feat0 + lane;
+      const float bias = (f < args.M) ? __bfloat162float(args.bias[(size_t)c.e * args.M + f]) : 0.f;
+      const uint32_t t_base =
+          tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c0 = 0; c0 < rows; c0 += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
+        ptx::tmem_ld_wait();
+        // destination row and gate of column (c0 + lane)
+        const int col = c0 + lane;
+        int dst = row0 + col;
+        float g = 1.f;
+        if (args.mode == 1) {
+          dst = (col < rows) ? __ldg(args.slot_token + row0 + col) : 0;
+          g = (col < rows) ? __ldg(args.gate + dst) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float v = __uint_as_float(r[j]) + bias;
+          if (args.mode == 0) {
+            v = fmaxf(v, 0.f);
+          } else {
+            v *= __shfl_sync(0xffffffffu, g, j);
+          }
+          st[j * 32 + lane] = __float2bfloat16_rn(v);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int idx = lane + 32 * i;
+          const int j = idx >> 2, part = idx & 3;
+          const int drow = __shfl_sync(0xffffffffu, dst, j);
+          if (c0 + j < rows && feat0 + part * 8 < args.M) {
+            *reinterpret_cast<uint4*>(args.out + (size_t)drow * args.M + feat0 + part * 8) =
+                *reinterpret_cast<const uint4*>(st + j * 32 + part * 8);
+          }
+        }
+        __syncwarp();
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) { acc = 0; aph ^= 1u; }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+size_t gemm_smem_bytes(int bn, int stages) {
+  return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
+         kEpiStageBytes + (2 * kMaxStages + 5) * sizeof(uint64_t) + 2 * sizeof(uint32_t);
+}
+
+}  // namespace
+
+int bf16_tile_rows(int64_t C_eff) {
+  int64_t r = (C_eff + 15) / 16 * 16;
+  if (r < 16) r = 16;
+  if (r > 256) r = 256;
+  return static_cast<int>(r);
+}
+
+cudaError_t launch_expert_gemm_bf16(const Shape& s, const Workspace& ws, int which,
+                                    const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                    const void* bias, const float* gate, void* out, int num_sms,
+                                    cudaStream_t stream) {
+  constexpr size_t kMaxSmem = 232448;   // 227 KiB opt-in per block
+  GemmArgs a;
+  a.tile_prefix = ws.tile_prefix;
+  a.exp_rows = ws.exp_rows;
+  a.exp_base = ws.exp_base;
+  a.bias = static_cast<const __nv_bfloat16*>(bias);
+  a.gate = gate;
+  a.slot_token = ws.slot_token;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.err = &ws.hdr->err;
+  a.num_experts = static_cast<int>(s.N);
+  const int64_t M = which == 0 ? s.d_ff : s.d;
+  const int64_t K = which == 0 ? s.d : s.d_ff;
+  a.M = static_cast<int>(M);
+  a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
+  a.k_blocks = static_cast<int>((K + kBK - 1) / kBK);
+  a.bn = s.tile_rows;
+  a.mode = which;
+  int stages = kMaxStages;
+  while (stages > 2 && gemm_smem_bytes(a.bn, stages) > kMaxSmem) --stages;
+  a.stages = stages;
+  const size_t smem = gemm_smem_bytes(a.bn, stages);
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_sm100_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  expert_gemm_sm100_kernel<<<num_sms, kThreads, smem, stream>>>(tmA, tmB, a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace swl

@@ -1,0 +1,91 @@
+// Internal interface between the C-ABI host code (switch_layer.cu) and the
+// kernels of the Switch-layer forward.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace swl {
+
+// Device error word values (first int of the workspace header).
+enum DeviceError : int {
+  kDevOk = 0,
+  kDevPipelineTimeout = 1,   // a GEMM pipeline wait exceeded its time limit
+  kDevIndexOutOfRange = 2,   // an index check failed (should never happen)
+  kDevNonFiniteLogits = 3,   // a token had no finite maximum logit (NaN/Inf input)
+};
+
+constexpr int kTokensPerBlock = 128;   // token block of the softmax / rank / gather stages
+constexpr int kMaxExperts = 1 << 20;
+
+// Workspace header (256 bytes at offset 0).
+struct WsHeader {
+  int err;            // DeviceError of the last call
+  unsigned int done;  // arrival counter of the dispatch-scan kernel (self-resetting)
+  int pad[62];
+};
+
+// Device pointers carved out of the caller's workspace.
+struct Workspace {
+  WsHeader* hdr;
+  float* logits;        // [T, N] fp32
+  int* blk_count;       // [nblk, N] tokens of block b routed to expert e
+  int* blk_off;         // [nblk, N] tokens of earlier blocks routed to e
+  float* blk_psum;      // [nblk, N] sum over block b of p_{t,e}
+  int* exp_count;       // [N] tokens whose argmax is e (before capacity)
+  int* exp_rows;        // [N] kept rows m_e = min(count_e, C)
+  int* exp_base;        // [N] first packed row of expert e
+  int* tile_prefix;     // [N+1] prefix over experts of ceil(m_e / tile_rows)
+  double* psum64;       // [N] sum over all tokens of p_{t,e}
+  int* slot_token;      // [T] packed row -> token
+  void* xbuf;           // [T, d] packed expert inputs (act dtype)
+  void* hbuf;           // [T, d_ff] packed hidden activations (act dtype)
+  // host-I/O staging (only with SWL_WS_HOST_IO)
+  void* x_dev;
+  void* out_dev;
+  int* idx_dev;
+  float* gate_dev;
+  int* pos_dev;
+  float* aux_dev;
+  size_t total_bytes;
+};
+
+struct Shape {
+  int64_t T, d, d_ff, N;
+  int dtype;      // 0 = fp32, 1 = bf16
+  int64_t C;      // capacity (formula value)
+  int64_t C_eff;  // min(C, T): rows an expert can actually keep
+  int nblk;       // ceil(T / kTokensPerBlock)
+  int tile_rows;  // token rows per GEMM tile (N of the UMMA, or the SIMT tile)
+};
+
+size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
+
+// ---- stage launchers (all asynchronous on `stream`; return cudaGetLastError()).
+cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
+                                 const float* W_r, const float* b_r, cudaStream_t stream);
+cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, int* expert_idx,
+                                  float* gate, int* local_rank, cudaStream_t stream);
+cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
+                                 cudaStream_t stream);
+cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
+                                   const int* expert_idx, int* pos_in_expert, void* out,
+                                   cudaStream_t stream);
+cudaError_t launch_expert_gemm_bf16(const Shape& s, const Workspace& ws, int which,
+                                    const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                    const void* bias, const float* gate, void* out,
+                                    int num_sms, cudaStream_t stream);
+cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int which,
+                                   const void* W, const void* bias, const float* gate, void* out,
+                                   cudaStream_t stream);
+
+// Tile rows for the bf16 tcgen05 GEMMs given the effective capacity.
+int bf16_tile_rows(int64_t C_eff);
+constexpr int kF32TileRows = 32;
+
+// Number of kernel launches issued by this library since load.
+void count_launch(int n = 1);
+
+}  // namespace swl

@@ -1,0 +1,369 @@
+// C-ABI host side of the Switch-layer forward: argument validation, exact
+// capacity, workspace layout, TMA descriptors and the launch sequence.
+//
+// Stage order on the caller's stream (no host synchronisation inside):
+//   0 router logits        fp32 FFMA GEMM            (router.cu)
+//   1 router softmax       max/argmax/gate, ranks     (router.cu)
+//   2 dispatch scan        offsets, capacity, aux     (dispatch.cu)
+//   3 dispatch gather      pos, packed expert rows    (dispatch.cu)
+//   4 expert GEMM1         bias + ReLU                (expert_gemm_sm100.cu / expert_gemm_f32.cu)
+//   5 expert GEMM2         bias, gate, combine        (same)
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "switch_layer.h"
+#include "kernels.h"
+
+namespace swl {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws) {
+  const size_t elem = s.dtype == SWL_BF16 ? 2 : 4;
+  const size_t T = static_cast<size_t>(s.T), N = static_cast<size_t>(s.N);
+  const size_t nb = static_cast<size_t>(s.nblk);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return base + o;
+  };
+  Workspace w{};
+  w.hdr = reinterpret_cast<WsHeader*>(take(sizeof(WsHeader)));
+  w.logits = reinterpret_cast<float*>(take(T * N * 4));
+  w.blk_count = reinterpret_cast<int*>(take(nb * N * 4));
+  w.blk_off = reinterpret_cast<int*>(take(nb * N * 4));
+  w.blk_psum = reinterpret_cast<float*>(take(nb * N * 4));
+  w.exp_count = reinterpret_cast<int*>(take(N * 4));
+  w.exp_rows = reinterpret_cast<int*>(take(N * 4));
+  w.exp_base = reinterpret_cast<int*>(take(N * 4));
+  w.tile_prefix = reinterpret_cast<int*>(take((N + 1) * 4));
+  w.psum64 = reinterpret_cast<double*>(take(N * 8));
+  w.slot_token = reinterpret_cast<int*>(take(T * 4));
+  w.xbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
+  w.hbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d_ff) * elem));
+  if (host_io) {
+    w.x_dev = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
+    w.out_dev = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
+    w.idx_dev = reinterpret_cast<int*>(take(T * 4));
+    w.gate_dev = reinterpret_cast<float*>(take(T * 4));
+    w.pos_dev = reinterpret_cast<int*>(take(T * 4));
+    w.aux_dev = reinterpret_cast<float*>(take(4));
+  }
+  w.total_bytes = off;
+  if (ws) *ws = w;
+  return off;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode_tiled() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, inner] (inner contiguous), box [box_rows, 64], 128-byte swizzle.
+static bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                           uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int num_sms_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+static bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+// Fills Shape; returns SWL_OK or the validation error.
+static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype, double cf,
+                             Shape* s) {
+  if (T < 0 || d <= 0 || d_ff <= 0 || N <= 0) return SWL_ERR_INVALID_ARG;
+  if (dtype != SWL_F32 && dtype != SWL_BF16) return SWL_ERR_INVALID_ARG;
+  if (!std::isfinite(cf) || !(cf > 0.0)) return SWL_ERR_INVALID_ARG;
+  if (dtype == SWL_BF16 && (d % 8 != 0 || d_ff % 8 != 0)) return SWL_ERR_UNSUPPORTED;
+  if (N > kMaxExperts) return SWL_ERR_UNSUPPORTED;
+  const int64_t lim = INT32_MAX;
+  if (T > lim / 2 || d > lim / 2 || d_ff > lim / 2) return SWL_ERR_UNSUPPORTED;
+  if (N * (d > d_ff ? d : d_ff) > lim) return SWL_ERR_UNSUPPORTED;   // TMA row coordinates
+  s->T = T;
+  s->d = d;
+  s->d_ff = d_ff;
+  s->N = N;
+  s->dtype = dtype;
+  s->C = switch_layer_capacity(T, N, cf);
+  s->C_eff = s->C < T ? s->C : T;
+  s->nblk = static_cast<int>((T + kTokensPerBlock - 1) / kTokensPerBlock);
+  s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
+  return SWL_OK;
+}
+
+static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x,
+                              const float* W_r, const void* W1, const void* b1, const void* W2,
+                              const void* b2, void* out, int32_t* expert_idx, float* gate,
+                              int32_t* pos_in_expert, float* aux_loss, const float* b_r,
+                              cudaStream_t stream, void* const* ev) {
+  auto rec = [&](int k) -> bool {
+    return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[k]), stream) == cudaSuccess;
+  };
+  if (!rec(0)) return SWL_ERR_CUDA;
+  if (launch_router_logits(s, ws, x, W_r, b_r, stream) != cudaSuccess) return SWL_ERR_CUDA;
+  if (!rec(1)) return SWL_ERR_CUDA;
+  if (launch_router_softmax(s, ws, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  if (!rec(2)) return SWL_ERR_CUDA;
+  if (launch_dispatch_scan(s, ws, aux_loss, stream) != cudaSuccess) return SWL_ERR_CUDA;
+  if (!rec(3)) return SWL_ERR_CUDA;
+  if (launch_dispatch_gather(s, ws, x, expert_idx, pos_in_expert, out, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  if (!rec(4)) return SWL_ERR_CUDA;
+  if (s.dtype == SWL_BF16) {
+    const int sms = num_sms_current();
+    if (sms <= 0) return SWL_ERR_CUDA;
+    CUtensorMap a1, b1m, a2, b2m;
+    if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff, 128) ||
+        !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T, s.tile_rows) ||
+        !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
+        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T, s.tile_rows))
+      return SWL_ERR_CUDA;
+    if (launch_expert_gemm_bf16(s, ws, 0, a1, b1m, b1, gate, ws.hbuf, sms, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (!rec(5)) return SWL_ERR_CUDA;
+    if (launch_expert_gemm_bf16(s, ws, 1, a2, b2m, b2, gate, out, sms, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+  } else {
+    if (launch_expert_gemm_f32(s, ws, 0, W1, b1, gate, ws.hbuf, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (!rec(5)) return SWL_ERR_CUDA;
+    if (launch_expert_gemm_f32(s, ws, 1, W2, b2, gate, out, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+  }
+  if (!rec(6)) return SWL_ERR_CUDA;
+  return SWL_OK;
+}
+
+static swl_status validate_io(const Shape& s, const void* x, const float* W_r, const void* W1,
+                              const void* b1, const void* W2, const void* b2, const void* out,
+                              const void* expert_idx, const void* gate, const void* pos,
+                              const void* aux, const void* workspace, size_t workspace_bytes,
+                              bool host_io) {
+  if (!W_r || !W1 || !b1 || !W2 || !b2 || !aux || !workspace) return SWL_ERR_INVALID_ARG;
+  // per-token buffers may be NULL only for an empty batch
+  if (s.T > 0 && (!x || !out || !expert_idx || !gate || !pos)) return SWL_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return SWL_ERR_UNSUPPORTED;
+  const uintptr_t a = s.dtype == SWL_BF16 ? 16 : 4;
+  if (!aligned(W1, a) || !aligned(W2, a) || !aligned(W_r, 4) || !aligned(b1, s.dtype ? 2 : 4) ||
+      !aligned(b2, s.dtype ? 2 : 4))
+    return SWL_ERR_UNSUPPORTED;
+  if (!host_io && (!aligned(x, a) || !aligned(out, a))) return SWL_ERR_UNSUPPORTED;
+  if (!aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(pos, 4) || !aligned(aux, 4))
+    return SWL_ERR_UNSUPPORTED;
+  if (workspace_bytes < workspace_layout(s, host_io, 0, nullptr)) return SWL_ERR_WORKSPACE;
+  return SWL_OK;
+}
+
+static swl_status forward_impl(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                               const void* x, const float* W_r, const void* W1, const void* b1,
+                               const void* W2, const void* b2, double cf, void* out,
+                               int32_t* expert_idx, float* gate, int32_t* pos, float* aux,
+                               const float* b_r, void* workspace, size_t workspace_bytes,
+                               void* stream_v, void* const* ev) {
+  Shape s;
+  swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s);
+  if (st != SWL_OK) return st;
+  st = validate_io(s, x, W_r, W1, b1, W2, b2, out, expert_idx, gate, pos, aux, workspace,
+                   workspace_bytes, false);
+  if (st != SWL_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (T == 0) {
+    if (cudaMemsetAsync(aux, 0, sizeof(float), stream) != cudaSuccess) return SWL_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (ev)
+      for (int k = 0; k <= SWL_NUM_STAGES; ++k)
+        if (cudaEventRecord(static_cast<cudaEvent_t>(ev[k]), stream) != cudaSuccess)
+          return SWL_ERR_CUDA;
+    return SWL_OK;
+  }
+  Workspace ws;
+  workspace_layout(s, false, reinterpret_cast<uintptr_t>(workspace), &ws);
+  return run_forward(s, ws, x, W_r, W1, b1, W2, b2, out, expert_idx, gate, pos, aux, b_r, stream,
+                     ev);
+}
+
+}  // namespace swl
+
+using namespace swl;
+
+extern "C" {
+
+int64_t switch_layer_capacity(int64_t T, int64_t N, double cf) {
+  if (T < 0 || N <= 0 || !std::isfinite(cf) || !(cf > 0.0)) return -1;
+  if (T == 0) return 0;
+  // cf = mant * 2^e2 exactly, mant < 2^53
+  int e = 0;
+  const double m = std::frexp(cf, &e);
+  const uint64_t mant = static_cast<uint64_t>(std::ldexp(m, 53));
+  const int e2 = e - 53;
+  unsigned __int128 num = static_cast<unsigned __int128>(mant) * static_cast<uint64_t>(T);
+  if (e2 >= 0) {
+    if (e2 >= 127 || (num >> (127 - e2)) != 0) return INT64_MAX;
+    num <<= e2;
+  } else {
+    // ceil(num / (N 2^s)) = ceil(ceil(num / 2^s) / N)
+    const int sh = -e2;
+    if (sh >= 127) {
+      num = 1;   // 0 < num < 2^117 <= 2^sh
+    } else {
+      const unsigned __int128 one = 1;
+      num = (num + ((one << sh) - 1)) >> sh;
+    }
+  }
+  const unsigned __int128 n = static_cast<uint64_t>(N);
+  const unsigned __int128 q = (num + n - 1) / n;
+  if (q > static_cast<unsigned __int128>(INT64_MAX)) return INT64_MAX;
+  return static_cast<int64_t>(q);
+}
+
+swl_status switch_layer_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                       double cf, int flags, size_t* bytes) {
+  if (!bytes) return SWL_ERR_INVALID_ARG;
+  Shape s;
+  const swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s);
+  if (st != SWL_OK) return st;
+  *bytes = workspace_layout(s, (flags & SWL_WS_HOST_IO) != 0, 0, nullptr);
+  return SWL_OK;
+}
+
+swl_status switch_layer_forward(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                const void* x, const float* W_r, const void* W1, const void* b1,
+                                const void* W2, const void* b2, double capacity_factor,
+                                void* out, int32_t* expert_idx, float* gate,
+                                int32_t* pos_in_expert, float* aux_loss, const float* b_r,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
+                      expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
+                      stream, nullptr);
+}
+
+swl_status switch_layer_forward_timed(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                      const void* x, const float* W_r, const void* W1,
+                                      const void* b1, const void* W2, const void* b2,
+                                      double capacity_factor, void* out, int32_t* expert_idx,
+                                      float* gate, int32_t* pos_in_expert, float* aux_loss,
+                                      const float* b_r, void* workspace, size_t workspace_bytes,
+                                      void* stream, void* const* stage_events) {
+  if (!stage_events) return SWL_ERR_INVALID_ARG;
+  for (int k = 0; k <= SWL_NUM_STAGES; ++k)
+    if (!stage_events[k]) return SWL_ERR_INVALID_ARG;
+  return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
+                      expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
+                      stream, stage_events);
+}
+
+swl_status switch_layer_forward_host_io(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                        const void* x_host, const float* W_r, const void* W1,
+                                        const void* b1, const void* W2, const void* b2,
+                                        double capacity_factor, void* out_host,
+                                        int32_t* expert_idx_host, float* gate_host,
+                                        int32_t* pos_host, float* aux_host, const float* b_r,
+                                        void* workspace, size_t workspace_bytes, void* stream_v) {
+  Shape s;
+  swl_status st = make_shape(T, d, d_ff, N, dtype, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  st = validate_io(s, x_host, W_r, W1, b1, W2, b2, out_host, expert_idx_host, gate_host, pos_host,
+                   aux_host, workspace, workspace_bytes, true);
+  if (st != SWL_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (T == 0) {
+    *aux_host = 0.f;
+    return SWL_OK;
+  }
+  Workspace ws;
+  workspace_layout(s, true, reinterpret_cast<uintptr_t>(workspace), &ws);
+  const size_t elem = dtype == SWL_BF16 ? 2 : 4;
+  const size_t xb = static_cast<size_t>(T) * static_cast<size_t>(d) * elem;
+  const size_t tb = static_cast<size_t>(T) * 4;
+  if (cudaMemcpyAsync(ws.x_dev, x_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  st = run_forward(s, ws, ws.x_dev, W_r, W1, b1, W2, b2, ws.out_dev, ws.idx_dev, ws.gate_dev,
+                   ws.pos_dev, ws.aux_dev, b_r, stream, nullptr);
+  if (st != SWL_OK) return st;
+  if (cudaMemcpyAsync(out_host, ws.out_dev, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemcpyAsync(expert_idx_host, ws.idx_dev, tb, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(gate_host, ws.gate_dev, tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemcpyAsync(pos_host, ws.pos_dev, tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemcpyAsync(aux_host, ws.aux_dev, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  return SWL_OK;
+}
+
+swl_status switch_layer_device_status(const void* workspace, void* stream) {
+  if (!workspace) return SWL_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SWL_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  return err == kDevOk ? SWL_OK : SWL_ERR_DEVICE;
+}
+
+const char* switch_layer_status_string(swl_status status) {
+  switch (status) {
+    case SWL_OK: return "ok";
+    case SWL_ERR_INVALID_ARG: return "invalid argument";
+    case SWL_ERR_UNSUPPORTED: return "unsupported shape, dtype or alignment";
+    case SWL_ERR_WORKSPACE: return "workspace too small";
+    case SWL_ERR_CUDA: return "CUDA runtime error";
+    case SWL_ERR_DEVICE: return "device-side failure reported by a kernel";
+  }
+  return "unknown status";
+}
+
+const char* switch_layer_stage_name(int k) {
+  static const char* names[SWL_NUM_STAGES] = {"router_logits", "router_softmax",
+                                              "dispatch_scan",  "dispatch_gather",
+                                              "expert_gemm1",   "expert_gemm2"};
+  return (k >= 0 && k < SWL_NUM_STAGES) ? names[k] : nullptr;
+}
+
+uint64_t switch_layer_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,249 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, on seeded inputs.
+
+Routing (expert_idx, pos_in_expert, drop mask) must match bit for bit; gate,
+aux loss and outputs within the stated tolerances (see helpers.py).  The five
+named workloads run at full size, in the launch configuration the bench uses;
+the two largest compare routing for every token and outputs on sampled tokens.
+"""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import sparse_mixture_experts_argmax_b200 as swl
+from sparse_mixture_experts_argmax_b200 import build as swl_build
+
+from helpers import check_close, check_routing, gap_redraws
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    swl_build.build()
+    swl.lib()
+
+
+def _run(inputs_gpu, cf):
+    out = swl.forward(inputs_gpu, cf)
+    torch.cuda.synchronize()
+    return out
+
+
+def _np(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _full_parity(spec: synth.LayerSpec, redraws, seed=0):
+    ig = synth.make_layer_inputs(spec, seed, device="cuda", redraws=redraws)
+    got = _run(ig, spec.cf)
+    ic = synth.make_layer_inputs(spec, seed, device="cpu", redraws=redraws)
+    ref = oracle.switch_forward(ic["x"], ic["W_r"], ic["W1"], ic["b1"], ic["W2"], ic["b2"],
+                                spec.cf, b_r=ic["b_r"])
+    C = oracle.capacity(spec.T, spec.N, spec.cf)
+    assert swl.switch_layer_capacity(spec.T, spec.N, spec.cf) == C
+    check_routing(got, ref, C, spec.T)
+    check_close(_np(got["out"]), ref["out"], spec.dtype)
+    return got, ref
+
+
+# ------------------------------------------------------------------ generator
+def test_generator_gpu_equals_cpu():
+    spec = synth.WORKLOADS["base_T4096_d768_N64"]
+    rd = synth.load_gap_redraws(spec.name)
+    xg = synth.make_x(spec, device="cuda", redraws=rd).cpu()
+    xc = synth.make_x(spec, device="cpu", redraws=rd)
+    assert torch.equal(xg, xc)
+    eg = synth.expert_slice(spec, [0, 17, 63], device="cuda")
+    ec = synth.expert_slice(spec, [0, 17, 63], device="cpu")
+    for k in eg:
+        assert torch.equal(eg[k].cpu(), ec[k]), k
+    rg = synth.make_router(spec, device="cuda")
+    assert torch.equal(rg["W_r"].cpu(), synth.make_router(spec)["W_r"])
+
+
+# ------------------------------------------------------------------ named workloads, full size
+@pytest.mark.parametrize("name", ["tiny_f32_T64_d32_N4", "base_T4096_d768_N64",
+                                  "large_T16384_d1024_N128"])
+def test_named_workload_full(name):
+    spec = synth.WORKLOADS[name]
+    rd = synth.load_gap_redraws(spec.name)
+    got, ref = _full_parity(spec, rd)
+    assert (~ref["kept"]).sum() >= 0
+
+
+def _sampled_parity(spec: synth.LayerSpec, n_sample: int, seed=0, extra_tokens=()):
+    rd = synth.load_gap_redraws(spec.name)
+    ig = synth.make_layer_inputs(spec, seed, device="cuda", redraws=rd)
+    got = _run(ig, spec.cf)
+    del ig
+    torch.cuda.empty_cache()
+    x = synth.make_x(spec, seed, redraws=rd)
+    r = synth.make_router(spec, seed)
+    rng = np.random.default_rng(1234)
+    sample = set(rng.choice(spec.T, size=n_sample, replace=False).tolist())
+    sample |= {0, spec.T - 1} | set(int(t) for t in extra_tokens)
+
+    @functools.lru_cache(maxsize=None)
+    def weights(e):
+        w = synth.expert_slice(spec, [e], seed)
+        return {k: v[0] for k, v in w.items()}
+
+    ref = oracle.switch_forward_sampled(x, r["W_r"], spec.cf, sorted(sample), weights,
+                                        b_r=r["b_r"])
+    check_routing(got, ref, ref["capacity"], spec.T)
+    toks = sorted(ref["out_rows"])
+    g = _np(got["out"][torch.tensor(toks, device=got["out"].device)])
+    want = np.stack([ref["out_rows"][t] for t in toks])
+    check_close(g, want, spec.dtype)
+    return got, ref
+
+
+def test_skewed_workload_sampled():
+    spec = synth.WORKLOADS["skewed_T32768_d2048_N64"]
+    # tokens of the lightly loaded experts, and expert 0's last kept / first dropped tokens
+    r = synth.make_router(spec)
+    x = synth.make_x(spec, redraws=synth.load_gap_redraws(spec.name))
+    e = np.argmax(oracle.router_logits(x, r["W_r"], r["b_r"]), axis=1)
+    others = np.nonzero(e != 0)[0][:96].tolist()
+    zero = np.nonzero(e == 0)[0]
+    C = oracle.capacity(spec.T, spec.N, spec.cf)
+    edge = zero[C - 3:C + 3].tolist()
+    got, ref = _sampled_parity(spec, 160, extra_tokens=others + edge)
+    assert (~ref["kept"]).sum() > 0
+
+
+def test_many_expert_workload_sampled():
+    spec = synth.WORKLOADS["many_T65536_d1024_N2048"]
+    _sampled_parity(spec, 80)
+
+
+# ------------------------------------------------------------------ random shapes, ragged tails
+def _random_specs():
+    rng = np.random.default_rng(2024)
+    specs = []
+    for i in range(10):
+        specs.append(synth.random_spec(rng, "rand_bf16_%d" % i, "bf16"))
+    for i in range(5):
+        specs.append(synth.random_spec(rng, "rand_f32_%d" % i, "f32", max_T=300))
+    return specs
+
+
+@pytest.mark.parametrize("spec", _random_specs(), ids=lambda s: "%s_T%d_d%d_f%d_N%d_cf%g" % (
+    s.name, s.T, s.d, s.d_ff, s.N, s.cf))
+def test_random_shapes(spec):
+    _full_parity(spec, gap_redraws(spec))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("case", ["one_token", "one_expert", "tiny_capacity", "no_drops",
+                                  "ragged_tiles", "wide_ffn"])
+def test_edge_cases(dtype, case):
+    shapes = {
+        "one_token": (1, 64, 128, 4, 1.0),
+        "one_expert": (300, 64, 128, 1, 1.0),       # dense FFN, gate 1
+        "tiny_capacity": (257, 64, 64, 3, 0.01),    # C = 1
+        "no_drops": (300, 48, 80, 5, 5.0),          # C = T
+        "ragged_tiles": (333, 200, 136, 6, 1.5),    # d, d_ff not multiples of 64 / 128
+        "wide_ffn": (130, 128, 1032, 2, 2.0),
+    }
+    T, d, d_ff, N, cf = shapes[case]
+    spec = synth.LayerSpec("edge_%s_%s" % (case, dtype), T, d, d_ff, N, cf, dtype, bias_std=0.05)
+    _full_parity(spec, gap_redraws(spec))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_collapse_multi_tile_expert(dtype):
+    """Every token picks expert 0 (router bias), C = T: one expert with several
+    256-row token tiles, the others empty."""
+    T, d, d_ff, N = 700, 64, 192, 4
+    spec = synth.LayerSpec("collapse_%s" % dtype, T, d, d_ff, N, float(N), dtype, bias_std=0.05)
+    rd = gap_redraws(spec)
+    ig = synth.make_layer_inputs(spec, device="cuda", redraws=rd)
+    ic = synth.make_layer_inputs(spec, device="cpu", redraws=rd)
+    b_r = torch.tensor([30.0] + [0.0] * (N - 1), dtype=torch.float32)
+    ig["b_r"], ic["b_r"] = b_r.cuda(), b_r
+    got = _run(ig, spec.cf)
+    ref = oracle.switch_forward(ic["x"], ic["W_r"], ic["W1"], ic["b1"], ic["W2"], ic["b2"],
+                                spec.cf, b_r=b_r)
+    assert np.all(ref["expert_idx"] == 0) and ref["kept"].all()
+    check_routing(got, ref, oracle.capacity(T, N, spec.cf), T)
+    check_close(_np(got["out"]), ref["out"], dtype)
+
+
+def test_empty_batch():
+    spec = synth.LayerSpec("empty", 0, 16, 16, 3, 1.0, "bf16")
+    ig = synth.make_layer_inputs(spec, device="cuda")
+    got = _run(ig, 1.0)
+    assert float(got["aux_loss"].cpu()[0]) == 0.0
+
+
+# ------------------------------------------------------------------ API variants and status
+def test_host_io_and_timed_variants_match():
+    spec = synth.WORKLOADS["base_T4096_d768_N64"]
+    ig = synth.make_layer_inputs(spec, device="cuda", redraws=synth.load_gap_redraws(spec.name))
+    a = _run(ig, spec.cf)
+    b = _run(ig, spec.cf)                  # repeat: deterministic
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+    T, d = ig["x"].shape
+    N, d_ff, _ = ig["W1"].shape
+    ws = swl.alloc_workspace(T, d, d_ff, N, ig["x"].dtype, spec.cf, host_io=True)
+    xh = ig["x"].cpu().pin_memory()
+    oh = {"out": torch.empty((T, d), dtype=ig["x"].dtype).pin_memory(),
+          "expert_idx": torch.empty(T, dtype=torch.int32).pin_memory(),
+          "gate": torch.empty(T, dtype=torch.float32).pin_memory(),
+          "pos_in_expert": torch.empty(T, dtype=torch.int32).pin_memory(),
+          "aux_loss": torch.empty(1, dtype=torch.float32).pin_memory()}
+    swl.switch_layer_forward_host_io(xh, ig["W_r"], ig["W1"], ig["b1"], ig["W2"], ig["b2"],
+                                     spec.cf, oh["out"], oh["expert_idx"], oh["gate"],
+                                     oh["pos_in_expert"], oh["aux_loss"], b_r=ig["b_r"],
+                                     workspace=ws)
+    torch.cuda.synchronize()
+    assert swl.switch_layer_device_status(ws) == 0
+    for k in a:
+        assert torch.equal(a[k].cpu(), oh[k]), k
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(swl.SWL_NUM_STAGES + 1)]
+    c = swl.alloc_outputs(T, d, ig["x"].dtype)
+    ws2 = swl.alloc_workspace(T, d, d_ff, N, ig["x"].dtype, spec.cf)
+    swl.switch_layer_forward(ig["x"], ig["W_r"], ig["W1"], ig["b1"], ig["W2"], ig["b2"], spec.cf,
+                             c["out"], c["expert_idx"], c["gate"], c["pos_in_expert"],
+                             c["aux_loss"], b_r=ig["b_r"], workspace=ws2, stage_events=evs)
+    torch.cuda.synchronize()
+    for k in a:
+        assert torch.equal(a[k], c[k]), k
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(swl.SWL_NUM_STAGES)]
+    assert all(t >= 0 for t in times)
+
+
+def test_small_workspace_is_rejected():
+    spec = synth.WORKLOADS["tiny_f32_T64_d32_N4"]
+    ig = synth.make_layer_inputs(spec, device="cuda")
+    o = swl.alloc_outputs(spec.T, spec.d, ig["x"].dtype)
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    before = swl.switch_layer_launch_count()
+    with pytest.raises(swl.SwitchLayerError) as ei:
+        swl.switch_layer_forward(ig["x"], ig["W_r"], ig["W1"], ig["b1"], ig["W2"], ig["b2"],
+                                 spec.cf, o["out"], o["expert_idx"], o["gate"],
+                                 o["pos_in_expert"], o["aux_loss"], workspace=ws)
+    assert ei.value.status == 3
+    assert swl.switch_layer_launch_count() == before
+
+
+def test_nonfinite_router_input_reports_device_status():
+    spec = synth.LayerSpec("nan_row", 200, 32, 64, 4, 1.0, "bf16")
+    ig = synth.make_layer_inputs(spec, device="cuda")
+    ig["x"][7] = float("nan")
+    with pytest.raises(swl.SwitchLayerError) as ei:
+        swl.forward(ig, spec.cf)
+    assert ei.value.status == 5
+    # the context is still usable
+    ig["x"][7] = 0.5
+    swl.forward(ig, spec.cf)
