@@ -27,7 +27,8 @@
  *  - Memory: every tensor pointer is a DEVICE pointer owned by the caller
  *    (except the *_host arguments of switch_layer_forward_host_io, which are
  *    host pointers, ideally pinned).  The library allocates nothing and keeps no
- *    state between calls besides a launch counter.
+ *    state between calls besides a launch counter and the fixed scratch array of
+ *    switch_layer_forward_noalloc.
  *  - Layouts: contiguous row-major.  x [T,d]; W_r [N,d] fp32; b_r [N] fp32;
  *    W1 [N,d_ff,d]; b1 [N,d_ff]; W2 [N,d,d_ff]; b2 [N,d]; out [T,d];
  *    expert_idx, pos_in_expert [T] int32; gate [T] fp32; aux_loss [1] fp32.
@@ -140,6 +141,38 @@ swl_status switch_layer_forward_host_io(int64_t T, int64_t d, int64_t d_ff, int6
  * failure (a bounded pipeline wait expired, or non-finite router logits).
  * SWL_ERR_CUDA if the synchronisation itself failed. */
 swl_status switch_layer_device_status(const void* workspace, void* stream);
+
+/* Bytes of the fixed device scratch used by switch_layer_forward_noalloc. */
+#define SWL_NOALLOC_MAX_BYTES (64u << 20)
+
+/* Forward pass for callers that cannot call cudaMalloc: plugin code running
+ * inside a host framework that owns all device memory and forbids allocations
+ * outside its own allocator, and latency-critical loops where an allocation (a
+ * synchronising, device-wide call) is not acceptable.  The paper has no
+ * counterpart of this entry point: it is switch_layer_forward
+ * with the workspace taken from a fixed-size static device array inside this
+ * library (SWL_NOALLOC_MAX_BYTES, held by every GPU that loads the library until
+ * the process exits).  Inputs and outputs are still passed by the caller, with
+ * the same meaning, layouts and checks as switch_layer_forward.
+ *  - Shapes whose workspace (switch_layer_workspace_size with flags 0) exceeds
+ *    SWL_NOALLOC_MAX_BYTES are rejected with SWL_ERR_WORKSPACE before anything
+ *    is enqueued.
+ *  - The first call on a device looks up the device address of the static
+ *    array for the current device (which must be the device of `stream`); make
+ *    that first call before any stream capture.
+ *  - All calls on a device share the one array, and it keeps the contents of the
+ *    last call; the call re-initialises what must start at zero.  Calls that
+ *    overlap on the GPU (different streams, or host threads without ordering)
+ *    race on the array and give wrong results: serialise them.
+ *  - Device-side failures of this variant are not visible to
+ *    switch_layer_device_status (it has no workspace pointer to read).
+ *  - Allocates nothing: no cudaMalloc / cudaFree or allocating library call. */
+swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                        const void* x, const float* W_r, const void* W1,
+                                        const void* b1, const void* W2, const void* b2,
+                                        double capacity_factor, void* out, int32_t* expert_idx,
+                                        float* gate, int32_t* pos_in_expert, float* aux_loss,
+                                        const float* b_r, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* switch_layer_status_string(swl_status status);

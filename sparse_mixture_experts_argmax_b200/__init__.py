@@ -31,7 +31,9 @@ STATUS = {0: "SWL_OK", 1: "SWL_ERR_INVALID_ARG", 2: "SWL_ERR_UNSUPPORTED",
 EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer_forward",
            "switch_layer_forward_timed", "switch_layer_forward_host_io",
            "switch_layer_device_status", "switch_layer_status_string",
-           "switch_layer_stage_name", "switch_layer_launch_count")
+           "switch_layer_stage_name", "switch_layer_launch_count",
+           "switch_layer_forward_noalloc")
+SWL_NOALLOC_MAX_BYTES = 64 << 20
 
 
 class SwitchLayerError(RuntimeError):
@@ -80,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_stage_name.argtypes = [_i32]
     L.switch_layer_launch_count.restype = ctypes.c_uint64
     L.switch_layer_launch_count.argtypes = []
+    L.switch_layer_forward_noalloc.restype = _i32
+    L.switch_layer_forward_noalloc.argtypes = _FWD_ARGS[:17] + [_vp, _vp]
     _lib = L
     return L
 

@@ -228,6 +228,27 @@ static swl_status forward_impl(int64_t T, int64_t d, int64_t d_ff, int64_t N, in
                      ev);
 }
 
+// ---------------------------------------------------------------- no-alloc scratch
+// Fixed device scratch for switch_layer_forward_noalloc.  In host code the
+// symbol is only a stand-in: its device address is looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SWL_NOALLOC_MAX_BYTES];
+
+static void* noalloc_scratch_for_current_device() {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* ptrs[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
 }  // namespace swl
 
 using namespace swl;
@@ -365,5 +386,23 @@ const char* switch_layer_stage_name(int k) {
 }
 
 uint64_t switch_layer_launch_count(void) { return g_launches.load(); }
+
+swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                        const void* x, const float* W_r, const void* W1,
+                                        const void* b1, const void* W2, const void* b2,
+                                        double capacity_factor, void* out, int32_t* expert_idx,
+                                        float* gate, int32_t* pos_in_expert, float* aux_loss,
+                                        const float* b_r, void* stream) {
+  Shape s;
+  const swl_status st = make_shape(T, d, d_ff, N, dtype, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (workspace_layout(s, false, 0, nullptr) > static_cast<size_t>(SWL_NOALLOC_MAX_BYTES))
+    return SWL_ERR_WORKSPACE;   // shape too large for the fixed scratch
+  void* scratch = noalloc_scratch_for_current_device();
+  if (scratch == nullptr) return SWL_ERR_CUDA;
+  return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
+                      expert_idx, gate, pos_in_expert, aux_loss, b_r, scratch,
+                      static_cast<size_t>(SWL_NOALLOC_MAX_BYTES), stream, nullptr);
+}
 
 }  // extern "C"
