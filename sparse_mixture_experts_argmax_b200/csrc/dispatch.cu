@@ -30,8 +30,37 @@
 namespace swl {
 namespace {
 
-constexpr int kScanThreads = 256;
+constexpr int kScanThreads = 512;
 constexpr int kScanWarps = kScanThreads / 32;
+
+// Inclusive warp scan (Hillis-Steele with shuffles; fixed order, deterministic).
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += u;
+  }
+  return v;
+}
+
+// Exclusive scan over the block of one int per thread; returns the exclusive
+// prefix and writes the block total to *total.  Uses s_warp[kScanWarps].
+__device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int incl = warp_incl_scan(v, lane);
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = lane < kScanWarps ? s_warp[lane] : 0;
+    const int wi = warp_incl_scan(w, lane);
+    if (lane < kScanWarps) s_warp[lane] = wi - w;   // exclusive warp offsets
+    if (lane == kScanWarps - 1) *total = wi;
+  }
+  __syncthreads();
+  const int r = s_warp[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
 
 __global__ void __launch_bounds__(kScanThreads)
 dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict__ blk_psum,
@@ -89,9 +118,9 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
   __threadfence();
 
   // ---- last CTA: scan over experts, tile prefix, aux loss
-  __shared__ int s_rows[kScanThreads];
-  __shared__ int s_tiles[kScanThreads];
-  __shared__ double s_aux[kScanThreads];
+  __shared__ int s_warp[kScanWarps];
+  __shared__ int s_tot_rows, s_tot_tiles;
+  __shared__ double s_aux[kScanWarps];
   const int chunk = (N + kScanThreads - 1) / kScanThreads;
   const int e0 = threadIdx.x * chunk, e1 = min(N, e0 + chunk);
   int rows = 0, tiles = 0;
@@ -103,71 +132,80 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     tiles += (m + tile_rows - 1) / tile_rows;
     aux += (double)c * __ldcg(psum64 + i);
   }
-  s_rows[threadIdx.x] = rows;
-  s_tiles[threadIdx.x] = tiles;
-  s_aux[threadIdx.x] = aux;
+  int base_rows = block_excl_scan(rows, s_warp, &s_tot_rows);
+  int base_tiles = block_excl_scan(tiles, s_warp, &s_tot_tiles);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) aux += __shfl_xor_sync(0xffffffffu, aux, off);
+  if (lane == 0) s_aux[warp] = aux;
   __syncthreads();
   if (threadIdx.x == 0) {
-    // serial exclusive scan over the 256 partials (fixed order, deterministic)
-    int r = 0, t = 0;
     double a = 0.0;
-    for (int i = 0; i < kScanThreads; ++i) {
-      const int rr = s_rows[i], tt = s_tiles[i];
-      s_rows[i] = r;
-      s_tiles[i] = t;
-      r += rr;
-      t += tt;
-      a += s_aux[i];
-    }
-    tile_prefix[N] = t;
+    for (int w = 0; w < kScanWarps; ++w) a += s_aux[w];
+    tile_prefix[N] = s_tot_tiles;
     // aux = N * sum_i (count_i / T) * (psum_i / T)
     *aux_loss = (float)((double)N * a / ((double)T * (double)T));
     hdr->done = 0u;   // ready for the next call
   }
-  __syncthreads();
-  rows = s_rows[threadIdx.x];
-  tiles = s_tiles[threadIdx.x];
   for (int i = e0; i < e1; ++i) {
     const int m = min(__ldcg(exp_count + i), C_eff);
     exp_rows[i] = m;
-    exp_base[i] = rows;
-    tile_prefix[i] = tiles;
-    rows += m;
-    tiles += (m + tile_rows - 1) / tile_rows;
+    exp_base[i] = base_rows;
+    tile_prefix[i] = base_tiles;
+    base_rows += m;
+    base_tiles += (m + tile_rows - 1) / tile_rows;
   }
 }
 
 constexpr int kGatherThreads = 256;
 constexpr int kGatherWarps = kGatherThreads / 32;
+constexpr int kGatherMaxVecPerLane = 8;   // rows up to 8 x 32 x 16 B = 4 KiB held in registers
 
 // One warp per token.  VEC = bytes per vector move (16 for bf16 rows, 4 for fp32).
+// The token's row is loaded before its destination is known (it does not depend
+// on the routing), then either stored to its packed expert row or dropped and
+// the output row zeroed.
 template <int VEC>
 __global__ void __launch_bounds__(kGatherThreads)
 dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ expert_idx,
                        int* __restrict__ pos_in_expert, const int* __restrict__ blk_off,
                        const int* __restrict__ exp_base, int* __restrict__ slot_token,
                        uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out, int T, int N,
-                       int C_eff, int row_bytes, WsHeader* hdr) {
+                       int C_eff, int row_bytes, int tpb, WsHeader* hdr) {
+  using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kGatherWarps + warp;
   if (t >= T) return;
+  const int nv = row_bytes / VEC;
+  const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
+  V reg[kGatherMaxVecPerLane];
+  const bool in_regs = nv <= 32 * kGatherMaxVecPerLane;
+  if (in_regs) {
+#pragma unroll
+    for (int j = 0; j < kGatherMaxVecPerLane; ++j)
+      if (lane + 32 * j < nv) reg[j] = src[lane + 32 * j];
+  }
   const int e = expert_idx[t];
+  const int rank = pos_in_expert[t];            // holds the in-block rank
   if (e < 0 || e >= N) {          // cannot happen: the router clamps its choice
     if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
     return;
   }
-  const int b = t / kTokensPerBlock;
-  const int pos = blk_off[(size_t)b * N + e] + pos_in_expert[t];   // holds the in-block rank
+  const int b = t / tpb;
+  const int pos = blk_off[(size_t)b * N + e] + rank;
+  const int base = exp_base[e];
   __syncwarp();
   if (lane == 0) pos_in_expert[t] = pos;
-  using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
-  const int nv = row_bytes / VEC;
   if (pos < C_eff) {
-    const int row = exp_base[e] + pos;
+    const int row = base + pos;
     if (lane == 0) slot_token[row] = t;
-    const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
     V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
-    for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kGatherMaxVecPerLane; ++j)
+        if (lane + 32 * j < nv) dst[lane + 32 * j] = reg[j];
+    } else {
+      for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    }
   } else {
     V* dst = reinterpret_cast<V*>(out + (size_t)t * row_bytes);
     V z;
@@ -201,12 +239,12 @@ cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const vo
     dispatch_gather_kernel<16><<<grid, kGatherThreads, 0, stream>>>(
         static_cast<const uint8_t*>(x), expert_idx, pos_in_expert, ws.blk_off, ws.exp_base,
         ws.slot_token, static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
-        (int)s.N, (int)s.C_eff, row_bytes, ws.hdr);
+        (int)s.N, (int)s.C_eff, row_bytes, s.tpb, ws.hdr);
   else
     dispatch_gather_kernel<4><<<grid, kGatherThreads, 0, stream>>>(
         static_cast<const uint8_t*>(x), expert_idx, pos_in_expert, ws.blk_off, ws.exp_base,
         ws.slot_token, static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
-        (int)s.N, (int)s.C_eff, row_bytes, ws.hdr);
+        (int)s.N, (int)s.C_eff, row_bytes, s.tpb, ws.hdr);
   count_launch();
   return cudaGetLastError();
 }

@@ -17,7 +17,7 @@ enum DeviceError : int {
   kDevNonFiniteLogits = 3,   // a token had no finite maximum logit (NaN/Inf input)
 };
 
-constexpr int kTokensPerBlock = 128;   // token block of the softmax / rank / gather stages
+constexpr int kTokensPerBlock = 128;   // largest token block of the softmax / rank / gather stages
 constexpr int kMaxExperts = 1 << 20;
 
 // Workspace header (256 bytes at offset 0).
@@ -30,7 +30,7 @@ struct WsHeader {
 // Device pointers carved out of the caller's workspace.
 struct Workspace {
   WsHeader* hdr;
-  float* logits;        // [T, N] fp32
+  float* logits;        // [ksplit_eff, T, N] fp32 partial logits (slice 0 reused for p)
   int* blk_count;       // [nblk, N] tokens of block b routed to expert e
   int* blk_off;         // [nblk, N] tokens of earlier blocks routed to e
   float* blk_psum;      // [nblk, N] sum over block b of p_{t,e}
@@ -57,17 +57,24 @@ struct Shape {
   int dtype;      // 0 = fp32, 1 = bf16
   int64_t C;      // capacity (formula value)
   int64_t C_eff;  // min(C, T): rows an expert can actually keep
-  int nblk;       // ceil(T / kTokensPerBlock)
+  int tpb;        // tokens per block of the softmax / rank / gather stages (<= kTokensPerBlock)
+  int nblk;       // ceil(T / tpb)
+  int kslice;     // K elements per slice of the router logits GEMM (multiple of 16)
+  int ksplit_eff; // K slices of the router logits GEMM (partials summed by the softmax)
   int tile_rows;  // token rows per GEMM tile (N of the UMMA, or the SIMT tile)
 };
+
+// Router logits K slice length for a shape (a pure function of the shape).
+int router_kslice(int64_t T, int64_t d, int64_t N);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 
 // ---- stage launchers (all asynchronous on `stream`; return cudaGetLastError()).
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
                                  const float* W_r, const float* b_r, cudaStream_t stream);
-cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, int* expert_idx,
-                                  float* gate, int* local_rank, cudaStream_t stream);
+cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
+                                  int* expert_idx, float* gate, int* local_rank,
+                                  cudaStream_t stream);
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
                                  cudaStream_t stream);
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,

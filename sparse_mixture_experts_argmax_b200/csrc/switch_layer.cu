@@ -40,7 +40,7 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   };
   Workspace w{};
   w.hdr = reinterpret_cast<WsHeader*>(take(sizeof(WsHeader)));
-  w.logits = reinterpret_cast<float*>(take(T * N * 4));
+  w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(s.ksplit_eff) * T * N * 4));
   w.blk_count = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_off = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_psum = reinterpret_cast<float*>(take(nb * N * 4));
@@ -130,7 +130,13 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->dtype = dtype;
   s->C = switch_layer_capacity(T, N, cf);
   s->C_eff = s->C < T ? s->C : T;
-  s->nblk = static_cast<int>((T + kTokensPerBlock - 1) / kTokensPerBlock);
+  // token block: the largest of 128/64/32 that still gives >= 2 CTAs per SM
+  s->tpb = 32;
+  for (int tpb = kTokensPerBlock; tpb > 32; tpb /= 2)
+    if ((T + tpb - 1) / tpb >= 2 * 148) { s->tpb = tpb; break; }
+  s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
+  s->kslice = router_kslice(T, d, N);
+  s->ksplit_eff = static_cast<int>((d + s->kslice - 1) / s->kslice);
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
   return SWL_OK;
 }
@@ -146,7 +152,7 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
   if (!rec(0)) return SWL_ERR_CUDA;
   if (launch_router_logits(s, ws, x, W_r, b_r, stream) != cudaSuccess) return SWL_ERR_CUDA;
   if (!rec(1)) return SWL_ERR_CUDA;
-  if (launch_router_softmax(s, ws, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
+  if (launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
     return SWL_ERR_CUDA;
   if (!rec(2)) return SWL_ERR_CUDA;
   if (launch_dispatch_scan(s, ws, aux_loss, stream) != cudaSuccess) return SWL_ERR_CUDA;
