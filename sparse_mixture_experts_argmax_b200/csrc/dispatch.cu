@@ -72,18 +72,33 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
   __shared__ int wc[kScanWarps][32];
   __shared__ double wp[kScanWarps][32];
   __shared__ int is_last;
+  pdl_trigger();
+  pdl_wait();   // block statistics come from the router
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * 32 + lane;
   const int per = (nblk + kScanWarps - 1) / kScanWarps;
   const int b0 = warp * per, b1 = min(nblk, b0 + per);
 
-  // pass 1: this warp's share of blocks, per expert (lane)
+  // pass 1: this warp's share of blocks, per expert (lane); the counts of up to
+  // kRegBlocks blocks stay in registers for pass 2, loads issued before use
+  constexpr int kRegBlocks = 16;
+  int creg[kRegBlocks];
   int csum = 0;
   double psum = 0.0;
   if (e < N) {
-    for (int b = b0; b < b1; ++b) {
-      csum += blk_count[(size_t)b * N + e];
-      psum += (double)blk_psum[(size_t)b * N + e];
+    for (int bb = b0; bb < b1; bb += kRegBlocks) {
+      float preg[kRegBlocks];
+#pragma unroll
+      for (int j = 0; j < kRegBlocks; ++j) {
+        const int b = bb + j;
+        creg[j] = b < b1 ? blk_count[(size_t)b * N + e] : 0;
+        preg[j] = b < b1 ? blk_psum[(size_t)b * N + e] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < kRegBlocks; ++j) {
+        csum += creg[j];
+        psum += (double)preg[j];
+      }
     }
   }
   wc[warp][lane] = csum;
@@ -93,11 +108,22 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
   if (e < N) {
     int off = 0;
     for (int w = 0; w < warp; ++w) off += wc[w][lane];
-    for (int b = b0; b < b1; ++b) {
-      const size_t i = (size_t)b * N + e;
-      const int c = blk_count[i];
-      blk_off[i] = off;
-      off += c;
+    if (b1 - b0 <= kRegBlocks) {
+#pragma unroll
+      for (int j = 0; j < kRegBlocks; ++j) {
+        const int b = b0 + j;
+        if (b < b1) {
+          blk_off[(size_t)b * N + e] = off;
+          off += creg[j];
+        }
+      }
+    } else {
+      for (int b = b0; b < b1; ++b) {
+        const size_t i = (size_t)b * N + e;
+        const int c = blk_count[i];
+        blk_off[i] = off;
+        off += c;
+      }
     }
     if (warp == 0) {
       int tot = 0;
@@ -172,6 +198,8 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
                        uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out, int T, int N,
                        int C_eff, int row_bytes, int tpb, WsHeader* hdr) {
   using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
+  pdl_trigger();
+  pdl_wait();   // offsets come from the scan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kGatherWarps + warp;
   if (t >= T) return;
@@ -219,11 +247,12 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
                                  cudaStream_t stream) {
   const int grid = (int)((s.N + 31) / 32);
-  dispatch_scan_kernel<<<grid, kScanThreads, 0, stream>>>(
-      ws.blk_count, ws.blk_psum, ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base,
-      ws.tile_prefix, aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows);
+  const cudaError_t e = launch_dependent(
+      dispatch_scan_kernel, dim3(grid), dim3(kScanThreads), 0, stream, ws.blk_count, ws.blk_psum,
+      ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base, ws.tile_prefix, aux_loss,
+      ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
@@ -235,18 +264,14 @@ cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const vo
   const bool vec16 = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0) &&
                      ((reinterpret_cast<uintptr_t>(out) & 15) == 0) &&
                      ((reinterpret_cast<uintptr_t>(ws.xbuf) & 15) == 0);
-  if (vec16)
-    dispatch_gather_kernel<16><<<grid, kGatherThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(x), expert_idx, pos_in_expert, ws.blk_off, ws.exp_base,
-        ws.slot_token, static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
-        (int)s.N, (int)s.C_eff, row_bytes, s.tpb, ws.hdr);
-  else
-    dispatch_gather_kernel<4><<<grid, kGatherThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(x), expert_idx, pos_in_expert, ws.blk_off, ws.exp_base,
-        ws.slot_token, static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
-        (int)s.N, (int)s.C_eff, row_bytes, s.tpb, ws.hdr);
+  const cudaError_t e = launch_dependent(
+      vec16 ? dispatch_gather_kernel<16> : dispatch_gather_kernel<4>, dim3(grid),
+      dim3(kGatherThreads), 0, stream, static_cast<const uint8_t*>(x), expert_idx, pos_in_expert,
+      static_cast<const int*>(ws.blk_off), static_cast<const int*>(ws.exp_base), ws.slot_token,
+      static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T, (int)s.N,
+      (int)s.C_eff, row_bytes, s.tpb, ws.hdr);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace swl

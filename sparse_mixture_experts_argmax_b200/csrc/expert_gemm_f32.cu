@@ -27,6 +27,8 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
                        float* __restrict__ out, int num_experts, int M, int K, int mode) {
   __shared__ float As[kTile][kTile + 1];   // [row][k]
   __shared__ float Ws[kTile][kTile + 1];   // [feature][k]
+  pdl_trigger();
+  pdl_wait();   // packed rows and tile prefix come from the dispatch
   const int g = blockIdx.x;
   if (g >= tile_prefix[num_experts]) return;
   int lo = 0, hi = num_experts;            // last e with prefix[e] <= g
@@ -86,12 +88,14 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
   // upper bound on row tiles: sum_e ceil(m_e / 32) <= T / 32 + N
   const int64_t max_tiles = (s.T + kTile - 1) / kTile + s.N;
   dim3 grid(static_cast<unsigned>(max_tiles), (M + kTile - 1) / kTile);
-  expert_gemm_f32_kernel<<<grid, 256, 0, stream>>>(
-      act, static_cast<const float*>(W), static_cast<const float*>(bias), ws.tile_prefix,
-      ws.exp_rows, ws.exp_base, ws.slot_token, gate, static_cast<float*>(out),
+  const cudaError_t e = launch_dependent(
+      expert_gemm_f32_kernel, grid, dim3(256), 0, stream, act, static_cast<const float*>(W),
+      static_cast<const float*>(bias), static_cast<const int*>(ws.tile_prefix),
+      static_cast<const int*>(ws.exp_rows), static_cast<const int*>(ws.exp_base),
+      static_cast<const int*>(ws.slot_token), gate, static_cast<float*>(out),
       static_cast<int>(s.N), M, K, which);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace swl

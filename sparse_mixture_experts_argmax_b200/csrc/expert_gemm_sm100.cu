@@ -113,7 +113,13 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = __ldg(args.tile_prefix + args.num_experts) * args.m_tiles;
+  pdl_trigger();
+  if (threadIdx.x == 0) {   // independent of the previous kernel: overlaps its tail
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  pdl_wait();   // tile prefix, packed rows and gate come from earlier kernels
+  const int total = args.tile_prefix[args.num_experts] * args.m_tiles;
   if (static_cast<int>(blockIdx.x) >= total) return;   // uniform per CTA: nothing to do
 
   if (threadIdx.x == 0) {
@@ -129,8 +135,6 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
-    ptx::prefetch_tmap(&tmA);
-    ptx::prefetch_tmap(&tmB);
   }
   if (warp == 2) {
     ptx::tmem_alloc(tmem_slot, kTmemCols);
@@ -332,9 +336,10 @@ cudaError_t launch_expert_gemm_bf16(const Shape& s, const Workspace& ws, int whi
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  expert_gemm_sm100_kernel<<<num_sms, kThreads, smem, stream>>>(tmA, tmB, a);
+  err = launch_dependent(expert_gemm_sm100_kernel, dim3(num_sms), dim3(kThreads), smem, stream,
+                         tmA, tmB, a);
   count_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace swl

@@ -64,14 +64,20 @@ struct Shape {
   int tile_rows;  // token rows per GEMM tile (N of the UMMA, or the SIMT tile)
 };
 
-// Router logits K slice length for a shape (a pure function of the shape).
+// Router logits K slice length for a shape (a pure function of the shape), and
+// the tokens per tile (= per dispatch block) of the fused router (N <= 128).
 int router_kslice(int64_t T, int64_t d, int64_t N);
+int fused_router_tile_tokens(int64_t N);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 
 // ---- stage launchers (all asynchronous on `stream`; return cudaGetLastError()).
+// N <= kFusedRouterMaxN: one fused kernel (logits + softmax + block statistics);
+// launch_router_softmax is then not called.  Wider N: logits here, softmax after.
+constexpr int kFusedRouterMaxN = 128;
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
-                                 const float* W_r, const float* b_r, cudaStream_t stream);
+                                 const float* W_r, const float* b_r, int* expert_idx, float* gate,
+                                 int* local_rank, cudaStream_t stream);
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);
@@ -94,5 +100,32 @@ constexpr int kF32TileRows = 32;
 
 // Number of kernel launches issued by this library since load.
 void count_launch(int n = 1);
+
+// Programmatic dependent launch: a kernel launched with launch_dependent() may
+// start while the previous kernel on the stream is still finishing; it must call
+// pdl_wait() before touching memory that kernel reads or writes.  Every kernel
+// calls pdl_trigger() early so that its dependent can be scheduled.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+#endif
 
 }  // namespace swl

@@ -18,6 +18,7 @@
 
 #include "kernels.h"
 
+
 namespace swl {
 namespace {
 
@@ -52,32 +53,22 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* row, int k, int d, bo
   }
 }
 
-// Partial logits over one K slice: zpart[ks][t][n] = sum_{k in slice ks} x[t,k] W_r[n,k].
-// CTA tile BM tokens x BN experts, (BM/8)*(BN/8) threads with 8 x 8 outputs each,
-// K staged through shared memory in chunks of 16 with register prefetch of the
-// next chunk.  Splitting K (blockIdx.z) gives enough CTAs to fill the GPU when T
-// and N are small; the softmax kernel adds the slices in order, then the bias.
+// Main loop of one logits tile: acc[i][j] = sum_{k in [k_lo, k_hi)} x[m0 + ty*8 + i, k] *
+// W_r[n(j), k] with n(j) = n0 + tx*4 + j for j < 4 and n0 + BN/2 + tx*4 + (j-4) for
+// j >= 4 (the two halves keep the float4 reads of a quarter-warp on distinct banks).  THREADS = (BM/8)*(BN/8) threads with 8 x 8 outputs each; K
+// staged through shared memory (As[2][kBK][BM], Bs[2][kBK][BN], transposed so the
+// inner loop reads float4 vectors) in chunks of 16 with register prefetch of the
+// next chunk.  Rows >= T, experts >= N and k >= k_hi read as zero.
 template <typename TX, int BM, int BN>
-__global__ void __launch_bounds__((BM / 8) * (BN / 8))
-router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
-                     float* __restrict__ zpart, int T, int d, int N, int kslice,
-                     WsHeader* hdr) {
+__device__ __forceinline__ void logits_mainloop(const TX* __restrict__ x,
+                                                const float* __restrict__ W_r, int T, int d, int N,
+                                                int m0, int n0, int k_lo, int k_hi,
+                                                float (*As)[kBK][BM], float (*Bs)[kBK][BN],
+                                                float (&acc)[8][8]) {
   constexpr int kThreads = (BM / 8) * (BN / 8);
-  __shared__ __align__(16) float As[2][kBK][BM];
-  __shared__ __align__(16) float Bs[2][kBK][BN];
-
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
-    hdr->err = kDevOk;   // per-call device status
-    hdr->done = 0u;      // arrival counter of the dispatch scan
-  }
-
   const int tid = threadIdx.x;
   const int tx = tid % (BN / 8);
   const int ty = tid / (BN / 8);
-  const int m0 = blockIdx.x * BM;
-  const int n0 = blockIdx.y * BN;
-  const int k_lo = blockIdx.z * kslice;
-  const int k_hi = min(d, k_lo + kslice);
   const bool xvec = ((d * (int)sizeof(TX)) % 16 == 0) &&
                     ((reinterpret_cast<uintptr_t>(x) & 15) == 0);
   const bool wvec = ((d % 4) == 0) && ((reinterpret_cast<uintptr_t>(W_r) & 15) == 0);
@@ -139,13 +130,13 @@ router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
     }
   };
 
-  float acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
   const int nk = (k_hi - k_lo + kBK - 1) / kBK;
+  if (nk <= 0) return;
   gload(k_lo);
   sstore(0);
   __syncthreads();
@@ -158,9 +149,9 @@ router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
       *reinterpret_cast<float4*>(&a[0]) = *reinterpret_cast<const float4*>(&As[buf][k][ty * 8]);
       *reinterpret_cast<float4*>(&a[4]) =
           *reinterpret_cast<const float4*>(&As[buf][k][ty * 8 + 4]);
-      *reinterpret_cast<float4*>(&b[0]) = *reinterpret_cast<const float4*>(&Bs[buf][k][tx * 8]);
+      *reinterpret_cast<float4*>(&b[0]) = *reinterpret_cast<const float4*>(&Bs[buf][k][tx * 4]);
       *reinterpret_cast<float4*>(&b[4]) =
-          *reinterpret_cast<const float4*>(&Bs[buf][k][tx * 8 + 4]);
+          *reinterpret_cast<const float4*>(&Bs[buf][k][BN / 2 + tx * 4]);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -169,22 +160,52 @@ router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
     if (kc + 1 < nk) sstore(buf ^ 1);
     __syncthreads();
   }
+}
 
+// Partial logits over one K slice: zpart[ks][t][n] = sum_{k in slice ks} x[t,k] W_r[n,k]
+// (used when N is too wide for one CTA to hold a token's whole row; the softmax
+// kernel adds the slices in order, then the bias).
+template <typename TX, int BM, int BN>
+__global__ void __launch_bounds__((BM / 8) * (BN / 8))
+router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
+                     float* __restrict__ zpart, int T, int d, int N, int kslice,
+                     WsHeader* hdr) {
+  __shared__ __align__(16) float As[2][kBK][BM];
+  __shared__ __align__(16) float Bs[2][kBK][BN];
+  pdl_trigger();
+  pdl_wait();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
+    hdr->err = kDevOk;   // per-call device status
+    hdr->done = 0u;      // arrival counter of the dispatch scan
+  }
+  const int tx = threadIdx.x % (BN / 8);
+  const int ty = threadIdx.x / (BN / 8);
+  const int m0 = blockIdx.x * BM;
+  const int n0 = blockIdx.y * BN;
+  const int k_lo = blockIdx.z * kslice;
+  const int k_hi = min(d, k_lo + kslice);
+  float acc[8][8];
+  logits_mainloop<TX, BM, BN>(x, W_r, T, d, N, m0, n0, k_lo, k_hi, As, Bs, acc);
+
+  // lane tx holds experts n0 + tx*4 + {0..3} and n0 + BN/2 + tx*4 + {0..3}
   float* zs = zpart + (size_t)blockIdx.z * T * N;
   const bool vec_out = (N % 4) == 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int t = m0 + ty * 8 + i;
     if (t >= T) continue;
-    float* zr = zs + (size_t)t * N + n0 + tx * 8;
-    if (vec_out && n0 + tx * 8 + 8 <= N) {
-      *reinterpret_cast<float4*>(zr) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-      *reinterpret_cast<float4*>(zr + 4) =
-          make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-    } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (n0 + tx * 8 + j < N) zr[j] = acc[i][j];
+    for (int h = 0; h < 2; ++h) {
+      const int nb = n0 + h * (BN / 2) + tx * 4;
+      float* zr = zs + (size_t)t * N + nb;
+      if (vec_out && nb + 4 <= N) {
+        *reinterpret_cast<float4*>(zr) =
+            make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (nb + j < N) zr[j] = acc[i][4 * h + j];
+      }
     }
   }
 }
@@ -233,6 +254,8 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
   float* s_psum = smem_f + N;             // [kSoftmaxWarps][N]
   __shared__ int eid[kTokensPerBlock];
   __shared__ int lead_count[kTokensPerBlock];
+  pdl_trigger();
+  pdl_wait();   // partial logits come from the logits kernel
   const int b = blockIdx.x;
   const int t0 = b * tpb;
   const int ntok = min(tpb, T - t0);
@@ -327,6 +350,8 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
                            WsHeader* hdr) {
   __shared__ int eid[kTokensPerBlock];
   __shared__ int lead_count[kTokensPerBlock];
+  pdl_trigger();
+  pdl_wait();   // partial logits come from the logits kernel
   const int b = blockIdx.x;
   const int t0 = b * tpb;
   const int ntok = min(tpb, T - t0);
@@ -392,6 +417,259 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
   }
 }
 
+// Fused router for N <= BN (BN = 32, 64 or 128): logits, softmax, argmax and the
+// block statistics in one kernel, one CTA per tile of TM = 2048/BN tokens.
+// The 8 warps split K: warp w accumulates the whole TM x BN tile over the
+// K chunks c = w, w+8, ... (8 x 8 register outer products per lane, staged
+// through warp-private shared memory, so the main loop has no block barrier).
+// The 8 partial tiles are then summed in warp order (deterministic), the bias
+// added, and each token's softmax run by one warp.  The tile's TM tokens form
+// one token block of the dispatch statistics.
+template <typename TX, int BN>
+__global__ void __launch_bounds__(256)
+router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
+                    const float* __restrict__ b_r, int T, int d, int N,
+                    int* __restrict__ expert_idx, float* __restrict__ gate,
+                    int* __restrict__ local_rank, int* __restrict__ blk_count,
+                    float* __restrict__ blk_psum, WsHeader* hdr) {
+  constexpr int kWarps = 8;
+  constexpr int TM = 2048 / BN;                 // tokens per tile
+  constexpr int KC = BN <= 64 ? 16 : 8;         // K per chunk
+  constexpr int TXN = BN / 8;                   // lanes along the expert axis
+  constexpr int NPL = (BN + 31) / 32;           // logits per lane in the softmax
+  constexpr int XS = TM * KC / 8;               // x slots of 8 k-values per chunk
+  constexpr int WS = BN * KC / 4;               // W_r slots of 4 k-values per chunk
+  constexpr int XPER = (XS + 31) / 32, WPER = (WS + 31) / 32;
+  constexpr int STAGE = KC * (TM + BN);         // floats per warp buffer
+  static_assert(TM * BN == 32 * 64, "one warp holds the whole tile");
+  extern __shared__ __align__(16) float fsm[];
+  __shared__ int eid[kTokensPerBlock];
+  __shared__ int lead_count[kTokensPerBlock];
+  __shared__ float s_psum[kWarps][BN];
+
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    hdr->err = kDevOk;   // per-call device status
+    hdr->done = 0u;      // arrival counter of the dispatch scan
+  }
+  const int t0 = blockIdx.x * TM;
+  float* wbuf = fsm + warp * 2 * STAGE;         // this warp's two staging buffers
+  const int tx = lane % TXN, ty = lane / TXN;
+  const bool xvec = ((d * (int)sizeof(TX)) % 16 == 0) &&
+                    ((reinterpret_cast<uintptr_t>(x) & 15) == 0);
+  const bool wvec = ((d % 4) == 0) && ((reinterpret_cast<uintptr_t>(W_r) & 15) == 0);
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  float rx[XPER][8];
+  float4 rw[WPER];
+  auto gload = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < XPER; ++q) {
+      const int sl = lane + 32 * q;
+      if (sl < XS) {
+        const int m = sl % TM, kq = sl / TM;
+        const int t = t0 + m;
+        if (t < T) {
+          load8(x + (size_t)t * d, k0 + kq * 8, d, xvec, rx[q]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) rx[q][j] = 0.f;
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < WPER; ++q) {
+      const int sl = lane + 32 * q;
+      if (sl < WS) {
+        const int n = sl % BN, kq = sl / BN;
+        const int k = k0 + kq * 4;
+        const float* wr = W_r + (size_t)n * d;
+        if (n >= N) {
+          rw[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else if (wvec && k + 4 <= d) {
+          rw[q] = *reinterpret_cast<const float4*>(wr + k);
+        } else {
+          rw[q] = make_float4(k < d ? wr[k] : 0.f, k + 1 < d ? wr[k + 1] : 0.f,
+                              k + 2 < d ? wr[k + 2] : 0.f, k + 3 < d ? wr[k + 3] : 0.f);
+        }
+      }
+    }
+  };
+  auto sstore = [&](float* buf) {
+    float* As = buf;              // [KC][TM]
+    float* Bs = buf + KC * TM;    // [KC][BN]
+#pragma unroll
+    for (int q = 0; q < XPER; ++q) {
+      const int sl = lane + 32 * q;
+      if (sl < XS) {
+        const int m = sl % TM, kq = sl / TM;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) As[(kq * 8 + j) * TM + m] = rx[q][j];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < WPER; ++q) {
+      const int sl = lane + 32 * q;
+      if (sl < WS) {
+        const int n = sl % BN, kq = sl / BN;
+        Bs[(kq * 4 + 0) * BN + n] = rw[q].x;
+        Bs[(kq * 4 + 1) * BN + n] = rw[q].y;
+        Bs[(kq * 4 + 2) * BN + n] = rw[q].z;
+        Bs[(kq * 4 + 3) * BN + n] = rw[q].w;
+      }
+    }
+  };
+
+  const int nchunks = (d + KC - 1) / KC;
+  int buf = 0;
+  if (warp < nchunks) {
+    gload(warp * KC);
+    sstore(wbuf);
+    __syncwarp();
+    for (int c = warp; c < nchunks; c += kWarps) {
+      const bool more = c + kWarps < nchunks;
+      if (more) gload((c + kWarps) * KC);
+      const float* As = wbuf + buf * STAGE;
+      const float* Bs = As + KC * TM;
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        float a[8], b[8];
+        *reinterpret_cast<float4*>(&a[0]) = *reinterpret_cast<const float4*>(&As[k * TM + ty * 8]);
+        *reinterpret_cast<float4*>(&a[4]) =
+            *reinterpret_cast<const float4*>(&As[k * TM + ty * 8 + 4]);
+        *reinterpret_cast<float4*>(&b[0]) = *reinterpret_cast<const float4*>(&Bs[k * BN + tx * 4]);
+        *reinterpret_cast<float4*>(&b[4]) =
+            *reinterpret_cast<const float4*>(&Bs[k * BN + BN / 2 + tx * 4]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      }
+      if (more) {
+        buf ^= 1;
+        sstore(wbuf + buf * STAGE);
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();   // all warps are done with their staging buffers
+
+  // partial tiles P[w][TM][BN] (aliases the staging area), summed in warp order
+  float* P = fsm;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float* pr = P + (size_t)warp * TM * BN + (ty * 8 + i) * BN + tx * 4;
+    *reinterpret_cast<float4*>(pr) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    *reinterpret_cast<float4*>(pr + BN / 2) =
+        make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < TM * BN; idx += 256) {
+    float v = P[idx];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) v += P[(size_t)w * TM * BN + idx];
+    const int n = idx % BN;
+    P[idx] = (n < N) ? v + (b_r ? b_r[n] : 0.f) : -INFINITY;   // in place: Z = P[0]
+  }
+  __syncthreads();
+
+  // softmax, one warp per token
+  const int ntok = max(0, min(TM, T - t0));
+  float pacc[NPL];
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) pacc[j] = 0.f;
+  for (int i = warp; i < TM; i += kWarps) {
+    if (i >= ntok) {
+      if (lane == 0) eid[i] = -1;
+      continue;
+    }
+    float v[NPL];
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      const int n = lane + 32 * j;
+      v[j] = (n < BN) ? P[i * BN + n] : -INFINITY;
+    }
+    float best = -INFINITY;
+    int bidx = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+      if (v[j] > best) { best = v[j]; bidx = lane + 32 * j; }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+      if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+    }
+    float ssum = 0.f;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      v[j] = (lane + 32 * j < N) ? expf(v[j] - best) : 0.f;
+      ssum += v[j];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+    const float inv = 1.0f / ssum;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) pacc[j] += v[j] * inv;
+    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
+      bidx = 0;
+      if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
+    }
+    if (lane == 0) {
+      expert_idx[t0 + i] = bidx;
+      gate[t0 + i] = inv;       // p at the argmax: exp(0) / s
+      eid[i] = bidx;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    const int n = lane + 32 * j;
+    if (n < BN) s_psum[warp][n] = pacc[j];
+  }
+  __syncthreads();
+  block_ranks(eid, lead_count, ntok, TM, t0, local_rank);
+  const int b = blockIdx.x;
+  int* cnt_row = blk_count + (size_t)b * N;
+  float* ps_row = blk_psum + (size_t)b * N;
+  for (int n = threadIdx.x; n < N; n += 256) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) a += s_psum[w][n];
+    ps_row[n] = a;
+    cnt_row[n] = 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < ntok; i += 256) {
+    if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
+  }
+}
+
+template <typename TX, int BN>
+cudaError_t launch_fused_t(const Shape& s, const Workspace& ws, const void* x, const float* W_r,
+                           const float* b_r, int* expert_idx, float* gate, int* local_rank,
+                           cudaStream_t stream) {
+  constexpr int TM = 2048 / BN;
+  constexpr int KC = BN <= 64 ? 16 : 8;
+  const size_t stage_bytes = (size_t)8 * 2 * KC * (TM + BN) * sizeof(float);
+  const size_t part_bytes = (size_t)8 * TM * BN * sizeof(float);
+  const size_t smem = stage_bytes > part_bytes ? stage_bytes : part_bytes;
+  cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<TX, BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((s.T + TM - 1) / TM);
+  router_fused_kernel<TX, BN><<<grid, 256, smem, stream>>>(
+      static_cast<const TX*>(x), W_r, b_r, (int)s.T, (int)s.d, (int)s.N, expert_idx, gate,
+      local_rank, ws.blk_count, ws.blk_psum, ws.hdr);
+  return cudaGetLastError();
+}
+
 template <typename TX, int BM, int BN>
 cudaError_t launch_logits_t(const Shape& s, const Workspace& ws, const void* x, const float* W_r,
                             cudaStream_t stream) {
@@ -413,13 +691,16 @@ cudaError_t launch_softmax_t(const Shape& s, const Workspace& ws, const float* b
         router_softmax_kernel<NPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  router_softmax_kernel<NPL><<<s.nblk, kSoftmaxThreads, smem, stream>>>(
-      ws.logits, s.ksplit_eff, b_r, (int)s.T, (int)s.N, s.tpb, expert_idx, gate, local_rank,
-      ws.blk_count, ws.blk_psum, ws.hdr);
-  return cudaGetLastError();
+  return launch_dependent(router_softmax_kernel<NPL>, dim3(s.nblk), dim3(kSoftmaxThreads), smem,
+                          stream, static_cast<const float*>(ws.logits), s.ksplit_eff, b_r,
+                          (int)s.T, (int)s.N, s.tpb, expert_idx, gate, local_rank, ws.blk_count,
+                          ws.blk_psum, ws.hdr);
 }
 
 }  // namespace
+
+// Tokens per fused-router tile for N (the tile's tokens are one dispatch block).
+int fused_router_tile_tokens(int64_t N) { return N <= 32 ? 64 : (N <= 64 ? 32 : 16); }
 
 int router_kslice(int64_t T, int64_t d, int64_t N) {
   // CTAs of the logits kernel before splitting K; aim for ~3 per SM on 148 SMs
@@ -429,21 +710,32 @@ int router_kslice(int64_t T, int64_t d, int64_t N) {
   int64_t ks = (3 * 148 + tiles - 1) / tiles;
   const int64_t max_ks = d / 64 > 0 ? d / 64 : 1;   // each slice keeps >= 64 of K
   if (ks > max_ks) ks = max_ks;
+  if (N <= kFusedRouterMaxN) ks = 1;   // fused path: K is split across warps, not CTAs
   if (ks > 16) ks = 16;
   if (ks < 1) ks = 1;
   return (int)(((d + ks - 1) / ks + kBK - 1) / kBK * kBK);
 }
 
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
-                                 const float* W_r, const float* b_r, cudaStream_t stream) {
-  (void)b_r;   // the bias is added by the softmax kernel after the K slices
+                                 const float* W_r, const float* b_r, int* expert_idx, float* gate,
+                                 int* local_rank, cudaStream_t stream) {
   cudaError_t e;
-  if (s.N > 64) {
-    e = s.dtype == 1 ? launch_logits_t<__nv_bfloat16, 128, 128>(s, ws, x, W_r, stream)
-                     : launch_logits_t<float, 128, 128>(s, ws, x, W_r, stream);
+  const bool bf = s.dtype == 1;
+  if (s.N <= 32) {
+    e = bf ? launch_fused_t<__nv_bfloat16, 32>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                                stream)
+           : launch_fused_t<float, 32>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank, stream);
+  } else if (s.N <= 64) {
+    e = bf ? launch_fused_t<__nv_bfloat16, 64>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                                stream)
+           : launch_fused_t<float, 64>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank, stream);
+  } else if (s.N <= kFusedRouterMaxN) {
+    e = bf ? launch_fused_t<__nv_bfloat16, 128>(s, ws, x, W_r, b_r, expert_idx, gate,
+                                                 local_rank, stream)
+           : launch_fused_t<float, 128>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank, stream);
   } else {
-    e = s.dtype == 1 ? launch_logits_t<__nv_bfloat16, 128, 64>(s, ws, x, W_r, stream)
-                     : launch_logits_t<float, 128, 64>(s, ws, x, W_r, stream);
+    e = bf ? launch_logits_t<__nv_bfloat16, 128, 128>(s, ws, x, W_r, stream)
+           : launch_logits_t<float, 128, 128>(s, ws, x, W_r, stream);
   }
   count_launch();
   return e;
@@ -462,10 +754,9 @@ cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const flo
   else if (npl <= 32) e = launch_softmax_t<32>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 64) e = launch_softmax_t<64>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else {
-    router_softmax_wide_kernel<<<s.nblk, kSoftmaxThreads, 0, stream>>>(
-        ws.logits, s.ksplit_eff, b_r, (int)s.T, (int)s.N, s.tpb, expert_idx, gate, local_rank,
-        ws.blk_count, ws.blk_psum, ws.hdr);
-    e = cudaGetLastError();
+    e = launch_dependent(router_softmax_wide_kernel, dim3(s.nblk), dim3(kSoftmaxThreads), 0,
+                         stream, ws.logits, s.ksplit_eff, b_r, (int)s.T, (int)s.N, s.tpb,
+                         expert_idx, gate, local_rank, ws.blk_count, ws.blk_psum, ws.hdr);
   }
   count_launch();
   return e;

@@ -40,7 +40,8 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   };
   Workspace w{};
   w.hdr = reinterpret_cast<WsHeader*>(take(sizeof(WsHeader)));
-  w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(s.ksplit_eff) * T * N * 4));
+  w.logits = reinterpret_cast<float*>(
+      take(s.N <= kFusedRouterMaxN ? 0 : static_cast<size_t>(s.ksplit_eff) * T * N * 4));
   w.blk_count = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_off = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_psum = reinterpret_cast<float*>(take(nb * N * 4));
@@ -130,13 +131,19 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->dtype = dtype;
   s->C = switch_layer_capacity(T, N, cf);
   s->C_eff = s->C < T ? s->C : T;
-  // token block: the largest of 128/64/32 that still gives >= 2 CTAs per SM
-  s->tpb = 32;
-  for (int tpb = kTokensPerBlock; tpb > 32; tpb /= 2)
-    if ((T + tpb - 1) / tpb >= 2 * 148) { s->tpb = tpb; break; }
-  s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
   s->kslice = router_kslice(T, d, N);
   s->ksplit_eff = static_cast<int>((d + s->kslice - 1) / s->kslice);
+  if (N <= kFusedRouterMaxN) {
+    // fused router: one CTA (= one dispatch block) per tile of tokens
+    s->tpb = fused_router_tile_tokens(N);
+    s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
+  } else {
+    // token block: the largest of 128/64/32 that still gives >= 2 CTAs per SM
+    s->tpb = 32;
+    for (int tpb = kTokensPerBlock; tpb > 32; tpb /= 2)
+      if ((T + tpb - 1) / tpb >= 2 * 148) { s->tpb = tpb; break; }
+    s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
+  }
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
   return SWL_OK;
 }
@@ -146,13 +153,19 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
                               const void* b2, void* out, int32_t* expert_idx, float* gate,
                               int32_t* pos_in_expert, float* aux_loss, const float* b_r,
                               cudaStream_t stream, void* const* ev) {
+  // External records: under stream capture they become event-record nodes of
+  // the graph (timable on replay); outside capture they are ordinary records.
   auto rec = [&](int k) -> bool {
-    return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[k]), stream) == cudaSuccess;
+    return ev == nullptr || cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev[k]), stream,
+                                                     cudaEventRecordExternal) == cudaSuccess;
   };
   if (!rec(0)) return SWL_ERR_CUDA;
-  if (launch_router_logits(s, ws, x, W_r, b_r, stream) != cudaSuccess) return SWL_ERR_CUDA;
+  if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert, stream) !=
+      cudaSuccess)
+    return SWL_ERR_CUDA;
   if (!rec(1)) return SWL_ERR_CUDA;
-  if (launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
+  if (s.N > kFusedRouterMaxN &&
+      launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
     return SWL_ERR_CUDA;
   if (!rec(2)) return SWL_ERR_CUDA;
   if (launch_dispatch_scan(s, ws, aux_loss, stream) != cudaSuccess) return SWL_ERR_CUDA;

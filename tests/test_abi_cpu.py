@@ -56,8 +56,8 @@ def test_capacity_matches_oracle(L):
 
 def test_workspace_size_and_validation(L):
     n = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25)
-    # logits + packed x/h buffers dominate
-    assert n >= 4096 * 64 * 4 + 4096 * (768 + 3072) * 2
+    # the packed expert input / hidden buffers dominate
+    assert n >= 4096 * (768 + 3072) * 2
     n2 = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25,
                                          swl.SWL_WS_HOST_IO)
     assert n2 > n
