@@ -71,9 +71,10 @@ typedef enum swl_dtype { SWL_F32 = 0, SWL_BF16 = 1 } swl_dtype;
 #define SWL_WS_HOST_IO 1
 
 /* Number of timed stages and their order (see switch_layer_forward_timed):
- * 0 router logits, 1 router softmax/argmax/rank, 2 dispatch scan + aux loss,
- * 3 dispatch gather, 4 expert GEMM1 (+bias, ReLU), 5 expert GEMM2 (+bias, gate, combine). */
-#define SWL_NUM_STAGES 6
+ * 0 router (logits; for N <= 128 also softmax/argmax/ranks), 1 router softmax for N > 128
+ * (empty otherwise), 2 dispatch scan + aux loss, 3 dispatch gather, 4 expert FFN
+ * (GEMM1 + bias + ReLU and GEMM2 + bias + gate + combine). */
+#define SWL_NUM_STAGES 5
 
 /* Expert capacity C = ceil(capacity_factor * T / N) ("Capacity Factor" section
  * of the reading note), evaluated exactly on the binary value of the double

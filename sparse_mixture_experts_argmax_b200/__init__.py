@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libswitchlayer.so")
 
 SWL_F32, SWL_BF16 = 0, 1
 SWL_WS_HOST_IO = 1
-SWL_NUM_STAGES = 6
+SWL_NUM_STAGES = 5
 STATUS = {0: "SWL_OK", 1: "SWL_ERR_INVALID_ARG", 2: "SWL_ERR_UNSUPPORTED",
           3: "SWL_ERR_WORKSPACE", 4: "SWL_ERR_CUDA", 5: "SWL_ERR_DEVICE"}
 

@@ -67,8 +67,8 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
                      int* __restrict__ blk_off, int* __restrict__ exp_count,
                      double* __restrict__ psum64, int* __restrict__ exp_rows,
                      int* __restrict__ exp_base, int* __restrict__ tile_prefix,
-                     float* __restrict__ aux_loss, WsHeader* hdr, int nblk, int N, int T,
-                     int C_eff, int tile_rows) {
+                     int* __restrict__ ready, float* __restrict__ aux_loss, WsHeader* hdr,
+                     int nblk, int N, int T, int C_eff, int tile_rows) {
   __shared__ int wc[kScanWarps][32];
   __shared__ double wp[kScanWarps][32];
   __shared__ int is_last;
@@ -164,10 +164,13 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
   for (int off = 16; off > 0; off >>= 1) aux += __shfl_xor_sync(0xffffffffu, aux, off);
   if (lane == 0) s_aux[warp] = aux;
   __syncthreads();
+  // per-call state of the expert FFN kernel: token-tile readiness and work counter
+  for (int i = threadIdx.x; i < s_tot_tiles; i += kScanThreads) ready[i] = 0;
   if (threadIdx.x == 0) {
     double a = 0.0;
     for (int w = 0; w < kScanWarps; ++w) a += s_aux[w];
     tile_prefix[N] = s_tot_tiles;
+    hdr->next_tile = 0u;
     // aux = N * sum_i (count_i / T) * (psum_i / T)
     *aux_loss = (float)((double)N * a / ((double)T * (double)T));
     hdr->done = 0u;   // ready for the next call
@@ -249,8 +252,8 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
   const int grid = (int)((s.N + 31) / 32);
   const cudaError_t e = launch_dependent(
       dispatch_scan_kernel, dim3(grid), dim3(kScanThreads), 0, stream, ws.blk_count, ws.blk_psum,
-      ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base, ws.tile_prefix, aux_loss,
-      ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows);
+      ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base, ws.tile_prefix, ws.ready,
+      aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows);
   count_launch();
   return e;
 }

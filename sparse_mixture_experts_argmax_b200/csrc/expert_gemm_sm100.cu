@@ -50,50 +50,78 @@ constexpr int kTmemCols = 512;
 constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KiB
 constexpr int kEpiStageBytes = 4 * 32 * 32 * 2;   // per-warp 32x32 bf16 transpose tiles
 
-struct GemmArgs {
-  const int* tile_prefix;      // [N+1]
-  const int* exp_rows;         // [N]
-  const int* exp_base;         // [N]
+// One GEMM of the expert FFN.
+struct PhaseArgs {
   const __nv_bfloat16* bias;   // [N, M]
-  const float* gate;           // [T]       (GEMM2)
-  const int* slot_token;       // [T]       (GEMM2)
   __nv_bfloat16* out;          // GEMM1: hbuf [T, M] (packed rows); GEMM2: out [T, M]
-  int* err;
-  int num_experts;
   int M;          // output features per expert
   int m_tiles;    // ceil(M / 128)
   int k_blocks;   // ceil(K / 64)
-  int bn;         // token rows per tile (multiple of 16, <= 256)
-  int stages;
   int mode;       // 0: bias + ReLU, packed rows; 1: bias, gate, scatter to token rows
 };
 
-struct TileCoord {
-  int e, mt, nt;
+struct FfnArgs {
+  const int* tile_prefix;      // [N+1] token tiles before expert e
+  const int* exp_rows;         // [N]
+  const int* exp_base;         // [N]
+  const float* gate;           // [T]
+  const int* slot_token;       // [T]
+  int* ready;                  // [token tiles] GEMM1 epilogue warps finished (zeroed by the scan)
+  unsigned int* next_tile;     // work counter (zeroed by the scan)
+  int* err;
+  int num_experts;
+  int bn;         // token rows per tile (multiple of 16, <= 256)
+  int stages;
+  PhaseArgs ph[2];
 };
 
-// Tile t of expert e occupies [P[e]*m_tiles, P[e+1]*m_tiles) with P the tile
-// prefix; inside, token blocks vary fastest so concurrent CTAs share weights.
-__device__ __forceinline__ TileCoord decode_tile(int tile, const GemmArgs& a) {
-  const int q = tile / a.m_tiles;
-  int lo = 0, hi = a.num_experts;     // find last e with P[e] <= q  (P[N] > q)
+struct TileCoord {
+  int phase, e, mt, nt, g;   // g: global token-tile index P[e] + nt
+};
+
+constexpr int kTileRing = 4;    // tile ids handed from the producer to the MMA / epilogue
+
+// Work item t: GEMM1 tiles [0, total0) then GEMM2 tiles.  Within a phase, the
+// tiles of expert e occupy [P[e]*m_tiles, P[e+1]*m_tiles) (P = tile prefix) with
+// token blocks fastest, so CTAs working at the same time share weights.
+__device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int total0) {
+  TileCoord c;
+  c.phase = t < total0 ? 0 : 1;
+  const int tile = c.phase == 0 ? t : t - total0;
+  const int m_tiles = a.ph[c.phase].m_tiles;
+  const int q = tile / m_tiles;
+  int lo = 0, hi = a.num_experts;     // last e with P[e] <= q  (P[N] > q)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (__ldg(a.tile_prefix + mid) <= q) lo = mid; else hi = mid;
   }
   const int p0 = __ldg(a.tile_prefix + lo);
   const int nts = __ldg(a.tile_prefix + lo + 1) - p0;
-  const int local = tile - p0 * a.m_tiles;
-  TileCoord c;
+  const int local = tile - p0 * m_tiles;
   c.e = lo;
   c.mt = local / nts;
   c.nt = local - c.mt * nts;
+  c.g = p0 + c.nt;
   return c;
 }
 
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Both GEMMs of the expert FFN in one persistent launch.  GEMM2 tiles of token
+// tile g wait until every GEMM1 epilogue warp of g has stored its rows of hbuf.
 __global__ void __launch_bounds__(kThreads, 1)
-expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmB1, const FfnArgs args) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -104,24 +132,19 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* smem_b = smem_a + stages * kABytes;
   __nv_bfloat16* epi = reinterpret_cast<__nv_bfloat16*>(smem_b + stages * b_bytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(epi) + kEpiStageBytes);
-  uint64_t* full_bar = bars;                    // [kMaxStages]
-  uint64_t* empty_bar = bars + kMaxStages;      // [kMaxStages]
-  uint64_t* tfull_bar = bars + 2 * kMaxStages;  // [2]
-  uint64_t* tempty_bar = tfull_bar + 2;         // [2]
-  uint64_t* drain_bar = tempty_bar + 2;         // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* full_bar = bars;                      // [kMaxStages]
+  uint64_t* empty_bar = bars + kMaxStages;        // [kMaxStages]
+  uint64_t* tfull_bar = bars + 2 * kMaxStages;    // [2]
+  uint64_t* tempty_bar = tfull_bar + 2;           // [2]
+  uint64_t* drain_bar = tempty_bar + 2;           // [1]
+  uint64_t* tile_full = drain_bar + 1;            // [kTileRing]
+  uint64_t* tile_empty = tile_full + kTileRing;   // [kTileRing]
+  int* tile_ring = reinterpret_cast<int*>(tile_empty + kTileRing);   // [kTileRing]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_ring + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  if (threadIdx.x == 0) {   // independent of the previous kernel: overlaps its tail
-    ptx::prefetch_tmap(&tmA);
-    ptx::prefetch_tmap(&tmB);
-  }
-  pdl_wait();   // tile prefix, packed rows and gate come from earlier kernels
-  const int total = args.tile_prefix[args.num_experts] * args.m_tiles;
-  if (static_cast<int>(blockIdx.x) >= total) return;   // uniform per CTA: nothing to do
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(&full_bar[s], 1);
@@ -132,9 +155,17 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
       ptx::mbar_init(&tempty_bar[i], 4);      // one arrive per epilogue warp
     }
     ptx::mbar_init(drain_bar, 1);
+    for (int i = 0; i < kTileRing; ++i) {
+      ptx::mbar_init(&tile_full[i], 1);        // the producer publishes a tile id
+      ptx::mbar_init(&tile_empty[i], 4);       // the epilogue warps retire it
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmA0);
+    ptx::prefetch_tmap(&tmB0);
+    ptx::prefetch_tmap(&tmA1);
+    ptx::prefetch_tmap(&tmB1);
   }
   if (warp == 2) {
     ptx::tmem_alloc(tmem_slot, kTmemCols);
@@ -144,6 +175,10 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // tile prefix, packed rows, gate and counters come from earlier kernels
+  const int ntiles = args.tile_prefix[args.num_experts];
+  const int total0 = ntiles * args.ph[0].m_tiles;
+  const int total = total0 + ntiles * args.ph[1].m_tiles;
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -160,19 +195,52 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
       int stage = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const TileCoord c = decode_tile(tile, args);
-        const int arow = c.e * args.M + c.mt * kBM;
+      for (int i = 0; ok; ++i) {
+        const int slot = i % kTileRing;
+        if (!ptx::mbar_wait(&tile_empty[slot], ((i / kTileRing) & 1) ^ 1u, abort_flag)) {
+          fail();
+          break;
+        }
+        int t = static_cast<int>(atomicAdd(args.next_tile, 1u));
+        if (t >= total) t = -1;
+        tile_ring[slot] = t;
+        ptx::mbar_arrive(&tile_full[slot]);
+        if (t < 0) break;
+        const TileCoord c = decode_tile(t, args, total0);
+        const PhaseArgs& P = args.ph[c.phase];
+        const CUtensorMap* tA = c.phase == 0 ? &tmA0 : &tmA1;
+        const CUtensorMap* tB = c.phase == 0 ? &tmB0 : &tmB1;
+        if (c.phase == 1) {
+          // hbuf rows of token tile g: all GEMM1 epilogue warps of g have stored them
+          const int target = 4 * args.ph[0].m_tiles;
+          if (ld_acquire(args.ready + c.g) < target) {
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (ld_acquire(args.ready + c.g) < target) {
+              if (*abort_flag || ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs) {
+                fail();
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
+          }
+          fence_proxy_async_global();   // generic-proxy stores -> the TMA reads below
+        }
+        const int arow = c.e * P.M + c.mt * kBM;
         const int brow = __ldg(args.exp_base + c.e) + c.nt * args.bn;
-        for (int kb = 0; kb < args.k_blocks; ++kb) {
+        for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag)) { fail(); ok = false; break; }
           ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
-          ptx::tma_load_2d(smem_a + stage * kABytes, &tmA, &full_bar[stage], kb * kBK, arow, pol_w);
-          ptx::tma_load_2d(smem_b + stage * b_bytes, &tmB, &full_bar[stage], kb * kBK, brow, pol_x);
+          ptx::tma_load_2d(smem_a + stage * kABytes, tA, &full_bar[stage], kb * kBK, arow, pol_w);
+          ptx::tma_load_2d(smem_b + stage * b_bytes, tB, &full_bar[stage], kb * kBK, brow, pol_x);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (ph << stage);
           if (++stage == stages) { stage = 0; ph ^= 1u; }
         }
+      }
+      if (!ok) {
+        // unblock the consumers: every ring slot they may still read says "stop"
+        for (int j = 0; j < kTileRing; ++j) tile_ring[j] = -1;
       }
       // drain: every issued load must land before the CTA may exit
       for (int s = 0; s < stages; ++s) {
@@ -193,15 +261,20 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
       int acc = 0;
       uint32_t aph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const TileCoord c = decode_tile(tile, args);
+      for (int i = 0; ok; ++i) {
+        const int slot = i % kTileRing;
+        if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) { fail(); break; }
+        const int t = tile_ring[slot];
+        if (t < 0) break;
+        const TileCoord c = decode_tile(t, args, total0);
+        const PhaseArgs& P = args.ph[c.phase];
         const int rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
         const uint32_t n_mma = static_cast<uint32_t>((rows + 15) & ~15);
         const uint32_t idesc = ptx::umma_idesc_bf16_f32(n_mma);
         if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { fail(); break; }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
-        for (int kb = 0; kb < args.k_blocks; ++kb) {
+        for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag)) { fail(); ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(smem_a + stage * kABytes);
@@ -231,15 +304,20 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
     __nv_bfloat16* st = epi + q * 32 * 32;         // [32 tokens][32 features]
     int acc = 0;
     uint32_t aph = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileCoord c = decode_tile(tile, args);
+    for (int i = 0;; ++i) {
+      const int slot = i % kTileRing;
+      if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) { fail(); break; }
+      const int t = tile_ring[slot];
+      if (t < 0) break;
+      const TileCoord c = decode_tile(t, args, total0);
+      const PhaseArgs& P = args.ph[c.phase];
       const int rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
       const int row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
       if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
       ptx::tc_fence_after();
       const int feat0 = c.mt * kBM + q * 32;       // first feature of this warp
       const int f = feat0 + lane;
-      const float bias = (f < args.M) ? __bfloat162float(args.bias[(size_t)c.e * args.M + f]) : 0.f;
+      const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)c.e * P.M + f]) : 0.f;
       const uint32_t t_base =
           tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < rows; c0 += 32) {
@@ -250,14 +328,14 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         const int col = c0 + lane;
         int dst = row0 + col;
         float g = 1.f;
-        if (args.mode == 1) {
+        if (P.mode == 1) {
           dst = (col < rows) ? __ldg(args.slot_token + row0 + col) : 0;
           g = (col < rows) ? __ldg(args.gate + dst) : 0.f;
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float v = __uint_as_float(r[j]) + bias;
-          if (args.mode == 0) {
+          if (P.mode == 0) {
             v = fmaxf(v, 0.f);
           } else {
             v *= __shfl_sync(0xffffffffu, g, j);
@@ -266,20 +344,29 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int idx = lane + 32 * i;
+        for (int k = 0; k < 4; ++k) {
+          const int idx = lane + 32 * k;
           const int j = idx >> 2, part = idx & 3;
           const int drow = __shfl_sync(0xffffffffu, dst, j);
-          if (c0 + j < rows && feat0 + part * 8 < args.M) {
-            *reinterpret_cast<uint4*>(args.out + (size_t)drow * args.M + feat0 + part * 8) =
+          if (c0 + j < rows && feat0 + part * 8 < P.M) {
+            *reinterpret_cast<uint4*>(P.out + (size_t)drow * P.M + feat0 + part * 8) =
                 *reinterpret_cast<const uint4*>(st + j * 32 + part * 8);
           }
         }
         __syncwarp();
       }
       ptx::tc_fence_before();
+      if (c.phase == 0) {
+        // publish this warp's rows of hbuf to GEMM2 tiles (TMA reads, other CTAs)
+        fence_proxy_async_global();
+        __threadfence();
+      }
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&tempty_bar[acc]);
+      if (lane == 0) {
+        if (c.phase == 0) atomicAdd(args.ready + c.g, 1);
+        ptx::mbar_arrive(&tempty_bar[acc]);
+        ptx::mbar_arrive(&tile_empty[slot]);
+      }
       if (++acc == 2) { acc = 0; aph ^= 1u; }
     }
   }
@@ -292,9 +379,10 @@ expert_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA,
   }
 }
 
-size_t gemm_smem_bytes(int bn, int stages) {
+size_t ffn_smem_bytes(int bn, int stages) {
   return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
-         kEpiStageBytes + (2 * kMaxStages + 5) * sizeof(uint64_t) + 2 * sizeof(uint32_t);
+         kEpiStageBytes + (2 * kMaxStages + 5 + 2 * kTileRing) * sizeof(uint64_t) +
+         kTileRing * sizeof(int) + 2 * sizeof(uint32_t);
 }
 
 }  // namespace
@@ -306,38 +394,43 @@ int bf16_tile_rows(int64_t C_eff) {
   return static_cast<int>(r);
 }
 
-cudaError_t launch_expert_gemm_bf16(const Shape& s, const Workspace& ws, int which,
-                                    const CUtensorMap& tmA, const CUtensorMap& tmB,
-                                    const void* bias, const float* gate, void* out, int num_sms,
-                                    cudaStream_t stream) {
+cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CUtensorMap& tmA1,
+                                   const CUtensorMap& tmB1, const CUtensorMap& tmA2,
+                                   const CUtensorMap& tmB2, const void* b1, const void* b2,
+                                   const float* gate, void* out, int num_sms,
+                                   cudaStream_t stream) {
   constexpr size_t kMaxSmem = 232448;   // 227 KiB opt-in per block
-  GemmArgs a;
+  FfnArgs a;
   a.tile_prefix = ws.tile_prefix;
   a.exp_rows = ws.exp_rows;
   a.exp_base = ws.exp_base;
-  a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.gate = gate;
   a.slot_token = ws.slot_token;
-  a.out = static_cast<__nv_bfloat16*>(out);
+  a.ready = ws.ready;
+  a.next_tile = &ws.hdr->next_tile;
   a.err = &ws.hdr->err;
   a.num_experts = static_cast<int>(s.N);
-  const int64_t M = which == 0 ? s.d_ff : s.d;
-  const int64_t K = which == 0 ? s.d : s.d_ff;
-  a.M = static_cast<int>(M);
-  a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
-  a.k_blocks = static_cast<int>((K + kBK - 1) / kBK);
   a.bn = s.tile_rows;
-  a.mode = which;
+  for (int p = 0; p < 2; ++p) {
+    const int64_t M = p == 0 ? s.d_ff : s.d;
+    const int64_t K = p == 0 ? s.d : s.d_ff;
+    a.ph[p].bias = static_cast<const __nv_bfloat16*>(p == 0 ? b1 : b2);
+    a.ph[p].out = static_cast<__nv_bfloat16*>(p == 0 ? ws.hbuf : out);
+    a.ph[p].M = static_cast<int>(M);
+    a.ph[p].m_tiles = static_cast<int>((M + kBM - 1) / kBM);
+    a.ph[p].k_blocks = static_cast<int>((K + kBK - 1) / kBK);
+    a.ph[p].mode = p;
+  }
   int stages = kMaxStages;
-  while (stages > 2 && gemm_smem_bytes(a.bn, stages) > kMaxSmem) --stages;
+  while (stages > 2 && ffn_smem_bytes(a.bn, stages) > kMaxSmem) --stages;
   a.stages = stages;
-  const size_t smem = gemm_smem_bytes(a.bn, stages);
-  cudaError_t err = cudaFuncSetAttribute(expert_gemm_sm100_kernel,
+  const size_t smem = ffn_smem_bytes(a.bn, stages);
+  cudaError_t err = cudaFuncSetAttribute(expert_ffn_sm100_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  err = launch_dependent(expert_gemm_sm100_kernel, dim3(num_sms), dim3(kThreads), smem, stream,
-                         tmA, tmB, a);
+  err = launch_dependent(expert_ffn_sm100_kernel, dim3(num_sms), dim3(kThreads), smem, stream,
+                         tmA1, tmB1, tmA2, tmB2, a);
   count_launch();
   return err;
 }

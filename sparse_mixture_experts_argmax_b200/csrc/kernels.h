@@ -22,9 +22,10 @@ constexpr int kMaxExperts = 1 << 20;
 
 // Workspace header (256 bytes at offset 0).
 struct WsHeader {
-  int err;            // DeviceError of the last call
-  unsigned int done;  // arrival counter of the dispatch-scan kernel (self-resetting)
-  int pad[62];
+  int err;                  // DeviceError of the last call
+  unsigned int done;        // arrival counter of the dispatch-scan kernel (self-resetting)
+  unsigned int next_tile;   // work counter of the expert FFN kernel (zeroed by the scan)
+  int pad[61];
 };
 
 // Device pointers carved out of the caller's workspace.
@@ -40,6 +41,7 @@ struct Workspace {
   int* tile_prefix;     // [N+1] prefix over experts of ceil(m_e / tile_rows)
   double* psum64;       // [N] sum over all tokens of p_{t,e}
   int* slot_token;      // [T] packed row -> token
+  int* ready;           // [T/16 + N + 1] per token tile: GEMM1 epilogue warps done
   void* xbuf;           // [T, d] packed expert inputs (act dtype)
   void* hbuf;           // [T, d_ff] packed hidden activations (act dtype)
   // host-I/O staging (only with SWL_WS_HOST_IO)
@@ -86,10 +88,13 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
                                    const int* expert_idx, int* pos_in_expert, void* out,
                                    cudaStream_t stream);
-cudaError_t launch_expert_gemm_bf16(const Shape& s, const Workspace& ws, int which,
-                                    const CUtensorMap& tmA, const CUtensorMap& tmB,
-                                    const void* bias, const float* gate, void* out,
-                                    int num_sms, cudaStream_t stream);
+// Both expert GEMMs (bf16, tcgen05) in one persistent launch: GEMM1 + bias + ReLU
+// into hbuf, GEMM2 + bias + gate scattered to out.
+cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CUtensorMap& tmA1,
+                                   const CUtensorMap& tmB1, const CUtensorMap& tmA2,
+                                   const CUtensorMap& tmB2, const void* b1, const void* b2,
+                                   const float* gate, void* out, int num_sms,
+                                   cudaStream_t stream);
 cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int which,
                                    const void* W, const void* bias, const float* gate, void* out,
                                    cudaStream_t stream);

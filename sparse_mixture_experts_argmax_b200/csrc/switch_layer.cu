@@ -6,8 +6,9 @@
 //   1 router softmax       max/argmax/gate, ranks     (router.cu)
 //   2 dispatch scan        offsets, capacity, aux     (dispatch.cu)
 //   3 dispatch gather      pos, packed expert rows    (dispatch.cu)
-//   4 expert GEMM1         bias + ReLU                (expert_gemm_sm100.cu / expert_gemm_f32.cu)
-//   5 expert GEMM2         bias, gate, combine        (same)
+//   4 expert FFN           GEMM1 + bias + ReLU, GEMM2 + bias + gate + combine
+//                          (one tcgen05 launch: expert_gemm_sm100.cu; fp32: two
+//                          launches of expert_gemm_f32.cu)
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -51,6 +52,7 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.tile_prefix = reinterpret_cast<int*>(take((N + 1) * 4));
   w.psum64 = reinterpret_cast<double*>(take(N * 8));
   w.slot_token = reinterpret_cast<int*>(take(T * 4));
+  w.ready = reinterpret_cast<int*>(take((T / 16 + N + 1) * 4));
   w.xbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
   w.hbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d_ff) * elem));
   if (host_io) {
@@ -153,11 +155,19 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
                               const void* b2, void* out, int32_t* expert_idx, float* gate,
                               int32_t* pos_in_expert, float* aux_loss, const float* b_r,
                               cudaStream_t stream, void* const* ev) {
-  // External records: under stream capture they become event-record nodes of
-  // the graph (timable on replay); outside capture they are ordinary records.
+  // Under stream capture the records are made external, so that they become
+  // event-record nodes of the graph (timable on replay); otherwise plain records.
+  bool capturing = false;
+  if (ev != nullptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return SWL_ERR_CUDA;
+    capturing = cs == cudaStreamCaptureStatusActive;
+  }
   auto rec = [&](int k) -> bool {
-    return ev == nullptr || cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev[k]), stream,
-                                                     cudaEventRecordExternal) == cudaSuccess;
+    if (ev == nullptr) return true;
+    cudaEvent_t e = static_cast<cudaEvent_t>(ev[k]);
+    return (capturing ? cudaEventRecordWithFlags(e, stream, cudaEventRecordExternal)
+                      : cudaEventRecord(e, stream)) == cudaSuccess;
   };
   if (!rec(0)) return SWL_ERR_CUDA;
   if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert, stream) !=
@@ -182,19 +192,16 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
         !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
         !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T, s.tile_rows))
       return SWL_ERR_CUDA;
-    if (launch_expert_gemm_bf16(s, ws, 0, a1, b1m, b1, gate, ws.hbuf, sms, stream) != cudaSuccess)
-      return SWL_ERR_CUDA;
-    if (!rec(5)) return SWL_ERR_CUDA;
-    if (launch_expert_gemm_bf16(s, ws, 1, a2, b2m, b2, gate, out, sms, stream) != cudaSuccess)
+    if (launch_expert_ffn_bf16(s, ws, a1, b1m, a2, b2m, b1, b2, gate, out, sms, stream) !=
+        cudaSuccess)
       return SWL_ERR_CUDA;
   } else {
     if (launch_expert_gemm_f32(s, ws, 0, W1, b1, gate, ws.hbuf, stream) != cudaSuccess)
       return SWL_ERR_CUDA;
-    if (!rec(5)) return SWL_ERR_CUDA;
     if (launch_expert_gemm_f32(s, ws, 1, W2, b2, gate, out, stream) != cudaSuccess)
       return SWL_ERR_CUDA;
   }
-  if (!rec(6)) return SWL_ERR_CUDA;
+  if (!rec(5)) return SWL_ERR_CUDA;
   return SWL_OK;
 }
 
@@ -399,8 +406,7 @@ const char* switch_layer_status_string(swl_status status) {
 
 const char* switch_layer_stage_name(int k) {
   static const char* names[SWL_NUM_STAGES] = {"router_logits", "router_softmax",
-                                              "dispatch_scan",  "dispatch_gather",
-                                              "expert_gemm1",   "expert_gemm2"};
+                                              "dispatch_scan", "dispatch_gather", "expert_ffn"};
   return (k >= 0 && k < SWL_NUM_STAGES) ? names[k] : nullptr;
 }
 
