@@ -34,6 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
+from sparse_mixture_experts_argmax_b200 import dist as swl_dist  # noqa: E402
 
 DEFAULT_WORKLOAD = "base_T4096_d768_N64"
 METRIC = "Switch-layer fwd tokens/sec on 1 B200; expert-GEMM % of bf16 tensor peak"
@@ -111,33 +112,16 @@ class ClockSampler:
 
 
 def _dist_init():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(local)
-    return ws, rank, local
+    info = swl_dist.init("nccl")
+    return info.world_size, info.rank, info.local_rank
 
 
 def _barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    swl_dist.barrier(swl_dist.rank_info())
 
 
 def _max_over_ranks(ws, v: float) -> float:
-    if ws == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return swl_dist.max_over_ranks(swl_dist.rank_info(), v)
 
 
 def _traffic_entry(kernel: str, workload: str):
@@ -246,7 +230,7 @@ def run_gpu(args):
     step_ms = np.array([a.elapsed_time(b) for a, b in step_ev])
     total_ms = _max_over_ranks(ws_n, float(step_ms.sum()))
     ms_per_step = total_ms / args.steps
-    value = ws_n * T * args.steps / (total_ms / 1e3)
+    value = swl_dist.aggregate_throughput(swl_dist.rank_info(), T, args.steps, total_ms)
     if swl.switch_layer_device_status(work, stream) != 0:
         raise RuntimeError("device status not OK after the timed steps")
 
@@ -365,9 +349,7 @@ def run_gpu(args):
         res["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(res), flush=True)
-    if ws_n > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    swl_dist.finalize(swl_dist.rank_info())
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -452,11 +434,19 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--shape", default=None,
+                    help="ad-hoc bf16 layer T,d,d_ff,N,capacity_factor instead of a named workload")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    if args.shape:
+        T, d, d_ff, N, cf = args.shape.split(",")
+        spec = synth.LayerSpec("shape_T%s_d%s_f%s_N%s_cf%s" % (T, d, d_ff, N, cf), int(T), int(d),
+                               int(d_ff), int(N), float(cf), "bf16")
+        synth.WORKLOADS[spec.name] = spec
+        args.workload = spec.name
     if args.impl == "reference":
         run_reference(args)
     else:

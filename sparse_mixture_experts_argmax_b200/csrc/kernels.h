@@ -17,7 +17,7 @@ enum DeviceError : int {
   kDevNonFiniteLogits = 3,   // a token had no finite maximum logit (NaN/Inf input)
 };
 
-constexpr int kTokensPerBlock = 128;   // largest token block of the softmax / rank / gather stages
+constexpr int kTokensPerBlock = 256;   // largest token block of the softmax / rank / gather stages
 constexpr int kMaxExperts = 1 << 20;
 
 // Workspace header (256 bytes at offset 0).
@@ -59,6 +59,7 @@ struct Shape {
   int dtype;      // 0 = fp32, 1 = bf16
   int64_t C;      // capacity (formula value)
   int64_t C_eff;  // min(C, T): rows an expert can actually keep
+  int router_path;  // RouterPath
   int tpb;        // tokens per block of the softmax / rank / gather stages (<= kTokensPerBlock)
   int nblk;       // ceil(T / tpb)
   int kslice;     // K elements per slice of the router logits GEMM (multiple of 16)
@@ -66,10 +67,19 @@ struct Shape {
   int tile_rows;  // token rows per GEMM tile (N of the UMMA, or the SIMT tile)
 };
 
-// Router logits K slice length for a shape (a pure function of the shape), and
-// the tokens per tile (= per dispatch block) of the fused router (N <= 128).
-int router_kslice(int64_t T, int64_t d, int64_t N);
-int fused_router_tile_tokens(int64_t N);
+// Router kernel choice for a shape (a pure function of the shape).
+enum RouterPath : int {
+  kRouterWarpSplit = 0,   // N <= 128, small T: one CTA per 2048/BN tokens, K split over warps
+  kRouterTile = 1,        // N <= 128, large T: 256x64 / 128x128 tiles, whole K per CTA
+  kRouterWide = 2,        // N > 128: logits GEMM (K slices) + softmax kernel
+};
+struct RouterPlan {
+  int path;     // RouterPath
+  int tpb;      // tokens per dispatch block
+  int kslice;   // K per logits slice (wide path)
+  int ksplit;   // logits slices (wide path; 1 otherwise)
+};
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 

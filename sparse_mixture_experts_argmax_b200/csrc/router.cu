@@ -13,10 +13,14 @@
 //   token row (held in registers) for max/argmax/sum via warp shuffles; then, per
 //   block, the in-block rank of every token among the block's tokens with the
 //   same expert, the block's per-expert token counts, and per-expert sums of p.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
+
+namespace cg = cooperative_groups;
+
 
 
 namespace swl {
@@ -274,17 +278,27 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
     }
     const int t = t0 + i;
     const float* row = zpart + (size_t)t * N;
+    // all loads of a slice are issued before any is used (one round trip per slice)
     float v[NPL];
 #pragma unroll
     for (int j = 0; j < NPL; ++j) {
       const int n = lane + 32 * j;
-      if (n < N) {
-        float a = row[n];
-        for (int s = 1; s < nsplit; ++s) a += row[s * slice + n];
-        v[j] = a + s_bias[n];
-      } else {
-        v[j] = -INFINITY;
+      v[j] = (n < N) ? row[n] : 0.f;
+    }
+    for (int s = 1; s < nsplit; ++s) {
+      float u[NPL];
+#pragma unroll
+      for (int j = 0; j < NPL; ++j) {
+        const int n = lane + 32 * j;
+        u[j] = (n < N) ? row[s * slice + n] : 0.f;
       }
+#pragma unroll
+      for (int j = 0; j < NPL; ++j) v[j] += u[j];
+    }
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      const int n = lane + 32 * j;
+      v[j] = (n < N) ? v[j] + s_bias[n] : -INFINITY;
     }
     float best = -INFINITY;
     int bidx = 0x7fffffff;
@@ -417,8 +431,9 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
   }
 }
 
-// Fused router for N <= BN (BN = 32, 64 or 128): logits, softmax, argmax and the
-// block statistics in one kernel, one CTA per tile of TM = 2048/BN tokens.
+// Warp-split router for small T and N <= BN (BN = 32, 64 or 128): logits,
+// softmax, argmax and the block statistics in one kernel, one CTA per tile of
+// TM = 2048/BN tokens.
 // The 8 warps split K: warp w accumulates the whole TM x BN tile over the
 // K chunks c = w, w+8, ... (8 x 8 register outer products per lane, staged
 // through warp-private shared memory, so the main loop has no block barrier).
@@ -427,7 +442,7 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
 // one token block of the dispatch statistics.
 template <typename TX, int BN>
 __global__ void __launch_bounds__(256)
-router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
+router_warpsplit_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
                     const float* __restrict__ b_r, int T, int d, int N,
                     int* __restrict__ expert_idx, float* __restrict__ gate,
                     int* __restrict__ local_rank, int* __restrict__ blk_count,
@@ -652,7 +667,7 @@ router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
 }
 
 template <typename TX, int BN>
-cudaError_t launch_fused_t(const Shape& s, const Workspace& ws, const void* x, const float* W_r,
+cudaError_t launch_warpsplit_t(const Shape& s, const Workspace& ws, const void* x, const float* W_r,
                            const float* b_r, int* expert_idx, float* gate, int* local_rank,
                            cudaStream_t stream) {
   constexpr int TM = 2048 / BN;
@@ -660,14 +675,181 @@ cudaError_t launch_fused_t(const Shape& s, const Workspace& ws, const void* x, c
   const size_t stage_bytes = (size_t)8 * 2 * KC * (TM + BN) * sizeof(float);
   const size_t part_bytes = (size_t)8 * TM * BN * sizeof(float);
   const size_t smem = stage_bytes > part_bytes ? stage_bytes : part_bytes;
-  cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<TX, BN>,
+  cudaError_t e = cudaFuncSetAttribute(router_warpsplit_kernel<TX, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((s.T + TM - 1) / TM);
-  router_fused_kernel<TX, BN><<<grid, 256, smem, stream>>>(
+  router_warpsplit_kernel<TX, BN><<<grid, 256, smem, stream>>>(
       static_cast<const TX*>(x), W_r, b_r, (int)s.T, (int)s.d, (int)s.N, expert_idx, gate,
       local_rank, ws.blk_count, ws.blk_psum, ws.hdr);
   return cudaGetLastError();
+}
+
+// Big-tile router for large T and N <= BN: a cluster of S CTAs (S = 1 or 2,
+// along z) owns BM tokens x BN experts; CTA r accumulates K slice r with 8 x 8
+// register tiles (256 threads, main loop above) into its partial tile, then -
+// after a cluster barrier - reduces rows [r*R, r*R+R) (R = BM/S) over the S
+// partial tiles through distributed shared memory in rank order
+// (deterministic), adds the bias and runs each token's softmax with one warp.
+// Its R tokens form dispatch block tile*S + r.
+template <typename TX, int BM, int BN>
+__global__ void __launch_bounds__((BM / 8) * (BN / 8), 2)
+router_tile_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
+                   const float* __restrict__ b_r, int T, int d, int N, int kslice,
+                   int* __restrict__ expert_idx, float* __restrict__ gate,
+                   int* __restrict__ local_rank, int* __restrict__ blk_count,
+                   float* __restrict__ blk_psum, WsHeader* hdr) {
+  constexpr int kThreads = (BM / 8) * (BN / 8), kWarps = kThreads / 32;
+  static_assert(kThreads == 256, "256 threads");
+  constexpr int NPL = BN / 32;
+  constexpr int PS = BN;                      // row stride of the partial tile
+  constexpr int STAGE = 2 * kBK * (BM + BN);  // floats of the staging buffers
+  extern __shared__ __align__(16) float fsm[];
+  auto As = reinterpret_cast<float (*)[kBK][BM]>(fsm);                    // [2][kBK][BM]
+  auto Bs = reinterpret_cast<float (*)[kBK][BN]>(fsm + 2 * kBK * BM);     // [2][kBK][BN]
+  float* Ps = fsm + STAGE;                    // [BM][PS] this CTA's partial tile
+  __shared__ float s_psum[kWarps][BN];
+  __shared__ int eid[kTokensPerBlock];
+  __shared__ int lead_count[kTokensPerBlock];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = (int)cluster.num_blocks();
+  const int r = (int)cluster.block_rank();
+  pdl_trigger();
+  pdl_wait();
+  if (blockIdx.x == 0 && r == 0 && threadIdx.x == 0) {
+    hdr->err = kDevOk;   // per-call device status
+    hdr->done = 0u;      // arrival counter of the dispatch scan
+  }
+  const int tid = threadIdx.x;
+  const int tx = tid % (BN / 8), ty = tid / (BN / 8);
+  const int m0 = blockIdx.x * BM;
+  const int k_lo = r * kslice;
+  const int k_hi = min(d, k_lo + kslice);
+  float acc[8][8];
+  logits_mainloop<TX, BM, BN>(x, W_r, T, d, N, m0, 0, k_lo, k_hi, As, Bs, acc);
+  // lane tx holds experts tx*4 + {0..3} and BN/2 + tx*4 + {0..3} (main loop layout)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float* pr = Ps + (ty * 8 + i) * PS + tx * 4;
+    *reinterpret_cast<float4*>(pr) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    *reinterpret_cast<float4*>(pr + BN / 2) =
+        make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+  }
+  cluster.sync();   // every partial tile of the cluster is complete
+
+  // Z: this CTA's R rows of logits + bias; in place in Ps when S == 1, else in
+  // the (now free) staging area, which holds R x BN floats for R = BM/2.
+  const int R = BM / S;
+  const int row0 = r * R;
+  float* Z = (S == 1) ? Ps : fsm;
+  const int zs = (S == 1) ? PS : BN;
+  const float* peer1 = cluster.map_shared_rank(Ps, S > 1 ? 1 : 0);
+  const float* peer0 = cluster.map_shared_rank(Ps, 0);
+  for (int idx = tid; idx < R * (BN / 4); idx += kThreads) {
+    const int i = idx / (BN / 4), n = (idx % (BN / 4)) * 4;
+    const int off = (row0 + i) * PS + n;
+    float4 v = *reinterpret_cast<const float4*>(peer0 + off);
+    if (S > 1) {
+      const float4 u = *reinterpret_cast<const float4*>(peer1 + off);
+      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+    }
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      Z[i * zs + n + c] = (n + c < N) ? vv[c] + (b_r ? b_r[n + c] : 0.f) : -INFINITY;
+  }
+  __syncthreads();
+
+  const int warp = tid >> 5, lane = tid & 31;
+  const int t0 = m0 + row0;
+  const int ntok = max(0, min(R, T - t0));
+  float pacc[NPL];
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) pacc[j] = 0.f;
+  for (int i = warp; i < R; i += kWarps) {
+    if (i >= ntok) {
+      if (lane == 0) eid[i] = -1;
+      continue;
+    }
+    float v[NPL];
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) v[j] = Z[i * zs + lane + 32 * j];
+    float best = -INFINITY;
+    int bidx = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+      if (v[j] > best) { best = v[j]; bidx = lane + 32 * j; }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+      if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+    }
+    float ssum = 0.f;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      v[j] = (lane + 32 * j < N) ? expf(v[j] - best) : 0.f;
+      ssum += v[j];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+    const float inv = 1.0f / ssum;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) pacc[j] += v[j] * inv;
+    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
+      bidx = 0;
+      if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
+    }
+    if (lane == 0) {
+      expert_idx[t0 + i] = bidx;
+      gate[t0 + i] = inv;       // p at the argmax: exp(0) / s
+      eid[i] = bidx;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) s_psum[warp][lane + 32 * j] = pacc[j];
+  __syncthreads();
+  const int b = blockIdx.x * S + r;
+  int* cnt_row = blk_count + (size_t)b * N;
+  float* ps_row = blk_psum + (size_t)b * N;
+  if (t0 < T) block_ranks(eid, lead_count, ntok, R, t0, local_rank);
+  for (int n = tid; n < N; n += kThreads) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) a += s_psum[w][n];
+    ps_row[n] = a;
+    cnt_row[n] = 0;
+  }
+  __syncthreads();
+  for (int i = tid; i < ntok; i += kThreads) {
+    if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
+  }
+  cluster.sync();   // the peer has finished reading this CTA's partial tile
+}
+
+template <typename TX, int BM, int BN>
+cudaError_t launch_tile_t(const Shape& s, const Workspace& ws, const void* x, const float* W_r,
+                          const float* b_r, int* expert_idx, float* gate, int* local_rank,
+                          cudaStream_t stream) {
+  const size_t smem = ((size_t)2 * kBK * (BM + BN) + (size_t)BM * BN) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(router_tile_kernel<TX, BM, BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((s.T + BM - 1) / BM), 1, (unsigned)s.ksplit_eff);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)s.ksplit_eff;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, router_tile_kernel<TX, BM, BN>, static_cast<const TX*>(x), W_r,
+                            b_r, (int)s.T, (int)s.d, (int)s.N, s.kslice, expert_idx, gate,
+                            local_rank, ws.blk_count, ws.blk_psum, ws.hdr);
 }
 
 template <typename TX, int BM, int BN>
@@ -699,21 +881,43 @@ cudaError_t launch_softmax_t(const Shape& s, const Workspace& ws, const float* b
 
 }  // namespace
 
-// Tokens per fused-router tile for N (the tile's tokens are one dispatch block).
-int fused_router_tile_tokens(int64_t N) { return N <= 32 ? 64 : (N <= 64 ? 32 : 16); }
-
-int router_kslice(int64_t T, int64_t d, int64_t N) {
-  // CTAs of the logits kernel before splitting K; aim for ~3 per SM on 148 SMs
-  int64_t tiles = N > 64 ? ((T + 127) / 128) * ((N + 127) / 128)
-                         : ((T + 127) / 128) * ((N + 63) / 64);
-  if (tiles < 1) tiles = 1;   // empty batch
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N) {
+  RouterPlan p;
+  if (N <= kFusedRouterMaxN) {
+    // one fused kernel; big tiles once there are enough of them to fill the GPU
+    const int64_t bm = N <= 64 ? 256 : 128;
+    const int64_t tiles = (T + bm - 1) / bm;
+    if (N > 32 && tiles >= 100) {
+      // two K slices over a 2-CTA cluster until there are ~2 CTAs per SM
+      p.path = kRouterTile;
+      p.ksplit = (tiles < 2 * 148 && d >= 128) ? 2 : 1;
+      p.kslice = (int)(((d + p.ksplit - 1) / p.ksplit + kBK - 1) / kBK * kBK);
+      p.ksplit = (int)((d + p.kslice - 1) / p.kslice);
+      p.tpb = (int)(bm / p.ksplit);
+    } else {
+      p.path = kRouterWarpSplit;
+      p.tpb = N <= 32 ? 64 : (N <= 64 ? 32 : 16);
+      p.kslice = (int)((d + kBK - 1) / kBK * kBK);
+      p.ksplit = 1;
+    }
+    return p;
+  }
+  // wide N: logits GEMM in 128 x 128 tiles with K slices for ~3 CTAs per SM, then
+  // the softmax kernel over blocks of 128/64/32 tokens
+  p.path = kRouterWide;
+  int64_t tiles = ((T + 127) / 128) * ((N + 127) / 128);
+  if (tiles < 1) tiles = 1;
   int64_t ks = (3 * 148 + tiles - 1) / tiles;
-  const int64_t max_ks = d / 64 > 0 ? d / 64 : 1;   // each slice keeps >= 64 of K
+  const int64_t max_ks = d / 64 > 0 ? d / 64 : 1;
   if (ks > max_ks) ks = max_ks;
-  if (N <= kFusedRouterMaxN) ks = 1;   // fused path: K is split across warps, not CTAs
   if (ks > 16) ks = 16;
   if (ks < 1) ks = 1;
-  return (int)(((d + ks - 1) / ks + kBK - 1) / kBK * kBK);
+  p.kslice = (int)(((d + ks - 1) / ks + kBK - 1) / kBK * kBK);
+  p.ksplit = (int)((d + p.kslice - 1) / p.kslice);
+  p.tpb = 32;
+  for (int tpb = 128; tpb > 32; tpb /= 2)
+    if ((T + tpb - 1) / tpb >= 2 * 148) { p.tpb = tpb; break; }
+  return p;
 }
 
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
@@ -721,18 +925,33 @@ cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void
                                  int* local_rank, cudaStream_t stream) {
   cudaError_t e;
   const bool bf = s.dtype == 1;
-  if (s.N <= 32) {
-    e = bf ? launch_fused_t<__nv_bfloat16, 32>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
-                                                stream)
-           : launch_fused_t<float, 32>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank, stream);
-  } else if (s.N <= 64) {
-    e = bf ? launch_fused_t<__nv_bfloat16, 64>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
-                                                stream)
-           : launch_fused_t<float, 64>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank, stream);
-  } else if (s.N <= kFusedRouterMaxN) {
-    e = bf ? launch_fused_t<__nv_bfloat16, 128>(s, ws, x, W_r, b_r, expert_idx, gate,
-                                                 local_rank, stream)
-           : launch_fused_t<float, 128>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank, stream);
+  if (s.router_path == kRouterTile) {
+    if (s.N <= 64)
+      e = bf ? launch_tile_t<__nv_bfloat16, 256, 64>(s, ws, x, W_r, b_r, expert_idx, gate,
+                                                      local_rank, stream)
+             : launch_tile_t<float, 256, 64>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                              stream);
+    else
+      e = bf ? launch_tile_t<__nv_bfloat16, 128, 128>(s, ws, x, W_r, b_r, expert_idx, gate,
+                                                       local_rank, stream)
+             : launch_tile_t<float, 128, 128>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                               stream);
+  } else if (s.router_path == kRouterWarpSplit) {
+    if (s.N <= 32)
+      e = bf ? launch_warpsplit_t<__nv_bfloat16, 32>(s, ws, x, W_r, b_r, expert_idx, gate,
+                                                      local_rank, stream)
+             : launch_warpsplit_t<float, 32>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                              stream);
+    else if (s.N <= 64)
+      e = bf ? launch_warpsplit_t<__nv_bfloat16, 64>(s, ws, x, W_r, b_r, expert_idx, gate,
+                                                      local_rank, stream)
+             : launch_warpsplit_t<float, 64>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                              stream);
+    else
+      e = bf ? launch_warpsplit_t<__nv_bfloat16, 128>(s, ws, x, W_r, b_r, expert_idx, gate,
+                                                       local_rank, stream)
+             : launch_warpsplit_t<float, 128>(s, ws, x, W_r, b_r, expert_idx, gate, local_rank,
+                                               stream);
   } else {
     e = bf ? launch_logits_t<__nv_bfloat16, 128, 128>(s, ws, x, W_r, stream)
            : launch_logits_t<float, 128, 128>(s, ws, x, W_r, stream);

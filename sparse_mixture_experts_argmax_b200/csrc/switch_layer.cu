@@ -42,7 +42,7 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   Workspace w{};
   w.hdr = reinterpret_cast<WsHeader*>(take(sizeof(WsHeader)));
   w.logits = reinterpret_cast<float*>(
-      take(s.N <= kFusedRouterMaxN ? 0 : static_cast<size_t>(s.ksplit_eff) * T * N * 4));
+      take(s.router_path != kRouterWide ? 0 : static_cast<size_t>(s.ksplit_eff) * T * N * 4));
   w.blk_count = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_off = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_psum = reinterpret_cast<float*>(take(nb * N * 4));
@@ -133,19 +133,12 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->dtype = dtype;
   s->C = switch_layer_capacity(T, N, cf);
   s->C_eff = s->C < T ? s->C : T;
-  s->kslice = router_kslice(T, d, N);
-  s->ksplit_eff = static_cast<int>((d + s->kslice - 1) / s->kslice);
-  if (N <= kFusedRouterMaxN) {
-    // fused router: one CTA (= one dispatch block) per tile of tokens
-    s->tpb = fused_router_tile_tokens(N);
-    s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
-  } else {
-    // token block: the largest of 128/64/32 that still gives >= 2 CTAs per SM
-    s->tpb = 32;
-    for (int tpb = kTokensPerBlock; tpb > 32; tpb /= 2)
-      if ((T + tpb - 1) / tpb >= 2 * 148) { s->tpb = tpb; break; }
-    s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
-  }
+  const RouterPlan rp = router_plan(T, d, N);
+  s->router_path = rp.path;
+  s->kslice = rp.kslice;
+  s->ksplit_eff = rp.ksplit;
+  s->tpb = rp.tpb;
+  s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
   return SWL_OK;
 }

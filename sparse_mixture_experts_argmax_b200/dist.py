@@ -1,0 +1,82 @@
+"""Multi-process plumbing for running the layer on several GPUs of one node.
+
+One process per GPU (torchrun).  The Switch layer's forward pass needs no data
+exchange between ranks when each rank routes its own batch: in the pages'
+design every core computes routing, positions and capacity for the tokens it
+holds (the dispatch mask is laid out per core).  So ranks run independent
+forward passes and only the measurement is combined: a barrier around the
+timed region and the maximum of the per-rank device times.
+
+Everything here is device agnostic (NCCL on GPUs, gloo on CPUs for the tests).
+"""
+from __future__ import annotations
+
+import datetime
+import os
+from dataclasses import dataclass
+
+import torch
+import torch.distributed as dist
+
+
+@dataclass
+class RankInfo:
+    rank: int
+    world_size: int
+    local_rank: int
+
+    @property
+    def distributed(self) -> bool:
+        return self.world_size > 1
+
+
+def rank_info() -> RankInfo:
+    """RANK / WORLD_SIZE / LOCAL_RANK from the environment (torchrun sets them)."""
+    return RankInfo(int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+                    int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init(backend: str = "nccl", timeout_s: float = 120.0) -> RankInfo:
+    """Join the process group when more than one rank is running."""
+    info = rank_info()
+    if info.distributed and not dist.is_initialized():
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(info.local_rank)
+            kw["device_id"] = torch.device("cuda", info.local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    elif backend == "nccl" and torch.cuda.is_available():
+        torch.cuda.set_device(info.local_rank)
+    return info
+
+
+def barrier(info: RankInfo) -> None:
+    if info.distributed:
+        dist.barrier()
+
+
+def max_over_ranks(info: RankInfo, value: float, device=None) -> float:
+    """Largest value over all ranks (the slowest rank decides a timed region)."""
+    if not info.distributed:
+        return float(value)
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(info: RankInfo, units_per_rank: int, steps: int,
+                         max_total_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest time."""
+    return info.world_size * units_per_rank * steps / (max_total_ms / 1e3)
+
+
+def rank_seed(info: RankInfo, base_seed: int = 0) -> int:
+    """Seed of this rank's batch (independent batches; rank 0 keeps the base seed)."""
+    return base_seed + info.rank
+
+
+def finalize(info: RankInfo) -> None:
+    if info.distributed and dist.is_initialized():
+        dist.destroy_process_group()
