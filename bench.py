@@ -200,7 +200,9 @@ def run_gpu(args):
                                      outs["aux_loss"], b_r=inputs["b_r"], workspace=work,
                                      stream=cap, stage_events=S_EV)
     stream.wait_stream(cap)
-    launches_per_forward = (4 if N <= 128 else 5) + (1 if act == torch.bfloat16 else 2)
+    # router (fused for N <= 128, logits + softmax otherwise), scan, gather, expert FFN (bf16: one
+    # launch for both GEMMs; fp32: two)
+    launches_per_forward = (3 if N <= 128 else 4) + (1 if act == torch.bfloat16 else 2)
     for _ in range(args.warmup):
         flush.fill_(1)
         graph.replay()
