@@ -168,9 +168,12 @@ def run_gpu(args):
                                  outs["aux_loss"], b_r=inputs["b_r"], workspace=work,
                                  stream=stream, stage_events=events)
 
+    launches_per_forward = 0          # kernels one forward enqueues (library's own count)
     for _ in range(args.warmup):
         flush.fill_(1)
+        c0 = swl.switch_layer_launch_count()
         step()
+        launches_per_forward = swl.switch_layer_launch_count() - c0
     torch.cuda.synchronize()
     if swl.switch_layer_device_status(work, stream) != 0:
         raise RuntimeError("device status not OK after warm-up")
@@ -200,9 +203,6 @@ def run_gpu(args):
                                      outs["aux_loss"], b_r=inputs["b_r"], workspace=work,
                                      stream=cap, stage_events=S_EV)
     stream.wait_stream(cap)
-    # router (fused for N <= 128, logits + softmax otherwise), scan, gather, expert FFN (bf16: one
-    # launch for both GEMMs; fp32: two)
-    launches_per_forward = (3 if N <= 128 else 4) + (1 if act == torch.bfloat16 else 2)
     for _ in range(args.warmup):
         flush.fill_(1)
         graph.replay()

@@ -24,11 +24,14 @@
 //               ring of shared-memory stages (128-byte swizzle)
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
 //   warp 2      TMEM allocator (512 columns: two 256-column accumulators)
+//   warp 3      tile scheduler (one thread): claims, decodes and publishes tiles
 //   warps 4..7  epilogue: tcgen05.ld, bias / ReLU / gate in fp32, bf16 pack,
 //               transpose through shared memory, 16-byte stores
 // Tiles (expert, 128-feature block, token block) are numbered expert-major and
-// handed out round-robin; the token-block count of each expert comes from the
-// device tile prefix written by the dispatch scan.  Every wait is bounded; a
+// handed out in order by a device counter; the token-block count of each expert
+// comes from the device tile prefix written by the dispatch scan.  The
+// scheduler keeps the claim, the decode (dependent loads of the prefix) and the
+// GEMM2 readiness wait off the producer's path.  Every wait is bounded; a
 // stuck pipeline sets the device error word and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -79,7 +82,15 @@ struct TileCoord {
   int phase, e, mt, nt, g;   // g: global token-tile index P[e] + nt
 };
 
-constexpr int kTileRing = 4;    // tile ids handed from the producer to the MMA / epilogue
+// A decoded work item, published by the scheduler warp in shared memory.
+struct TileSlot {
+  int t;          // tile id; -1: no more work
+  int phase, e, mt, nt, g;
+  int rows;       // valid token rows of the tile
+  int row0;       // first packed row of the tile
+};
+
+constexpr int kTileRing = 4;    // decoded tiles handed to the producer, MMA and epilogue
 
 // Work item t: GEMM1 tiles [0, total0) then GEMM2 tiles.  Within a phase, the
 // tiles of expert e occupy [P[e]*m_tiles, P[e+1]*m_tiles) (P = tile prefix) with
@@ -139,7 +150,8 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   uint64_t* drain_bar = tempty_bar + 2;           // [1]
   uint64_t* tile_full = drain_bar + 1;            // [kTileRing]
   uint64_t* tile_empty = tile_full + kTileRing;   // [kTileRing]
-  int* tile_ring = reinterpret_cast<int*>(tile_empty + kTileRing);   // [kTileRing]
+  uint64_t* take_bar = tile_empty + kTileRing;    // [1] the producer took a tile
+  TileSlot* tile_ring = reinterpret_cast<TileSlot*>(take_bar + 1);   // [kTileRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_ring + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -156,9 +168,10 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     }
     ptx::mbar_init(drain_bar, 1);
     for (int i = 0; i < kTileRing; ++i) {
-      ptx::mbar_init(&tile_full[i], 1);        // the producer publishes a tile id
+      ptx::mbar_init(&tile_full[i], 1);        // the scheduler publishes a tile
       ptx::mbar_init(&tile_empty[i], 4);       // the epilogue warps retire it
     }
+    ptx::mbar_init(take_bar, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
@@ -185,7 +198,57 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     atomicExch(args.err, kDevPipelineTimeout);
   };
 
-  if (warp == 0) {
+  if (warp == 3) {
+    // ------------------------------------------------------------ tile scheduler
+    // Claims the next tile only once the producer has taken the previous one (so
+    // a CTA holds at most one claimed tile it has not started), decodes it, waits
+    // for its GEMM1 rows when it is a GEMM2 tile, and publishes it in the ring.
+    if (lane == 0) {
+      for (int i = 0;; ++i) {
+        const int slot = i % kTileRing;
+        if (i > 0 && !ptx::mbar_wait(take_bar, static_cast<uint32_t>(i - 1) & 1u, abort_flag)) {
+          fail();
+          break;
+        }
+        if (!ptx::mbar_wait(&tile_empty[slot], ((i / kTileRing) & 1) ^ 1u, abort_flag)) {
+          fail();
+          break;
+        }
+        const unsigned int claimed = atomicAdd(args.next_tile, 1u);
+        TileSlot ts;
+        ts.t = claimed < static_cast<unsigned int>(total) ? static_cast<int>(claimed) : -1;
+        ts.phase = ts.e = ts.mt = ts.nt = ts.g = ts.rows = ts.row0 = 0;
+        if (ts.t >= 0) {
+          const TileCoord c = decode_tile(ts.t, args, total0);
+          ts.phase = c.phase;
+          ts.e = c.e;
+          ts.mt = c.mt;
+          ts.nt = c.nt;
+          ts.g = c.g;
+          ts.rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
+          ts.row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
+          if (c.phase == 1) {
+            // hbuf rows of token tile g: every GEMM1 epilogue warp of g has stored them
+            const int target = 4 * args.ph[0].m_tiles;
+            bool ready = ld_acquire(args.ready + c.g) >= target;
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (!ready) {
+              if (*abort_flag || ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs) break;
+              ready = ld_acquire(args.ready + c.g) >= target;
+            }
+            if (!ready) {
+              fail();
+              break;
+            }
+          }
+        }
+        tile_ring[slot] = ts;
+        ptx::mbar_arrive(&tile_full[slot]);
+        if (ts.t < 0) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_w = ptx::l2_policy_evict_first();
@@ -197,37 +260,21 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int slot = i % kTileRing;
-        if (!ptx::mbar_wait(&tile_empty[slot], ((i / kTileRing) & 1) ^ 1u, abort_flag)) {
+        if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) {
           fail();
           break;
         }
-        int t = static_cast<int>(atomicAdd(args.next_tile, 1u));
-        if (t >= total) t = -1;
-        tile_ring[slot] = t;
-        ptx::mbar_arrive(&tile_full[slot]);
-        if (t < 0) break;
-        const TileCoord c = decode_tile(t, args, total0);
-        const PhaseArgs& P = args.ph[c.phase];
-        const CUtensorMap* tA = c.phase == 0 ? &tmA0 : &tmA1;
-        const CUtensorMap* tB = c.phase == 0 ? &tmB0 : &tmB1;
-        if (c.phase == 1) {
-          // hbuf rows of token tile g: all GEMM1 epilogue warps of g have stored them
-          const int target = 4 * args.ph[0].m_tiles;
-          if (ld_acquire(args.ready + c.g) < target) {
-            const uint64_t t0 = ptx::globaltimer_ns();
-            while (ld_acquire(args.ready + c.g) < target) {
-              if (*abort_flag || ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs) {
-                fail();
-                ok = false;
-                break;
-              }
-            }
-            if (!ok) break;
-          }
-          fence_proxy_async_global();   // generic-proxy stores -> the TMA reads below
-        }
-        const int arow = c.e * P.M + c.mt * kBM;
-        const int brow = __ldg(args.exp_base + c.e) + c.nt * args.bn;
+        const TileSlot ts = tile_ring[slot];
+        if (ts.t < 0) break;
+        ptx::mbar_arrive(take_bar);
+        const PhaseArgs& P = args.ph[ts.phase];
+        const CUtensorMap* tA = ts.phase == 0 ? &tmA0 : &tmA1;
+        const CUtensorMap* tB = ts.phase == 0 ? &tmB0 : &tmB1;
+        // GEMM2 tile: the scheduler saw the hbuf rows published (generic-proxy
+        // stores of other CTAs); order them before the TMA reads below
+        if (ts.phase == 1) fence_proxy_async_global();
+        const int arow = ts.e * P.M + ts.mt * kBM;
+        const int brow = ts.row0;
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag)) { fail(); ok = false; break; }
           ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
@@ -237,10 +284,6 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           last_par = (last_par & ~(1u << stage)) | (ph << stage);
           if (++stage == stages) { stage = 0; ph ^= 1u; }
         }
-      }
-      if (!ok) {
-        // unblock the consumers: every ring slot they may still read says "stop"
-        for (int j = 0; j < kTileRing; ++j) tile_ring[j] = -1;
       }
       // drain: every issued load must land before the CTA may exit
       for (int s = 0; s < stages; ++s) {
@@ -264,12 +307,10 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       for (int i = 0; ok; ++i) {
         const int slot = i % kTileRing;
         if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) { fail(); break; }
-        const int t = tile_ring[slot];
-        if (t < 0) break;
-        const TileCoord c = decode_tile(t, args, total0);
-        const PhaseArgs& P = args.ph[c.phase];
-        const int rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
-        const uint32_t n_mma = static_cast<uint32_t>((rows + 15) & ~15);
+        const TileSlot ts = tile_ring[slot];
+        if (ts.t < 0) break;
+        const PhaseArgs& P = args.ph[ts.phase];
+        const uint32_t n_mma = static_cast<uint32_t>((ts.rows + 15) & ~15);
         const uint32_t idesc = ptx::umma_idesc_bf16_f32(n_mma);
         if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { fail(); break; }
         ptx::tc_fence_after();
@@ -307,31 +348,40 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     for (int i = 0;; ++i) {
       const int slot = i % kTileRing;
       if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) { fail(); break; }
-      const int t = tile_ring[slot];
-      if (t < 0) break;
-      const TileCoord c = decode_tile(t, args, total0);
-      const PhaseArgs& P = args.ph[c.phase];
-      const int rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
-      const int row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
-      if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
-      ptx::tc_fence_after();
-      const int feat0 = c.mt * kBM + q * 32;       // first feature of this warp
+      const TileSlot ts = tile_ring[slot];
+      if (ts.t < 0) break;
+      const PhaseArgs& P = args.ph[ts.phase];
+      const int rows = ts.rows;
+      const int row0 = ts.row0;
+      const int feat0 = ts.mt * kBM + q * 32;      // first feature of this warp
       const int f = feat0 + lane;
-      const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)c.e * P.M + f]) : 0.f;
-      const uint32_t t_base =
-          tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 0; c0 < rows; c0 += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
-        ptx::tmem_ld_wait();
-        // destination row and gate of column (c0 + lane)
+      // operands of the epilogue, fetched before the accumulator is ready:
+      // this lane's bias, and the destination row / gate of column (c0 + lane)
+      const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.M + f]) : 0.f;
+      auto fetch_col = [&](int c0, int& dst, float& g) {
         const int col = c0 + lane;
-        int dst = row0 + col;
-        float g = 1.f;
         if (P.mode == 1) {
           dst = (col < rows) ? __ldg(args.slot_token + row0 + col) : 0;
           g = (col < rows) ? __ldg(args.gate + dst) : 0.f;
+        } else {
+          dst = row0 + col;
+          g = 1.f;
         }
+      };
+      int dst_next;
+      float g_next;
+      fetch_col(0, dst_next, g_next);
+      if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
+      ptx::tc_fence_after();
+      const uint32_t t_base =
+          tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c0 = 0; c0 < rows; c0 += 32) {
+        const int dst = dst_next;
+        const float g = g_next;
+        if (c0 + 32 < rows) fetch_col(c0 + 32, dst_next, g_next);
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
+        ptx::tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float v = __uint_as_float(r[j]) + bias;
@@ -356,21 +406,20 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         __syncwarp();
       }
       ptx::tc_fence_before();
-      if (c.phase == 0) {
+      if (ts.phase == 0) {
         // publish this warp's rows of hbuf to GEMM2 tiles (TMA reads, other CTAs)
         fence_proxy_async_global();
         __threadfence();
       }
       __syncwarp();
       if (lane == 0) {
-        if (c.phase == 0) atomicAdd(args.ready + c.g, 1);
+        if (ts.phase == 0) atomicAdd(args.ready + ts.g, 1);
         ptx::mbar_arrive(&tempty_bar[acc]);
         ptx::mbar_arrive(&tile_empty[slot]);
       }
       if (++acc == 2) { acc = 0; aph ^= 1u; }
     }
   }
-
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 2) {
@@ -381,8 +430,8 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
 
 size_t ffn_smem_bytes(int bn, int stages) {
   return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
-         kEpiStageBytes + (2 * kMaxStages + 5 + 2 * kTileRing) * sizeof(uint64_t) +
-         kTileRing * sizeof(int) + 2 * sizeof(uint32_t);
+         kEpiStageBytes + (2 * kMaxStages + 6 + 2 * kTileRing) * sizeof(uint64_t) +
+         kTileRing * sizeof(TileSlot) + 2 * sizeof(uint32_t);
 }
 
 }  // namespace

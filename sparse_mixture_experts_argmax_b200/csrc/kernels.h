@@ -42,6 +42,7 @@ struct Workspace {
   double* psum64;       // [N] sum over all tokens of p_{t,e}
   int* slot_token;      // [T] packed row -> token
   int* ready;           // [T/16 + N + 1] per token tile: GEMM1 epilogue warps done
+  void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
   void* xbuf;           // [T, d] packed expert inputs (act dtype)
   void* hbuf;           // [T, d_ff] packed hidden activations (act dtype)
   // host-I/O staging (only with SWL_WS_HOST_IO)
@@ -72,14 +73,18 @@ enum RouterPath : int {
   kRouterWarpSplit = 0,   // N <= 128, small T: one CTA per 2048/BN tokens, K split over warps
   kRouterTile = 1,        // N <= 128, large T: 256x64 / 128x128 tiles, whole K per CTA
   kRouterWide = 2,        // N > 128: logits GEMM (K slices) + softmax kernel
+  kRouterTC = 3,          // bf16 layers, N <= 128: tcgen05 logits from a 3-piece bf16 split
+                          // of W_r, 128-token tiles, K split over a cluster of 1/2/4 CTAs
+  kRouterTCWide = 4,      // bf16 layers, N > 128: tcgen05 logits tiles (128 x 128) to the
+                          // workspace, then the softmax kernel
 };
 struct RouterPlan {
   int path;     // RouterPath
   int tpb;      // tokens per dispatch block
-  int kslice;   // K per logits slice (wide path)
-  int ksplit;   // logits slices (wide path; 1 otherwise)
+  int kslice;   // K per logits slice (wide, tile and tensor-core paths)
+  int ksplit;   // logits slices (CTAs of a cluster on the tile / tensor-core paths)
 };
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N);
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int dtype);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 
@@ -90,6 +95,13 @@ constexpr int kFusedRouterMaxN = 128;
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
                                  const float* W_r, const float* b_r, int* expert_idx, float* gate,
                                  int* local_rank, cudaStream_t stream);
+// Tensor-core router (kRouterTC, kRouterTCWide): splits W_r into ws.w3, then routes.
+// tmX = x as bf16 [T, d] (box 64 x 128), tmW = ws.w3 as bf16 [3N, d] (box 64 x
+// router_tc_padded_experts(N)), both with 128-byte swizzle.  Two launches.
+int router_tc_padded_experts(int64_t N);
+cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
+                             const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
+                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream);
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);

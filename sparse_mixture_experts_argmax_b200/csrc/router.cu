@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include "kernels.h"
+#include "router_common.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -216,28 +217,6 @@ router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
 
 constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = kSoftmaxThreads / 32;
-
-// Block-level bookkeeping shared by both softmax kernels: in-block stable rank
-// of each token among the block's earlier tokens with the same expert, and the
-// block's per-expert token counts (written by the first token of each expert).
-// eid[i] < 0 marks an absent token.  Caller zeroes cnt_row before calling and
-// synchronises the block after.
-__device__ __forceinline__ void block_ranks(const int* eid, int* lead_count, int ntok, int tpb,
-                                            int t0, int* __restrict__ local_rank) {
-  for (int i = threadIdx.x; i < tpb; i += blockDim.x) {
-    const int e = eid[i];
-    lead_count[i] = 0;
-    if (e < 0) continue;
-    int rank = 0;
-    for (int j = 0; j < i; ++j) rank += (eid[j] == e);
-    local_rank[t0 + i] = rank;
-    if (rank == 0) {
-      int c = 1;
-      for (int j = i + 1; j < ntok; ++j) c += (eid[j] == e);
-      lead_count[i] = c;
-    }
-  }
-}
 
 // One CTA per block of tpb tokens; one warp per token with the row of logits
 // held in registers (NPL = logits per lane, N <= 32*NPL):
@@ -760,70 +739,10 @@ router_tile_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
   }
   __syncthreads();
 
-  const int warp = tid >> 5, lane = tid & 31;
   const int t0 = m0 + row0;
   const int ntok = max(0, min(R, T - t0));
-  float pacc[NPL];
-#pragma unroll
-  for (int j = 0; j < NPL; ++j) pacc[j] = 0.f;
-  for (int i = warp; i < R; i += kWarps) {
-    if (i >= ntok) {
-      if (lane == 0) eid[i] = -1;
-      continue;
-    }
-    float v[NPL];
-#pragma unroll
-    for (int j = 0; j < NPL; ++j) v[j] = Z[i * zs + lane + 32 * j];
-    float best = -INFINITY;
-    int bidx = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NPL; ++j)
-      if (v[j] > best) { best = v[j]; bidx = lane + 32 * j; }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-      if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
-    }
-    float ssum = 0.f;
-#pragma unroll
-    for (int j = 0; j < NPL; ++j) {
-      v[j] = (lane + 32 * j < N) ? expf(v[j] - best) : 0.f;
-      ssum += v[j];
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
-    const float inv = 1.0f / ssum;
-#pragma unroll
-    for (int j = 0; j < NPL; ++j) pacc[j] += v[j] * inv;
-    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
-      bidx = 0;
-      if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
-    }
-    if (lane == 0) {
-      expert_idx[t0 + i] = bidx;
-      gate[t0 + i] = inv;       // p at the argmax: exp(0) / s
-      eid[i] = bidx;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < NPL; ++j) s_psum[warp][lane + 32 * j] = pacc[j];
-  __syncthreads();
-  const int b = blockIdx.x * S + r;
-  int* cnt_row = blk_count + (size_t)b * N;
-  float* ps_row = blk_psum + (size_t)b * N;
-  if (t0 < T) block_ranks(eid, lead_count, ntok, R, t0, local_rank);
-  for (int n = tid; n < N; n += kThreads) {
-    float a = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) a += s_psum[w][n];
-    ps_row[n] = a;
-    cnt_row[n] = 0;
-  }
-  __syncthreads();
-  for (int i = tid; i < ntok; i += kThreads) {
-    if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
-  }
+  route_rows<NPL, kWarps>(Z, zs, R, ntok, t0, N, blockIdx.x * S + r, expert_idx, gate,
+                          local_rank, blk_count, blk_psum, hdr, eid, lead_count, &s_psum[0][0]);
   cluster.sync();   // the peer has finished reading this CTA's partial tile
 }
 
@@ -881,8 +800,22 @@ cudaError_t launch_softmax_t(const Shape& s, const Workspace& ws, const float* b
 
 }  // namespace
 
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N) {
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int dtype) {
   RouterPlan p;
+  if (dtype == 1 && N <= kFusedRouterMaxN) {
+    // tensor cores: 128-token tiles; K split over 2 or 4 CTAs of a cluster while
+    // the tiles alone would leave most SMs idle (and each CTA keeps >= 2 k-blocks)
+    const int64_t tiles = (T + 127) / 128;
+    const int64_t nkb = (d + 63) / 64;
+    int64_t S = 1;
+    while (S < 4 && tiles * S * 2 <= 160 && 2 * S * 2 <= nkb) S *= 2;
+    const int64_t kb_per = (nkb + S - 1) / S;
+    p.path = kRouterTC;
+    p.ksplit = (int)S;
+    p.kslice = (int)(kb_per * 64);
+    p.tpb = (int)(128 / S);
+    return p;
+  }
   if (N <= kFusedRouterMaxN) {
     // one fused kernel; big tiles once there are enough of them to fill the GPU
     const int64_t bm = N <= 64 ? 256 : 128;
@@ -902,8 +835,18 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N) {
     }
     return p;
   }
-  // wide N: logits GEMM in 128 x 128 tiles with K slices for ~3 CTAs per SM, then
-  // the softmax kernel over blocks of 128/64/32 tokens
+  // wide N: logits GEMM in 128 x 128 tiles (bf16 layers: tensor cores over the
+  // whole K; fp32 layers: FFMA with K slices for ~3 CTAs per SM), then the softmax
+  // kernel over blocks of 128/64/32 tokens
+  p.tpb = 32;
+  for (int tpb = 128; tpb > 32; tpb /= 2)
+    if ((T + tpb - 1) / tpb >= 2 * 148) { p.tpb = tpb; break; }
+  if (dtype == 1) {
+    p.path = kRouterTCWide;
+    p.ksplit = 1;
+    p.kslice = (int)((d + 63) / 64 * 64);
+    return p;
+  }
   p.path = kRouterWide;
   int64_t tiles = ((T + 127) / 128) * ((N + 127) / 128);
   if (tiles < 1) tiles = 1;

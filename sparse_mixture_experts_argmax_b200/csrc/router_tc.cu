@@ -1,0 +1,443 @@
+// fp32 router of the Switch layer on the 5th-generation tensor cores, for bf16
+// layers: fused routing for N <= 128 experts, logits only for wider layers.
+//
+// The router computes z_t = W_r x_t (+ b_r) in float32, then p_t = softmax(z_t),
+// e_t = argmax_i p_t,i (lowest index on ties) and g_t = p_t,e_t (Switch
+// Transformer, explained, recipe step 2 "Route in float32"; paper-graph summary
+// of arXiv 2101.03961, "The selective precision solution").
+//
+// float32 logits from bf16 tensor-core products: every fp32 router weight is
+// split exactly into three bf16 numbers, w = hi + mid + lo with
+//   hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)
+// (each residual is exact in fp32, and 3 x 8 significand bits cover fp32's 24).
+// The layer input x is bf16 already, so every product x_k * piece_k is exact in
+// fp32 and the tensor core accumulates the three dot products in fp32 (TMEM).
+// z = D_hi + (D_mid + D_lo) is then the fp32 dot product up to the rounding of
+// the fp32 accumulation, the same class of error as an fp32 FFMA loop.
+//
+// router_wsplit_kernel writes the pieces once per call, W3 = [hi; mid; lo] as a
+// bf16 [3N, d] matrix; the router kernel then streams them with TMA.
+//
+// Fused routing (N <= 128): one cluster of S CTAs (S = 1, 2 or 4, along z) owns
+// a tile of 128 tokens; CTA r takes k-blocks [r*kb_per, (r+1)*kb_per).
+//   warp 0       TMA producer: x tile [128 tokens x 64 k] and the three piece
+//                tiles [NP experts x 64 k] (bf16, 128-byte swizzle) per stage
+//   warp 1       MMA issuer: per 16-wide k step, three tcgen05.mma (M = 128
+//                tokens, N = NP experts), one per piece, into three TMEM
+//                accumulators
+//   warp 2       TMEM allocator
+//   warps 4..7   TMEM epilogue (thread = token row): z = D_hi + (D_mid + D_lo)
+// Partial logits of the cluster are added in rank order through distributed
+// shared memory (deterministic), the bias is added, and each CTA routes its
+// 128/S rows (softmax, argmax, block ranks, per-expert counts and sums of p).
+// Every mbarrier wait is bounded; a stuck pipeline sets the device error word.
+#include <cooperative_groups.h>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "router_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace swl {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBM = 128;          // tokens per tile (UMMA M)
+constexpr int kBK = 64;           // k per stage (one 128-byte swizzle row of bf16)
+constexpr int kUmmaK = 16;
+constexpr int kPieces = 3;        // hi, mid, lo
+constexpr int kMaxStages = 4;
+constexpr size_t kMaxDynSmem = 232448 - 8192;   // leave room for the static arrays
+
+template <int NP>
+struct TcCfg {
+  static constexpr uint32_t kABytes = kBM * kBK * 2;             // x tile, bf16
+  static constexpr uint32_t kPieceBytes = NP * kBK * 2;          // one piece tile, bf16
+  static constexpr uint32_t kStage = kABytes + kPieces * kPieceBytes;
+  static constexpr int kPS = NP + 4;                             // row stride of the logits tile
+  static constexpr uint32_t kTmemCols = 3 * NP <= 128 ? 128 : (3 * NP <= 256 ? 256 : 512);
+};
+
+struct TcArgs {
+  const float* b_r;       // [N] or null
+  float* logits;          // wide layout only: [T, N] fp32 logits (without the bias)
+  int T, N;
+  int piece_rows;         // rows of one piece in W3 (= N)
+  int nkb;                // k-blocks of 64 over d
+  int kb_per;             // k-blocks per cluster rank
+  int stages;
+  int* expert_idx;
+  float* gate;
+  int* local_rank;
+  int* blk_count;
+  float* blk_psum;
+  WsHeader* hdr;
+};
+
+__device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 h) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(h));
+}
+
+// w = hi + mid + lo exactly (see the file comment).
+__device__ __forceinline__ void split3(float w, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(w);
+  const float r1 = w - __bfloat162float(h);
+  const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(m);
+  hi = bf16_bits(h);
+  mid = bf16_bits(m);
+  lo = bf16_bits(__float2bfloat16_rn(r2));
+}
+
+// W3[p*N + n, k] = piece p of W_r[n, k]; 8 consecutive k per thread (d % 8 == 0).
+__global__ void __launch_bounds__(256)
+router_wsplit_kernel(const float* __restrict__ W_r, __nv_bfloat16* __restrict__ W3, int N, int d) {
+  pdl_trigger();
+  const size_t chunks = static_cast<size_t>(N) * (d / 8);
+  const size_t plane = static_cast<size_t>(N) * d;
+  for (size_t c = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; c < chunks;
+       c += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t off = c * 8;
+    const float4 u0 = *reinterpret_cast<const float4*>(W_r + off);
+    const float4 u1 = *reinterpret_cast<const float4*>(W_r + off + 4);
+    const float w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    uint32_t hi[4], mi[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t h0, m0, l0, h1, m1, l1;
+      split3(w[2 * q], h0, m0, l0);
+      split3(w[2 * q + 1], h1, m1, l1);
+      hi[q] = h0 | (h1 << 16);
+      mi[q] = m0 | (m1 << 16);
+      lo[q] = l0 | (l1 << 16);
+    }
+    *reinterpret_cast<uint4*>(W3 + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(W3 + plane + off) = make_uint4(mi[0], mi[1], mi[2], mi[3]);
+    *reinterpret_cast<uint4*>(W3 + 2 * plane + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+// kWide = false: fused routing of N <= NP experts (cluster of S CTAs along z).
+// kWide = true: logits only, CTA (x, y) writes tokens [128y, 128y+128) x experts
+// [NP*x, NP*x + NP) to a.logits (expert tiles fastest, so the CTAs that run
+// together share the x tile in L2); the softmax kernel routes from there.
+template <int NP, bool kWide>
+__global__ void __launch_bounds__(kThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const TcArgs a) {
+  // tmW: W3 = [hi; mid; lo] as bf16 [3N, d], box [NP rows, 64 k], 128-byte swizzle
+  using C = TcCfg<NP>;
+  constexpr int NPL = NP / 32;
+  constexpr int PS = C::kPS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int stages = a.stages;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + stages * C::kStage);
+  uint64_t* empty_bar = full_bar + kMaxStages;
+  uint64_t* accf_bar = empty_bar + kMaxStages;
+  uint64_t* drain_bar = accf_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* Ps = reinterpret_cast<float*>(smem);   // [kBM][PS] logits, after the main loop
+  __shared__ int eid[kBM];
+  __shared__ int lead_count[kBM];
+  __shared__ float s_psum[kWarps * NP];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = static_cast<int>(cluster.num_blocks());
+  const int r = static_cast<int>(cluster.block_rank());
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && r == 0 && threadIdx.x == 0) {
+    a.hdr->err = kDevOk;   // per-call device status
+    a.hdr->done = 0u;      // arrival counter of the dispatch scan
+  }
+  const int m0 = (kWide ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x)) * kBM;
+  const int n0 = kWide ? static_cast<int>(blockIdx.x) * NP : 0;
+  const int kb0 = r * a.kb_per;
+  const int nk = max(0, min(a.nkb, kb0 + a.kb_per) - kb0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(&full_bar[s], 1);
+      ptx::mbar_init(&empty_bar[s], 1);
+    }
+    ptx::mbar_init(accf_bar, 1);
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmX);
+    ptx::prefetch_tmap(&tmW);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicExch(&a.hdr->err, kDevPipelineTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_x = ptx::l2_policy_evict_last();    // x: the gather reads it again
+      const uint64_t pol_w = ptx::l2_policy_evict_last();    // W3: read by every tile
+      uint32_t issued = 0u, last_par = 0u;
+      pdl_wait();   // W3 comes from the split kernel
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
+        if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) {
+          fail();
+          break;
+        }
+        uint8_t* st = smem + s * C::kStage;
+        const int kc = (kb0 + i) * kBK;
+        ptx::mbar_arrive_expect_tx(&full_bar[s], C::kStage);
+        ptx::tma_load_2d(st, &tmX, &full_bar[s], kc, m0, pol_x);
+#pragma unroll
+        for (int p = 0; p < kPieces; ++p)
+          ptx::tma_load_2d(st + C::kABytes + p * C::kPieceBytes, &tmW, &full_bar[s], kc,
+                           p * a.piece_rows + n0, pol_w);
+        issued |= 1u << s;
+        last_par = (last_par & ~(1u << s)) | (ph << s);
+      }
+      // every issued load lands before the stage memory is reused or the CTA exits
+      for (int s = 0; s < stages; ++s) {
+        if (issued & (1u << s)) {
+          volatile int never = 0;
+          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never))
+            atomicExch(&a.hdr->err, kDevPipelineTimeout);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = ptx::umma_idesc_bf16_f32(NP);
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
+        if (!ptx::mbar_wait(&full_bar[s], ph, abort_flag)) {
+          fail();
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a_addr = ptx::smem_u32(smem + s * C::kStage);
+        const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+        for (int k = 0; k < kBK / kUmmaK; ++k) {
+          const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + k * kUmmaK * 2);
+#pragma unroll
+          for (int p = 0; p < kPieces; ++p) {
+            const uint64_t bd =
+                ptx::umma_desc_sw128_kmajor(b_addr + p * C::kPieceBytes + k * kUmmaK * 2);
+            ptx::umma_bf16(tmem_base + static_cast<uint32_t>(p * NP), ad, bd, idesc,
+                           (i | k) != 0 ? 1u : 0u);
+          }
+        }
+        ptx::umma_commit(&empty_bar[s]);    // frees the stage once these MMAs are done
+      }
+      if (ok && nk > 0) ptx::umma_commit(accf_bar);
+      // all MMAs of this thread complete before TMEM is released
+      ptx::umma_commit(drain_bar);
+      volatile int never = 0;
+      if (!ptx::mbar_wait(drain_bar, 0u, &never)) atomicExch(&a.hdr->err, kDevPipelineTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ TMEM epilogue
+    bool have = false;
+    if (nk > 0) {
+      const bool got = ptx::mbar_wait(accf_bar, 0u, abort_flag);
+      have = __all_sync(0xffffffffu, got);
+      if (!have && lane == 0) fail();
+    }
+    ptx::tc_fence_after();
+    const int q = warp & 3;
+    const int row = q * 32 + lane;                 // TMEM lane = token row of the tile
+#pragma unroll 1
+    for (int c0 = 0; c0 < NP; c0 += 32) {
+      float z[32];
+      if (have) {
+        uint32_t r0[32], r1[32], r2[32];
+        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                            static_cast<uint32_t>(c0);
+        ptx::tmem_ld_32x32b_x32(ta, r0);
+        ptx::tmem_ld_32x32b_x32(ta + NP, r1);
+        ptx::tmem_ld_32x32b_x32(ta + 2 * NP, r2);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          z[j] = __uint_as_float(r0[j]) + (__uint_as_float(r1[j]) + __uint_as_float(r2[j]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = 0.f;
+      }
+      float* pr = Ps + row * PS + c0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(pr + j) = make_float4(z[j], z[j + 1], z[j + 2], z[j + 3]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if constexpr (kWide) {
+    // coalesced rows of the logits tile (the bias is added by the softmax kernel)
+    const bool vec = (a.N % 4) == 0;
+    for (int idx = threadIdx.x; idx < kBM * (NP / 4); idx += kThreads) {
+      const int i = idx / (NP / 4), n = (idx % (NP / 4)) * 4;
+      const int t = m0 + i;
+      if (t >= a.T || n0 + n >= a.N) continue;
+      const float4 v = *reinterpret_cast<const float4*>(Ps + i * PS + n);
+      float* dst = a.logits + static_cast<size_t>(t) * a.N + n0 + n;
+      if (vec) {
+        *reinterpret_cast<float4*>(dst) = v;
+      } else {
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (n0 + n + c < a.N) dst[c] = vv[c];
+      }
+    }
+    return;
+  }
+  cluster.sync();   // every partial logits tile of the cluster is complete
+
+  // this CTA's rows [r*R, r*R + R): partials added in rank order, plus the bias;
+  // written in place (the peers read only their own rows of this tile)
+  const int R = kBM / S;
+  const int row0 = r * R;
+  const float* part[4];
+#pragma unroll
+  for (int s2 = 0; s2 < 4; ++s2) part[s2] = cluster.map_shared_rank(Ps, s2 < S ? s2 : 0);
+  for (int idx = threadIdx.x; idx < R * (NP / 4); idx += kThreads) {
+    const int i = idx / (NP / 4), n = (idx % (NP / 4)) * 4;
+    const int off = (row0 + i) * PS + n;
+    float4 v = *reinterpret_cast<const float4*>(part[0] + off);
+#pragma unroll
+    for (int s2 = 1; s2 < 4; ++s2) {
+      if (s2 < S) {
+        const float4 u = *reinterpret_cast<const float4*>(part[s2] + off);
+        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+      }
+    }
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      Ps[off + c] = (n + c < a.N) ? vv[c] + (a.b_r ? a.b_r[n + c] : 0.f) : -INFINITY;
+  }
+  cluster.sync();   // the peers have finished reading this CTA's partial tile
+
+  const int t0 = m0 + row0;
+  const int ntok = max(0, min(R, a.T - t0));
+  route_rows<NPL, kWarps>(Ps + row0 * PS, PS, R, ntok, t0, a.N, blockIdx.x * S + r,
+                          a.expert_idx, a.gate, a.local_rank, a.blk_count, a.blk_psum, a.hdr, eid,
+                          lead_count, s_psum);
+}
+
+template <int NP>
+size_t tc_smem_bytes(int stages) {
+  return 1024 + static_cast<size_t>(stages) * TcCfg<NP>::kStage +
+         (2 * kMaxStages + 2) * sizeof(uint64_t) + 2 * sizeof(uint32_t);
+}
+
+template <int NP, bool kWide>
+cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
+                        const CUtensorMap& tmW, const float* b_r, int* expert_idx, float* gate,
+                        int* local_rank, cudaStream_t stream) {
+  TcArgs a;
+  a.b_r = b_r;
+  a.logits = ws.logits;
+  a.T = static_cast<int>(s.T);
+  a.N = static_cast<int>(s.N);
+  a.piece_rows = static_cast<int>(s.N);
+  a.nkb = static_cast<int>((s.d + kBK - 1) / kBK);
+  a.kb_per = s.kslice / kBK;
+  a.expert_idx = expert_idx;
+  a.gate = gate;
+  a.local_rank = local_rank;
+  a.blk_count = ws.blk_count;
+  a.blk_psum = ws.blk_psum;
+  a.hdr = ws.hdr;
+  int stages = kMaxStages;
+  while (stages > 2 && tc_smem_bytes<NP>(stages) > kMaxDynSmem) --stages;
+  a.stages = stages;
+  const size_t smem = tc_smem_bytes<NP>(stages);
+  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NP, kWide>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned t_tiles = static_cast<unsigned>((s.T + kBM - 1) / kBM);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = kWide ? dim3(static_cast<unsigned>((s.N + NP - 1) / NP), t_tiles, 1)
+                      : dim3(t_tiles, 1, static_cast<unsigned>(s.ksplit_eff));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = kWide ? 1u : static_cast<unsigned>(s.ksplit_eff);
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, router_tc_kernel<NP, kWide>, tmX, tmW, a);
+}
+
+}  // namespace
+
+int router_tc_padded_experts(int64_t N) {
+  return N > kFusedRouterMaxN ? 128 : static_cast<int>((N + 31) / 32 * 32);
+}
+
+cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
+                             const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
+                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
+  // the three bf16 pieces of W_r, then the router (programmatic dependent launch)
+  const size_t chunks = static_cast<size_t>(s.N) * static_cast<size_t>(s.d / 8);
+  size_t blocks = (chunks + 255) / 256;
+  if (blocks > 4 * 148) blocks = 4 * 148;
+  if (blocks < 1) blocks = 1;
+  router_wsplit_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      W_r, static_cast<__nv_bfloat16*>(ws.w3), static_cast<int>(s.N), static_cast<int>(s.d));
+  cudaError_t e = cudaGetLastError();
+  count_launch();
+  if (e != cudaSuccess) return e;
+  if (s.router_path == kRouterTCWide) {
+    e = launch_tc_t<128, true>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream);
+  } else {
+    switch (router_tc_padded_experts(s.N)) {
+      case 32: e = launch_tc_t<32, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
+      case 64: e = launch_tc_t<64, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
+      case 96: e = launch_tc_t<96, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
+      case 128: e = launch_tc_t<128, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
+      default: e = cudaErrorInvalidValue; break;
+    }
+  }
+  count_launch();
+  return e;
+}
+
+}  // namespace swl

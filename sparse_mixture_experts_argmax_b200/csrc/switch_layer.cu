@@ -2,8 +2,10 @@
 // capacity, workspace layout, TMA descriptors and the launch sequence.
 //
 // Stage order on the caller's stream (no host synchronisation inside):
-//   0 router logits        fp32 FFMA GEMM            (router.cu)
-//   1 router softmax       max/argmax/gate, ranks     (router.cu)
+//   0 router               fp32 logits + softmax/argmax/gate + block ranks; bf16
+//                          layers with N <= 128: one tcgen05 kernel (router_tc.cu),
+//                          fp32 layers: FFMA kernels (router.cu)
+//   1 router softmax       N > 128 only: max/argmax/gate, ranks (router.cu)
 //   2 dispatch scan        offsets, capacity, aux     (dispatch.cu)
 //   3 dispatch gather      pos, packed expert rows    (dispatch.cu)
 //   4 expert FFN           GEMM1 + bias + ReLU, GEMM2 + bias + gate + combine
@@ -42,7 +44,9 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   Workspace w{};
   w.hdr = reinterpret_cast<WsHeader*>(take(sizeof(WsHeader)));
   w.logits = reinterpret_cast<float*>(
-      take(s.router_path != kRouterWide ? 0 : static_cast<size_t>(s.ksplit_eff) * T * N * 4));
+      take(s.router_path != kRouterWide && s.router_path != kRouterTCWide
+               ? 0
+               : static_cast<size_t>(s.ksplit_eff) * T * N * 4));
   w.blk_count = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_off = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_psum = reinterpret_cast<float*>(take(nb * N * 4));
@@ -53,6 +57,10 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.psum64 = reinterpret_cast<double*>(take(N * 8));
   w.slot_token = reinterpret_cast<int*>(take(T * 4));
   w.ready = reinterpret_cast<int*>(take((T / 16 + N + 1) * 4));
+  w.w3 = reinterpret_cast<void*>(
+      take(s.router_path == kRouterTC || s.router_path == kRouterTCWide
+               ? 3 * N * static_cast<size_t>(s.d) * 2
+               : 0));
   w.xbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
   w.hbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d_ff) * elem));
   if (host_io) {
@@ -133,7 +141,7 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->dtype = dtype;
   s->C = switch_layer_capacity(T, N, cf);
   s->C_eff = s->C < T ? s->C : T;
-  const RouterPlan rp = router_plan(T, d, N);
+  const RouterPlan rp = router_plan(T, d, N, dtype);
   s->router_path = rp.path;
   s->kslice = rp.kslice;
   s->ksplit_eff = rp.ksplit;
@@ -163,9 +171,18 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
                       : cudaEventRecord(e, stream)) == cudaSuccess;
   };
   if (!rec(0)) return SWL_ERR_CUDA;
-  if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert, stream) !=
-      cudaSuccess)
+  if (s.router_path == kRouterTC || s.router_path == kRouterTCWide) {
+    CUtensorMap tx, tw;
+    if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
+        !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N, router_tc_padded_experts(s.N)))
+      return SWL_ERR_CUDA;
+    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, stream) !=
+        cudaSuccess)
+      return SWL_ERR_CUDA;
+  } else if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert,
+                                  stream) != cudaSuccess) {
     return SWL_ERR_CUDA;
+  }
   if (!rec(1)) return SWL_ERR_CUDA;
   if (s.N > kFusedRouterMaxN &&
       launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
@@ -208,7 +225,8 @@ static swl_status validate_io(const Shape& s, const void* x, const float* W_r, c
   if (s.T > 0 && (!x || !out || !expert_idx || !gate || !pos)) return SWL_ERR_INVALID_ARG;
   if (!aligned(workspace, 256)) return SWL_ERR_UNSUPPORTED;
   const uintptr_t a = s.dtype == SWL_BF16 ? 16 : 4;
-  if (!aligned(W1, a) || !aligned(W2, a) || !aligned(W_r, 4) || !aligned(b1, s.dtype ? 2 : 4) ||
+  if (!aligned(W1, a) || !aligned(W2, a) ||
+      !aligned(W_r, s.router_path == kRouterTC || s.router_path == kRouterTCWide ? 16 : 4) || !aligned(b1, s.dtype ? 2 : 4) ||
       !aligned(b2, s.dtype ? 2 : 4))
     return SWL_ERR_UNSUPPORTED;
   if (!host_io && (!aligned(x, a) || !aligned(out, a))) return SWL_ERR_UNSUPPORTED;
