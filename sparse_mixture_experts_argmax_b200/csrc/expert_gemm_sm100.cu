@@ -23,7 +23,8 @@
 //   warp 0      TMA producer (one thread): A and B k-blocks of 64 elements into a
 //               ring of shared-memory stages (128-byte swizzle)
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
-//   warp 2      TMEM allocator (512 columns: two 256-column accumulators)
+//   warp 2      TMEM allocator (512 columns: four 128-column accumulators for
+//               token tiles of up to 128 rows, else two of 256)
 //   warp 3      tile scheduler (one thread): claims, decodes and publishes tiles
 //   warps 4..7  epilogue: tcgen05.ld, bias / ReLU / gate in fp32, bf16 pack,
 //               transpose through shared memory, 16-byte stores
@@ -48,7 +49,7 @@ constexpr int kBM = 128;              // UMMA M: output features per tile
 constexpr int kBK = 64;               // K elements per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 16;            // K per tcgen05.mma (bf16)
 constexpr int kMaxStages = 12;
-constexpr int kAccCols = 256;         // TMEM columns per accumulator buffer
+constexpr int kMaxAcc = 4;            // TMEM accumulator buffers (512 / acc_cols)
 constexpr int kTmemCols = 512;
 constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KiB
 constexpr int kEpiStageBytes = 4 * 32 * 32 * 2;   // per-warp 32x32 bf16 transpose tiles
@@ -75,6 +76,7 @@ struct FfnArgs {
   int num_experts;
   int bn;         // token rows per tile (multiple of 16, <= 256)
   int stages;
+  int num_acc;    // TMEM accumulators: 4 of 128 columns when bn <= 128, else 2 of 256
   PhaseArgs ph[2];
 };
 
@@ -90,7 +92,7 @@ struct TileSlot {
   int row0;       // first packed row of the tile
 };
 
-constexpr int kTileRing = 4;    // decoded tiles handed to the producer, MMA and epilogue
+constexpr int kTileRing = 8;    // decoded tiles handed to the producer, MMA and epilogue
 
 // Work item t: GEMM1 tiles [0, total0) then GEMM2 tiles.  Within a phase, the
 // tiles of expert e occupy [P[e]*m_tiles, P[e+1]*m_tiles) (P = tile prefix) with
@@ -145,9 +147,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(epi) + kEpiStageBytes);
   uint64_t* full_bar = bars;                      // [kMaxStages]
   uint64_t* empty_bar = bars + kMaxStages;        // [kMaxStages]
-  uint64_t* tfull_bar = bars + 2 * kMaxStages;    // [2]
-  uint64_t* tempty_bar = tfull_bar + 2;           // [2]
-  uint64_t* drain_bar = tempty_bar + 2;           // [1]
+  uint64_t* tfull_bar = bars + 2 * kMaxStages;    // [kMaxAcc]
+  uint64_t* tempty_bar = tfull_bar + kMaxAcc;     // [kMaxAcc]
+  uint64_t* drain_bar = tempty_bar + kMaxAcc;     // [1]
   uint64_t* tile_full = drain_bar + 1;            // [kTileRing]
   uint64_t* tile_empty = tile_full + kTileRing;   // [kTileRing]
   uint64_t* take_bar = tile_empty + kTileRing;    // [1] the producer took a tile
@@ -162,7 +164,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       ptx::mbar_init(&full_bar[s], 1);
       ptx::mbar_init(&empty_bar[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxAcc; ++i) {
       ptx::mbar_init(&tfull_bar[i], 1);
       ptx::mbar_init(&tempty_bar[i], 4);      // one arrive per epilogue warp
     }
@@ -188,6 +190,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int acc_cols = kTmemCols / args.num_acc;
   pdl_wait();   // tile prefix, packed rows, gate and counters come from earlier kernels
   const int ntiles = args.tile_prefix[args.num_experts];
   const int total0 = ntiles * args.ph[0].m_tiles;
@@ -314,7 +317,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         const uint32_t idesc = ptx::umma_idesc_bf16_f32(n_mma);
         if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { fail(); break; }
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * acc_cols);
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag)) { fail(); ok = false; break; }
           ptx::tc_fence_after();
@@ -331,7 +334,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         }
         if (!ok) break;
         ptx::umma_commit(&tfull_bar[acc]);          // accumulator ready for the epilogue
-        if (++acc == 2) { acc = 0; aph ^= 1u; }
+        if (++acc == args.num_acc) { acc = 0; aph ^= 1u; }
       }
       // drain: all MMAs issued by this thread complete before TMEM is released
       ptx::umma_commit(drain_bar);
@@ -374,7 +377,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
       ptx::tc_fence_after();
       const uint32_t t_base =
-          tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
+          tmem_base + static_cast<uint32_t>(acc * acc_cols) + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < rows; c0 += 32) {
         const int dst = dst_next;
         const float g = g_next;
@@ -417,7 +420,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         ptx::mbar_arrive(&tempty_bar[acc]);
         ptx::mbar_arrive(&tile_empty[slot]);
       }
-      if (++acc == 2) { acc = 0; aph ^= 1u; }
+      if (++acc == args.num_acc) { acc = 0; aph ^= 1u; }
     }
   }
   ptx::tc_fence_before();
@@ -430,7 +433,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
 
 size_t ffn_smem_bytes(int bn, int stages) {
   return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
-         kEpiStageBytes + (2 * kMaxStages + 6 + 2 * kTileRing) * sizeof(uint64_t) +
+         kEpiStageBytes + (2 * kMaxStages + 2 * kMaxAcc + 2 + 2 * kTileRing) * sizeof(uint64_t) +
          kTileRing * sizeof(TileSlot) + 2 * sizeof(uint32_t);
 }
 
@@ -460,6 +463,7 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.err = &ws.hdr->err;
   a.num_experts = static_cast<int>(s.N);
   a.bn = s.tile_rows;
+  a.num_acc = a.bn <= kTmemCols / kMaxAcc ? kMaxAcc : 2;
   for (int p = 0; p < 2; ++p) {
     const int64_t M = p == 0 ? s.d_ff : s.d;
     const int64_t K = p == 0 ? s.d : s.d_ff;

@@ -97,11 +97,17 @@ cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void
                                  int* local_rank, cudaStream_t stream);
 // Tensor-core router (kRouterTC, kRouterTCWide): splits W_r into ws.w3, then routes.
 // tmX = x as bf16 [T, d] (box 64 x 128), tmW = ws.w3 as bf16 [3N, d] (box 64 x
-// router_tc_padded_experts(N)), both with 128-byte swizzle.  Two launches.
+// router_tc_padded_experts(N)), both with 128-byte swizzle.  Two launches.  The
+// router CTAs also prefetch [l2_prefetch, +l2_prefetch_bytes) into L2 once their
+// own loads have landed (16-byte aligned, a multiple of 16 bytes; 0 bytes: none).
 int router_tc_padded_experts(int64_t N);
 cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
                              const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
-                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream);
+                             int* expert_idx, float* gate, int* local_rank,
+                             const void* l2_prefetch, size_t l2_prefetch_bytes,
+                             cudaStream_t stream);
+// Expert weights fetched into L2 during the router and dispatch stages.
+constexpr size_t kL2PrefetchBytes = 64u << 20;
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);

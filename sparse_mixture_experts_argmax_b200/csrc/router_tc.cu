@@ -77,6 +77,8 @@ struct TcArgs {
   int* blk_count;
   float* blk_psum;
   WsHeader* hdr;
+  const uint8_t* pf;      // bytes fetched into L2 once this CTA's loads have landed
+  size_t pf_bytes;        // (the expert weights the FFN streams first; 0: none)
 };
 
 __device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 h) {
@@ -222,6 +224,21 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             atomicExch(&a.hdr->err, kDevPipelineTimeout);
         }
       }
+      // HBM is idle from here until the expert FFN starts: this CTA's share of the
+      // weights the FFN streams first goes to L2 meanwhile (no completion needed)
+      if (a.pf_bytes > 0) {
+        constexpr size_t kChunk = 64 << 10;
+        const size_t nct = static_cast<size_t>(gridDim.x) * gridDim.y * gridDim.z;
+        const size_t id = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x +
+                          blockIdx.x;
+        const size_t share = ((a.pf_bytes + nct - 1) / nct + 15) & ~static_cast<size_t>(15);
+        const size_t lo = id * share;
+        const size_t hi = lo + share < a.pf_bytes ? lo + share : a.pf_bytes;
+        for (size_t o = lo; o < hi; o += kChunk) {
+          const size_t n = (hi - o < kChunk ? hi - o : kChunk) & ~static_cast<size_t>(15);
+          if (n > 0) ptx::prefetch_l2_bulk(a.pf + o, static_cast<uint32_t>(n));
+        }
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -365,8 +382,10 @@ size_t tc_smem_bytes(int stages) {
 template <int NP, bool kWide>
 cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
                         const CUtensorMap& tmW, const float* b_r, int* expert_idx, float* gate,
-                        int* local_rank, cudaStream_t stream) {
+                        int* local_rank, const void* pf, size_t pf_bytes, cudaStream_t stream) {
   TcArgs a;
+  a.pf = static_cast<const uint8_t*>(pf);
+  a.pf_bytes = pf_bytes;
   a.b_r = b_r;
   a.logits = ws.logits;
   a.T = static_cast<int>(s.T);
@@ -414,7 +433,9 @@ int router_tc_padded_experts(int64_t N) {
 
 cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
                              const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
-                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
+                             int* expert_idx, float* gate, int* local_rank,
+                             const void* l2_prefetch, size_t l2_prefetch_bytes,
+                             cudaStream_t stream) {
   // the three bf16 pieces of W_r, then the router (programmatic dependent launch)
   const size_t chunks = static_cast<size_t>(s.N) * static_cast<size_t>(s.d / 8);
   size_t blocks = (chunks + 255) / 256;
@@ -426,13 +447,14 @@ cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W
   count_launch();
   if (e != cudaSuccess) return e;
   if (s.router_path == kRouterTCWide) {
-    e = launch_tc_t<128, true>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream);
+    e = launch_tc_t<128, true>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch,
+                               l2_prefetch_bytes, stream);
   } else {
     switch (router_tc_padded_experts(s.N)) {
-      case 32: e = launch_tc_t<32, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
-      case 64: e = launch_tc_t<64, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
-      case 96: e = launch_tc_t<96, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
-      case 128: e = launch_tc_t<128, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, stream); break;
+      case 32: e = launch_tc_t<32, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
+      case 64: e = launch_tc_t<64, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
+      case 96: e = launch_tc_t<96, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
+      case 128: e = launch_tc_t<128, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
       default: e = cudaErrorInvalidValue; break;
     }
   }

@@ -114,6 +114,15 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* tmap, int3
                : "memory");
 }
 
+// Bring [addr, addr + bytes) into L2 (no completion; bytes a multiple of 16,
+// addr 16-byte aligned).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* addr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(addr)),
+               "r"(bytes)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -176,8 +176,11 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
     if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
         !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N, router_tc_padded_experts(s.N)))
       return SWL_ERR_CUDA;
-    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, stream) !=
-        cudaSuccess)
+    // the FFN's first tiles stream W1 from its start: fetch a slice into L2 now
+    const size_t w1_bytes = static_cast<size_t>(s.N) * s.d_ff * s.d * 2;
+    const size_t pf = w1_bytes < kL2PrefetchBytes ? w1_bytes : kL2PrefetchBytes;
+    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, W1, pf,
+                         stream) != cudaSuccess)
       return SWL_ERR_CUDA;
   } else if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert,
                                   stream) != cudaSuccess) {

@@ -247,3 +247,32 @@ def test_nonfinite_router_input_reports_device_status():
     # the context is still usable
     ig["x"][7] = 0.5
     swl.forward(ig, spec.cf)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_router_decision_needs_float32_weights(dtype):
+    """The router works in float32 (selective precision).  Experts 0 and 1 have
+    weights 1 + 2^-9 and 1 + 2^-9 + 2^-17: equal in bfloat16, and equal after
+    the first two bf16 pieces of an fp32 split (the 2^-17 lives only in the third
+    piece).  Their logits for x = c * ones(64) differ by c * 64 * 2^-17, about 64
+    ulps of the logit, far above the worst-case fp32 accumulation error
+    (64 * ulp/2), so a float32 router sends every token with c > 0 to expert 1,
+    while any router that drops the low piece ties them and takes expert 0."""
+    T, d, d_ff, N, cf = 256, 64, 64, 8, float(8)
+    spec = synth.LayerSpec("fp32_router_%s" % dtype, T, d, d_ff, N, cf, dtype)
+    ic = synth.make_layer_inputs(spec, device="cpu")
+    scale = torch.tensor([0.5, 1.0, 2.0, 4.0, -1.0])[torch.arange(T) % 5]
+    ic["x"] = (scale[:, None] * torch.ones(T, d)).to(ic["x"].dtype)
+    W_r = torch.zeros(N, d, dtype=torch.float32)
+    W_r[0] = 1.0 + 2.0 ** -9
+    W_r[1] = 1.0 + 2.0 ** -9 + 2.0 ** -17
+    assert float(W_r[1, 0]) - float(W_r[0, 0]) == 2.0 ** -17      # exact in fp32
+    assert torch.equal(W_r[0].to(torch.bfloat16), W_r[1].to(torch.bfloat16))
+    ic["W_r"], ic["b_r"] = W_r, None
+    ig = {k: (v.cuda() if v is not None else None) for k, v in ic.items()}
+    got = _run(ig, cf)
+    ref = oracle.switch_forward(ic["x"], ic["W_r"], ic["W1"], ic["b1"], ic["W2"], ic["b2"], cf)
+    pos = (scale > 0).numpy()
+    assert np.all(ref["expert_idx"][pos] == 1)
+    check_routing(got, ref, oracle.capacity(T, N, cf), T)
+    check_close(_np(got["out"]), ref["out"], dtype)
