@@ -44,7 +44,8 @@
 namespace swl {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kEpiWarps = 8;          // two per TMEM lane quarter, alternating column chunks
+constexpr int kThreads = 128 + 32 * kEpiWarps;
 constexpr int kBM = 128;              // UMMA M: output features per tile
 constexpr int kBK = 64;               // K elements per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 16;            // K per tcgen05.mma (bf16)
@@ -52,7 +53,8 @@ constexpr int kMaxStages = 12;
 constexpr int kMaxAcc = 4;            // TMEM accumulator buffers (512 / acc_cols)
 constexpr int kTmemCols = 512;
 constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KiB
-constexpr int kEpiStageBytes = 4 * 32 * 32 * 2;   // per-warp 32x32 bf16 transpose tiles
+constexpr int kEpiStageBytes = kEpiWarps * 32 * 32 * 2;   // per-warp 32x32 bf16 transpose tiles
+constexpr int kMaxPending = 2;        // GEMM1 tiles an epilogue warp publishes per fence
 
 // One GEMM of the expert FFN.
 struct PhaseArgs {
@@ -166,12 +168,12 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     }
     for (int i = 0; i < kMaxAcc; ++i) {
       ptx::mbar_init(&tfull_bar[i], 1);
-      ptx::mbar_init(&tempty_bar[i], 4);      // one arrive per epilogue warp
+      ptx::mbar_init(&tempty_bar[i], kEpiWarps);   // one arrive per epilogue warp
     }
     ptx::mbar_init(drain_bar, 1);
     for (int i = 0; i < kTileRing; ++i) {
       ptx::mbar_init(&tile_full[i], 1);        // the scheduler publishes a tile
-      ptx::mbar_init(&tile_empty[i], 4);       // the epilogue warps retire it
+      ptx::mbar_init(&tile_empty[i], kEpiWarps);   // the epilogue warps retire it
     }
     ptx::mbar_init(take_bar, 1);
     *abort_flag = 0;
@@ -232,7 +234,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           ts.row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
           if (c.phase == 1) {
             // hbuf rows of token tile g: every GEMM1 epilogue warp of g has stored them
-            const int target = 4 * args.ph[0].m_tiles;
+            const int target = kEpiWarps * args.ph[0].m_tiles;
             bool ready = ld_acquire(args.ready + c.g) >= target;
             const uint64_t t0 = ptx::globaltimer_ns();
             while (!ready) {
@@ -345,12 +347,35 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                        // TMEM lane quarter of this warp
-    __nv_bfloat16* st = epi + q * 32 * 32;         // [32 tokens][32 features]
+    const int half = (warp - 4) >> 2;              // column chunks half, half + 2, ...
+    __nv_bfloat16* st = epi + (warp - 4) * 32 * 32;   // [32 tokens][32 features]
+    // GEMM1 tiles whose hbuf rows this warp stored but has not yet published:
+    // one fence covers up to kMaxPending of them.  The warp publishes before it
+    // could block, so a GEMM2 tile never waits on a warp that is itself waiting.
+    int pend0 = 0, pend1 = 0;   // token tiles of the unpublished GEMM1 tiles (warp-uniform)
+    int npending = 0;
+    auto publish = [&]() {
+      if (npending == 0) return;
+      fence_proxy_async_global();   // generic-proxy stores -> other CTAs' TMA reads
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) {
+        atomicAdd(args.ready + pend0, 1);
+        if (npending > 1) atomicAdd(args.ready + pend1, 1);
+      }
+      npending = 0;
+    };
+    // publish before blocking on a barrier that is not yet complete (warp-uniform)
+    auto publish_if_blocked = [&](uint64_t* bar, uint32_t parity) {
+      if (npending > 0 && __any_sync(0xffffffffu, !ptx::mbar_try_wait(bar, parity))) publish();
+    };
     int acc = 0;
     uint32_t aph = 0;
     for (int i = 0;; ++i) {
       const int slot = i % kTileRing;
-      if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) { fail(); break; }
+      const uint32_t tpar = (i / kTileRing) & 1;
+      publish_if_blocked(&tile_full[slot], tpar);
+      if (!ptx::mbar_wait(&tile_full[slot], tpar, abort_flag)) { fail(); break; }
       const TileSlot ts = tile_ring[slot];
       if (ts.t < 0) break;
       const PhaseArgs& P = args.ph[ts.phase];
@@ -360,28 +385,36 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       const int f = feat0 + lane;
       // operands of the epilogue, fetched before the accumulator is ready:
       // this lane's bias, and the destination row / gate of column (c0 + lane)
+      // of each of this warp's column chunks
+      constexpr int kMaxChunks = 256 / 64;         // chunks of 32 per warp at 256 rows
       const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.M + f]) : 0.f;
-      auto fetch_col = [&](int c0, int& dst, float& g) {
-        const int col = c0 + lane;
+      int dsts[kMaxChunks];
+      float gs[kMaxChunks];
+#pragma unroll
+      for (int k = 0; k < kMaxChunks; ++k) {
+        const int col = (2 * k + half) * 32 + lane;
         if (P.mode == 1) {
-          dst = (col < rows) ? __ldg(args.slot_token + row0 + col) : 0;
-          g = (col < rows) ? __ldg(args.gate + dst) : 0.f;
+          dsts[k] = (col < rows) ? __ldg(args.slot_token + row0 + col) : 0;
         } else {
-          dst = row0 + col;
-          g = 1.f;
+          dsts[k] = row0 + col;
         }
-      };
-      int dst_next;
-      float g_next;
-      fetch_col(0, dst_next, g_next);
+      }
+#pragma unroll
+      for (int k = 0; k < kMaxChunks; ++k) {
+        const int col = (2 * k + half) * 32 + lane;
+        gs[k] = (P.mode == 1 && col < rows) ? __ldg(args.gate + dsts[k]) : 1.f;
+      }
+      publish_if_blocked(&tfull_bar[acc], aph);
       if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
       ptx::tc_fence_after();
       const uint32_t t_base =
           tmem_base + static_cast<uint32_t>(acc * acc_cols) + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 0; c0 < rows; c0 += 32) {
-        const int dst = dst_next;
-        const float g = g_next;
-        if (c0 + 32 < rows) fetch_col(c0 + 32, dst_next, g_next);
+#pragma unroll
+      for (int k = 0; k < kMaxChunks; ++k) {
+        const int c0 = (2 * k + half) * 32;
+        if (c0 >= rows) break;
+        const int dst = dsts[k];
+        const float g = gs[k];
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
         ptx::tmem_ld_wait();
@@ -397,8 +430,8 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         }
         __syncwarp();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int idx = lane + 32 * k;
+        for (int kk = 0; kk < 4; ++kk) {
+          const int idx = lane + 32 * kk;
           const int j = idx >> 2, part = idx & 3;
           const int drow = __shfl_sync(0xffffffffu, dst, j);
           if (c0 + j < rows && feat0 + part * 8 < P.M) {
@@ -409,19 +442,18 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         __syncwarp();
       }
       ptx::tc_fence_before();
-      if (ts.phase == 0) {
-        // publish this warp's rows of hbuf to GEMM2 tiles (TMA reads, other CTAs)
-        fence_proxy_async_global();
-        __threadfence();
-      }
       __syncwarp();
       if (lane == 0) {
-        if (ts.phase == 0) atomicAdd(args.ready + ts.g, 1);
         ptx::mbar_arrive(&tempty_bar[acc]);
         ptx::mbar_arrive(&tile_empty[slot]);
       }
+      if (ts.phase == 0) {
+        if (npending == 0) pend0 = ts.g; else pend1 = ts.g;
+        if (++npending == kMaxPending) publish();
+      }
       if (++acc == args.num_acc) { acc = 0; aph ^= 1u; }
     }
+    publish();
   }
   ptx::tc_fence_before();
   __syncthreads();

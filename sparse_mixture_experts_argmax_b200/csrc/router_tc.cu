@@ -197,18 +197,28 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       const uint64_t pol_x = ptx::l2_policy_evict_last();    // x: the gather reads it again
       const uint64_t pol_w = ptx::l2_policy_evict_last();    // W3: read by every tile
       uint32_t issued = 0u, last_par = 0u;
+      // x does not depend on the split kernel: the first stages' x tiles are
+      // requested before waiting for it, then their W3 pieces
+      const int first = nk < stages ? nk : stages;
+      for (int i = 0; i < first; ++i) {
+        ptx::mbar_arrive_expect_tx(&full_bar[i], C::kStage);
+        ptx::tma_load_2d(smem + i * C::kStage, &tmX, &full_bar[i], (kb0 + i) * kBK, m0, pol_x);
+        issued |= 1u << i;
+      }
       pdl_wait();   // W3 comes from the split kernel
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
-        if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) {
-          fail();
-          break;
-        }
         uint8_t* st = smem + s * C::kStage;
         const int kc = (kb0 + i) * kBK;
-        ptx::mbar_arrive_expect_tx(&full_bar[s], C::kStage);
-        ptx::tma_load_2d(st, &tmX, &full_bar[s], kc, m0, pol_x);
+        if (i >= first) {
+          if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) {
+            fail();
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full_bar[s], C::kStage);
+          ptx::tma_load_2d(st, &tmX, &full_bar[s], kc, m0, pol_x);
+        }
 #pragma unroll
         for (int p = 0; p < kPieces; ++p)
           ptx::tma_load_2d(st + C::kABytes + p * C::kPieceBytes, &tmW, &full_bar[s], kc,
