@@ -10,7 +10,10 @@
  * formula, "The routing mechanics in detail", "The selective precision
  * solution"; "Switch Transformer, explained." recipe steps 2-5):
  *
- *   z_t   = W_r x_t + b_r                     router logits, fp32
+ *   z_t   = W_r x_t + b_r                     router logits, fp32 (bf16 layers: computed
+ *                                             on the tensor cores from the exact split
+ *                                             W_r = hi + mid + lo into three bf16
+ *                                             matrices, products exact, fp32 accumulation)
  *   p_t   = softmax(z_t)                      fp32
  *   e_t   = argmax_i p_t,i                    lowest index on ties
  *   g_t   = p_t,e_t                           gate
@@ -71,9 +74,12 @@ typedef enum swl_dtype { SWL_F32 = 0, SWL_BF16 = 1 } swl_dtype;
 #define SWL_WS_HOST_IO 1
 
 /* Number of timed stages and their order (see switch_layer_forward_timed):
- * 0 router (logits; for N <= 128 also softmax/argmax/ranks), 1 router softmax for N > 128
- * (empty otherwise), 2 dispatch scan + aux loss, 3 dispatch gather, 4 expert FFN
- * (GEMM1 + bias + ReLU and GEMM2 + bias + gate + combine). */
+ * 0 router (logits; for N <= 128 also softmax/argmax/ranks; bf16 layers include
+ * the split of W_r into its bf16 pieces), 1 router softmax for N > 128 (empty
+ * otherwise), 2 dispatch scan + aux loss, 3 dispatch gather, 4 expert FFN
+ * (GEMM1 + bias + ReLU and GEMM2 + bias + gate + combine).  For N <= 128 and
+ * batches whose x is at most 16 MiB, scan and gather run as one kernel, timed in
+ * stage 2; stage 3 is then empty. */
 #define SWL_NUM_STAGES 5
 
 /* Expert capacity C = ceil(capacity_factor * T / N) ("Capacity Factor" section
@@ -104,7 +110,7 @@ swl_status switch_layer_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64
  *   workspace       device scratch of workspace_bytes >= switch_layer_workspace_size()
  *   stream          cudaStream_t to enqueue on
  * bf16 additionally requires d % 8 == 0, d_ff % 8 == 0 and 16-byte aligned x,
- * W1, W2 and out (TMA rows). */
+ * W1, W2, out and W_r (TMA rows, vector loads); otherwise SWL_ERR_UNSUPPORTED. */
 swl_status switch_layer_forward(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                 const void* x, const float* W_r, const void* W1, const void* b1,
                                 const void* W2, const void* b2, double capacity_factor,

@@ -245,7 +245,206 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
   }
 }
 
+constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kFusedMaxN = 128;
+constexpr int kFusedRegVec = 8;   // row vectors per lane held in registers (4 KiB rows at 16 B)
+
+// Scan and gather in one launch (N <= 128): CTA b owns router block b (tpb
+// tokens).  Every CTA sums the per-block counts itself - the expert totals and
+// the prefix over the blocks before b - so no CTA waits for another; CTA 0 also
+// writes the expert bases, the GEMM tile prefix, the aux loss and the expert
+// FFN's per-call counters.  Then one warp per token: pos = prefix + in-block
+// rank; a kept token records its packed row and is copied there, a dropped
+// token's output row is zeroed.  Integer sums are exact in any order; the fp64
+// sums of p run in a fixed order (deterministic).
+template <int VEC>
+__global__ void __launch_bounds__(kFusedThreads)
+dispatch_fused_kernel(const uint8_t* __restrict__ x, const int* __restrict__ expert_idx,
+                      int* __restrict__ pos_in_expert, const int* __restrict__ blk_count,
+                      const float* __restrict__ blk_psum, int* __restrict__ exp_rows,
+                      int* __restrict__ exp_base, int* __restrict__ tile_prefix,
+                      int* __restrict__ slot_token, int* __restrict__ ready,
+                      uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out,
+                      float* __restrict__ aux_loss, WsHeader* hdr, int T, int N, int nblk,
+                      int tpb, int C_eff, int tile_rows, int row_bytes, int copy_rows) {
+  using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
+  __shared__ int s_tot[kFusedMaxN], s_pre[kFusedMaxN], s_base[kFusedMaxN];
+  __shared__ double s_ps[kFusedThreads];
+  __shared__ double s_term[kFusedMaxN];
+  __shared__ int s_tiles;
+  pdl_trigger();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x;
+  const int t0 = b * tpb;
+  const int ntok = min(tpb, T - t0);
+  const int nv = row_bytes / VEC;
+  const bool in_regs = copy_rows && nv <= 32 * kFusedRegVec;
+  // this warp's first token row: x is a layer input, readable before the wait
+  V cur[kFusedRegVec];
+  auto load_row = [&](int t, V (&r)[kFusedRegVec]) {
+    const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
+#pragma unroll
+    for (int j = 0; j < kFusedRegVec; ++j)
+      if (lane + 32 * j < nv) r[j] = src[lane + 32 * j];
+  };
+  if (in_regs && warp < ntok) load_row(t0 + warp, cur);
+  pdl_wait();   // block statistics and ranks come from the router
+
+  for (int e = tid; e < N; e += kFusedThreads) {
+    s_tot[e] = 0;
+    s_pre[e] = 0;
+  }
+  __syncthreads();
+  // per expert: total over all blocks and prefix over blocks < b (G threads each)
+  const int G = kFusedThreads / N;
+  const int ee = tid % N, g = tid / N;
+  double ps = 0.0;
+  if (g < G) {
+    int tot = 0, pre = 0;
+    int bb = g;
+    for (; bb + 3 * G < nblk; bb += 4 * G) {
+      int c[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) c[u] = blk_count[(size_t)(bb + u * G) * N + ee];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        tot += c[u];
+        pre += (bb + u * G < b) ? c[u] : 0;
+      }
+    }
+    for (; bb < nblk; bb += G) {
+      const int c = blk_count[(size_t)bb * N + ee];
+      tot += c;
+      pre += (bb < b) ? c : 0;
+    }
+    if (b == 0)
+      for (int b2 = g; b2 < nblk; b2 += G) ps += (double)blk_psum[(size_t)b2 * N + ee];
+    atomicAdd(&s_tot[ee], tot);
+    atomicAdd(&s_pre[ee], pre);
+  }
+  if (b == 0) s_ps[tid] = ps;
+  __syncthreads();
+  // packed row bases (and, in CTA 0, the expert FFN's tile prefix): one warp
+  if (warp == 0) {
+    constexpr int EPL = kFusedMaxN / 32;
+    int rows[EPL], tiles[EPL];
+    int rs = 0, ts = 0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane * EPL + j;
+      rows[j] = e < N ? min(s_tot[e], C_eff) : 0;
+      tiles[j] = (rows[j] + tile_rows - 1) / tile_rows;
+      rs += rows[j];
+      ts += tiles[j];
+    }
+    const int rs_in = warp_incl_scan(rs, lane), ts_in = warp_incl_scan(ts, lane);
+    int run = rs_in - rs, trun = ts_in - ts;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane * EPL + j;
+      if (e < N) {
+        s_base[e] = run;
+        if (b == 0) {
+          exp_rows[e] = rows[j];
+          exp_base[e] = run;
+          tile_prefix[e] = trun;
+        }
+      }
+      run += rows[j];
+      trun += tiles[j];
+    }
+    const int total_tiles = __shfl_sync(0xffffffffu, ts_in, 31);
+    if (lane == 0) {
+      s_tiles = total_tiles;
+      if (b == 0) tile_prefix[N] = total_tiles;
+    }
+  }
+  __syncthreads();
+  if (b == 0) {
+    // per-call state of the expert FFN kernel: token-tile readiness, work counter
+    for (int i = tid; i < s_tiles; i += kFusedThreads) ready[i] = 0;
+    // aux = N * sum_i (count_i / T) * (sum_t p_t,i / T); sums in a fixed order
+    if (tid < N) {
+      double P = 0.0;
+      for (int g2 = 0; g2 < G; ++g2) P += s_ps[g2 * N + tid];
+      s_term[tid] = (double)s_tot[tid] * P;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double a = 0.0;
+      for (int e = 0; e < N; ++e) a += s_term[e];
+      *aux_loss = (float)((double)N * a / ((double)T * (double)T));
+      hdr->next_tile = 0u;
+    }
+  }
+  // one warp per token; the next token's row is requested before this one's
+  // destination is known
+  for (int i = warp; i < ntok; i += kFusedWarps) {
+    const int t = t0 + i;
+    V nxt[kFusedRegVec];
+    const bool more = i + kFusedWarps < ntok;
+    if (in_regs && more) load_row(t + kFusedWarps, nxt);
+    const int e = expert_idx[t];
+    if (e < 0 || e >= N) {        // cannot happen: the router clamps its choice
+      if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
+      return;
+    }
+    const int pos = s_pre[e] + pos_in_expert[t];   // prefix + in-block rank
+    __syncwarp();
+    if (lane == 0) pos_in_expert[t] = pos;
+    if (pos < C_eff) {
+      const int row = s_base[e] + pos;
+      if (lane == 0) slot_token[row] = t;
+      if (copy_rows) {
+        V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
+        if (in_regs) {
+#pragma unroll
+          for (int j = 0; j < kFusedRegVec; ++j)
+            if (lane + 32 * j < nv) dst[lane + 32 * j] = cur[j];
+        } else {
+          const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
+          for (int j = lane; j < nv; j += 32) dst[j] = src[j];
+        }
+      }
+    } else {
+      V* dst = reinterpret_cast<V*>(out + (size_t)t * row_bytes);
+      V z;
+      memset(&z, 0, sizeof(V));
+      for (int j = lane; j < nv; j += 32) dst[j] = z;
+    }
+    if (in_regs && more) {
+#pragma unroll
+      for (int j = 0; j < kFusedRegVec; ++j) cur[j] = nxt[j];
+    }
+  }
+}
+
 }  // namespace
+
+bool dispatch_fused_ok(const Shape& s) {
+  const int64_t elem = s.dtype == 1 ? 2 : 4;
+  return s.N <= kFusedMaxN && s.T * s.d * elem <= (int64_t{16} << 20);
+}
+
+cudaError_t launch_dispatch_fused(const Shape& s, const Workspace& ws, const void* x,
+                                  const int* expert_idx, int* pos_in_expert, void* out,
+                                  float* aux_loss, cudaStream_t stream) {
+  const int elem = s.dtype == 1 ? 2 : 4;
+  const int row_bytes = (int)(s.d * elem);
+  const bool vec16 = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(out) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ws.xbuf) & 15) == 0);
+  const cudaError_t e = launch_dependent(
+      vec16 ? dispatch_fused_kernel<16> : dispatch_fused_kernel<4>, dim3(s.nblk),
+      dim3(kFusedThreads), 0, stream, static_cast<const uint8_t*>(x), expert_idx, pos_in_expert,
+      static_cast<const int*>(ws.blk_count), static_cast<const float*>(ws.blk_psum), ws.exp_rows,
+      ws.exp_base, ws.tile_prefix, ws.slot_token, ws.ready, static_cast<uint8_t*>(ws.xbuf),
+      static_cast<uint8_t*>(out), aux_loss, ws.hdr, (int)s.T, (int)s.N, s.nblk, s.tpb,
+      (int)s.C_eff, s.tile_rows, row_bytes, 1);
+  count_launch();
+  return e;
+}
 
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
                                  cudaStream_t stream) {

@@ -116,6 +116,13 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
                                    const int* expert_idx, int* pos_in_expert, void* out,
                                    cudaStream_t stream);
+// Scan and gather in one launch, for N <= 128 and small batches (one CTA per
+// router block copies its tokens' rows; the two-kernel path spreads large copies
+// over more warps).
+bool dispatch_fused_ok(const Shape& s);
+cudaError_t launch_dispatch_fused(const Shape& s, const Workspace& ws, const void* x,
+                                  const int* expert_idx, int* pos_in_expert, void* out,
+                                  float* aux_loss, cudaStream_t stream);
 // Both expert GEMMs (bf16, tcgen05) in one persistent launch: GEMM1 + bias + ReLU
 // into hbuf, GEMM2 + bias + gate scattered to out.
 cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CUtensorMap& tmA1,

@@ -191,10 +191,18 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
       launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
     return SWL_ERR_CUDA;
   if (!rec(2)) return SWL_ERR_CUDA;
-  if (launch_dispatch_scan(s, ws, aux_loss, stream) != cudaSuccess) return SWL_ERR_CUDA;
-  if (!rec(3)) return SWL_ERR_CUDA;
-  if (launch_dispatch_gather(s, ws, x, expert_idx, pos_in_expert, out, stream) != cudaSuccess)
-    return SWL_ERR_CUDA;
+  if (dispatch_fused_ok(s)) {
+    // one launch for scan and gather (timed in the scan stage; the gather stage is empty)
+    if (launch_dispatch_fused(s, ws, x, expert_idx, pos_in_expert, out, aux_loss, stream) !=
+        cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (!rec(3)) return SWL_ERR_CUDA;
+  } else {
+    if (launch_dispatch_scan(s, ws, aux_loss, stream) != cudaSuccess) return SWL_ERR_CUDA;
+    if (!rec(3)) return SWL_ERR_CUDA;
+    if (launch_dispatch_gather(s, ws, x, expert_idx, pos_in_expert, out, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+  }
   if (!rec(4)) return SWL_ERR_CUDA;
   if (s.dtype == SWL_BF16) {
     const int sms = num_sms_current();
