@@ -295,31 +295,36 @@ dispatch_fused_kernel(const uint8_t* __restrict__ x, const int* __restrict__ exp
     s_tot[e] = 0;
     s_pre[e] = 0;
   }
+  // this warp's tokens (i = warp + 16 j): expert and in-block rank, lane j holds
+  // token j's, all requested now
+  const int my_i = warp + kFusedWarps * lane;
+  const int my_e = my_i < ntok ? expert_idx[t0 + my_i] : 0;
+  const int my_rank = my_i < ntok ? pos_in_expert[t0 + my_i] : 0;
   __syncthreads();
-  // per expert: total over all blocks and prefix over blocks < b (G threads each)
+  // per expert: total over all blocks and prefix over blocks < b (G threads
+  // each); the counts are requested in batches of kBatch before they are summed
   const int G = kFusedThreads / N;
   const int ee = tid % N, g = tid / N;
   double ps = 0.0;
   if (g < G) {
+    constexpr int kBatch = 16;
     int tot = 0, pre = 0;
-    int bb = g;
-    for (; bb + 3 * G < nblk; bb += 4 * G) {
-      int c[4];
+    for (int bb0 = g; bb0 < nblk; bb0 += kBatch * G) {
+      int c[kBatch];
+      float q[kBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) c[u] = blk_count[(size_t)(bb + u * G) * N + ee];
+      for (int u = 0; u < kBatch; ++u) {
+        const int bb = bb0 + u * G;
+        c[u] = bb < nblk ? blk_count[(size_t)bb * N + ee] : 0;
+        q[u] = (b == 0 && bb < nblk) ? blk_psum[(size_t)bb * N + ee] : 0.f;
+      }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kBatch; ++u) {
         tot += c[u];
-        pre += (bb + u * G < b) ? c[u] : 0;
+        pre += (bb0 + u * G < b) ? c[u] : 0;
+        ps += (double)q[u];
       }
     }
-    for (; bb < nblk; bb += G) {
-      const int c = blk_count[(size_t)bb * N + ee];
-      tot += c;
-      pre += (bb < b) ? c : 0;
-    }
-    if (b == 0)
-      for (int b2 = g; b2 < nblk; b2 += G) ps += (double)blk_psum[(size_t)b2 * N + ee];
     atomicAdd(&s_tot[ee], tot);
     atomicAdd(&s_pre[ee], pre);
   }
@@ -380,17 +385,17 @@ dispatch_fused_kernel(const uint8_t* __restrict__ x, const int* __restrict__ exp
   }
   // one warp per token; the next token's row is requested before this one's
   // destination is known
-  for (int i = warp; i < ntok; i += kFusedWarps) {
+  for (int i = warp, j = 0; i < ntok; i += kFusedWarps, ++j) {
     const int t = t0 + i;
     V nxt[kFusedRegVec];
     const bool more = i + kFusedWarps < ntok;
     if (in_regs && more) load_row(t + kFusedWarps, nxt);
-    const int e = expert_idx[t];
+    const int e = __shfl_sync(0xffffffffu, my_e, j);
     if (e < 0 || e >= N) {        // cannot happen: the router clamps its choice
       if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
       return;
     }
-    const int pos = s_pre[e] + pos_in_expert[t];   // prefix + in-block rank
+    const int pos = s_pre[e] + __shfl_sync(0xffffffffu, my_rank, j);   // prefix + in-block rank
     __syncwarp();
     if (lane == 0) pos_in_expert[t] = pos;
     if (pos < C_eff) {

@@ -46,7 +46,6 @@ namespace swl {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBM = 128;          // tokens per tile (UMMA M)
 constexpr int kBK = 64;           // k per stage (one 128-byte swizzle row of bf16)
 constexpr int kUmmaK = 16;
@@ -134,7 +133,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                  const TcArgs a) {
   // tmW: W3 = [hi; mid; lo] as bf16 [3N, d], box [NP rows, 64 k], 128-byte swizzle
   using C = TcCfg<NP>;
-  constexpr int NPL = NP / 32;
   constexpr int PS = C::kPS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -148,8 +146,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* Ps = reinterpret_cast<float*>(smem);   // [kBM][PS] logits, after the main loop
   __shared__ int eid[kBM];
-  __shared__ int lead_count[kBM];
-  __shared__ float s_psum[kWarps * NP];
+  __shared__ int wcnt[(kBM / 32) * NP];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int S = static_cast<int>(cluster.num_blocks());
@@ -232,21 +229,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           volatile int never = 0;
           if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never))
             atomicExch(&a.hdr->err, kDevPipelineTimeout);
-        }
-      }
-      // HBM is idle from here until the expert FFN starts: this CTA's share of the
-      // weights the FFN streams first goes to L2 meanwhile (no completion needed)
-      if (a.pf_bytes > 0) {
-        constexpr size_t kChunk = 64 << 10;
-        const size_t nct = static_cast<size_t>(gridDim.x) * gridDim.y * gridDim.z;
-        const size_t id = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x +
-                          blockIdx.x;
-        const size_t share = ((a.pf_bytes + nct - 1) / nct + 15) & ~static_cast<size_t>(15);
-        const size_t lo = id * share;
-        const size_t hi = lo + share < a.pf_bytes ? lo + share : a.pf_bytes;
-        for (size_t o = lo; o < hi; o += kChunk) {
-          const size_t n = (hi - o < kChunk ? hi - o : kChunk) & ~static_cast<size_t>(15);
-          if (n > 0) ptx::prefetch_l2_bulk(a.pf + o, static_cast<uint32_t>(n));
         }
       }
     }
@@ -378,9 +360,25 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 
   const int t0 = m0 + row0;
   const int ntok = max(0, min(R, a.T - t0));
-  route_rows<NPL, kWarps>(Ps + row0 * PS, PS, R, ntok, t0, a.N, blockIdx.x * S + r,
-                          a.expert_idx, a.gate, a.local_rank, a.blk_count, a.blk_psum, a.hdr, eid,
-                          lead_count, s_psum);
+  route_rows_grouped<NP>(Ps + row0 * PS, PS, R, ntok, t0, a.N, blockIdx.x * S + r, a.expert_idx,
+                         a.gate, a.local_rank, a.blk_count, a.blk_psum, a.hdr, eid, wcnt);
+  // HBM is idle from here until the expert FFN starts (every CTA's loads have
+  // landed by now): this CTA's share of the weights the FFN streams first goes
+  // to L2 meanwhile (no completion needed).  Issued last, so that no warp of
+  // the routing above waits for it.
+  if (threadIdx.x == 0 && a.pf_bytes > 0) {
+    constexpr size_t kChunk = 64 << 10;
+    const size_t nct = static_cast<size_t>(gridDim.x) * gridDim.y * gridDim.z;
+    const size_t id = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x +
+                      blockIdx.x;
+    const size_t share = ((a.pf_bytes + nct - 1) / nct + 15) & ~static_cast<size_t>(15);
+    const size_t lo = id * share;
+    const size_t hi = lo + share < a.pf_bytes ? lo + share : a.pf_bytes;
+    for (size_t o = lo; o < hi; o += kChunk) {
+      const size_t n = (hi - o < kChunk ? hi - o : kChunk) & ~static_cast<size_t>(15);
+      if (n > 0) ptx::prefetch_l2_bulk(a.pf + o, static_cast<uint32_t>(n));
+    }
+  }
 }
 
 template <int NP>

@@ -176,9 +176,15 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
     if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
         !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N, router_tc_padded_experts(s.N)))
       return SWL_ERR_CUDA;
-    // the FFN's first tiles stream W1 from its start: fetch a slice into L2 now
+    // the FFN's first tiles stream W1 from its start: fetch a slice into L2 while
+    // routing and dispatch run, when the router is a single wave of CTAs (with a
+    // second wave the prefetch would compete with that wave's loads)
     const size_t w1_bytes = static_cast<size_t>(s.N) * s.d_ff * s.d * 2;
-    const size_t pf = w1_bytes < kL2PrefetchBytes ? w1_bytes : kL2PrefetchBytes;
+    const int sms = num_sms_current();
+    const int64_t router_ctas = s.router_path == kRouterTC ? (s.T + 127) / 128 * s.ksplit_eff : 0;
+    const size_t pf = (router_ctas > 0 && router_ctas <= sms)
+                          ? (w1_bytes < kL2PrefetchBytes ? w1_bytes : kL2PrefetchBytes)
+                          : 0;
     if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, W1, pf,
                          stream) != cudaSuccess)
       return SWL_ERR_CUDA;
