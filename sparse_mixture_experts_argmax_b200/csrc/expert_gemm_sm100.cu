@@ -76,6 +76,7 @@ struct FfnArgs {
   unsigned int* next_tile;     // work counter (zeroed by the scan)
   int* err;
   int num_experts;
+  int cache_prefix;   // 1: the scheduler keeps the tile prefix in shared memory
   int bn;         // token rows per tile (multiple of 16, <= 256)
   int stages;
   int num_acc;    // TMEM accumulators: 4 of 128 columns when bn <= 128, else 2 of 256
@@ -99,7 +100,9 @@ constexpr int kTileRing = 8;    // decoded tiles handed to the producer, MMA and
 // Work item t: GEMM1 tiles [0, total0) then GEMM2 tiles.  Within a phase, the
 // tiles of expert e occupy [P[e]*m_tiles, P[e+1]*m_tiles) (P = tile prefix) with
 // token blocks fastest, so CTAs working at the same time share weights.
-__device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int total0) {
+// P is the tile prefix, in shared memory when it fits there, else global.
+__device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int total0,
+                                                 const int* P) {
   TileCoord c;
   c.phase = t < total0 ? 0 : 1;
   const int tile = c.phase == 0 ? t : t - total0;
@@ -108,10 +111,10 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int to
   int lo = 0, hi = a.num_experts;     // last e with P[e] <= q  (P[N] > q)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(a.tile_prefix + mid) <= q) lo = mid; else hi = mid;
+    if (P[mid] <= q) lo = mid; else hi = mid;
   }
-  const int p0 = __ldg(a.tile_prefix + lo);
-  const int nts = __ldg(a.tile_prefix + lo + 1) - p0;
+  const int p0 = P[lo];
+  const int nts = P[lo + 1] - p0;
   const int local = tile - p0 * m_tiles;
   c.e = lo;
   c.mt = local / nts;
@@ -156,7 +159,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   uint64_t* tile_empty = tile_full + kTileRing;   // [kTileRing]
   uint64_t* take_bar = tile_empty + kTileRing;    // [1] the producer took a tile
   TileSlot* tile_ring = reinterpret_cast<TileSlot*>(take_bar + 1);   // [kTileRing]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_ring + kTileRing);
+  int* s_prefix = reinterpret_cast<int*>(tile_ring + kTileRing);      // [N+1] if cached
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(s_prefix + (args.cache_prefix ? args.num_experts + 1 : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -208,6 +213,13 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     // Claims the next tile only once the producer has taken the previous one (so
     // a CTA holds at most one claimed tile it has not started), decodes it, waits
     // for its GEMM1 rows when it is a GEMM2 tile, and publishes it in the ring.
+    // CTA c starts with tile c; the counter hands out tiles from gridDim.x on.
+    const int* P = args.tile_prefix;
+    if (args.cache_prefix) {
+      for (int e = lane; e <= args.num_experts; e += 32) s_prefix[e] = args.tile_prefix[e];
+      __syncwarp();
+      P = s_prefix;
+    }
     if (lane == 0) {
       for (int i = 0;; ++i) {
         const int slot = i % kTileRing;
@@ -219,12 +231,13 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           fail();
           break;
         }
-        const unsigned int claimed = atomicAdd(args.next_tile, 1u);
+        const unsigned int claimed =
+            i == 0 ? blockIdx.x : gridDim.x + atomicAdd(args.next_tile, 1u);
         TileSlot ts;
         ts.t = claimed < static_cast<unsigned int>(total) ? static_cast<int>(claimed) : -1;
         ts.phase = ts.e = ts.mt = ts.nt = ts.g = ts.rows = ts.row0 = 0;
         if (ts.t >= 0) {
-          const TileCoord c = decode_tile(ts.t, args, total0);
+          const TileCoord c = decode_tile(ts.t, args, total0, P);
           ts.phase = c.phase;
           ts.e = c.e;
           ts.mt = c.mt;
@@ -463,8 +476,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   }
 }
 
-size_t ffn_smem_bytes(int bn, int stages) {
-  return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
+size_t ffn_smem_bytes(int bn, int stages, int cached_prefix_ints) {
+  return 1024 + static_cast<size_t>(cached_prefix_ints) * sizeof(int) +
+         static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
          kEpiStageBytes + (2 * kMaxStages + 2 * kMaxAcc + 2 + 2 * kTileRing) * sizeof(uint64_t) +
          kTileRing * sizeof(TileSlot) + 2 * sizeof(uint32_t);
 }
@@ -507,9 +521,12 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
     a.ph[p].mode = p;
   }
   int stages = kMaxStages;
-  while (stages > 2 && ffn_smem_bytes(a.bn, stages) > kMaxSmem) --stages;
+  while (stages > 2 && ffn_smem_bytes(a.bn, stages, 0) > kMaxSmem) --stages;
   a.stages = stages;
-  const size_t smem = ffn_smem_bytes(a.bn, stages);
+  // the tile prefix goes to shared memory when it fits beside the stage ring
+  const int prefix_ints = static_cast<int>(s.N) + 1;
+  a.cache_prefix = ffn_smem_bytes(a.bn, stages, prefix_ints) <= kMaxSmem ? 1 : 0;
+  const size_t smem = ffn_smem_bytes(a.bn, stages, a.cache_prefix ? prefix_ints : 0);
   cudaError_t err = cudaFuncSetAttribute(expert_ffn_sm100_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
