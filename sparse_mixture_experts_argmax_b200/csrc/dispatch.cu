@@ -19,7 +19,9 @@
 //                         row bases, GEMM tile prefix) and writes the aux loss.
 // dispatch_gather_kernel: pos = block offset + in-block rank; kept tokens are
 //                         copied into their packed row of the expert buffer with
-//                         16-byte vector moves, dropped tokens' output rows zeroed.
+//                         16-byte vector moves (rows requested early when x is
+//                         small enough to still be in L2), dropped tokens' output
+//                         rows zeroed.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -199,7 +201,7 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
                        int* __restrict__ pos_in_expert, const int* __restrict__ blk_off,
                        const int* __restrict__ exp_base, int* __restrict__ slot_token,
                        uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out, int T, int N,
-                       int C_eff, int row_bytes, int tpb, WsHeader* hdr) {
+                       int C_eff, int row_bytes, int tpb, int prefetch, WsHeader* hdr) {
   using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
   pdl_trigger();
   pdl_wait();   // offsets come from the scan
@@ -209,7 +211,9 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
   const int nv = row_bytes / VEC;
   const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
   V reg[kGatherMaxVecPerLane];
-  const bool in_regs = nv <= 32 * kGatherMaxVecPerLane;
+  // prefetch: the row is requested before its destination is known (x is still
+  // in L2 after the router); otherwise only kept tokens' rows are read
+  const bool in_regs = prefetch && nv <= 32 * kGatherMaxVecPerLane;
   if (in_regs) {
 #pragma unroll
     for (int j = 0; j < kGatherMaxVecPerLane; ++j)
@@ -476,7 +480,8 @@ cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const vo
       dim3(kGatherThreads), 0, stream, static_cast<const uint8_t*>(x), expert_idx, pos_in_expert,
       static_cast<const int*>(ws.blk_off), static_cast<const int*>(ws.exp_base), ws.slot_token,
       static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T, (int)s.N,
-      (int)s.C_eff, row_bytes, s.tpb, ws.hdr);
+      (int)s.C_eff, row_bytes, s.tpb, s.T * (int64_t)row_bytes <= (int64_t{48} << 20) ? 1 : 0,
+      ws.hdr);
   count_launch();
   return e;
 }
