@@ -276,3 +276,30 @@ def test_router_decision_needs_float32_weights(dtype):
     assert np.all(ref["expert_idx"][pos] == 1)
     check_routing(got, ref, oracle.capacity(T, N, cf), T)
     check_close(_np(got["out"]), ref["out"], dtype)
+
+
+# Shapes chosen to reach each kernel variant of the path (see the router plan,
+# the dispatch choice and the expert FFN accumulator count in csrc/):
+#   bf16 N = 80 (96-expert router tiles), K split over a 4-CTA cluster
+#   bf16 N = 128, K split over a 2-CTA cluster
+#   bf16 N = 200: tensor-core logits tiles with a ragged last expert tile + softmax kernel
+#   fp32 N = 150: FFMA logits with K slices + softmax kernel
+#   fp32 N = 48, ~100 big router tiles: FFMA tile router, fused dispatch
+#   fp32 N = 8, x > 16 MiB: warp-split router, two-kernel dispatch (scan + gather)
+#   bf16 N = 4, capacity > 128 rows: two 256-column TMEM accumulators
+_VARIANT_SHAPES = [
+    ("tc_np96_s4", 1000, 1024, 256, 80, 1.25, "bf16"),
+    ("tc_np128_s2", 2000, 256, 128, 128, 1.25, "bf16"),
+    ("tc_wide_ragged", 700, 256, 128, 200, 2.0, "bf16"),
+    ("ffma_wide", 300, 48, 40, 150, 2.0, "f32"),
+    ("ffma_tile", 25700, 32, 32, 48, 1.0, "f32"),
+    ("two_kernel_dispatch", 20000, 256, 32, 8, 1.0, "f32"),
+    ("two_accumulators", 900, 64, 64, 4, 1.0, "bf16"),
+]
+
+
+@pytest.mark.parametrize("shape", _VARIANT_SHAPES, ids=lambda s: s[0])
+def test_kernel_variant_shapes(shape):
+    name, T, d, d_ff, N, cf, dtype = shape
+    spec = synth.LayerSpec("variant_" + name, T, d, d_ff, N, cf, dtype, bias_std=0.05)
+    _full_parity(spec, gap_redraws(spec))
