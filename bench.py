@@ -152,6 +152,11 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     spec = synth.WORKLOADS[args.workload]
     T, d, d_ff, N, cf = spec.T, spec.d, spec.d_ff, spec.N, spec.cf
+    # set before the workspace is sized (the two routers need different scratch)
+    swl.switch_layer_set_router_mode(swl.SWL_ROUTER_FFMA if args.router == "ffma"
+                                     else swl.SWL_ROUTER_TENSOR)
+    router_desc = ("fp32 FFMA" if args.router == "ffma" or spec.dtype != "bf16" else
+                   "fp32 on tensor cores (exact three-piece bf16 split of W_r, fp32 accumulation)")
     redraws = synth.load_gap_redraws(spec.name) if rank == 0 else {}
     inputs = synth.make_layer_inputs(spec, seed=rank, device=dev, redraws=redraws)
     act = inputs["x"].dtype
@@ -320,7 +325,7 @@ def run_gpu(args):
         "config": {
             "workload": spec.name, "T": T, "d": d, "d_ff": d_ff, "N": N,
             "capacity_factor": cf, "capacity": swl.switch_layer_capacity(T, N, cf),
-            "router": "fp32", "parallelism": "dp%d (independent batches)" % ws_n,
+            "router": router_desc, "parallelism": "dp%d (independent batches)" % ws_n,
             "l2": "flushed between timed steps (256 MiB write, outside the step events); "
                   "expert weights %.0f MB > 126 MB L2" % (2 * N * d * d_ff * elem / 1e6),
         },
@@ -441,6 +446,9 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router", default="tensor", choices=["tensor", "ffma"],
+                    help="fp32 router logits of bf16 layers: tensor cores on the exact bf16 "
+                         "split of W_r (default) or FFMA on the CUDA cores")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.shape:

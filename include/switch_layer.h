@@ -190,6 +190,19 @@ const char* switch_layer_stage_name(int k);
 /* Number of kernel launches this library has issued since it was loaded. */
 uint64_t switch_layer_launch_count(void);
 
+/* How the fp32 router logits of bf16 layers are computed (process-wide; fp32
+ * layers always use FFMA).  Both give the float32 dot product up to the rounding
+ * of fp32 accumulation ("The selective precision solution"):
+ *   SWL_ROUTER_TENSOR (default): tcgen05 tensor cores on the exact split of
+ *     W_r into three bf16 pieces (hi + mid + lo), fp32 accumulation in TMEM;
+ *   SWL_ROUTER_FFMA: fp32 FMA on the CUDA cores, no tensor cores.
+ * The choice changes the workspace size: set it before
+ * switch_layer_workspace_size and keep it for the calls that use that
+ * workspace.  Returns SWL_ERR_INVALID_ARG for an unknown mode. */
+typedef enum swl_router_mode { SWL_ROUTER_TENSOR = 0, SWL_ROUTER_FFMA = 1 } swl_router_mode;
+swl_status switch_layer_set_router_mode(int mode);
+int switch_layer_router_mode(void);
+
 #ifdef __cplusplus
 }
 #endif

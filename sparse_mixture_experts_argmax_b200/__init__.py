@@ -32,7 +32,10 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_forward_timed", "switch_layer_forward_host_io",
            "switch_layer_device_status", "switch_layer_status_string",
            "switch_layer_stage_name", "switch_layer_launch_count",
-           "switch_layer_forward_noalloc")
+           "switch_layer_forward_noalloc", "switch_layer_set_router_mode",
+           "switch_layer_router_mode")
+SWL_ROUTER_TENSOR = 0
+SWL_ROUTER_FFMA = 1
 SWL_NOALLOC_MAX_BYTES = 64 << 20
 
 
@@ -82,6 +85,10 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_stage_name.argtypes = [_i32]
     L.switch_layer_launch_count.restype = ctypes.c_uint64
     L.switch_layer_launch_count.argtypes = []
+    L.switch_layer_set_router_mode.restype = ctypes.c_int
+    L.switch_layer_set_router_mode.argtypes = [_i32]
+    L.switch_layer_router_mode.restype = ctypes.c_int
+    L.switch_layer_router_mode.argtypes = []
     L.switch_layer_forward_noalloc.restype = _i32
     L.switch_layer_forward_noalloc.argtypes = _FWD_ARGS[:17] + [_vp, _vp]
     _lib = L
@@ -229,6 +236,15 @@ def switch_layer_stage_name(k: int) -> Optional[str]:
 
 def switch_layer_launch_count() -> int:
     return int(lib().switch_layer_launch_count())
+
+
+def switch_layer_set_router_mode(mode: int) -> None:
+    """SWL_ROUTER_TENSOR (default) or SWL_ROUTER_FFMA for bf16 layers (process-wide)."""
+    _check(lib().switch_layer_set_router_mode(int(mode)), "switch_layer_set_router_mode")
+
+
+def switch_layer_router_mode() -> int:
+    return int(lib().switch_layer_router_mode())
 
 
 # ---------------------------------------------------------------------------

@@ -84,7 +84,8 @@ struct RouterPlan {
   int kslice;   // K per logits slice (wide, tile and tensor-core paths)
   int ksplit;   // logits slices (CTAs of a cluster on the tile / tensor-core paths)
 };
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int dtype);
+// tensor != 0: the tensor-core router (bf16 layers); else the FFMA kernels.
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 

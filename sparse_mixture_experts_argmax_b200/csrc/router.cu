@@ -800,9 +800,9 @@ cudaError_t launch_softmax_t(const Shape& s, const Workspace& ws, const float* b
 
 }  // namespace
 
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int dtype) {
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor) {
   RouterPlan p;
-  if (dtype == 1 && N <= kFusedRouterMaxN) {
+  if (tensor && N <= kFusedRouterMaxN) {
     // tensor cores: 128-token tiles; K split over 2 or 4 CTAs of a cluster while
     // the tiles alone would leave most SMs idle (and each CTA keeps >= 2 k-blocks)
     const int64_t tiles = (T + 127) / 128;
@@ -841,7 +841,7 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int dtype) {
   p.tpb = 32;
   for (int tpb = 128; tpb > 32; tpb /= 2)
     if ((T + tpb - 1) / tpb >= 2 * 148) { p.tpb = tpb; break; }
-  if (dtype == 1) {
+  if (tensor) {
     p.path = kRouterTCWide;
     p.ksplit = 1;
     p.kslice = (int)((d + 63) / 64 * 64);

@@ -27,6 +27,7 @@
 namespace swl {
 
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<int> g_router_mode{SWL_ROUTER_TENSOR};   // switch_layer_set_router_mode
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -141,7 +142,9 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->dtype = dtype;
   s->C = switch_layer_capacity(T, N, cf);
   s->C_eff = s->C < T ? s->C : T;
-  const RouterPlan rp = router_plan(T, d, N, dtype);
+  // the tensor-core router serves bf16 layers unless the FFMA router was chosen
+  const bool tensor_router = dtype == SWL_BF16 && g_router_mode.load() == SWL_ROUTER_TENSOR;
+  const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0);
   s->router_path = rp.path;
   s->kslice = rp.kslice;
   s->ksplit_eff = rp.ksplit;
@@ -439,6 +442,14 @@ const char* switch_layer_stage_name(int k) {
 }
 
 uint64_t switch_layer_launch_count(void) { return g_launches.load(); }
+
+swl_status switch_layer_set_router_mode(int mode) {
+  if (mode != SWL_ROUTER_TENSOR && mode != SWL_ROUTER_FFMA) return SWL_ERR_INVALID_ARG;
+  swl::g_router_mode.store(mode);
+  return SWL_OK;
+}
+
+int switch_layer_router_mode(void) { return swl::g_router_mode.load(); }
 
 swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                         const void* x, const float* W_r, const void* W1,

@@ -97,3 +97,23 @@ def test_forward_rejects_bad_arguments_without_launching(L):
     assert L.switch_layer_forward_timed(16, 8, 8, 2, 0, *([0x1000] * 6), 1.0, *([0x1000] * 5),
                                         None, 0x10000, 1 << 30, None, None) == 1
     assert swl.switch_layer_status_string(3) == "workspace too small"
+
+
+def test_router_mode_switch(L):
+    assert swl.switch_layer_router_mode() == swl.SWL_ROUTER_TENSOR
+    n_tensor = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25)
+    swl.switch_layer_set_router_mode(swl.SWL_ROUTER_FFMA)
+    try:
+        assert swl.switch_layer_router_mode() == swl.SWL_ROUTER_FFMA
+        n_ffma = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25)
+        # the tensor-core router keeps the three bf16 pieces of W_r in the workspace
+        assert n_tensor - n_ffma >= 3 * 64 * 768 * 2
+        # fp32 layers use the FFMA router in both modes
+        assert (swl.switch_layer_workspace_size(64, 32, 64, 4, swl.SWL_F32, 1.0) ==
+                swl.switch_layer_workspace_size(64, 32, 64, 4, swl.SWL_F32, 1.0))
+    finally:
+        swl.switch_layer_set_router_mode(swl.SWL_ROUTER_TENSOR)
+    with pytest.raises(swl.SwitchLayerError) as ei:
+        swl.switch_layer_set_router_mode(7)
+    assert ei.value.status == 1
+    assert swl.switch_layer_router_mode() == swl.SWL_ROUTER_TENSOR

@@ -303,3 +303,25 @@ def test_kernel_variant_shapes(shape):
     name, T, d, d_ff, N, cf, dtype = shape
     spec = synth.LayerSpec("variant_" + name, T, d, d_ff, N, cf, dtype, bias_std=0.05)
     _full_parity(spec, gap_redraws(spec))
+
+
+# ------------------------------------------------------------------ FFMA router for bf16 layers
+@pytest.fixture
+def ffma_router():
+    swl.switch_layer_set_router_mode(swl.SWL_ROUTER_FFMA)
+    yield
+    swl.switch_layer_set_router_mode(swl.SWL_ROUTER_TENSOR)
+
+
+def test_base_workload_ffma_router(ffma_router):
+    spec = synth.WORKLOADS["base_T4096_d768_N64"]
+    _full_parity(spec, synth.load_gap_redraws(spec.name))
+
+
+@pytest.mark.parametrize("spec", _random_specs()[:5], ids=lambda s: s.name)
+def test_random_shapes_ffma_router(spec, ffma_router):
+    _full_parity(spec, gap_redraws(spec))
+
+
+def test_router_decision_needs_float32_weights_ffma(ffma_router):
+    test_router_decision_needs_float32_weights("bf16")
