@@ -308,6 +308,14 @@ def run_gpu(args):
     traffic = _traffic_entry(dom, spec.name)
     gemm_flops = 4.0 * K_kept * d * d_ff
     tensor_frac = gemm_flops / dom_s / (peaks["bf16_tflops"] * 1e12)
+    # whole layer: the slower of its GEMM FLOPs at the bf16 peak and its bytes at
+    # the HBM peak, against the measured step time.  Bytes: router (x, W_r, bias),
+    # dispatch (x rows of kept tokens in and out of the packed buffer, zero rows of
+    # dropped tokens, per-token outputs), the expert FFN's bytes above, and out.
+    layer_bytes = (T * d * elem + N * d * 4 + N * 4 + 2 * K_kept * d * elem +
+                   (T - K_kept) * d * elem + 3 * 4 * T + ffn_bytes)
+    layer_floor_s = max(layer_bytes / (peaks["hbm_gbs"] * 1e9),
+                        (gemm_flops + 2.0 * T * d * N) / (peaks["bf16_tflops"] * 1e12))
 
     res = {
         "metric": METRIC,
@@ -337,6 +345,13 @@ def run_gpu(args):
             "kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
             "algorithmic_bytes": ffn_bytes, "peak_source": peaks["source"] + " (burst copy)",
+        },
+        "layer_roofline": {
+            "bytes": layer_bytes, "flops": gemm_flops + 2.0 * T * d * N,
+            "floor_us": layer_floor_s * 1e6, "step_us": ms_per_step * 1e3,
+            "frac": layer_floor_s / (ms_per_step / 1e3),
+            "note": "the slower of the layer's FLOPs at the measured bf16 peak and its bytes at "
+                    "the measured HBM copy bandwidth, over the measured step time",
         },
         "expert_gemm_tensor_frac": {
             "value": tensor_frac, "flops_per_step": gemm_flops,

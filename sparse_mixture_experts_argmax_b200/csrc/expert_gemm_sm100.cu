@@ -388,7 +388,12 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       const int slot = i % kTileRing;
       const uint32_t tpar = (i / kTileRing) & 1;
       publish_if_blocked(&tile_full[slot], tpar);
-      if (!ptx::mbar_wait(&tile_full[slot], tpar, abort_flag)) { fail(); break; }
+      // every wait result is made warp-uniform: the warp then leaves together (the
+      // TMEM loads below are warp-collective)
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tile_full[slot], tpar, abort_flag))) {
+        fail();
+        break;
+      }
       const TileSlot ts = tile_ring[slot];
       if (ts.t < 0) break;
       const PhaseArgs& P = args.ph[ts.phase];
@@ -418,7 +423,10 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         gs[k] = (P.mode == 1 && col < rows) ? __ldg(args.gate + dsts[k]) : 1.f;
       }
       publish_if_blocked(&tfull_bar[acc], aph);
-      if (!ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag)) { fail(); break; }
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag))) {
+        fail();
+        break;
+      }
       ptx::tc_fence_after();
       const uint32_t t_base =
           tmem_base + static_cast<uint32_t>(acc * acc_cols) + (static_cast<uint32_t>(q * 32) << 16);
