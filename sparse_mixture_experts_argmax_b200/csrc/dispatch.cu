@@ -22,6 +22,7 @@
 //                         16-byte vector moves (rows requested early when x is
 //                         small enough to still be in L2), dropped tokens' output
 //                         rows zeroed.
+// dispatch_fused_kernel:  both in one launch for N <= 128 and small batches.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

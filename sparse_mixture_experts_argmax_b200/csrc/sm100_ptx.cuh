@@ -105,15 +105,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* t
       : "memory");
 }
 
-// Bring a 2-D tile into L2 ahead of its load (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* tmap, int32_t c0,
-                                                   int32_t c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // Bring [addr, addr + bytes) into L2 (no completion; bytes a multiple of 16,
 // addr 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* addr, uint32_t bytes) {

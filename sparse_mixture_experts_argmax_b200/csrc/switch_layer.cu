@@ -2,11 +2,13 @@
 // capacity, workspace layout, TMA descriptors and the launch sequence.
 //
 // Stage order on the caller's stream (no host synchronisation inside):
-//   0 router               fp32 logits + softmax/argmax/gate + block ranks; bf16
-//                          layers with N <= 128: one tcgen05 kernel (router_tc.cu),
-//                          fp32 layers: FFMA kernels (router.cu)
+//   0 router               fp32 logits + softmax/argmax/gate + block ranks.  bf16
+//                          layers: the split of W_r into bf16 pieces, then the
+//                          tcgen05 router (router_tc.cu; logits only for N > 128);
+//                          fp32 layers or SWL_ROUTER_FFMA: FFMA kernels (router.cu)
 //   1 router softmax       N > 128 only: max/argmax/gate, ranks (router.cu)
-//   2 dispatch scan        offsets, capacity, aux     (dispatch.cu)
+//   2 dispatch scan        offsets, capacity, aux     (dispatch.cu); for N <= 128
+//                          and small batches scan and gather are one kernel here
 //   3 dispatch gather      pos, packed expert rows    (dispatch.cu)
 //   4 expert FFN           GEMM1 + bias + ReLU, GEMM2 + bias + gate + combine
 //                          (one tcgen05 launch: expert_gemm_sm100.cu; fp32: two
