@@ -114,55 +114,76 @@ __device__ __forceinline__ void route_rows(const float* Z, int zs, int R, int nt
   }
 }
 
-// Routing of R <= 128 token rows (R a multiple of 32, NT = 256 threads) from fp32
-// logits Z[R][zs] (bias added; columns N .. NP-1 hold -inf), with TPT = 256 / R
-// threads per token, each holding NP / TPT logits: max/argmax (lowest index on
-// ties), exp-sum and gate reduced over the token's thread group with shuffles;
-// p overwrites Z in place.  In-block ranks: match_any over each warp's 32
-// tokens, plus the counts of the earlier warps.  Per-expert counts and sums of
-// p (rows in token order: deterministic).  Rows at or beyond ntok are skipped;
-// a block that starts beyond the batch writes nothing.  Shared scratch: eid[R],
-// wcnt[R/32][NP].  Every thread of the CTA (256) calls this.
-template <int NP>
-__device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int R, int ntok, int t0,
-                                                   int N, int b, int* __restrict__ expert_idx,
+// Routing of R token rows (R = 128, 64 or 32; 256 threads) from fp32 logits
+// Z[R][zs] (bias added; columns N .. NP-1 hold -inf), TPT = 256 / R threads per
+// token.  Thread `sub` of a token's group holds the columns sub, sub + TPT, ...
+// in registers: max/argmax (lowest index on ties) and exp-sum in four
+// interleaved partial chains, then reduced over the group with shuffles; gate =
+// 1 / sum; p overwrites Z in place.  With zs = NP + TPT (mod 32)
+// the group's lanes read 32 distinct banks.  In-block ranks: match_any over
+// each warp's 32 tokens, plus the counts of the earlier warps.  Per-expert
+// counts, and per-expert sums of p over the rows in a fixed order (contiguous
+// row ranges summed in parallel, then the ranges in order: deterministic).
+// Rows at or beyond ntok are skipped; a block that starts beyond the batch
+// writes nothing.  Shared scratch: eid[R], wcnt[R/32][NP], red[256].  Every
+// thread of the CTA (256) calls this.
+template <int NP, int R>
+__device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int ntok, int t0, int N,
+                                                   int b, int* __restrict__ expert_idx,
                                                    float* __restrict__ gate,
                                                    int* __restrict__ local_rank,
                                                    int* __restrict__ blk_count,
                                                    float* __restrict__ blk_psum, WsHeader* hdr,
-                                                   int* eid, int* wcnt) {
+                                                   int* eid, int* wcnt, float* red) {
+  static_assert(R == 128 || R == 64 || R == 32, "tile rows");
+  constexpr int TPT = 256 / R;             // threads per token: 2, 4 or 8
+  constexpr int EPT = NP / TPT;            // logits per thread
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tpt = 256 / R;                 // threads per token: 8, 4 or 2
-  const int ept = NP / tpt;                // logits per thread
-  const int i = tid / tpt, sub = tid % tpt;
+  const int i = tid / TPT, sub = tid % TPT;
   const bool valid = i < ntok;
   for (int k = tid; k < (R / 32) * NP; k += 256) wcnt[k] = 0;
-  float* zr = Z + i * zs + sub * ept;
-  float best = -INFINITY;
-  int bidx = 0x7fffffff;
+  float* zr = Z + i * zs + sub;
+  static_assert(EPT % 4 == 0, "four interleaved partial maxima and sums");
+  float v[EPT];
+  // four independent max/argmax chains (column j goes to chain j % 4; each
+  // keeps its lowest index among equal maxima), then merged the same way
+  float bq[4];
+  int iq[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) { bq[q] = -INFINITY; iq[q] = 0x7fffffff; }
   if (valid) {
-    for (int j = 0; j < ept; ++j) {
-      const float v = zr[j];
-      if (v > best) { best = v; bidx = sub * ept + j; }
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      v[j] = zr[j * TPT];
+      if (v[j] > bq[j & 3]) { bq[j & 3] = v[j]; iq[j & 3] = sub + j * TPT; }
     }
   }
-  for (int off = 1; off < tpt; off <<= 1) {   // the group's lanes are consecutive
+  float best = bq[0];
+  int bidx = iq[0];
+#pragma unroll
+  for (int q = 1; q < 4; ++q)
+    if (bq[q] > best || (bq[q] == best && iq[q] < bidx)) { best = bq[q]; bidx = iq[q]; }
+#pragma unroll
+  for (int off = 1; off < TPT; off <<= 1) {   // the group's lanes are consecutive
     const float ov = __shfl_xor_sync(0xffffffffu, best, off);
     const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
     if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
   }
-  float ssum = 0.f;
+  float sq[4] = {0.f, 0.f, 0.f, 0.f};
   if (valid) {
-    for (int j = 0; j < ept; ++j) {
-      const float e = (sub * ept + j < N) ? expf(zr[j] - best) : 0.f;
-      zr[j] = e;
-      ssum += e;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      v[j] = (sub + j * TPT < N) ? expf(v[j] - best) : 0.f;
+      sq[j & 3] += v[j];
     }
   }
-  for (int off = 1; off < tpt; off <<= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+  float ssum = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+#pragma unroll
+  for (int off = 1; off < TPT; off <<= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
   const float inv = 1.0f / ssum;
   if (valid) {
-    for (int j = 0; j < ept; ++j) zr[j] *= inv;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) zr[j * TPT] = v[j] * inv;
     if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
       bidx = 0;
       if (sub == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
@@ -184,6 +205,18 @@ __device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int R, int 
     mask = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && (mask & lanes_below) == 0u) wcnt[warp * NP + e] = __popc(mask);
   }
+  // partial sums of p: thread (g, n) adds rows [g*RPG, g*RPG + RPG) of column n
+  constexpr int G = 256 / NP;
+  constexpr int RPG = (R + G - 1) / G;
+  {
+    const int g = tid / NP, n = tid % NP;
+    if (g < G) {
+      float acc = 0.f;
+      const int r1 = min(ntok, (g + 1) * RPG);
+      for (int rr = g * RPG; rr < r1; ++rr) acc += Z[rr * zs + n];
+      red[g * NP + n] = acc;
+    }
+  }
   __syncthreads();
   if (warp < R / 32 && e >= 0) {
     int rank = __popc(mask & lanes_below);
@@ -194,10 +227,12 @@ __device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int R, int 
   float* ps_row = blk_psum + (size_t)b * N;
   for (int n = tid; n < N; n += 256) {
     int c = 0;
+#pragma unroll
     for (int w = 0; w < R / 32; ++w) c += wcnt[w * NP + n];
     cnt_row[n] = c;
     float a = 0.f;
-    for (int r = 0; r < ntok; ++r) a += Z[r * zs + n];
+#pragma unroll
+    for (int g = 0; g < G; ++g) a += red[g * NP + n];
     ps_row[n] = a;
   }
 }

@@ -22,14 +22,16 @@
 // a tile of 128 tokens; CTA r takes k-blocks [r*kb_per, (r+1)*kb_per).
 //   warp 0       TMA producer: x tile [128 tokens x 64 k] and the three piece
 //                tiles [NP experts x 64 k] (bf16, 128-byte swizzle) per stage
-//   warp 1       MMA issuer: per 16-wide k step, three tcgen05.mma (M = 128
-//                tokens, N = NP experts), one per piece, into three TMEM
-//                accumulators
+//   warp 1       MMA issuer: the three piece tiles lie contiguous in shared
+//                memory, one B operand of 3*NP rows; per 16-wide k step one
+//                tcgen05.mma (M = 128 tokens, N = 3*NP; two MMAs when 3*NP >
+//                256) into the three TMEM accumulators [hi | mid | lo]
 //   warp 2       TMEM allocator
 //   warps 4..7   TMEM epilogue (thread = token row): z = D_hi + (D_mid + D_lo)
-// Partial logits of the cluster are added in rank order through distributed
-// shared memory (deterministic), the bias is added, and each CTA routes its
-// 128/S rows (softmax, argmax, block ranks, per-expert counts and sums of p).
+// For S > 1 the partial logits of the cluster are added in rank order through
+// distributed shared memory (deterministic); the bias is added, and each CTA
+// routes its 128/S rows (softmax, argmax, block ranks, per-expert counts and
+// sums of p).
 // Every mbarrier wait is bounded; a stuck pipeline sets the device error word.
 #include <cooperative_groups.h>
 #include <cuda.h>
@@ -58,7 +60,6 @@ struct TcCfg {
   static constexpr uint32_t kABytes = kBM * kBK * 2;             // x tile, bf16
   static constexpr uint32_t kPieceBytes = NP * kBK * 2;          // one piece tile, bf16
   static constexpr uint32_t kStage = kABytes + kPieces * kPieceBytes;
-  static constexpr int kPS = NP + 4;                             // row stride of the logits tile
   static constexpr uint32_t kTmemCols = 3 * NP <= 128 ? 128 : (3 * NP <= 256 ? 256 : 512);
 };
 
@@ -133,7 +134,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                  const TcArgs a) {
   // tmW: W3 = [hi; mid; lo] as bf16 [3N, d], box [NP rows, 64 k], 128-byte swizzle
   using C = TcCfg<NP>;
-  constexpr int PS = C::kPS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -147,10 +147,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   float* Ps = reinterpret_cast<float*>(smem);   // [kBM][PS] logits, after the main loop
   __shared__ int eid[kBM];
   __shared__ int wcnt[(kBM / 32) * NP];
+  __shared__ float red[256];
+  __shared__ float bias_s[NP];   // b_r, 0 without a bias, -inf in the padded columns
 
   cg::cluster_group cluster = cg::this_cluster();
   const int S = static_cast<int>(cluster.num_blocks());
   const int r = static_cast<int>(cluster.block_rank());
+  // row stride of the logits tile: NP + 2S (= NP + threads per token in the
+  // routing below, so that a warp's reads fall in distinct banks); NP + 4 for
+  // the logits-only layout
+  const int PS = kWide ? NP + 4 : NP + 2 * S;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   if (blockIdx.x == 0 && blockIdx.y == 0 && r == 0 && threadIdx.x == 0) {
@@ -236,7 +242,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = ptx::umma_idesc_bf16_f32(NP);
+      // the three piece tiles are contiguous in shared memory: one operand of
+      // 3*NP rows, issued as MMAs of at most 256 rows (N <= 256)
+      constexpr int kRows = kPieces * NP;
+      constexpr int kChunks = (kRows + 255) / 256;
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
@@ -253,11 +262,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         for (int k = 0; k < kBK / kUmmaK; ++k) {
           const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + k * kUmmaK * 2);
 #pragma unroll
-          for (int p = 0; p < kPieces; ++p) {
-            const uint64_t bd =
-                ptx::umma_desc_sw128_kmajor(b_addr + p * C::kPieceBytes + k * kUmmaK * 2);
-            ptx::umma_bf16(tmem_base + static_cast<uint32_t>(p * NP), ad, bd, idesc,
-                           (i | k) != 0 ? 1u : 0u);
+          for (int c = 0; c < kChunks; ++c) {
+            constexpr uint32_t kRowBytes = kBK * 2;
+            const uint32_t n = kRows - c * 256 < 256 ? kRows - c * 256 : 256;
+            const uint64_t bd = ptx::umma_desc_sw128_kmajor(b_addr + c * 256 * kRowBytes +
+                                                            k * kUmmaK * 2);
+            ptx::umma_bf16(tmem_base + static_cast<uint32_t>(c * 256), ad, bd,
+                           ptx::umma_idesc_bf16_f32(n), (i | k) != 0 ? 1u : 0u);
           }
         }
         ptx::umma_commit(&empty_bar[s]);    // frees the stage once these MMAs are done
@@ -269,6 +280,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       if (!ptx::mbar_wait(drain_bar, 0u, &never)) atomicExch(&a.hdr->err, kDevPipelineTimeout);
     }
     __syncwarp();
+  } else if (warp == 3) {
+    // bias row for the read-out below (named barrier 1: this warp + warps 4..7)
+    if constexpr (!kWide) {
+      for (int n = lane; n < NP; n += 32)
+        bias_s[n] = n < a.N ? (a.b_r ? a.b_r[n] : 0.f) : -INFINITY;
+      ptx::named_bar_arrive(1, 160);
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ TMEM epilogue
     bool have = false;
@@ -277,6 +295,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       have = __all_sync(0xffffffffu, got);
       if (!have && lane == 0) fail();
     }
+    if constexpr (!kWide) ptx::named_bar_sync(1, 160);
+    // a lone CTA (S = 1) holds the whole sum: the bias goes in here
+    const bool add_bias = !kWide && S == 1;
     ptx::tc_fence_after();
     const int q = warp & 3;
     const int row = q * 32 + lane;                 // TMEM lane = token row of the tile
@@ -298,10 +319,20 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 32; ++j) z[j] = 0.f;
       }
-      float* pr = Ps + row * PS + c0;
+      if (add_bias) {
 #pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(pr + j) = make_float4(z[j], z[j + 1], z[j + 2], z[j + 3]);
+        for (int j = 0; j < 32; ++j) z[j] = c0 + j < a.N ? z[j] + bias_s[c0 + j] : -INFINITY;
+      }
+      float* pr = Ps + row * PS + c0;
+      if ((PS & 3) == 0) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(pr + j) = make_float4(z[j], z[j + 1], z[j + 2], z[j + 3]);
+      } else {   // PS = NP + 2: rows 8-byte aligned
+#pragma unroll
+        for (int j = 0; j < 32; j += 2)
+          *reinterpret_cast<float2*>(pr + j) = make_float2(z[j], z[j + 1]);
+      }
     }
   }
 
@@ -331,37 +362,48 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     }
     return;
   }
-  cluster.sync();   // every partial logits tile of the cluster is complete
-
-  // this CTA's rows [r*R, r*R + R): partials added in rank order, plus the bias;
-  // written in place (the peers read only their own rows of this tile)
+  // this CTA's rows [r*R, r*R + R), with the bias added and -inf in the padded
+  // columns (S > 1: written in place, the peers read only their own rows of
+  // this tile; S = 1: added by the read-out above)
   const int R = kBM / S;
   const int row0 = r * R;
-  const float* part[4];
+  if (S > 1) {
+    cluster.sync();   // every partial logits tile of the cluster is complete
+    // partials added in rank order (PS = NP + 2S is a multiple of 4 here)
+    const float* part[4];
 #pragma unroll
-  for (int s2 = 0; s2 < 4; ++s2) part[s2] = cluster.map_shared_rank(Ps, s2 < S ? s2 : 0);
-  for (int idx = threadIdx.x; idx < R * (NP / 4); idx += kThreads) {
-    const int i = idx / (NP / 4), n = (idx % (NP / 4)) * 4;
-    const int off = (row0 + i) * PS + n;
-    float4 v = *reinterpret_cast<const float4*>(part[0] + off);
+    for (int s2 = 0; s2 < 4; ++s2) part[s2] = cluster.map_shared_rank(Ps, s2 < S ? s2 : 0);
+    for (int idx = threadIdx.x; idx < R * (NP / 4); idx += kThreads) {
+      const int i = idx / (NP / 4), n = (idx % (NP / 4)) * 4;
+      const int off = (row0 + i) * PS + n;
+      float4 v = *reinterpret_cast<const float4*>(part[0] + off);
 #pragma unroll
-    for (int s2 = 1; s2 < 4; ++s2) {
-      if (s2 < S) {
-        const float4 u = *reinterpret_cast<const float4*>(part[s2] + off);
-        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+      for (int s2 = 1; s2 < 4; ++s2) {
+        if (s2 < S) {
+          const float4 u = *reinterpret_cast<const float4*>(part[s2] + off);
+          v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
       }
-    }
-    const float vv[4] = {v.x, v.y, v.z, v.w};
+      const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      Ps[off + c] = (n + c < a.N) ? vv[c] + (a.b_r ? a.b_r[n + c] : 0.f) : -INFINITY;
+      for (int c = 0; c < 4; ++c)
+        Ps[off + c] = (n + c < a.N) ? vv[c] + bias_s[n + c] : -INFINITY;
+    }
+    cluster.sync();   // the peers have finished reading this CTA's partial tile
   }
-  cluster.sync();   // the peers have finished reading this CTA's partial tile
 
   const int t0 = m0 + row0;
   const int ntok = max(0, min(R, a.T - t0));
-  route_rows_grouped<NP>(Ps + row0 * PS, PS, R, ntok, t0, a.N, blockIdx.x * S + r, a.expert_idx,
-                         a.gate, a.local_rank, a.blk_count, a.blk_psum, a.hdr, eid, wcnt);
+  const int blk = blockIdx.x * S + r;
+  if (S == 1)
+    route_rows_grouped<NP, 128>(Ps, PS, ntok, t0, a.N, blk, a.expert_idx, a.gate, a.local_rank,
+                                a.blk_count, a.blk_psum, a.hdr, eid, wcnt, red);
+  else if (S == 2)
+    route_rows_grouped<NP, 64>(Ps + row0 * PS, PS, ntok, t0, a.N, blk, a.expert_idx, a.gate,
+                               a.local_rank, a.blk_count, a.blk_psum, a.hdr, eid, wcnt, red);
+  else
+    route_rows_grouped<NP, 32>(Ps + row0 * PS, PS, ntok, t0, a.N, blk, a.expert_idx, a.gate,
+                               a.local_rank, a.blk_count, a.blk_psum, a.hdr, eid, wcnt, red);
   // HBM is idle from here until the expert FFN starts (every CTA's loads have
   // landed by now): this CTA's share of the weights the FFN streams first goes
   // to L2 meanwhile (no completion needed).  Issued last, so that no warp of
