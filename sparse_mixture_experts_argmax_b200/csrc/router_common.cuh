@@ -169,11 +169,13 @@ __device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int ntok, i
     const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
     if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
   }
+  // the padded columns hold -inf: exp gives exactly 0 there, with no branch
+  // per column (a finite maximum exists unless the row is flagged below)
   float sq[4] = {0.f, 0.f, 0.f, 0.f};
   if (valid) {
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
-      v[j] = (sub + j * TPT < N) ? expf(v[j] - best) : 0.f;
+      v[j] = expf(v[j] - best);
       sq[j & 3] += v[j];
     }
   }
@@ -212,8 +214,13 @@ __device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int ntok, i
     const int g = tid / NP, n = tid % NP;
     if (g < G) {
       float acc = 0.f;
-      const int r1 = min(ntok, (g + 1) * RPG);
-      for (int rr = g * RPG; rr < r1; ++rr) acc += Z[rr * zs + n];
+      const int r0 = g * RPG, r1 = min(ntok, r0 + RPG);
+      if (r1 - r0 == RPG) {     // full range: loads issued ahead of the adds
+#pragma unroll
+        for (int rr = 0; rr < RPG; ++rr) acc += Z[(r0 + rr) * zs + n];
+      } else {
+        for (int rr = r0; rr < r1; ++rr) acc += Z[rr * zs + n];
+      }
       red[g * NP + n] = acc;
     }
   }
