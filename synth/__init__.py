@@ -68,7 +68,7 @@ class LayerSpec:
     cf: float         # capacity factor
     dtype: str        # "f32" or "bf16": dtype of x, W1, b1, W2, b2, out
     bias_std: float = 0.0       # std of b1 / b2 (0 -> zero biases)
-    router_bias: Optional[str] = None  # None or "zipf1.5": b_r[i] = 1.5*ln(1/(i+1))
+    router_bias: Optional[str] = None  # None or "zipf<a>": b_r[i] = a*ln(1/(i+1))
 
     def to_json(self) -> dict:
         return asdict(self)
@@ -200,11 +200,13 @@ def _sigmas(spec: LayerSpec) -> dict:
 
 
 def router_bias_values(spec: LayerSpec) -> Optional[torch.Tensor]:
-    """Router-logit bias b_r[i] = 1.5 * ln(1/(i+1)) (skewed workload), fp32."""
+    """Router-logit bias b_r[i] = a * ln(1/(i+1)) for router_bias "zipf<a>" (the
+    skewed workload uses a = 1.5), fp32."""
     if spec.router_bias is None:
         return None
-    if spec.router_bias == "zipf1.5":
-        v = np.array([1.5 * math.log(1.0 / (i + 1)) for i in range(spec.N)], dtype=np.float64)
+    if spec.router_bias.startswith("zipf"):
+        a = float(spec.router_bias[4:])
+        v = np.array([a * math.log(1.0 / (i + 1)) for i in range(spec.N)], dtype=np.float64)
         return torch.from_numpy(v.astype(np.float32))
     raise ValueError(spec.router_bias)
 
