@@ -27,11 +27,13 @@
 //                tcgen05.mma (M = 128 tokens, N = 3*NP; two MMAs when 3*NP >
 //                256) into the three TMEM accumulators [hi | mid | lo]
 //   warp 2       TMEM allocator
-//   warps 4..7   TMEM epilogue (thread = token row): z = D_hi + (D_mid + D_lo)
+//   warp 3       stages the bias row in shared memory (-inf in padded columns)
+//   warps 4..7   TMEM epilogue (thread = token row): z = D_hi + (D_mid + D_lo),
+//                plus the bias when the tile has one CTA (S = 1)
 // For S > 1 the partial logits of the cluster are added in rank order through
-// distributed shared memory (deterministic); the bias is added, and each CTA
-// routes its 128/S rows (softmax, argmax, block ranks, per-expert counts and
-// sums of p).
+// distributed shared memory (deterministic), plus the bias.  Each CTA then
+// routes its 128/S rows with all 256 threads (softmax, argmax, block ranks,
+// per-expert counts and sums of p).
 // Every mbarrier wait is bounded; a stuck pipeline sets the device error word.
 #include <cooperative_groups.h>
 #include <cuda.h>
