@@ -22,7 +22,7 @@ stored fp32 / bf16 values.  Matrices act on column vectors as [ST-note] writes
 them: z_t = W_r x_t, W_1 in R^{d_ff x d}, W_2 in R^{d x d_ff}; stored row-major
 as W_r [N, d], W1 [N, d_ff, d], W2 [N, d, d_ff].
 
-Readings where the pages are silent or disagree (each also listed in the design doc):
+Readings where the pages are silent or disagree:
 
 * capacity: C = ceil(capacity_factor * T / N) with the exact rational value of
   the given double ([ST-note] "Capacity Factor"; [ST-paper] prints a floor
