@@ -105,7 +105,7 @@ int router_tc_padded_experts(int64_t N);
 cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
                              const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
                              int* expert_idx, float* gate, int* local_rank,
-                             const void* l2_prefetch, size_t l2_prefetch_bytes,
+                             const void* l2_prefetch, size_t l2_prefetch_bytes, int num_sms,
                              cudaStream_t stream);
 // Expert weights fetched into L2 during the router and dispatch stages.
 constexpr size_t kL2PrefetchBytes = 64u << 20;

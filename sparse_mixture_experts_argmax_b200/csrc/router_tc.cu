@@ -434,7 +434,8 @@ size_t tc_smem_bytes(int stages) {
 template <int NP, bool kWide>
 cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
                         const CUtensorMap& tmW, const float* b_r, int* expert_idx, float* gate,
-                        int* local_rank, const void* pf, size_t pf_bytes, cudaStream_t stream) {
+                        int* local_rank, const void* pf, size_t pf_bytes, int num_sms,
+                        cudaStream_t stream) {
   TcArgs a;
   a.pf = static_cast<const uint8_t*>(pf);
   a.pf_bytes = pf_bytes;
@@ -451,14 +452,23 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
   a.blk_count = ws.blk_count;
   a.blk_psum = ws.blk_psum;
   a.hdr = ws.hdr;
+  const unsigned t_tiles = static_cast<unsigned>((s.T + kBM - 1) / kBM);
   int stages = kMaxStages;
   while (stages > 2 && tc_smem_bytes<NP>(stages) > kMaxDynSmem) --stages;
+  // more one-CTA tiles than SMs: two stages each, so that two CTAs share an SM
+  // (their shared memory, registers and 2 x 256 TMEM columns fit) and all tiles
+  // are resident at once; each CTA's prologue and routing tail then overlap the
+  // other CTA's loads instead of forming a second wave
+  if (!kWide && s.ksplit_eff == 1 && 3 * NP <= 256 && t_tiles > static_cast<unsigned>(num_sms))
+    stages = 2;
+  // the logits tile reuses the stage memory
+  const size_t ps_bytes = static_cast<size_t>(kBM) * (NP + (kWide ? 4 : 2 * s.ksplit_eff)) * 4;
+  if (ps_bytes > static_cast<size_t>(stages) * TcCfg<NP>::kStage) return cudaErrorInvalidValue;
   a.stages = stages;
   const size_t smem = tc_smem_bytes<NP>(stages);
   cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NP, kWide>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const unsigned t_tiles = static_cast<unsigned>((s.T + kBM - 1) / kBM);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = kWide ? dim3(static_cast<unsigned>((s.N + NP - 1) / NP), t_tiles, 1)
                       : dim3(t_tiles, 1, static_cast<unsigned>(s.ksplit_eff));
@@ -486,7 +496,7 @@ int router_tc_padded_experts(int64_t N) {
 cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
                              const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
                              int* expert_idx, float* gate, int* local_rank,
-                             const void* l2_prefetch, size_t l2_prefetch_bytes,
+                             const void* l2_prefetch, size_t l2_prefetch_bytes, int num_sms,
                              cudaStream_t stream) {
   // the three bf16 pieces of W_r, then the router (programmatic dependent launch)
   const size_t chunks = static_cast<size_t>(s.N) * static_cast<size_t>(s.d / 8);
@@ -500,13 +510,13 @@ cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W
   if (e != cudaSuccess) return e;
   if (s.router_path == kRouterTCWide) {
     e = launch_tc_t<128, true>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch,
-                               l2_prefetch_bytes, stream);
+                               l2_prefetch_bytes, num_sms, stream);
   } else {
     switch (router_tc_padded_experts(s.N)) {
-      case 32: e = launch_tc_t<32, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
-      case 64: e = launch_tc_t<64, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
-      case 96: e = launch_tc_t<96, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
-      case 128: e = launch_tc_t<128, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, stream); break;
+      case 32: e = launch_tc_t<32, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 64: e = launch_tc_t<64, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 96: e = launch_tc_t<96, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 128: e = launch_tc_t<128, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
       default: e = cudaErrorInvalidValue; break;
     }
   }

@@ -190,7 +190,7 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
     const size_t pf = (router_ctas > 0 && router_ctas <= sms)
                           ? (w1_bytes < kL2PrefetchBytes ? w1_bytes : kL2PrefetchBytes)
                           : 0;
-    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, W1, pf,
+    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, W1, pf, sms,
                          stream) != cudaSuccess)
       return SWL_ERR_CUDA;
   } else if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert,

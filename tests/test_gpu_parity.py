@@ -306,12 +306,14 @@ def test_kernel_variant_shapes(shape):
 
 
 # Router bias on each tensor-core router path: one CTA per 128-token tile (bias
-# added at the TMEM read-out; d = 128 leaves K too short to split), 2- and 4-CTA
+# added at the TMEM read-out; d = 128 leaves K too short to split; with more
+# tiles than SMs, two CTAs of two stages each per SM), 2- and 4-CTA
 # clusters (bias added after the rank-ordered sum of the partial logits).  N is
 # not a multiple of 32 in two of them (padded expert columns), and every batch
 # ends in a ragged tile.  A mild bias (0.1 ln(1/(i+1))) keeps most experts in use.
 _ROUTER_BIAS_SHAPES = [
     ("tc_s1_bias_padded", 6000, 128, 64, 50, 1.25),
+    ("tc_s1_two_per_sm", 20000, 256, 64, 50, 1.25),   # 157 one-CTA tiles > 148 SMs: 2 stages
     ("tc_s2_bias_np128", 3000, 256, 64, 100, 1.0),
     ("tc_s4_bias_padded", 1000, 1024, 64, 40, 1.25),
 ]
