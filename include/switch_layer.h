@@ -203,6 +203,26 @@ typedef enum swl_router_mode { SWL_ROUTER_TENSOR = 0, SWL_ROUTER_FFMA = 1 } swl_
 swl_status switch_layer_set_router_mode(int mode);
 int switch_layer_router_mode(void);
 
+/* The kernels switch_layer_forward would launch for this shape on a GPU of
+ * num_sms SMs, under the current router mode, without touching the device
+ * (host-only; usable without a GPU).  Writes a NUL-terminated list of
+ * comma-separated key=value pairs into the caller's buffer buf of len bytes:
+ *   router            tc | tc_wide (tensor-core router, N <= 128 fused / wider
+ *                     logits only) | ffma_warpsplit | ffma_tile | ffma_wide
+ *   ksplit            CTAs per router tile (cluster size) or K slices
+ *   router_stages     operand stages per tensor-core router CTA (0: FFMA router)
+ *   tokens_per_block  tokens per router block (the dispatch's unit)
+ *   dispatch          fused (scan and gather in one launch) | two_kernel
+ *   ffn               sm100 (bf16, tcgen05) | f32 (SIMT)
+ *   tile_rows         token rows per expert GEMM tile
+ *   accumulators      TMEM accumulators of the bf16 expert FFN (0 for f32)
+ * Returns SWL_OK, the shape's validation error (as switch_layer_workspace_size),
+ * or SWL_ERR_INVALID_ARG when buf is NULL, num_sms <= 0 or len is too small
+ * (256 bytes always suffice). */
+swl_status switch_layer_describe_plan(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                      double capacity_factor, int num_sms, char* buf,
+                                      size_t len);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_device_status", "switch_layer_status_string",
            "switch_layer_stage_name", "switch_layer_launch_count",
            "switch_layer_forward_noalloc", "switch_layer_set_router_mode",
-           "switch_layer_router_mode")
+           "switch_layer_router_mode", "switch_layer_describe_plan")
 SWL_ROUTER_TENSOR = 0
 SWL_ROUTER_FFMA = 1
 SWL_NOALLOC_MAX_BYTES = 64 << 20
@@ -89,6 +89,9 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_set_router_mode.argtypes = [_i32]
     L.switch_layer_router_mode.restype = ctypes.c_int
     L.switch_layer_router_mode.argtypes = []
+    L.switch_layer_describe_plan.restype = _i32
+    L.switch_layer_describe_plan.argtypes = [_i64, _i64, _i64, _i64, _i32, _dbl, _i32,
+                                             ctypes.c_char_p, _sz]
     L.switch_layer_forward_noalloc.restype = _i32
     L.switch_layer_forward_noalloc.argtypes = _FWD_ARGS[:17] + [_vp, _vp]
     _lib = L
@@ -245,6 +248,20 @@ def switch_layer_set_router_mode(mode: int) -> None:
 
 def switch_layer_router_mode() -> int:
     return int(lib().switch_layer_router_mode())
+
+
+def switch_layer_describe_plan(T, d, d_ff, N, dtype: int, capacity_factor: float,
+                               num_sms: int = 148) -> dict:
+    """The kernels a forward call of this shape would launch (host-only), as a dict
+    of the C entry point's key=value pairs (integers converted)."""
+    buf = ctypes.create_string_buffer(256)
+    _check(lib().switch_layer_describe_plan(T, d, d_ff, N, dtype, capacity_factor, num_sms,
+                                            buf, len(buf)), "describe_plan")
+    out = {}
+    for kv in buf.value.decode().split(","):
+        k, v = kv.split("=", 1)
+        out[k] = int(v) if v.lstrip("-").isdigit() else v
+    return out
 
 
 # ---------------------------------------------------------------------------

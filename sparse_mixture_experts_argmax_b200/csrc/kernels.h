@@ -102,6 +102,9 @@ cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void
 // router CTAs also prefetch [l2_prefetch, +l2_prefetch_bytes) into L2 once their
 // own loads have landed (16-byte aligned, a multiple of 16 bytes; 0 bytes: none).
 int router_tc_padded_experts(int64_t N);
+// Pipeline stages of the tensor-core router kernel for this shape on a GPU of
+// num_sms SMs (what launch_router_tc uses).
+int router_tc_stages(const Shape& s, int num_sms);
 cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,
                              const CUtensorMap& tmX, const CUtensorMap& tmW, const float* b_r,
                              int* expert_idx, float* gate, int* local_rank,
@@ -137,6 +140,10 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
 
 // Tile rows for the bf16 tcgen05 GEMMs given the effective capacity.
 int bf16_tile_rows(int64_t C_eff);
+// TMEM accumulators of the bf16 expert FFN for a token tile of tile_rows rows:
+// four of 128 columns when the tile fits 128, else two of 256 (the rule the FFN
+// launcher applies to its 512 TMEM columns).
+inline int ffn_accumulators(int tile_rows) { return tile_rows <= 128 ? 4 : 2; }
 constexpr int kF32TileRows = 32;
 
 // Number of kernel launches issued by this library since load.

@@ -431,6 +431,20 @@ size_t tc_smem_bytes(int stages) {
          (2 * kMaxStages + 2) * sizeof(uint64_t) + 2 * sizeof(uint32_t);
 }
 
+// Stages of the operand ring: as many as fit, except that with more one-CTA
+// tiles than SMs each CTA gets two, so that two CTAs share an SM (their shared
+// memory, registers and 2 x 256 TMEM columns fit) and all tiles are resident at
+// once; each CTA's prologue and routing tail then overlap the other CTA's loads
+// instead of forming a second wave.
+template <int NP>
+int tc_stages(const Shape& s, bool wide, int num_sms) {
+  int stages = kMaxStages;
+  while (stages > 2 && tc_smem_bytes<NP>(stages) > kMaxDynSmem) --stages;
+  const int64_t t_tiles = (s.T + kBM - 1) / kBM;
+  if (!wide && s.ksplit_eff == 1 && 3 * NP <= 256 && t_tiles > num_sms) stages = 2;
+  return stages;
+}
+
 template <int NP, bool kWide>
 cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
                         const CUtensorMap& tmW, const float* b_r, int* expert_idx, float* gate,
@@ -453,14 +467,7 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
   a.blk_psum = ws.blk_psum;
   a.hdr = ws.hdr;
   const unsigned t_tiles = static_cast<unsigned>((s.T + kBM - 1) / kBM);
-  int stages = kMaxStages;
-  while (stages > 2 && tc_smem_bytes<NP>(stages) > kMaxDynSmem) --stages;
-  // more one-CTA tiles than SMs: two stages each, so that two CTAs share an SM
-  // (their shared memory, registers and 2 x 256 TMEM columns fit) and all tiles
-  // are resident at once; each CTA's prologue and routing tail then overlap the
-  // other CTA's loads instead of forming a second wave
-  if (!kWide && s.ksplit_eff == 1 && 3 * NP <= 256 && t_tiles > static_cast<unsigned>(num_sms))
-    stages = 2;
+  const int stages = tc_stages<NP>(s, kWide, num_sms);
   // the logits tile reuses the stage memory
   const size_t ps_bytes = static_cast<size_t>(kBM) * (NP + (kWide ? 4 : 2 * s.ksplit_eff)) * 4;
   if (ps_bytes > static_cast<size_t>(stages) * TcCfg<NP>::kStage) return cudaErrorInvalidValue;
@@ -491,6 +498,17 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
 
 int router_tc_padded_experts(int64_t N) {
   return N > kFusedRouterMaxN ? 128 : static_cast<int>((N + 31) / 32 * 32);
+}
+
+int router_tc_stages(const Shape& s, int num_sms) {
+  if (s.router_path == kRouterTCWide) return tc_stages<128>(s, true, num_sms);
+  switch (router_tc_padded_experts(s.N)) {
+    case 32: return tc_stages<32>(s, false, num_sms);
+    case 64: return tc_stages<64>(s, false, num_sms);
+    case 96: return tc_stages<96>(s, false, num_sms);
+    case 128: return tc_stages<128>(s, false, num_sms);
+    default: return 0;
+  }
 }
 
 cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W_r,

@@ -20,6 +20,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -452,6 +453,37 @@ swl_status switch_layer_set_router_mode(int mode) {
 }
 
 int switch_layer_router_mode(void) { return swl::g_router_mode.load(); }
+
+swl_status switch_layer_describe_plan(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                      double capacity_factor, int num_sms, char* buf,
+                                      size_t len) {
+  if (buf == nullptr || len == 0 || num_sms <= 0) return SWL_ERR_INVALID_ARG;
+  Shape s;
+  const swl_status st = make_shape(T, d, d_ff, N, dtype, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  const char* router = "?";
+  switch (s.router_path) {
+    case kRouterWarpSplit: router = "ffma_warpsplit"; break;
+    case kRouterTile: router = "ffma_tile"; break;
+    case kRouterWide: router = "ffma_wide"; break;
+    case kRouterTC: router = "tc"; break;
+    case kRouterTCWide: router = "tc_wide"; break;
+    default: break;
+  }
+  const bool tc = s.router_path == kRouterTC || s.router_path == kRouterTCWide;
+  const bool bf16 = s.dtype == SWL_BF16;
+  char tmp[256];
+  const int n = std::snprintf(
+      tmp, sizeof(tmp),
+      "router=%s,ksplit=%d,router_stages=%d,tokens_per_block=%d,dispatch=%s,ffn=%s,"
+      "tile_rows=%d,accumulators=%d",
+      router, s.ksplit_eff, tc ? router_tc_stages(s, num_sms) : 0, s.tpb,
+      dispatch_fused_ok(s) ? "fused" : "two_kernel", bf16 ? "sm100" : "f32", s.tile_rows,
+      bf16 ? ffn_accumulators(s.tile_rows) : 0);
+  if (n < 0 || static_cast<size_t>(n) >= len) return SWL_ERR_INVALID_ARG;
+  std::memcpy(buf, tmp, static_cast<size_t>(n) + 1);
+  return SWL_OK;
+}
 
 swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                         const void* x, const float* W_r, const void* W1,

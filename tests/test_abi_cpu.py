@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 
 import oracle
+import synth
 import sparse_mixture_experts_argmax_b200 as swl
 from sparse_mixture_experts_argmax_b200 import build as swl_build
 
@@ -117,3 +118,71 @@ def test_router_mode_switch(L):
         swl.switch_layer_set_router_mode(7)
     assert ei.value.status == 1
     assert swl.switch_layer_router_mode() == swl.SWL_ROUTER_TENSOR
+
+
+# Each GPU parity case is named for the kernel variant it exercises; the host's
+# plan (host logic only, no device) confirms that the shape takes that variant.
+_PLAN_CASES = [
+    # workloads
+    ("base_T4096_d768_N64", None, {"router": "tc", "ksplit": 4, "router_stages": 4,
+                                   "dispatch": "fused", "ffn": "sm100", "accumulators": 4}),
+    ("large_T16384_d1024_N128", None, {"router": "tc", "ksplit": 1, "router_stages": 3,
+                                       "dispatch": "two_kernel", "tile_rows": 128,
+                                       "accumulators": 4}),
+    ("skewed_T32768_d2048_N64", None, {"router": "tc", "ksplit": 1, "router_stages": 2,
+                                       "dispatch": "two_kernel", "tile_rows": 256,
+                                       "accumulators": 2}),
+    ("many_T65536_d1024_N2048", None, {"router": "tc_wide", "dispatch": "two_kernel"}),
+    ("tiny_f32_T64_d32_N4", None, {"router": "ffma_warpsplit", "ffn": "f32", "dispatch": "fused"}),
+    # test_kernel_variant_shapes
+    ("tc_np96_s4", (1000, 1024, 256, 80, 1.25, "bf16"), {"router": "tc", "ksplit": 4}),
+    ("tc_np128_s2", (2000, 256, 128, 128, 1.25, "bf16"), {"router": "tc", "ksplit": 2}),
+    ("tc_wide_ragged", (700, 256, 128, 200, 2.0, "bf16"), {"router": "tc_wide"}),
+    ("ffma_wide", (300, 48, 40, 150, 2.0, "f32"), {"router": "ffma_wide"}),
+    ("ffma_tile", (25700, 32, 32, 48, 1.0, "f32"), {"router": "ffma_tile"}),
+    ("two_kernel_dispatch", (20000, 256, 32, 8, 1.0, "f32"), {"dispatch": "two_kernel"}),
+    ("two_accumulators", (900, 64, 64, 4, 1.0, "bf16"), {"ffn": "sm100", "accumulators": 2}),
+    # test_router_bias_paths
+    ("tc_s1_bias_padded", (6000, 128, 64, 50, 1.25, "bf16"),
+     {"router": "tc", "ksplit": 1, "router_stages": 4}),
+    ("tc_s1_two_per_sm", (20000, 256, 64, 50, 1.25, "bf16"),
+     {"router": "tc", "ksplit": 1, "router_stages": 2}),
+    ("tc_s2_bias_np128", (3000, 256, 64, 100, 1.0, "bf16"), {"router": "tc", "ksplit": 2}),
+    ("tc_s4_bias_padded", (1000, 1024, 64, 40, 1.25, "bf16"), {"router": "tc", "ksplit": 4}),
+]
+
+
+@pytest.mark.parametrize("case", _PLAN_CASES, ids=lambda c: c[0])
+def test_parity_cases_take_their_kernel_variant(case):
+    name, shape, want = case
+    if shape is None:
+        w = synth.WORKLOADS[name]
+        shape = (w.T, w.d, w.d_ff, w.N, w.cf, w.dtype)
+    T, d, d_ff, N, cf, dt = shape
+    code = swl.SWL_BF16 if dt == "bf16" else swl.SWL_F32
+    plan = swl.switch_layer_describe_plan(T, d, d_ff, N, code, cf, num_sms=148)
+    assert {k: plan[k] for k in want} == want, plan
+
+
+def test_describe_plan_router_mode_and_errors(L):
+    base = (4096, 768, 3072, 64, swl.SWL_BF16, 1.25)
+    swl.switch_layer_set_router_mode(swl.SWL_ROUTER_FFMA)
+    try:
+        plan = swl.switch_layer_describe_plan(*base)
+        assert plan["router"].startswith("ffma_") and plan["router_stages"] == 0
+    finally:
+        swl.switch_layer_set_router_mode(swl.SWL_ROUTER_TENSOR)
+    # fewer SMs than one-CTA router tiles: two stages per CTA (two CTAs per SM)
+    assert swl.switch_layer_describe_plan(16384, 1024, 64, 64, swl.SWL_BF16, 1.25,
+                                          num_sms=100)["router_stages"] == 2
+    assert swl.switch_layer_describe_plan(16384, 1024, 64, 64, swl.SWL_BF16, 1.25,
+                                          num_sms=148)["router_stages"] == 4
+    small = ctypes.create_string_buffer(8)
+    assert L.switch_layer_describe_plan(*base, 148, small, len(small)) == 1   # too small
+    big = ctypes.create_string_buffer(256)
+    assert L.switch_layer_describe_plan(*base, 0, big, len(big)) == 1         # no SMs
+    assert L.switch_layer_describe_plan(*base, 148, None, 256) == 1           # no buffer
+    assert L.switch_layer_describe_plan(4096, 0, 3072, 64, swl.SWL_BF16, 1.25, 148, big,
+                                        len(big)) == 1                         # d = 0
+    assert L.switch_layer_describe_plan(4096, 764, 3072, 64, swl.SWL_BF16, 1.25, 148, big,
+                                        len(big)) != 0                         # d % 8 != 0
