@@ -145,6 +145,24 @@ def _traffic_entry(kernel: str, workload: str):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def algorithmic_bytes(T, d, d_ff, N, elem, touched, K_kept):
+    """(expert FFN launch bytes, whole-layer bytes) that the work needs at least.
+
+    FFN (both GEMMs): the weights and biases of every touched expert once,
+    (2*d*d_ff + d + d_ff) * elem each, and per kept token its packed row in, its
+    hidden row out and back in, its output row out, 2*(d + d_ff)*elem, plus its
+    destination index and gate (8 bytes).  Layer: the router (x, fp32 W_r and
+    bias), the dispatch (kept rows into and out of the packed buffer, zero rows of
+    dropped tokens, expert index / gate / position per token, the aux loss is
+    negligible) and the FFN above."""
+    w_bytes = touched * (2 * d * d_ff + d + d_ff) * elem
+    act_bytes = K_kept * (d + d_ff) * elem * 2 + K_kept * 8
+    ffn_bytes = w_bytes + act_bytes
+    layer_bytes = (T * d * elem + N * d * 4 + N * 4 + 2 * K_kept * d * elem +
+                   (T - K_kept) * d * elem + 3 * 4 * T + ffn_bytes)
+    return ffn_bytes, layer_bytes
+
+
 def run_gpu(args):
     import sparse_mixture_experts_argmax_b200 as swl
 
@@ -310,11 +328,7 @@ def run_gpu(args):
     K_kept = int(kept.sum())
     avg_stage = stage_ms.mean(axis=0)
     names = [swl.switch_layer_stage_name(i) for i in range(S)]
-    # algorithmic bytes of the expert FFN launch (both GEMMs): the weights and
-    # biases of every touched expert once, the packed activations in and out
-    w_bytes = touched * (2 * d * d_ff + d + d_ff) * elem
-    act_bytes = K_kept * (d + d_ff) * elem * 2 + K_kept * 8
-    ffn_bytes = w_bytes + act_bytes
+    ffn_bytes, layer_bytes = algorithmic_bytes(T, d, d_ff, N, elem, touched, K_kept)
     dom = "expert_ffn"
     dom_s = avg_stage[names.index(dom)] / 1e3
     peaks = _peaks()
@@ -323,11 +337,7 @@ def run_gpu(args):
     gemm_flops = 4.0 * K_kept * d * d_ff
     tensor_frac = gemm_flops / dom_s / (peaks["bf16_tflops"] * 1e12)
     # whole layer: the slower of its GEMM FLOPs at the bf16 peak and its bytes at
-    # the HBM peak, against the measured step time.  Bytes: router (x, W_r, bias),
-    # dispatch (x rows of kept tokens in and out of the packed buffer, zero rows of
-    # dropped tokens, per-token outputs), the expert FFN's bytes above, and out.
-    layer_bytes = (T * d * elem + N * d * 4 + N * 4 + 2 * K_kept * d * elem +
-                   (T - K_kept) * d * elem + 3 * 4 * T + ffn_bytes)
+    # the HBM peak, against the measured step time
     layer_floor_s = max(layer_bytes / (peaks["hbm_gbs"] * 1e9),
                         (gemm_flops + 2.0 * T * d * N) / (peaks["bf16_tflops"] * 1e12))
 

@@ -42,3 +42,28 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, "--steps", "1")
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_algorithmic_bytes_of_base_workload():
+    """The roofline's byte count for base_T4096_d768_N64: the oracle's routing of the
+    seeded batch keeps 4087 tokens over all 64 experts, and the FFN launch needs
+    9 444 864 B per touched expert plus 15 368 B per kept token: 667 280 312 B, the
+    figure the bench reports on the GPU."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import synth
+    import numpy as np
+    spec = synth.WORKLOADS["base_T4096_d768_N64"]
+    ic = synth.make_layer_inputs(spec, 0, device="cpu", redraws=synth.load_gap_redraws(spec.name))
+    ref = oracle.switch_forward(ic["x"], ic["W_r"], ic["W1"], ic["b1"], ic["W2"], ic["b2"],
+                                spec.cf, b_r=ic["b_r"])
+    C = oracle.capacity(spec.T, spec.N, spec.cf)
+    e = np.asarray(ref["expert_idx"])
+    kept = int((np.asarray(ref["pos_in_expert"]) < C).sum())
+    touched = int((np.bincount(e, minlength=spec.N) > 0).sum())
+    assert (touched, kept) == (64, 4087)
+    ffn, layer = bench.algorithmic_bytes(spec.T, spec.d, spec.d_ff, spec.N, 2, touched, kept)
+    assert ffn == 64 * 9_444_864 + 4087 * 15_368 == 667_280_312
+    # the layer adds the router's and the dispatch's bytes to the FFN's
+    assert ffn < layer < ffn + 4 * spec.T * spec.d * 2 + spec.N * spec.d * 4 + 16 * spec.T
