@@ -281,9 +281,55 @@ def pin_sampled_matches_full():
         assert np.allclose(part["out_rows"][int(t)], full["out"][t], rtol=1e-13, atol=1e-13)
 
 
+def _gap_bruteforce(z_row):
+    """max over experts i of min over j != i of (z_i - z_j), by explicit pairs:
+    for the winning expert this is its margin over the runner-up; every other
+    expert scores <= 0, and an exact tie at the top gives 0."""
+    N = len(z_row)
+    best = -np.inf
+    for i in range(N):
+        worst = np.inf
+        for j in range(N):
+            if j != i:
+                worst = min(worst, float(z_row[i]) - float(z_row[j]))
+        best = max(best, worst)
+    return best
+
+
+def pin_logit_gap():
+    """The router-logit gap that decides which seeded token rows are redrawn
+    (top-1 minus top-2 logit, on logits, not probabilities)."""
+    rng = np.random.default_rng(11)
+    # brute force over ordered pairs on small random rows, N = 2..6
+    for N in range(2, 7):
+        z = rng.normal(size=(40, N)) * 2.0
+        g = S.logit_gap(z)
+        want = np.array([_gap_bruteforce(r) for r in z])
+        assert np.array_equal(g, want), N
+    # N = 2: |z_0 - z_1| exactly
+    z = rng.normal(size=(100, 2))
+    assert np.array_equal(S.logit_gap(z), np.abs(z[:, 0] - z[:, 1]))
+    # a constructed exact tie at the top gives 0; a tie below the top does not matter
+    z = rng.normal(size=(30, 5))
+    top = z.max(axis=1) + 1.0
+    z[:, 1] = top
+    z[:, 3] = top
+    assert np.all(S.logit_gap(z) == 0.0)
+    z = np.array([[3.0, 1.0, 1.0, 0.5], [0.0, -2.0, 5.0, -2.0]])
+    assert np.array_equal(S.logit_gap(z), [2.0, 5.0])
+    # a gap of logits: unchanged by a per-row shift, scaled by a positive scale
+    # (a gap of probabilities is neither)
+    z = rng.normal(size=(50, 7))
+    shift = rng.normal(size=(50, 1)) * 10
+    assert np.allclose(S.logit_gap(z + shift), S.logit_gap(z), rtol=0, atol=1e-12)
+    assert np.allclose(S.logit_gap(4.0 * z), 4.0 * S.logit_gap(z), rtol=0, atol=1e-12)
+    # one expert: no runner-up, never redrawn
+    assert np.all(np.isinf(S.logit_gap(rng.normal(size=(4, 1)))))
+
+
 ALL_PINS = [
     pin_lb_worked_example, pin_even_routing_is_one, pin_collapse_tends_to_N,
     pin_not_a_lower_bound, pin_softmax_rows_and_closed_form, pin_ties_lowest_index,
     pin_capacity, pin_positions_bruteforce, pin_drops, pin_single_expert_is_dense_ffn,
-    pin_identical_experts_scale_by_gate, pin_sampled_matches_full,
+    pin_identical_experts_scale_by_gate, pin_sampled_matches_full, pin_logit_gap,
 ]

@@ -71,6 +71,29 @@ def _gate_is_one(p):
     return e.astype(np.int64), np.ones(p.shape[0])
 
 
+def _gap_top1_minus_min(z):
+    if z.shape[1] < 2:
+        return np.full(z.shape[0], np.inf)
+    return z.max(axis=1) - z.min(axis=1)
+
+
+def _gap_on_probs(z):
+    if z.shape[1] < 2:
+        return np.full(z.shape[0], np.inf)
+    s = np.sort(S.router_probs(z), axis=1)
+    return s[:, -1] - s[:, -2]
+
+
+def _gap_distinct_values(z):
+    # mistake: the runner-up is the largest value *different* from the top, so
+    # an exact tie at the top does not read as a zero gap
+    out = []
+    for r in z:
+        u = np.unique(r)
+        out.append(np.inf if len(u) < 2 else u[-1] - u[-2])
+    return np.asarray(out)
+
+
 MUTATIONS = {
     "ties_to_highest": ("top1", _top1_highest_tie),
     "positions_one_based": ("positions", _positions_one_based),
@@ -83,6 +106,9 @@ MUTATIONS = {
     "f_after_cut": ("load_balance_stats", _stats_after_cut),
     "logit_sign": ("router_logits", _logits_sign),
     "gate_one": ("top1", _gate_is_one),
+    "gap_top1_minus_min": ("logit_gap", _gap_top1_minus_min),
+    "gap_on_probs": ("logit_gap", _gap_on_probs),
+    "gap_ties_ignored": ("logit_gap", _gap_distinct_values),
 }
 
 
