@@ -3,11 +3,9 @@
 Routing (expert_idx, pos_in_expert, drop mask) must match bit for bit; gate,
 aux loss and outputs within the stated tolerances (see helpers.py).  The five
 named workloads run at full size, in the launch configuration the bench uses;
-the two largest compare routing for every token and outputs on sampled tokens.
+the two largest regenerate each expert's weights on demand in the oracle.
 """
 from __future__ import annotations
-
-import functools
 
 import numpy as np
 import pytest
@@ -79,50 +77,53 @@ def test_named_workload_full(name):
     assert (~ref["kept"]).sum() >= 0
 
 
-def _sampled_parity(spec: synth.LayerSpec, n_sample: int, seed=0, extra_tokens=()):
+def _every_token_parity(spec: synth.LayerSpec, seed=0):
+    """Full-size parity for layers whose fp64 weights would not fit in host
+    memory at once: the oracle routes every token, then computes the output row
+    of every kept token one expert at a time (dropped rows must be zero).  Each
+    expert's weights are the seeded inputs themselves, copied from the device
+    one expert at a time (the generator is bit-identical on CPU and GPU; see
+    test_generator_gpu_equals_cpu)."""
     rd = synth.load_gap_redraws(spec.name)
     ig = synth.make_layer_inputs(spec, seed, device="cuda", redraws=rd)
     got = _run(ig, spec.cf)
-    del ig
-    torch.cuda.empty_cache()
-    x = synth.make_x(spec, seed, redraws=rd)
-    r = synth.make_router(spec, seed)
-    rng = np.random.default_rng(1234)
-    sample = set(rng.choice(spec.T, size=n_sample, replace=False).tolist())
-    sample |= {0, spec.T - 1} | set(int(t) for t in extra_tokens)
 
-    @functools.lru_cache(maxsize=None)
     def weights(e):
-        w = synth.expert_slice(spec, [e], seed)
-        return {k: v[0] for k, v in w.items()}
+        return {k: ig[k][e].cpu() for k in ("W1", "b1", "W2", "b2")}
 
-    ref = oracle.switch_forward_sampled(x, r["W_r"], spec.cf, sorted(sample), weights,
-                                        b_r=r["b_r"])
+    x = ig["x"].cpu()
+    b_r = ig["b_r"].cpu() if ig["b_r"] is not None else None
+    ref = oracle.switch_forward_sampled(x, ig["W_r"].cpu(), spec.cf, range(spec.T), weights,
+                                        b_r=b_r)
     check_routing(got, ref, ref["capacity"], spec.T)
-    toks = sorted(ref["out_rows"])
-    g = _np(got["out"][torch.tensor(toks, device=got["out"].device)])
-    want = np.stack([ref["out_rows"][t] for t in toks])
-    check_close(g, want, spec.dtype)
+    out = got["out"]
+    kept = ref["kept"]
+    # every dropped row is exactly zero; every kept row within tolerance
+    dropped = torch.from_numpy(np.nonzero(~kept)[0]).to(out.device)
+    assert not out[dropped].any(), "a dropped token has a non-zero output row"
+    toks = np.nonzero(kept)[0]
+    want = np.stack([ref["out_rows"][int(t)] for t in toks])
+    check_close(_np(out[torch.from_numpy(toks).to(out.device)]), want, spec.dtype)
+    # every touched expert contributes compared rows, first and last kept ones included
+    touched = np.unique(ref["expert_idx"][kept])
+    assert len(touched) == len(np.unique(ref["expert_idx"]))
     return got, ref
 
 
-def test_skewed_workload_sampled():
+def test_skewed_workload_every_token():
     spec = synth.WORKLOADS["skewed_T32768_d2048_N64"]
-    # tokens of the lightly loaded experts, and expert 0's last kept / first dropped tokens
-    r = synth.make_router(spec)
-    x = synth.make_x(spec, redraws=synth.load_gap_redraws(spec.name))
-    e = np.argmax(oracle.router_logits(x, r["W_r"], r["b_r"]), axis=1)
-    others = np.nonzero(e != 0)[0][:96].tolist()
-    zero = np.nonzero(e == 0)[0]
-    C = oracle.capacity(spec.T, spec.N, spec.cf)
-    edge = zero[C - 3:C + 3].tolist()
-    got, ref = _sampled_parity(spec, 160, extra_tokens=others + edge)
+    got, ref = _every_token_parity(spec)
+    C = ref["capacity"]
+    zero = np.nonzero(ref["expert_idx"] == 0)[0]
+    # expert 0 overflows: its last kept and first dropped tokens are in the comparison
+    assert len(zero) > C and ref["kept"][zero[C - 1]] and not ref["kept"][zero[C]]
     assert (~ref["kept"]).sum() > 0
 
 
-def test_many_expert_workload_sampled():
+def test_many_expert_workload_every_token():
     spec = synth.WORKLOADS["many_T65536_d1024_N2048"]
-    _sampled_parity(spec, 80)
+    got, ref = _every_token_parity(spec)
+    assert len(np.unique(ref["expert_idx"][ref["kept"]])) == spec.N
 
 
 # ------------------------------------------------------------------ random shapes, ragged tails
@@ -250,6 +251,24 @@ def test_nonfinite_router_input_reports_device_status():
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("N", [4, 200])
+def test_infinite_router_weight_reports_device_status(dtype, N):
+    """An infinite router weight gives tokens an infinite maximum logit (+inf
+    minus +inf in the softmax would make the gate NaN): the call reports
+    SWL_ERR_DEVICE, and the context stays usable.  N = 200 takes the wide
+    router with its separate softmax kernel."""
+    spec = synth.LayerSpec("inf_wr_%s_N%d" % (dtype, N), 300, 64, 64, N, 1.0, dtype)
+    ig = synth.make_layer_inputs(spec, device="cuda")
+    w = ig["W_r"][2, 0].item()
+    ig["W_r"][2, 0] = float("inf")
+    with pytest.raises(swl.SwitchLayerError) as ei:
+        swl.forward(ig, spec.cf)
+    assert ei.value.status == 5
+    ig["W_r"][2, 0] = w
+    swl.forward(ig, spec.cf)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_router_decision_needs_float32_weights(dtype):
     """The router works in float32 (selective precision).  Experts 0 and 1 have
     weights 1 + 2^-9 and 1 + 2^-9 + 2^-17: equal in bfloat16, and equal after
@@ -282,7 +301,9 @@ def test_router_decision_needs_float32_weights(dtype):
 # the dispatch choice and the expert FFN accumulator count in csrc/):
 #   bf16 N = 80 (96-expert router tiles), K split over a 4-CTA cluster
 #   bf16 N = 128, K split over a 2-CTA cluster
-#   bf16 N = 200: tensor-core logits tiles with a ragged last expert tile + softmax kernel
+#   bf16 N = 200: tensor-core logits tiles with a ragged last expert tile + streaming softmax
+#   bf16 N = 202 (not a multiple of 4): softmax with the row held in registers
+#   bf16 N = 2100 (beyond the register row): three-pass softmax
 #   fp32 N = 150: FFMA logits with K slices + softmax kernel
 #   fp32 N = 48, ~100 big router tiles: FFMA tile router, fused dispatch
 #   fp32 N = 8, x > 16 MiB: warp-split router, two-kernel dispatch (scan + gather)
@@ -291,6 +312,8 @@ _VARIANT_SHAPES = [
     ("tc_np96_s4", 1000, 1024, 256, 80, 1.25, "bf16"),
     ("tc_np128_s2", 2000, 256, 128, 128, 1.25, "bf16"),
     ("tc_wide_ragged", 700, 256, 128, 200, 2.0, "bf16"),
+    ("tc_wide_rows", 500, 128, 64, 202, 2.0, "bf16"),
+    ("tc_wide_threepass", 300, 64, 64, 2100, 8.0, "bf16"),
     ("ffma_wide", 300, 48, 40, 150, 2.0, "f32"),
     ("ffma_tile", 25700, 32, 32, 48, 1.0, "f32"),
     ("two_kernel_dispatch", 20000, 256, 32, 8, 1.0, "f32"),
@@ -316,6 +339,7 @@ _ROUTER_BIAS_SHAPES = [
     ("tc_s1_two_per_sm", 20000, 256, 64, 50, 1.25),   # 157 one-CTA tiles > 148 SMs: 2 stages
     ("tc_s2_bias_np128", 3000, 256, 64, 100, 1.0),
     ("tc_s4_bias_padded", 1000, 1024, 64, 40, 1.25),
+    ("tc_wide_stream_bias", 3000, 256, 64, 300, 1.25),   # bias added by the streaming softmax
 ]
 
 
