@@ -5,15 +5,18 @@
 One step = one full forward pass of the layer (router logits, softmax/argmax,
 dispatch scan + aux loss, gather, expert GEMM1, expert GEMM2 + combine) over
 one batch of seeded synthetic tokens already resident in HBM.  Default
-workload: the Switch-Base-like layer (T=4096 tokens, d=768, d_ff=3072, N=64
-experts, capacity factor 1.25, bf16 with an fp32 router).
+workload: the many-expert layer, the largest of the five that fits one GPU
+(T=65536 tokens, d=1024, d_ff=2048, N=2048 experts, capacity factor 1.0, C=32,
+17 GB of bf16 expert weights, fp32 router); the other four are reachable with
+--workload.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the layer on its own
 batch (independent problems, weak scaling, no collective on the data path);
 the timed region is bracketed by barriers and the max over ranks is reported.
 
-``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), each step
-a bounded token sample of the same workload.
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only): every
+token routed, the expert FFNs of a bounded sample of experts, scaled to the
+whole batch.
 """
 from __future__ import annotations
 
@@ -36,7 +39,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 from sparse_mixture_experts_argmax_b200 import dist as swl_dist  # noqa: E402
 
-DEFAULT_WORKLOAD = "base_T4096_d768_N64"
+DEFAULT_WORKLOAD = "many_T65536_d1024_N2048"
 METRIC = "Switch-layer fwd tokens/sec on 1 B200; expert-GEMM % of bf16 tensor peak"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -149,14 +152,14 @@ def algorithmic_bytes(T, d, d_ff, N, elem, touched, K_kept):
     """(expert FFN launch bytes, whole-layer bytes) that the work needs at least.
 
     FFN (both GEMMs): the weights and biases of every touched expert once,
-    (2*d*d_ff + d + d_ff) * elem each, and per kept token its packed row in, its
-    hidden row out and back in, its output row out, 2*(d + d_ff)*elem, plus its
-    destination index and gate (8 bytes).  Layer: the router (x, fp32 W_r and
-    bias), the dispatch (kept rows into and out of the packed buffer, zero rows of
-    dropped tokens, expert index / gate / position per token, the aux loss is
-    negligible) and the FFN above."""
+    (2*d*d_ff + d + d_ff) * elem each, and per kept token its packed input row
+    in and its output row out, 2*d*elem, plus its destination index and gate
+    (8 bytes).  The hidden rows between the two GEMMs are an intermediate, not
+    algorithmic traffic.  Layer: the router (x, fp32 W_r and bias), the dispatch
+    (kept rows into the packed buffer, zero rows of dropped tokens, expert index
+    / gate / position per token; the aux loss is negligible) and the FFN above."""
     w_bytes = touched * (2 * d * d_ff + d + d_ff) * elem
-    act_bytes = K_kept * (d + d_ff) * elem * 2 + K_kept * 8
+    act_bytes = K_kept * 2 * d * elem + K_kept * 8
     ffn_bytes = w_bytes + act_bytes
     layer_bytes = (T * d * elem + N * d * 4 + N * 4 + 2 * K_kept * d * elem +
                    (T - K_kept) * d * elem + 3 * 4 * T + ffn_bytes)
@@ -273,30 +276,41 @@ def run_gpu(args):
     del graph, graph_timed
 
     # ---- end to end through the host-I/O entry point (pinned host x and outputs).
-    # Two streams, each with its own workspace and pinned buffers, take alternate
-    # steps, so one step's copies overlap the other's kernels (host-to-device and
-    # device-to-host run on separate copy engines).  Every step still copies its x
-    # in and its outputs back inside the timed region; the expert weights (larger
-    # than L2) stream from HBM in every step, so no L2 flush is interposed.
+    # Two streams, each with its own workspace, take alternate steps, so one
+    # step's copies overlap the other's kernels (host-to-device and
+    # device-to-host run on separate copy engines).  Every step copies its x in
+    # and its outputs back inside the timed region, into host buffers of its own
+    # (up to 32 sets, reused in order), and every step's outputs are compared
+    # with the device-resident run afterwards.  The expert weights (larger than
+    # L2) stream from HBM in every step, so no L2 flush is interposed.
     e2e_streams = [stream, torch.cuda.Stream(dev)]
     work_h = [swl.alloc_workspace(T, d, d_ff, N, act, cf, host_io=True, device=dev)
               for _ in range(2)]
     xh = [inputs["x"].cpu().pin_memory() for _ in range(2)]
-    oh = [[torch.empty((T, d), dtype=act).pin_memory(),
-           torch.empty(T, dtype=torch.int32).pin_memory(),
-           torch.empty(T, dtype=torch.float32).pin_memory(),
-           torch.empty(T, dtype=torch.int32).pin_memory(),
-           torch.empty(1, dtype=torch.float32).pin_memory()] for _ in range(2)]
+    n_sets = min(32, args.steps + args.steps % 2)     # even: a set stays on one stream
 
-    def step_e2e(j):
+    def out_set():
+        return [torch.empty((T, d), dtype=act).pin_memory(),
+                torch.empty(T, dtype=torch.int32).pin_memory(),
+                torch.empty(T, dtype=torch.float32).pin_memory(),
+                torch.empty(T, dtype=torch.int32).pin_memory(),
+                torch.empty(1, dtype=torch.float32).pin_memory()]
+
+    oh = [out_set() for _ in range(max(2, n_sets))]
+
+    def step_e2e(k):
+        j = k % 2
         swl.switch_layer_forward_host_io(xh[j], inputs["W_r"], inputs["W1"], inputs["b1"],
-                                         inputs["W2"], inputs["b2"], cf, *oh[j],
+                                         inputs["W2"], inputs["b2"], cf, *oh[k % len(oh)],
                                          b_r=inputs["b_r"], workspace=work_h[j],
                                          stream=e2e_streams[j])
 
     for k in range(max(2, args.warmup)):
-        step_e2e(k % 2)
+        step_e2e(k)
     torch.cuda.synchronize()
+    for o in oh:
+        o[0].fill_(0)
+        o[1].fill_(-1)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_side = torch.cuda.Event()
     _barrier(ws_n)
@@ -304,7 +318,7 @@ def run_gpu(args):
     e_start.record(e2e_streams[0])
     e2e_streams[1].wait_event(e_start)
     for k in range(args.steps):
-        step_e2e(k % 2)
+        step_e2e(k)
     e_side.record(e2e_streams[1])
     e2e_streams[0].wait_event(e_side)
     e_end.record(e2e_streams[0])
@@ -312,10 +326,15 @@ def run_gpu(args):
     _barrier(ws_n)
     e2e_total = _max_over_ranks(ws_n, float(e_start.elapsed_time(e_end)))
     e2e_value = ws_n * T * args.steps / (e2e_total / 1e3)
-    last = oh[(args.steps - 1) % 2]
-    if not torch.equal(last[0], outs["out"].cpu()) or not torch.equal(last[1],
-                                                                      outs["expert_idx"].cpu()):
-        raise RuntimeError("end-to-end outputs differ from the device-resident run")
+    for j in range(2):
+        if swl.switch_layer_device_status(work_h[j], e2e_streams[j]) != 0:
+            raise RuntimeError("device status not OK after the end-to-end steps (stream %d)" % j)
+    ref_host = [outs[k].cpu() for k in ("out", "expert_idx", "gate", "pos_in_expert",
+                                        "aux_loss")]
+    for k in range(max(0, args.steps - len(oh)), args.steps):
+        if not all(torch.equal(a, b) for a, b in zip(oh[k % len(oh)], ref_host)):
+            raise RuntimeError("end-to-end outputs of step %d differ from the device-resident "
+                               "run" % k)
     elem = 2 if act == torch.bfloat16 else 4
     h2d = T * d * elem
     d2h = T * d * elem + 3 * 4 * T + 4
@@ -328,6 +347,13 @@ def run_gpu(args):
     K_kept = int(kept.sum())
     avg_stage = stage_ms.mean(axis=0)
     names = [swl.switch_layer_stage_name(i) for i in range(S)]
+    # stages that launch no kernel for this shape report 0, not the event gap
+    plan = swl.switch_layer_describe_plan(T, d, d_ff, N, swl.dtype_code(act), cf,
+                                          torch.cuda.get_device_properties(dev).multi_processor_count)
+    if plan["softmax"] == "fused":
+        avg_stage[names.index("router_softmax")] = 0.0
+    if plan["dispatch"] == "fused":
+        avg_stage[names.index("dispatch_gather")] = 0.0
     ffn_bytes, layer_bytes = algorithmic_bytes(T, d, d_ff, N, elem, touched, K_kept)
     dom = "expert_ffn"
     dom_s = avg_stage[names.index(dom)] / 1e3
@@ -395,7 +421,7 @@ def run_gpu(args):
         "clocks": clk,
     }
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(spec, budget_s=args.cpu_budget)
+        res["cpu_baseline"] = cpu_baseline(spec, inputs, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(res), flush=True)
     swl_dist.finalize(swl_dist.rank_info())
@@ -411,28 +437,62 @@ def _blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def _oracle_step(spec, inputs, n_tok: int):
+def oracle_estimate(spec, x, W_r, b_r, weights, ffn_budget_s=None, experts=None) -> dict:
+    """The fp64 oracle on a bounded sample of one batch, scaled to the batch.
+
+    Every token is routed (fp64 logits, softmax, argmax, positions and the
+    capacity cut: oracle.switch_forward_sampled with no output rows); then the
+    oracle's expert FFN and gate scaling run on the kept rows of the experts in
+    ``experts`` (or of experts 0, 1, ... until ``ffn_budget_s`` of FFN time).
+    The whole-batch time estimate is the routing time plus the FFN time scaled
+    by (kept tokens / sampled kept tokens).  ``weights(e)`` supplies expert e's
+    host tensors outside the timed part."""
     import oracle
-    x = inputs["x"][:n_tok]
-    oracle.switch_forward(x, inputs["W_r"], inputs["W1"], inputs["b1"], inputs["W2"],
-                          inputs["b2"], spec.cf, b_r=inputs["b_r"])
-
-
-def cpu_baseline(spec, budget_s: float = 20.0, steps: int = None):
-    """The fp64 oracle on the host cores: full-batch forwards until ~budget_s."""
-    inputs = synth.make_layer_inputs(spec, 0, device="cpu",
-                                     redraws=synth.load_gap_redraws(spec.name))
     t0 = time.perf_counter()
-    _oracle_step(spec, inputs, spec.T)
-    dt = [time.perf_counter() - t0]
-    while sum(dt) < budget_s * 0.5 and len(dt) < 50:
-        t0 = time.perf_counter()
-        _oracle_step(spec, inputs, spec.T)
-        dt.append(time.perf_counter() - t0)
-    return {"value": spec.T * len(dt) / sum(dt), "unit": "tokens/s", "cores": _blas_threads(),
-            "kind": "oracle",
-            "sample": "%d full-batch fp64 oracle forwards of %s (T=%d), %.1f s wall" % (
-                len(dt), spec.name, spec.T, sum(dt))}
+    r = oracle.switch_forward_sampled(x, W_r, spec.cf, [], weights, b_r=b_r)
+    t_route = time.perf_counter() - t0
+    e, kept, g = r["expert_idx"], r["kept"], r["gate"]
+    K = int(kept.sum())
+    t_ffn, K_s, used = 0.0, 0, []
+    for i in (experts if experts is not None else range(spec.N)):
+        rows = np.nonzero((e == i) & kept)[0]
+        used.append(int(i))
+        if rows.size == 0:
+            continue
+        w = weights(int(i))
+        t1 = time.perf_counter()
+        u = oracle.expert_ffn(x[torch.from_numpy(rows)], w["W1"], w["b1"], w["W2"], w["b2"])
+        y = g[rows, None] * u
+        t_ffn += time.perf_counter() - t1
+        K_s += int(rows.size)
+        del y
+        if experts is None and t_ffn >= ffn_budget_s:
+            break
+    est = t_route + (t_ffn * K / K_s if K_s else 0.0)
+    return {"t_route": t_route, "t_ffn": t_ffn, "kept": K, "kept_sampled": K_s,
+            "experts": used, "estimate_s": est}
+
+
+def _sample_text(spec, m) -> str:
+    return ("every one of the %d tokens routed by the fp64 oracle (%.2f s); its expert FFN "
+            "timed on the %d kept rows of experts %d..%d (%.2f s) and scaled to all %d kept "
+            "rows" % (spec.T, m["t_route"], m["kept_sampled"], m["experts"][0],
+                      m["experts"][-1], m["t_ffn"], m["kept"]))
+
+
+def cpu_baseline(spec, inputs, budget_s: float = 20.0):
+    """The fp64 oracle on the host cores, on a bounded sample of the batch that
+    the GPU arm ran (its seeded inputs, copied to the host)."""
+    x = inputs["x"].cpu()
+    W_r = inputs["W_r"].cpu()
+    b_r = inputs["b_r"].cpu() if inputs["b_r"] is not None else None
+
+    def weights(e):
+        return {k: inputs[k][e].cpu() for k in ("W1", "b1", "W2", "b2")}
+
+    m = oracle_estimate(spec, x, W_r, b_r, weights, ffn_budget_s=0.6 * budget_s)
+    return {"value": spec.T / m["estimate_s"], "unit": "tokens/s", "cores": _blas_threads(),
+            "kind": "oracle", "sample": _sample_text(spec, m)}
 
 
 def run_reference(args):
@@ -440,28 +500,29 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import functools
     spec = synth.WORKLOADS[args.workload]
-    inputs = synth.make_layer_inputs(spec, 0, device="cpu",
-                                     redraws=synth.load_gap_redraws(spec.name))
-    # calibrate a token sample so warm-up + timed steps stay within ~budget seconds
-    budget = args.cpu_budget * 6
-    t0 = time.perf_counter()
-    _oracle_step(spec, inputs, spec.T)
-    t_full = time.perf_counter() - t0
-    frac = min(1.0, budget / max(1e-9, (args.steps + args.warmup) * t_full))
-    n_tok = max(128, int(spec.T * frac) // 128 * 128)
+    rd = synth.load_gap_redraws(spec.name)
+    x = synth.make_x(spec, 0, "cpu", rd)
+    r = synth.make_router(spec, 0, "cpu")
+
+    @functools.lru_cache(maxsize=None)
+    def weights(e):
+        w = synth.expert_slice(spec, [e], 0, "cpu")
+        return {k: v[0] for k, v in w.items()}
+
+    # the expert sample is fixed by a first (untimed) pass with a small FFN budget,
+    # so that warm-up and timed steps stay within a few minutes
+    m0 = oracle_estimate(spec, x, r["W_r"], r["b_r"], weights, ffn_budget_s=args.cpu_budget / 10)
+    experts = m0["experts"]
     for _ in range(args.warmup):
-        _oracle_step(spec, inputs, n_tok)
-    dts = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        _oracle_step(spec, inputs, n_tok)
-        dts.append(time.perf_counter() - t0)
-    total = sum(dts)
-    v = n_tok * args.steps / total
+        oracle_estimate(spec, x, r["W_r"], r["b_r"], weights, experts=experts)
+    ms = [oracle_estimate(spec, x, r["W_r"], r["b_r"], weights, experts=experts)
+          for _ in range(args.steps)]
+    total = sum(m["estimate_s"] for m in ms)
+    v = spec.T * args.steps / total
     cores = _blas_threads()
-    sample = ("each step: fp64 oracle forward on the first %d of %d tokens of %s "
-              "(same weights, capacity from the formula)" % (n_tok, spec.T, spec.name))
+    sample = "each step: " + _sample_text(spec, ms[-1])
     res = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
         "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,

@@ -171,8 +171,13 @@ swl_status switch_layer_device_status(const void* workspace, void* stream);
  *    last call; the call re-initialises what must start at zero.  Calls that
  *    overlap on the GPU (different streams, or host threads without ordering)
  *    race on the array and give wrong results: serialise them.
- *  - Device-side failures of this variant are not visible to
- *    switch_layer_device_status (it has no workspace pointer to read).
+ *  - The device address of the array is looked up once per device and kept
+ *    for the life of the process: after cudaDeviceReset (which unloads the
+ *    library's device code) this entry point and switch_layer_noalloc_status
+ *    must not be called again on that device.
+ *  - Device-side failures of this variant are read with
+ *    switch_layer_noalloc_status (switch_layer_device_status needs a workspace
+ *    pointer, which this variant has none of).
  *  - Allocates nothing: no cudaMalloc / cudaFree or allocating library call. */
 swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                         const void* x, const float* W_r, const void* W1,
@@ -180,6 +185,14 @@ swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int6
                                         double capacity_factor, void* out, int32_t* expert_idx,
                                         float* gate, int32_t* pos_in_expert, float* aux_loss,
                                         const float* b_r, void* stream);
+
+/* Synchronises `stream` and returns the device status of the last
+ * switch_layer_forward_noalloc call on the current device: SWL_OK, or
+ * SWL_ERR_DEVICE if one of its kernels reported a failure (a bounded pipeline
+ * wait expired, or non-finite router logits); SWL_ERR_CUDA if the
+ * synchronisation or the read failed.  Like the entry point it reports on, it
+ * allocates nothing.  The paper has no counterpart of this call either. */
+swl_status switch_layer_noalloc_status(void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* switch_layer_status_string(swl_status status);
@@ -211,6 +224,9 @@ int switch_layer_router_mode(void);
  *                     logits only) | ffma_warpsplit | ffma_tile | ffma_wide
  *   ksplit            CTAs per router tile (cluster size) or K slices
  *   router_stages     operand stages per tensor-core router CTA (0: FFMA router)
+ *   softmax           fused (in the router, N <= 128) | stream (N > 128, one
+ *                     logits slice, N % 4 == 0, N <= 2048: bulk-copied row
+ *                     chunks) | rows (row in registers) | wide (three passes)
  *   tokens_per_block  tokens per router block (the dispatch's unit)
  *   dispatch          fused (scan and gather in one launch) | two_kernel
  *   ffn               sm100 (bf16, tcgen05) | f32 (SIMT)

@@ -33,7 +33,8 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_device_status", "switch_layer_status_string",
            "switch_layer_stage_name", "switch_layer_launch_count",
            "switch_layer_forward_noalloc", "switch_layer_set_router_mode",
-           "switch_layer_router_mode", "switch_layer_describe_plan")
+           "switch_layer_router_mode", "switch_layer_describe_plan",
+           "switch_layer_noalloc_status")
 SWL_ROUTER_TENSOR = 0
 SWL_ROUTER_FFMA = 1
 SWL_NOALLOC_MAX_BYTES = 64 << 20
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
                                              ctypes.c_char_p, _sz]
     L.switch_layer_forward_noalloc.restype = _i32
     L.switch_layer_forward_noalloc.argtypes = _FWD_ARGS[:17] + [_vp, _vp]
+    L.switch_layer_noalloc_status.restype = _i32
+    L.switch_layer_noalloc_status.argtypes = [_vp]
     _lib = L
     return L
 

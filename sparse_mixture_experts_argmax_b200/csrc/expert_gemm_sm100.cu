@@ -19,18 +19,20 @@
 // streamed from HBM once per token tile no matter how few tokens an expert has.
 // D[feature, token] accumulates in TMEM.
 //
-// Persistent kernel, one CTA per SM, 256 threads:
+// Persistent kernel, one CTA per SM, 384 threads:
 //   warp 0      TMA producer (one thread): A and B k-blocks of 64 elements into a
 //               ring of shared-memory stages (128-byte swizzle)
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
 //   warp 2      TMEM allocator (512 columns: four 128-column accumulators for
 //               token tiles of up to 128 rows, else two of 256)
 //   warp 3      tile scheduler (one thread): claims, decodes and publishes tiles
-//   warps 4..7  epilogue: tcgen05.ld, bias / ReLU / gate in fp32, bf16 pack,
-//               transpose through shared memory, 16-byte stores
+//   warps 4..11 epilogue, two warps per TMEM lane quarter taking alternate
+//               32-column chunks: tcgen05.ld, bias / ReLU / gate in fp32, bf16
+//               pack, transpose through shared memory, 16-byte stores
 // Tiles (expert, 128-feature block, token block) are numbered expert-major and
-// handed out in order by a device counter; the token-block count of each expert
-// comes from the device tile prefix written by the dispatch scan.  The
+// handed out in order by a device counter, every tile (a CTA's first included)
+// claimed by a CTA that is already running; the token-block count of each
+// expert comes from the device tile prefix written by the dispatch scan.  The
 // scheduler keeps the claim, the decode (dependent loads of the prefix) and the
 // GEMM2 readiness wait off the producer's path.  Every wait is bounded; a
 // stuck pipeline sets the device error word and the CTA drains and exits.
@@ -213,7 +215,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     // Claims the next tile only once the producer has taken the previous one (so
     // a CTA holds at most one claimed tile it has not started), decodes it, waits
     // for its GEMM1 rows when it is a GEMM2 tile, and publishes it in the ring.
-    // CTA c starts with tile c; the counter hands out tiles from gridDim.x on.
+    // Every tile comes from the counter, so only a running CTA owns a tile: when
+    // a GEMM2 tile is claimed, every GEMM1 tile (lower numbers) has already been
+    // claimed by a running CTA, whose pipeline finishes it without waiting on
+    // anything but its own stages (its epilogue publishes before it blocks), so
+    // the readiness wait below ends even when other kernels hold some SMs.
     const int* P = args.tile_prefix;
     if (args.cache_prefix) {
       for (int e = lane; e <= args.num_experts; e += 32) s_prefix[e] = args.tile_prefix[e];
@@ -231,8 +237,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           fail();
           break;
         }
-        const unsigned int claimed =
-            i == 0 ? blockIdx.x : gridDim.x + atomicAdd(args.next_tile, 1u);
+        const unsigned int claimed = atomicAdd(args.next_tile, 1u);
         TileSlot ts;
         ts.t = claimed < static_cast<unsigned int>(total) ? static_cast<int>(claimed) : -1;
         ts.phase = ts.e = ts.mt = ts.nt = ts.g = ts.rows = ts.row0 = 0;

@@ -112,6 +112,13 @@ cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W
                              cudaStream_t stream);
 // Expert weights fetched into L2 during the router and dispatch stages.
 constexpr size_t kL2PrefetchBytes = 64u << 20;
+// Softmax kernel of a shape: none (fused into the router, N <= 128), the
+// streaming kernel (one logits slice, N % 4 == 0, N <= kStreamSoftmaxMaxN), the
+// register-row kernel (N <= 2048) or the three-pass kernel (any N).
+enum SoftmaxVariant : int { kSoftmaxFused = 0, kSoftmaxStream = 1, kSoftmaxRows = 2,
+                            kSoftmaxWide = 3 };
+constexpr int kStreamSoftmaxMaxN = 2048;
+int softmax_variant(const Shape& s);
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);

@@ -19,6 +19,7 @@
 
 #include "kernels.h"
 #include "router_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -301,8 +302,10 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
     const float inv = 1.0f / ssum;
 #pragma unroll
     for (int j = 0; j < NPL; ++j) acc[j] += v[j] * inv;
-    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
-      bidx = 0;
+    // a non-finite logit (NaN, or an infinite maximum that makes the exp sum
+    // NaN) is flagged; an index with no finite maximum is kept in range
+    if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
+      if (bidx >= N) bidx = 0;
       if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
     }
     if (lane == 0) {
@@ -383,8 +386,10 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
     for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
     const float inv = 1.0f / ssum;
     for (int j = lane; j < N; j += 32) row[j] *= inv;
-    if (bidx >= N) {
-      bidx = 0;
+    // a non-finite logit (NaN, or an infinite maximum that makes the exp sum
+    // NaN) is flagged; an index with no finite maximum is kept in range
+    if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
+      if (bidx >= N) bidx = 0;
       if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
     }
     if (lane == 0) {
@@ -407,6 +412,212 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
   __syncthreads();
   for (int i = threadIdx.x; i < ntok; i += kSoftmaxThreads) {
     if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
+  }
+}
+
+// Streaming softmax for N > 128 whose logits come in one slice (ksplit = 1)
+// with N % 4 == 0: a persistent CTA per SM takes dispatch blocks b =
+// blockIdx.x, blockIdx.x + gridDim.x, ...; each block's rows arrive in chunks
+// of kStreamChunk consecutive token rows (contiguous in [T, N]) through a ring
+// of kStreamBufs shared-memory buffers filled by single bulk copies
+// (cp.async.bulk), so a whole chunk is in flight while the previous ones are
+// processed.  Per chunk:
+//   pass A, one warp per token row: lane l holds the float4 columns l, l + 32,
+//     ... in registers (+ b_r); max with the lowest index on ties and the exp
+//     sum in four interleaved chains, warp-reduced; gate = 1/s; p = exp(z - m)/s
+//     written back over the row;
+//   pass B, each thread owns the float4 columns tid, tid + 256, ... and adds
+//     the chunk's p rows to its per-block sums in token order.
+// At the end of a block: in-block ranks, per-expert counts and the block's
+// sums of p (each column owned by one thread: no reduction needed).
+constexpr int kStreamThreads = 256;
+constexpr int kStreamChunk = kStreamThreads / 32;   // token rows per chunk (one per warp)
+constexpr int kStreamBufs = 3;
+
+__host__ __device__ constexpr size_t stream_softmax_smem(int N) {
+  return 128 + (static_cast<size_t>(kStreamBufs) * kStreamChunk + 1) * N * sizeof(float);
+}
+
+template <int V4>   // float4 columns per lane in pass A: N <= 128 * V4
+__global__ void __launch_bounds__(kStreamThreads, 1)
+router_softmax_stream_kernel(const float* __restrict__ z, const float* __restrict__ b_r, int T,
+                             int N, int tpb, int nblk, int* __restrict__ expert_idx,
+                             float* __restrict__ gate, int* __restrict__ local_rank,
+                             int* __restrict__ blk_count, float* __restrict__ blk_psum,
+                             WsHeader* hdr) {
+  constexpr int VPT = (V4 * 32 + kStreamThreads - 1) / kStreamThreads;   // pass-B float4 / thread
+  extern __shared__ uint8_t smem_raw[];
+  float* buf = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  float* s_bias = buf + static_cast<size_t>(kStreamBufs) * kStreamChunk * N;   // [N]
+  __shared__ uint64_t full[kStreamBufs];
+  __shared__ int eid[kTokensPerBlock];
+  __shared__ int lead_count[kTokensPerBlock];
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NV = N >> 2;   // float4 per row
+  pdl_trigger();
+  if (tid == 0) {
+    for (int i = 0; i < kStreamBufs; ++i) ptx::mbar_init(&full[i], 1);
+    s_abort = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+  }
+  for (int n = tid; n < N; n += kStreamThreads) s_bias[n] = b_r ? b_r[n] : 0.f;
+  __syncthreads();
+  pdl_wait();   // the logits come from the logits kernel
+
+  // chunk sequence of this CTA (the producer's copy of the consumers' order)
+  int pb = blockIdx.x, pc = 0, issued = 0;
+  auto issue_next = [&](int slot) {
+    if (pb >= nblk) return;
+    const int tb = pb * tpb, nb = min(tpb, T - tb);
+    const int t0 = tb + pc * kStreamChunk;
+    const int n = min(kStreamChunk, tb + nb - t0);
+    const uint32_t bytes = static_cast<uint32_t>(n) * static_cast<uint32_t>(N) * 4u;
+    ptx::mbar_arrive_expect_tx(&full[slot], bytes);
+    ptx::bulk_load_g2s(buf + static_cast<size_t>(slot) * kStreamChunk * N,
+                       z + static_cast<size_t>(t0) * N, bytes, &full[slot]);
+    ++issued;
+    if (++pc * kStreamChunk >= nb) { pc = 0; pb += gridDim.x; }
+  };
+  if (tid == 0)
+    for (int i = 0; i < kStreamBufs - 1; ++i) issue_next(i);
+
+  int ci = 0;   // chunks consumed
+  bool failed = false;
+  for (int b = blockIdx.x; b < nblk && !failed; b += gridDim.x) {
+    const int t0b = b * tpb, ntb = min(tpb, T - t0b);
+    float4 acc[VPT];
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c * kStreamChunk < ntb; ++c, ++ci) {
+      const int slot = ci % kStreamBufs;
+      if (tid == 0) {
+        // the buffer of chunk ci - 1 is free (barrier below): refill it ahead
+        ptx::fence_proxy_async_smem();
+        issue_next((ci + kStreamBufs - 1) % kStreamBufs);
+      }
+      volatile int* ab = &s_abort;
+      const bool ok = ptx::mbar_wait(&full[slot], static_cast<uint32_t>(ci / kStreamBufs) & 1u, ab);
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      float* zc = buf + static_cast<size_t>(slot) * kStreamChunk * N;
+      const int nt = min(kStreamChunk, ntb - c * kStreamChunk);
+      if (warp < nt) {
+        float4* row = reinterpret_cast<float4*>(zc + static_cast<size_t>(warp) * N);
+        const float4* bias4 = reinterpret_cast<const float4*>(s_bias);
+        float4 v[V4];
+        float bq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        int iq[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+#pragma unroll
+        for (int k = 0; k < V4; ++k) {
+          const int q = lane + 32 * k;
+          if (q < NV) {
+            const float4 a = row[q], bb = bias4[q];
+            v[k] = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
+          } else {
+            v[k] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+          }
+          // chain c holds column 4q + c: ascending columns per chain, so the
+          // strict compare keeps each chain's lowest index among equal maxima
+          if (v[k].x > bq[0]) { bq[0] = v[k].x; iq[0] = 4 * q; }
+          if (v[k].y > bq[1]) { bq[1] = v[k].y; iq[1] = 4 * q + 1; }
+          if (v[k].z > bq[2]) { bq[2] = v[k].z; iq[2] = 4 * q + 2; }
+          if (v[k].w > bq[3]) { bq[3] = v[k].w; iq[3] = 4 * q + 3; }
+        }
+        float best = bq[0];
+        int bidx = iq[0];
+#pragma unroll
+        for (int c4 = 1; c4 < 4; ++c4)
+          if (bq[c4] > best || (bq[c4] == best && iq[c4] < bidx)) { best = bq[c4]; bidx = iq[c4]; }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+          if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+        }
+        float sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < V4; ++k) {
+          v[k].x = expf(v[k].x - best);
+          v[k].y = expf(v[k].y - best);
+          v[k].z = expf(v[k].z - best);
+          v[k].w = expf(v[k].w - best);
+          sq[0] += v[k].x;
+          sq[1] += v[k].y;
+          sq[2] += v[k].z;
+          sq[3] += v[k].w;
+        }
+        float ssum = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+        const float inv = 1.0f / ssum;
+#pragma unroll
+        for (int k = 0; k < V4; ++k) {
+          const int q = lane + 32 * k;
+          if (q < NV)
+            row[q] = make_float4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
+        }
+        // a non-finite logit (NaN, or an infinite maximum that makes the exp
+        // sum NaN) is flagged; an index with no finite maximum is kept in range
+        if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
+          if (bidx >= N) bidx = 0;
+          if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
+        }
+        if (lane == 0) {
+          const int t = t0b + c * kStreamChunk + warp;
+          expert_idx[t] = bidx;
+          gate[t] = inv;          // p at the argmax: exp(0) / s
+          eid[c * kStreamChunk + warp] = bidx;
+        }
+      }
+      __syncthreads();
+      const float4* zc4 = reinterpret_cast<const float4*>(zc);
+#pragma unroll
+      for (int v = 0; v < VPT; ++v) {
+        const int q = tid + kStreamThreads * v;
+        if (q < NV) {
+          for (int r = 0; r < nt; ++r) {
+            const float4 p = zc4[static_cast<size_t>(r) * NV + q];
+            acc[v].x += p.x;
+            acc[v].y += p.y;
+            acc[v].z += p.z;
+            acc[v].w += p.w;
+          }
+        }
+      }
+      __syncthreads();   // the chunk buffer is free again
+    }
+    if (failed) break;
+    // block bookkeeping: ranks, the block's per-expert counts and sums of p
+    block_ranks(eid, lead_count, ntb, ntb, t0b, local_rank);
+    int* cnt_row = blk_count + static_cast<size_t>(b) * N;
+    float* ps_row = blk_psum + static_cast<size_t>(b) * N;
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+      const int q = tid + kStreamThreads * v;
+      if (q < NV) {
+        reinterpret_cast<float4*>(ps_row)[q] = acc[v];
+        reinterpret_cast<int4*>(cnt_row)[q] = make_int4(0, 0, 0, 0);
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < ntb; i += kStreamThreads)
+      if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
+    __syncthreads();   // eid / lead_count are reused by the next block
+  }
+  if (failed) {
+    atomicExch(&hdr->err, kDevPipelineTimeout);
+    // every issued copy must land before the CTA's shared memory goes away
+    if (tid == 0) {
+      volatile int never = 0;
+      for (int j = ci; j < issued; ++j)
+        ptx::mbar_wait(&full[j % kStreamBufs], static_cast<uint32_t>(j / kStreamBufs) & 1u, &never);
+    }
+    __syncthreads();
   }
 }
 
@@ -612,8 +823,10 @@ router_warpsplit_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
     const float inv = 1.0f / ssum;
 #pragma unroll
     for (int j = 0; j < NPL; ++j) pacc[j] += v[j] * inv;
-    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
-      bidx = 0;
+    // a non-finite logit (NaN, or an infinite maximum that makes the exp sum
+    // NaN) is flagged; an index with no finite maximum is kept in range
+    if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
+      if (bidx >= N) bidx = 0;
       if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
     }
     if (lane == 0) {
@@ -903,12 +1116,43 @@ cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void
   return e;
 }
 
+int softmax_variant(const Shape& s) {
+  if (s.N <= kFusedRouterMaxN) return kSoftmaxFused;
+  if (s.ksplit_eff == 1 && s.N % 4 == 0 && s.N <= kStreamSoftmaxMaxN) return kSoftmaxStream;
+  return (s.N + 31) / 32 <= 64 ? kSoftmaxRows : kSoftmaxWide;
+}
+
+template <int V4>
+cudaError_t launch_stream_t(const Shape& s, const Workspace& ws, const float* b_r,
+                            int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
+  const size_t smem = stream_softmax_smem(static_cast<int>(s.N));
+  cudaError_t e = cudaFuncSetAttribute(router_softmax_stream_kernel<V4>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const int grid = s.nblk < sms ? s.nblk : sms;
+  return launch_dependent(router_softmax_stream_kernel<V4>, dim3(grid), dim3(kStreamThreads),
+                          smem, stream, static_cast<const float*>(ws.logits), b_r, (int)s.T,
+                          (int)s.N, s.tpb, s.nblk, expert_idx, gate, local_rank, ws.blk_count,
+                          ws.blk_psum, ws.hdr);
+}
+
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream) {
   cudaError_t e;
   const int64_t npl = (s.N + 31) / 32;
-  if (npl <= 1) e = launch_softmax_t<1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+  if (softmax_variant(s) == kSoftmaxStream) {
+    const int64_t v4 = (s.N / 4 + 31) / 32;
+    if (v4 <= 2) e = launch_stream_t<2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else if (v4 <= 4) e = launch_stream_t<4>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else if (v4 <= 8) e = launch_stream_t<8>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else e = launch_stream_t<16>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+  } else if (npl <= 1) e = launch_softmax_t<1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 2) e = launch_softmax_t<2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 4) e = launch_softmax_t<4>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 8) e = launch_softmax_t<8>(s, ws, b_r, expert_idx, gate, local_rank, stream);

@@ -84,8 +84,10 @@ __device__ __forceinline__ void route_rows(const float* Z, int zs, int R, int nt
     const float inv = 1.0f / ssum;
 #pragma unroll
     for (int j = 0; j < NPL; ++j) pacc[j] += v[j] * inv;
-    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
-      bidx = 0;
+    // a non-finite logit (NaN, or an infinite maximum that makes the exp sum
+    // NaN) is flagged; an index with no finite maximum is kept in range
+    if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
+      if (bidx >= N) bidx = 0;
       if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
     }
     if (lane == 0) {
@@ -186,8 +188,10 @@ __device__ __forceinline__ void route_rows_grouped(float* Z, int zs, int ntok, i
   if (valid) {
 #pragma unroll
     for (int j = 0; j < EPT; ++j) zr[j * TPT] = v[j] * inv;
-    if (bidx >= N) {          // no finite maximum (non-finite logits): flag, keep in range
-      bidx = 0;
+    // a non-finite logit (NaN, or an infinite maximum that makes the exp sum
+    // NaN) is flagged; an index with no finite maximum is kept in range
+    if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
+      if (bidx >= N) bidx = 0;
       if (sub == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
     }
     if (sub == 0) {

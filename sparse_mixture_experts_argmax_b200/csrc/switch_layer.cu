@@ -472,12 +472,14 @@ swl_status switch_layer_describe_plan(int64_t T, int64_t d, int64_t d_ff, int64_
   }
   const bool tc = s.router_path == kRouterTC || s.router_path == kRouterTCWide;
   const bool bf16 = s.dtype == SWL_BF16;
+  static const char* const softmax_names[4] = {"fused", "stream", "rows", "wide"};
   char tmp[256];
   const int n = std::snprintf(
       tmp, sizeof(tmp),
-      "router=%s,ksplit=%d,router_stages=%d,tokens_per_block=%d,dispatch=%s,ffn=%s,"
-      "tile_rows=%d,accumulators=%d",
-      router, s.ksplit_eff, tc ? router_tc_stages(s, num_sms) : 0, s.tpb,
+      "router=%s,ksplit=%d,router_stages=%d,softmax=%s,tokens_per_block=%d,dispatch=%s,"
+      "ffn=%s,tile_rows=%d,accumulators=%d",
+      router, s.ksplit_eff, tc ? router_tc_stages(s, num_sms) : 0,
+      softmax_names[softmax_variant(s)], s.tpb,
       dispatch_fused_ok(s) ? "fused" : "two_kernel", bf16 ? "sm100" : "f32", s.tile_rows,
       bf16 ? ffn_accumulators(s.tile_rows) : 0);
   if (n < 0 || static_cast<size_t>(n) >= len) return SWL_ERR_INVALID_ARG;
@@ -501,6 +503,12 @@ swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int6
   return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
                       expert_idx, gate, pos_in_expert, aux_loss, b_r, scratch,
                       static_cast<size_t>(SWL_NOALLOC_MAX_BYTES), stream, nullptr);
+}
+
+swl_status switch_layer_noalloc_status(void* stream) {
+  void* scratch = noalloc_scratch_for_current_device();
+  if (scratch == nullptr) return SWL_ERR_CUDA;
+  return switch_layer_device_status(scratch, stream);   // reads the scratch's header word
 }
 
 }  // extern "C"

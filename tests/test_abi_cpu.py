@@ -132,13 +132,19 @@ _PLAN_CASES = [
     ("skewed_T32768_d2048_N64", None, {"router": "tc", "ksplit": 1, "router_stages": 2,
                                        "dispatch": "two_kernel", "tile_rows": 256,
                                        "accumulators": 2}),
-    ("many_T65536_d1024_N2048", None, {"router": "tc_wide", "dispatch": "two_kernel"}),
+    ("many_T65536_d1024_N2048", None, {"router": "tc_wide", "softmax": "stream",
+                                       "dispatch": "two_kernel"}),
     ("tiny_f32_T64_d32_N4", None, {"router": "ffma_warpsplit", "ffn": "f32", "dispatch": "fused"}),
     # test_kernel_variant_shapes
     ("tc_np96_s4", (1000, 1024, 256, 80, 1.25, "bf16"), {"router": "tc", "ksplit": 4}),
     ("tc_np128_s2", (2000, 256, 128, 128, 1.25, "bf16"), {"router": "tc", "ksplit": 2}),
-    ("tc_wide_ragged", (700, 256, 128, 200, 2.0, "bf16"), {"router": "tc_wide"}),
-    ("ffma_wide", (300, 48, 40, 150, 2.0, "f32"), {"router": "ffma_wide"}),
+    ("tc_wide_ragged", (700, 256, 128, 200, 2.0, "bf16"), {"router": "tc_wide",
+                                                            "softmax": "stream"}),
+    ("tc_wide_rows", (500, 128, 64, 202, 2.0, "bf16"), {"router": "tc_wide",
+                                                         "softmax": "rows"}),
+    ("tc_wide_threepass", (300, 64, 64, 2100, 8.0, "bf16"), {"router": "tc_wide",
+                                                              "softmax": "wide"}),
+    ("ffma_wide", (300, 48, 40, 150, 2.0, "f32"), {"router": "ffma_wide", "softmax": "rows"}),
     ("ffma_tile", (25700, 32, 32, 48, 1.0, "f32"), {"router": "ffma_tile"}),
     ("two_kernel_dispatch", (20000, 256, 32, 8, 1.0, "f32"), {"dispatch": "two_kernel"}),
     ("two_accumulators", (900, 64, 64, 4, 1.0, "bf16"), {"ffn": "sm100", "accumulators": 2}),
@@ -149,6 +155,8 @@ _PLAN_CASES = [
      {"router": "tc", "ksplit": 1, "router_stages": 2}),
     ("tc_s2_bias_np128", (3000, 256, 64, 100, 1.0, "bf16"), {"router": "tc", "ksplit": 2}),
     ("tc_s4_bias_padded", (1000, 1024, 64, 40, 1.25, "bf16"), {"router": "tc", "ksplit": 4}),
+    ("tc_wide_stream_bias", (3000, 256, 64, 300, 1.25, "bf16"),
+     {"router": "tc_wide", "softmax": "stream"}),
 ]
 
 

@@ -17,7 +17,8 @@ def _run(env_extra, *args):
 
 
 def test_reference_arm_line():
-    r = _run({}, "--steps", "1", "--warmup", "0", "--cpu-budget", "0.5")
+    r = _run({}, "--workload", "base_T4096_d768_N64", "--steps", "1", "--warmup", "0",
+             "--cpu-budget", "0.5")
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1, r.stdout
@@ -44,11 +45,20 @@ def test_reference_arm_other_ranks_exit_quietly():
     assert r.stdout.strip() == ""
 
 
+def test_default_workload_is_the_largest_single_gpu_layer():
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    big = max(synth.WORKLOADS.values(), key=lambda w: w.T * w.d + 2 * w.N * w.d * w.d_ff)
+    assert bench.DEFAULT_WORKLOAD == big.name == "many_T65536_d1024_N2048"
+
+
 def test_algorithmic_bytes_of_base_workload():
     """The roofline's byte count for base_T4096_d768_N64: the oracle's routing of the
     seeded batch keeps 4087 tokens over all 64 experts, and the FFN launch needs
-    9 444 864 B per touched expert plus 15 368 B per kept token: 667 280 312 B, the
-    figure the bench reports on the GPU."""
+    9 444 864 B per touched expert (weights and biases) plus 3 080 B per kept token
+    (its input row in, its output row out, destination index and gate):
+    617 059 256 B.  The hidden rows between the GEMMs are not counted."""
     sys.path.insert(0, ROOT)
     import bench
     import oracle
@@ -64,6 +74,6 @@ def test_algorithmic_bytes_of_base_workload():
     touched = int((np.bincount(e, minlength=spec.N) > 0).sum())
     assert (touched, kept) == (64, 4087)
     ffn, layer = bench.algorithmic_bytes(spec.T, spec.d, spec.d_ff, spec.N, 2, touched, kept)
-    assert ffn == 64 * 9_444_864 + 4087 * 15_368 == 667_280_312
+    assert ffn == 64 * 9_444_864 + 4087 * 3_080 == 617_059_256
     # the layer adds the router's and the dispatch's bytes to the FFN's
     assert ffn < layer < ffn + 4 * spec.T * spec.d * 2 + spec.N * spec.d * 4 + 16 * spec.T
