@@ -10,9 +10,11 @@ workload: the many-expert layer, the largest of the five that fits one GPU
 17 GB of bf16 expert weights, fp32 router); the other four are reachable with
 --workload.
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs the layer on its own
-batch (independent problems, weak scaling, no collective on the data path);
-the timed region is bracketed by barriers and the max over ranks is reported.
+Multi-GPU (torchrun, one rank per GPU): one global batch, each rank holding a
+contiguous range of T tokens and all weights; one NCCL all-gather of
+per-expert counts and sums of p per step gives every rank the whole batch's
+positions, capacity and aux loss (weak scaling: per-GPU work fixed).  The
+timed region is bracketed by barriers and the max over ranks is reported.
 
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only): every
 token routed, the expert FFNs of a bounded sample of experts, scaled to the
@@ -383,7 +385,7 @@ def run_gpu(args):
         "config": {
             "workload": spec.name, "T": T, "d": d, "d_ff": d_ff, "N": N,
             "capacity_factor": cf, "capacity": swl.switch_layer_capacity(T, N, cf),
-            "router": router_desc, "parallelism": "dp%d (independent batches)" % ws_n,
+            "router": router_desc, "parallelism": "single GPU",
             "l2": "flushed between timed steps (256 MiB write, outside the step events); "
                   "expert weights %.0f MB > 126 MB L2" % (2 * N * d * d_ff * elem / 1e6),
         },
@@ -425,6 +427,171 @@ def run_gpu(args):
     if rank == 0:
         print(json.dumps(res), flush=True)
     swl_dist.finalize(swl_dist.rank_info())
+
+
+def run_gpu_sharded(args):
+    """N > 1 ranks: ONE global batch of N x T tokens, rank g holding the g-th
+    contiguous range of T tokens (rank 0 the workload's own seeded tokens, rank
+    g > 0 tokens drawn with seed g) and a full copy of the weights (seed 0).
+    Positions, capacity C = ceil(cf * N * T / experts) and the aux loss are
+    those of the whole batch: a step is the library's shard step 1 (routing and
+    this rank's exchange record), an NCCL all-gather of the records (12 bytes
+    per expert and rank), and shard step 3 (offsets of earlier ranks, dispatch,
+    expert FFN).  Per-GPU work is fixed as N grows: weak scaling."""
+    import sparse_mixture_experts_argmax_b200 as swl
+
+    ws_n, rank, local = _dist_init()
+    info = swl_dist.rank_info()
+    dev = torch.device("cuda", local)
+    spec = synth.WORKLOADS[args.workload]
+    T, d, d_ff, N, cf = spec.T, spec.d, spec.d_ff, spec.N, spec.cf
+    T_total = ws_n * T
+    swl.switch_layer_set_router_mode(swl.SWL_ROUTER_FFMA if args.router == "ffma"
+                                     else swl.SWL_ROUTER_TENSOR)
+    inputs = synth.make_layer_inputs(spec, seed=0, device=dev,
+                                     redraws=synth.load_gap_redraws(spec.name))
+    if rank > 0:
+        inputs["x"] = synth.make_x(spec, seed=rank, device=dev)
+    act = inputs["x"].dtype
+    elem = 2 if act == torch.bfloat16 else 4
+    work = swl.alloc_workspace(T, d, d_ff, N, act, cf, device=dev)
+    outs = swl.alloc_outputs(T, d, act, device=dev)
+    record = torch.empty(swl.switch_layer_shard_record_bytes(N), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x, ev=None):
+        swl.switch_layer_forward_shard_begin(x, inputs["W_r"], cf, T_total, outs["expert_idx"],
+                                             outs["gate"], outs["pos_in_expert"], record, d_ff,
+                                             b_r=inputs["b_r"], workspace=work, stream=stream)
+        gathered = swl_dist.exchange_records(info, record)
+        if ev is not None:
+            ev.record(stream)
+        swl.switch_layer_forward_shard_end(x, inputs["W1"], inputs["b1"], inputs["W2"],
+                                           inputs["b2"], cf, T_total, rank, ws_n, gathered,
+                                           outs["out"], outs["expert_idx"], outs["gate"],
+                                           outs["pos_in_expert"], outs["aux_loss"],
+                                           workspace=work, stream=stream)
+
+    launches_per_step = 0
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        c0 = swl.switch_layer_launch_count()
+        step(inputs["x"])
+        launches_per_step = swl.switch_layer_launch_count() - c0
+    torch.cuda.synchronize()
+    if swl.switch_layer_device_status(work, stream) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    # ---- timed region: K steps, L2 flushed between steps (outside the step events)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for e3 in ev:
+        for e in e3:
+            e.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    _barrier(ws_n)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record(stream)
+        step(inputs["x"], ev[k][1])
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    _barrier(ws_n)
+    clk = clocks.stop()
+    step_ms = np.array([a.elapsed_time(c) for a, _, c in ev])
+    end_ms = np.array([b.elapsed_time(c) for _, b, c in ev])
+    total_ms = _max_over_ranks(ws_n, float(step_ms.sum()))
+    ms_per_step = total_ms / args.steps
+    value = swl_dist.aggregate_throughput(info, T, args.steps, total_ms)
+    if swl.switch_layer_device_status(work, stream) != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+    ref_host = [outs[k].cpu() for k in ("out", "expert_idx", "gate", "pos_in_expert",
+                                        "aux_loss")]
+
+    # ---- end to end through the public API: pinned host x copied in, the two
+    # shard steps and the all-gather, outputs copied back, every step
+    xh = inputs["x"].cpu().pin_memory()
+    x_dev = torch.empty_like(inputs["x"])
+    oh = [[torch.empty_like(t, device="cpu").pin_memory() for t in ref_host]
+          for _ in range(min(32, args.steps))]
+
+    def step_e2e(k):
+        x_dev.copy_(xh, non_blocking=True)
+        step(x_dev)
+        for h, key in zip(oh[k % len(oh)], ("out", "expert_idx", "gate", "pos_in_expert",
+                                            "aux_loss")):
+            h.copy_(outs[key], non_blocking=True)
+
+    for k in range(args.warmup):
+        step_e2e(k)
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws_n)
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for k in range(args.steps):
+        step_e2e(k)
+    e_end.record(stream)
+    e_end.synchronize()
+    _barrier(ws_n)
+    e2e_total = _max_over_ranks(ws_n, float(e_start.elapsed_time(e_end)))
+    e2e_value = ws_n * T * args.steps / (e2e_total / 1e3)
+    if swl.switch_layer_device_status(work, stream) != 0:
+        raise RuntimeError("device status not OK after the end-to-end steps")
+    for k in range(max(0, args.steps - len(oh)), args.steps):
+        if not all(torch.equal(a, b) for a, b in zip(oh[k % len(oh)], ref_host)):
+            raise RuntimeError("end-to-end outputs of step %d differ" % k)
+
+    C = swl.switch_layer_capacity(T_total, N, cf)
+    kept = outs["pos_in_expert"].long() < C
+    counts = torch.bincount(outs["expert_idx"].long()[kept], minlength=N)
+    touched = int((counts > 0).sum())
+    K_kept = int(kept.sum())
+    ffn_bytes, layer_bytes = algorithmic_bytes(T, d, d_ff, N, elem, touched, K_kept)
+    gather_bytes = 2 * K_kept * d * elem + (T - K_kept) * d * elem
+    end_s = float(end_ms.mean()) / 1e3
+    peaks = _peaks()
+    achieved = (ffn_bytes + gather_bytes) / end_s / 1e9
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if act == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded; x ~ N(0,1), T5 truncated-normal init s=0.1)",
+        "config": {
+            "workload": spec.name, "T": T, "d": d, "d_ff": d_ff, "N": N, "capacity_factor": cf,
+            "global_batch": T_total, "capacity": C,
+            "parallelism": "dp%d: one global batch, contiguous token range per rank, weights "
+                           "replicated; one all-gather of per-expert counts and sums of p "
+                           "per step" % ws_n,
+            "l2": "flushed between timed steps (256 MiB write, outside the step events); "
+                  "expert weights %.0f MB > 126 MB L2" % (2 * N * d * d_ff * elem / 1e6),
+        },
+        "stages_us": {"shard_end": round(float(end_ms.mean()) * 1e3, 2),
+                      "begin_and_exchange": round(float((step_ms - end_ms).mean()) * 1e3, 2)},
+        "roofline": {
+            "kernel": "shard step 3 (combine, gather, expert FFN)", "bound": "hbm",
+            "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "algorithmic_bytes": ffn_bytes + gather_bytes,
+            "peak_source": peaks["source"] + " (burst copy)",
+        },
+        "routing": {"experts_touched_here": touched, "kept_tokens_here": K_kept,
+                    "aux_loss": float(outs["aux_loss"][0])},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * elem,
+                "d2h_bytes_per_step": T * d * elem + 3 * 4 * T + 4,
+                "note": "per step: pinned host x in, both shard steps and the all-gather, "
+                        "out / expert_idx / gate / pos_in_expert / aux_loss back"},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    swl_dist.finalize(info)
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -552,6 +719,9 @@ def main():
     ap.add_argument("--router", default="tensor", choices=["tensor", "ffma"],
                     help="fp32 router logits of bf16 layers: tensor cores on the exact bf16 "
                          "split of W_r (default) or FFMA on the CUDA cores")
+    ap.add_argument("--global-batch", action="store_true",
+                    help="use the multi-rank global-batch path (shard steps and the record "
+                         "all-gather) also on a single GPU")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.shape:
@@ -562,6 +732,8 @@ def main():
         args.workload = spec.name
     if args.impl == "reference":
         run_reference(args)
+    elif int(os.environ.get("WORLD_SIZE", "1")) > 1 or args.global_batch:
+        run_gpu_sharded(args)
     else:
         run_gpu(args)
 

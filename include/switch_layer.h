@@ -149,6 +149,62 @@ swl_status switch_layer_forward_host_io(int64_t T, int64_t d, int64_t d_ff, int6
  * SWL_ERR_CUDA if the synchronisation itself failed. */
 swl_status switch_layer_device_status(const void* workspace, void* stream);
 
+/* ---- One global batch sharded over ranks by contiguous token ranges ----
+ *
+ * Data parallelism over the tokens of ONE batch: rank g of `world` ranks holds
+ * the g-th contiguous range of the batch's T_total tokens (rank order = token
+ * order) and a full copy of the weights.  Positions, the capacity cut and the
+ * aux loss are those of the unsharded batch: a token's position is the number
+ * of tokens of its expert on earlier ranks plus its position among this rank's
+ * tokens (the cumulative sum over the expert's column of the dispatch mask in
+ * token order, "The routing mechanics in detail"), C = ceil(cf * T_total / N),
+ * and f_i, P_i count the whole batch ("The loss formulation").  One exchange is
+ * needed: every rank's per-expert token counts and sums of p.  A forward pass is
+ * three steps on every rank:
+ *   1. switch_layer_forward_shard_begin: routing of the local tokens, and this
+ *      rank's exchange record (switch_layer_shard_record_bytes(N) bytes, a
+ *      multiple of 16: N int32 token counts, then N fp64 sums of p at the next
+ *      16-byte boundary);
+ *   2. the caller gathers the records of all ranks, in rank order, into one
+ *      device buffer of world * record bytes (an all-gather: NCCL
+ *      ncclAllGather, torch.distributed.all_gather_into_tensor);
+ *   3. switch_layer_forward_shard_end: offsets of earlier ranks, the capacity
+ *      cut, the aux loss (the same value on every rank), dispatch and the expert
+ *      FFN of the local kept tokens.
+ * Both calls take the local T and the same workspace (sized by
+ * switch_layer_workspace_size for the local T); expert_idx, gate and
+ * pos_in_expert written by step 1 are read and completed by step 3 (pos_in_expert
+ * holds in-block ranks in between and the global position after).  A record set
+ * whose counts do not add up to T_total, or to this rank's T, makes the device
+ * status SWL_ERR_DEVICE.  With world = 1 the result equals switch_layer_forward's. */
+
+/* Bytes of one rank's exchange record for N experts (0 for invalid N). */
+size_t switch_layer_shard_record_bytes(int64_t N);
+
+/* Step 1 of a sharded forward (see above).  T: this rank's tokens (may be 0),
+ * T_total >= T: tokens of the whole batch; x, W_r, b_r, expert_idx, gate,
+ * pos_in_expert as for switch_layer_forward; record: device, 16-byte aligned,
+ * switch_layer_shard_record_bytes(N) bytes, written by the call. */
+swl_status switch_layer_forward_shard_begin(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                            int dtype, int64_t T_total, const void* x,
+                                            const float* W_r, const float* b_r,
+                                            double capacity_factor, int32_t* expert_idx,
+                                            float* gate, int32_t* pos_in_expert, void* record,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream);
+
+/* Step 3 of a sharded forward.  rank in [0, world); gathered: device, 16-byte
+ * aligned, the world records in rank order; the remaining arguments as for
+ * switch_layer_forward, with the tensors of step 1. */
+swl_status switch_layer_forward_shard_end(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                          int dtype, int64_t T_total, int rank, int world,
+                                          const void* gathered, const void* x, const void* W1,
+                                          const void* b1, const void* W2, const void* b2,
+                                          double capacity_factor, void* out,
+                                          int32_t* expert_idx, float* gate,
+                                          int32_t* pos_in_expert, float* aux_loss,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of the fixed device scratch used by switch_layer_forward_noalloc. */
 #define SWL_NOALLOC_MAX_BYTES (64u << 20)
 
@@ -215,6 +271,20 @@ uint64_t switch_layer_launch_count(void);
 typedef enum swl_router_mode { SWL_ROUTER_TENSOR = 0, SWL_ROUTER_FFMA = 1 } swl_router_mode;
 swl_status switch_layer_set_router_mode(int mode);
 int switch_layer_router_mode(void);
+
+/* ---- Failure-path test hooks (process-wide; not for production use) ----
+ * Every wait inside the kernels (pipeline barriers, the expert FFN's wait for
+ * another CTA's hidden rows) gives up after a time limit, sets the device
+ * status to SWL_ERR_DEVICE and lets the kernel drain and return, so the CUDA
+ * context stays usable.  switch_layer_set_wait_limit_ns sets that limit (0
+ * restores the default of 2 s).  switch_layer_set_stall_test(1) makes the
+ * expert FFN wait for one GEMM1 epilogue warp more than token tile 0 has, a
+ * signal that never comes: the wait runs out after the limit and the call
+ * reports SWL_ERR_DEVICE through switch_layer_device_status (outputs of that
+ * call are undefined).  switch_layer_set_stall_test(0) (the default) turns it
+ * off; other values return SWL_ERR_INVALID_ARG. */
+swl_status switch_layer_set_wait_limit_ns(uint64_t ns);
+swl_status switch_layer_set_stall_test(int on);
 
 /* The kernels switch_layer_forward would launch for this shape on a GPU of
  * num_sms SMs, under the current router mode, without touching the device

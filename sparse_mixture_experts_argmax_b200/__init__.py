@@ -34,7 +34,9 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_stage_name", "switch_layer_launch_count",
            "switch_layer_forward_noalloc", "switch_layer_set_router_mode",
            "switch_layer_router_mode", "switch_layer_describe_plan",
-           "switch_layer_noalloc_status")
+           "switch_layer_noalloc_status", "switch_layer_shard_record_bytes",
+           "switch_layer_forward_shard_begin", "switch_layer_forward_shard_end",
+           "switch_layer_set_wait_limit_ns", "switch_layer_set_stall_test")
 SWL_ROUTER_TENSOR = 0
 SWL_ROUTER_FFMA = 1
 SWL_NOALLOC_MAX_BYTES = 64 << 20
@@ -97,6 +99,20 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_forward_noalloc.argtypes = _FWD_ARGS[:17] + [_vp, _vp]
     L.switch_layer_noalloc_status.restype = _i32
     L.switch_layer_noalloc_status.argtypes = [_vp]
+    L.switch_layer_set_wait_limit_ns.restype = _i32
+    L.switch_layer_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.switch_layer_set_stall_test.restype = _i32
+    L.switch_layer_set_stall_test.argtypes = [_i32]
+    L.switch_layer_shard_record_bytes.restype = _sz
+    L.switch_layer_shard_record_bytes.argtypes = [_i64]
+    L.switch_layer_forward_shard_begin.restype = _i32
+    L.switch_layer_forward_shard_begin.argtypes = [_i64, _i64, _i64, _i64, _i32, _i64,
+                                                   _vp, _vp, _vp, _dbl, _vp, _vp, _vp, _vp,
+                                                   _vp, _sz, _vp]
+    L.switch_layer_forward_shard_end.restype = _i32
+    L.switch_layer_forward_shard_end.argtypes = [_i64, _i64, _i64, _i64, _i32, _i64, _i32,
+                                                 _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dbl,
+                                                 _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     _lib = L
     return L
 
@@ -267,6 +283,61 @@ def switch_layer_describe_plan(T, d, d_ff, N, dtype: int, capacity_factor: float
     return out
 
 
+def switch_layer_set_wait_limit_ns(ns: int) -> None:
+    """Failure-path test hook: bound of every wait inside the kernels (0: 2 s)."""
+    _check(lib().switch_layer_set_wait_limit_ns(int(ns)), "set_wait_limit_ns")
+
+
+def switch_layer_set_stall_test(on: bool) -> None:
+    """Failure-path test hook: make the expert FFN's first GEMM2 wait run out."""
+    _check(lib().switch_layer_set_stall_test(1 if on else 0), "set_stall_test")
+
+
+def switch_layer_shard_record_bytes(N: int) -> int:
+    return int(lib().switch_layer_shard_record_bytes(N))
+
+
+def switch_layer_forward_shard_begin(x, W_r, capacity_factor, T_total, expert_idx, gate,
+                                     pos_in_expert, record, d_ff, b_r=None, workspace=None,
+                                     stream=None) -> None:
+    """Step 1 of a forward over one rank's token range of a global batch."""
+    T, d = x.shape
+    N = W_r.shape[0]
+    _require(x, "x")
+    _require(W_r, "W_r", torch.float32)
+    if b_r is not None:
+        _require(b_r, "b_r", torch.float32)
+    _require(record, "record", torch.uint8)
+    _require(workspace, "workspace", torch.uint8)
+    if record.numel() != switch_layer_shard_record_bytes(N):
+        raise ValueError("record must hold %d bytes" % switch_layer_shard_record_bytes(N))
+    _check(lib().switch_layer_forward_shard_begin(
+        T, d, d_ff, N, dtype_code(x.dtype), int(T_total), _ptr(x), _ptr(W_r), _ptr(b_r),
+        float(capacity_factor), _ptr(expert_idx), _ptr(gate), _ptr(pos_in_expert),
+        _ptr(record), _ptr(workspace), workspace.numel(), _stream_handle(stream)),
+        "forward_shard_begin")
+
+
+def switch_layer_forward_shard_end(x, W1, b1, W2, b2, capacity_factor, T_total, rank, world,
+                                   gathered, out, expert_idx, gate, pos_in_expert, aux_loss,
+                                   workspace=None, stream=None) -> None:
+    """Step 3 of a forward over one rank's token range of a global batch."""
+    T, d = x.shape
+    N, d_ff, _ = W1.shape
+    act = x.dtype
+    for t, n in ((x, "x"), (W1, "W1"), (b1, "b1"), (W2, "W2"), (b2, "b2"), (out, "out")):
+        _require(t, n, act)
+    _require(gathered, "gathered", torch.uint8)
+    _require(workspace, "workspace", torch.uint8)
+    if gathered.numel() != world * switch_layer_shard_record_bytes(N):
+        raise ValueError("gathered must hold world * record bytes")
+    _check(lib().switch_layer_forward_shard_end(
+        T, d, d_ff, N, dtype_code(act), int(T_total), int(rank), int(world), _ptr(gathered),
+        _ptr(x), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), float(capacity_factor), _ptr(out),
+        _ptr(expert_idx), _ptr(gate), _ptr(pos_in_expert), _ptr(aux_loss), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)), "forward_shard_end")
+
+
 # ---------------------------------------------------------------------------
 # convenience: allocate outputs + workspace with torch and run
 # ---------------------------------------------------------------------------
@@ -301,6 +372,37 @@ def forward(inputs: dict, capacity_factor: float, workspace: Optional[torch.Tens
                          capacity_factor, outputs["out"], outputs["expert_idx"], outputs["gate"],
                          outputs["pos_in_expert"], outputs["aux_loss"], b_r=inputs.get("b_r"),
                          workspace=workspace, stream=stream)
+    if check:
+        _check(switch_layer_device_status(workspace, stream), "device status")
+    return outputs
+
+
+def forward_shard(inputs: dict, capacity_factor: float, T_total: int, rank: int, world: int,
+                  exchange, workspace: Optional[torch.Tensor] = None,
+                  outputs: Optional[dict] = None, stream=None, check: bool = True) -> dict:
+    """One rank's part of a forward over a global batch: ``inputs`` holds this
+    rank's token range (x) and the full weights; ``exchange(record)`` returns
+    the records of all ranks in rank order (an all-gather)."""
+    x, W1 = inputs["x"], inputs["W1"]
+    T, d = x.shape
+    N, d_ff, _ = W1.shape
+    if workspace is None:
+        workspace = alloc_workspace(max(T, 1), d, d_ff, N, x.dtype, capacity_factor,
+                                    device=W1.device)
+    if outputs is None:
+        outputs = alloc_outputs(T, d, x.dtype, device=W1.device)
+    record = torch.empty(switch_layer_shard_record_bytes(N), dtype=torch.uint8,
+                         device=W1.device)
+    switch_layer_forward_shard_begin(x, inputs["W_r"], capacity_factor, T_total,
+                                     outputs["expert_idx"], outputs["gate"],
+                                     outputs["pos_in_expert"], record, d_ff,
+                                     b_r=inputs.get("b_r"), workspace=workspace, stream=stream)
+    gathered = exchange(record)
+    switch_layer_forward_shard_end(x, W1, inputs["b1"], inputs["W2"], inputs["b2"],
+                                   capacity_factor, T_total, rank, world, gathered,
+                                   outputs["out"], outputs["expert_idx"], outputs["gate"],
+                                   outputs["pos_in_expert"], outputs["aux_loss"],
+                                   workspace=workspace, stream=stream)
     if check:
         _check(switch_layer_device_status(workspace, stream), "device status")
     return outputs

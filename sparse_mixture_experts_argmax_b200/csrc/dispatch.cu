@@ -65,13 +65,18 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
   return r;
 }
 
+// record != nullptr (a shard of a global batch): the expert totals of this
+// rank's tokens also go to the exchange record (int32 counts, then fp64 sums
+// at record_psum_offset), and the expert-level part (capacity, bases, aux) is
+// left to shard_combine_kernel, which needs every rank's record.
 __global__ void __launch_bounds__(kScanThreads)
 dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict__ blk_psum,
                      int* __restrict__ blk_off, int* __restrict__ exp_count,
                      double* __restrict__ psum64, int* __restrict__ exp_rows,
                      int* __restrict__ exp_base, int* __restrict__ tile_prefix,
                      int* __restrict__ ready, float* __restrict__ aux_loss, WsHeader* hdr,
-                     int nblk, int N, int T, int C_eff, int tile_rows) {
+                     int nblk, int N, int T, int C_eff, int tile_rows,
+                     uint8_t* __restrict__ record, int record_psum_offset) {
   __shared__ int wc[kScanWarps][32];
   __shared__ double wp[kScanWarps][32];
   __shared__ int is_last;
@@ -134,8 +139,13 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
       for (int w = 0; w < kScanWarps; ++w) { tot += wc[w][lane]; ps += wp[w][lane]; }
       exp_count[e] = tot;
       psum64[e] = ps;
+      if (record != nullptr) {
+        reinterpret_cast<int*>(record)[e] = tot;
+        reinterpret_cast<double*>(record + record_psum_offset)[e] = ps;
+      }
     }
   }
+  if (record != nullptr) return;
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -200,9 +210,10 @@ template <int VEC>
 __global__ void __launch_bounds__(kGatherThreads)
 dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ expert_idx,
                        int* __restrict__ pos_in_expert, const int* __restrict__ blk_off,
-                       const int* __restrict__ exp_base, int* __restrict__ slot_token,
-                       uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out, int T, int N,
-                       int C_eff, int row_bytes, int tpb, int prefetch, WsHeader* hdr) {
+                       const int* __restrict__ exp_base, const int* __restrict__ exp_off,
+                       int* __restrict__ slot_token, uint8_t* __restrict__ xbuf,
+                       uint8_t* __restrict__ out, int T, int N, int C_eff, int row_bytes,
+                       int tpb, int prefetch, WsHeader* hdr) {
   using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
   pdl_trigger();
   pdl_wait();   // offsets come from the scan
@@ -227,12 +238,14 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
     return;
   }
   const int b = t / tpb;
-  const int pos = blk_off[(size_t)b * N + e] + rank;
+  // a shard of a global batch: the tokens of earlier ranks come first
+  const int off = exp_off != nullptr ? exp_off[e] : 0;
+  const int pos = off + blk_off[(size_t)b * N + e] + rank;
   const int base = exp_base[e];
   __syncwarp();
   if (lane == 0) pos_in_expert[t] = pos;
   if (pos < C_eff) {
-    const int row = base + pos;
+    const int row = base + pos - off;
     if (lane == 0) slot_token[row] = t;
     V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
     if (in_regs) {
@@ -430,6 +443,109 @@ dispatch_fused_kernel(const uint8_t* __restrict__ x, const int* __restrict__ exp
   }
 }
 
+constexpr int kCombineThreads = 512;
+constexpr int kCombineWarps = kCombineThreads / 32;
+
+// A global batch sharded over `world` ranks by contiguous token ranges, rank
+// order = token order.  From every rank's exchange record (expert totals of its
+// tokens and their sums of p), one CTA computes for this rank:
+//   exp_off[e]   tokens of expert e on earlier ranks, so that a local token's
+//                position is exp_off[e] + its position among this rank's tokens
+//                (the cumulative sum over the expert's column in global token
+//                order, "The routing mechanics in detail");
+//   exp_rows[e]  this rank's kept tokens of e: those whose global position is
+//                below C, min(count, max(0, C - exp_off[e]));
+//   packed bases, the GEMM tile prefix and the FFN's per-call state;
+//   the aux loss N * sum_i f_i P_i over the whole batch, with each expert's
+//   totals summed in rank order (every rank computes the same value).
+// C_cap = min(C, T_total).  A record set whose counts do not add up to
+// T_total (ranks disagreeing on the batch) or to this rank's T raises
+// kDevIndexOutOfRange; the rows are then clamped to stay in range.
+__global__ void __launch_bounds__(kCombineThreads)
+shard_combine_kernel(const uint8_t* __restrict__ gathered, int record_bytes,
+                     int record_psum_offset, int rank, int world, int N, int T_local,
+                     int T_total, int C_cap, int tile_rows,
+                     const int* __restrict__ exp_count, int* __restrict__ exp_off,
+                     int* __restrict__ exp_rows, int* __restrict__ exp_base,
+                     int* __restrict__ tile_prefix, int* __restrict__ ready,
+                     float* __restrict__ aux_loss, WsHeader* hdr) {
+  __shared__ int s_warp[kCombineWarps];
+  __shared__ int s_tot_rows, s_tot_tiles;
+  __shared__ double s_aux[kCombineWarps];
+  __shared__ long long s_cnt[2][kCombineWarps];
+  pdl_trigger();
+  pdl_wait();   // the records were gathered after the local scan
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = (N + kCombineThreads - 1) / kCombineThreads;
+  const int e0 = threadIdx.x * chunk, e1 = min(N, e0 + chunk);
+  int rows = 0, tiles = 0;
+  long long all_tok = 0, my_tok = 0;
+  double aux = 0.0;
+  bool consistent = true;
+  for (int i = e0; i < e1; ++i) {
+    long long before = 0, tot = 0;
+    int mine = 0;
+    double ps = 0.0;
+    for (int g = 0; g < world; ++g) {
+      const uint8_t* rec = gathered + static_cast<size_t>(g) * record_bytes;
+      const int c = reinterpret_cast<const int*>(rec)[i];
+      tot += c;
+      if (g < rank) before += c;
+      if (g == rank) mine = c;
+      ps += reinterpret_cast<const double*>(rec + record_psum_offset)[i];
+    }
+    // this rank's own count comes from its scan (the record should repeat it):
+    // the kept rows then never exceed the rows this rank holds
+    const int own = exp_count != nullptr ? exp_count[i] : 0;   // null: no local tokens
+    consistent = consistent && own == mine && before >= 0 && before <= T_total;
+    const long long room = static_cast<long long>(C_cap) - before;
+    const int m = static_cast<int>(max(0ll, min(static_cast<long long>(own), room)));
+    rows += m;
+    tiles += (m + tile_rows - 1) / tile_rows;
+    aux += static_cast<double>(tot) * ps;
+    all_tok += tot;
+    my_tok += own;
+    exp_off[i] = static_cast<int>(min(max(before, 0ll), static_cast<long long>(T_total)));
+    exp_rows[i] = m;
+  }
+  if (!consistent) atomicExch(&hdr->err, kDevIndexOutOfRange);
+  int base_rows = block_excl_scan(rows, s_warp, &s_tot_rows);
+  int base_tiles = block_excl_scan(tiles, s_warp, &s_tot_tiles);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    aux += __shfl_xor_sync(0xffffffffu, aux, off);
+    all_tok += __shfl_xor_sync(0xffffffffu, all_tok, off);
+    my_tok += __shfl_xor_sync(0xffffffffu, my_tok, off);
+  }
+  if (lane == 0) {
+    s_aux[warp] = aux;
+    s_cnt[0][warp] = all_tok;
+    s_cnt[1][warp] = my_tok;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < s_tot_tiles; i += kCombineThreads) ready[i] = 0;
+  if (threadIdx.x == 0) {
+    double a = 0.0;
+    long long at = 0, mt = 0;
+    for (int w = 0; w < kCombineWarps; ++w) {
+      a += s_aux[w];
+      at += s_cnt[0][w];
+      mt += s_cnt[1][w];
+    }
+    if (at != T_total || mt != T_local) atomicExch(&hdr->err, kDevIndexOutOfRange);
+    tile_prefix[N] = s_tot_tiles;
+    hdr->next_tile = 0u;
+    *aux_loss = (float)((double)N * a / ((double)T_total * (double)T_total));
+  }
+  for (int i = e0; i < e1; ++i) {
+    const int m = exp_rows[i];
+    exp_base[i] = base_rows;
+    tile_prefix[i] = base_tiles;
+    base_rows += m;
+    base_tiles += (m + tile_rows - 1) / tile_rows;
+  }
+}
+
 }  // namespace
 
 bool dispatch_fused_ok(const Shape& s) {
@@ -457,12 +573,34 @@ cudaError_t launch_dispatch_fused(const Shape& s, const Workspace& ws, const voi
 }
 
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
-                                 cudaStream_t stream) {
+                                 void* record, cudaStream_t stream) {
   const int grid = (int)((s.N + 31) / 32);
   const cudaError_t e = launch_dependent(
       dispatch_scan_kernel, dim3(grid), dim3(kScanThreads), 0, stream, ws.blk_count, ws.blk_psum,
       ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base, ws.tile_prefix, ws.ready,
-      aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows);
+      aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows,
+      static_cast<uint8_t*>(record), (int)shard_record_psum_offset(s.N));
+  count_launch();
+  return e;
+}
+
+size_t shard_record_psum_offset(int64_t N) {
+  return (static_cast<size_t>(N) * 4 + 15) / 16 * 16;
+}
+
+size_t shard_record_bytes(int64_t N) {   // a multiple of 16, so records can sit back to back
+  return (shard_record_psum_offset(N) + static_cast<size_t>(N) * 8 + 15) / 16 * 16;
+}
+
+cudaError_t launch_shard_combine(const Shape& s, const Workspace& ws, const void* gathered,
+                                 int rank, int world, float* aux_loss, cudaStream_t stream) {
+  const cudaError_t e = launch_dependent(
+      shard_combine_kernel, dim3(1), dim3(kCombineThreads), 0, stream,
+      static_cast<const uint8_t*>(gathered), (int)shard_record_bytes(s.N),
+      (int)shard_record_psum_offset(s.N), rank, world, (int)s.N, (int)s.T, (int)s.T_total,
+      (int)s.C_cmp, s.tile_rows, s.T > 0 ? static_cast<const int*>(ws.exp_count) : nullptr,
+      ws.exp_off, ws.exp_rows,
+      ws.exp_base, ws.tile_prefix, ws.ready, aux_loss, ws.hdr);
   count_launch();
   return e;
 }
@@ -479,9 +617,10 @@ cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const vo
   const cudaError_t e = launch_dependent(
       vec16 ? dispatch_gather_kernel<16> : dispatch_gather_kernel<4>, dim3(grid),
       dim3(kGatherThreads), 0, stream, static_cast<const uint8_t*>(x), expert_idx, pos_in_expert,
-      static_cast<const int*>(ws.blk_off), static_cast<const int*>(ws.exp_base), ws.slot_token,
+      static_cast<const int*>(ws.blk_off), static_cast<const int*>(ws.exp_base),
+      static_cast<const int*>(s.sharded ? ws.exp_off : nullptr), ws.slot_token,
       static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T, (int)s.N,
-      (int)s.C_eff, row_bytes, s.tpb, s.T * (int64_t)row_bytes <= (int64_t{48} << 20) ? 1 : 0,
+      (int)s.C_cmp, row_bytes, s.tpb, s.T * (int64_t)row_bytes <= (int64_t{48} << 20) ? 1 : 0,
       ws.hdr);
   count_launch();
   return e;

@@ -77,6 +77,9 @@ struct FfnArgs {
   int* ready;                  // [token tiles] GEMM1 epilogue warps finished (zeroed by the scan)
   unsigned int* next_tile;     // work counter (zeroed by the scan)
   int* err;
+  unsigned long long wait_ns;  // bound of every wait
+  int stall_test;  // 1: token tile 0's GEMM2 readiness target is one warp too high (the
+                   // wait runs out: a test of the failure path)
   int num_experts;
   int cache_prefix;   // 1: the scheduler keeps the tile prefix in shared memory
   int bn;         // token rows per tile (multiple of 16, <= 256)
@@ -229,11 +232,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     if (lane == 0) {
       for (int i = 0;; ++i) {
         const int slot = i % kTileRing;
-        if (i > 0 && !ptx::mbar_wait(take_bar, static_cast<uint32_t>(i - 1) & 1u, abort_flag)) {
+        if (i > 0 && !ptx::mbar_wait(take_bar, static_cast<uint32_t>(i - 1) & 1u, abort_flag, args.wait_ns)) {
           fail();
           break;
         }
-        if (!ptx::mbar_wait(&tile_empty[slot], ((i / kTileRing) & 1) ^ 1u, abort_flag)) {
+        if (!ptx::mbar_wait(&tile_empty[slot], ((i / kTileRing) & 1) ^ 1u, abort_flag, args.wait_ns)) {
           fail();
           break;
         }
@@ -252,11 +255,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           ts.row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
           if (c.phase == 1) {
             // hbuf rows of token tile g: every GEMM1 epilogue warp of g has stored them
-            const int target = kEpiWarps * args.ph[0].m_tiles;
+            const int target = kEpiWarps * args.ph[0].m_tiles + (args.stall_test && c.g == 0);
             bool ready = ld_acquire(args.ready + c.g) >= target;
             const uint64_t t0 = ptx::globaltimer_ns();
             while (!ready) {
-              if (*abort_flag || ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs) break;
+              if (*abort_flag || ptx::globaltimer_ns() - t0 > args.wait_ns) break;
               ready = ld_acquire(args.ready + c.g) >= target;
             }
             if (!ready) {
@@ -283,7 +286,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int slot = i % kTileRing;
-        if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) {
+        if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag, args.wait_ns)) {
           fail();
           break;
         }
@@ -299,7 +302,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         const int arow = ts.e * P.M + ts.mt * kBM;
         const int brow = ts.row0;
         for (int kb = 0; kb < P.k_blocks; ++kb) {
-          if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag)) { fail(); ok = false; break; }
+          if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
           ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
           ptx::tma_load_2d(smem_a + stage * kABytes, tA, &full_bar[stage], kb * kBK, arow, pol_w);
           ptx::tma_load_2d(smem_b + stage * b_bytes, tB, &full_bar[stage], kb * kBK, brow, pol_x);
@@ -312,7 +315,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       for (int s = 0; s < stages; ++s) {
         if (issued & (1u << s)) {
           volatile int never = 0;
-          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never)) {
+          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never, args.wait_ns)) {
             atomicExch(args.err, kDevPipelineTimeout);
           }
         }
@@ -329,17 +332,17 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int slot = i % kTileRing;
-        if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag)) { fail(); break; }
+        if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag, args.wait_ns)) { fail(); break; }
         const TileSlot ts = tile_ring[slot];
         if (ts.t < 0) break;
         const PhaseArgs& P = args.ph[ts.phase];
         const uint32_t n_mma = static_cast<uint32_t>((ts.rows + 15) & ~15);
         const uint32_t idesc = ptx::umma_idesc_bf16_f32(n_mma);
-        if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { fail(); break; }
+        if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag, args.wait_ns)) { fail(); break; }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * acc_cols);
         for (int kb = 0; kb < P.k_blocks; ++kb) {
-          if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag)) { fail(); ok = false; break; }
+          if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(smem_a + stage * kABytes);
           const uint32_t b_addr = ptx::smem_u32(smem_b + stage * b_bytes);
@@ -359,7 +362,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       // drain: all MMAs issued by this thread complete before TMEM is released
       ptx::umma_commit(drain_bar);
       volatile int never = 0;
-      if (!ptx::mbar_wait(drain_bar, 0u, &never)) atomicExch(args.err, kDevPipelineTimeout);
+      if (!ptx::mbar_wait(drain_bar, 0u, &never, args.wait_ns)) atomicExch(args.err, kDevPipelineTimeout);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -395,7 +398,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       publish_if_blocked(&tile_full[slot], tpar);
       // every wait result is made warp-uniform: the warp then leaves together (the
       // TMEM loads below are warp-collective)
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tile_full[slot], tpar, abort_flag))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tile_full[slot], tpar, abort_flag, args.wait_ns))) {
         fail();
         break;
       }
@@ -428,7 +431,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         gs[k] = (P.mode == 1 && col < rows) ? __ldg(args.gate + dsts[k]) : 1.f;
       }
       publish_if_blocked(&tfull_bar[acc], aph);
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&tfull_bar[acc], aph, abort_flag, args.wait_ns))) {
         fail();
         break;
       }
@@ -520,6 +523,8 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.ready = ws.ready;
   a.next_tile = &ws.hdr->next_tile;
   a.err = &ws.hdr->err;
+  a.wait_ns = wait_limit_ns();
+  a.stall_test = stall_test_enabled() ? 1 : 0;
   a.num_experts = static_cast<int>(s.N);
   a.bn = s.tile_rows;
   a.num_acc = a.bn <= kTmemCols / kMaxAcc ? kMaxAcc : 2;

@@ -38,6 +38,7 @@ struct Workspace {
   int* exp_count;       // [N] tokens whose argmax is e (before capacity)
   int* exp_rows;        // [N] kept rows m_e = min(count_e, C)
   int* exp_base;        // [N] first packed row of expert e
+  int* exp_off;         // [N] shard of a global batch: tokens of e on earlier ranks
   int* tile_prefix;     // [N+1] prefix over experts of ceil(m_e / tile_rows)
   double* psum64;       // [N] sum over all tokens of p_{t,e}
   int* slot_token;      // [T] packed row -> token
@@ -58,8 +59,11 @@ struct Workspace {
 struct Shape {
   int64_t T, d, d_ff, N;
   int dtype;      // 0 = fp32, 1 = bf16
-  int64_t C;      // capacity (formula value)
-  int64_t C_eff;  // min(C, T): rows an expert can actually keep
+  int64_t C;      // capacity (formula value, from the batch's T_total tokens)
+  int64_t C_eff;  // min(C, T): rows an expert can actually keep on this rank
+  int64_t T_total;  // tokens of the whole batch (T unless a shard of a global batch)
+  int64_t C_cmp;  // min(C, T_total): a token is kept iff its position is below it
+  int sharded;    // 1: a shard of a global batch (positions offset by earlier ranks)
   int router_path;  // RouterPath
   int tpb;        // tokens per block of the softmax / rank / gather stages (<= kTokensPerBlock)
   int nblk;       // ceil(T / tpb)
@@ -122,8 +126,18 @@ int softmax_variant(const Shape& s);
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);
+// record != nullptr: a shard of a global batch; the expert totals go to the
+// exchange record and the expert-level part waits for launch_shard_combine.
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
-                                 cudaStream_t stream);
+                                 void* record, cudaStream_t stream);
+// Exchange record of one rank: int32 counts [N], then fp64 sums of p [N] at a
+// 16-byte aligned offset.
+size_t shard_record_psum_offset(int64_t N);
+size_t shard_record_bytes(int64_t N);
+// Offsets of earlier ranks, kept rows, bases, tile prefix and the global aux
+// loss from the records of all `world` ranks (gathered in rank order).
+cudaError_t launch_shard_combine(const Shape& s, const Workspace& ws, const void* gathered,
+                                 int rank, int world, float* aux_loss, cudaStream_t stream);
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
                                    const int* expert_idx, int* pos_in_expert, void* out,
                                    cudaStream_t stream);
@@ -155,6 +169,10 @@ constexpr int kF32TileRows = 32;
 
 // Number of kernel launches issued by this library since load.
 void count_launch(int n = 1);
+// Bound of every wait inside the kernels, in ns (switch_layer_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+// Failure-path test of the expert FFN (switch_layer_set_stall_test).
+bool stall_test_enabled();
 
 // Programmatic dependent launch: a kernel launched with launch_dependent() may
 // start while the previous kernel on the stream is still finishing; it must call

@@ -444,7 +444,7 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
                              int N, int tpb, int nblk, int* __restrict__ expert_idx,
                              float* __restrict__ gate, int* __restrict__ local_rank,
                              int* __restrict__ blk_count, float* __restrict__ blk_psum,
-                             WsHeader* hdr) {
+                             WsHeader* hdr, unsigned long long wait_ns) {
   constexpr int VPT = (V4 * 32 + kStreamThreads - 1) / kStreamThreads;   // pass-B float4 / thread
   extern __shared__ uint8_t smem_raw[];
   float* buf = reinterpret_cast<float*>(
@@ -499,7 +499,8 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
         issue_next((ci + kStreamBufs - 1) % kStreamBufs);
       }
       volatile int* ab = &s_abort;
-      const bool ok = ptx::mbar_wait(&full[slot], static_cast<uint32_t>(ci / kStreamBufs) & 1u, ab);
+      const bool ok = ptx::mbar_wait(&full[slot], static_cast<uint32_t>(ci / kStreamBufs) & 1u, ab,
+                                     wait_ns);
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
@@ -615,7 +616,8 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
     if (tid == 0) {
       volatile int never = 0;
       for (int j = ci; j < issued; ++j)
-        ptx::mbar_wait(&full[j % kStreamBufs], static_cast<uint32_t>(j / kStreamBufs) & 1u, &never);
+        ptx::mbar_wait(&full[j % kStreamBufs], static_cast<uint32_t>(j / kStreamBufs) & 1u, &never,
+                       wait_ns);
     }
     __syncthreads();
   }
@@ -1138,7 +1140,7 @@ cudaError_t launch_stream_t(const Shape& s, const Workspace& ws, const float* b_
   return launch_dependent(router_softmax_stream_kernel<V4>, dim3(grid), dim3(kStreamThreads),
                           smem, stream, static_cast<const float*>(ws.logits), b_r, (int)s.T,
                           (int)s.N, s.tpb, s.nblk, expert_idx, gate, local_rank, ws.blk_count,
-                          ws.blk_psum, ws.hdr);
+                          ws.blk_psum, ws.hdr, wait_limit_ns());
 }
 
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,

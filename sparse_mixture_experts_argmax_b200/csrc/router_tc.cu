@@ -79,6 +79,7 @@ struct TcArgs {
   int* blk_count;
   float* blk_psum;
   WsHeader* hdr;
+  unsigned long long wait_ns;   // bound of every wait
   const uint8_t* pf;      // bytes fetched into L2 once this CTA's loads have landed
   size_t pf_bytes;        // (the expert weights the FFN streams first; 0: none)
 };
@@ -217,7 +218,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         uint8_t* st = smem + s * C::kStage;
         const int kc = (kb0 + i) * kBK;
         if (i >= first) {
-          if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) {
+          if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, a.wait_ns)) {
             fail();
             break;
           }
@@ -235,7 +236,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       for (int s = 0; s < stages; ++s) {
         if (issued & (1u << s)) {
           volatile int never = 0;
-          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never))
+          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never, a.wait_ns))
             atomicExch(&a.hdr->err, kDevPipelineTimeout);
         }
       }
@@ -252,7 +253,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t ph = static_cast<uint32_t>(i / stages) & 1u;
-        if (!ptx::mbar_wait(&full_bar[s], ph, abort_flag)) {
+        if (!ptx::mbar_wait(&full_bar[s], ph, abort_flag, a.wait_ns)) {
           fail();
           ok = false;
           break;
@@ -279,7 +280,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       // all MMAs of this thread complete before TMEM is released
       ptx::umma_commit(drain_bar);
       volatile int never = 0;
-      if (!ptx::mbar_wait(drain_bar, 0u, &never)) atomicExch(&a.hdr->err, kDevPipelineTimeout);
+      if (!ptx::mbar_wait(drain_bar, 0u, &never, a.wait_ns)) atomicExch(&a.hdr->err, kDevPipelineTimeout);
     }
     __syncwarp();
   } else if (warp == 3) {
@@ -293,7 +294,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     // ------------------------------------------------------------ TMEM epilogue
     bool have = false;
     if (nk > 0) {
-      const bool got = ptx::mbar_wait(accf_bar, 0u, abort_flag);
+      const bool got = ptx::mbar_wait(accf_bar, 0u, abort_flag, a.wait_ns);
       have = __all_sync(0xffffffffu, got);
       if (!have && lane == 0) fail();
     }
@@ -466,6 +467,7 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
   a.blk_count = ws.blk_count;
   a.blk_psum = ws.blk_psum;
   a.hdr = ws.hdr;
+  a.wait_ns = wait_limit_ns();
   const unsigned t_tiles = static_cast<unsigned>((s.T + kBM - 1) / kBM);
   const int stages = tc_stages<NP>(s, kWide, num_sms);
   // the logits tile reuses the stage memory

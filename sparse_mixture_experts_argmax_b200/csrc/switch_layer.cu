@@ -31,7 +31,11 @@ namespace swl {
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<int> g_router_mode{SWL_ROUTER_TENSOR};   // switch_layer_set_router_mode
+static std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+static std::atomic<int> g_stall_test{0};
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(); }
+bool stall_test_enabled() { return g_stall_test.load() != 0; }
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -57,6 +61,7 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.exp_count = reinterpret_cast<int*>(take(N * 4));
   w.exp_rows = reinterpret_cast<int*>(take(N * 4));
   w.exp_base = reinterpret_cast<int*>(take(N * 4));
+  w.exp_off = reinterpret_cast<int*>(take(N * 4));
   w.tile_prefix = reinterpret_cast<int*>(take((N + 1) * 4));
   w.psum64 = reinterpret_cast<double*>(take(N * 8));
   w.slot_token = reinterpret_cast<int*>(take(T * 4));
@@ -145,6 +150,9 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->dtype = dtype;
   s->C = switch_layer_capacity(T, N, cf);
   s->C_eff = s->C < T ? s->C : T;
+  s->T_total = T;
+  s->C_cmp = s->C_eff;
+  s->sharded = 0;
   // the tensor-core router serves bf16 layers unless the FFMA router was chosen
   const bool tensor_router = dtype == SWL_BF16 && g_router_mode.load() == SWL_ROUTER_TENSOR;
   const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0);
@@ -154,6 +162,84 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->tpb = rp.tpb;
   s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
+  return SWL_OK;
+}
+
+// Shape of one rank's shard of a global batch of T_total tokens: the kernels
+// run over the T local tokens, the capacity comes from T_total.
+static swl_status make_shard_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                   int64_t T_total, double cf, Shape* s) {
+  swl_status st = make_shape(T, d, d_ff, N, dtype, cf, s);
+  if (st != SWL_OK) return st;
+  if (T_total < T) return SWL_ERR_INVALID_ARG;
+  if (T_total > INT32_MAX / 2) return SWL_ERR_UNSUPPORTED;
+  s->T_total = T_total;
+  s->C = switch_layer_capacity(T_total, N, cf);
+  s->C_eff = s->C < T ? s->C : T;
+  s->C_cmp = s->C < T_total ? s->C : T_total;
+  s->sharded = 1;
+  s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
+  return SWL_OK;
+}
+
+// Stages 0-1: router logits, softmax, argmax, gate, block ranks and statistics.
+// rec(k) records stage event k (a no-op without events).
+template <typename Rec>
+static swl_status run_routing(const Shape& s, const Workspace& ws, const void* x,
+                              const float* W_r, const void* W1, int32_t* expert_idx, float* gate,
+                              int32_t* pos_in_expert, const float* b_r, cudaStream_t stream,
+                              Rec& rec) {
+  if (s.router_path == kRouterTC || s.router_path == kRouterTCWide) {
+    CUtensorMap tx, tw;
+    if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
+        !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N, router_tc_padded_experts(s.N)))
+      return SWL_ERR_CUDA;
+    // the FFN's first tiles stream W1 from its start: fetch a slice into L2 while
+    // routing and dispatch run, when the router is a single wave of CTAs (with a
+    // second wave the prefetch would compete with that wave's loads)
+    const size_t w1_bytes = static_cast<size_t>(s.N) * s.d_ff * s.d * 2;
+    const int sms = num_sms_current();
+    const int64_t router_ctas = s.router_path == kRouterTC ? (s.T + 127) / 128 * s.ksplit_eff : 0;
+    const size_t pf = (W1 != nullptr && router_ctas > 0 && router_ctas <= sms)
+                          ? (w1_bytes < kL2PrefetchBytes ? w1_bytes : kL2PrefetchBytes)
+                          : 0;
+    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, W1, pf, sms,
+                         stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+  } else if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert,
+                                  stream) != cudaSuccess) {
+    return SWL_ERR_CUDA;
+  }
+  if (!rec(1)) return SWL_ERR_CUDA;
+  if (s.N > kFusedRouterMaxN &&
+      launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  if (!rec(2)) return SWL_ERR_CUDA;
+  return SWL_OK;
+}
+
+// Stage 4: both expert GEMMs over the packed rows, combine in the epilogue.
+static swl_status run_ffn(const Shape& s, const Workspace& ws, const void* W1, const void* b1,
+                          const void* W2, const void* b2, const float* gate, void* out,
+                          cudaStream_t stream) {
+  if (s.dtype == SWL_BF16) {
+    const int sms = num_sms_current();
+    if (sms <= 0) return SWL_ERR_CUDA;
+    CUtensorMap a1, b1m, a2, b2m;
+    if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff, 128) ||
+        !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T, s.tile_rows) ||
+        !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
+        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T, s.tile_rows))
+      return SWL_ERR_CUDA;
+    if (launch_expert_ffn_bf16(s, ws, a1, b1m, a2, b2m, b1, b2, gate, out, sms, stream) !=
+        cudaSuccess)
+      return SWL_ERR_CUDA;
+  } else {
+    if (launch_expert_gemm_f32(s, ws, 0, W1, b1, gate, ws.hbuf, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (launch_expert_gemm_f32(s, ws, 1, W2, b2, gate, out, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+  }
   return SWL_OK;
 }
 
@@ -177,32 +263,9 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
                       : cudaEventRecord(e, stream)) == cudaSuccess;
   };
   if (!rec(0)) return SWL_ERR_CUDA;
-  if (s.router_path == kRouterTC || s.router_path == kRouterTCWide) {
-    CUtensorMap tx, tw;
-    if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
-        !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N, router_tc_padded_experts(s.N)))
-      return SWL_ERR_CUDA;
-    // the FFN's first tiles stream W1 from its start: fetch a slice into L2 while
-    // routing and dispatch run, when the router is a single wave of CTAs (with a
-    // second wave the prefetch would compete with that wave's loads)
-    const size_t w1_bytes = static_cast<size_t>(s.N) * s.d_ff * s.d * 2;
-    const int sms = num_sms_current();
-    const int64_t router_ctas = s.router_path == kRouterTC ? (s.T + 127) / 128 * s.ksplit_eff : 0;
-    const size_t pf = (router_ctas > 0 && router_ctas <= sms)
-                          ? (w1_bytes < kL2PrefetchBytes ? w1_bytes : kL2PrefetchBytes)
-                          : 0;
-    if (launch_router_tc(s, ws, W_r, tx, tw, b_r, expert_idx, gate, pos_in_expert, W1, pf, sms,
-                         stream) != cudaSuccess)
-      return SWL_ERR_CUDA;
-  } else if (launch_router_logits(s, ws, x, W_r, b_r, expert_idx, gate, pos_in_expert,
-                                  stream) != cudaSuccess) {
-    return SWL_ERR_CUDA;
-  }
-  if (!rec(1)) return SWL_ERR_CUDA;
-  if (s.N > kFusedRouterMaxN &&
-      launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
-    return SWL_ERR_CUDA;
-  if (!rec(2)) return SWL_ERR_CUDA;
+  swl_status st = run_routing(s, ws, x, W_r, W1, expert_idx, gate, pos_in_expert, b_r, stream,
+                              rec);
+  if (st != SWL_OK) return st;
   if (dispatch_fused_ok(s)) {
     // one launch for scan and gather (timed in the scan stage; the gather stage is empty)
     if (launch_dispatch_fused(s, ws, x, expert_idx, pos_in_expert, out, aux_loss, stream) !=
@@ -210,30 +273,15 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
       return SWL_ERR_CUDA;
     if (!rec(3)) return SWL_ERR_CUDA;
   } else {
-    if (launch_dispatch_scan(s, ws, aux_loss, stream) != cudaSuccess) return SWL_ERR_CUDA;
+    if (launch_dispatch_scan(s, ws, aux_loss, nullptr, stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
     if (!rec(3)) return SWL_ERR_CUDA;
     if (launch_dispatch_gather(s, ws, x, expert_idx, pos_in_expert, out, stream) != cudaSuccess)
       return SWL_ERR_CUDA;
   }
   if (!rec(4)) return SWL_ERR_CUDA;
-  if (s.dtype == SWL_BF16) {
-    const int sms = num_sms_current();
-    if (sms <= 0) return SWL_ERR_CUDA;
-    CUtensorMap a1, b1m, a2, b2m;
-    if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff, 128) ||
-        !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T, s.tile_rows) ||
-        !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
-        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T, s.tile_rows))
-      return SWL_ERR_CUDA;
-    if (launch_expert_ffn_bf16(s, ws, a1, b1m, a2, b2m, b1, b2, gate, out, sms, stream) !=
-        cudaSuccess)
-      return SWL_ERR_CUDA;
-  } else {
-    if (launch_expert_gemm_f32(s, ws, 0, W1, b1, gate, ws.hbuf, stream) != cudaSuccess)
-      return SWL_ERR_CUDA;
-    if (launch_expert_gemm_f32(s, ws, 1, W2, b2, gate, out, stream) != cudaSuccess)
-      return SWL_ERR_CUDA;
-  }
+  st = run_ffn(s, ws, W1, b1, W2, b2, gate, out, stream);
+  if (st != SWL_OK) return st;
   if (!rec(5)) return SWL_ERR_CUDA;
   return SWL_OK;
 }
@@ -454,6 +502,17 @@ swl_status switch_layer_set_router_mode(int mode) {
 
 int switch_layer_router_mode(void) { return swl::g_router_mode.load(); }
 
+swl_status switch_layer_set_wait_limit_ns(uint64_t ns) {
+  swl::g_wait_limit_ns.store(ns == 0 ? 2000000000ull : ns);
+  return SWL_OK;
+}
+
+swl_status switch_layer_set_stall_test(int on) {
+  if (on != 0 && on != 1) return SWL_ERR_INVALID_ARG;
+  swl::g_stall_test.store(on);
+  return SWL_OK;
+}
+
 swl_status switch_layer_describe_plan(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                       double capacity_factor, int num_sms, char* buf,
                                       size_t len) {
@@ -503,6 +562,87 @@ swl_status switch_layer_forward_noalloc(int64_t T, int64_t d, int64_t d_ff, int6
   return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
                       expert_idx, gate, pos_in_expert, aux_loss, b_r, scratch,
                       static_cast<size_t>(SWL_NOALLOC_MAX_BYTES), stream, nullptr);
+}
+
+size_t switch_layer_shard_record_bytes(int64_t N) {
+  return N > 0 && N <= kMaxExperts ? shard_record_bytes(N) : 0;
+}
+
+swl_status switch_layer_forward_shard_begin(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                            int dtype, int64_t T_total, const void* x,
+                                            const float* W_r, const float* b_r,
+                                            double capacity_factor, int32_t* expert_idx,
+                                            float* gate, int32_t* pos_in_expert, void* record,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream_v) {
+  Shape s;
+  swl_status st = make_shard_shape(T, d, d_ff, N, dtype, T_total, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (!W_r || !record || !workspace) return SWL_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !expert_idx || !gate || !pos_in_expert)) return SWL_ERR_INVALID_ARG;
+  const bool tc = s.router_path == kRouterTC || s.router_path == kRouterTCWide;
+  if (!aligned(workspace, 256) || !aligned(record, 16) || !aligned(W_r, tc ? 16 : 4) ||
+      !aligned(x, dtype == SWL_BF16 ? 16 : 4) || !aligned(expert_idx, 4) || !aligned(gate, 4) ||
+      !aligned(pos_in_expert, 4))
+    return SWL_ERR_UNSUPPORTED;
+  if (workspace_bytes < workspace_layout(s, false, 0, nullptr)) return SWL_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (T == 0) {   // no tokens here: an all-zero record
+    return cudaMemsetAsync(record, 0, shard_record_bytes(N), stream) == cudaSuccess
+               ? SWL_OK
+               : SWL_ERR_CUDA;
+  }
+  Workspace ws;
+  workspace_layout(s, false, reinterpret_cast<uintptr_t>(workspace), &ws);
+  auto no_events = [](int) { return true; };
+  st = run_routing(s, ws, x, W_r, nullptr, expert_idx, gate, pos_in_expert, b_r, stream,
+                   no_events);
+  if (st != SWL_OK) return st;
+  return launch_dispatch_scan(s, ws, nullptr, record, stream) == cudaSuccess ? SWL_OK
+                                                                             : SWL_ERR_CUDA;
+}
+
+swl_status switch_layer_forward_shard_end(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                          int dtype, int64_t T_total, int rank, int world,
+                                          const void* gathered, const void* x, const void* W1,
+                                          const void* b1, const void* W2, const void* b2,
+                                          double capacity_factor, void* out,
+                                          int32_t* expert_idx, float* gate,
+                                          int32_t* pos_in_expert, float* aux_loss,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* stream_v) {
+  Shape s;
+  swl_status st = make_shard_shape(T, d, d_ff, N, dtype, T_total, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (world < 1 || rank < 0 || rank >= world) return SWL_ERR_INVALID_ARG;
+  if (!gathered || !W1 || !b1 || !W2 || !b2 || !aux_loss || !workspace)
+    return SWL_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out || !expert_idx || !gate || !pos_in_expert)) return SWL_ERR_INVALID_ARG;
+  const uintptr_t a = dtype == SWL_BF16 ? 16 : 4;
+  if (!aligned(workspace, 256) || !aligned(gathered, 16) || !aligned(W1, a) ||
+      !aligned(W2, a) || !aligned(b1, dtype == SWL_BF16 ? 2 : 4) ||
+      !aligned(b2, dtype == SWL_BF16 ? 2 : 4) || !aligned(x, a) || !aligned(out, a) ||
+      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(pos_in_expert, 4) ||
+      !aligned(aux_loss, 4))
+    return SWL_ERR_UNSUPPORTED;
+  if (workspace_bytes < workspace_layout(s, false, 0, nullptr)) return SWL_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (T_total == 0) {
+    if (cudaMemsetAsync(aux_loss, 0, sizeof(float), stream) != cudaSuccess ||
+        cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream) != cudaSuccess)
+      return SWL_ERR_CUDA;
+    return SWL_OK;
+  }
+  Workspace ws;
+  workspace_layout(s, false, reinterpret_cast<uintptr_t>(workspace), &ws);
+  if (T == 0 && cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream) != cudaSuccess)
+    return SWL_ERR_CUDA;   // no router ran here to reset the header
+  if (launch_shard_combine(s, ws, gathered, rank, world, aux_loss, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  if (T == 0) return SWL_OK;
+  if (launch_dispatch_gather(s, ws, x, expert_idx, pos_in_expert, out, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  return run_ffn(s, ws, W1, b1, W2, b2, gate, out, stream);
 }
 
 swl_status switch_layer_noalloc_status(void* stream) {

@@ -1,11 +1,13 @@
 """Multi-process plumbing for running the layer on several GPUs of one node.
 
-One process per GPU (torchrun).  The Switch layer's forward pass needs no data
-exchange between ranks when each rank routes its own batch: in the pages'
-design every core computes routing, positions and capacity for the tokens it
-holds (the dispatch mask is laid out per core).  So ranks run independent
-forward passes and only the measurement is combined: a barrier around the
-timed region and the maximum of the per-rank device times.
+One process per GPU (torchrun).  Ranks hold contiguous token ranges of one
+global batch and a full copy of the weights (data parallelism over tokens).
+Positions, the capacity cut and the aux loss of the global batch need one
+exchange per forward pass: every rank's per-expert token counts and sums of p
+(the library's exchange record, 12 bytes per expert), all-gathered in rank
+order (``exchange_records``; ncclAllGather over NVLink on GPUs).  The
+measurement adds a barrier around the timed region and the maximum of the
+per-rank device times.
 
 Everything here is device agnostic (NCCL on GPUs, gloo on CPUs for the tests).
 """
@@ -70,6 +72,23 @@ def aggregate_throughput(info: RankInfo, units_per_rank: int, steps: int,
                          max_total_ms: float) -> float:
     """Units per second of the whole job: every rank's units over the slowest time."""
     return info.world_size * units_per_rank * steps / (max_total_ms / 1e3)
+
+
+def exchange_records(info: RankInfo, record: torch.Tensor) -> torch.Tensor:
+    """All-gather of one equally sized 1-D record per rank: the records of all
+    ranks, concatenated in rank order (a copy of ``record`` on a single rank)."""
+    record = record.reshape(-1).contiguous()
+    if not info.distributed:
+        return record.clone()
+    out = torch.empty(info.world_size * record.numel(), dtype=record.dtype,
+                      device=record.device)
+    dist.all_gather_into_tensor(out, record)
+    return out
+
+
+def token_range(info: RankInfo, T_per_rank: int) -> tuple:
+    """[start, stop) of this rank's tokens in a global batch of world * T_per_rank."""
+    return info.rank * T_per_rank, (info.rank + 1) * T_per_rank
 
 
 def rank_seed(info: RankInfo, base_seed: int = 0) -> int:

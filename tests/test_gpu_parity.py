@@ -371,3 +371,24 @@ def test_random_shapes_ffma_router(spec, ffma_router):
 
 def test_router_decision_needs_float32_weights_ffma(ffma_router):
     test_router_decision_needs_float32_weights("bf16")
+
+
+# ------------------------------------------------------------------ failure path (bounded waits)
+def test_wait_that_runs_out_reports_device_status_and_context_survives():
+    """The expert FFN is made to wait for a GEMM1 epilogue warp that does not
+    exist (test hook): the wait gives up after its (shortened) limit, the call
+    reports SWL_ERR_DEVICE, and the next normal call on the same context passes
+    parity."""
+    spec = synth.LayerSpec("stall_wait", 600, 128, 256, 4, 1.25, "bf16", bias_std=0.05)
+    rd = gap_redraws(spec)
+    ig = synth.make_layer_inputs(spec, device="cuda", redraws=rd)
+    swl.switch_layer_set_wait_limit_ns(1_000_000)          # 1 ms
+    swl.switch_layer_set_stall_test(True)
+    try:
+        with pytest.raises(swl.SwitchLayerError) as ei:
+            swl.forward(ig, spec.cf)
+        assert ei.value.status == 5
+    finally:
+        swl.switch_layer_set_stall_test(False)
+        swl.switch_layer_set_wait_limit_ns(0)
+    _full_parity(spec, rd)
