@@ -19,7 +19,10 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libswitchlayer.so")
+# SWL_LIBRARY=checked loads the range-checked build (see build.py)
+LIB_PATH = os.path.join(_HERE, "libswitchlayer_checked.so"
+                        if os.environ.get("SWL_LIBRARY", "") == "checked"
+                        else "libswitchlayer.so")
 
 SWL_F32, SWL_BF16 = 0, 1
 SWL_WS_HOST_IO = 1
@@ -66,8 +69,9 @@ def lib() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise RuntimeError("libswitchlayer.so is missing: build it with "
-                           "`python -m sparse_mixture_experts_argmax_b200.build`")
+        raise RuntimeError("%s is missing: build it with "
+                           "`python -m sparse_mixture_experts_argmax_b200.build`"
+                           % os.path.basename(LIB_PATH))
     L = ctypes.CDLL(LIB_PATH)
     L.switch_layer_capacity.restype = _i64
     L.switch_layer_capacity.argtypes = [_i64, _i64, _dbl]

@@ -1,8 +1,12 @@
 """Build libswitchlayer.so (sm_100a) in-tree with nvcc.
 
-Usage: python -m sparse_mixture_experts_argmax_b200.build [--force]
+Usage: python -m sparse_mixture_experts_argmax_b200.build [--force] [--checked]
 Objects go to _build/ at the repository root; the shared library is written
-next to this file, where the Python binding loads it.
+next to this file, where the Python binding loads it.  ``--checked`` builds
+libswitchlayer_checked.so with -DSWL_CHECKED: every computed index of the
+dispatch and the expert GEMMs is range-checked, a failed check sets the device
+status to SWL_ERR_DEVICE and the access is skipped (the binding loads it when
+SWL_LIBRARY=checked).
 """
 from __future__ import annotations
 
@@ -19,6 +23,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libswitchlayer.so")
+LIB_CHECKED = os.path.join(PKG, "libswitchlayer_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -42,22 +47,30 @@ def _deps():
             [os.path.abspath(__file__)])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(checked: bool = False) -> bool:
+    lib = LIB_CHECKED if checked else LIB
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile every CUDA source for sm_100a and link the shared library."""
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra_flags=(), checked=None) -> str:
+    """Compile every CUDA source for sm_100a and link the shared library
+    (``checked``: the range-checked variant; None: the one SWL_LIBRARY selects)."""
+    if checked is None:
+        checked = os.environ.get("SWL_LIBRARY", "") == "checked"
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(checked):
+        return lib
+    bdir = os.path.join(BUILD, "checked") if checked else BUILD
+    os.makedirs(bdir, exist_ok=True)
     nvcc = _nvcc()
+    if checked:
+        extra_flags = tuple(extra_flags) + ("-DSWL_CHECKED",)
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -70,15 +83,16 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []
-    print(build(force="--force" in sys.argv or bool(extra), verbose=True, extra_flags=extra))
+    print(build(force="--force" in sys.argv or bool(extra), verbose=True, extra_flags=extra,
+                checked="--checked" in sys.argv))

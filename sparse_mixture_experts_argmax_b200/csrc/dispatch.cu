@@ -246,6 +246,7 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
   if (lane == 0) pos_in_expert[t] = pos;
   if (pos < C_eff) {
     const int row = base + pos - off;
+    if (!checked_index(row >= 0 && row < T, &hdr->err)) return;
     if (lane == 0) slot_token[row] = t;
     V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
     if (in_regs) {
@@ -418,6 +419,7 @@ dispatch_fused_kernel(const uint8_t* __restrict__ x, const int* __restrict__ exp
     if (lane == 0) pos_in_expert[t] = pos;
     if (pos < C_eff) {
       const int row = s_base[e] + pos;
+      if (!checked_index(row >= 0 && row < T, &hdr->err)) return;
       if (lane == 0) slot_token[row] = t;
       if (copy_rows) {
         V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
@@ -533,6 +535,7 @@ shard_combine_kernel(const uint8_t* __restrict__ gathered, int record_bytes,
       mt += s_cnt[1][w];
     }
     if (at != T_total || mt != T_local) atomicExch(&hdr->err, kDevIndexOutOfRange);
+    checked_index(s_tot_rows <= T_local, &hdr->err);
     tile_prefix[N] = s_tot_tiles;
     hdr->next_tile = 0u;
     *aux_loss = (float)((double)N * a / ((double)T_total * (double)T_total));

@@ -24,7 +24,8 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
                        const float* __restrict__ bias, const int* __restrict__ tile_prefix,
                        const int* __restrict__ exp_rows, const int* __restrict__ exp_base,
                        const int* __restrict__ slot_token, const float* __restrict__ gate,
-                       float* __restrict__ out, int num_experts, int M, int K, int mode) {
+                       float* __restrict__ out, int num_experts, int M, int K, int mode,
+                       int T_rows, int* err) {
   __shared__ float As[kTile][kTile + 1];   // [row][k]
   __shared__ float Ws[kTile][kTile + 1];   // [feature][k]
   pdl_trigger();
@@ -67,11 +68,13 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
   for (int i = 0; i < 4; ++i) {
     const int rr = ty * 4 + i;
     if (rr >= nrows) continue;
+    if (!checked_index(r0 + rr >= 0 && r0 + rr < T_rows, err)) continue;
     const float v = acc[i] + bm;
     if (mode == 0) {
       out[(size_t)(r0 + rr) * M + m] = fmaxf(v, 0.f);
     } else {
       const int tok = slot_token[r0 + rr];
+      if (!checked_index(tok >= 0 && tok < T_rows, err)) continue;
       out[(size_t)tok * M + m] = gate[tok] * v;
     }
   }
@@ -93,7 +96,7 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
       static_cast<const float*>(bias), static_cast<const int*>(ws.tile_prefix),
       static_cast<const int*>(ws.exp_rows), static_cast<const int*>(ws.exp_base),
       static_cast<const int*>(ws.slot_token), gate, static_cast<float*>(out),
-      static_cast<int>(s.N), M, K, which);
+      static_cast<int>(s.N), M, K, which, static_cast<int>(s.T), &ws.hdr->err);
   count_launch();
   return e;
 }

@@ -81,6 +81,7 @@ struct FfnArgs {
   int stall_test;  // 1: token tile 0's GEMM2 readiness target is one warp too high (the
                    // wait runs out: a test of the failure path)
   int num_experts;
+  int T_rows;         // rows of the packed buffers and of out (range checks)
   int cache_prefix;   // 1: the scheduler keeps the tile prefix in shared memory
   int bn;         // token rows per tile (multiple of 16, <= 256)
   int stages;
@@ -301,6 +302,12 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         if (ts.phase == 1) fence_proxy_async_global();
         const int arow = ts.e * P.M + ts.mt * kBM;
         const int brow = ts.row0;
+        if (!checked_index(ts.e >= 0 && ts.e < args.num_experts && brow >= 0 &&
+                               brow + ts.rows <= args.T_rows && ts.rows > 0,
+                           args.err)) {
+          fail();
+          break;
+        }
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
           ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
@@ -424,6 +431,8 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         } else {
           dsts[k] = row0 + col;
         }
+        if (col < rows && !checked_index(dsts[k] >= 0 && dsts[k] < args.T_rows, args.err))
+          dsts[k] = 0;
       }
 #pragma unroll
       for (int k = 0; k < kMaxChunks; ++k) {
@@ -526,6 +535,7 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.wait_ns = wait_limit_ns();
   a.stall_test = stall_test_enabled() ? 1 : 0;
   a.num_experts = static_cast<int>(s.N);
+  a.T_rows = static_cast<int>(s.T);
   a.bn = s.tile_rows;
   a.num_acc = a.bn <= kTmemCols / kMaxAcc ? kMaxAcc : 2;
   for (int p = 0; p < 2; ++p) {

@@ -174,6 +174,22 @@ unsigned long long wait_limit_ns();
 // Failure-path test of the expert FFN (switch_layer_set_stall_test).
 bool stall_test_enabled();
 
+#ifdef __CUDACC__
+// Range check of a computed index.  In a checked build (-DSWL_CHECKED) a failed
+// check records kDevIndexOutOfRange in the device error word and returns false,
+// and the caller skips the access; other builds compile it to `true`.
+__device__ __forceinline__ bool checked_index(bool ok, int* err) {
+#ifdef SWL_CHECKED
+  if (!ok) atomicExch(err, kDevIndexOutOfRange);
+  return ok;
+#else
+  (void)ok;
+  (void)err;
+  return true;
+#endif
+}
+#endif
+
 // Programmatic dependent launch: a kernel launched with launch_dependent() may
 // start while the previous kernel on the stream is still finishing; it must call
 // pdl_wait() before touching memory that kernel reads or writes.  Every kernel

@@ -194,3 +194,14 @@ def test_describe_plan_router_mode_and_errors(L):
                                         len(big)) == 1                         # d = 0
     assert L.switch_layer_describe_plan(4096, 764, 3072, 64, swl.SWL_BF16, 1.25, 148, big,
                                         len(big)) != 0                         # d % 8 != 0
+
+
+def test_checked_build_exports_the_same_symbols():
+    """The range-checked variant (SWL_CHECKED) builds and exports every symbol
+    the header declares."""
+    import ctypes
+    path = swl_build.build(checked=True)
+    assert path.endswith("libswitchlayer_checked.so")
+    L2 = ctypes.CDLL(path)
+    for name in swl.EXPORTS:
+        assert hasattr(L2, name), name
