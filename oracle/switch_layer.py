@@ -37,6 +37,22 @@ Readings where the pages are silent or disagree:
 * b_2 sits inside the gate: y = g * (W_2 relu(W_1 x + b_1) + b_2)
   ([ST-note] "Expert FFN Layer" and "Router": y_t = g_t E_{e_t}(x_t)).
 * an empty batch (T = 0) gives no outputs and aux = 0.
+
+Top-2 variant (the earlier-MoE routing the pages compare Switch with):
+
+* [ST-note] "Comparison to Earlier MoE": y_t = sum over the two largest p_t,i
+  of p_t,i E_i(x_t) (gates unnormalised); [MoE-note] the attention-and-MoE note
+  (doc.liz6.com), "From Dense FFN to Sparse Experts": the two selected weights
+  are normalised within the selected set ([0.6, 0.3, 0.1] -> [2/3, 1/3]).  Both
+  are provided (``normalize``).
+* capacity: proportional to k * tokens / N * capacity factor for top-k
+  ([ST-paper] "Expert capacity can be at least halved"): C = ceil(2 cf T / N).
+* positions: the cumulative sum over each expert's column of the top-2
+  dispatch mask in token order (a token's two experts differ, so its two
+  assignments never compete for one column); an assignment is dropped iff its
+  position >= C; a token's output sums its kept assignments.
+* f_i still counts the argmax (first choice), as the loss formula's indicator
+  does; P_i is the mean router probability.
 """
 from __future__ import annotations
 
@@ -215,3 +231,70 @@ def switch_forward_sampled(x, W_r, capacity_factor: float, sample_tokens,
     return {"out_rows": out, "expert_idx": e_all, "gate": g_all, "pos_in_expert": pos,
             "kept": kept, "capacity": C, "f": f, "P": P, "aux": aux_loss(f, P)}
 
+
+# ---------------------------------------------------------------------------
+# top-2 routing ([ST-note] "Comparison to Earlier MoE"; [MoE-note] top-2 example)
+# ---------------------------------------------------------------------------
+def capacity_k(T: int, N: int, capacity_factor: float, k: int) -> int:
+    """Capacity of top-k routing, ceil(k * cf * T / N), exact on the double cf."""
+    if N <= 0 or T < 0 or k < 1 or not math.isfinite(capacity_factor) or capacity_factor <= 0:
+        raise ValueError("invalid capacity arguments")
+    return math.ceil(Fraction(capacity_factor) * k * T / N)
+
+
+def top2(p: np.ndarray, normalize: bool = True):
+    """First choice e1 = argmax_i p_i and second choice e2 = argmax over i != e1
+    (lowest index on ties for both); gates p_e1, p_e2, divided by their sum when
+    ``normalize``.  Returns e [T, 2] and g [T, 2]."""
+    T, N = p.shape
+    if N < 2:
+        raise ValueError("top-2 routing needs at least two experts")
+    rows = np.arange(T)
+    e1 = np.argmax(p, axis=1)
+    rest = p.copy()
+    rest[rows, e1] = -np.inf
+    e2 = np.argmax(rest, axis=1)
+    g = np.stack([p[rows, e1], p[rows, e2]], axis=1)
+    if normalize:
+        g = g / g.sum(axis=1, keepdims=True)
+    return np.stack([e1, e2], axis=1).astype(np.int64), g
+
+
+def positions_top2(e: np.ndarray, N: int) -> np.ndarray:
+    """pos[t, k] = number of assignments to expert e[t, k] by tokens before t
+    (token order; a token's two experts differ)."""
+    seen = [0] * N
+    pos = np.zeros(e.shape, dtype=np.int64)
+    for t in range(e.shape[0]):
+        for k in range(e.shape[1]):
+            pos[t, k] = seen[int(e[t, k])]
+        for k in range(e.shape[1]):
+            seen[int(e[t, k])] += 1
+    return pos
+
+
+def switch_forward_top2(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None,
+                        normalize: bool = True) -> Dict:
+    """Top-2 layer in float64: out [T, d], expert_idx [T, 2], gate [T, 2],
+    pos_in_expert [T, 2], kept [T, 2], capacity, f, P, aux."""
+    xs = _f64(x)
+    T = xs.shape[0]
+    N = _f64(W_r).shape[0]
+    z = router_logits(xs, W_r, b_r)
+    p = router_probs(z) if T else np.zeros((0, N))
+    e, g = top2(p, normalize) if T else (np.zeros((0, 2), np.int64), np.zeros((0, 2)))
+    C = capacity_k(T, N, capacity_factor, 2)
+    pos = positions_top2(e, N)
+    kept = pos < C
+    out = np.zeros((T, xs.shape[1]))
+    for i in range(N):
+        for k in range(2):
+            rows = np.nonzero((e[:, k] == i) & kept[:, k])[0]
+            if rows.size == 0:
+                continue
+            u = expert_ffn(xs[rows], W1[i], b1[i], W2[i], b2[i])
+            out[rows] += g[rows, k, None] * u
+    f, P = load_balance_stats(e[:, 0], p)
+    aux = aux_loss(f, P) if T else 0.0
+    return {"out": out, "expert_idx": e, "gate": g, "pos_in_expert": pos, "kept": kept,
+            "capacity": C, "f": f, "P": P, "aux": aux, "probs": p, "logits": z}

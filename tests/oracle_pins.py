@@ -327,9 +327,125 @@ def pin_logit_gap():
     assert np.all(np.isinf(S.logit_gap(rng.normal(size=(4, 1)))))
 
 
+# ---------------------------------------------------------------------------
+# top-2 routing (the earlier-MoE variant)
+# ---------------------------------------------------------------------------
+def _const_experts(outputs, d, extra):
+    """Experts whose output is a constant row: W1 = 0, b1 = 1 (h = 1), W2 = 0,
+    b2 = the row.  outputs: list of d-vectors; extra: further constant rows."""
+    rows = np.array(list(outputs) + list(extra), dtype=np.float64)
+    N = rows.shape[0]
+    return (np.zeros((N, 1, d)), np.ones((N, 1)), np.zeros((N, d, 1)), rows)
+
+
+def pin_top2_worked_example():
+    """The attention-and-MoE note's example: router weights [0.6, 0.3, 0.1],
+    top-2 normalised to [2/3, 1/3]; expert outputs [3,0] and [0,6] merge to
+    [2,2].  Unnormalised (the reading note's formula): [1.8, 1.8]."""
+    g = _gold("top2_worked_example.json")
+    p = np.array([g["router_weights"]])
+    x = np.log(p)                          # W_r = I: softmax(W_r x) = p
+    W1, b1, W2, b2 = _const_experts([o + [0.0] for o in g["expert_outputs"]], 3,
+                                    [[1.0, 1.0, 1.0]])
+    r = S.switch_forward_top2(x, np.eye(3), W1, b1, W2, b2, capacity_factor=1.0)
+    assert r["expert_idx"].tolist() == [[0, 1]]
+    assert np.allclose(r["gate"][0], g["normalised_gates"], rtol=0, atol=1e-15)
+    assert np.allclose(r["out"][0, :2], g["merged_output"], rtol=0, atol=1e-14)
+    assert r["out"][0, 2] == 0.0
+    r = S.switch_forward_top2(x, np.eye(3), W1, b1, W2, b2, capacity_factor=1.0,
+                              normalize=False)
+    assert np.allclose(r["out"][0, :2], g["merged_output_unnormalised"], rtol=0, atol=1e-14)
+
+
+def pin_top2_choices_and_capacity():
+    """Second choice = the runner-up logit (torch.topk), ties to the lowest
+    index; capacity ceil(2 cf T / N) by exact search."""
+    rng = np.random.default_rng(12)
+    z = rng.normal(size=(300, 6))
+    e, g = S.top2(S.router_probs(z), normalize=False)
+    tk = torch.topk(torch.from_numpy(z), 2, dim=1)
+    assert np.array_equal(e, tk.indices.numpy())
+    assert np.allclose(g, torch.softmax(torch.from_numpy(z), 1).gather(1, tk.indices).numpy(),
+                       rtol=0, atol=1e-15)
+    # exact ties: three equal largest logits -> experts 1 and 2; two equal
+    # runners-up below a clear winner -> the lower of them
+    z = np.array([[0.0, 5.0, 5.0, 5.0], [9.0, 1.0, 3.0, 3.0]])
+    e, _ = S.top2(S.router_probs(z))
+    assert e.tolist() == [[1, 2], [0, 2]]
+    for T in (0, 1, 7, 64, 97):
+        for N in (2, 3, 8):
+            for cf in (0.25, 1.0, 1.25, 2.0):
+                want = _smallest_integer_at_least(Fraction(cf) * 2 * T / N)
+                assert S.capacity_k(T, N, cf, 2) == want
+    assert S.capacity_k(4096, 64, 1.25, 1) == S.capacity(4096, 64, 1.25)
+
+
+def pin_top2_positions_bruteforce():
+    """All top-2 assignments of T <= 5 tokens to N = 3 experts: each expert's
+    kept assignments are its first min(count, C) in token order."""
+    pairs = [(a, b) for a in range(3) for b in range(3) if a != b]
+    for T in range(0, 5):
+        for assign in itertools.product(pairs, repeat=T):
+            e = np.array(assign, dtype=np.int64).reshape(T, 2)
+            pos = S.positions_top2(e, 3)
+            for i in range(3):
+                toks = [t for t in range(T) if i in assign[t]]
+                got = [int(pos[t, assign[t].index(i)]) for t in toks]
+                assert got == list(range(len(toks)))
+
+
+def pin_top2_closed_forms():
+    """Identical experts, normalised gates, no drops: y = E(x) exactly (the two
+    gates sum to one).  Two experts, no drops: y = p_0 E_0(x) + p_1 E_1(x)."""
+    rng = np.random.default_rng(13)
+    T, d, d_ff, N = 40, 6, 7, 4
+    x = rng.normal(size=(T, d))
+    W1, b1, W2, b2 = _rand_ffn(rng, 1, d, d_ff)
+    rep = lambda a: np.repeat(a, N, axis=0)
+    r = S.switch_forward_top2(x, rng.normal(size=(N, d)), rep(W1), rep(b1), rep(W2), rep(b2),
+                              capacity_factor=float(N))
+    assert r["kept"].all()
+    assert np.allclose(r["out"], _torch_ffn(x, W1[0], b1[0], W2[0], b2[0]), rtol=1e-13,
+                       atol=1e-13)
+    W1, b1, W2, b2 = _rand_ffn(rng, 2, d, d_ff)
+    Wr = rng.normal(size=(2, d))
+    for norm in (True, False):
+        r = S.switch_forward_top2(x, Wr, W1, b1, W2, b2, capacity_factor=2.0, normalize=norm)
+        p = torch.softmax(torch.from_numpy(x @ Wr.T), dim=1).numpy()
+        ref = (p[:, :1] * _torch_ffn(x, W1[0], b1[0], W2[0], b2[0]) +
+               p[:, 1:] * _torch_ffn(x, W1[1], b1[1], W2[1], b2[1]))
+        assert np.allclose(r["out"], ref, rtol=1e-13, atol=1e-13)
+    # the aux loss counts first choices: it equals the top-1 layer's
+    top1 = S.switch_forward(x, Wr, W1, b1, W2, b2, capacity_factor=2.0)
+    assert abs(r["aux"] - top1["aux"]) < 1e-15
+
+
+def pin_top2_drops():
+    """A capacity cut removes assignments only: kept assignments contribute
+    exactly what they contribute without the cut."""
+    rng = np.random.default_rng(14)
+    T, d, d_ff, N = 60, 5, 6, 4
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(N, d))
+    Wr[0] *= 3
+    W1, b1, W2, b2 = _rand_ffn(rng, N, d, d_ff)
+    full = S.switch_forward_top2(x, Wr, W1, b1, W2, b2, capacity_factor=float(N))
+    cut = S.switch_forward_top2(x, Wr, W1, b1, W2, b2, capacity_factor=0.5)
+    assert full["kept"].all() and (~cut["kept"]).any() and cut["capacity"] == 15
+    for t in range(T):
+        want = np.zeros(d)
+        for k in range(2):
+            if cut["kept"][t, k]:
+                e = cut["expert_idx"][t, k]
+                want += cut["gate"][t, k] * _torch_ffn(x[t:t + 1], W1[e], b1[e], W2[e], b2[e])[0]
+        assert np.allclose(cut["out"][t], want, rtol=1e-13, atol=1e-13)
+
+
 ALL_PINS = [
     pin_lb_worked_example, pin_even_routing_is_one, pin_collapse_tends_to_N,
     pin_not_a_lower_bound, pin_softmax_rows_and_closed_form, pin_ties_lowest_index,
     pin_capacity, pin_positions_bruteforce, pin_drops, pin_single_expert_is_dense_ffn,
     pin_identical_experts_scale_by_gate, pin_sampled_matches_full, pin_logit_gap,
+    pin_top2_worked_example, pin_top2_choices_and_capacity, pin_top2_positions_bruteforce,
+    pin_top2_closed_forms, pin_top2_drops,
 ]

@@ -94,6 +94,37 @@ def _gap_distinct_values(z):
     return np.asarray(out)
 
 
+def _top2_second_is_last(p, normalize=True):
+    # mistake: the second choice is the smallest probability
+    T, N = p.shape
+    e1 = np.argmax(p, axis=1)
+    e2 = np.argmin(p, axis=1)
+    rows = np.arange(T)
+    g = np.stack([p[rows, e1], p[rows, e2]], axis=1)
+    if normalize:
+        g = g / g.sum(axis=1, keepdims=True)
+    return np.stack([e1, e2], axis=1).astype(np.int64), g
+
+
+def _top2_never_normalised(p, normalize=True):
+    return _orig_top2(p, False)
+
+
+def _capacity_k_ignores_k(T, N, cf, k):
+    return S.capacity(T, N, cf)
+
+
+def _positions_top2_firsts_first(e, N):
+    # mistake: all first choices claim slots before any second choice
+    seen = [0] * N
+    pos = np.zeros(e.shape, dtype=np.int64)
+    for k in range(e.shape[1]):
+        for t in range(e.shape[0]):
+            pos[t, k] = seen[int(e[t, k])]
+            seen[int(e[t, k])] += 1
+    return pos
+
+
 MUTATIONS = {
     "ties_to_highest": ("top1", _top1_highest_tie),
     "positions_one_based": ("positions", _positions_one_based),
@@ -109,7 +140,13 @@ MUTATIONS = {
     "gap_top1_minus_min": ("logit_gap", _gap_top1_minus_min),
     "gap_on_probs": ("logit_gap", _gap_on_probs),
     "gap_ties_ignored": ("logit_gap", _gap_distinct_values),
+    "top2_second_is_last": ("top2", _top2_second_is_last),
+    "top2_never_normalised": ("top2", _top2_never_normalised),
+    "top2_capacity_ignores_k": ("capacity_k", _capacity_k_ignores_k),
+    "top2_firsts_first": ("positions_top2", _positions_top2_firsts_first),
 }
+
+_orig_top2 = S.top2
 
 
 def _orig_positions(expert_idx, N):
