@@ -72,6 +72,8 @@ typedef enum swl_dtype { SWL_F32 = 0, SWL_BF16 = 1 } swl_dtype;
 
 /* Workspace flag: also reserve device staging buffers for switch_layer_forward_host_io. */
 #define SWL_WS_HOST_IO 1
+/* Workspace flag: size for switch_layer_forward_top2 (not combinable with SWL_WS_HOST_IO). */
+#define SWL_WS_TOP2 2
 
 /* Number of timed stages and their order (see switch_layer_forward_timed):
  * 0 router (logits; for N <= 128 also softmax/argmax/ranks; bf16 layers include
@@ -117,6 +119,31 @@ swl_status switch_layer_forward(int64_t T, int64_t d, int64_t d_ff, int64_t N, i
                                 void* out, int32_t* expert_idx, float* gate,
                                 int32_t* pos_in_expert, float* aux_loss, const float* b_r,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Top-2 variant: the earlier-MoE routing the pages compare the Switch layer
+ * with ("Switch Transformer" reading note, "Comparison to Earlier MoE":
+ * y_t = sum over the two largest p_t,i of p_t,i E_i(x_t); the attention-and-MoE
+ * note's example normalises the two weights within the selected set).
+ *   e_t,0 = argmax_i p_t,i, e_t,1 = argmax over i != e_t,0 (lowest index on ties)
+ *   g_t,k = p_t,e_t,k, divided by (p_t,e_t,0 + p_t,e_t,1) when normalize = 1
+ *   C     = ceil(2 * capacity_factor * T / N)  (capacity grows with k: paper-graph
+ *           summary, "Expert capacity can be at least halved")
+ *   pos_t,k = assignments to e_t,k by tokens before t (token order; a token's two
+ *           experts differ); assignment (t, k) is dropped iff pos_t,k >= C
+ *   out_t = sum over kept k of g_t,k E_e_t,k(x_t)   (zero if both are dropped)
+ *   aux   = N * sum_i f_i P_i with f_i counting FIRST choices (the loss
+ *           formula's argmax indicator)
+ * expert_idx, gate and pos_in_expert are [T, 2] (row-major: first choice,
+ * second choice).  Requires 2 <= N <= 2048 (SWL_ERR_INVALID_ARG /
+ * SWL_ERR_UNSUPPORTED) and a workspace sized with SWL_WS_TOP2; normalize is 0
+ * or 1.  Other arguments, layouts and errors as switch_layer_forward. */
+swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                     const void* x, const float* W_r, const void* W1,
+                                     const void* b1, const void* W2, const void* b2,
+                                     double capacity_factor, int normalize, void* out,
+                                     int32_t* expert_idx, float* gate, int32_t* pos_in_expert,
+                                     float* aux_loss, const float* b_r, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /* As switch_layer_forward, and records cudaEvent_t stage_events[k] on `stream`
  * before stage 0 (k = 0) and after stage k-1 (k = 1..SWL_NUM_STAGES): an array

@@ -76,7 +76,8 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
                      int* __restrict__ exp_base, int* __restrict__ tile_prefix,
                      int* __restrict__ ready, float* __restrict__ aux_loss, WsHeader* hdr,
                      int nblk, int N, int T, int C_eff, int tile_rows,
-                     uint8_t* __restrict__ record, int record_psum_offset) {
+                     uint8_t* __restrict__ record, int record_psum_offset,
+                     const int* __restrict__ blk_count1, int* __restrict__ exp_count1) {
   __shared__ int wc[kScanWarps][32];
   __shared__ double wp[kScanWarps][32];
   __shared__ int is_last;
@@ -109,6 +110,12 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
       }
     }
   }
+  // top-2: first choices alone, for the aux loss's f
+  int c1sum = 0;
+  if (blk_count1 != nullptr && e < N)
+    for (int b = b0; b < b1; ++b) c1sum += blk_count1[(size_t)b * N + e];
+  __shared__ int wc1[kScanWarps][32];
+  wc1[warp][lane] = c1sum;
   wc[warp][lane] = csum;
   wp[warp][lane] = psum;
   __syncthreads();
@@ -139,6 +146,11 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
       for (int w = 0; w < kScanWarps; ++w) { tot += wc[w][lane]; ps += wp[w][lane]; }
       exp_count[e] = tot;
       psum64[e] = ps;
+      if (exp_count1 != nullptr) {
+        int t1 = 0;
+        for (int w = 0; w < kScanWarps; ++w) t1 += wc1[w][lane];
+        exp_count1[e] = t1;
+      }
       if (record != nullptr) {
         reinterpret_cast<int*>(record)[e] = tot;
         reinterpret_cast<double*>(record + record_psum_offset)[e] = ps;
@@ -169,7 +181,8 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     const int m = min(c, C_eff);
     rows += m;
     tiles += (m + tile_rows - 1) / tile_rows;
-    aux += (double)c * __ldcg(psum64 + i);
+    const int cf = exp_count1 != nullptr ? __ldcg(exp_count1 + i) : c;   // argmax counts
+    aux += (double)cf * __ldcg(psum64 + i);
   }
   int base_rows = block_excl_scan(rows, s_warp, &s_tot_rows);
   int base_tiles = block_excl_scan(tiles, s_warp, &s_tot_tiles);
@@ -213,13 +226,16 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
                        const int* __restrict__ exp_base, const int* __restrict__ exp_off,
                        int* __restrict__ slot_token, uint8_t* __restrict__ xbuf,
                        uint8_t* __restrict__ out, int T, int N, int C_eff, int row_bytes,
-                       int tpb, int prefetch, WsHeader* hdr) {
+                       int tpb, int prefetch, int kk, WsHeader* hdr) {
   using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
   pdl_trigger();
   pdl_wait();   // offsets come from the scan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kGatherWarps + warp;
-  if (t >= T) return;
+  // one warp per assignment a = kk t + k (kk = 1: per token; top-2: kk = 2, and a
+  // dropped assignment writes nothing: the combine kernel sums the kept ones)
+  const int a = blockIdx.x * kGatherWarps + warp;
+  if (a >= T * kk) return;
+  const int t = a / kk;
   const int nv = row_bytes / VEC;
   const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
   V reg[kGatherMaxVecPerLane];
@@ -231,8 +247,8 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
     for (int j = 0; j < kGatherMaxVecPerLane; ++j)
       if (lane + 32 * j < nv) reg[j] = src[lane + 32 * j];
   }
-  const int e = expert_idx[t];
-  const int rank = pos_in_expert[t];            // holds the in-block rank
+  const int e = expert_idx[a];
+  const int rank = pos_in_expert[a];            // holds the in-block rank
   if (e < 0 || e >= N) {          // cannot happen: the router clamps its choice
     if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
     return;
@@ -243,11 +259,11 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
   const int pos = off + blk_off[(size_t)b * N + e] + rank;
   const int base = exp_base[e];
   __syncwarp();
-  if (lane == 0) pos_in_expert[t] = pos;
+  if (lane == 0) pos_in_expert[a] = pos;
   if (pos < C_eff) {
     const int row = base + pos - off;
-    if (!checked_index(row >= 0 && row < T, &hdr->err)) return;
-    if (lane == 0) slot_token[row] = t;
+    if (!checked_index(row >= 0 && row < T * kk, &hdr->err)) return;
+    if (lane == 0) slot_token[row] = a;
     V* dst = reinterpret_cast<V*>(xbuf + (size_t)row * row_bytes);
     if (in_regs) {
 #pragma unroll
@@ -256,11 +272,36 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
     } else {
       for (int i = lane; i < nv; i += 32) dst[i] = src[i];
     }
-  } else {
+  } else if (kk == 1) {
     V* dst = reinterpret_cast<V*>(out + (size_t)t * row_bytes);
     V z;
     memset(&z, 0, sizeof(V));
     for (int i = lane; i < nv; i += 32) dst[i] = z;
+  }
+}
+
+// Top-2 combine: out[t] = sum over k of (assignment 2t+k kept ? ybuf[2t+k] : 0),
+// the gated rows the GEMM2 epilogue wrote, added in fp32 in choice order and
+// rounded once to the activation dtype (a dropped assignment contributes 0; a
+// token with both dropped gets a zero row).  One warp per token.
+template <typename TA>
+__global__ void __launch_bounds__(kGatherThreads)
+combine_top2_kernel(const TA* __restrict__ ybuf, const int* __restrict__ pos_in_expert,
+                    TA* __restrict__ out, int T, int d, int C_cmp) {
+  pdl_trigger();
+  pdl_wait();   // rows come from the expert FFN
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kGatherWarps + warp;
+  if (t >= T) return;
+  const bool k0 = pos_in_expert[2 * t] < C_cmp, k1 = pos_in_expert[2 * t + 1] < C_cmp;
+  const TA* y0 = ybuf + (size_t)(2 * t) * d;
+  const TA* y1 = y0 + d;
+  TA* o = out + (size_t)t * d;
+  for (int j = lane; j < d; j += 32) {
+    float v = 0.f;
+    if (k0) v += static_cast<float>(y0[j]);
+    if (k1) v += static_cast<float>(y1[j]);
+    o[j] = static_cast<TA>(v);
   }
 }
 
@@ -553,7 +594,7 @@ shard_combine_kernel(const uint8_t* __restrict__ gathered, int record_bytes,
 
 bool dispatch_fused_ok(const Shape& s) {
   const int64_t elem = s.dtype == 1 ? 2 : 4;
-  return s.N <= kFusedMaxN && s.T * s.d * elem <= (int64_t{16} << 20);
+  return s.topk == 1 && !s.sharded && s.N <= kFusedMaxN && s.T * s.d * elem <= (int64_t{16} << 20);
 }
 
 cudaError_t launch_dispatch_fused(const Shape& s, const Workspace& ws, const void* x,
@@ -582,7 +623,9 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
       dispatch_scan_kernel, dim3(grid), dim3(kScanThreads), 0, stream, ws.blk_count, ws.blk_psum,
       ws.blk_off, ws.exp_count, ws.psum64, ws.exp_rows, ws.exp_base, ws.tile_prefix, ws.ready,
       aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows,
-      static_cast<uint8_t*>(record), (int)shard_record_psum_offset(s.N));
+      static_cast<uint8_t*>(record), (int)shard_record_psum_offset(s.N),
+      static_cast<const int*>(s.topk == 2 ? ws.blk_count1 : nullptr),
+      s.topk == 2 ? ws.exp_count1 : nullptr);
   count_launch();
   return e;
 }
@@ -611,7 +654,7 @@ cudaError_t launch_shard_combine(const Shape& s, const Workspace& ws, const void
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
                                    const int* expert_idx, int* pos_in_expert, void* out,
                                    cudaStream_t stream) {
-  const int grid = (int)((s.T + kGatherWarps - 1) / kGatherWarps);
+  const int grid = (int)((s.T * s.topk + kGatherWarps - 1) / kGatherWarps);
   const int elem = s.dtype == 1 ? 2 : 4;
   const int row_bytes = (int)(s.d * elem);
   const bool vec16 = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0) &&
@@ -624,7 +667,24 @@ cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const vo
       static_cast<const int*>(s.sharded ? ws.exp_off : nullptr), ws.slot_token,
       static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T, (int)s.N,
       (int)s.C_cmp, row_bytes, s.tpb, s.T * (int64_t)row_bytes <= (int64_t{48} << 20) ? 1 : 0,
-      ws.hdr);
+      s.topk, ws.hdr);
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_combine_top2(const Shape& s, const Workspace& ws, const int* pos_in_expert,
+                                void* out, cudaStream_t stream) {
+  const int grid = (int)((s.T + kGatherWarps - 1) / kGatherWarps);
+  cudaError_t e;
+  if (s.dtype == 1) {
+    e = launch_dependent(combine_top2_kernel<__nv_bfloat16>, dim3(grid), dim3(kGatherThreads), 0,
+                         stream, static_cast<const __nv_bfloat16*>(ws.ybuf), pos_in_expert,
+                         static_cast<__nv_bfloat16*>(out), (int)s.T, (int)s.d, (int)s.C_cmp);
+  } else {
+    e = launch_dependent(combine_top2_kernel<float>, dim3(grid), dim3(kGatherThreads), 0,
+                         stream, static_cast<const float*>(ws.ybuf), pos_in_expert,
+                         static_cast<float*>(out), (int)s.T, (int)s.d, (int)s.C_cmp);
+  }
   count_launch();
   return e;
 }

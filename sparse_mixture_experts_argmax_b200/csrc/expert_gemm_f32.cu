@@ -88,15 +88,15 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
   const int M = static_cast<int>(which == 0 ? s.d_ff : s.d);
   const int K = static_cast<int>(which == 0 ? s.d : s.d_ff);
   const float* act = static_cast<const float*>(which == 0 ? ws.xbuf : ws.hbuf);
-  // upper bound on row tiles: sum_e ceil(m_e / 32) <= T / 32 + N
-  const int64_t max_tiles = (s.T + kTile - 1) / kTile + s.N;
+  // upper bound on row tiles: sum_e ceil(m_e / 32) <= A / 32 + N (A = T * topk rows)
+  const int64_t max_tiles = (s.T * s.topk + kTile - 1) / kTile + s.N;
   dim3 grid(static_cast<unsigned>(max_tiles), (M + kTile - 1) / kTile);
   const cudaError_t e = launch_dependent(
       expert_gemm_f32_kernel, grid, dim3(256), 0, stream, act, static_cast<const float*>(W),
       static_cast<const float*>(bias), static_cast<const int*>(ws.tile_prefix),
       static_cast<const int*>(ws.exp_rows), static_cast<const int*>(ws.exp_base),
       static_cast<const int*>(ws.slot_token), gate, static_cast<float*>(out),
-      static_cast<int>(s.N), M, K, which, static_cast<int>(s.T), &ws.hdr->err);
+      static_cast<int>(s.N), M, K, which, static_cast<int>(s.T * s.topk), &ws.hdr->err);
   count_launch();
   return e;
 }

@@ -32,20 +32,23 @@ struct WsHeader {
 struct Workspace {
   WsHeader* hdr;
   float* logits;        // [ksplit_eff, T, N] fp32 partial logits (slice 0 reused for p)
-  int* blk_count;       // [nblk, N] tokens of block b routed to expert e
+  int* blk_count;       // [nblk, N] assignments of block b's tokens to expert e
+  int* blk_count1;      // top-2: [nblk, N] first choices of block b's tokens for e
   int* blk_off;         // [nblk, N] tokens of earlier blocks routed to e
   float* blk_psum;      // [nblk, N] sum over block b of p_{t,e}
-  int* exp_count;       // [N] tokens whose argmax is e (before capacity)
+  int* exp_count;       // [N] assignments to e (tokens whose argmax is e for top-1)
+  int* exp_count1;      // top-2: [N] tokens whose first choice is e
   int* exp_rows;        // [N] kept rows m_e = min(count_e, C)
   int* exp_base;        // [N] first packed row of expert e
   int* exp_off;         // [N] shard of a global batch: tokens of e on earlier ranks
   int* tile_prefix;     // [N+1] prefix over experts of ceil(m_e / tile_rows)
   double* psum64;       // [N] sum over all tokens of p_{t,e}
-  int* slot_token;      // [T] packed row -> token
+  int* slot_token;      // [A] packed row -> assignment (token t, choice k: t * topk + k)
   int* ready;           // [T/16 + N + 1] per token tile: GEMM1 epilogue warps done
   void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
-  void* xbuf;           // [T, d] packed expert inputs (act dtype)
-  void* hbuf;           // [T, d_ff] packed hidden activations (act dtype)
+  void* xbuf;           // [A, d] packed expert inputs (act dtype), A = T * topk
+  void* hbuf;           // [A, d_ff] packed hidden activations (act dtype)
+  void* ybuf;           // top-2: [A, d] gated expert output per assignment (act dtype)
   // host-I/O staging (only with SWL_WS_HOST_IO)
   void* x_dev;
   void* out_dev;
@@ -64,6 +67,8 @@ struct Shape {
   int64_t T_total;  // tokens of the whole batch (T unless a shard of a global batch)
   int64_t C_cmp;  // min(C, T_total): a token is kept iff its position is below it
   int sharded;    // 1: a shard of a global batch (positions offset by earlier ranks)
+  int topk;       // experts per token: 1 (Switch) or 2 (the top-2 variant)
+  int normalize;  // top-2: gates divided by their sum
   int router_path;  // RouterPath
   int tpb;        // tokens per block of the softmax / rank / gather stages (<= kTokensPerBlock)
   int nblk;       // ceil(T / tpb)
@@ -89,7 +94,7 @@ struct RouterPlan {
   int ksplit;   // logits slices (CTAs of a cluster on the tile / tensor-core paths)
 };
 // tensor != 0: the tensor-core router (bf16 layers); else the FFMA kernels.
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor);
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk = 1);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 
@@ -141,6 +146,9 @@ cudaError_t launch_shard_combine(const Shape& s, const Workspace& ws, const void
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
                                    const int* expert_idx, int* pos_in_expert, void* out,
                                    cudaStream_t stream);
+// Top-2: out[t] = sum over the token's kept assignments of their gated rows.
+cudaError_t launch_combine_top2(const Shape& s, const Workspace& ws, const int* pos_in_expert,
+                                void* out, cudaStream_t stream);
 // Scan and gather in one launch, for N <= 128 and small batches (one CTA per
 // router block copies its tokens' rows; the two-kernel path spreads large copies
 // over more warps).

@@ -219,25 +219,49 @@ router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ W_r,
 constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = kSoftmaxThreads / 32;
 
+// Order of (value, expert) pairs for the top-2 choice: larger value first,
+// lower expert index first among equal values.
+__device__ __forceinline__ bool rank_before(float v, int i, float w, int j) {
+  return v > w || (v == w && i < j);
+}
+
+// (b1, i1) >= (b2, i2) and (c1, j1) >= (c2, j2) in the (value desc, index asc)
+// order: the two largest of the four, in order, into (b1, i1), (b2, i2).
+__device__ __forceinline__ void top2_merge(float& b1, int& i1, float& b2, int& i2, float c1,
+                                           int j1, float c2, int j2) {
+  if (rank_before(c1, j1, b1, i1)) {
+    if (rank_before(b1, i1, c2, j2)) { b2 = b1; i2 = i1; } else { b2 = c2; i2 = j2; }
+    b1 = c1;
+    i1 = j1;
+  } else if (rank_before(c1, j1, b2, i2)) {
+    b2 = c1;
+    i2 = j1;
+  }
+}
+
+
 // One CTA per block of tpb tokens; one warp per token with the row of logits
 // held in registers (NPL = logits per lane, N <= 32*NPL):
 //   z = sum of the K-slice partials + b_r; m = max with the lowest index;
 //   s = sum exp(z - m); gate = p at the argmax = 1/s; p_i = exp(z_i - m)/s is
 //   accumulated per lane into per-expert sums.
 // Then per block: ranks, counts blk_count[b][e], probability sums blk_psum[b][e]
-// (each warp's tokens in order, warps in order).
-template <int NPL>
+// (each warp's tokens in order, warps in order).  TOP2: as the streaming
+// kernel's top-2 form (below), with [T, 2] outputs.
+template <int NPL, bool TOP2>
 __global__ void __launch_bounds__(kSoftmaxThreads)
 router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* __restrict__ b_r,
                       int T, int N, int tpb, int* __restrict__ expert_idx,
                       float* __restrict__ gate, int* __restrict__ local_rank,
                       int* __restrict__ blk_count, float* __restrict__ blk_psum,
-                      WsHeader* hdr) {
+                      int* __restrict__ blk_count1, int normalize, WsHeader* hdr) {
+  constexpr int K = TOP2 ? 2 : 1;
   extern __shared__ float smem_f[];
   float* s_bias = smem_f;                 // [N]
   float* s_psum = smem_f + N;             // [kSoftmaxWarps][N]
-  __shared__ int eid[kTokensPerBlock];
-  __shared__ int lead_count[kTokensPerBlock];
+  __shared__ int eid[K][kTokensPerBlock];
+  __shared__ int lead_count[K * kTokensPerBlock];
+  __shared__ int lead_first[TOP2 ? kTokensPerBlock : 1];
   pdl_trigger();
   pdl_wait();   // partial logits come from the logits kernel
   const int b = blockIdx.x;
@@ -253,7 +277,10 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
   const size_t slice = (size_t)T * N;
   for (int i = warp; i < tpb; i += kSoftmaxWarps) {
     if (i >= ntok) {
-      if (lane == 0) eid[i] = -1;
+      if (lane == 0) {
+        eid[0][i] = -1;
+        eid[K - 1][i] = -1;
+      }
       continue;
     }
     const int t = t0 + i;
@@ -280,16 +307,31 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
       const int n = lane + 32 * j;
       v[j] = (n < N) ? v[j] + s_bias[n] : -INFINITY;
     }
-    float best = -INFINITY;
-    int bidx = 0x7fffffff;
+    float best = -INFINITY, second = -INFINITY;
+    int bidx = 0x7fffffff, sidx = 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < NPL; ++j)
-      if (v[j] > best) { best = v[j]; bidx = lane + 32 * j; }   // first index within a lane
+    for (int j = 0; j < NPL; ++j) {     // ascending columns: strict compares keep the lowest index
+      if (v[j] > best) {
+        if (TOP2) { second = best; sidx = bidx; }
+        best = v[j];
+        bidx = lane + 32 * j;
+      } else if (TOP2 && v[j] > second) {
+        second = v[j];
+        sidx = lane + 32 * j;
+      }
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, best, off);
       const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-      if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+      if (TOP2) {
+        const float os = __shfl_xor_sync(0xffffffffu, second, off);
+        const int oj = __shfl_xor_sync(0xffffffffu, sidx, off);
+        top2_merge(best, bidx, second, sidx, ov, oi, os, oj);
+      } else if (ov > best || (ov == best && oi < bidx)) {
+        best = ov;
+        bidx = oi;
+      }
     }
     float ssum = 0.f;
 #pragma unroll
@@ -304,14 +346,27 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
     for (int j = 0; j < NPL; ++j) acc[j] += v[j] * inv;
     // a non-finite logit (NaN, or an infinite maximum that makes the exp sum
     // NaN) is flagged; an index with no finite maximum is kept in range
-    if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
-      if (bidx >= N) bidx = 0;
-      if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
+    bool bad = bidx >= N || !isfinite(best) || !isfinite(ssum);
+    if (bidx >= N) bidx = 0;
+    if (TOP2) {
+      bad = bad || sidx >= N || sidx == bidx;
+      if (sidx >= N || sidx == bidx) sidx = bidx == 0 ? 1 : 0;
     }
+    if (bad && lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
     if (lane == 0) {
-      expert_idx[t] = bidx;
-      gate[t] = inv;            // p at the argmax: exp(0) / s
-      eid[i] = bidx;
+      if (TOP2) {
+        const float e2 = expf(second - best);      // p_e2 / p_e1
+        expert_idx[2 * t] = bidx;
+        expert_idx[2 * t + 1] = sidx;
+        gate[2 * t] = normalize ? 1.0f / (1.0f + e2) : inv;
+        gate[2 * t + 1] = normalize ? e2 / (1.0f + e2) : e2 * inv;
+        eid[0][i] = bidx;
+        eid[K - 1][i] = sidx;
+      } else {
+        expert_idx[t] = bidx;
+        gate[t] = inv;            // p at the argmax: exp(0) / s
+        eid[0][i] = bidx;
+      }
     }
   }
 #pragma unroll
@@ -320,8 +375,13 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
     if (n < N) s_psum[warp * N + n] = acc[j];
   }
   __syncthreads();
-  block_ranks(eid, lead_count, ntok, tpb, t0, local_rank);
+  if (TOP2) {
+    block_ranks_top2(eid[0], eid[K - 1], lead_count, lead_first, ntok, tpb, t0, local_rank);
+  } else {
+    block_ranks(eid[0], lead_count, ntok, tpb, t0, local_rank);
+  }
   int* cnt_row = blk_count + (size_t)b * N;
+  int* cnt1_row = TOP2 ? blk_count1 + (size_t)b * N : nullptr;
   float* ps_row = blk_psum + (size_t)b * N;
   for (int n = threadIdx.x; n < N; n += kSoftmaxThreads) {
     float a = 0.f;
@@ -329,10 +389,15 @@ router_softmax_kernel(const float* __restrict__ zpart, int nsplit, const float* 
     for (int w = 0; w < kSoftmaxWarps; ++w) a += s_psum[w * N + n];
     ps_row[n] = a;
     cnt_row[n] = 0;
+    if (TOP2) cnt1_row[n] = 0;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < ntok; i += kSoftmaxThreads) {
-    if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
+    if (lead_count[i] > 0) cnt_row[eid[0][i]] = lead_count[i];
+    if (TOP2) {
+      if (lead_count[tpb + i] > 0) cnt_row[eid[K - 1][i]] = lead_count[tpb + i];
+      if (lead_first[i] > 0) cnt1_row[eid[0][i]] = lead_first[i];
+    }
   }
 }
 
@@ -438,21 +503,29 @@ __host__ __device__ constexpr size_t stream_softmax_smem(int N) {
   return 128 + (static_cast<size_t>(kStreamBufs) * kStreamChunk + 1) * N * sizeof(float);
 }
 
-template <int V4>   // float4 columns per lane in pass A: N <= 128 * V4
+// TOP2: the first choice and the runner-up (lowest index on ties for both,
+// two experts per token, see top2_merge), gates p_e1 and p_e2, divided by
+// their sum when `normalize`; outputs are [T, 2] (first choice, then second),
+// the block statistics count both choices (blk_count) and, for the aux loss,
+// first choices alone (blk_count1).
+template <int V4, bool TOP2>   // V4: float4 columns per lane in pass A, N <= 128 * V4
 __global__ void __launch_bounds__(kStreamThreads, 1)
 router_softmax_stream_kernel(const float* __restrict__ z, const float* __restrict__ b_r, int T,
                              int N, int tpb, int nblk, int* __restrict__ expert_idx,
                              float* __restrict__ gate, int* __restrict__ local_rank,
                              int* __restrict__ blk_count, float* __restrict__ blk_psum,
-                             WsHeader* hdr, unsigned long long wait_ns) {
+                             int* __restrict__ blk_count1, int normalize, WsHeader* hdr,
+                             unsigned long long wait_ns) {
   constexpr int VPT = (V4 * 32 + kStreamThreads - 1) / kStreamThreads;   // pass-B float4 / thread
+  constexpr int K = TOP2 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   float* buf = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
   float* s_bias = buf + static_cast<size_t>(kStreamBufs) * kStreamChunk * N;   // [N]
   __shared__ uint64_t full[kStreamBufs];
-  __shared__ int eid[kTokensPerBlock];
-  __shared__ int lead_count[kTokensPerBlock];
+  __shared__ int eid[K][kTokensPerBlock];
+  __shared__ int lead_count[K * kTokensPerBlock];
+  __shared__ int lead_first[TOP2 ? kTokensPerBlock : 1];
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NV = N >> 2;   // float4 per row
@@ -511,8 +584,22 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
         float4* row = reinterpret_cast<float4*>(zc + static_cast<size_t>(warp) * N);
         const float4* bias4 = reinterpret_cast<const float4*>(s_bias);
         float4 v[V4];
+        // chain c holds column 4q + c: ascending columns per chain, so a strict
+        // compare keeps each chain's lowest index among equal values
         float bq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         int iq[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+        float sq2[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // runner-up (TOP2)
+        int jq[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+        auto insert = [&](int c4, float val, int col) {
+          if (val > bq[c4]) {
+            if (TOP2) { sq2[c4] = bq[c4]; jq[c4] = iq[c4]; }
+            bq[c4] = val;
+            iq[c4] = col;
+          } else if (TOP2 && val > sq2[c4]) {
+            sq2[c4] = val;
+            jq[c4] = col;
+          }
+        };
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
           const int q = lane + 32 * k;
@@ -522,23 +609,34 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
           } else {
             v[k] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
           }
-          // chain c holds column 4q + c: ascending columns per chain, so the
-          // strict compare keeps each chain's lowest index among equal maxima
-          if (v[k].x > bq[0]) { bq[0] = v[k].x; iq[0] = 4 * q; }
-          if (v[k].y > bq[1]) { bq[1] = v[k].y; iq[1] = 4 * q + 1; }
-          if (v[k].z > bq[2]) { bq[2] = v[k].z; iq[2] = 4 * q + 2; }
-          if (v[k].w > bq[3]) { bq[3] = v[k].w; iq[3] = 4 * q + 3; }
+          insert(0, v[k].x, 4 * q);
+          insert(1, v[k].y, 4 * q + 1);
+          insert(2, v[k].z, 4 * q + 2);
+          insert(3, v[k].w, 4 * q + 3);
         }
-        float best = bq[0];
-        int bidx = iq[0];
+        float best = bq[0], second = sq2[0];
+        int bidx = iq[0], sidx = jq[0];
 #pragma unroll
-        for (int c4 = 1; c4 < 4; ++c4)
-          if (bq[c4] > best || (bq[c4] == best && iq[c4] < bidx)) { best = bq[c4]; bidx = iq[c4]; }
+        for (int c4 = 1; c4 < 4; ++c4) {
+          if (TOP2) {
+            top2_merge(best, bidx, second, sidx, bq[c4], iq[c4], sq2[c4], jq[c4]);
+          } else if (rank_before(bq[c4], iq[c4], best, bidx)) {
+            best = bq[c4];
+            bidx = iq[c4];
+          }
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
           const float ov = __shfl_xor_sync(0xffffffffu, best, off);
           const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-          if (ov > best || (ov == best && oi < bidx)) { best = ov; bidx = oi; }
+          if (TOP2) {
+            const float os = __shfl_xor_sync(0xffffffffu, second, off);
+            const int oj = __shfl_xor_sync(0xffffffffu, sidx, off);
+            top2_merge(best, bidx, second, sidx, ov, oi, os, oj);
+          } else if (rank_before(ov, oi, best, bidx)) {
+            best = ov;
+            bidx = oi;
+          }
         }
         float sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -564,15 +662,31 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
         }
         // a non-finite logit (NaN, or an infinite maximum that makes the exp
         // sum NaN) is flagged; an index with no finite maximum is kept in range
-        if (bidx >= N || !isfinite(best) || !isfinite(ssum)) {
-          if (bidx >= N) bidx = 0;
-          if (lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
+        bool bad = bidx >= N || !isfinite(best) || !isfinite(ssum);
+        if (bidx >= N) bidx = 0;
+        if (TOP2) {
+          bad = bad || sidx >= N || sidx == bidx;
+          if (sidx >= N || sidx == bidx) sidx = bidx == 0 ? 1 : 0;
         }
+        if (bad && lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
         if (lane == 0) {
           const int t = t0b + c * kStreamChunk + warp;
-          expert_idx[t] = bidx;
-          gate[t] = inv;          // p at the argmax: exp(0) / s
-          eid[c * kStreamChunk + warp] = bidx;
+          const int i = c * kStreamChunk + warp;
+          if (TOP2) {
+            const float e2 = expf(second - best);      // p_e2 / p_e1
+            const float g1 = normalize ? 1.0f / (1.0f + e2) : inv;
+            const float g2 = normalize ? e2 / (1.0f + e2) : e2 * inv;
+            expert_idx[2 * t] = bidx;
+            expert_idx[2 * t + 1] = sidx;
+            gate[2 * t] = g1;
+            gate[2 * t + 1] = g2;
+            eid[0][i] = bidx;
+            eid[K - 1][i] = sidx;
+          } else {
+            expert_idx[t] = bidx;
+            gate[t] = inv;          // p at the argmax: exp(0) / s
+            eid[0][i] = bidx;
+          }
         }
       }
       __syncthreads();
@@ -594,8 +708,13 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
     }
     if (failed) break;
     // block bookkeeping: ranks, the block's per-expert counts and sums of p
-    block_ranks(eid, lead_count, ntb, ntb, t0b, local_rank);
+    if (TOP2) {
+      block_ranks_top2(eid[0], eid[K - 1], lead_count, lead_first, ntb, ntb, t0b, local_rank);
+    } else {
+      block_ranks(eid[0], lead_count, ntb, ntb, t0b, local_rank);
+    }
     int* cnt_row = blk_count + static_cast<size_t>(b) * N;
+    int* cnt1_row = TOP2 ? blk_count1 + static_cast<size_t>(b) * N : nullptr;
     float* ps_row = blk_psum + static_cast<size_t>(b) * N;
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
@@ -603,11 +722,17 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
       if (q < NV) {
         reinterpret_cast<float4*>(ps_row)[q] = acc[v];
         reinterpret_cast<int4*>(cnt_row)[q] = make_int4(0, 0, 0, 0);
+        if (TOP2) reinterpret_cast<int4*>(cnt1_row)[q] = make_int4(0, 0, 0, 0);
       }
     }
     __syncthreads();
-    for (int i = tid; i < ntb; i += kStreamThreads)
-      if (lead_count[i] > 0) cnt_row[eid[i]] = lead_count[i];
+    for (int i = tid; i < ntb; i += kStreamThreads) {
+      if (lead_count[i] > 0) cnt_row[eid[0][i]] = lead_count[i];
+      if (TOP2) {
+        if (lead_count[ntb + i] > 0) cnt_row[eid[K - 1][i]] = lead_count[ntb + i];
+        if (lead_first[i] > 0) cnt1_row[eid[0][i]] = lead_first[i];
+      }
+    }
     __syncthreads();   // eid / lead_count are reused by the next block
   }
   if (failed) {
@@ -1002,22 +1127,23 @@ template <int NPL>
 cudaError_t launch_softmax_t(const Shape& s, const Workspace& ws, const float* b_r,
                              int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
   const size_t smem = (size_t)(kSoftmaxWarps + 1) * s.N * sizeof(float);
+  auto kern = s.topk == 2 ? router_softmax_kernel<NPL, true> : router_softmax_kernel<NPL, false>;
   if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        router_softmax_kernel<NPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_dependent(router_softmax_kernel<NPL>, dim3(s.nblk), dim3(kSoftmaxThreads), smem,
-                          stream, static_cast<const float*>(ws.logits), s.ksplit_eff, b_r,
-                          (int)s.T, (int)s.N, s.tpb, expert_idx, gate, local_rank, ws.blk_count,
-                          ws.blk_psum, ws.hdr);
+  return launch_dependent(kern, dim3(s.nblk), dim3(kSoftmaxThreads), smem, stream,
+                          static_cast<const float*>(ws.logits), s.ksplit_eff, b_r, (int)s.T,
+                          (int)s.N, s.tpb, expert_idx, gate, local_rank, ws.blk_count,
+                          ws.blk_psum, ws.blk_count1, s.normalize, ws.hdr);
 }
 
 }  // namespace
 
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor) {
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk) {
   RouterPlan p;
-  if (tensor && N <= kFusedRouterMaxN) {
+  if (tensor && N <= kFusedRouterMaxN && topk == 1) {
     // tensor cores: 128-token tiles; K split over 2 or 4 CTAs of a cluster while
     // the tiles alone would leave most SMs idle (and each CTA keeps >= 2 k-blocks)
     const int64_t tiles = (T + 127) / 128;
@@ -1031,7 +1157,7 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor) {
     p.tpb = (int)(128 / S);
     return p;
   }
-  if (N <= kFusedRouterMaxN) {
+  if (N <= kFusedRouterMaxN && topk == 1) {
     // one fused kernel; big tiles once there are enough of them to fill the GPU
     const int64_t bm = N <= 64 ? 256 : 128;
     const int64_t tiles = (T + bm - 1) / bm;
@@ -1050,9 +1176,9 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor) {
     }
     return p;
   }
-  // wide N: logits GEMM in 128 x 128 tiles (bf16 layers: tensor cores over the
-  // whole K; fp32 layers: FFMA with K slices for ~3 CTAs per SM), then the softmax
-  // kernel over blocks of 128/64/32 tokens
+  // wide N (and every top-2 layer): logits GEMM in 128 x 128 tiles (bf16
+  // layers: tensor cores over the whole K; fp32 layers: FFMA with K slices for
+  // ~3 CTAs per SM), then the softmax kernel over blocks of 128/64/32 tokens
   p.tpb = 32;
   for (int tpb = 128; tpb > 32; tpb /= 2)
     if ((T + tpb - 1) / tpb >= 2 * 148) { p.tpb = tpb; break; }
@@ -1119,7 +1245,7 @@ cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void
 }
 
 int softmax_variant(const Shape& s) {
-  if (s.N <= kFusedRouterMaxN) return kSoftmaxFused;
+  if (s.router_path != kRouterWide && s.router_path != kRouterTCWide) return kSoftmaxFused;
   if (s.ksplit_eff == 1 && s.N % 4 == 0 && s.N <= kStreamSoftmaxMaxN) return kSoftmaxStream;
   return (s.N + 31) / 32 <= 64 ? kSoftmaxRows : kSoftmaxWide;
 }
@@ -1128,8 +1254,9 @@ template <int V4>
 cudaError_t launch_stream_t(const Shape& s, const Workspace& ws, const float* b_r,
                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
   const size_t smem = stream_softmax_smem(static_cast<int>(s.N));
-  cudaError_t e = cudaFuncSetAttribute(router_softmax_stream_kernel<V4>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = s.topk == 2 ? router_softmax_stream_kernel<V4, true>
+                          : router_softmax_stream_kernel<V4, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -1137,10 +1264,10 @@ cudaError_t launch_stream_t(const Shape& s, const Workspace& ws, const float* b_
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
   const int grid = s.nblk < sms ? s.nblk : sms;
-  return launch_dependent(router_softmax_stream_kernel<V4>, dim3(grid), dim3(kStreamThreads),
-                          smem, stream, static_cast<const float*>(ws.logits), b_r, (int)s.T,
-                          (int)s.N, s.tpb, s.nblk, expert_idx, gate, local_rank, ws.blk_count,
-                          ws.blk_psum, ws.hdr, wait_limit_ns());
+  return launch_dependent(kern, dim3(grid), dim3(kStreamThreads), smem, stream,
+                          static_cast<const float*>(ws.logits), b_r, (int)s.T, (int)s.N, s.tpb,
+                          s.nblk, expert_idx, gate, local_rank, ws.blk_count, ws.blk_psum,
+                          ws.blk_count1, s.normalize, ws.hdr, wait_limit_ns());
 }
 
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,

@@ -32,6 +32,46 @@ __device__ __forceinline__ void block_ranks(const int* eid, int* lead_count, int
   }
 }
 
+// Top-2 form of block_ranks: token i of the block holds assignments to experts
+// eid1[i] (first choice) and eid2[i] (second; always a different expert).  The
+// rank of assignment (i, k) is the number of earlier tokens of the block with
+// an assignment to the same expert (token order, the dispatch mask's column
+// cumsum), written to local_rank[2 (t0 + i) + k].  lead_count[i] (k = 0) /
+// lead_count[tpb + i] (k = 1) is set on the block's first assignment to an
+// expert to that expert's number of assignments in the block, and lead_first[i]
+// on a token that is the first with that expert as FIRST choice to the number
+// of first choices of it.  eid1[i] < 0 marks an absent token.
+__device__ __forceinline__ void block_ranks_top2(const int* eid1, const int* eid2,
+                                                 int* lead_count, int* lead_first, int ntok,
+                                                 int tpb, int t0, int* __restrict__ local_rank) {
+  for (int i = threadIdx.x; i < tpb; i += blockDim.x) {
+    lead_count[i] = 0;
+    lead_count[tpb + i] = 0;
+    lead_first[i] = 0;
+    if (i >= ntok || eid1[i] < 0) continue;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = k == 0 ? eid1[i] : eid2[i];
+      int rank = 0, first = 0;
+      for (int j = 0; j < i; ++j) {
+        rank += (eid1[j] == e) | (eid2[j] == e);
+        first += (eid1[j] == e);
+      }
+      local_rank[2 * (t0 + i) + k] = rank;
+      if (rank == 0) {
+        int c = 1;
+        for (int j = i + 1; j < ntok; ++j) c += (eid1[j] == e) | (eid2[j] == e);
+        lead_count[k * tpb + i] = c;
+      }
+      if (k == 0 && first == 0) {
+        int c = 1;
+        for (int j = i + 1; j < ntok; ++j) c += (eid1[j] == e);
+        lead_first[i] = c;
+      }
+    }
+  }
+}
+
 // Routing of R token rows t0 .. t0+R-1 (dispatch block b) from fp32 logits Z
 // (row stride zs; bias already added; columns N .. 32*NPL-1 hold -inf):
 //   m = max_i z_i with the lowest index on ties; s = sum_i exp(z_i - m);

@@ -42,6 +42,8 @@ static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws) {
   const size_t elem = s.dtype == SWL_BF16 ? 2 : 4;
   const size_t T = static_cast<size_t>(s.T), N = static_cast<size_t>(s.N);
+  const size_t A = T * static_cast<size_t>(s.topk);   // expert assignments
+  const bool top2 = s.topk == 2;
   const size_t nb = static_cast<size_t>(s.nblk);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -56,6 +58,8 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
                ? 0
                : static_cast<size_t>(s.ksplit_eff) * T * N * 4));
   w.blk_count = reinterpret_cast<int*>(take(nb * N * 4));
+  w.blk_count1 = reinterpret_cast<int*>(take(top2 ? nb * N * 4 : 0));
+  w.exp_count1 = reinterpret_cast<int*>(take(top2 ? N * 4 : 0));
   w.blk_off = reinterpret_cast<int*>(take(nb * N * 4));
   w.blk_psum = reinterpret_cast<float*>(take(nb * N * 4));
   w.exp_count = reinterpret_cast<int*>(take(N * 4));
@@ -64,14 +68,15 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.exp_off = reinterpret_cast<int*>(take(N * 4));
   w.tile_prefix = reinterpret_cast<int*>(take((N + 1) * 4));
   w.psum64 = reinterpret_cast<double*>(take(N * 8));
-  w.slot_token = reinterpret_cast<int*>(take(T * 4));
-  w.ready = reinterpret_cast<int*>(take((T / 16 + N + 1) * 4));
+  w.slot_token = reinterpret_cast<int*>(take(A * 4));
+  w.ready = reinterpret_cast<int*>(take((A / 16 + N + 1) * 4));
   w.w3 = reinterpret_cast<void*>(
       take(s.router_path == kRouterTC || s.router_path == kRouterTCWide
                ? 3 * N * static_cast<size_t>(s.d) * 2
                : 0));
-  w.xbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
-  w.hbuf = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d_ff) * elem));
+  w.xbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d) * elem));
+  w.hbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d_ff) * elem));
+  w.ybuf = reinterpret_cast<void*>(take(top2 ? A * static_cast<size_t>(s.d) * elem : 0));
   if (host_io) {
     w.x_dev = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
     w.out_dev = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
@@ -134,8 +139,11 @@ static bool aligned(const void* p, uintptr_t a) {
 
 // Fills Shape; returns SWL_OK or the validation error.
 static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype, double cf,
-                             Shape* s) {
+                             Shape* s, int topk = 1, int normalize = 1) {
   if (T < 0 || d <= 0 || d_ff <= 0 || N <= 0) return SWL_ERR_INVALID_ARG;
+  if (topk != 1 && topk != 2) return SWL_ERR_INVALID_ARG;
+  if (topk == 2 && N < 2) return SWL_ERR_INVALID_ARG;                    // two experts needed
+  if (topk == 2 && N > kStreamSoftmaxMaxN) return SWL_ERR_UNSUPPORTED;
   if (dtype != SWL_F32 && dtype != SWL_BF16) return SWL_ERR_INVALID_ARG;
   if (!std::isfinite(cf) || !(cf > 0.0)) return SWL_ERR_INVALID_ARG;
   if (dtype == SWL_BF16 && (d % 8 != 0 || d_ff % 8 != 0)) return SWL_ERR_UNSUPPORTED;
@@ -148,14 +156,17 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->d_ff = d_ff;
   s->N = N;
   s->dtype = dtype;
-  s->C = switch_layer_capacity(T, N, cf);
-  s->C_eff = s->C < T ? s->C : T;
+  // top-k capacity ceil(k cf T / N) = the formula's value for k T tokens
+  s->C = switch_layer_capacity(T * topk, N, cf);
+  s->C_eff = s->C < T ? s->C : T;   // a token has at most one assignment per expert
   s->T_total = T;
   s->C_cmp = s->C_eff;
   s->sharded = 0;
+  s->topk = topk;
+  s->normalize = normalize ? 1 : 0;
   // the tensor-core router serves bf16 layers unless the FFMA router was chosen
   const bool tensor_router = dtype == SWL_BF16 && g_router_mode.load() == SWL_ROUTER_TENSOR;
-  const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0);
+  const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0, topk);
   s->router_path = rp.path;
   s->kslice = rp.kslice;
   s->ksplit_eff = rp.ksplit;
@@ -192,7 +203,8 @@ static swl_status run_routing(const Shape& s, const Workspace& ws, const void* x
   if (s.router_path == kRouterTC || s.router_path == kRouterTCWide) {
     CUtensorMap tx, tw;
     if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
-        !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N, router_tc_padded_experts(s.N)))
+        !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N,
+                        s.router_path == kRouterTCWide ? 128 : router_tc_padded_experts(s.N)))
       return SWL_ERR_CUDA;
     // the FFN's first tiles stream W1 from its start: fetch a slice into L2 while
     // routing and dispatch run, when the router is a single wave of CTAs (with a
@@ -211,7 +223,7 @@ static swl_status run_routing(const Shape& s, const Workspace& ws, const void* x
     return SWL_ERR_CUDA;
   }
   if (!rec(1)) return SWL_ERR_CUDA;
-  if (s.N > kFusedRouterMaxN &&
+  if (softmax_variant(s) != kSoftmaxFused &&
       launch_router_softmax(s, ws, b_r, expert_idx, gate, pos_in_expert, stream) != cudaSuccess)
     return SWL_ERR_CUDA;
   if (!rec(2)) return SWL_ERR_CUDA;
@@ -227,9 +239,9 @@ static swl_status run_ffn(const Shape& s, const Workspace& ws, const void* W1, c
     if (sms <= 0) return SWL_ERR_CUDA;
     CUtensorMap a1, b1m, a2, b2m;
     if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff, 128) ||
-        !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T, s.tile_rows) ||
+        !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T * s.topk, s.tile_rows) ||
         !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
-        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T, s.tile_rows))
+        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T * s.topk, s.tile_rows))
       return SWL_ERR_CUDA;
     if (launch_expert_ffn_bf16(s, ws, a1, b1m, a2, b2m, b1, b2, gate, out, sms, stream) !=
         cudaSuccess)
@@ -280,8 +292,12 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
       return SWL_ERR_CUDA;
   }
   if (!rec(4)) return SWL_ERR_CUDA;
-  st = run_ffn(s, ws, W1, b1, W2, b2, gate, out, stream);
+  // top-2: the GEMM2 epilogue writes each assignment's gated row to ybuf and
+  // the combine kernel adds a token's kept rows
+  st = run_ffn(s, ws, W1, b1, W2, b2, gate, s.topk == 2 ? ws.ybuf : out, stream);
   if (st != SWL_OK) return st;
+  if (s.topk == 2 && launch_combine_top2(s, ws, pos_in_expert, out, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
   if (!rec(5)) return SWL_ERR_CUDA;
   return SWL_OK;
 }
@@ -312,9 +328,10 @@ static swl_status forward_impl(int64_t T, int64_t d, int64_t d_ff, int64_t N, in
                                const void* W2, const void* b2, double cf, void* out,
                                int32_t* expert_idx, float* gate, int32_t* pos, float* aux,
                                const float* b_r, void* workspace, size_t workspace_bytes,
-                               void* stream_v, void* const* ev) {
+                               void* stream_v, void* const* ev, int topk = 1,
+                               int normalize = 1) {
   Shape s;
-  swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s);
+  swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s, topk, normalize);
   if (st != SWL_OK) return st;
   st = validate_io(s, x, W_r, W1, b1, W2, b2, out, expert_idx, gate, pos, aux, workspace,
                    workspace_bytes, false);
@@ -394,8 +411,9 @@ int64_t switch_layer_capacity(int64_t T, int64_t N, double cf) {
 swl_status switch_layer_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                        double cf, int flags, size_t* bytes) {
   if (!bytes) return SWL_ERR_INVALID_ARG;
+  if ((flags & SWL_WS_TOP2) && (flags & SWL_WS_HOST_IO)) return SWL_ERR_INVALID_ARG;
   Shape s;
-  const swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s);
+  const swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s, (flags & SWL_WS_TOP2) ? 2 : 1);
   if (st != SWL_OK) return st;
   *bytes = workspace_layout(s, (flags & SWL_WS_HOST_IO) != 0, 0, nullptr);
   return SWL_OK;
@@ -410,6 +428,19 @@ swl_status switch_layer_forward(int64_t T, int64_t d, int64_t d_ff, int64_t N, i
   return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
                       expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
                       stream, nullptr);
+}
+
+swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                     const void* x, const float* W_r, const void* W1,
+                                     const void* b1, const void* W2, const void* b2,
+                                     double capacity_factor, int normalize, void* out,
+                                     int32_t* expert_idx, float* gate, int32_t* pos_in_expert,
+                                     float* aux_loss, const float* b_r, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (normalize != 0 && normalize != 1) return SWL_ERR_INVALID_ARG;
+  return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
+                      expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
+                      stream, nullptr, 2, normalize);
 }
 
 swl_status switch_layer_forward_timed(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,

@@ -205,3 +205,20 @@ def test_checked_build_exports_the_same_symbols():
     L2 = ctypes.CDLL(path)
     for name in swl.EXPORTS:
         assert hasattr(L2, name), name
+
+
+def test_top2_workspace_and_validation(L):
+    """Top-2 workspaces hold twice the packed rows plus the per-assignment output
+    rows; one expert, or top-2 beyond 2048 experts, is refused on the host."""
+    import ctypes
+    n1 = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25)
+    n2 = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25, swl.SWL_WS_TOP2)
+    assert n2 > n1 + 4096 * (768 + 3072 + 768) * 2
+    n = ctypes.c_size_t(0)
+    assert L.switch_layer_workspace_size(64, 32, 32, 1, swl.SWL_BF16, 1.0, swl.SWL_WS_TOP2,
+                                         ctypes.byref(n)) == 1
+    assert L.switch_layer_workspace_size(64, 32, 32, 4096, swl.SWL_BF16, 1.0, swl.SWL_WS_TOP2,
+                                         ctypes.byref(n)) == 2
+    assert L.switch_layer_workspace_size(64, 32, 32, 4, swl.SWL_BF16, 1.0,
+                                         swl.SWL_WS_TOP2 | swl.SWL_WS_HOST_IO,
+                                         ctypes.byref(n)) == 1
