@@ -232,6 +232,69 @@ swl_status switch_layer_forward_shard_end(int64_t T, int64_t d, int64_t d_ff, in
                                           int32_t* pos_in_expert, float* aux_loss,
                                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Expert parallelism over ranks (experts sharded, tokens sharded) ----
+ *
+ * The pages' multi-device design: every device hosts a subset of the experts,
+ * and tokens travel to the device of their expert and back in an all-to-all
+ * (paper-graph summary, "The routing mechanics in detail": dispatch, expert
+ * computation, output recombination; "Switch Transformer, explained", recipe
+ * step 4).  Rank r of `world` ranks (N % world == 0) holds the weights of
+ * experts [r L, r L + L), L = N / world, as W1_local [L, d_ff, d], b1_local
+ * [L, d_ff], W2_local [L, d, d_ff], b2_local [L, d], the full router W_r, and
+ * the r-th contiguous token range of one global batch of T_total tokens.  The
+ * result is the unsharded layer's: the same positions, capacity cut, aux loss
+ * and outputs.  A forward pass on every rank:
+ *   1. switch_layer_forward_shard_begin (routing, exchange record);
+ *   2. all-gather of the records (as for the global-batch split), and a host
+ *      copy of them for the all-to-all sizes: switch_layer_ep_counts gives, per
+ *      peer, the rows this rank sends and receives (kept tokens only);
+ *   3. switch_layer_ep_dispatch: positions and aux loss from the records, and
+ *      this rank's kept token rows packed into send_rows [sum send, d] in the
+ *      order peer, expert, position;
+ *   4. all-to-all: peer g's block of send_rows goes to peer g (NCCL
+ *      ncclSend/ncclRecv or torch.distributed.all_to_all_single with the counts
+ *      of step 2), arriving in recv_rows [sum recv, d] in source-rank order;
+ *   5. switch_layer_ep_experts: the received rows of this rank's experts through
+ *      their FFN (bias, no gate), written back in the receive order into
+ *      ret_rows [sum recv, d];
+ *   6. the reverse all-to-all (recv counts become send counts) into
+ *      back_rows [sum send, d];
+ *   7. switch_layer_ep_combine: out_t = g_t * (the token's returned row), or 0
+ *      for a dropped token.
+ * Every rank's workspace is sized by switch_layer_ep_workspace_size (its own
+ * tokens plus room for L * min(C, T_total) received rows:
+ * switch_layer_ep_max_recv_rows).  Row buffers are device memory in the
+ * activation dtype, 16-byte aligned for bf16. */
+int64_t switch_layer_ep_max_recv_rows(int64_t N, int world, int64_t T_total,
+                                      double capacity_factor);
+swl_status switch_layer_ep_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                          int dtype, int world, int64_t T_total,
+                                          double capacity_factor, size_t* bytes);
+/* Host-only: rows this rank sends to (send_rows[g]) and receives from
+ * (recv_rows[g]) every peer g, from a host copy of the gathered records. */
+swl_status switch_layer_ep_counts(int64_t N, int world, int rank, int64_t T_total,
+                                  double capacity_factor, const void* gathered_host,
+                                  int64_t* send_rows, int64_t* recv_rows);
+swl_status switch_layer_ep_dispatch(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                    int world, int rank, int64_t T_total,
+                                    double capacity_factor, const void* gathered, const void* x,
+                                    int32_t* expert_idx, int32_t* pos_in_expert,
+                                    float* aux_loss, void* send_rows, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+/* n_recv: rows in recv_rows (the sum of recv counts); ret_rows holds as many. */
+swl_status switch_layer_ep_experts(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                   int world, int rank, int64_t T_total, double capacity_factor,
+                                   const void* gathered, void* recv_rows, int64_t n_recv,
+                                   const void* W1_local, const void* b1_local,
+                                   const void* W2_local, const void* b2_local, void* ret_rows,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+swl_status switch_layer_ep_combine(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                   int world, int rank, int64_t T_total,
+                                   double capacity_factor, const void* back_rows,
+                                   const int32_t* expert_idx, const float* gate,
+                                   const int32_t* pos_in_expert, void* out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Bytes of the fixed device scratch used by switch_layer_forward_noalloc. */
 #define SWL_NOALLOC_MAX_BYTES (64u << 20)
 

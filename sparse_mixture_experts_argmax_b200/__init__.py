@@ -41,7 +41,9 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_noalloc_status", "switch_layer_shard_record_bytes",
            "switch_layer_forward_shard_begin", "switch_layer_forward_shard_end",
            "switch_layer_set_wait_limit_ns", "switch_layer_set_stall_test",
-           "switch_layer_forward_top2")
+           "switch_layer_forward_top2", "switch_layer_ep_max_recv_rows",
+           "switch_layer_ep_workspace_size", "switch_layer_ep_counts",
+           "switch_layer_ep_dispatch", "switch_layer_ep_experts", "switch_layer_ep_combine")
 SWL_ROUTER_TENSOR = 0
 SWL_ROUTER_FFMA = 1
 SWL_NOALLOC_MAX_BYTES = 64 << 20
@@ -105,6 +107,24 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_forward_noalloc.argtypes = _FWD_ARGS[:17] + [_vp, _vp]
     L.switch_layer_noalloc_status.restype = _i32
     L.switch_layer_noalloc_status.argtypes = [_vp]
+    L.switch_layer_ep_max_recv_rows.restype = _i64
+    L.switch_layer_ep_max_recv_rows.argtypes = [_i64, _i32, _i64, _dbl]
+    L.switch_layer_ep_workspace_size.restype = _i32
+    L.switch_layer_ep_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i32, _i32, _i64, _dbl,
+                                                 ctypes.POINTER(_sz)]
+    L.switch_layer_ep_counts.restype = _i32
+    L.switch_layer_ep_counts.argtypes = [_i64, _i32, _i32, _i64, _dbl, _vp,
+                                         ctypes.POINTER(_i64), ctypes.POINTER(_i64)]
+    L.switch_layer_ep_dispatch.restype = _i32
+    L.switch_layer_ep_dispatch.argtypes = [_i64, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _dbl,
+                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    L.switch_layer_ep_experts.restype = _i32
+    L.switch_layer_ep_experts.argtypes = [_i64, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _dbl,
+                                          _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                          _vp]
+    L.switch_layer_ep_combine.restype = _i32
+    L.switch_layer_ep_combine.argtypes = [_i64, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _dbl,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     L.switch_layer_forward_top2.restype = _i32
     L.switch_layer_forward_top2.argtypes = _FWD_ARGS[:12] + [_i32] + _FWD_ARGS[12:]
     L.switch_layer_set_wait_limit_ns.restype = _i32
@@ -327,6 +347,61 @@ def switch_layer_set_stall_test(on: bool) -> None:
     _check(lib().switch_layer_set_stall_test(1 if on else 0), "set_stall_test")
 
 
+def switch_layer_ep_max_recv_rows(N, world, T_total, capacity_factor) -> int:
+    return int(lib().switch_layer_ep_max_recv_rows(N, world, T_total, capacity_factor))
+
+
+def switch_layer_ep_workspace_size(T, d, d_ff, N, dtype, world, T_total, capacity_factor) -> int:
+    n = _sz(0)
+    _check(lib().switch_layer_ep_workspace_size(T, d, d_ff, N, dtype, world, T_total,
+                                                capacity_factor, ctypes.byref(n)),
+           "ep_workspace_size")
+    return int(n.value)
+
+
+def switch_layer_ep_counts(N, world, rank, T_total, capacity_factor, gathered_host):
+    """(send rows per peer, receive rows per peer) from a host copy of the records."""
+    _require(gathered_host, "gathered_host", torch.uint8, device="cpu")
+    send = (_i64 * world)()
+    recv = (_i64 * world)()
+    _check(lib().switch_layer_ep_counts(N, world, rank, int(T_total), float(capacity_factor),
+                                        _ptr(gathered_host), send, recv), "ep_counts")
+    return [int(v) for v in send], [int(v) for v in recv]
+
+
+def switch_layer_ep_dispatch(x, d_ff, N, world, rank, T_total, capacity_factor, gathered,
+                             expert_idx, pos_in_expert, aux_loss, send_rows, workspace,
+                             stream=None) -> None:
+    T, d = x.shape
+    _check(lib().switch_layer_ep_dispatch(
+        T, d, d_ff, N, dtype_code(x.dtype), world, rank, int(T_total), float(capacity_factor),
+        _ptr(gathered), _ptr(x), _ptr(expert_idx), _ptr(pos_in_expert), _ptr(aux_loss),
+        _ptr(send_rows), _ptr(workspace), workspace.numel(), _stream_handle(stream)),
+        "ep_dispatch")
+
+
+def switch_layer_ep_experts(T, d, d_ff, N, act_dtype, world, rank, T_total, capacity_factor,
+                            gathered, recv_rows, W1_local, b1_local, W2_local, b2_local, ret_rows,
+                            workspace, stream=None) -> None:
+    for t, n in ((W1_local, "W1_local"), (b1_local, "b1_local"), (W2_local, "W2_local"),
+                 (b2_local, "b2_local")):
+        _require(t, n, act_dtype)
+    _check(lib().switch_layer_ep_experts(
+        T, d, d_ff, N, dtype_code(act_dtype), world, rank, int(T_total), float(capacity_factor),
+        _ptr(gathered), _ptr(recv_rows), recv_rows.shape[0], _ptr(W1_local), _ptr(b1_local),
+        _ptr(W2_local), _ptr(b2_local), _ptr(ret_rows), _ptr(workspace), workspace.numel(),
+        _stream_handle(stream)), "ep_experts")
+
+
+def switch_layer_ep_combine(T, d, d_ff, N, act_dtype, world, rank, T_total, capacity_factor,
+                            back_rows, expert_idx, gate, pos_in_expert, out, workspace,
+                            stream=None) -> None:
+    _check(lib().switch_layer_ep_combine(
+        T, d, d_ff, N, dtype_code(act_dtype), world, rank, int(T_total), float(capacity_factor),
+        _ptr(back_rows), _ptr(expert_idx), _ptr(gate), _ptr(pos_in_expert), _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream_handle(stream)), "ep_combine")
+
+
 def switch_layer_shard_record_bytes(N: int) -> int:
     return int(lib().switch_layer_shard_record_bytes(N))
 
@@ -464,4 +539,44 @@ def forward_top2(inputs: dict, capacity_factor: float, normalize: bool = True,
                               workspace=workspace, stream=stream)
     if check:
         _check(switch_layer_device_status(workspace, stream), "device status")
+    return o
+
+
+def forward_ep(inputs: dict, capacity_factor: float, N: int, T_total: int, rank: int,
+               world: int, allgather, alltoall, stream=None, check: bool = True) -> dict:
+    """One rank's part of an expert-parallel forward pass.  ``inputs``: this
+    rank's token range x, the full W_r (and b_r), and the weights of this
+    rank's experts W1/b1/W2/b2 ([N / world, ...]).  ``allgather(record)``
+    returns every rank's record in rank order (device); ``alltoall(rows,
+    send_counts, recv_counts)`` exchanges row blocks between ranks (rows [sum
+    send, d] -> [sum recv, d])."""
+    x, W1 = inputs["x"], inputs["W1"]
+    T, d = x.shape
+    d_ff = W1.shape[1]
+    dev = W1.device
+    ws = torch.empty(switch_layer_ep_workspace_size(T, d, d_ff, N, dtype_code(x.dtype), world,
+                                                    T_total, capacity_factor),
+                     dtype=torch.uint8, device=dev)
+    o = alloc_outputs(T, d, x.dtype, device=dev)
+    record = torch.empty(switch_layer_shard_record_bytes(N), dtype=torch.uint8, device=dev)
+    switch_layer_forward_shard_begin(x, inputs["W_r"], capacity_factor, T_total, o["expert_idx"],
+                                     o["gate"], o["pos_in_expert"], record, d_ff,
+                                     b_r=inputs.get("b_r"), workspace=ws, stream=stream)
+    gathered = allgather(record)
+    send_c, recv_c = switch_layer_ep_counts(N, world, rank, T_total, capacity_factor,
+                                            gathered.cpu())
+    send = torch.empty((sum(send_c), d), dtype=x.dtype, device=dev)
+    switch_layer_ep_dispatch(x, d_ff, N, world, rank, T_total, capacity_factor, gathered,
+                             o["expert_idx"], o["pos_in_expert"], o["aux_loss"], send, ws,
+                             stream)
+    recv = alltoall(send, send_c, recv_c)
+    ret = torch.empty_like(recv)
+    switch_layer_ep_experts(T, d, d_ff, N, x.dtype, world, rank, T_total, capacity_factor,
+                            gathered, recv, W1, inputs["b1"], inputs["W2"], inputs["b2"], ret, ws,
+                            stream)
+    back = alltoall(ret, recv_c, send_c)
+    switch_layer_ep_combine(T, d, d_ff, N, x.dtype, world, rank, T_total, capacity_factor, back,
+                            o["expert_idx"], o["gate"], o["pos_in_expert"], o["out"], ws, stream)
+    if check:
+        _check(switch_layer_device_status(ws, stream), "device status")
     return o

@@ -272,7 +272,7 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
     } else {
       for (int i = lane; i < nv; i += 32) dst[i] = src[i];
     }
-  } else if (kk == 1) {
+  } else if (kk == 1 && out != nullptr) {   // (expert parallel: the combine writes zeros)
     V* dst = reinterpret_cast<V*>(out + (size_t)t * row_bytes);
     V z;
     memset(&z, 0, sizeof(V));
@@ -590,6 +590,152 @@ shard_combine_kernel(const uint8_t* __restrict__ gathered, int record_bytes,
   }
 }
 
+// ------------------------------------------------------------------ expert parallel
+// Experts are split over `world` ranks, rank r owning experts [r L, r L + L)
+// (L = N / world); the tokens of one global batch are split by contiguous
+// ranges as in shard_combine_kernel.  From the gathered exchange records every
+// rank knows, for every rank g and expert e, how many of g's tokens of e are
+// kept: m[g][e] = min(count[g][e], max(0, C - offset[g][e])), the kept global
+// positions of e being [offset[g][e], offset[g][e] + m[g][e]).  Rank g sends
+// its kept rows packed by expert (its own packed buffer), so the rows for owner
+// r form one contiguous segment; the owner receives, source by source, blocks
+// (g, local expert l) of m[g][e] rows, and ep_plan_kernel lays out where each
+// block goes in the owner's per-expert packed buffer: expert e's rows in global
+// position order (source rank, then token order), exactly the rows and order
+// of the unsharded layer.
+__global__ void __launch_bounds__(kCombineThreads)
+ep_plan_kernel(const uint8_t* __restrict__ gathered, int record_bytes, int record_psum_offset,
+               int rank, int world, int L, int C_cap, int tile_rows, int* __restrict__ blk_src,
+               int* __restrict__ blk_dst, int* __restrict__ blk_n, int* __restrict__ ep_rows,
+               int* __restrict__ ep_base, int* __restrict__ ep_tile_prefix,
+               int* __restrict__ ready, int max_rows, WsHeader* hdr) {
+  __shared__ int s_warp[kCombineWarps];
+  __shared__ int s_tot_rows, s_tot_tiles, s_seg_total;
+  pdl_trigger();
+  pdl_wait();
+  const int chunk = (L + kCombineThreads - 1) / kCombineThreads;
+  const int l0 = threadIdx.x * chunk, l1 = min(L, l0 + chunk);
+  // per local expert: the kept rows of every source (their positions tile
+  // [0, K_e) in source order)
+  int rows = 0, tiles = 0;
+  for (int l = l0; l < l1; ++l) {
+    const int e = rank * L + l;
+    long long before = 0;
+    int kept = 0;
+    for (int g = 0; g < world; ++g) {
+      const int c = reinterpret_cast<const int*>(gathered + static_cast<size_t>(g) * record_bytes)[e];
+      const long long room = static_cast<long long>(C_cap) - before;
+      const int m = static_cast<int>(max(0ll, min(static_cast<long long>(c), room)));
+      blk_n[g * L + l] = m;
+      blk_dst[g * L + l] = static_cast<int>(min(before, static_cast<long long>(C_cap)));
+      before += c;
+      kept += m;
+    }
+    ep_rows[l] = kept;
+    rows += kept;
+    tiles += (kept + tile_rows - 1) / tile_rows;
+  }
+  int base_rows = block_excl_scan(rows, s_warp, &s_tot_rows);
+  int base_tiles = block_excl_scan(tiles, s_warp, &s_tot_tiles);
+  for (int l = l0; l < l1; ++l) {
+    ep_base[l] = base_rows;
+    ep_tile_prefix[l] = base_tiles;
+    for (int g = 0; g < world; ++g) blk_dst[g * L + l] += base_rows;
+    base_rows += ep_rows[l];
+    base_tiles += (ep_rows[l] + tile_rows - 1) / tile_rows;
+  }
+  // receive order: source g, then local expert l; blk_src = exclusive prefix
+  int seg_base = 0;
+  for (int g = 0; g < world; ++g) {
+    int part = 0;
+    for (int l = l0; l < l1; ++l) part += blk_n[g * L + l];
+    int off = block_excl_scan(part, s_warp, &s_seg_total) + seg_base;
+    for (int l = l0; l < l1; ++l) {
+      blk_src[g * L + l] = off;
+      off += blk_n[g * L + l];
+    }
+    seg_base += s_seg_total;
+    __syncthreads();
+  }
+  if (s_tot_rows > max_rows) atomicExch(&hdr->err, kDevIndexOutOfRange);   // cannot happen
+  for (int i = threadIdx.x; i < s_tot_tiles; i += kCombineThreads) ready[i] = 0;
+  if (threadIdx.x == 0) {
+    ep_tile_prefix[L] = s_tot_tiles;
+    hdr->next_tile = 0u;
+  }
+}
+
+// Moves rows between the receive order (source rank, local expert) and the
+// owner's per-expert packed buffer: dir 0 copies recv[i] to packed[dst], dir 1
+// copies packed[dst] back to recv[i] (the return trip).  One warp per row i of
+// the receive order; its block is the last entry whose start is <= i.
+template <int VEC>
+__global__ void __launch_bounds__(kGatherThreads)
+ep_permute_kernel(uint8_t* __restrict__ recv, uint8_t* __restrict__ packed,
+                  const int* __restrict__ blk_src, const int* __restrict__ blk_dst,
+                  const int* __restrict__ blk_n, int nblocks, int n_recv, int max_rows,
+                  int row_bytes, int dir, WsHeader* hdr) {
+  using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kGatherWarps + warp;
+  const int total = blk_src[nblocks - 1] + blk_n[nblocks - 1];
+  if (i >= total) return;
+  if (i >= n_recv) {              // more rows than the caller's receive buffer holds
+    if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
+    return;
+  }
+  int lo = 0, hi = nblocks;       // last j with blk_src[j] <= i
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (blk_src[mid] <= i) lo = mid; else hi = mid;
+  }
+  const int row = blk_dst[lo] + (i - blk_src[lo]);
+  if (row < 0 || row >= max_rows) {
+    if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
+    return;
+  }
+  const int nv = row_bytes / VEC;
+  V* r = reinterpret_cast<V*>(recv + static_cast<size_t>(i) * row_bytes);
+  V* p = reinterpret_cast<V*>(packed + static_cast<size_t>(row) * row_bytes);
+  if (dir == 0) {
+    for (int j = lane; j < nv; j += 32) p[j] = r[j];
+  } else {
+    for (int j = lane; j < nv; j += 32) r[j] = p[j];
+  }
+}
+
+// Source side of the return trip: the rows came back in this rank's packed
+// order (expert, then token order): out[t] = g_t * row for a kept token, zero
+// for a dropped one.  One warp per token.
+template <typename TA>
+__global__ void __launch_bounds__(kGatherThreads)
+ep_combine_kernel(const TA* __restrict__ ret, const int* __restrict__ expert_idx,
+                  const float* __restrict__ gate, const int* __restrict__ pos_in_expert,
+                  const int* __restrict__ exp_base, const int* __restrict__ exp_off,
+                  TA* __restrict__ out, int T, int d, int C_cmp, WsHeader* hdr) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kGatherWarps + warp;
+  if (t >= T) return;
+  const int e = expert_idx[t], pos = pos_in_expert[t];
+  TA* o = out + static_cast<size_t>(t) * d;
+  if (pos < C_cmp) {
+    const int row = exp_base[e] + pos - exp_off[e];
+    if (row < 0 || row >= T) {
+      if (lane == 0) atomicExch(&hdr->err, kDevIndexOutOfRange);
+      return;
+    }
+    const float g = gate[t];
+    const TA* y = ret + static_cast<size_t>(row) * d;
+    for (int j = lane; j < d; j += 32) o[j] = static_cast<TA>(g * static_cast<float>(y[j]));
+  } else {
+    for (int j = lane; j < d; j += 32) o[j] = static_cast<TA>(0.f);
+  }
+}
+
 }  // namespace
 
 bool dispatch_fused_ok(const Shape& s) {
@@ -684,6 +830,56 @@ cudaError_t launch_combine_top2(const Shape& s, const Workspace& ws, const int* 
     e = launch_dependent(combine_top2_kernel<float>, dim3(grid), dim3(kGatherThreads), 0,
                          stream, static_cast<const float*>(ws.ybuf), pos_in_expert,
                          static_cast<float*>(out), (int)s.T, (int)s.d, (int)s.C_cmp);
+  }
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_ep_plan(const EpPlan& ep, const void* gathered, cudaStream_t stream) {
+  const cudaError_t e = launch_dependent(
+      ep_plan_kernel, dim3(1), dim3(kCombineThreads), 0, stream,
+      static_cast<const uint8_t*>(gathered), (int)shard_record_bytes(ep.N),
+      (int)shard_record_psum_offset(ep.N), ep.rank, ep.world, ep.L, (int)ep.C_cmp,
+      ep.tile_rows, ep.blk_src, ep.blk_dst, ep.blk_n, ep.rows, ep.base, ep.tile_prefix, ep.ready,
+      (int)ep.max_rows, ep.hdr);
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_ep_permute(const EpPlan& ep, void* recv, void* packed, int64_t n_recv,
+                              int row_bytes, int dir, cudaStream_t stream) {
+  if (n_recv <= 0) return cudaSuccess;
+  const int grid = (int)((n_recv + kGatherWarps - 1) / kGatherWarps);
+  const bool vec16 = row_bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(recv) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(packed) & 15) == 0;
+  const cudaError_t e = launch_dependent(
+      vec16 ? ep_permute_kernel<16> : ep_permute_kernel<4>, dim3(grid), dim3(kGatherThreads), 0,
+      stream, static_cast<uint8_t*>(recv), static_cast<uint8_t*>(packed),
+      static_cast<const int*>(ep.blk_src), static_cast<const int*>(ep.blk_dst),
+      static_cast<const int*>(ep.blk_n), ep.world * ep.L, (int)n_recv, (int)ep.max_rows,
+      row_bytes, dir, ep.hdr);
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_ep_combine(const Shape& s, const Workspace& ws, const void* ret,
+                              const int* expert_idx, const float* gate,
+                              const int* pos_in_expert, void* out, cudaStream_t stream) {
+  if (s.T <= 0) return cudaSuccess;
+  const int grid = (int)((s.T + kGatherWarps - 1) / kGatherWarps);
+  cudaError_t e;
+  if (s.dtype == 1) {
+    e = launch_dependent(ep_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kGatherThreads), 0,
+                         stream, static_cast<const __nv_bfloat16*>(ret), expert_idx, gate,
+                         pos_in_expert, static_cast<const int*>(ws.exp_base),
+                         static_cast<const int*>(ws.exp_off), static_cast<__nv_bfloat16*>(out),
+                         (int)s.T, (int)s.d, (int)s.C_cmp, ws.hdr);
+  } else {
+    e = launch_dependent(ep_combine_kernel<float>, dim3(grid), dim3(kGatherThreads), 0, stream,
+                         static_cast<const float*>(ret), expert_idx, gate, pos_in_expert,
+                         static_cast<const int*>(ws.exp_base),
+                         static_cast<const int*>(ws.exp_off), static_cast<float*>(out),
+                         (int)s.T, (int)s.d, (int)s.C_cmp, ws.hdr);
   }
   count_launch();
   return e;

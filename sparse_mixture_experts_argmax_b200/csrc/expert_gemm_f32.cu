@@ -72,6 +72,8 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
     const float v = acc[i] + bm;
     if (mode == 0) {
       out[(size_t)(r0 + rr) * M + m] = fmaxf(v, 0.f);
+    } else if (mode == 2) {        // packed rows without the gate (expert-parallel)
+      out[(size_t)(r0 + rr) * M + m] = v;
     } else {
       const int tok = slot_token[r0 + rr];
       if (!checked_index(tok >= 0 && tok < T_rows, err)) continue;
@@ -96,7 +98,8 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
       static_cast<const float*>(bias), static_cast<const int*>(ws.tile_prefix),
       static_cast<const int*>(ws.exp_rows), static_cast<const int*>(ws.exp_base),
       static_cast<const int*>(ws.slot_token), gate, static_cast<float*>(out),
-      static_cast<int>(s.N), M, K, which, static_cast<int>(s.T * s.topk), &ws.hdr->err);
+      static_cast<int>(s.N), M, K, which == 1 && gate == nullptr ? 2 : which,
+      static_cast<int>(s.T * s.topk), &ws.hdr->err);
   count_launch();
   return e;
 }

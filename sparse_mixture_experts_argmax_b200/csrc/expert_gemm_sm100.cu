@@ -65,7 +65,9 @@ struct PhaseArgs {
   int M;          // output features per expert
   int m_tiles;    // ceil(M / 128)
   int k_blocks;   // ceil(K / 64)
-  int mode;       // 0: bias + ReLU, packed rows; 1: bias, gate, scatter to token rows
+  int mode;       // 0: bias + ReLU, packed rows; 1: bias, gate, scatter to token rows;
+                  // 2: bias only, packed rows (expert-parallel: the gate is applied
+                  //    on the rank that holds the token)
 };
 
 struct FfnArgs {
@@ -546,7 +548,7 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
     a.ph[p].M = static_cast<int>(M);
     a.ph[p].m_tiles = static_cast<int>((M + kBM - 1) / kBM);
     a.ph[p].k_blocks = static_cast<int>((K + kBK - 1) / kBK);
-    a.ph[p].mode = p;
+    a.ph[p].mode = p == 0 ? 0 : (gate != nullptr ? 1 : 2);
   }
   int stages = kMaxStages;
   while (stages > 2 && ffn_smem_bytes(a.bn, stages, 0) > kMaxSmem) --stages;

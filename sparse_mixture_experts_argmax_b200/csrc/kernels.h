@@ -146,6 +146,32 @@ cudaError_t launch_shard_combine(const Shape& s, const Workspace& ws, const void
 cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const void* x,
                                    const int* expert_idx, int* pos_in_expert, void* out,
                                    cudaStream_t stream);
+// Expert parallelism: where the owner rank's received rows go (see
+// ep_plan_kernel in dispatch.cu).  The arrays live in the owner's workspace.
+struct EpPlan {
+  int64_t N;        // experts of the layer
+  int world, rank;  // ranks; this rank owns experts [rank L, rank L + L)
+  int L;            // experts per rank
+  int64_t C_cmp;    // min(C, T_total)
+  int64_t max_rows; // rows of the owner's packed buffers: L * C_cmp
+  int tile_rows;
+  int* blk_src;     // [world L] first receive row of block (source g, local expert l)
+  int* blk_dst;     // [world L] its first packed row
+  int* blk_n;       // [world L] its rows
+  int* rows;        // [L] kept rows of each local expert (all sources)
+  int* base;        // [L] first packed row of each local expert
+  int* tile_prefix; // [L + 1]
+  int* ready;       // [max_rows / 16 + L + 1]
+  WsHeader* hdr;
+};
+cudaError_t launch_ep_plan(const EpPlan& ep, const void* gathered, cudaStream_t stream);
+// dir 0: receive order -> packed buffer; dir 1: packed buffer -> receive order.
+cudaError_t launch_ep_permute(const EpPlan& ep, void* recv, void* packed, int64_t n_recv,
+                              int row_bytes, int dir, cudaStream_t stream);
+// Source side: out[t] = gate * returned row (kept) or 0 (dropped).
+cudaError_t launch_ep_combine(const Shape& s, const Workspace& ws, const void* ret,
+                              const int* expert_idx, const float* gate,
+                              const int* pos_in_expert, void* out, cudaStream_t stream);
 // Top-2: out[t] = sum over the token's kept assignments of their gated rows.
 cudaError_t launch_combine_top2(const Shape& s, const Workspace& ws, const int* pos_in_expert,
                                 void* out, cudaStream_t stream);
@@ -157,7 +183,8 @@ cudaError_t launch_dispatch_fused(const Shape& s, const Workspace& ws, const voi
                                   const int* expert_idx, int* pos_in_expert, void* out,
                                   float* aux_loss, cudaStream_t stream);
 // Both expert GEMMs (bf16, tcgen05) in one persistent launch: GEMM1 + bias + ReLU
-// into hbuf, GEMM2 + bias + gate scattered to out.
+// into hbuf, GEMM2 + bias + gate scattered to out (gate == nullptr: GEMM2 +
+// bias written to the packed rows of out, for the expert-parallel path).
 cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CUtensorMap& tmA1,
                                    const CUtensorMap& tmB1, const CUtensorMap& tmA2,
                                    const CUtensorMap& tmB2, const void* b1, const void* b2,

@@ -193,6 +193,54 @@ static swl_status make_shard_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N
   return SWL_OK;
 }
 
+// Expert parallelism: the owner-side region of the workspace, after the
+// layout of this rank's own tokens (a shard of the global batch).
+struct EpLayout {
+  EpPlan plan;
+  void* xbuf;   // [max_rows, d] received rows, packed by local expert
+  void* hbuf;   // [max_rows, d_ff]
+  void* ybuf;   // [max_rows, d] expert outputs (bias, no gate)
+  size_t total_bytes;
+};
+
+static swl_status ep_check(int64_t N, int world, int rank) {
+  if (world < 1 || rank < 0 || rank >= world || N % world != 0) return SWL_ERR_INVALID_ARG;
+  return SWL_OK;
+}
+
+static EpLayout ep_layout(const Shape& s, int world, int rank, uintptr_t base) {
+  EpLayout e{};
+  const size_t elem = s.dtype == SWL_BF16 ? 2 : 4;
+  size_t off = workspace_layout(s, false, 0, nullptr);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return base + o;
+  };
+  const int L = static_cast<int>(s.N / world);
+  e.plan.N = s.N;
+  e.plan.world = world;
+  e.plan.rank = rank;
+  e.plan.L = L;
+  e.plan.C_cmp = s.C_cmp;
+  e.plan.max_rows = static_cast<int64_t>(L) * s.C_cmp;
+  e.plan.tile_rows = s.dtype == SWL_BF16 ? bf16_tile_rows(s.C_cmp) : kF32TileRows;
+  const size_t WL = static_cast<size_t>(world) * L, R = static_cast<size_t>(e.plan.max_rows);
+  e.plan.blk_src = reinterpret_cast<int*>(take(WL * 4));
+  e.plan.blk_dst = reinterpret_cast<int*>(take(WL * 4));
+  e.plan.blk_n = reinterpret_cast<int*>(take(WL * 4));
+  e.plan.rows = reinterpret_cast<int*>(take(static_cast<size_t>(L) * 4));
+  e.plan.base = reinterpret_cast<int*>(take(static_cast<size_t>(L) * 4));
+  e.plan.tile_prefix = reinterpret_cast<int*>(take(static_cast<size_t>(L + 1) * 4));
+  e.plan.ready = reinterpret_cast<int*>(take((R / 16 + L + 1) * 4));
+  e.plan.hdr = reinterpret_cast<WsHeader*>(base);   // shared with this rank's own stages
+  e.xbuf = reinterpret_cast<void*>(take(R * static_cast<size_t>(s.d) * elem));
+  e.hbuf = reinterpret_cast<void*>(take(R * static_cast<size_t>(s.d_ff) * elem));
+  e.ybuf = reinterpret_cast<void*>(take(R * static_cast<size_t>(s.d) * elem));
+  e.total_bytes = off;
+  return e;
+}
+
 // Stages 0-1: router logits, softmax, argmax, gate, block ranks and statistics.
 // rec(k) records stage event k (a no-op without events).
 template <typename Rec>
@@ -674,6 +722,175 @@ swl_status switch_layer_forward_shard_end(int64_t T, int64_t d, int64_t d_ff, in
   if (launch_dispatch_gather(s, ws, x, expert_idx, pos_in_expert, out, stream) != cudaSuccess)
     return SWL_ERR_CUDA;
   return run_ffn(s, ws, W1, b1, W2, b2, gate, out, stream);
+}
+
+int64_t switch_layer_ep_max_recv_rows(int64_t N, int world, int64_t T_total,
+                                      double capacity_factor) {
+  if (N <= 0 || world < 1 || N % world != 0 || T_total < 0) return -1;
+  const int64_t C = switch_layer_capacity(T_total, N, capacity_factor);
+  if (C < 0) return -1;
+  return (N / world) * (C < T_total ? C : T_total);
+}
+
+swl_status switch_layer_ep_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                          int dtype, int world, int64_t T_total,
+                                          double capacity_factor, size_t* bytes) {
+  if (!bytes) return SWL_ERR_INVALID_ARG;
+  swl_status st = ep_check(N, world, 0);
+  if (st != SWL_OK) return st;
+  Shape s;
+  st = make_shard_shape(T, d, d_ff, N, dtype, T_total, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  *bytes = ep_layout(s, world, 0, 0).total_bytes;
+  return SWL_OK;
+}
+
+swl_status switch_layer_ep_counts(int64_t N, int world, int rank, int64_t T_total,
+                                  double capacity_factor, const void* gathered_host,
+                                  int64_t* send_rows, int64_t* recv_rows) {
+  swl_status st = ep_check(N, world, rank);
+  if (st != SWL_OK) return st;
+  if (!gathered_host || !send_rows || !recv_rows || T_total < 0) return SWL_ERR_INVALID_ARG;
+  const int64_t C = switch_layer_capacity(T_total, N, capacity_factor);
+  if (C < 0) return SWL_ERR_INVALID_ARG;
+  const int64_t C_cmp = C < T_total ? C : T_total;
+  const size_t R = shard_record_bytes(N);
+  const int64_t L = N / world;
+  const uint8_t* g0 = static_cast<const uint8_t*>(gathered_host);
+  for (int r = 0; r < world; ++r) send_rows[r] = recv_rows[r] = 0;
+  for (int64_t e = 0; e < N; ++e) {
+    const int owner = static_cast<int>(e / L);
+    int64_t before = 0;
+    for (int g = 0; g < world; ++g) {
+      int32_t c;
+      std::memcpy(&c, g0 + static_cast<size_t>(g) * R + static_cast<size_t>(e) * 4, 4);
+      int64_t m = C_cmp - before;
+      if (m < 0) m = 0;
+      if (m > c) m = c;
+      if (g == rank) send_rows[owner] += m;       // my kept rows of e go to its owner
+      if (owner == rank) recv_rows[g] += m;       // g's kept rows of my expert e
+      before += c;
+    }
+  }
+  return SWL_OK;
+}
+
+swl_status switch_layer_ep_dispatch(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                    int world, int rank, int64_t T_total,
+                                    double capacity_factor, const void* gathered, const void* x,
+                                    int32_t* expert_idx, int32_t* pos_in_expert,
+                                    float* aux_loss, void* send_rows, void* workspace,
+                                    size_t workspace_bytes, void* stream_v) {
+  swl_status st = ep_check(N, world, rank);
+  if (st != SWL_OK) return st;
+  Shape s;
+  st = make_shard_shape(T, d, d_ff, N, dtype, T_total, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (!gathered || !aux_loss || !workspace) return SWL_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !expert_idx || !pos_in_expert || !send_rows)) return SWL_ERR_INVALID_ARG;
+  const uintptr_t a = dtype == SWL_BF16 ? 16 : 4;
+  if (!aligned(workspace, 256) || !aligned(gathered, 16) || !aligned(x, a) ||
+      !aligned(send_rows, a) || !aligned(expert_idx, 4) || !aligned(pos_in_expert, 4) ||
+      !aligned(aux_loss, 4))
+    return SWL_ERR_UNSUPPORTED;
+  if (workspace_bytes < ep_layout(s, world, rank, 0).total_bytes) return SWL_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (T_total == 0) {
+    return cudaMemsetAsync(aux_loss, 0, sizeof(float), stream) == cudaSuccess ? SWL_OK
+                                                                              : SWL_ERR_CUDA;
+  }
+  Workspace ws;
+  workspace_layout(s, false, reinterpret_cast<uintptr_t>(workspace), &ws);
+  if (T == 0 && cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  if (launch_shard_combine(s, ws, gathered, rank, world, aux_loss, stream) != cudaSuccess)
+    return SWL_ERR_CUDA;
+  if (T == 0) return SWL_OK;
+  // this rank's kept rows, packed by expert: the send buffer (experts of one
+  // owner are consecutive, so each owner's rows form one segment)
+  Workspace wsend = ws;
+  wsend.xbuf = send_rows;
+  return launch_dispatch_gather(s, wsend, x, expert_idx, pos_in_expert, nullptr, stream) ==
+                 cudaSuccess
+             ? SWL_OK
+             : SWL_ERR_CUDA;
+}
+
+swl_status switch_layer_ep_experts(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                   int world, int rank, int64_t T_total, double capacity_factor,
+                                   const void* gathered, void* recv_rows, int64_t n_recv,
+                                   const void* W1_local, const void* b1_local,
+                                   const void* W2_local, const void* b2_local, void* ret_rows,
+                                   void* workspace, size_t workspace_bytes, void* stream_v) {
+  swl_status st = ep_check(N, world, rank);
+  if (st != SWL_OK) return st;
+  Shape s;
+  st = make_shard_shape(T, d, d_ff, N, dtype, T_total, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (!gathered || !W1_local || !b1_local || !W2_local || !b2_local || !workspace || n_recv < 0)
+    return SWL_ERR_INVALID_ARG;
+  if (n_recv > 0 && (!recv_rows || !ret_rows)) return SWL_ERR_INVALID_ARG;
+  const uintptr_t a = dtype == SWL_BF16 ? 16 : 4;
+  if (!aligned(workspace, 256) || !aligned(gathered, 16) || !aligned(recv_rows, a) ||
+      !aligned(ret_rows, a) || !aligned(W1_local, a) || !aligned(W2_local, a))
+    return SWL_ERR_UNSUPPORTED;
+  const EpLayout ep = ep_layout(s, world, rank, reinterpret_cast<uintptr_t>(workspace));
+  if (workspace_bytes < ep.total_bytes) return SWL_ERR_WORKSPACE;
+  if (n_recv > ep.plan.max_rows) return SWL_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (T_total == 0 || ep.plan.max_rows == 0) return SWL_OK;
+  const int row_bytes = static_cast<int>(d * (dtype == SWL_BF16 ? 2 : 4));
+  if (launch_ep_plan(ep.plan, gathered, stream) != cudaSuccess) return SWL_ERR_CUDA;
+  if (launch_ep_permute(ep.plan, recv_rows, ep.xbuf, n_recv, row_bytes, 0, stream) !=
+      cudaSuccess)
+    return SWL_ERR_CUDA;
+  // the owner's experts over their packed rows: an ordinary FFN of L experts
+  // and max_rows rows whose GEMM2 writes bias-added packed rows (no gate)
+  Shape so = s;
+  so.T = ep.plan.max_rows;
+  so.N = ep.plan.L;
+  so.topk = 1;
+  so.tile_rows = ep.plan.tile_rows;
+  Workspace wo{};
+  wo.hdr = ep.plan.hdr;
+  wo.tile_prefix = ep.plan.tile_prefix;
+  wo.exp_rows = ep.plan.rows;
+  wo.exp_base = ep.plan.base;
+  wo.ready = ep.plan.ready;
+  wo.xbuf = ep.xbuf;
+  wo.hbuf = ep.hbuf;
+  st = run_ffn(so, wo, W1_local, b1_local, W2_local, b2_local, nullptr, ep.ybuf, stream);
+  if (st != SWL_OK) return st;
+  return launch_ep_permute(ep.plan, ret_rows, ep.ybuf, n_recv, row_bytes, 1, stream) ==
+                 cudaSuccess
+             ? SWL_OK
+             : SWL_ERR_CUDA;
+}
+
+swl_status switch_layer_ep_combine(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                   int world, int rank, int64_t T_total,
+                                   double capacity_factor, const void* ret_rows,
+                                   const int32_t* expert_idx, const float* gate,
+                                   const int32_t* pos_in_expert, void* out, void* workspace,
+                                   size_t workspace_bytes, void* stream_v) {
+  swl_status st = ep_check(N, world, rank);
+  if (st != SWL_OK) return st;
+  Shape s;
+  st = make_shard_shape(T, d, d_ff, N, dtype, T_total, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (!workspace) return SWL_ERR_INVALID_ARG;
+  if (T > 0 && (!ret_rows || !expert_idx || !gate || !pos_in_expert || !out))
+    return SWL_ERR_INVALID_ARG;
+  const uintptr_t a = dtype == SWL_BF16 ? 16 : 4;
+  if (!aligned(workspace, 256) || !aligned(ret_rows, a) || !aligned(out, a))
+    return SWL_ERR_UNSUPPORTED;
+  if (workspace_bytes < ep_layout(s, world, rank, 0).total_bytes) return SWL_ERR_WORKSPACE;
+  Workspace ws;
+  workspace_layout(s, false, reinterpret_cast<uintptr_t>(workspace), &ws);
+  return launch_ep_combine(s, ws, ret_rows, expert_idx, gate, pos_in_expert, out,
+                           static_cast<cudaStream_t>(stream_v)) == cudaSuccess
+             ? SWL_OK
+             : SWL_ERR_CUDA;
 }
 
 swl_status switch_layer_noalloc_status(void* stream) {

@@ -86,6 +86,19 @@ def exchange_records(info: RankInfo, record: torch.Tensor) -> torch.Tensor:
     return out
 
 
+def alltoall_rows(info: RankInfo, rows: torch.Tensor, send_counts, recv_counts) -> torch.Tensor:
+    """Row blocks between ranks: block g of ``rows`` (send_counts[g] rows) goes
+    to rank g; the result holds recv_counts[g] rows from each rank g, in rank
+    order (expert-parallel dispatch and return)."""
+    if not info.distributed:
+        return rows.clone()
+    out = torch.empty((int(sum(recv_counts)),) + tuple(rows.shape[1:]), dtype=rows.dtype,
+                      device=rows.device)
+    dist.all_to_all_single(out, rows.contiguous(), output_split_sizes=[int(c) for c in recv_counts],
+                           input_split_sizes=[int(c) for c in send_counts])
+    return out
+
+
 def token_range(info: RankInfo, T_per_rank: int) -> tuple:
     """[start, stop) of this rank's tokens in a global batch of world * T_per_rank."""
     return info.rank * T_per_rank, (info.rank + 1) * T_per_rank

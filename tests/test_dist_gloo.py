@@ -158,3 +158,63 @@ def test_sharded_batch_routing_equals_unsharded(world):
     assert all(o["C"] == ref["capacity"] for o in outs)
     assert len({o["aux"] for o in outs}) == 1
     assert abs(outs[0]["aux"] - ref["aux"]) <= 1e-13 * ref["aux"]
+
+
+# ---------------------------------------------------------------------------
+# expert parallelism: per-peer row counts from the gathered records, and the
+# row all-to-all that carries kept tokens to the owners of their experts
+# ---------------------------------------------------------------------------
+EP_WORKER = textwrap.dedent("""
+    import sys, json
+    sys.path.insert(0, %r)
+    import numpy as np, torch
+    import sparse_mixture_experts_argmax_b200 as swl
+    from sparse_mixture_experts_argmax_b200 import dist as d
+    info = d.init("gloo", timeout_s=60)
+    W, N, cf = info.world_size, 6, 1.0
+    rng = np.random.default_rng(5)
+    counts = rng.integers(0, 9, size=(W, N)).astype(np.int32)     # every rank's record
+    T_total = int(counts.sum())
+    R = swl.switch_layer_shard_record_bytes(N)
+    rec = np.zeros(R, dtype=np.uint8)
+    rec[:4 * N] = counts[info.rank].view(np.uint8)
+    gathered = d.exchange_records(info, torch.from_numpy(rec))
+    send, recv = swl.switch_layer_ep_counts(N, W, info.rank, T_total, cf, gathered)
+    # rows labelled (source rank, expert, global position), packed by expert
+    C = swl.switch_layer_capacity(T_total, N, cf)
+    before = counts[:info.rank].sum(axis=0)
+    labels = []
+    for e in range(N):
+        m = max(0, min(int(counts[info.rank, e]), C - int(before[e])))
+        labels += [[info.rank, e, int(before[e]) + j] for j in range(m)]
+    rows = torch.tensor(labels, dtype=torch.int64).reshape(-1, 3)
+    got = d.alltoall_rows(info, rows, send, recv)
+    print(json.dumps({"rank": info.rank, "send": send, "recv": recv, "got": got.tolist(),
+                      "C": C, "counts": counts.tolist()}), flush=True)
+    d.finalize(info)
+""") % ROOT
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_expert_parallel_counts_and_row_exchange(world):
+    """Every rank's send count to a peer equals that peer's receive count from
+    it, and each owner receives exactly the kept (expert, position) pairs of
+    its experts, source by source, positions ascending: the global position
+    order of the unsharded layer once permuted per expert."""
+    outs = _run_ranks(EP_WORKER, world)
+    N = 6
+    L = N // world
+    counts = outs[0]["counts"]
+    C = outs[0]["C"]
+    for g in range(world):
+        for r in range(world):
+            assert outs[g]["send"][r] == outs[r]["recv"][g]
+    for r in range(world):
+        got = outs[r]["got"]
+        want = []
+        for g in range(world):
+            for e in range(r * L, r * L + L):
+                before = sum(counts[h][e] for h in range(g))
+                m = max(0, min(counts[g][e], C - before))
+                want += [[g, e, before + j] for j in range(m)]
+        assert got == want
