@@ -53,6 +53,18 @@ Top-2 variant (the earlier-MoE routing the pages compare Switch with):
   position >= C; a token's output sums its kept assignments.
 * f_i still counts the argmax (first choice), as the loss formula's indicator
   does; P_i is the mean router probability.
+
+GEGLU experts and router input jitter ([ST-paper] architecture paragraph: "ReLU
+or GEGLU"; Table 11: input jitter, multiplicative noise on the router input,
+a training-time exploration, off at inference).  The pages name both without
+defining them; the readings taken:
+
+* GEGLU expert: E(x) = W_2 (GELU(W_g x + b_g) * (W_v x + b_v)) + b_2, stored as
+  W1 = [W_g; W_v] [2 d_ff, d] and b1 = [b_g; b_v] [2 d_ff], with the exact
+  GELU(u) = u Phi(u) = u (1 + erf(u / sqrt 2)) / 2.
+* jitter: the router sees x * n for a caller-supplied multiplicative noise n
+  [T, d] (the noise law is not stated; the tests draw n ~ U(1 - eps, 1 + eps));
+  the experts see x itself.  No noise (None) is the inference layer.
 """
 from __future__ import annotations
 
@@ -140,6 +152,30 @@ def expert_ffn(x_rows, W1e, b1e, W2e, b2e) -> np.ndarray:
     return h @ _f64(W2e).T + _f64(b2e)[None, :]
 
 
+def gelu(u: np.ndarray) -> np.ndarray:
+    """GELU(u) = u Phi(u) = u (1 + erf(u / sqrt 2)) / 2 (the exact form)."""
+    from scipy.special import erf
+    u = np.asarray(u, dtype=np.float64)
+    return 0.5 * u * (1.0 + erf(u / math.sqrt(2.0)))
+
+
+def expert_ffn_geglu(x_rows, W1e, b1e, W2e, b2e) -> np.ndarray:
+    """GEGLU expert for rows of x: W1e = [W_g; W_v] [2 d_ff, d], b1e = [b_g; b_v];
+    (GELU(x W_g^T + b_g) * (x W_v^T + b_v)) W2^T + b2, float64."""
+    a = _f64(x_rows) @ _f64(W1e).T + _f64(b1e)[None, :]
+    d_ff = a.shape[1] // 2
+    h = gelu(a[:, :d_ff]) * a[:, d_ff:]
+    return h @ _f64(W2e).T + _f64(b2e)[None, :]
+
+
+def _ffn_of(activation: str):
+    if activation == "relu":
+        return expert_ffn
+    if activation == "geglu":
+        return expert_ffn_geglu
+    raise ValueError(activation)
+
+
 # ---------------------------------------------------------------------------
 # load-balancing loss ([ST-paper] "The loss formulation"; [LB-card])
 # ---------------------------------------------------------------------------
@@ -162,15 +198,19 @@ def aux_loss(f: np.ndarray, P: np.ndarray) -> float:
 # ---------------------------------------------------------------------------
 # the whole layer
 # ---------------------------------------------------------------------------
-def switch_forward(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None) -> Dict:
-    """Full forward pass in float64.
+def switch_forward(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None,
+                   activation: str = "relu", router_noise=None) -> Dict:
+    """Full forward pass in float64 (``activation``: "relu" or "geglu";
+    ``router_noise``: multiplicative noise [T, d] on the router input, or None).
 
     Returns out [T, d] (float64; zero rows for dropped tokens), expert_idx,
     gate, pos_in_expert, kept, capacity, f, P, aux, probs, logits."""
     xs = _f64(x)
     T = xs.shape[0]
     N = _f64(W_r).shape[0]
-    z = router_logits(xs, W_r, b_r)
+    ffn = _ffn_of(activation)
+    xr = xs if router_noise is None else xs * _f64(router_noise)
+    z = router_logits(xr, W_r, b_r)
     p = router_probs(z) if T else np.zeros((0, N))
     e, g = top1(p) if T else (np.zeros(0, np.int64), np.zeros(0))
     C = capacity(T, N, capacity_factor)
@@ -181,7 +221,7 @@ def switch_forward(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None) -> 
         rows = np.nonzero((e == i) & kept)[0]
         if rows.size == 0:
             continue
-        u = expert_ffn(xs[rows], W1[i], b1[i], W2[i], b2[i])
+        u = ffn(xs[rows], W1[i], b1[i], W2[i], b2[i])
         out[rows] = g[rows, None] * u
     f, P = load_balance_stats(e, p)
     aux = aux_loss(f, P) if T else 0.0
@@ -191,7 +231,7 @@ def switch_forward(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None) -> 
 
 def switch_forward_sampled(x, W_r, capacity_factor: float, sample_tokens,
                            expert_weights: Callable[[int], Dict], b_r=None,
-                           chunk: int = 4096) -> Dict:
+                           chunk: int = 4096, activation: str = "relu") -> Dict:
     """Routing for every token, expert outputs only for ``sample_tokens``.
 
     ``expert_weights(e)`` returns {"W1","b1","W2","b2"} of expert e, so large
@@ -225,7 +265,7 @@ def switch_forward_sampled(x, W_r, capacity_factor: float, sample_tokens,
             out[int(t)] = np.zeros(xs.shape[1])
     for i, toks in sorted(by_expert.items()):
         w = expert_weights(i)
-        u = expert_ffn(_f64(xs[toks]), w["W1"], w["b1"], w["W2"], w["b2"])
+        u = _ffn_of(activation)(_f64(xs[toks]), w["W1"], w["b1"], w["W2"], w["b2"])
         for j, t in enumerate(toks):
             out[t] = g_all[t] * u[j]
     return {"out_rows": out, "expert_idx": e_all, "gate": g_all, "pos_in_expert": pos,

@@ -441,11 +441,77 @@ def pin_top2_drops():
         assert np.allclose(cut["out"][t], want, rtol=1e-13, atol=1e-13)
 
 
+# ---------------------------------------------------------------------------
+# GEGLU experts and router input jitter
+# ---------------------------------------------------------------------------
+def pin_gelu():
+    """Exact GELU: torch's erf form (a library routine), GELU(u) - GELU(-u) = u,
+    GELU(0) = 0, and the limits u and 0 far from zero."""
+    u = np.linspace(-8, 8, 1001)
+    lib = F.gelu(torch.from_numpy(u), approximate="none").numpy()
+    assert np.allclose(S.gelu(u), lib, rtol=0, atol=1e-15)
+    assert np.allclose(S.gelu(u) - S.gelu(-u), u, rtol=0, atol=1e-14)
+    assert S.gelu(np.array([0.0]))[0] == 0.0
+    assert abs(S.gelu(np.array([40.0]))[0] - 40.0) < 1e-12 and S.gelu(np.array([-40.0]))[0] == 0
+
+
+def pin_geglu_special_cases():
+    """W_v = 0, b_v = 1: the GEGLU expert is the GELU FFN W2 GELU(W_g x + b_g) + b2
+    (torch linear / gelu); scaling the value branch by c scales E(x) - b2 by c."""
+    rng = np.random.default_rng(15)
+    T, d, d_ff = 17, 6, 5
+    x = rng.normal(size=(T, d))
+    Wg = rng.normal(size=(d_ff, d))
+    bg = rng.normal(size=d_ff) * 0.3
+    W2 = rng.normal(size=(d, d_ff))
+    b2 = rng.normal(size=d) * 0.1
+    W1 = np.concatenate([Wg, np.zeros((d_ff, d))])
+    b1 = np.concatenate([bg, np.ones(d_ff)])
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    ref = F.linear(F.gelu(F.linear(t(x), t(Wg), t(bg))), t(W2), t(b2)).numpy()
+    assert np.allclose(S.expert_ffn_geglu(x, W1, b1, W2, b2), ref, rtol=1e-13, atol=1e-13)
+    Wv = rng.normal(size=(d_ff, d))
+    bv = rng.normal(size=d_ff)
+    base = S.expert_ffn_geglu(x, np.concatenate([Wg, Wv]), np.concatenate([bg, bv]), W2, b2)
+    scaled = S.expert_ffn_geglu(x, np.concatenate([Wg, 3 * Wv]), np.concatenate([bg, 3 * bv]),
+                                W2, b2)
+    assert np.allclose(scaled - b2, 3 * (base - b2), rtol=1e-12, atol=1e-12)
+    # the layer with one expert and GEGLU is that expert's FFN
+    r = S.switch_forward(x, rng.normal(size=(1, d)), W1[None], b1[None], W2[None], b2[None], 1.0,
+                         activation="geglu")
+    assert np.allclose(r["out"], ref, rtol=1e-13, atol=1e-13)
+
+
+def pin_router_jitter():
+    """Jitter multiplies the router input only.  Unit noise is the inference
+    layer; a constant noise c scales every logit by c (gate = max softmax(c z),
+    torch), while the experts still see x itself."""
+    rng = np.random.default_rng(16)
+    T, d, d_ff, N = 30, 6, 7, 4
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(N, d))
+    W1, b1, W2, b2 = _rand_ffn(rng, N, d, d_ff)
+    plain = S.switch_forward(x, Wr, W1, b1, W2, b2, float(N))
+    ones = S.switch_forward(x, Wr, W1, b1, W2, b2, float(N), router_noise=np.ones((T, d)))
+    for k in ("out", "gate", "expert_idx", "aux"):
+        assert np.array_equal(np.asarray(plain[k]), np.asarray(ones[k])), k
+    c = 3.5
+    r = S.switch_forward(x, Wr, W1, b1, W2, b2, float(N), router_noise=np.full((T, d), c))
+    z = c * (torch.from_numpy(x) @ torch.from_numpy(Wr).T)
+    g = torch.softmax(z, dim=1).max(dim=1).values.numpy()
+    e = z.argmax(dim=1).numpy()
+    assert np.array_equal(r["expert_idx"], e)
+    assert np.allclose(r["gate"], g, rtol=0, atol=1e-15)
+    for t0 in range(T):
+        want = g[t0] * _torch_ffn(x[t0:t0 + 1], W1[e[t0]], b1[e[t0]], W2[e[t0]], b2[e[t0]])[0]
+        assert np.allclose(r["out"][t0], want, rtol=1e-13, atol=1e-13)
+
+
 ALL_PINS = [
     pin_lb_worked_example, pin_even_routing_is_one, pin_collapse_tends_to_N,
     pin_not_a_lower_bound, pin_softmax_rows_and_closed_form, pin_ties_lowest_index,
     pin_capacity, pin_positions_bruteforce, pin_drops, pin_single_expert_is_dense_ffn,
     pin_identical_experts_scale_by_gate, pin_sampled_matches_full, pin_logit_gap,
     pin_top2_worked_example, pin_top2_choices_and_capacity, pin_top2_positions_bruteforce,
-    pin_top2_closed_forms, pin_top2_drops,
+    pin_top2_closed_forms, pin_top2_drops, pin_gelu, pin_geglu_special_cases, pin_router_jitter,
 ]

@@ -125,6 +125,26 @@ def _positions_top2_firsts_first(e, N):
     return pos
 
 
+def _gelu_tanh(u):
+    u = np.asarray(u, dtype=np.float64)
+    return 0.5 * u * (1 + np.tanh(np.sqrt(2 / np.pi) * (u + 0.044715 * u ** 3)))
+
+
+def _geglu_gate_on_value(x_rows, W1e, b1e, W2e, b2e):
+    a = S._f64(x_rows) @ S._f64(W1e).T + S._f64(b1e)[None, :]
+    d_ff = a.shape[1] // 2
+    h = a[:, :d_ff] * S.gelu(a[:, d_ff:])
+    return h @ S._f64(W2e).T + S._f64(b2e)[None, :]
+
+
+def _forward_noise_everywhere(x, W_r, W1, b1, W2, b2, capacity_factor, b_r=None,
+                              activation="relu", router_noise=None):
+    # mistake: the experts also see the jittered input
+    xs = x if router_noise is None else S._f64(x) * S._f64(router_noise)
+    return _orig_forward(xs, W_r, W1, b1, W2, b2, capacity_factor, b_r=b_r,
+                         activation=activation)
+
+
 MUTATIONS = {
     "ties_to_highest": ("top1", _top1_highest_tie),
     "positions_one_based": ("positions", _positions_one_based),
@@ -144,7 +164,12 @@ MUTATIONS = {
     "top2_never_normalised": ("top2", _top2_never_normalised),
     "top2_capacity_ignores_k": ("capacity_k", _capacity_k_ignores_k),
     "top2_firsts_first": ("positions_top2", _positions_top2_firsts_first),
+    "gelu_tanh_approximation": ("gelu", _gelu_tanh),
+    "geglu_gate_on_value": ("expert_ffn_geglu", _geglu_gate_on_value),
+    "jitter_reaches_experts": ("switch_forward", _forward_noise_everywhere),
 }
+
+_orig_forward = S.switch_forward
 
 _orig_top2 = S.top2
 
