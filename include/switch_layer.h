@@ -145,6 +145,41 @@ swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t
                                      float* aux_loss, const float* b_r, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* Layer variants the pages name beside the Switch layer, in one call:
+ *   top_k = 2     the top-2 routing of switch_layer_forward_top2 (routing outputs
+ *                 [T, 2]), with normalize as there;
+ *   activation    SWL_ACT_RELU (the Switch expert) or SWL_ACT_GEGLU: the paper-graph
+ *                 summary's "ReLU or GEGLU" expert, read as
+ *                 E(x) = W2 (GELU(W_g x + b_g) * (W_v x + b_v)) + b2 with the exact
+ *                 GELU(u) = u Phi(u); W1 is then [N, 2 d_ff, d] (W_g rows, then W_v
+ *                 rows) and b1 [N, 2 d_ff] (b_g, then b_v);
+ *   router_noise  NULL (inference), or [T, d] fp32 multiplicative noise on the
+ *                 router input ("input jitter", Table 11 of the paper-graph
+ *                 summary, a training-time exploration): the router sees x * noise
+ *                 (fp32, routed with the FFMA router), the experts see x.
+ * A NULL variant is switch_layer_forward.  The workspace is sized by
+ * switch_layer_variant_workspace_size with the same variant (only whether
+ * router_noise is NULL matters there).  Invalid fields: SWL_ERR_INVALID_ARG. */
+#define SWL_ACT_RELU 0
+#define SWL_ACT_GEGLU 1
+typedef struct swl_variant {
+  int top_k;
+  int normalize;
+  int activation;
+  const float* router_noise;
+} swl_variant;
+swl_status switch_layer_variant_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                               int dtype, double capacity_factor,
+                                               const swl_variant* variant, size_t* bytes);
+swl_status switch_layer_forward_variant(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                        int dtype, const void* x, const float* W_r,
+                                        const void* W1, const void* b1, const void* W2,
+                                        const void* b2, double capacity_factor, void* out,
+                                        int32_t* expert_idx, float* gate,
+                                        int32_t* pos_in_expert, float* aux_loss,
+                                        const float* b_r, const swl_variant* variant,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* As switch_layer_forward, and records cudaEvent_t stage_events[k] on `stream`
  * before stage 0 (k = 0) and after stage k-1 (k = 1..SWL_NUM_STAGES): an array
  * of SWL_NUM_STAGES + 1 events created by the caller (timing enabled). */

@@ -43,7 +43,15 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_set_wait_limit_ns", "switch_layer_set_stall_test",
            "switch_layer_forward_top2", "switch_layer_ep_max_recv_rows",
            "switch_layer_ep_workspace_size", "switch_layer_ep_counts",
-           "switch_layer_ep_dispatch", "switch_layer_ep_experts", "switch_layer_ep_combine")
+           "switch_layer_ep_dispatch", "switch_layer_ep_experts", "switch_layer_ep_combine",
+           "switch_layer_variant_workspace_size", "switch_layer_forward_variant")
+SWL_ACT_RELU, SWL_ACT_GEGLU = 0, 1
+
+
+class Variant(ctypes.Structure):
+    """struct swl_variant of include/switch_layer.h."""
+    _fields_ = [("top_k", ctypes.c_int), ("normalize", ctypes.c_int),
+                ("activation", ctypes.c_int), ("router_noise", ctypes.c_void_p)]
 SWL_ROUTER_TENSOR = 0
 SWL_ROUTER_FFMA = 1
 SWL_NOALLOC_MAX_BYTES = 64 << 20
@@ -125,6 +133,13 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_ep_combine.restype = _i32
     L.switch_layer_ep_combine.argtypes = [_i64, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _dbl,
                                           _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    L.switch_layer_variant_workspace_size.restype = _i32
+    L.switch_layer_variant_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i32, _dbl,
+                                                      ctypes.POINTER(Variant),
+                                                      ctypes.POINTER(_sz)]
+    L.switch_layer_forward_variant.restype = _i32
+    L.switch_layer_forward_variant.argtypes = (_FWD_ARGS[:18] + [ctypes.POINTER(Variant)] +
+                                               _FWD_ARGS[18:])
     L.switch_layer_forward_top2.restype = _i32
     L.switch_layer_forward_top2.argtypes = _FWD_ARGS[:12] + [_i32] + _FWD_ARGS[12:]
     L.switch_layer_set_wait_limit_ns.restype = _i32
@@ -579,4 +594,57 @@ def forward_ep(inputs: dict, capacity_factor: float, N: int, T_total: int, rank:
                             o["expert_idx"], o["gate"], o["pos_in_expert"], o["out"], ws, stream)
     if check:
         _check(switch_layer_device_status(ws, stream), "device status")
+    return o
+
+
+def make_variant(top_k: int = 1, normalize: bool = True, activation: str = "relu",
+                 router_noise: Optional[torch.Tensor] = None) -> Variant:
+    if router_noise is not None:
+        _require(router_noise, "router_noise", torch.float32)
+    return Variant(int(top_k), 1 if normalize else 0,
+                   {"relu": SWL_ACT_RELU, "geglu": SWL_ACT_GEGLU}[activation],
+                   None if router_noise is None else router_noise.data_ptr())
+
+
+def switch_layer_variant_workspace_size(T, d, d_ff, N, dtype, capacity_factor,
+                                        variant: Variant) -> int:
+    n = _sz(0)
+    _check(lib().switch_layer_variant_workspace_size(T, d, d_ff, N, dtype, capacity_factor,
+                                                     ctypes.byref(variant), ctypes.byref(n)),
+           "variant_workspace_size")
+    return int(n.value)
+
+
+def forward_variant(inputs: dict, capacity_factor: float, top_k: int = 1, normalize: bool = True,
+                    activation: str = "relu", router_noise: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None,
+                    check: bool = True) -> dict:
+    """Run a layer variant (top-2 routing, GEGLU experts, router input jitter)."""
+    x, W1 = inputs["x"], inputs["W1"]
+    T, d = x.shape
+    N = W1.shape[0]
+    d_ff = W1.shape[1] // (2 if activation == "geglu" else 1)
+    v = make_variant(top_k, normalize, activation, router_noise)
+    if workspace is None:
+        workspace = torch.empty(max(256, switch_layer_variant_workspace_size(
+            T, d, d_ff, N, dtype_code(x.dtype), capacity_factor, v)), dtype=torch.uint8,
+            device=x.device)
+    shape_k = (T, top_k) if top_k == 2 else (T,)
+    o = {"out": torch.empty((T, d), dtype=x.dtype, device=x.device),
+         "expert_idx": torch.empty(shape_k, dtype=torch.int32, device=x.device),
+         "gate": torch.empty(shape_k, dtype=torch.float32, device=x.device),
+         "pos_in_expert": torch.empty(shape_k, dtype=torch.int32, device=x.device),
+         "aux_loss": torch.empty(1, dtype=torch.float32, device=x.device)}
+    for t, n in ((x, "x"), (W1, "W1"), (inputs["b1"], "b1"), (inputs["W2"], "W2"),
+                 (inputs["b2"], "b2")):
+        _require(t, n, x.dtype)
+    _require(inputs["W_r"], "W_r", torch.float32)
+    _check(lib().switch_layer_forward_variant(
+        T, d, d_ff, N, dtype_code(x.dtype), _ptr(x), _ptr(inputs["W_r"]), _ptr(W1),
+        _ptr(inputs["b1"]), _ptr(inputs["W2"]), _ptr(inputs["b2"]), float(capacity_factor),
+        _ptr(o["out"]), _ptr(o["expert_idx"]), _ptr(o["gate"]), _ptr(o["pos_in_expert"]),
+        _ptr(o["aux_loss"]), _ptr(inputs.get("b_r")), ctypes.byref(v), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)), "forward_variant")
+    if check:
+        _check(switch_layer_device_status(workspace, stream), "device status")
     return o

@@ -19,6 +19,9 @@ namespace {
 
 constexpr int kTile = kF32TileRows;   // 32
 
+// GLU (GEMM1 of GEGLU experts): W is [N, 2M, K], gate rows then value rows;
+// out = GELU(gate + b_g) * (value + b_v) with the biases [N, 2M] laid out the same.
+template <bool GLU>
 __global__ void __launch_bounds__(256)
 expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ W,
                        const float* __restrict__ bias, const int* __restrict__ tile_prefix,
@@ -28,6 +31,7 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
                        int T_rows, int* err) {
   __shared__ float As[kTile][kTile + 1];   // [row][k]
   __shared__ float Ws[kTile][kTile + 1];   // [feature][k]
+  __shared__ float Wv[GLU ? kTile : 1][kTile + 1];   // value rows (GLU)
   pdl_trigger();
   pdl_wait();   // packed rows and tile prefix come from the dispatch
   const int g = blockIdx.x;
@@ -43,14 +47,18 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
   const int nrows = min(kTile, exp_rows[e] - nt * kTile);
   const int m0 = blockIdx.y * kTile;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // feature, row group
-  const float* We = W + (size_t)e * M * K;
+  const int rows_e = GLU ? 2 * M : M;       // weight rows (and biases) per expert
+  const float* We = W + (size_t)e * rows_e * K;
 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float accv[4] = {0.f, 0.f, 0.f, 0.f};
   for (int k0 = 0; k0 < K; k0 += kTile) {
     for (int i = threadIdx.x; i < kTile * kTile; i += 256) {
       const int rr = i / kTile, kk = i % kTile;
       As[rr][kk] = (rr < nrows && k0 + kk < K) ? act[(size_t)(r0 + rr) * K + k0 + kk] : 0.f;
       Ws[rr][kk] = (m0 + rr < M && k0 + kk < K) ? We[(size_t)(m0 + rr) * K + k0 + kk] : 0.f;
+      if (GLU)
+        Wv[rr][kk] = (m0 + rr < M && k0 + kk < K) ? We[(size_t)(M + m0 + rr) * K + k0 + kk] : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -58,12 +66,30 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
       const float w = Ws[tx][kk];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = fmaf(As[ty * 4 + i][kk], w, acc[i]);
+      if (GLU) {
+        const float wv = Wv[tx][kk];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) accv[i] = fmaf(As[ty * 4 + i][kk], wv, accv[i]);
+      }
     }
     __syncthreads();
   }
   const int m = m0 + tx;
   if (m >= M) return;
-  const float bm = bias[(size_t)e * M + m];
+  const float bm = bias[(size_t)e * rows_e + m];
+  if constexpr (GLU) {
+    const float bv = bias[(size_t)e * rows_e + M + m];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rr = ty * 4 + i;
+      if (rr >= nrows) continue;
+      if (!checked_index(r0 + rr >= 0 && r0 + rr < T_rows, err)) continue;
+      const float g = acc[i] + bm;
+      out[(size_t)(r0 + rr) * M + m] = 0.5f * g * (1.0f + erff(g * 0.70710678118654752f)) *
+                                       (accv[i] + bv);
+    }
+    return;
+  } else {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rr = ty * 4 + i;
@@ -80,6 +106,7 @@ expert_gemm_f32_kernel(const float* __restrict__ act, const float* __restrict__ 
       out[(size_t)tok * M + m] = gate[tok] * v;
     }
   }
+  }
 }
 
 }  // namespace
@@ -93,8 +120,10 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
   // upper bound on row tiles: sum_e ceil(m_e / 32) <= A / 32 + N (A = T * topk rows)
   const int64_t max_tiles = (s.T * s.topk + kTile - 1) / kTile + s.N;
   dim3 grid(static_cast<unsigned>(max_tiles), (M + kTile - 1) / kTile);
+  const bool glu = which == 0 && s.glu;
   const cudaError_t e = launch_dependent(
-      expert_gemm_f32_kernel, grid, dim3(256), 0, stream, act, static_cast<const float*>(W),
+      glu ? expert_gemm_f32_kernel<true> : expert_gemm_f32_kernel<false>, grid, dim3(256), 0,
+      stream, act, static_cast<const float*>(W),
       static_cast<const float*>(bias), static_cast<const int*>(ws.tile_prefix),
       static_cast<const int*>(ws.exp_rows), static_cast<const int*>(ws.exp_base),
       static_cast<const int*>(ws.slot_token), gate, static_cast<float*>(out),

@@ -63,6 +63,8 @@ struct PhaseArgs {
   const __nv_bfloat16* bias;   // [N, M]
   __nv_bfloat16* out;          // GEMM1: hbuf [T, M] (packed rows); GEMM2: out [T, M]
   int M;          // output features per expert
+  int a_rows;     // rows of the A operand per expert: M, or 2 M for GEGLU (gate rows,
+                  // then value rows); also the bias stride per expert
   int m_tiles;    // ceil(M / 128)
   int k_blocks;   // ceil(K / 64)
   int mode;       // 0: bias + ReLU, packed rows; 1: bias, gate, scatter to token rows;
@@ -88,6 +90,10 @@ struct FfnArgs {
   int bn;         // token rows per tile (multiple of 16, <= 256)
   int stages;
   int num_acc;    // TMEM accumulators: 4 of 128 columns when bn <= 128, else 2 of 256
+                  // (GEGLU: 512 / the next power of two >= max(128, 2 bn))
+  int glu;        // 1: GEMM1 is GEGLU: each tile multiplies the gate and the value
+                  // rows of W1 for the same 128 features into the two halves of
+                  // its accumulator, and the epilogue stores GELU(gate) * value
   PhaseArgs ph[2];
 };
 
@@ -154,8 +160,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int stages = args.stages;
   const uint32_t b_bytes = static_cast<uint32_t>(args.bn) * kBK * 2;
+  const uint32_t a_stage = args.glu ? 2 * kABytes : kABytes;   // A bytes per stage
   uint8_t* smem_a = smem;
-  uint8_t* smem_b = smem_a + stages * kABytes;
+  uint8_t* smem_b = smem_a + stages * a_stage;
   __nv_bfloat16* epi = reinterpret_cast<__nv_bfloat16*>(smem_b + stages * b_bytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(epi) + kEpiStageBytes);
   uint64_t* full_bar = bars;                      // [kMaxStages]
@@ -302,8 +309,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         // GEMM2 tile: the scheduler saw the hbuf rows published (generic-proxy
         // stores of other CTAs); order them before the TMA reads below
         if (ts.phase == 1) fence_proxy_async_global();
-        const int arow = ts.e * P.M + ts.mt * kBM;
+        const int arow = ts.e * P.a_rows + ts.mt * kBM;
         const int brow = ts.row0;
+        const bool two_a = args.glu && ts.phase == 0;   // gate and value rows
         if (!checked_index(ts.e >= 0 && ts.e < args.num_experts && brow >= 0 &&
                                brow + ts.rows <= args.T_rows && ts.rows > 0,
                            args.err)) {
@@ -312,8 +320,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         }
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + b_bytes);
-          ptx::tma_load_2d(smem_a + stage * kABytes, tA, &full_bar[stage], kb * kBK, arow, pol_w);
+          ptx::mbar_arrive_expect_tx(&full_bar[stage], (two_a ? 2 * kABytes : kABytes) + b_bytes);
+          ptx::tma_load_2d(smem_a + stage * a_stage, tA, &full_bar[stage], kb * kBK, arow, pol_w);
+          if (two_a)
+            ptx::tma_load_2d(smem_a + stage * a_stage + kABytes, tA, &full_bar[stage], kb * kBK,
+                             arow + P.M, pol_w);
           ptx::tma_load_2d(smem_b + stage * b_bytes, tB, &full_bar[stage], kb * kBK, brow, pol_x);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (ph << stage);
@@ -350,16 +361,22 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag, args.wait_ns)) { fail(); break; }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * acc_cols);
+        const bool two_a = args.glu && ts.phase == 0;   // value rows into the upper half
+        const uint32_t d_val = d_tmem + static_cast<uint32_t>(acc_cols / 2);
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t a_addr = ptx::smem_u32(smem_a + stage * kABytes);
+          const uint32_t a_addr = ptx::smem_u32(smem_a + stage * a_stage);
           const uint32_t b_addr = ptx::smem_u32(smem_b + stage * b_bytes);
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + k * kUmmaK * 2);
             const uint64_t bd = ptx::umma_desc_sw128_kmajor(b_addr + k * kUmmaK * 2);
             ptx::umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            if (two_a) {
+              const uint64_t av = ptx::umma_desc_sw128_kmajor(a_addr + kABytes + k * kUmmaK * 2);
+              ptx::umma_bf16(d_val, av, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
           }
           ptx::umma_commit(&empty_bar[stage]);      // frees the stage when these MMAs finish
           if (++stage == stages) { stage = 0; ph ^= 1u; }
@@ -422,7 +439,10 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       // this lane's bias, and the destination row / gate of column (c0 + lane)
       // of each of this warp's column chunks
       constexpr int kMaxChunks = 256 / 64;         // chunks of 32 per warp at 256 rows
-      const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.M + f]) : 0.f;
+      const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.a_rows + f]) : 0.f;
+      const bool glu = args.glu && ts.phase == 0;
+      const float bias_v =
+          (glu && f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.a_rows + P.M + f]) : 0.f;
       int dsts[kMaxChunks];
       float gs[kMaxChunks];
 #pragma unroll
@@ -457,16 +477,30 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         const float g = gs[k];
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
-        ptx::tmem_ld_wait();
+        if (glu) {
+          // GELU(gate) * value, the value accumulator in the upper half
+          uint32_t rv[32];
+          ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(acc_cols / 2 + c0), rv);
+          ptx::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float v = __uint_as_float(r[j]) + bias;
-          if (P.mode == 0) {
-            v = fmaxf(v, 0.f);
-          } else {
-            v *= __shfl_sync(0xffffffffu, g, j);
+          for (int j = 0; j < 32; ++j) {
+            const float gt = __uint_as_float(r[j]) + bias;
+            const float vl = __uint_as_float(rv[j]) + bias_v;
+            const float h = 0.5f * gt * (1.0f + erff(gt * 0.70710678118654752f)) * vl;
+            st[j * 32 + lane] = __float2bfloat16_rn(h);
           }
-          st[j * 32 + lane] = __float2bfloat16_rn(v);
+        } else {
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float v = __uint_as_float(r[j]) + bias;
+            if (P.mode == 0) {
+              v = fmaxf(v, 0.f);
+            } else {
+              v *= __shfl_sync(0xffffffffu, g, j);
+            }
+            st[j * 32 + lane] = __float2bfloat16_rn(v);
+          }
         }
         __syncwarp();
 #pragma unroll
@@ -503,9 +537,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   }
 }
 
-size_t ffn_smem_bytes(int bn, int stages, int cached_prefix_ints) {
+size_t ffn_smem_bytes(int bn, int stages, int cached_prefix_ints, int a_tiles = 1) {
   return 1024 + static_cast<size_t>(cached_prefix_ints) * sizeof(int) +
-         static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(bn) * kBK * 2) +
+         static_cast<size_t>(stages) * (a_tiles * kABytes + static_cast<size_t>(bn) * kBK * 2) +
          kEpiStageBytes + (2 * kMaxStages + 2 * kMaxAcc + 2 + 2 * kTileRing) * sizeof(uint64_t) +
          kTileRing * sizeof(TileSlot) + 2 * sizeof(uint32_t);
 }
@@ -539,24 +573,33 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.num_experts = static_cast<int>(s.N);
   a.T_rows = static_cast<int>(s.T * s.topk);   // packed rows; top-2 writes per assignment
   a.bn = s.tile_rows;
-  a.num_acc = a.bn <= kTmemCols / kMaxAcc ? kMaxAcc : 2;
+  a.glu = s.glu ? 1 : 0;
+  if (a.glu) {
+    int cols = 128;
+    while (cols < 2 * a.bn) cols *= 2;          // gate and value halves of one accumulator
+    a.num_acc = kTmemCols / cols;
+  } else {
+    a.num_acc = a.bn <= kTmemCols / kMaxAcc ? kMaxAcc : 2;
+  }
   for (int p = 0; p < 2; ++p) {
     const int64_t M = p == 0 ? s.d_ff : s.d;
     const int64_t K = p == 0 ? s.d : s.d_ff;
     a.ph[p].bias = static_cast<const __nv_bfloat16*>(p == 0 ? b1 : b2);
     a.ph[p].out = static_cast<__nv_bfloat16*>(p == 0 ? ws.hbuf : out);
     a.ph[p].M = static_cast<int>(M);
+    a.ph[p].a_rows = static_cast<int>(p == 0 && a.glu ? 2 * M : M);
     a.ph[p].m_tiles = static_cast<int>((M + kBM - 1) / kBM);
     a.ph[p].k_blocks = static_cast<int>((K + kBK - 1) / kBK);
     a.ph[p].mode = p == 0 ? 0 : (gate != nullptr ? 1 : 2);
   }
+  const int a_tiles = a.glu ? 2 : 1;
   int stages = kMaxStages;
-  while (stages > 2 && ffn_smem_bytes(a.bn, stages, 0) > kMaxSmem) --stages;
+  while (stages > 2 && ffn_smem_bytes(a.bn, stages, 0, a_tiles) > kMaxSmem) --stages;
   a.stages = stages;
   // the tile prefix goes to shared memory when it fits beside the stage ring
   const int prefix_ints = static_cast<int>(s.N) + 1;
-  a.cache_prefix = ffn_smem_bytes(a.bn, stages, prefix_ints) <= kMaxSmem ? 1 : 0;
-  const size_t smem = ffn_smem_bytes(a.bn, stages, a.cache_prefix ? prefix_ints : 0);
+  a.cache_prefix = ffn_smem_bytes(a.bn, stages, prefix_ints, a_tiles) <= kMaxSmem ? 1 : 0;
+  const size_t smem = ffn_smem_bytes(a.bn, stages, a.cache_prefix ? prefix_ints : 0, a_tiles);
   cudaError_t err = cudaFuncSetAttribute(expert_ffn_sm100_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

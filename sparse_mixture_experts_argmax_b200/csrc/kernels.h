@@ -46,6 +46,7 @@ struct Workspace {
   int* slot_token;      // [A] packed row -> assignment (token t, choice k: t * topk + k)
   int* ready;           // [T/16 + N + 1] per token tile: GEMM1 epilogue warps done
   void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
+  float* xj;            // jittered router input x * noise [T, d] fp32 (jitter only)
   void* xbuf;           // [A, d] packed expert inputs (act dtype), A = T * topk
   void* hbuf;           // [A, d_ff] packed hidden activations (act dtype)
   void* ybuf;           // top-2: [A, d] gated expert output per assignment (act dtype)
@@ -68,6 +69,8 @@ struct Shape {
   int64_t C_cmp;  // min(C, T_total): a token is kept iff its position is below it
   int sharded;    // 1: a shard of a global batch (positions offset by earlier ranks)
   int topk;       // experts per token: 1 (Switch) or 2 (the top-2 variant)
+  int glu;        // 1: GEGLU experts (W1 [N, 2 d_ff, d]: gate rows, then value rows)
+  int jitter;     // 1: the router sees x * noise (a jittered fp32 copy of x, FFMA router)
   int normalize;  // top-2: gates divided by their sum
   int router_path;  // RouterPath
   int tpb;        // tokens per block of the softmax / rank / gather stages (<= kTokensPerBlock)
@@ -102,6 +105,9 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
 // N <= kFusedRouterMaxN: one fused kernel (logits + softmax + block statistics);
 // launch_router_softmax is then not called.  Wider N: logits here, softmax after.
 constexpr int kFusedRouterMaxN = 128;
+// Jittered router input: ws.xj = x * noise (fp32, element by element).
+cudaError_t launch_router_jitter(const Shape& s, const Workspace& ws, const void* x,
+                                 const float* noise, cudaStream_t stream);
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
                                  const float* W_r, const float* b_r, int* expert_idx, float* gate,
                                  int* local_rank, cudaStream_t stream);

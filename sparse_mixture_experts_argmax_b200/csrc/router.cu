@@ -1204,11 +1204,36 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk) {
   return p;
 }
 
+template <typename TX>
+__global__ void __launch_bounds__(256)
+router_jitter_kernel(const TX* __restrict__ x, const float* __restrict__ noise,
+                     float* __restrict__ xj, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    xj[i] = static_cast<float>(x[i]) * noise[i];
+}
+
+cudaError_t launch_router_jitter(const Shape& s, const Workspace& ws, const void* x,
+                                 const float* noise, cudaStream_t stream) {
+  const size_t n = static_cast<size_t>(s.T) * static_cast<size_t>(s.d);
+  size_t blocks = (n + 255) / 256;
+  if (blocks > 8 * 148) blocks = 8 * 148;
+  if (blocks < 1) blocks = 1;
+  if (s.dtype == 1)
+    router_jitter_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), noise, ws.xj, n);
+  else
+    router_jitter_kernel<float><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const float*>(x), noise, ws.xj, n);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits(const Shape& s, const Workspace& ws, const void* x,
                                  const float* W_r, const float* b_r, int* expert_idx, float* gate,
                                  int* local_rank, cudaStream_t stream) {
   cudaError_t e;
-  const bool bf = s.dtype == 1;
+  const bool bf = s.dtype == 1 && !s.jitter;   // a jittered input is fp32
   if (s.router_path == kRouterTile) {
     if (s.N <= 64)
       e = bf ? launch_tile_t<__nv_bfloat16, 256, 64>(s, ws, x, W_r, b_r, expert_idx, gate,

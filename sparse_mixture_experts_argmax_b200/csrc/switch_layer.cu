@@ -74,6 +74,7 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
       take(s.router_path == kRouterTC || s.router_path == kRouterTCWide
                ? 3 * N * static_cast<size_t>(s.d) * 2
                : 0));
+  w.xj = reinterpret_cast<float*>(take(s.jitter ? T * static_cast<size_t>(s.d) * 4 : 0));
   w.xbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d) * elem));
   w.hbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d_ff) * elem));
   w.ybuf = reinterpret_cast<void*>(take(top2 ? A * static_cast<size_t>(s.d) * elem : 0));
@@ -139,7 +140,8 @@ static bool aligned(const void* p, uintptr_t a) {
 
 // Fills Shape; returns SWL_OK or the validation error.
 static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype, double cf,
-                             Shape* s, int topk = 1, int normalize = 1) {
+                             Shape* s, int topk = 1, int normalize = 1, int glu = 0,
+                             int jitter = 0) {
   if (T < 0 || d <= 0 || d_ff <= 0 || N <= 0) return SWL_ERR_INVALID_ARG;
   if (topk != 1 && topk != 2) return SWL_ERR_INVALID_ARG;
   if (topk == 2 && N < 2) return SWL_ERR_INVALID_ARG;                    // two experts needed
@@ -164,8 +166,13 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->sharded = 0;
   s->topk = topk;
   s->normalize = normalize ? 1 : 0;
-  // the tensor-core router serves bf16 layers unless the FFMA router was chosen
-  const bool tensor_router = dtype == SWL_BF16 && g_router_mode.load() == SWL_ROUTER_TENSOR;
+  s->glu = glu ? 1 : 0;
+  s->jitter = jitter ? 1 : 0;
+  if (glu && N * 2 * d_ff > INT32_MAX) return SWL_ERR_UNSUPPORTED;   // TMA row coordinates
+  // the tensor-core router serves bf16 layers unless the FFMA router was chosen;
+  // a jittered router input (x * noise, fp32) always takes the FFMA router
+  const bool tensor_router =
+      dtype == SWL_BF16 && !jitter && g_router_mode.load() == SWL_ROUTER_TENSOR;
   const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0, topk);
   s->router_path = rp.path;
   s->kslice = rp.kslice;
@@ -247,7 +254,12 @@ template <typename Rec>
 static swl_status run_routing(const Shape& s, const Workspace& ws, const void* x,
                               const float* W_r, const void* W1, int32_t* expert_idx, float* gate,
                               int32_t* pos_in_expert, const float* b_r, cudaStream_t stream,
-                              Rec& rec) {
+                              Rec& rec, const float* router_noise = nullptr) {
+  if (s.jitter) {
+    // the router sees x * noise (fp32); the experts keep x
+    if (launch_router_jitter(s, ws, x, router_noise, stream) != cudaSuccess) return SWL_ERR_CUDA;
+    x = ws.xj;
+  }
   if (s.router_path == kRouterTC || s.router_path == kRouterTCWide) {
     CUtensorMap tx, tw;
     if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
@@ -286,7 +298,7 @@ static swl_status run_ffn(const Shape& s, const Workspace& ws, const void* W1, c
     const int sms = num_sms_current();
     if (sms <= 0) return SWL_ERR_CUDA;
     CUtensorMap a1, b1m, a2, b2m;
-    if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff, 128) ||
+    if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff * (s.glu ? 2 : 1), 128) ||
         !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T * s.topk, s.tile_rows) ||
         !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
         !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T * s.topk, s.tile_rows))
@@ -307,7 +319,8 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
                               const float* W_r, const void* W1, const void* b1, const void* W2,
                               const void* b2, void* out, int32_t* expert_idx, float* gate,
                               int32_t* pos_in_expert, float* aux_loss, const float* b_r,
-                              cudaStream_t stream, void* const* ev) {
+                              cudaStream_t stream, void* const* ev,
+                              const float* router_noise = nullptr) {
   // Under stream capture the records are made external, so that they become
   // event-record nodes of the graph (timable on replay); otherwise plain records.
   bool capturing = false;
@@ -324,7 +337,7 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
   };
   if (!rec(0)) return SWL_ERR_CUDA;
   swl_status st = run_routing(s, ws, x, W_r, W1, expert_idx, gate, pos_in_expert, b_r, stream,
-                              rec);
+                              rec, router_noise);
   if (st != SWL_OK) return st;
   if (dispatch_fused_ok(s)) {
     // one launch for scan and gather (timed in the scan stage; the gather stage is empty)
@@ -377,9 +390,11 @@ static swl_status forward_impl(int64_t T, int64_t d, int64_t d_ff, int64_t N, in
                                int32_t* expert_idx, float* gate, int32_t* pos, float* aux,
                                const float* b_r, void* workspace, size_t workspace_bytes,
                                void* stream_v, void* const* ev, int topk = 1,
-                               int normalize = 1) {
+                               int normalize = 1, int glu = 0,
+                               const float* router_noise = nullptr) {
   Shape s;
-  swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s, topk, normalize);
+  swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s, topk, normalize, glu,
+                             router_noise != nullptr ? 1 : 0);
   if (st != SWL_OK) return st;
   st = validate_io(s, x, W_r, W1, b1, W2, b2, out, expert_idx, gate, pos, aux, workspace,
                    workspace_bytes, false);
@@ -397,8 +412,9 @@ static swl_status forward_impl(int64_t T, int64_t d, int64_t d_ff, int64_t N, in
   }
   Workspace ws;
   workspace_layout(s, false, reinterpret_cast<uintptr_t>(workspace), &ws);
+  if (router_noise != nullptr && !aligned(router_noise, 4)) return SWL_ERR_UNSUPPORTED;
   return run_forward(s, ws, x, W_r, W1, b1, W2, b2, out, expert_idx, gate, pos, aux, b_r, stream,
-                     ev);
+                     ev, router_noise);
 }
 
 // ---------------------------------------------------------------- no-alloc scratch
@@ -476,6 +492,53 @@ swl_status switch_layer_forward(int64_t T, int64_t d, int64_t d_ff, int64_t N, i
   return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
                       expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
                       stream, nullptr);
+}
+
+static swl_status variant_args(const swl_variant* v, int* topk, int* normalize, int* glu) {
+  *topk = 1;
+  *normalize = 1;
+  *glu = 0;
+  if (v == nullptr) return SWL_OK;
+  if (v->top_k != 1 && v->top_k != 2) return SWL_ERR_INVALID_ARG;
+  if (v->normalize != 0 && v->normalize != 1) return SWL_ERR_INVALID_ARG;
+  if (v->activation != SWL_ACT_RELU && v->activation != SWL_ACT_GEGLU) return SWL_ERR_INVALID_ARG;
+  *topk = v->top_k;
+  *normalize = v->normalize;
+  *glu = v->activation == SWL_ACT_GEGLU ? 1 : 0;
+  return SWL_OK;
+}
+
+swl_status switch_layer_variant_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                               int dtype, double cf, const swl_variant* v,
+                                               size_t* bytes) {
+  if (!bytes) return SWL_ERR_INVALID_ARG;
+  int topk, normalize, glu;
+  swl_status st = variant_args(v, &topk, &normalize, &glu);
+  if (st != SWL_OK) return st;
+  Shape s;
+  st = make_shape(T, d, d_ff, N, dtype, cf, &s, topk, normalize, glu,
+                  v != nullptr && v->router_noise != nullptr ? 1 : 0);
+  if (st != SWL_OK) return st;
+  *bytes = workspace_layout(s, false, 0, nullptr);
+  return SWL_OK;
+}
+
+swl_status switch_layer_forward_variant(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                        int dtype, const void* x, const float* W_r,
+                                        const void* W1, const void* b1, const void* W2,
+                                        const void* b2, double capacity_factor, void* out,
+                                        int32_t* expert_idx, float* gate,
+                                        int32_t* pos_in_expert, float* aux_loss,
+                                        const float* b_r, const swl_variant* variant,
+                                        void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  int topk, normalize, glu;
+  const swl_status st = variant_args(variant, &topk, &normalize, &glu);
+  if (st != SWL_OK) return st;
+  return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
+                      expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
+                      stream, nullptr, topk, normalize, glu,
+                      variant != nullptr ? variant->router_noise : nullptr);
 }
 
 swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,

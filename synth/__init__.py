@@ -50,7 +50,7 @@ import torch
 
 __all__ = [
     "LayerSpec", "WORKLOADS", "make_layer_inputs", "expert_slice", "draw",
-    "load_gap_redraws", "TABLE_BITS",
+    "load_gap_redraws", "TABLE_BITS", "router_noise",
 ]
 
 TABLE_BITS = 20
@@ -69,6 +69,7 @@ class LayerSpec:
     dtype: str        # "f32" or "bf16": dtype of x, W1, b1, W2, b2, out
     bias_std: float = 0.0       # std of b1 / b2 (0 -> zero biases)
     router_bias: Optional[str] = None  # None or "zipf<a>": b_r[i] = a*ln(1/(i+1))
+    activation: str = "relu"    # "relu" or "geglu" (W1 [N, 2 d_ff, d]: gate rows, value rows)
 
     def to_json(self) -> dict:
         return asdict(self)
@@ -127,6 +128,8 @@ def _std_quantiles(kind: str) -> np.ndarray:
     if kind == "trunc2":
         lo, hi = ndtr(-2.0), ndtr(2.0)
         return ndtri(lo + u * (hi - lo))
+    if kind == "uniform":          # U(-1, 1)
+        return 2.0 * u - 1.0
     raise ValueError(kind)
 
 
@@ -220,23 +223,31 @@ def expert_slice(spec: LayerSpec, experts, seed: int = 0, device="cpu") -> dict:
     sg = _sigmas(spec)
     ce = _chunk_elems(device)
     base = (seed, spec.name)
+    h = 2 * spec.d_ff if spec.activation == "geglu" else spec.d_ff   # GEGLU: gate and value rows
     out = {
-        "W1": _draw_experts(base + ("W1",), experts, (spec.d_ff, spec.d), "trunc2",
+        "W1": _draw_experts(base + ("W1",), experts, (h, spec.d), "trunc2",
                             sg["W1"], spec.dtype, device, ce),
         "W2": _draw_experts(base + ("W2",), experts, (spec.d, spec.d_ff), "trunc2",
                             sg["W2"], spec.dtype, device, ce),
     }
     if spec.bias_std > 0:
-        out["b1"] = _draw_experts(base + ("b1",), experts, (spec.d_ff,), "normal",
+        out["b1"] = _draw_experts(base + ("b1",), experts, (h,), "normal",
                                   spec.bias_std, spec.dtype, device, ce)
         out["b2"] = _draw_experts(base + ("b2",), experts, (spec.d,), "normal",
                                   spec.bias_std, spec.dtype, device, ce)
     else:
-        out["b1"] = torch.zeros((len(list(experts)), spec.d_ff), dtype=_torch_dtype(spec.dtype),
+        out["b1"] = torch.zeros((len(list(experts)), h), dtype=_torch_dtype(spec.dtype),
                                 device=device)
         out["b2"] = torch.zeros((len(list(experts)), spec.d), dtype=_torch_dtype(spec.dtype),
                                 device=device)
     return out
+
+
+def router_noise(spec: LayerSpec, eps: float = 1e-2, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Multiplicative router-input noise [T, d] fp32, uniform on [1 - eps, 1 + eps]
+    (the input jitter of the router exploration experiments; off at inference)."""
+    u = draw((seed, spec.name, "router_noise"), (spec.T, spec.d), "uniform", eps, "f32", device)
+    return 1.0 + u
 
 
 def make_x(spec: LayerSpec, seed: int = 0, device="cpu",
