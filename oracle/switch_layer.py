@@ -54,6 +54,23 @@ Top-2 variant (the earlier-MoE routing the pages compare Switch with):
 * f_i still counts the argmax (first choice), as the loss formula's indicator
   does; P_i is the mean router probability.
 
+Backward pass ([ST-explained] "Why one expert is enough": the chosen expert's
+output is scaled by its own probability, so the gradient reaches the router
+through the gate; [ST-paper] "The loss formulation": f_i is a count with no
+gradient, the balancing gradient flows through P_i only; argmax, positions and
+the capacity cut are piecewise constant and pass no gradient):
+
+* upstream gradients dout [T, d] of the layer output and daux of the aux loss;
+* kept token t (expert e, gate g, a = W1[e] x + b1[e], h = relu(a),
+  u = W2[e] h + b2[e], y = g u): du = g dout_t, dW2[e] += du h^T, db2[e] += du,
+  da = (W2[e]^T du) * [a > 0] (ReLU'(0) = 0), dW1[e] += da x^T, db1[e] += da,
+  dx_t += W1[e]^T da, and the gate's gradient dg_t = dout_t . u;
+* router logits: dz_t,j = dg_t g (delta_{j e} - p_t,j) for kept t, plus
+  daux (N / T) p_t,j (f_j - sum_i f_i p_t,i) for every t (aux = N sum f_i P_i,
+  P_i = mean_t p_t,i);
+* dW_r = sum_t dz_t x_t^T (the router's input: x, or x * noise), db_r = sum_t dz_t,
+  dx_t += W_r^T dz_t.
+
 GEGLU experts and router input jitter ([ST-paper] architecture paragraph: "ReLU
 or GEGLU"; Table 11: input jitter, multiplicative noise on the router input,
 a training-time exploration, off at inference).  The pages name both without
@@ -338,3 +355,51 @@ def switch_forward_top2(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None
     aux = aux_loss(f, P) if T else 0.0
     return {"out": out, "expert_idx": e, "gate": g, "pos_in_expert": pos, "kept": kept,
             "capacity": C, "f": f, "P": P, "aux": aux, "probs": p, "logits": z}
+
+
+# ---------------------------------------------------------------------------
+# backward ([ST-explained] gate gradient; [ST-paper] "The loss formulation")
+# ---------------------------------------------------------------------------
+def switch_backward(x, W_r, W1, b1, W2, b2, capacity_factor: float, dout, daux: float = 0.0,
+                    b_r=None) -> Dict:
+    """Gradients of L = sum(dout * out) + daux * aux for the top-1 ReLU layer:
+    dx [T, d], dW_r [N, d], db_r [N], dW1, db1, dW2, db2 (the shapes of the
+    weights), all float64."""
+    xs = _f64(x)
+    T, d = xs.shape
+    Wr = _f64(W_r)
+    N = Wr.shape[0]
+    fw = switch_forward(xs, W_r, W1, b1, W2, b2, capacity_factor, b_r=b_r)
+    p, e, g, kept, f = fw["probs"], fw["expert_idx"], fw["gate"], fw["kept"], fw["f"]
+    dy = _f64(dout)
+    W1s, b1s, W2s, b2s = _f64(W1), _f64(b1), _f64(W2), _f64(b2)
+    dx = np.zeros((T, d))
+    dW1, db1 = np.zeros_like(W1s), np.zeros_like(b1s)
+    dW2, db2 = np.zeros_like(W2s), np.zeros_like(b2s)
+    dg = np.zeros(T)
+    for i in range(N):
+        rows = np.nonzero((e == i) & kept)[0]
+        if rows.size == 0:
+            continue
+        a = xs[rows] @ W1s[i].T + b1s[i][None, :]
+        h = np.maximum(a, 0.0)
+        u = h @ W2s[i].T + b2s[i][None, :]
+        dg[rows] = np.sum(dy[rows] * u, axis=1)
+        du = g[rows, None] * dy[rows]
+        dW2[i] = du.T @ h
+        db2[i] = du.sum(axis=0)
+        da = (du @ W2s[i]) * (a > 0)
+        dW1[i] = da.T @ xs[rows]
+        db1[i] = da.sum(axis=0)
+        dx[rows] += da @ W1s[i]
+    dz = np.zeros((T, N))
+    if T:
+        onehot = np.zeros((T, N))
+        onehot[np.arange(T), e] = 1.0
+        dz += (dg * g)[:, None] * (onehot - p)                 # zero for dropped tokens
+        dz += daux * (N / T) * p * (f[None, :] - (p @ f)[:, None])
+    dW_r = dz.T @ xs
+    db_r = dz.sum(axis=0)
+    dx += dz @ Wr
+    return {"dx": dx, "dW_r": dW_r, "db_r": db_r, "dW1": dW1, "db1": db1, "dW2": dW2,
+            "db2": db2, "dgate": dg, "dlogits": dz}

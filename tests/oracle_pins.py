@@ -507,6 +507,65 @@ def pin_router_jitter():
         assert np.allclose(r["out"][t0], want, rtol=1e-13, atol=1e-13)
 
 
+# ---------------------------------------------------------------------------
+# backward: central finite differences of L = sum(dout * out) + daux * aux
+# (routing is piecewise constant; inputs keep every decision far from a switch)
+# ---------------------------------------------------------------------------
+def _loss(x, Wr, W1, b1, W2, b2, cf, dout, daux, b_r):
+    r = S.switch_forward(x, Wr, W1, b1, W2, b2, cf, b_r=b_r)
+    return float(np.sum(dout * r["out"]) + daux * r["aux"]), r
+
+
+def pin_backward_finite_differences():
+    rng = np.random.default_rng(17)
+    T, d, d_ff, N, cf = 12, 4, 5, 3, 1.0        # C = 4: some tokens are dropped
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(N, d))
+    b_r = rng.normal(size=N) * 0.2
+    W1, b1, W2, b2 = _rand_ffn(rng, N, d, d_ff)
+    b1 = b1 + 0.05                              # keep pre-activations away from 0 ...
+    dout = rng.normal(size=(T, d))
+    daux = 0.7
+    base, r = _loss(x, Wr, W1, b1, W2, b2, cf, dout, daux, b_r)
+    assert (~r["kept"]).any() and r["kept"].any()
+    gr = S.switch_backward(x, Wr, W1, b1, W2, b2, cf, dout, daux, b_r=b_r)
+    eps = 1e-6
+    params = {"dx": x, "dW_r": Wr, "db_r": b_r, "dW1": W1, "db1": b1, "dW2": W2, "db2": b2}
+    for name, arr in params.items():
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + eps
+            lp, rp = _loss(x, Wr, W1, b1, W2, b2, cf, dout, daux, b_r)
+            arr[idx] = old - eps
+            lm, rm = _loss(x, Wr, W1, b1, W2, b2, cf, dout, daux, b_r)
+            arr[idx] = old
+            # the perturbation must not move a routing decision or a ReLU kink
+            assert np.array_equal(rp["expert_idx"], r["expert_idx"])
+            assert np.array_equal(rm["kept"], r["kept"])
+            num[idx] = (lp - lm) / (2 * eps)
+        assert np.allclose(gr[name], num, rtol=1e-6, atol=1e-7), name
+
+
+def pin_backward_dense_ffn():
+    """N = 1: no router gradient (p = 1), and dx, dW1, db1, dW2, db2 are torch
+    autograd's of the dense FFN."""
+    rng = np.random.default_rng(18)
+    T, d, d_ff = 9, 5, 6
+    x = rng.normal(size=(T, d))
+    W1, b1, W2, b2 = _rand_ffn(rng, 1, d, d_ff)
+    dout = rng.normal(size=(T, d))
+    gr = S.switch_backward(x, rng.normal(size=(1, d)), W1, b1, W2, b2, 1.0, dout, daux=0.5)
+    t = [torch.tensor(a, dtype=torch.float64, requires_grad=True)
+         for a in (x, W1[0], b1[0], W2[0], b2[0])]
+    y = F.linear(F.relu(F.linear(t[0], t[1], t[2])), t[3], t[4])
+    (y * torch.from_numpy(dout)).sum().backward()
+    for k, ten in zip(("dx", "dW1", "db1", "dW2", "db2"), t):
+        got = gr[k] if k == "dx" else gr[k][0]
+        assert np.allclose(got, ten.grad.numpy(), rtol=1e-12, atol=1e-12), k
+    assert np.all(gr["dW_r"] == 0) and np.all(gr["db_r"] == 0)
+
+
 ALL_PINS = [
     pin_lb_worked_example, pin_even_routing_is_one, pin_collapse_tends_to_N,
     pin_not_a_lower_bound, pin_softmax_rows_and_closed_form, pin_ties_lowest_index,
@@ -514,4 +573,5 @@ ALL_PINS = [
     pin_identical_experts_scale_by_gate, pin_sampled_matches_full, pin_logit_gap,
     pin_top2_worked_example, pin_top2_choices_and_capacity, pin_top2_positions_bruteforce,
     pin_top2_closed_forms, pin_top2_drops, pin_gelu, pin_geglu_special_cases, pin_router_jitter,
+    pin_backward_finite_differences, pin_backward_dense_ffn,
 ]

@@ -145,6 +145,16 @@ def _forward_noise_everywhere(x, W_r, W1, b1, W2, b2, capacity_factor, b_r=None,
                          activation=activation)
 
 
+def _patched_backward(old_line: str, new_line: str):
+    """The oracle's switch_backward with one line replaced (a planted mistake)."""
+    import inspect
+    src = inspect.getsource(_orig_backward)
+    assert old_line in src, old_line
+    ns = dict(vars(S))
+    exec(src.replace(old_line, new_line), ns)
+    return ns["switch_backward"]
+
+
 MUTATIONS = {
     "ties_to_highest": ("top1", _top1_highest_tie),
     "positions_one_based": ("positions", _positions_one_based),
@@ -168,6 +178,21 @@ MUTATIONS = {
     "geglu_gate_on_value": ("expert_ffn_geglu", _geglu_gate_on_value),
     "jitter_reaches_experts": ("switch_forward", _forward_noise_everywhere),
 }
+
+_orig_backward = S.switch_backward
+_BACKWARD_MUTATIONS = {
+    "backward_no_gate_path": ("dz += (dg * g)[:, None] * (onehot - p)",
+                              "dz += 0.0 * (onehot - p)"),
+    "backward_no_aux_path": ("dz += daux * (N / T) * p * (f[None, :] - (p @ f)[:, None])",
+                             "dz += 0.0"),
+    "backward_aux_without_mean": ("dz += daux * (N / T) * p * (f[None, :] - (p @ f)[:, None])",
+                                  "dz += daux * (N / T) * p * f[None, :]"),
+    "backward_gate_not_scaling_du": ("du = g[rows, None] * dy[rows]", "du = dy[rows]"),
+    "backward_relu_mask_dropped": ("da = (du @ W2s[i]) * (a > 0)", "da = du @ W2s[i]"),
+    "backward_router_grad_to_x_dropped": ("dx += dz @ Wr", "dx += 0.0"),
+}
+for _name, (_old, _new) in _BACKWARD_MUTATIONS.items():
+    MUTATIONS[_name] = ("switch_backward", _patched_backward(_old, _new))
 
 _orig_forward = S.switch_forward
 
