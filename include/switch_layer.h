@@ -145,6 +145,42 @@ swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t
                                      float* aux_loss, const float* b_r, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* Backward pass of switch_layer_forward (top-1 routing, ReLU experts): the
+ * gradients of L = sum(dout * out) + daux * aux_loss.  The router's gradient
+ * flows through the gate only ("Switch Transformer, explained", "Why one expert
+ * is enough": the chosen expert's output is scaled by its router probability)
+ * and through P_i of the aux loss, f_i being a count without gradient
+ * (paper-graph summary, "The loss formulation"); argmax, positions and the
+ * capacity cut pass no gradient.  For a kept token t of expert e, gate g,
+ * h = relu(W1[e] x + b1[e]), u = W2[e] h + b2[e]:
+ *   du = g dout_t, dW2[e] += du h^T, db2[e] += du,
+ *   da = (W2[e]^T du) * [h > 0], dW1[e] += da x^T, db1[e] += da, dx_t += W1[e]^T da,
+ *   dg_t = dout_t . u (computed as (dout_t . out_t) / g from the bf16 output);
+ * for every token, with p_t = softmax(W_r x_t + b_r) recomputed in fp32:
+ *   dz_t,j = dg_t g (delta_{j e} - p_t,j) [kept] + daux (N / T) p_t,j (f_j - sum_i f_i p_t,i)
+ *   dW_r = sum_t dz_t x_t^T, db_r = sum_t dz_t, dx_t += W_r^T dz_t.
+ * Arguments: the forward's inputs and outputs (out, expert_idx, gate,
+ * pos_in_expert) and its workspace, unchanged since that call (the packed
+ * expert inputs, hidden rows and expert bases are read from it); dout [T, d]
+ * (activation dtype), daux (host value); outputs dx [T, d], dW1, db1, dW2, db2
+ * in the activation dtype and the weights' layouts, dW_r [N, d] and db_r [N]
+ * fp32 (db_r may be NULL).  bwd_workspace: switch_layer_backward_workspace_size
+ * bytes, 256-byte aligned.  Every output is written (experts without kept
+ * tokens get zero gradients).  Errors as switch_layer_forward. */
+swl_status switch_layer_backward_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                                int dtype, double capacity_factor,
+                                                size_t* bytes);
+swl_status switch_layer_backward(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                 const void* x, const float* W_r, const float* b_r,
+                                 const void* W1, const void* b1, const void* W2, const void* b2,
+                                 double capacity_factor, const void* out,
+                                 const int32_t* expert_idx, const float* gate,
+                                 const int32_t* pos_in_expert, const void* fwd_workspace,
+                                 size_t fwd_workspace_bytes, const void* dout, float daux,
+                                 void* dx, float* dW_r, float* db_r, void* dW1, void* db1,
+                                 void* dW2, void* db2, void* bwd_workspace,
+                                 size_t bwd_workspace_bytes, void* stream);
+
 /* Layer variants the pages name beside the Switch layer, in one call:
  *   top_k = 2     the top-2 routing of switch_layer_forward_top2 (routing outputs
  *                 [T, 2]), with normalize as there;

@@ -44,7 +44,8 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_forward_top2", "switch_layer_ep_max_recv_rows",
            "switch_layer_ep_workspace_size", "switch_layer_ep_counts",
            "switch_layer_ep_dispatch", "switch_layer_ep_experts", "switch_layer_ep_combine",
-           "switch_layer_variant_workspace_size", "switch_layer_forward_variant")
+           "switch_layer_variant_workspace_size", "switch_layer_forward_variant",
+           "switch_layer_backward_workspace_size", "switch_layer_backward")
 SWL_ACT_RELU, SWL_ACT_GEGLU = 0, 1
 
 
@@ -133,6 +134,13 @@ def lib() -> ctypes.CDLL:
     L.switch_layer_ep_combine.restype = _i32
     L.switch_layer_ep_combine.argtypes = [_i64, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _dbl,
                                           _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    L.switch_layer_backward_workspace_size.restype = _i32
+    L.switch_layer_backward_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i32, _dbl,
+                                                       ctypes.POINTER(_sz)]
+    L.switch_layer_backward.restype = _i32
+    L.switch_layer_backward.argtypes = ([_i64, _i64, _i64, _i64, _i32] + [_vp] * 7 + [_dbl] +
+                                        [_vp] * 5 + [_sz, _vp, ctypes.c_float] + [_vp] * 8 +
+                                        [_sz, _vp])
     L.switch_layer_variant_workspace_size.restype = _i32
     L.switch_layer_variant_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i32, _dbl,
                                                       ctypes.POINTER(Variant),
@@ -648,3 +656,34 @@ def forward_variant(inputs: dict, capacity_factor: float, top_k: int = 1, normal
     if check:
         _check(switch_layer_device_status(workspace, stream), "device status")
     return o
+
+
+def backward(inputs: dict, capacity_factor: float, fwd: dict, fwd_workspace: torch.Tensor,
+             dout: torch.Tensor, daux: float = 0.0, stream=None, check: bool = True) -> dict:
+    """Gradients of sum(dout * out) + daux * aux for a forward call made with
+    ``fwd_workspace`` (its outputs ``fwd``): dx, dW_r, db_r, dW1, db1, dW2, db2."""
+    x, W1 = inputs["x"], inputs["W1"]
+    T, d = x.shape
+    N, d_ff, _ = W1.shape
+    dev = x.device
+    n = _sz(0)
+    _check(lib().switch_layer_backward_workspace_size(T, d, d_ff, N, dtype_code(x.dtype),
+                                                      float(capacity_factor), ctypes.byref(n)),
+           "backward_workspace_size")
+    bws = torch.empty(max(256, int(n.value)), dtype=torch.uint8, device=dev)
+    g = {"dx": torch.empty_like(x), "dW_r": torch.empty_like(inputs["W_r"]),
+         "db_r": torch.empty(N, dtype=torch.float32, device=dev),
+         "dW1": torch.empty_like(W1), "db1": torch.empty_like(inputs["b1"]),
+         "dW2": torch.empty_like(inputs["W2"]), "db2": torch.empty_like(inputs["b2"])}
+    _require(dout, "dout", x.dtype)
+    _check(lib().switch_layer_backward(
+        T, d, d_ff, N, dtype_code(x.dtype), _ptr(x), _ptr(inputs["W_r"]), _ptr(inputs.get("b_r")),
+        _ptr(W1), _ptr(inputs["b1"]), _ptr(inputs["W2"]), _ptr(inputs["b2"]),
+        float(capacity_factor), _ptr(fwd["out"]), _ptr(fwd["expert_idx"]), _ptr(fwd["gate"]),
+        _ptr(fwd["pos_in_expert"]), _ptr(fwd_workspace), fwd_workspace.numel(), _ptr(dout),
+        float(daux), _ptr(g["dx"]), _ptr(g["dW_r"]), _ptr(g["db_r"]), _ptr(g["dW1"]),
+        _ptr(g["db1"]), _ptr(g["dW2"]), _ptr(g["db2"]), _ptr(bws), bws.numel(),
+        _stream_handle(stream)), "backward")
+    if check:
+        _check(switch_layer_device_status(fwd_workspace, stream), "device status")
+    return g

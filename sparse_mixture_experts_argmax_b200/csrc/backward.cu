@@ -1,0 +1,440 @@
+// Backward pass of the Switch layer (top-1, ReLU experts).
+//
+// The gradient reaches the router only through the gate: the chosen expert's
+// output is scaled by its router probability, so dL/dp_e = dout . u with
+// u = E_e(x) ("Switch Transformer, explained", "Why one expert is enough").
+// The load-balancing loss N sum_i f_i P_i passes its gradient through P_i only;
+// f_i is a count (paper-graph summary of arXiv 2101.03961, "The loss
+// formulation").  The argmax, the positions and the capacity cut are piecewise
+// constant and pass nothing.  For a kept token t of expert e with gate g,
+// a = W1[e] x + b1[e], h = relu(a), u = W2[e] h + b2[e]:
+//   du = g dout_t                dW2[e] += du h^T        db2[e] += du
+//   da = (W2[e]^T du) * [h > 0]  dW1[e] += da x^T        db1[e] += da
+//   dx_t += W1[e]^T da           dg_t = dout_t . u = (dout_t . out_t) / g
+// and for every token, with p_t = softmax(W_r x_t + b_r) recomputed in fp32:
+//   dz_t,j = dg_t g (delta_{j e} - p_t,j) [kept t]
+//          + daux (N / T) p_t,j (f_j - sum_i f_i p_t,i)
+//   dW_r += dz_t x_t^T, db_r += dz_t, dx_t += W_r^T dz_t.
+//
+// Kernels:
+//   bwd_gate_kernel     per token: dg (fp32), the packed row du = g dout, f counts
+//   bwd_router_kernel   per token: logits, softmax, dz (fp32, [T, N])
+//   grouped_gemm_kernel SIMT tiles with fp32 accumulation over packed row
+//                       groups (one group per expert), two forms:
+//                       WGRAD  C[g] = sum over the group's rows of A_r^T B_r
+//                       DGRAD  C_r  = A_r W[g] (+ an epilogue per use)
+//   bias_grad_kernel    db[g] = sum over the group's rows of A_r
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+
+namespace swl {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ld(const T* p) { return static_cast<float>(*p); }
+template <typename T>
+__device__ __forceinline__ T cvt(float v) { return static_cast<T>(v); }
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdWarps = kBwdThreads / 32;
+
+// dg_t = (dout_t . out_t) / g_t for kept tokens (0 for dropped ones), the
+// packed row du[r] = g_t dout_t (r = the token's packed row), and the argmax
+// counts of f.  One warp per token.
+template <typename TA>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_gate_kernel(const TA* __restrict__ dout, const TA* __restrict__ out,
+                const int* __restrict__ expert_idx, const float* __restrict__ gate,
+                const int* __restrict__ pos_in_expert, const int* __restrict__ exp_base,
+                int T, int d, int C_cmp, float* __restrict__ dg, TA* __restrict__ du,
+                int* __restrict__ counts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kBwdWarps + warp;
+  if (t >= T) return;
+  const int e = expert_idx[t];
+  if (lane == 0) atomicAdd(&counts[e], 1);
+  const int pos = pos_in_expert[t];
+  if (pos >= C_cmp) {
+    if (lane == 0) dg[t] = 0.f;
+    return;
+  }
+  const float g = gate[t];
+  const TA* dy = dout + static_cast<size_t>(t) * d;
+  const TA* y = out + static_cast<size_t>(t) * d;
+  TA* u = du + static_cast<size_t>(exp_base[e] + pos) * d;
+  float acc = 0.f;
+  for (int j = lane; j < d; j += 32) {
+    const float a = ld(dy + j);
+    acc += a * ld(y + j);
+    u[j] = cvt<TA>(g * a);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) dg[t] = acc / g;
+}
+
+// Router gradient, one CTA per token: z = W_r x_t + b_r (fp32), p = softmax(z),
+// dz_j = kg (delta_{j e} - p_j) + daux (N / T) p_j (f_j - sum_i f_i p_i) with
+// kg = dg_t g_t (0 for a dropped token), f_j = counts_j / T.  Shared scratch: N floats.
+template <typename TA>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_router_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
+                  const float* __restrict__ b_r, const int* __restrict__ expert_idx,
+                  const float* __restrict__ gate, const float* __restrict__ dg,
+                  const int* __restrict__ counts, int T, int d, int N, float daux,
+                  float* __restrict__ dz) {
+  extern __shared__ float sz[];   // [N] logits, then p
+  __shared__ float red[kBwdWarps];
+  __shared__ float s_bcast;
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const TA* xt = x + static_cast<size_t>(t) * d;
+  // logits: one warp per expert row of W_r
+  for (int n = warp; n < N; n += kBwdWarps) {
+    const float* w = W_r + static_cast<size_t>(n) * d;
+    float acc = 0.f;
+    for (int k = lane; k < d; k += 32) acc = fmaf(ld(xt + k), w[k], acc);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) sz[n] = acc + (b_r ? b_r[n] : 0.f);
+  }
+  __syncthreads();
+  auto block_reduce = [&](float v, bool is_max) -> float {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, v, off);
+      v = is_max ? fmaxf(v, o) : v + o;
+    }
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float r = red[0];
+      for (int w = 1; w < kBwdWarps; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+      s_bcast = r;
+    }
+    __syncthreads();
+    const float r = s_bcast;
+    __syncthreads();
+    return r;
+  };
+  float m = -INFINITY;
+  for (int n = threadIdx.x; n < N; n += kBwdThreads) m = fmaxf(m, sz[n]);
+  m = block_reduce(m, true);
+  float s = 0.f;
+  for (int n = threadIdx.x; n < N; n += kBwdThreads) {
+    const float e = expf(sz[n] - m);
+    sz[n] = e;
+    s += e;
+  }
+  s = block_reduce(s, false);
+  const float inv = 1.0f / s;
+  const float invT = 1.0f / static_cast<float>(T);
+  float fp = 0.f;   // sum_i f_i p_i
+  for (int n = threadIdx.x; n < N; n += kBwdThreads) {
+    const float p = sz[n] * inv;
+    sz[n] = p;
+    fp += static_cast<float>(counts[n]) * invT * p;
+  }
+  fp = block_reduce(fp, false);
+  const int e = expert_idx[t];
+  const float kg = dg[t] * gate[t];
+  const float ca = daux * static_cast<float>(N) * invT;
+  float* dzt = dz + static_cast<size_t>(t) * N;
+  for (int n = threadIdx.x; n < N; n += kBwdThreads) {
+    const float p = sz[n];
+    const float f = static_cast<float>(counts[n]) * invT;
+    dzt[n] = kg * ((n == e ? 1.f : 0.f) - p) + ca * p * (f - fp);
+  }
+}
+
+// Tiled SIMT GEMM over groups of packed rows, fp32 accumulation.  64 x 64
+// outputs per CTA, 256 threads with 4 x 4 each, K staged through shared memory
+// in steps of 16.
+//   WGRAD (kWgrad = true): group g owns rows [base[g], base[g] + rows[g]) of A
+//     [*, P] and B [*, Q]; C[g] [P, Q] = sum over those rows r of A[r]^T B[r]
+//     (C written, not accumulated).  Grid: (Q/64, P/64, groups).
+//   DGRAD: C[r] [Q] = A[r] [K] x W[g] [K, Q] for the group's rows; the epilogue
+//     by `epi`: 0 store; 1 multiply by [mask[r] > 0] and store (da from dh);
+//     2 add into the fp32 accumulator row dst_row[r] (dx).  Grid: (Q/64,
+//     row tiles of 64 listed by tile_prefix, 1).
+// A single group with base = nullptr covers rows [0, rows0).
+constexpr int kGT = 64, kGK = 16;
+
+template <typename TAin, typename TBin, typename TC, bool kWgrad>
+__global__ void __launch_bounds__(256)
+grouped_gemm_kernel(const TAin* __restrict__ A, const TBin* __restrict__ B, TC* __restrict__ C,
+                    int P, int Q, int K, const int* __restrict__ base,
+                    const int* __restrict__ rows, int rows0, const int* __restrict__ tile_prefix,
+                    int groups, int epi, const TC* __restrict__ mask,
+                    const int* __restrict__ dst_row, float* __restrict__ acc_out) {
+  __shared__ float As[kGK][kGT + 1];
+  __shared__ float Bs[kGK][kGT + 1];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  int g, r0, nr;
+  int m0, n0 = blockIdx.x * kGT;
+  if (kWgrad) {
+    g = blockIdx.z;
+    r0 = base ? base[g] : 0;
+    nr = rows ? rows[g] : rows0;
+    m0 = blockIdx.y * kGT;
+    if (nr == 0) {      // an expert with no kept rows has a zero gradient
+      for (int i = threadIdx.x; i < kGT * kGT; i += 256) {
+        const int mm = m0 + i / kGT, nn = n0 + i % kGT;
+        if (mm < P && nn < Q) C[(static_cast<size_t>(g) * P + mm) * Q + nn] = cvt<TC>(0.f);
+      }
+      return;
+    }
+    // C[m][n] = sum_r A[r0 + r][m] B[r0 + r][n]
+    for (int k0 = 0; k0 < nr; k0 += kGK) {
+      for (int i = threadIdx.x; i < kGK * kGT; i += 256) {
+        const int kk = i / kGT, mm = i % kGT;
+        const int r = k0 + kk;
+        As[kk][mm] = (r < nr && m0 + mm < P) ? ld(A + static_cast<size_t>(r0 + r) * P + m0 + mm)
+                                             : 0.f;
+        Bs[kk][mm] = (r < nr && n0 + mm < Q) ? ld(B + static_cast<size_t>(r0 + r) * Q + n0 + mm)
+                                             : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < kGK; ++kk) {
+        float a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a[i] = As[kk][ty * 4 + i];
+          b[i] = Bs[kk][tx * 4 + i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int mm = m0 + ty * 4 + i;
+      if (mm >= P) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int nn = n0 + tx * 4 + j;
+        if (nn < Q) C[(static_cast<size_t>(g) * P + mm) * Q + nn] = cvt<TC>(acc[i][j]);
+      }
+    }
+    return;
+  }
+  // DGRAD: row tile blockIdx.y of the tile list
+  const int tile = blockIdx.y;
+  if (tile_prefix) {
+    if (tile >= tile_prefix[groups]) return;
+    int lo = 0, hi = groups;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_prefix[mid] <= tile) lo = mid; else hi = mid;
+    }
+    g = lo;
+    const int nt = tile - tile_prefix[g];
+    r0 = base[g] + nt * kGT;
+    nr = min(kGT, rows[g] - nt * kGT);
+  } else {
+    g = 0;
+    r0 = tile * kGT;
+    nr = min(kGT, rows0 - r0);
+    if (nr <= 0) return;
+  }
+  const TBin* W = B + static_cast<size_t>(g) * K * Q;
+  for (int k0 = 0; k0 < K; k0 += kGK) {
+    for (int i = threadIdx.x; i < kGK * kGT; i += 256) {
+      const int kk = i % kGK, rr = i / kGK;            // A: rows along i / kGK
+      As[kk][rr] = (rr < nr && k0 + kk < K) ? ld(A + static_cast<size_t>(r0 + rr) * K + k0 + kk)
+                                            : 0.f;
+      const int kb = i / kGT, nn = i % kGT;
+      Bs[kb][nn] = (k0 + kb < K && n0 + nn < Q) ? ld(W + static_cast<size_t>(k0 + kb) * Q + n0 + nn)
+                                                : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kGK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[kk][ty * 4 + i];
+        b[i] = Bs[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = ty * 4 + i;
+    if (rr >= nr) continue;
+    const int r = r0 + rr;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int nn = n0 + tx * 4 + j;
+      if (nn >= Q) continue;
+      const size_t o = static_cast<size_t>(r) * Q + nn;
+      if (epi == 0) {
+        C[o] = cvt<TC>(acc[i][j]);
+      } else if (epi == 1) {
+        C[o] = cvt<TC>(ld(mask + o) > 0.f ? acc[i][j] : 0.f);
+      } else {
+        const int t = dst_row ? dst_row[r] : r;
+        acc_out[static_cast<size_t>(t) * Q + nn] += acc[i][j];
+      }
+    }
+  }
+}
+
+// db[g][m] = sum over the group's rows r of A[r][m]; one thread per (g, m).
+template <typename TA, typename TC>
+__global__ void __launch_bounds__(256)
+bias_grad_kernel(const TA* __restrict__ A, int P, const int* __restrict__ base,
+                 const int* __restrict__ rows, int rows0, int groups, TC* __restrict__ db) {
+  const int g = blockIdx.y;
+  const int m = blockIdx.x * 256 + threadIdx.x;
+  if (g >= groups || m >= P) return;
+  const int r0 = base ? base[g] : 0, nr = rows ? rows[g] : rows0;
+  float s = 0.f;
+  for (int r = 0; r < nr; ++r) s += ld(A + static_cast<size_t>(r0 + r) * P + m);
+  db[static_cast<size_t>(g) * P + m] = cvt<TC>(s);
+}
+
+// Row tiles of 64 packed rows per expert for the DGRAD grid.
+__global__ void bwd_tile_prefix_kernel(const int* __restrict__ rows, int N,
+                                       int* __restrict__ prefix) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < N; ++e) {
+      prefix[e] = acc;
+      acc += (rows[e] + kGT - 1) / kGT;
+    }
+    prefix[N] = acc;
+  }
+}
+
+template <typename TA>
+__global__ void __launch_bounds__(256)
+dx_finish_kernel(const float* __restrict__ acc, TA* __restrict__ dx, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dx[i] = cvt<TA>(acc[i]);
+}
+
+template <typename TA>
+cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspace& bw,
+                           const BwdArgs& a, cudaStream_t stream) {
+  const int T = static_cast<int>(s.T), d = static_cast<int>(s.d), d_ff = static_cast<int>(s.d_ff);
+  const int N = static_cast<int>(s.N);
+  const TA* x = static_cast<const TA*>(a.x);
+  cudaError_t e;
+  int launches = 0;
+  if ((e = cudaMemsetAsync(bw.counts, 0, static_cast<size_t>(N) * 4, stream)) != cudaSuccess)
+    return e;
+  if ((e = cudaMemsetAsync(bw.dx_acc, 0, static_cast<size_t>(T) * d * 4, stream)) != cudaSuccess)
+    return e;
+  // dg, du rows, argmax counts
+  bwd_gate_kernel<TA><<<(T + kBwdWarps - 1) / kBwdWarps, kBwdThreads, 0, stream>>>(
+      static_cast<const TA*>(a.dout), static_cast<const TA*>(a.out), a.expert_idx, a.gate,
+      a.pos_in_expert, fw.exp_base, T, d, static_cast<int>(s.C_cmp), bw.dg,
+      static_cast<TA*>(bw.du), bw.counts);
+  ++launches;
+  // router: dz [T, N]
+  const size_t rsmem = static_cast<size_t>(N) * 4;
+  if (rsmem > 48 * 1024) {
+    if ((e = cudaFuncSetAttribute(bwd_router_kernel<TA>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(rsmem))) != cudaSuccess)
+      return e;
+  }
+  bwd_router_kernel<TA><<<T, kBwdThreads, rsmem, stream>>>(
+      x, a.W_r, a.b_r, a.expert_idx, a.gate, bw.dg, bw.counts, T, d, N, a.daux, bw.dz);
+  ++launches;
+  const dim3 blk(256);
+  auto tiles = [](int v) { return static_cast<unsigned>((v + kGT - 1) / kGT); };
+  // dW2[e] = du^T h, db2[e] = sum du
+  grouped_gemm_kernel<TA, TA, TA, true><<<dim3(tiles(d_ff), tiles(d), N), blk, 0, stream>>>(
+      static_cast<const TA*>(bw.du), static_cast<const TA*>(fw.hbuf), static_cast<TA*>(a.dW2), d,
+      d_ff, 0, fw.exp_base, fw.exp_rows, 0, nullptr, N, 0, nullptr, nullptr, nullptr);
+  bias_grad_kernel<TA, TA><<<dim3((d + 255) / 256, N), blk, 0, stream>>>(
+      static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, static_cast<TA*>(a.db2));
+  launches += 2;
+  // da = (du W2[e]) * [h > 0]   (W2[e] is [d, d_ff]: K = d, Q = d_ff)
+  bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, bw.tile_prefix);
+  const unsigned max_row_tiles = static_cast<unsigned>((T + kGT - 1) / kGT + N);
+  grouped_gemm_kernel<TA, TA, TA, false><<<dim3(tiles(d_ff), max_row_tiles, 1), blk, 0, stream>>>(
+      static_cast<const TA*>(bw.du), static_cast<const TA*>(a.W2), static_cast<TA*>(bw.da), 0,
+      d_ff, d, fw.exp_base, fw.exp_rows, 0, bw.tile_prefix, N, 1,
+      static_cast<const TA*>(fw.hbuf), nullptr, nullptr);
+  launches += 2;
+  // dW1[e] = da^T x (packed x rows), db1[e] = sum da
+  grouped_gemm_kernel<TA, TA, TA, true><<<dim3(tiles(d), tiles(d_ff), N), blk, 0, stream>>>(
+      static_cast<const TA*>(bw.da), static_cast<const TA*>(fw.xbuf), static_cast<TA*>(a.dW1),
+      d_ff, d, 0, fw.exp_base, fw.exp_rows, 0, nullptr, N, 0, nullptr, nullptr, nullptr);
+  bias_grad_kernel<TA, TA><<<dim3((d_ff + 255) / 256, N), blk, 0, stream>>>(
+      static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N,
+      static_cast<TA*>(a.db1));
+  launches += 2;
+  // dx (kept tokens) += da W1[e]   (W1[e] is [d_ff, d]: K = d_ff, Q = d), rows to tokens
+  grouped_gemm_kernel<TA, TA, TA, false><<<dim3(tiles(d), max_row_tiles, 1), blk, 0, stream>>>(
+      static_cast<const TA*>(bw.da), static_cast<const TA*>(a.W1), static_cast<TA*>(nullptr), 0, d,
+      d_ff, fw.exp_base, fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
+  ++launches;
+  // router: dW_r = dz^T x (one group of T rows), db_r = sum dz, dx += dz W_r
+  grouped_gemm_kernel<float, TA, float, true><<<dim3(tiles(d), tiles(N), 1), blk, 0, stream>>>(
+      bw.dz, x, a.dW_r, N, d, 0, nullptr, nullptr, T, nullptr, 1, 0, nullptr, nullptr, nullptr);
+  ++launches;
+  if (a.db_r) {
+    bias_grad_kernel<float, float><<<dim3((N + 255) / 256, 1), blk, 0, stream>>>(
+        bw.dz, N, nullptr, nullptr, T, 1, a.db_r);
+    ++launches;
+  }
+  grouped_gemm_kernel<float, float, float, false><<<dim3(tiles(d), tiles(T), 1), blk, 0, stream>>>(
+      bw.dz, a.W_r, static_cast<float*>(nullptr), 0, d, N, nullptr, nullptr, T, nullptr, 1, 2,
+      nullptr, nullptr, bw.dx_acc);
+  const size_t n = static_cast<size_t>(T) * d;
+  size_t blocks = (n + 255) / 256;
+  if (blocks > 8 * 148) blocks = 8 * 148;
+  dx_finish_kernel<TA><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      bw.dx_acc, static_cast<TA*>(a.dx), n);
+  launches += 2;
+  count_launch(launches);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_workspace_layout(const Shape& s, uintptr_t base, BwdWorkspace* w) {
+  const size_t elem = s.dtype == 1 ? 2 : 4;
+  const size_t T = static_cast<size_t>(s.T), N = static_cast<size_t>(s.N);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return base + o;
+  };
+  BwdWorkspace b{};
+  b.dg = reinterpret_cast<float*>(take(T * 4));
+  b.counts = reinterpret_cast<int*>(take(N * 4));
+  b.tile_prefix = reinterpret_cast<int*>(take((N + 1) * 4));
+  b.dz = reinterpret_cast<float*>(take(T * N * 4));
+  b.du = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
+  b.da = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d_ff) * elem));
+  b.dx_acc = reinterpret_cast<float*>(take(T * static_cast<size_t>(s.d) * 4));
+  if (w) *w = b;
+  return off;
+}
+
+cudaError_t launch_backward(const Shape& s, const Workspace& fw, const BwdWorkspace& bw,
+                            const BwdArgs& a, cudaStream_t stream) {
+  return s.dtype == 1 ? run_backward_t<__nv_bfloat16>(s, fw, bw, a, stream)
+                      : run_backward_t<float>(s, fw, bw, a, stream);
+}
+
+}  // namespace swl

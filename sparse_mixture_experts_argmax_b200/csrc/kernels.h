@@ -200,6 +200,40 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
                                    const void* W, const void* bias, const float* gate, void* out,
                                    cudaStream_t stream);
 
+// ---- backward pass (backward.cu)
+struct BwdWorkspace {
+  float* dg;          // [T] gradient of each token's gate (0 for dropped tokens)
+  int* counts;        // [N] argmax counts (f = counts / T)
+  int* tile_prefix;   // [N + 1] 64-row tiles of packed rows per expert
+  float* dz;          // [T, N] gradient of the router logits
+  void* du;           // [T, d] packed rows g * dout (act dtype)
+  void* da;           // [T, d_ff] packed rows of the gradient of the pre-activations
+  float* dx_acc;      // [T, d] fp32 accumulator of dx
+};
+struct BwdArgs {
+  const void* x;          // [T, d]
+  const float* W_r;       // [N, d]
+  const float* b_r;       // [N] or null
+  const void* W1;         // [N, d_ff, d]
+  const void* W2;         // [N, d, d_ff]
+  const void* out;        // [T, d] forward output
+  const int* expert_idx;
+  const float* gate;
+  const int* pos_in_expert;
+  const void* dout;       // [T, d]
+  float daux;
+  void* dx;               // [T, d]
+  float* dW_r;            // [N, d]
+  float* db_r;            // [N] or null
+  void* dW1;              // [N, d_ff, d]
+  void* db1;              // [N, d_ff]
+  void* dW2;              // [N, d, d_ff]
+  void* db2;              // [N, d]
+};
+size_t backward_workspace_layout(const Shape& s, uintptr_t base, BwdWorkspace* w);
+cudaError_t launch_backward(const Shape& s, const Workspace& fw, const BwdWorkspace& bw,
+                            const BwdArgs& a, cudaStream_t stream);
+
 // Tile rows for the bf16 tcgen05 GEMMs given the effective capacity.
 int bf16_tile_rows(int64_t C_eff);
 // TMEM accumulators of the bf16 expert FFN for a token tile of tile_rows rows:

@@ -956,6 +956,57 @@ swl_status switch_layer_ep_combine(int64_t T, int64_t d, int64_t d_ff, int64_t N
              : SWL_ERR_CUDA;
 }
 
+swl_status switch_layer_backward_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N,
+                                                int dtype, double capacity_factor,
+                                                size_t* bytes) {
+  if (!bytes) return SWL_ERR_INVALID_ARG;
+  Shape s;
+  const swl_status st = make_shape(T, d, d_ff, N, dtype, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  *bytes = backward_workspace_layout(s, 0, nullptr);
+  return SWL_OK;
+}
+
+swl_status switch_layer_backward(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                 const void* x, const float* W_r, const float* b_r,
+                                 const void* W1, const void* b1, const void* W2, const void* b2,
+                                 double capacity_factor, const void* out,
+                                 const int32_t* expert_idx, const float* gate,
+                                 const int32_t* pos_in_expert, const void* fwd_workspace,
+                                 size_t fwd_workspace_bytes, const void* dout, float daux,
+                                 void* dx, float* dW_r, float* db_r, void* dW1, void* db1,
+                                 void* dW2, void* db2, void* bwd_workspace,
+                                 size_t bwd_workspace_bytes, void* stream) {
+  Shape s;
+  swl_status st = make_shape(T, d, d_ff, N, dtype, capacity_factor, &s);
+  if (st != SWL_OK) return st;
+  if (!W_r || !W1 || !b1 || !W2 || !b2 || !fwd_workspace || !bwd_workspace || !dW_r || !dW1 ||
+      !db1 || !dW2 || !db2)
+    return SWL_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out || !expert_idx || !gate || !pos_in_expert || !dout || !dx))
+    return SWL_ERR_INVALID_ARG;
+  if (!std::isfinite(daux)) return SWL_ERR_INVALID_ARG;
+  if (!aligned(fwd_workspace, 256) || !aligned(bwd_workspace, 256)) return SWL_ERR_UNSUPPORTED;
+  const uintptr_t a = dtype == SWL_BF16 ? 2 : 4;
+  if (!aligned(x, a) || !aligned(out, a) || !aligned(dout, a) || !aligned(dx, a) ||
+      !aligned(W1, a) || !aligned(W2, a) || !aligned(dW1, a) || !aligned(dW2, a) ||
+      !aligned(db1, a) || !aligned(db2, a) || !aligned(W_r, 4) || !aligned(dW_r, 4))
+    return SWL_ERR_UNSUPPORTED;
+  if (fwd_workspace_bytes < workspace_layout(s, false, 0, nullptr) ||
+      bwd_workspace_bytes < backward_workspace_layout(s, 0, nullptr))
+    return SWL_ERR_WORKSPACE;
+  if (T == 0) return SWL_OK;
+  Workspace fw;
+  workspace_layout(s, false, reinterpret_cast<uintptr_t>(const_cast<void*>(fwd_workspace)), &fw);
+  BwdWorkspace bw;
+  backward_workspace_layout(s, reinterpret_cast<uintptr_t>(bwd_workspace), &bw);
+  BwdArgs args{x, W_r, b_r, W1, W2, out, expert_idx, gate, pos_in_expert, dout, daux,
+               dx, dW_r, db_r, dW1, db1, dW2, db2};
+  return launch_backward(s, fw, bw, args, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SWL_OK
+             : SWL_ERR_CUDA;
+}
+
 swl_status switch_layer_noalloc_status(void* stream) {
   void* scratch = noalloc_scratch_for_current_device();
   if (scratch == nullptr) return SWL_ERR_CUDA;
