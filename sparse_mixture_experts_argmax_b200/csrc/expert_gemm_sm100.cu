@@ -149,6 +149,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 // Both GEMMs of the expert FFN in one persistent launch.  GEMM2 tiles of token
 // tile g wait until every GEMM1 epilogue warp of g has stored its rows of hbuf.
+template <bool kGlu>   // GEMM1 is GEGLU (args.glu), a separate instantiation
 __global__ void __launch_bounds__(kThreads, 1)
 expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
                         const __grid_constant__ CUtensorMap tmB0,
@@ -160,7 +161,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int stages = args.stages;
   const uint32_t b_bytes = static_cast<uint32_t>(args.bn) * kBK * 2;
-  const uint32_t a_stage = args.glu ? 2 * kABytes : kABytes;   // A bytes per stage
+  constexpr uint32_t a_stage = kGlu ? 2 * kABytes : kABytes;   // A bytes per stage
   uint8_t* smem_a = smem;
   uint8_t* smem_b = smem_a + stages * a_stage;
   __nv_bfloat16* epi = reinterpret_cast<__nv_bfloat16*>(smem_b + stages * b_bytes);
@@ -311,7 +312,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         if (ts.phase == 1) fence_proxy_async_global();
         const int arow = ts.e * P.a_rows + ts.mt * kBM;
         const int brow = ts.row0;
-        const bool two_a = args.glu && ts.phase == 0;   // gate and value rows
+        const bool two_a = kGlu && ts.phase == 0;   // gate and value rows
         if (!checked_index(ts.e >= 0 && ts.e < args.num_experts && brow >= 0 &&
                                brow + ts.rows <= args.T_rows && ts.rows > 0,
                            args.err)) {
@@ -361,7 +362,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag, args.wait_ns)) { fail(); break; }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * acc_cols);
-        const bool two_a = args.glu && ts.phase == 0;   // value rows into the upper half
+        const bool two_a = kGlu && ts.phase == 0;   // value rows into the upper half
         const uint32_t d_val = d_tmem + static_cast<uint32_t>(acc_cols / 2);
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
@@ -440,9 +441,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       // of each of this warp's column chunks
       constexpr int kMaxChunks = 256 / 64;         // chunks of 32 per warp at 256 rows
       const float bias = (f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.a_rows + f]) : 0.f;
-      const bool glu = args.glu && ts.phase == 0;
-      const float bias_v =
-          (glu && f < P.M) ? __bfloat162float(P.bias[(size_t)ts.e * P.a_rows + P.M + f]) : 0.f;
+      const bool glu = kGlu && ts.phase == 0;
+      float bias_v = 0.f;
+      if constexpr (kGlu) {
+        if (glu && f < P.M) bias_v = __bfloat162float(P.bias[(size_t)ts.e * P.a_rows + P.M + f]);
+      }
       int dsts[kMaxChunks];
       float gs[kMaxChunks];
 #pragma unroll
@@ -477,19 +480,24 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         const float g = gs[k];
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
-        if (glu) {
-          // GELU(gate) * value, the value accumulator in the upper half
-          uint32_t rv[32];
-          ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(acc_cols / 2 + c0), rv);
-          ptx::tmem_ld_wait();
+        bool stored = false;
+        if constexpr (kGlu) {
+          if (glu) {
+            // GELU(gate) * value, the value accumulator in the upper half
+            uint32_t rv[32];
+            ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(acc_cols / 2 + c0), rv);
+            ptx::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float gt = __uint_as_float(r[j]) + bias;
-            const float vl = __uint_as_float(rv[j]) + bias_v;
-            const float h = 0.5f * gt * (1.0f + erff(gt * 0.70710678118654752f)) * vl;
-            st[j * 32 + lane] = __float2bfloat16_rn(h);
+            for (int j = 0; j < 32; ++j) {
+              const float gt = __uint_as_float(r[j]) + bias;
+              const float vl = __uint_as_float(rv[j]) + bias_v;
+              const float h = 0.5f * gt * (1.0f + erff(gt * 0.70710678118654752f)) * vl;
+              st[j * 32 + lane] = __float2bfloat16_rn(h);
+            }
+            stored = true;
           }
-        } else {
+        }
+        if (!stored) {
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -600,12 +608,12 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   const int prefix_ints = static_cast<int>(s.N) + 1;
   a.cache_prefix = ffn_smem_bytes(a.bn, stages, prefix_ints, a_tiles) <= kMaxSmem ? 1 : 0;
   const size_t smem = ffn_smem_bytes(a.bn, stages, a.cache_prefix ? prefix_ints : 0, a_tiles);
-  cudaError_t err = cudaFuncSetAttribute(expert_ffn_sm100_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  cudaError_t err = cudaFuncSetAttribute(
+      a.glu ? expert_ffn_sm100_kernel<true> : expert_ffn_sm100_kernel<false>,
+      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  err = launch_dependent(expert_ffn_sm100_kernel, dim3(num_sms), dim3(kThreads), smem, stream,
-                         tmA1, tmB1, tmA2, tmB2, a);
+  err = launch_dependent(a.glu ? expert_ffn_sm100_kernel<true> : expert_ffn_sm100_kernel<false>,
+                         dim3(num_sms), dim3(kThreads), smem, stream, tmA1, tmB1, tmA2, tmB2, a);
   count_launch();
   return err;
 }

@@ -88,10 +88,15 @@ def test_variant_matches_oracle(case):
         check_routing(got, ref, ref["capacity"], T)
     else:
         xr = ic["x"].double() * noise.double() if jitter else ic["x"]
-        # the top-2 oracle with the jittered router input and the plain expert input:
-        # route on x * noise, experts on x (the top-2 layer has no noise argument)
-        routed = oracle.switch_forward_top2(xr, ic["W_r"], ic["W1"], ic["b1"], ic["W2"],
-                                            ic["b2"], cf, b_r=ic["b_r"])
+        # the oracle's top-2 routing of the jittered router input; the experts
+        # (GEGLU) see x itself
+        p = oracle.router_probs(oracle.router_logits(xr, ic["W_r"], ic["b_r"]))
+        e2, g2 = oracle.top2(p)
+        pos2 = oracle.positions_top2(e2, N)
+        C2 = oracle.capacity_k(T, N, cf, 2)
+        f, P = oracle.load_balance_stats(e2[:, 0], p)
+        routed = {"expert_idx": e2, "gate": g2, "pos_in_expert": pos2, "kept": pos2 < C2,
+                  "aux": oracle.aux_loss(f, P)}
         assert np.array_equal(got["expert_idx"].cpu().numpy(), routed["expert_idx"])
         assert np.array_equal(got["pos_in_expert"].cpu().numpy(), routed["pos_in_expert"])
         g = got["gate"].cpu().numpy().astype(np.float64)
