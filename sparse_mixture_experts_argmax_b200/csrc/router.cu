@@ -487,17 +487,22 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
 // of kStreamBufs shared-memory buffers filled by single bulk copies
 // (cp.async.bulk), so a whole chunk is in flight while the previous ones are
 // processed.  Per chunk:
-//   pass A, one warp per token row: lane l holds the float4 columns l, l + 32,
-//     ... in registers (+ b_r); max with the lowest index on ties and the exp
-//     sum in four interleaved chains, warp-reduced; gate = 1/s; p = exp(z - m)/s
-//     written back over the row;
-//   pass B, each thread owns the float4 columns tid, tid + 256, ... and adds
+//   pass A, two warps per token row, each holding half of its float4 columns in
+//     registers (+ b_r when there is one): each half's maximum with the lowest
+//     index on ties (and runner-up for top-2) in four interleaved chains and warp
+//     shuffles; the two halves combined through shared memory; then each half's
+//     exp(z - m) = exp2(z log2 e - m log2 e) and its sum, combined the same
+//     way; gate = 1/s; p = exp(z - m)/s written back over the row;
+//   pass B, each thread owns the float4 columns tid, tid + 512, ... and adds
 //     the chunk's p rows to its per-block sums in token order.
 // At the end of a block: in-block ranks, per-expert counts and the block's
 // sums of p (each column owned by one thread: no reduction needed).
-constexpr int kStreamThreads = 256;
-constexpr int kStreamChunk = kStreamThreads / 32;   // token rows per chunk (one per warp)
+constexpr int kStreamThreads = 512;
+constexpr int kStreamWarps = kStreamThreads / 32;
+constexpr int kStreamWPR = 2;                          // warps per token row in pass A
+constexpr int kStreamChunk = kStreamWarps / kStreamWPR;   // token rows per chunk
 constexpr int kStreamBufs = 3;
+constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr size_t stream_softmax_smem(int N) {
   return 128 + (static_cast<size_t>(kStreamBufs) * kStreamChunk + 1) * N * sizeof(float);
@@ -508,7 +513,7 @@ __host__ __device__ constexpr size_t stream_softmax_smem(int N) {
 // their sum when `normalize`; outputs are [T, 2] (first choice, then second),
 // the block statistics count both choices (blk_count) and, for the aux loss,
 // first choices alone (blk_count1).
-template <int V4, bool TOP2>   // V4: float4 columns per lane in pass A, N <= 128 * V4
+template <int V4, bool TOP2>   // V4: float4 columns per lane in pass A, N <= 2 * 128 * V4
 __global__ void __launch_bounds__(kStreamThreads, 1)
 router_softmax_stream_kernel(const float* __restrict__ z, const float* __restrict__ b_r, int T,
                              int N, int tpb, int nblk, int* __restrict__ expert_idx,
@@ -516,7 +521,7 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
                              int* __restrict__ blk_count, float* __restrict__ blk_psum,
                              int* __restrict__ blk_count1, int normalize, WsHeader* hdr,
                              unsigned long long wait_ns) {
-  constexpr int VPT = (V4 * 32 + kStreamThreads - 1) / kStreamThreads;   // pass-B float4 / thread
+  constexpr int VPT = (V4 * 32 * kStreamWPR + kStreamThreads - 1) / kStreamThreads;
   constexpr int K = TOP2 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   float* buf = reinterpret_cast<float*>(
@@ -526,9 +531,17 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
   __shared__ int eid[K][kTokensPerBlock];
   __shared__ int lead_count[K * kTokensPerBlock];
   __shared__ int lead_first[TOP2 ? kTokensPerBlock : 1];
+  // per row and half: maximum (and runner-up), their experts, the exp sum
+  __shared__ float x_b1[kStreamChunk][kStreamWPR], x_b2[kStreamChunk][kStreamWPR];
+  __shared__ int x_i1[kStreamChunk][kStreamWPR], x_i2[kStreamChunk][kStreamWPR];
+  __shared__ float x_s[kStreamChunk][kStreamWPR];
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NV = N >> 2;   // float4 per row
+  const int rw = warp / kStreamWPR, half = warp % kStreamWPR;   // row of the chunk, half
+  const int NV = N >> 2;                                       // float4 per row
+  const int NVh = (NV + kStreamWPR - 1) / kStreamWPR;         // float4 per half row
+  const int q_lo = half * NVh, q_hi = min(NV, q_lo + NVh);
+  const bool has_bias = b_r != nullptr;
   pdl_trigger();
   if (tid == 0) {
     for (int i = 0; i < kStreamBufs; ++i) ptx::mbar_init(&full[i], 1);
@@ -536,7 +549,8 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
   }
-  for (int n = tid; n < N; n += kStreamThreads) s_bias[n] = b_r ? b_r[n] : 0.f;
+  if (has_bias)
+    for (int n = tid; n < N; n += kStreamThreads) s_bias[n] = b_r[n];
   __syncthreads();
   pdl_wait();   // the logits come from the logits kernel
 
@@ -580,10 +594,13 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
       }
       float* zc = buf + static_cast<size_t>(slot) * kStreamChunk * N;
       const int nt = min(kStreamChunk, ntb - c * kStreamChunk);
-      if (warp < nt) {
-        float4* row = reinterpret_cast<float4*>(zc + static_cast<size_t>(warp) * N);
+      const bool active = rw < nt;
+      float4* row = reinterpret_cast<float4*>(zc + static_cast<size_t>(rw) * N);
+      float4 v[V4];
+      float best = -INFINITY, second = -INFINITY;
+      int bidx = 0x7fffffff, sidx = 0x7fffffff;
+      if (active) {
         const float4* bias4 = reinterpret_cast<const float4*>(s_bias);
-        float4 v[V4];
         // chain c holds column 4q + c: ascending columns per chain, so a strict
         // compare keeps each chain's lowest index among equal values
         float bq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -602,10 +619,14 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
         };
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
-          const int q = lane + 32 * k;
-          if (q < NV) {
-            const float4 a = row[q], bb = bias4[q];
-            v[k] = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
+          const int q = q_lo + lane + 32 * k;
+          if (q < q_hi) {
+            float4 a = row[q];
+            if (has_bias) {
+              const float4 bb = bias4[q];
+              a = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
+            }
+            v[k] = a;
           } else {
             v[k] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
           }
@@ -614,8 +635,10 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
           insert(2, v[k].z, 4 * q + 2);
           insert(3, v[k].w, 4 * q + 3);
         }
-        float best = bq[0], second = sq2[0];
-        int bidx = iq[0], sidx = jq[0];
+        best = bq[0];
+        second = sq2[0];
+        bidx = iq[0];
+        sidx = jq[0];
 #pragma unroll
         for (int c4 = 1; c4 < 4; ++c4) {
           if (TOP2) {
@@ -638,13 +661,38 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
             bidx = oi;
           }
         }
+        if (lane == 0) {
+          x_b1[rw][half] = best;
+          x_i1[rw][half] = bidx;
+          x_b2[rw][half] = second;
+          x_i2[rw][half] = sidx;
+        }
+      }
+      __syncthreads();
+      if (active) {
+        // both halves of the row: the same merge on both warps, in half order
+        best = x_b1[rw][0];
+        bidx = x_i1[rw][0];
+        second = x_b2[rw][0];
+        sidx = x_i2[rw][0];
+#pragma unroll
+        for (int h = 1; h < kStreamWPR; ++h) {
+          if (TOP2) {
+            top2_merge(best, bidx, second, sidx, x_b1[rw][h], x_i1[rw][h], x_b2[rw][h],
+                       x_i2[rw][h]);
+          } else if (rank_before(x_b1[rw][h], x_i1[rw][h], best, bidx)) {
+            best = x_b1[rw][h];
+            bidx = x_i1[rw][h];
+          }
+        }
+        const float ml = best * kLog2e;
         float sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
-          v[k].x = expf(v[k].x - best);
-          v[k].y = expf(v[k].y - best);
-          v[k].z = expf(v[k].z - best);
-          v[k].w = expf(v[k].w - best);
+          v[k].x = exp2f(fmaf(v[k].x, kLog2e, -ml));
+          v[k].y = exp2f(fmaf(v[k].y, kLog2e, -ml));
+          v[k].z = exp2f(fmaf(v[k].z, kLog2e, -ml));
+          v[k].w = exp2f(fmaf(v[k].w, kLog2e, -ml));
           sq[0] += v[k].x;
           sq[1] += v[k].y;
           sq[2] += v[k].z;
@@ -653,54 +701,63 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
         float ssum = (sq[0] + sq[1]) + (sq[2] + sq[3]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+        if (lane == 0) x_s[rw][half] = ssum;
+      }
+      __syncthreads();
+      if (active) {
+        float ssum = x_s[rw][0];
+#pragma unroll
+        for (int h = 1; h < kStreamWPR; ++h) ssum += x_s[rw][h];
         const float inv = 1.0f / ssum;
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
-          const int q = lane + 32 * k;
-          if (q < NV)
+          const int q = q_lo + lane + 32 * k;
+          if (q < q_hi)
             row[q] = make_float4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
         }
-        // a non-finite logit (NaN, or an infinite maximum that makes the exp
-        // sum NaN) is flagged; an index with no finite maximum is kept in range
-        bool bad = bidx >= N || !isfinite(best) || !isfinite(ssum);
-        if (bidx >= N) bidx = 0;
-        if (TOP2) {
-          bad = bad || sidx >= N || sidx == bidx;
-          if (sidx >= N || sidx == bidx) sidx = bidx == 0 ? 1 : 0;
-        }
-        if (bad && lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
-        if (lane == 0) {
-          const int t = t0b + c * kStreamChunk + warp;
-          const int i = c * kStreamChunk + warp;
+        if (half == 0) {
+          // a non-finite logit (NaN, or an infinite maximum that makes the exp
+          // sum NaN) is flagged; an index with no finite maximum is kept in range
+          bool bad = bidx >= N || !isfinite(best) || !isfinite(ssum);
+          if (bidx >= N) bidx = 0;
           if (TOP2) {
-            const float e2 = expf(second - best);      // p_e2 / p_e1
-            const float g1 = normalize ? 1.0f / (1.0f + e2) : inv;
-            const float g2 = normalize ? e2 / (1.0f + e2) : e2 * inv;
-            expert_idx[2 * t] = bidx;
-            expert_idx[2 * t + 1] = sidx;
-            gate[2 * t] = g1;
-            gate[2 * t + 1] = g2;
-            eid[0][i] = bidx;
-            eid[K - 1][i] = sidx;
-          } else {
-            expert_idx[t] = bidx;
-            gate[t] = inv;          // p at the argmax: exp(0) / s
-            eid[0][i] = bidx;
+            bad = bad || sidx >= N || sidx == bidx;
+            if (sidx >= N || sidx == bidx) sidx = bidx == 0 ? 1 : 0;
+          }
+          if (bad && lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
+          if (lane == 0) {
+            const int t = t0b + c * kStreamChunk + rw;
+            const int i = c * kStreamChunk + rw;
+            if (TOP2) {
+              const float e2 = exp2f((second - best) * kLog2e);   // p_e2 / p_e1
+              const float g1 = normalize ? 1.0f / (1.0f + e2) : inv;
+              const float g2 = normalize ? e2 / (1.0f + e2) : e2 * inv;
+              expert_idx[2 * t] = bidx;
+              expert_idx[2 * t + 1] = sidx;
+              gate[2 * t] = g1;
+              gate[2 * t + 1] = g2;
+              eid[0][i] = bidx;
+              eid[K - 1][i] = sidx;
+            } else {
+              expert_idx[t] = bidx;
+              gate[t] = inv;          // p at the argmax: exp(0) / s
+              eid[0][i] = bidx;
+            }
           }
         }
       }
       __syncthreads();
       const float4* zc4 = reinterpret_cast<const float4*>(zc);
 #pragma unroll
-      for (int v = 0; v < VPT; ++v) {
-        const int q = tid + kStreamThreads * v;
+      for (int vv = 0; vv < VPT; ++vv) {
+        const int q = tid + kStreamThreads * vv;
         if (q < NV) {
           for (int r = 0; r < nt; ++r) {
             const float4 p = zc4[static_cast<size_t>(r) * NV + q];
-            acc[v].x += p.x;
-            acc[v].y += p.y;
-            acc[v].z += p.z;
-            acc[v].w += p.w;
+            acc[vv].x += p.x;
+            acc[vv].y += p.y;
+            acc[vv].z += p.z;
+            acc[vv].w += p.w;
           }
         }
       }
@@ -717,10 +774,10 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
     int* cnt1_row = TOP2 ? blk_count1 + static_cast<size_t>(b) * N : nullptr;
     float* ps_row = blk_psum + static_cast<size_t>(b) * N;
 #pragma unroll
-    for (int v = 0; v < VPT; ++v) {
-      const int q = tid + kStreamThreads * v;
+    for (int vv = 0; vv < VPT; ++vv) {
+      const int q = tid + kStreamThreads * vv;
       if (q < NV) {
-        reinterpret_cast<float4*>(ps_row)[q] = acc[v];
+        reinterpret_cast<float4*>(ps_row)[q] = acc[vv];
         reinterpret_cast<int4*>(cnt_row)[q] = make_int4(0, 0, 0, 0);
         if (TOP2) reinterpret_cast<int4*>(cnt1_row)[q] = make_int4(0, 0, 0, 0);
       }
@@ -1301,11 +1358,11 @@ cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const flo
   cudaError_t e;
   const int64_t npl = (s.N + 31) / 32;
   if (softmax_variant(s) == kSoftmaxStream) {
-    const int64_t v4 = (s.N / 4 + 31) / 32;
+    const int64_t v4 = (s.N / 4 / kStreamWPR + 31) / 32;   // float4 per lane, half a row
     if (v4 <= 2) e = launch_stream_t<2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
     else if (v4 <= 4) e = launch_stream_t<4>(s, ws, b_r, expert_idx, gate, local_rank, stream);
     else if (v4 <= 8) e = launch_stream_t<8>(s, ws, b_r, expert_idx, gate, local_rank, stream);
-    else e = launch_stream_t<16>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else e = launch_stream_t<8>(s, ws, b_r, expert_idx, gate, local_rank, stream);   // N <= 2048
   } else if (npl <= 1) e = launch_softmax_t<1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 2) e = launch_softmax_t<2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 4) e = launch_softmax_t<4>(s, ws, b_r, expert_idx, gate, local_rank, stream);
