@@ -77,7 +77,8 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
                      int* __restrict__ ready, float* __restrict__ aux_loss, WsHeader* hdr,
                      int nblk, int N, int T, int C_eff, int tile_rows,
                      uint8_t* __restrict__ record, int record_psum_offset,
-                     const int* __restrict__ blk_count1, int* __restrict__ exp_count1) {
+                     const int* __restrict__ blk_count1, int* __restrict__ exp_count1,
+                     SplitPlan split) {
   __shared__ int wc[kScanWarps][32];
   __shared__ double wp[kScanWarps][32];
   __shared__ int is_last;
@@ -208,6 +209,42 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     tile_prefix[i] = base_tiles;
     base_rows += m;
     base_tiles += (m + tile_rows - 1) / tile_rows;
+  }
+  if (split.factor > 1) {
+    // GEMM2 split over K for experts with at least one full token tile, in
+    // expert order while the partial-tile groups fit the budget: the split tile
+    // prefix, each expert's first group (-1: not split), zeroed counters
+    __shared__ int s_tot_groups, s_tot_tiles2;
+    int groups = 0;
+    for (int i = e0; i < e1; ++i) {
+      const int m = min(__ldcg(exp_count + i), C_eff);
+      if (m >= tile_rows) groups += (m + tile_rows - 1) / tile_rows * split.m_tiles2;
+    }
+    int g = block_excl_scan(groups, s_warp, &s_tot_groups);
+    int tiles2 = 0;
+    for (int i = e0; i < e1; ++i) {
+      const int m = min(__ldcg(exp_count + i), C_eff);
+      const int tl = (m + tile_rows - 1) / tile_rows;
+      const int grp = m >= tile_rows ? tl * split.m_tiles2 : 0;
+      const bool on = grp > 0 && g + grp <= split.max_groups;
+      tiles2 += tl * (on ? split.factor : 1);
+      g += grp;
+    }
+    int base2 = block_excl_scan(tiles2, s_warp, &s_tot_tiles2);
+    g = block_excl_scan(groups, s_warp, &s_tot_groups);
+    for (int i = e0; i < e1; ++i) {
+      const int m = min(__ldcg(exp_count + i), C_eff);
+      const int tl = (m + tile_rows - 1) / tile_rows;
+      const int grp = m >= tile_rows ? tl * split.m_tiles2 : 0;
+      const bool on = grp > 0 && g + grp <= split.max_groups;
+      split.tile_prefix2[i] = base2;
+      split.split_base[i] = on ? g : -1;
+      base2 += tl * (on ? split.factor : 1);
+      g += grp;
+    }
+    if (threadIdx.x == 0) split.tile_prefix2[N] = s_tot_tiles2;
+    for (int i = threadIdx.x; i < split.max_groups * split.warps; i += kScanThreads)
+      split.counters[i] = 0;
   }
 }
 
@@ -771,7 +808,9 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
       aux_loss, ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff, s.tile_rows,
       static_cast<uint8_t*>(record), (int)shard_record_psum_offset(s.N),
       static_cast<const int*>(s.topk == 2 ? ws.blk_count1 : nullptr),
-      s.topk == 2 ? ws.exp_count1 : nullptr);
+      s.topk == 2 ? ws.exp_count1 : nullptr,
+      SplitPlan{s.ffn_split, (int)((s.d + 127) / 128), kSplitMaxGroups, kSplitWarps,
+                ws.tile_prefix2, ws.split_base, ws.part_cnt});
   count_launch();
   return e;
 }

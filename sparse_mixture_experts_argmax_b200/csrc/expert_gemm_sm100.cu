@@ -91,6 +91,16 @@ struct FfnArgs {
   int stages;
   int num_acc;    // TMEM accumulators: 4 of 128 columns when bn <= 128, else 2 of 256
                   // (GEGLU: 512 / the next power of two >= max(128, 2 bn))
+  // GEMM2 split over K (split > 1): the GEMM2 tiles of an expert that has at
+  // least one full token tile are cut into `split` sub-tiles of consecutive
+  // k-blocks; each sub-tile writes an fp32 partial, and for each epilogue warp's
+  // part of the tile the last of the split sub-tiles to finish adds the
+  // partials in k order and stores the result (bias, gate, scatter).
+  int split;
+  const int* tile_prefix2;     // [N+1] GEMM2 tile prefix counting split sub-tiles
+  const int* split_base;       // [N] first split group of expert e, -1: not split
+  float* part;                 // [groups][split][128][bn] fp32 partial tiles
+  int* part_cnt;               // [groups][kEpiWarps] sub-tiles done (zeroed by the scan)
   int glu;        // 1: GEMM1 is GEGLU: each tile multiplies the gate and the value
                   // rows of W1 for the same 128 features into the two halves of
                   // its accumulator, and the epilogue stores GELU(gate) * value
@@ -99,6 +109,7 @@ struct FfnArgs {
 
 struct TileCoord {
   int phase, e, mt, nt, g;   // g: global token-tile index P[e] + nt
+  int ks, nsplit;            // GEMM2 split: sub-tile ks of nsplit (1: not split)
 };
 
 // A decoded work item, published by the scheduler warp in shared memory.
@@ -107,6 +118,9 @@ struct TileSlot {
   int phase, e, mt, nt, g;
   int rows;       // valid token rows of the tile
   int row0;       // first packed row of the tile
+  int kb0, kb1;   // k-blocks [kb0, kb1) of this (sub-)tile
+  int ks, nsplit; // GEMM2 split: sub-tile ks of nsplit
+  int grp;        // split group (partials and counters), -1: not split
 };
 
 constexpr int kTileRing = 8;    // decoded tiles handed to the producer, MMA and epilogue
@@ -115,6 +129,9 @@ constexpr int kTileRing = 8;    // decoded tiles handed to the producer, MMA and
 // tiles of expert e occupy [P[e]*m_tiles, P[e+1]*m_tiles) (P = tile prefix) with
 // token blocks fastest, so CTAs working at the same time share weights.
 // P is the tile prefix, in shared memory when it fits there, else global.
+// With a GEMM2 split, GEMM2 tiles follow the split prefix P2 instead (an
+// expert's tiles there are its token tiles times its split factor).
+template <bool kSplit>
 __device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int total0,
                                                  const int* P) {
   TileCoord c;
@@ -122,17 +139,23 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int to
   const int tile = c.phase == 0 ? t : t - total0;
   const int m_tiles = a.ph[c.phase].m_tiles;
   const int q = tile / m_tiles;
-  int lo = 0, hi = a.num_experts;     // last e with P[e] <= q  (P[N] > q)
+  const int* Q = (kSplit && c.phase == 1) ? a.tile_prefix2 : P;
+  int lo = 0, hi = a.num_experts;     // last e with Q[e] <= q  (Q[N] > q)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (P[mid] <= q) lo = mid; else hi = mid;
+    if (Q[mid] <= q) lo = mid; else hi = mid;
   }
   const int p0 = P[lo];
   const int nts = P[lo + 1] - p0;
-  const int local = tile - p0 * m_tiles;
+  const int q0 = Q[lo];
+  const int nts2 = Q[lo + 1] - q0;     // token tiles times the split factor
+  const int local = tile - q0 * m_tiles;
   c.e = lo;
-  c.mt = local / nts;
-  c.nt = local - c.mt * nts;
+  c.mt = local / nts2;
+  const int r = local - c.mt * nts2;
+  c.nsplit = nts2 / nts;
+  c.nt = r / c.nsplit;
+  c.ks = r - c.nt * c.nsplit;
   c.g = p0 + c.nt;
   return c;
 }
@@ -149,7 +172,9 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 // Both GEMMs of the expert FFN in one persistent launch.  GEMM2 tiles of token
 // tile g wait until every GEMM1 epilogue warp of g has stored its rows of hbuf.
-template <bool kGlu>   // GEMM1 is GEGLU (args.glu), a separate instantiation
+// kGlu: GEMM1 is GEGLU (args.glu); kSplit: GEMM2 split over K (args.split > 1).
+// Each is a separate instantiation so the plain kernel keeps its register budget.
+template <bool kGlu, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
 expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
                         const __grid_constant__ CUtensorMap tmB0,
@@ -217,7 +242,8 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   pdl_wait();   // tile prefix, packed rows, gate and counters come from earlier kernels
   const int ntiles = args.tile_prefix[args.num_experts];
   const int total0 = ntiles * args.ph[0].m_tiles;
-  const int total = total0 + ntiles * args.ph[1].m_tiles;
+  const int ntiles2 = kSplit ? args.tile_prefix2[args.num_experts] : ntiles;
+  const int total = total0 + ntiles2 * args.ph[1].m_tiles;
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -255,8 +281,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         TileSlot ts;
         ts.t = claimed < static_cast<unsigned int>(total) ? static_cast<int>(claimed) : -1;
         ts.phase = ts.e = ts.mt = ts.nt = ts.g = ts.rows = ts.row0 = 0;
+        ts.kb0 = ts.kb1 = ts.ks = 0;
+        ts.nsplit = 1;
+        ts.grp = -1;
         if (ts.t >= 0) {
-          const TileCoord c = decode_tile(ts.t, args, total0, P);
+          const TileCoord c = decode_tile<kSplit>(ts.t, args, total0, P);
           ts.phase = c.phase;
           ts.e = c.e;
           ts.mt = c.mt;
@@ -264,6 +293,19 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           ts.g = c.g;
           ts.rows = min(args.bn, __ldg(args.exp_rows + c.e) - c.nt * args.bn);
           ts.row0 = __ldg(args.exp_base + c.e) + c.nt * args.bn;
+          const int kbs = args.ph[c.phase].k_blocks;
+          ts.ks = c.ks;
+          ts.nsplit = c.nsplit;
+          if (kSplit && c.nsplit > 1) {
+            const int per = (kbs + c.nsplit - 1) / c.nsplit;
+            ts.kb0 = c.ks * per;
+            ts.kb1 = min(kbs, ts.kb0 + per);
+            const int nts = P[c.e + 1] - P[c.e];
+            ts.grp = __ldg(args.split_base + c.e) + c.mt * nts + c.nt;
+          } else {
+            ts.kb0 = 0;
+            ts.kb1 = kbs;
+          }
           if (c.phase == 1) {
             // hbuf rows of token tile g: every GEMM1 epilogue warp of g has stored them
             const int target = kEpiWarps * args.ph[0].m_tiles + (args.stall_test && c.g == 0);
@@ -319,7 +361,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           fail();
           break;
         }
-        for (int kb = 0; kb < P.k_blocks; ++kb) {
+        for (int kb = ts.kb0; kb < ts.kb1; ++kb) {
           if (!ptx::mbar_wait(&empty_bar[stage], ph ^ 1u, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
           ptx::mbar_arrive_expect_tx(&full_bar[stage], (two_a ? 2 * kABytes : kABytes) + b_bytes);
           ptx::tma_load_2d(smem_a + stage * a_stage, tA, &full_bar[stage], kb * kBK, arow, pol_w);
@@ -364,7 +406,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * acc_cols);
         const bool two_a = kGlu && ts.phase == 0;   // value rows into the upper half
         const uint32_t d_val = d_tmem + static_cast<uint32_t>(acc_cols / 2);
-        for (int kb = 0; kb < P.k_blocks; ++kb) {
+        for (int kb = ts.kb0; kb < ts.kb1; ++kb) {
           if (!ptx::mbar_wait(&full_bar[stage], ph, abort_flag, args.wait_ns)) { fail(); ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(smem_a + stage * a_stage);
@@ -373,10 +415,11 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + k * kUmmaK * 2);
             const uint64_t bd = ptx::umma_desc_sw128_kmajor(b_addr + k * kUmmaK * 2);
-            ptx::umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            const uint32_t acc_on = (kb != ts.kb0 || k != 0) ? 1u : 0u;
+            ptx::umma_bf16(d_tmem, ad, bd, idesc, acc_on);
             if (two_a) {
               const uint64_t av = ptx::umma_desc_sw128_kmajor(a_addr + kABytes + k * kUmmaK * 2);
-              ptx::umma_bf16(d_val, av, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+              ptx::umma_bf16(d_val, av, bd, idesc, acc_on);
             }
           }
           ptx::umma_commit(&empty_bar[stage]);      // frees the stage when these MMAs finish
@@ -472,6 +515,83 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       ptx::tc_fence_after();
       const uint32_t t_base =
           tmem_base + static_cast<uint32_t>(acc * acc_cols) + (static_cast<uint32_t>(q * 32) << 16);
+      if (kSplit && ts.grp >= 0) {
+        // GEMM2 sub-tile of a split: this warp's fp32 partial (its 32 features,
+        // its column chunks) goes to the group's partial tile ks, the
+        // accumulator is released, and the last of the split's sub-tiles to
+        // reach this point for this warp's part adds the partials in k order
+        // and stores the result (bias, gate, scatter) as an unsplit tile would.
+        const int S = ts.nsplit;
+        const size_t feat_row = static_cast<size_t>(q * 32 + lane) * args.bn;
+        float* mine = args.part + (static_cast<size_t>(ts.grp) * S + ts.ks) * kBM * args.bn + feat_row;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks; ++k) {
+          const int c0 = (2 * k + half) * 32;
+          if (c0 >= rows) break;
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
+          ptx::tmem_ld_wait();
+          float4* d4 = reinterpret_cast<float4*>(mine + c0);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            d4[jj] = make_float4(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1]),
+                                 __uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3]));
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&tempty_bar[acc]);   // the accumulator is free
+        __threadfence();                                      // partial visible before the count
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(args.part_cnt + ts.grp * kEpiWarps + (warp - 4), 1);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == S - 1) {
+          __threadfence();
+          const float* base = args.part + static_cast<size_t>(ts.grp) * S * kBM * args.bn + feat_row;
+#pragma unroll 1
+          for (int k = 0; k < kMaxChunks; ++k) {
+            const int c0 = (2 * k + half) * 32;
+            if (c0 >= rows) break;
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            for (int sk = 0; sk < S; ++sk) {    // partials added in k order
+              const float4* s4 = reinterpret_cast<const float4*>(
+                  base + static_cast<size_t>(sk) * kBM * args.bn + c0);
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) {
+                const float4 w = __ldcg(s4 + jj);
+                v[4 * jj] += w.x;
+                v[4 * jj + 1] += w.y;
+                v[4 * jj + 2] += w.z;
+                v[4 * jj + 3] += w.w;
+              }
+            }
+            const int dst = dsts[k];
+            const float g = gs[k];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              st[j * 32 + lane] =
+                  __float2bfloat16_rn((v[j] + bias) * __shfl_sync(0xffffffffu, g, j));
+            __syncwarp();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int idx = lane + 32 * kk;
+              const int j = idx >> 2, part = idx & 3;
+              const int drow = __shfl_sync(0xffffffffu, dst, j);
+              if (c0 + j < rows && feat0 + part * 8 < P.M) {
+                *reinterpret_cast<uint4*>(P.out + (size_t)drow * P.M + feat0 + part * 8) =
+                    *reinterpret_cast<const uint4*>(st + j * 32 + part * 8);
+              }
+            }
+            __syncwarp();
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&tile_empty[slot]);
+        if (++acc == args.num_acc) { acc = 0; aph ^= 1u; }
+        continue;
+      }
 #pragma unroll
       for (int k = 0; k < kMaxChunks; ++k) {
         const int c0 = (2 * k + half) * 32;
@@ -576,6 +696,11 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.ready = ws.ready;
   a.next_tile = &ws.hdr->next_tile;
   a.err = &ws.hdr->err;
+  a.split = s.ffn_split;
+  a.tile_prefix2 = ws.tile_prefix2;
+  a.split_base = ws.split_base;
+  a.part = ws.part;
+  a.part_cnt = ws.part_cnt;
   a.wait_ns = wait_limit_ns();
   a.stall_test = stall_test_enabled() ? 1 : 0;
   a.num_experts = static_cast<int>(s.N);
@@ -608,12 +733,15 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   const int prefix_ints = static_cast<int>(s.N) + 1;
   a.cache_prefix = ffn_smem_bytes(a.bn, stages, prefix_ints, a_tiles) <= kMaxSmem ? 1 : 0;
   const size_t smem = ffn_smem_bytes(a.bn, stages, a.cache_prefix ? prefix_ints : 0, a_tiles);
-  cudaError_t err = cudaFuncSetAttribute(
-      a.glu ? expert_ffn_sm100_kernel<true> : expert_ffn_sm100_kernel<false>,
-      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (a.glu && a.split > 1) return cudaErrorInvalidValue;   // no such instantiation
+  auto kern = a.glu ? expert_ffn_sm100_kernel<true, false>
+                    : (a.split > 1 ? expert_ffn_sm100_kernel<false, true>
+                                   : expert_ffn_sm100_kernel<false, false>);
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  err = launch_dependent(a.glu ? expert_ffn_sm100_kernel<true> : expert_ffn_sm100_kernel<false>,
-                         dim3(num_sms), dim3(kThreads), smem, stream, tmA1, tmB1, tmA2, tmB2, a);
+  err = launch_dependent(kern, dim3(num_sms), dim3(kThreads), smem, stream, tmA1, tmB1, tmA2,
+                         tmB2, a);
   count_launch();
   return err;
 }

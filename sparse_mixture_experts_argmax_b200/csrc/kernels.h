@@ -45,6 +45,10 @@ struct Workspace {
   double* psum64;       // [N] sum over all tokens of p_{t,e}
   int* slot_token;      // [A] packed row -> assignment (token t, choice k: t * topk + k)
   int* ready;           // [T/16 + N + 1] per token tile: GEMM1 epilogue warps done
+  int* tile_prefix2;    // GEMM2 split: [N+1] tile prefix counting split sub-tiles
+  int* split_base;      // GEMM2 split: [N] first partial-tile group of e, -1: not split
+  float* part;          // GEMM2 split: [kSplitMaxGroups][split][128][tile_rows] fp32
+  int* part_cnt;        // GEMM2 split: [kSplitMaxGroups][kSplitWarps] sub-tiles done
   void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
   float* xj;            // jittered router input x * noise [T, d] fp32 (jitter only)
   void* xbuf;           // [A, d] packed expert inputs (act dtype), A = T * topk
@@ -68,6 +72,7 @@ struct Shape {
   int64_t T_total;  // tokens of the whole batch (T unless a shard of a global batch)
   int64_t C_cmp;  // min(C, T_total): a token is kept iff its position is below it
   int sharded;    // 1: a shard of a global batch (positions offset by earlier ranks)
+  int ffn_split;  // GEMM2 split over K of experts with full token tiles (1: none)
   int topk;       // experts per token: 1 (Switch) or 2 (the top-2 variant)
   int glu;        // 1: GEGLU experts (W1 [N, 2 d_ff, d]: gate rows, then value rows)
   int jitter;     // 1: the router sees x * noise (a jittered fp32 copy of x, FFMA router)
@@ -137,6 +142,20 @@ int softmax_variant(const Shape& s);
 cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const float* b_r,
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);
+// GEMM2 split over K (see expert_gemm_sm100.cu): at most kSplitMaxGroups groups
+// of kSplitWarps epilogue warps' partial tiles per call.
+constexpr int kSplitMaxGroups = 128;
+constexpr int kSplitWarps = 8;
+constexpr int kSplitFactor = 4;
+struct SplitPlan {
+  int factor;        // 1: no split
+  int m_tiles2;      // GEMM2 feature tiles (d / 128)
+  int max_groups;
+  int warps;
+  int* tile_prefix2;
+  int* split_base;
+  int* counters;
+};
 // record != nullptr: a shard of a global batch; the expert totals go to the
 // exchange record and the expert-level part waits for launch_shard_combine.
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,

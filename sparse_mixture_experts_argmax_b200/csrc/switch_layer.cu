@@ -70,6 +70,13 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.psum64 = reinterpret_cast<double*>(take(N * 8));
   w.slot_token = reinterpret_cast<int*>(take(A * 4));
   w.ready = reinterpret_cast<int*>(take((A / 16 + N + 1) * 4));
+  const bool split = s.ffn_split > 1;
+  w.tile_prefix2 = reinterpret_cast<int*>(take(split ? (N + 1) * 4 : 0));
+  w.split_base = reinterpret_cast<int*>(take(split ? N * 4 : 0));
+  w.part = reinterpret_cast<float*>(
+      take(split ? static_cast<size_t>(kSplitMaxGroups) * s.ffn_split * 128 * s.tile_rows * 4 : 0));
+  w.part_cnt = reinterpret_cast<int*>(
+      take(split ? static_cast<size_t>(kSplitMaxGroups) * kSplitWarps * 4 : 0));
   w.w3 = reinterpret_cast<void*>(
       take(s.router_path == kRouterTC || s.router_path == kRouterTCWide
                ? 3 * N * static_cast<size_t>(s.d) * 2
@@ -180,6 +187,12 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->tpb = rp.tpb;
   s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
+  // GEMM2 split over K: bf16 top-1 ReLU layers with full 256-row token tiles and
+  // a long GEMM2 reduction (d_ff >= 4096), whose dispatch is the scan kernel
+  s->ffn_split = 1;
+  if (dtype == SWL_BF16 && topk == 1 && !glu && s->tile_rows == 256 && d_ff >= 4096 &&
+      !dispatch_fused_ok(*s))
+    s->ffn_split = kSplitFactor;
   return SWL_OK;
 }
 
@@ -196,6 +209,7 @@ static swl_status make_shard_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N
   s->C_eff = s->C < T ? s->C : T;
   s->C_cmp = s->C < T_total ? s->C : T_total;
   s->sharded = 1;
+  s->ffn_split = 1;
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
   return SWL_OK;
 }
@@ -678,11 +692,11 @@ swl_status switch_layer_describe_plan(int64_t T, int64_t d, int64_t d_ff, int64_
   const int n = std::snprintf(
       tmp, sizeof(tmp),
       "router=%s,ksplit=%d,router_stages=%d,softmax=%s,tokens_per_block=%d,dispatch=%s,"
-      "ffn=%s,tile_rows=%d,accumulators=%d",
+      "ffn=%s,tile_rows=%d,accumulators=%d,gemm2_split=%d",
       router, s.ksplit_eff, tc ? router_tc_stages(s, num_sms) : 0,
       softmax_names[softmax_variant(s)], s.tpb,
       dispatch_fused_ok(s) ? "fused" : "two_kernel", bf16 ? "sm100" : "f32", s.tile_rows,
-      bf16 ? ffn_accumulators(s.tile_rows) : 0);
+      bf16 ? ffn_accumulators(s.tile_rows) : 0, s.ffn_split);
   if (n < 0 || static_cast<size_t>(n) >= len) return SWL_ERR_INVALID_ARG;
   std::memcpy(buf, tmp, static_cast<size_t>(n) + 1);
   return SWL_OK;
@@ -913,6 +927,7 @@ swl_status switch_layer_ep_experts(int64_t T, int64_t d, int64_t d_ff, int64_t N
   so.T = ep.plan.max_rows;
   so.N = ep.plan.L;
   so.topk = 1;
+  so.ffn_split = 1;
   so.tile_rows = ep.plan.tile_rows;
   Workspace wo{};
   wo.hdr = ep.plan.hdr;

@@ -125,13 +125,14 @@ def test_router_mode_switch(L):
 _PLAN_CASES = [
     # workloads
     ("base_T4096_d768_N64", None, {"router": "tc", "ksplit": 4, "router_stages": 4,
-                                   "dispatch": "fused", "ffn": "sm100", "accumulators": 4}),
+                                   "dispatch": "fused", "ffn": "sm100", "accumulators": 4,
+                                   "gemm2_split": 1}),
     ("large_T16384_d1024_N128", None, {"router": "tc", "ksplit": 1, "router_stages": 3,
                                        "dispatch": "two_kernel", "tile_rows": 128,
                                        "accumulators": 4}),
     ("skewed_T32768_d2048_N64", None, {"router": "tc", "ksplit": 1, "router_stages": 2,
                                        "dispatch": "two_kernel", "tile_rows": 256,
-                                       "accumulators": 2}),
+                                       "accumulators": 2, "gemm2_split": 4}),
     ("many_T65536_d1024_N2048", None, {"router": "tc_wide", "softmax": "stream",
                                        "dispatch": "two_kernel"}),
     ("tiny_f32_T64_d32_N4", None, {"router": "ffma_warpsplit", "ffn": "f32", "dispatch": "fused"}),
@@ -148,6 +149,8 @@ _PLAN_CASES = [
     ("ffma_tile", (25700, 32, 32, 48, 1.0, "f32"), {"router": "ffma_tile"}),
     ("two_kernel_dispatch", (20000, 256, 32, 8, 1.0, "f32"), {"dispatch": "two_kernel"}),
     ("two_accumulators", (900, 64, 64, 4, 1.0, "bf16"), {"ffn": "sm100", "accumulators": 2}),
+    ("gemm2_split_mixed", (12288, 768, 4096, 8, 1.0, "bf16"),
+     {"dispatch": "two_kernel", "tile_rows": 256, "gemm2_split": 4}),
     # test_router_bias_paths
     ("tc_s1_bias_padded", (6000, 128, 64, 50, 1.25, "bf16"),
      {"router": "tc", "ksplit": 1, "router_stages": 4}),
