@@ -211,40 +211,46 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     base_tiles += (m + tile_rows - 1) / tile_rows;
   }
   if (split.factor > 1) {
-    // GEMM2 split over K for experts with at least one full token tile, in
-    // expert order while the partial-tile groups fit the budget: the split tile
-    // prefix, each expert's first group (-1: not split), zeroed counters
+    // GEMM2 split over K, in expert order while the groups (an expert's
+    // 128-feature by token-tile GEMM2 tiles) fit the budget: the split tile
+    // prefix, each expert's first group (-1: not split) and the group table
     __shared__ int s_tot_groups, s_tot_tiles2;
+    for (int i = threadIdx.x; i < split.max_groups; i += kScanThreads)
+      reinterpret_cast<int4*>(split.groups)[i] = make_int4(-1, 0, 0, 0);
     int groups = 0;
     for (int i = e0; i < e1; ++i) {
       const int m = min(__ldcg(exp_count + i), C_eff);
-      if (m >= tile_rows) groups += (m + tile_rows - 1) / tile_rows * split.m_tiles2;
+      groups += (m + tile_rows - 1) / tile_rows * split.m_tiles2;
     }
     int g = block_excl_scan(groups, s_warp, &s_tot_groups);
     int tiles2 = 0;
     for (int i = e0; i < e1; ++i) {
       const int m = min(__ldcg(exp_count + i), C_eff);
       const int tl = (m + tile_rows - 1) / tile_rows;
-      const int grp = m >= tile_rows ? tl * split.m_tiles2 : 0;
+      const int grp = tl * split.m_tiles2;
       const bool on = grp > 0 && g + grp <= split.max_groups;
       tiles2 += tl * (on ? split.factor : 1);
       g += grp;
     }
     int base2 = block_excl_scan(tiles2, s_warp, &s_tot_tiles2);
-    g = block_excl_scan(groups, s_warp, &s_tot_groups);
+    g = block_excl_scan(groups, s_warp, &s_tot_groups);   // (its barriers order the -1 fill)
     for (int i = e0; i < e1; ++i) {
       const int m = min(__ldcg(exp_count + i), C_eff);
       const int tl = (m + tile_rows - 1) / tile_rows;
-      const int grp = m >= tile_rows ? tl * split.m_tiles2 : 0;
+      const int grp = tl * split.m_tiles2;
       const bool on = grp > 0 && g + grp <= split.max_groups;
       split.tile_prefix2[i] = base2;
       split.split_base[i] = on ? g : -1;
+      if (on) {
+        // group g + mt * tl + nt: m-tile mt of token tile nt (the FFN's numbering)
+        for (int mt = 0; mt < split.m_tiles2; ++mt)
+          for (int nt = 0; nt < tl; ++nt)
+            reinterpret_cast<int4*>(split.groups)[g + mt * tl + nt] = make_int4(i, mt, nt, 0);
+      }
       base2 += tl * (on ? split.factor : 1);
       g += grp;
     }
     if (threadIdx.x == 0) split.tile_prefix2[N] = s_tot_tiles2;
-    for (int i = threadIdx.x; i < split.max_groups * split.warps; i += kScanThreads)
-      split.counters[i] = 0;
   }
 }
 
@@ -809,8 +815,8 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
       static_cast<uint8_t*>(record), (int)shard_record_psum_offset(s.N),
       static_cast<const int*>(s.topk == 2 ? ws.blk_count1 : nullptr),
       s.topk == 2 ? ws.exp_count1 : nullptr,
-      SplitPlan{s.ffn_split, (int)((s.d + 127) / 128), kSplitMaxGroups, kSplitWarps,
-                ws.tile_prefix2, ws.split_base, ws.part_cnt});
+      SplitPlan{s.ffn_split, (int)((s.d + 127) / 128), kSplitMaxGroups, ws.tile_prefix2,
+                ws.split_base, ws.split_grp});
   count_launch();
   return e;
 }

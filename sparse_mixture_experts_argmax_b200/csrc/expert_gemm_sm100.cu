@@ -91,16 +91,20 @@ struct FfnArgs {
   int stages;
   int num_acc;    // TMEM accumulators: 4 of 128 columns when bn <= 128, else 2 of 256
                   // (GEGLU: 512 / the next power of two >= max(128, 2 bn))
-  // GEMM2 split over K (split > 1): the GEMM2 tiles of an expert that has at
-  // least one full token tile are cut into `split` sub-tiles of consecutive
-  // k-blocks; each sub-tile writes an fp32 partial, and for each epilogue warp's
-  // part of the tile the last of the split sub-tiles to finish adds the
-  // partials in k order and stores the result (bias, gate, scatter).
+  // GEMM2 split over K (split > 1): the GEMM2 tiles of the experts the
+  // dispatch scan marks (split_base >= 0) are cut into `split` sub-tiles of
+  // consecutive k-blocks; each sub-tile stores its fp32 partial tile, and
+  // ffn_split_reduce_kernel adds the partials in k order and stores the result
+  // (bias, gate, scatter) once the FFN has finished.
   int split;
   const int* tile_prefix2;     // [N+1] GEMM2 tile prefix counting split sub-tiles
   const int* split_base;       // [N] first split group of expert e, -1: not split
-  float* part;                 // [groups][split][128][bn] fp32 partial tiles
-  int* part_cnt;               // [groups][kEpiWarps] sub-tiles done (zeroed by the scan)
+  float* part;                 // [groups][split][bn][128] fp32 partial tiles
+  // 1: within an expert, tiles go token tile by token tile (all m-tiles of
+  // token tile 0 first), so that GEMM2 of the first token tiles can start
+  // while GEMM1 of the last ones runs; 0: m-tile by m-tile (token tiles
+  // fastest: the CTAs running together share a weight tile)
+  int tok_major;
   int glu;        // 1: GEMM1 is GEGLU: each tile multiplies the gate and the value
                   // rows of W1 for the same 128 features into the two halves of
                   // its accumulator, and the epilogue stores GELU(gate) * value
@@ -151,11 +155,19 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int to
   const int nts2 = Q[lo + 1] - q0;     // token tiles times the split factor
   const int local = tile - q0 * m_tiles;
   c.e = lo;
-  c.mt = local / nts2;
-  const int r = local - c.mt * nts2;
   c.nsplit = nts2 / nts;
-  c.nt = r / c.nsplit;
-  c.ks = r - c.nt * c.nsplit;
+  if (a.tok_major) {
+    const int per_nt = m_tiles * c.nsplit;   // the tiles of one token tile
+    c.nt = local / per_nt;
+    const int r = local - c.nt * per_nt;
+    c.mt = r / c.nsplit;
+    c.ks = r - c.mt * c.nsplit;
+  } else {
+    c.mt = local / nts2;
+    const int r = local - c.mt * nts2;
+    c.nt = r / c.nsplit;
+    c.ks = r - c.nt * c.nsplit;
+  }
   c.g = p0 + c.nt;
   return c;
 }
@@ -398,7 +410,6 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         if (!ptx::mbar_wait(&tile_full[slot], (i / kTileRing) & 1, abort_flag, args.wait_ns)) { fail(); break; }
         const TileSlot ts = tile_ring[slot];
         if (ts.t < 0) break;
-        const PhaseArgs& P = args.ph[ts.phase];
         const uint32_t n_mma = static_cast<uint32_t>((ts.rows + 15) & ~15);
         const uint32_t idesc = ptx::umma_idesc_bf16_f32(n_mma);
         if (!ptx::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag, args.wait_ns)) { fail(); break; }
@@ -516,14 +527,12 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       const uint32_t t_base =
           tmem_base + static_cast<uint32_t>(acc * acc_cols) + (static_cast<uint32_t>(q * 32) << 16);
       if (kSplit && ts.grp >= 0) {
-        // GEMM2 sub-tile of a split: this warp's fp32 partial (its 32 features,
-        // its column chunks) goes to the group's partial tile ks, the
-        // accumulator is released, and the last of the split's sub-tiles to
-        // reach this point for this warp's part adds the partials in k order
-        // and stores the result (bias, gate, scatter) as an unsplit tile would.
-        const int S = ts.nsplit;
-        const size_t feat_row = static_cast<size_t>(q * 32 + lane) * args.bn;
-        float* mine = args.part + (static_cast<size_t>(ts.grp) * S + ts.ks) * kBM * args.bn + feat_row;
+        // GEMM2 sub-tile of a split: the fp32 partial of this warp's 32
+        // features and column chunks goes to partial tile ks of the group, as
+        // [token column][feature] rows (a warp's stores cover 128 contiguous
+        // bytes); the reduce kernel finishes the tile
+        float* pt = args.part + (static_cast<size_t>(ts.grp) * ts.nsplit + ts.ks) * args.bn * kBM +
+                    q * 32 + lane;
 #pragma unroll
         for (int k = 0; k < kMaxChunks; ++k) {
           const int c0 = (2 * k + half) * 32;
@@ -531,64 +540,16 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           uint32_t r[32];
           ptx::tmem_ld_32x32b_x32(t_base + static_cast<uint32_t>(c0), r);
           ptx::tmem_ld_wait();
-          float4* d4 = reinterpret_cast<float4*>(mine + c0);
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj)
-            d4[jj] = make_float4(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1]),
-                                 __uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3]));
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < rows) pt[static_cast<size_t>(c0 + j) * kBM] = __uint_as_float(r[j]);
         }
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&tempty_bar[acc]);   // the accumulator is free
-        __threadfence();                                      // partial visible before the count
-        __syncwarp();
-        int prev = 0;
-        if (lane == 0) prev = atomicAdd(args.part_cnt + ts.grp * kEpiWarps + (warp - 4), 1);
-        prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == S - 1) {
-          __threadfence();
-          const float* base = args.part + static_cast<size_t>(ts.grp) * S * kBM * args.bn + feat_row;
-#pragma unroll 1
-          for (int k = 0; k < kMaxChunks; ++k) {
-            const int c0 = (2 * k + half) * 32;
-            if (c0 >= rows) break;
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.f;
-            for (int sk = 0; sk < S; ++sk) {    // partials added in k order
-              const float4* s4 = reinterpret_cast<const float4*>(
-                  base + static_cast<size_t>(sk) * kBM * args.bn + c0);
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) {
-                const float4 w = __ldcg(s4 + jj);
-                v[4 * jj] += w.x;
-                v[4 * jj + 1] += w.y;
-                v[4 * jj + 2] += w.z;
-                v[4 * jj + 3] += w.w;
-              }
-            }
-            const int dst = dsts[k];
-            const float g = gs[k];
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              st[j * 32 + lane] =
-                  __float2bfloat16_rn((v[j] + bias) * __shfl_sync(0xffffffffu, g, j));
-            __syncwarp();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int idx = lane + 32 * kk;
-              const int j = idx >> 2, part = idx & 3;
-              const int drow = __shfl_sync(0xffffffffu, dst, j);
-              if (c0 + j < rows && feat0 + part * 8 < P.M) {
-                *reinterpret_cast<uint4*>(P.out + (size_t)drow * P.M + feat0 + part * 8) =
-                    *reinterpret_cast<const uint4*>(st + j * 32 + part * 8);
-              }
-            }
-            __syncwarp();
-          }
+        if (lane == 0) {
+          ptx::mbar_arrive(&tempty_bar[acc]);
+          ptx::mbar_arrive(&tile_empty[slot]);
         }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&tile_empty[slot]);
         if (++acc == args.num_acc) { acc = 0; aph ^= 1u; }
         continue;
       }
@@ -665,6 +626,61 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   }
 }
 
+// The split GEMM2 tiles, finished: group blockIdx.x / kReduceParts (an expert's
+// 128 features by one token tile), token columns [part * bn / kReduceParts, ...)
+// of it.  Each thread takes 4 features of a column: the partials added in k
+// order (deterministic), then the bias, the token's gate and the bf16 store to
+// the token's output row.  Launched after the FFN (programmatic dependency).
+constexpr int kReduceParts = 4;
+constexpr int kReduceThreads = 256;
+__global__ void __launch_bounds__(kReduceThreads)
+ffn_split_reduce_kernel(const float* __restrict__ part, const int4* __restrict__ groups,
+                        const int* __restrict__ exp_rows, const int* __restrict__ exp_base,
+                        const int* __restrict__ slot_token, const float* __restrict__ gate,
+                        const __nv_bfloat16* __restrict__ b2, __nv_bfloat16* __restrict__ out,
+                        int S, int bn, int M, int T_rows, int* err) {
+  pdl_trigger();
+  pdl_wait();   // the partial tiles and the group table come from earlier kernels
+  const int grp = blockIdx.x / kReduceParts, quarter = blockIdx.x % kReduceParts;
+  const int4 gd = groups[grp];
+  if (gd.x < 0) return;
+  const int e = gd.x, mt = gd.y, nt = gd.z;
+  const int rows = min(bn, __ldg(exp_rows + e) - nt * bn);
+  const int row0 = __ldg(exp_base + e) + nt * bn;
+  const int per = (bn + kReduceParts - 1) / kReduceParts;
+  const int c_lo = quarter * per, c_hi = min(rows, c_lo + per);
+  const size_t tile = static_cast<size_t>(bn) * kBM;   // floats per partial tile
+  const float* base = part + static_cast<size_t>(grp) * S * tile;
+  for (int item = threadIdx.x; item < (c_hi - c_lo) * (kBM / 4); item += kReduceThreads) {
+    const int col = c_lo + item / (kBM / 4);
+    const int f4 = (item % (kBM / 4)) * 4;
+    const int f = mt * kBM + f4;
+    if (f >= M) continue;
+    const float* src = base + static_cast<size_t>(col) * kBM + f4;
+    float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+    for (int ks = 1; ks < S; ++ks) {   // partials added in k order
+      const float4 w = __ldcg(reinterpret_cast<const float4*>(src + ks * tile));
+      v.x += w.x;
+      v.y += w.y;
+      v.z += w.z;
+      v.w += w.w;
+    }
+    int dst = __ldg(slot_token + row0 + col);
+    if (!checked_index(dst >= 0 && dst < T_rows, err)) dst = 0;
+    const float g = __ldg(gate + dst);
+    const __nv_bfloat16* bb = b2 + static_cast<size_t>(e) * M + f;
+    const float o0 = (v.x + __bfloat162float(bb[0])) * g;
+    const float o1 = (v.y + __bfloat162float(bb[1])) * g;
+    const float o2 = (v.z + __bfloat162float(bb[2])) * g;
+    const float o3 = (v.w + __bfloat162float(bb[3])) * g;
+    __nv_bfloat162 lo2 = __floats2bfloat162_rn(o0, o1), hi2 = __floats2bfloat162_rn(o2, o3);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+    *reinterpret_cast<uint2*>(out + static_cast<size_t>(dst) * M + f) = pk;
+  }
+}
+
 size_t ffn_smem_bytes(int bn, int stages, int cached_prefix_ints, int a_tiles = 1) {
   return 1024 + static_cast<size_t>(cached_prefix_ints) * sizeof(int) +
          static_cast<size_t>(stages) * (a_tiles * kABytes + static_cast<size_t>(bn) * kBK * 2) +
@@ -700,7 +716,8 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.tile_prefix2 = ws.tile_prefix2;
   a.split_base = ws.split_base;
   a.part = ws.part;
-  a.part_cnt = ws.part_cnt;
+  // token-tile order within an expert when its weights sit in L2 anyway
+  a.tok_major = s.d * s.d_ff * 2 * (s.glu ? 2 : 1) <= (int64_t{32} << 20) ? 1 : 0;
   a.wait_ns = wait_limit_ns();
   a.stall_test = stall_test_enabled() ? 1 : 0;
   a.num_experts = static_cast<int>(s.N);
@@ -742,6 +759,14 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   if (err != cudaSuccess) return err;
   err = launch_dependent(kern, dim3(num_sms), dim3(kThreads), smem, stream, tmA1, tmB1, tmA2,
                          tmB2, a);
+  count_launch();
+  if (err != cudaSuccess || a.split <= 1) return err;
+  err = launch_dependent(ffn_split_reduce_kernel, dim3(kSplitMaxGroups * kReduceParts),
+                         dim3(kReduceThreads), 0, stream, static_cast<const float*>(ws.part),
+                         static_cast<const int4*>(static_cast<const void*>(ws.split_grp)),
+                         ws.exp_rows, ws.exp_base, ws.slot_token, gate,
+                         static_cast<const __nv_bfloat16*>(b2), static_cast<__nv_bfloat16*>(out),
+                         a.split, a.bn, a.ph[1].M, a.T_rows, &ws.hdr->err);
   count_launch();
   return err;
 }

@@ -47,8 +47,9 @@ struct Workspace {
   int* ready;           // [T/16 + N + 1] per token tile: GEMM1 epilogue warps done
   int* tile_prefix2;    // GEMM2 split: [N+1] tile prefix counting split sub-tiles
   int* split_base;      // GEMM2 split: [N] first partial-tile group of e, -1: not split
-  float* part;          // GEMM2 split: [kSplitMaxGroups][split][128][tile_rows] fp32
-  int* part_cnt;        // GEMM2 split: [kSplitMaxGroups][kSplitWarps] sub-tiles done
+  float* part;          // GEMM2 split: [kSplitMaxGroups][split][tile_rows][128] fp32
+  int* split_grp;       // GEMM2 split: [kSplitMaxGroups][4] (expert, m-tile, token tile,
+                        // 0) of each group, expert -1 past the last group
   void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
   float* xj;            // jittered router input x * noise [T, d] fp32 (jitter only)
   void* xbuf;           // [A, d] packed expert inputs (act dtype), A = T * topk
@@ -143,18 +144,16 @@ cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const flo
                                   int* expert_idx, float* gate, int* local_rank,
                                   cudaStream_t stream);
 // GEMM2 split over K (see expert_gemm_sm100.cu): at most kSplitMaxGroups groups
-// of kSplitWarps epilogue warps' partial tiles per call.
+// (an expert's 128-feature by token-tile GEMM2 tile) are split per call.
 constexpr int kSplitMaxGroups = 128;
-constexpr int kSplitWarps = 8;
 constexpr int kSplitFactor = 4;
 struct SplitPlan {
   int factor;        // 1: no split
   int m_tiles2;      // GEMM2 feature tiles (d / 128)
   int max_groups;
-  int warps;
   int* tile_prefix2;
   int* split_base;
-  int* counters;
+  int* groups;       // [max_groups][4]
 };
 // record != nullptr: a shard of a global batch; the expert totals go to the
 // exchange record and the expert-level part waits for launch_shard_combine.

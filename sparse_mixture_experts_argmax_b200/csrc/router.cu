@@ -482,30 +482,46 @@ router_softmax_wide_kernel(float* __restrict__ zpart, int nsplit, const float* _
 
 // Streaming softmax for N > 128 whose logits come in one slice (ksplit = 1)
 // with N % 4 == 0: a persistent CTA per SM takes dispatch blocks b =
-// blockIdx.x, blockIdx.x + gridDim.x, ...; each block's rows arrive in chunks
-// of kStreamChunk consecutive token rows (contiguous in [T, N]) through a ring
-// of kStreamBufs shared-memory buffers filled by single bulk copies
-// (cp.async.bulk), so a whole chunk is in flight while the previous ones are
-// processed.  Per chunk:
-//   pass A, two warps per token row, each holding half of its float4 columns in
-//     registers (+ b_r when there is one): each half's maximum with the lowest
-//     index on ties (and runner-up for top-2) in four interleaved chains and warp
-//     shuffles; the two halves combined through shared memory; then each half's
-//     exp(z - m) = exp2(z log2 e - m log2 e) and its sum, combined the same
-//     way; gate = 1/s; p = exp(z - m)/s written back over the row;
-//   pass B, each thread owns the float4 columns tid, tid + 512, ... and adds
-//     the chunk's p rows to its per-block sums in token order.
-// At the end of a block: in-block ranks, per-expert counts and the block's
-// sums of p (each column owned by one thread: no reduction needed).
+// blockIdx.x, blockIdx.x + gridDim.x, ...  Its 16 warps form row groups of WPR
+// warps (one warp per token row up to N = 1024, two up to 2048); group g takes
+// rows g, g + G, ... of each block (G = 16 / WPR groups) and runs on its own:
+// its leader streams each of its rows into a private ring of kStreamStages
+// row buffers with one bulk copy (cp.async.bulk) per row, so the next rows are
+// in flight while one is processed, and the only waits between warps are the
+// group's own (a named barrier when WPR = 2) and one block-wide barrier per
+// block.  Per row, each warp holds its part of the float4 columns in registers
+// (+ b_r when there is one):
+//   the maximum m (fmax in four chains, warp shuffles, the group's parts);
+//   the expert: the lowest column holding m (equal values keep the lowest
+//     index), found by comparing against m and a warp minimum;
+//   e = 2^(z log2 e - m log2 e) and its sum s; gate = 1/s (p at the expert);
+//   p = e/s added to the warp's per-column sums for the block (registers:
+//     a warp sees the same columns on every row).
+// At the end of a block the groups' column sums are added in group order
+// (deterministic), then the in-block ranks and per-expert counts are written.
 constexpr int kStreamThreads = 512;
 constexpr int kStreamWarps = kStreamThreads / 32;
-constexpr int kStreamWPR = 2;                          // warps per token row in pass A
-constexpr int kStreamChunk = kStreamWarps / kStreamWPR;   // token rows per chunk
-constexpr int kStreamBufs = 3;
+constexpr int kStreamStages = 3;                       // row buffers per row group
 constexpr float kLog2e = 1.4426950408889634f;
 
+__host__ __device__ constexpr int stream_wpr(int N) { return N <= 1024 ? 1 : 2; }
+
 __host__ __device__ constexpr size_t stream_softmax_smem(int N) {
-  return 128 + (static_cast<size_t>(kStreamBufs) * kStreamChunk + 1) * N * sizeof(float);
+  // every group's ring, then b_r and the block's column sums
+  return 128 + (static_cast<size_t>(kStreamStages) * (kStreamWarps / stream_wpr(N)) + 2) * N *
+                   sizeof(float);
+}
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz: relative error near
+// 2^-22; a result below the normal range is flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // TOP2: the first choice and the runner-up (lowest index on ties for both,
@@ -513,7 +529,7 @@ __host__ __device__ constexpr size_t stream_softmax_smem(int N) {
 // their sum when `normalize`; outputs are [T, 2] (first choice, then second),
 // the block statistics count both choices (blk_count) and, for the aux loss,
 // first choices alone (blk_count1).
-template <int V4, bool TOP2>   // V4: float4 columns per lane in pass A, N <= 2 * 128 * V4
+template <int V4, int WPR, bool TOP2>   // V4: float4 columns per lane, N <= 128 * WPR * V4
 __global__ void __launch_bounds__(kStreamThreads, 1)
 router_softmax_stream_kernel(const float* __restrict__ z, const float* __restrict__ b_r, int T,
                              int N, int tpb, int nblk, int* __restrict__ expert_idx,
@@ -521,30 +537,35 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
                              int* __restrict__ blk_count, float* __restrict__ blk_psum,
                              int* __restrict__ blk_count1, int normalize, WsHeader* hdr,
                              unsigned long long wait_ns) {
-  constexpr int VPT = (V4 * 32 * kStreamWPR + kStreamThreads - 1) / kStreamThreads;
+  constexpr int G = kStreamWarps / WPR;   // row groups
+  constexpr int S = kStreamStages;
   constexpr int K = TOP2 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   float* buf = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
-  float* s_bias = buf + static_cast<size_t>(kStreamBufs) * kStreamChunk * N;   // [N]
-  __shared__ uint64_t full[kStreamBufs];
+  float* s_bias = buf + static_cast<size_t>(G) * S * N;   // [N]
+  float* s_psum = s_bias + N;                             // [N]
+  __shared__ uint64_t full[G][S];
   __shared__ int eid[K][kTokensPerBlock];
   __shared__ int lead_count[K * kTokensPerBlock];
   __shared__ int lead_first[TOP2 ? kTokensPerBlock : 1];
-  // per row and half: maximum (and runner-up), their experts, the exp sum
-  __shared__ float x_b1[kStreamChunk][kStreamWPR], x_b2[kStreamChunk][kStreamWPR];
-  __shared__ int x_i1[kStreamChunk][kStreamWPR], x_i2[kStreamChunk][kStreamWPR];
-  __shared__ float x_s[kStreamChunk][kStreamWPR];
+  // per group and part: maximum (runner-up), their experts, the exp sum
+  __shared__ float x_m[G][WPR], x_m2[G][WPR], x_s[G][WPR];
+  __shared__ int x_h[G][WPR], x_h2[G][WPR];
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rw = warp / kStreamWPR, half = warp % kStreamWPR;   // row of the chunk, half
-  const int NV = N >> 2;                                       // float4 per row
-  const int NVh = (NV + kStreamWPR - 1) / kStreamWPR;         // float4 per half row
-  const int q_lo = half * NVh, q_hi = min(NV, q_lo + NVh);
+  const int grp = warp / WPR, part = warp % WPR;
+  const int NV = N >> 2;                       // float4 per row
+  const int NVp = (NV + WPR - 1) / WPR;        // float4 per part
+  const int q_lo = part * NVp, q_hi = min(NV, q_lo + NVp);
   const bool has_bias = b_r != nullptr;
+  const bool leader = part == 0 && lane == 0;
+  float* ring = buf + static_cast<size_t>(grp) * S * N;
+  volatile int* ab = &s_abort;
   pdl_trigger();
   if (tid == 0) {
-    for (int i = 0; i < kStreamBufs; ++i) ptx::mbar_init(&full[i], 1);
+    for (int g = 0; g < G; ++g)
+      for (int i = 0; i < S; ++i) ptx::mbar_init(&full[g][i], 1);
     s_abort = 0;
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
@@ -554,216 +575,238 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
   __syncthreads();
   pdl_wait();   // the logits come from the logits kernel
 
-  // chunk sequence of this CTA (the producer's copy of the consumers' order)
-  int pb = blockIdx.x, pc = 0, issued = 0;
-  auto issue_next = [&](int slot) {
+  // the leader's cursor over its group's rows, in the consumers' order
+  int pb = blockIdx.x, pr = grp, issued = 0;
+  auto issue_next = [&]() {
+    while (pb < nblk && pr >= min(tpb, T - pb * tpb)) {
+      pr = grp;
+      pb += gridDim.x;
+    }
     if (pb >= nblk) return;
-    const int tb = pb * tpb, nb = min(tpb, T - tb);
-    const int t0 = tb + pc * kStreamChunk;
-    const int n = min(kStreamChunk, tb + nb - t0);
-    const uint32_t bytes = static_cast<uint32_t>(n) * static_cast<uint32_t>(N) * 4u;
-    ptx::mbar_arrive_expect_tx(&full[slot], bytes);
-    ptx::bulk_load_g2s(buf + static_cast<size_t>(slot) * kStreamChunk * N,
-                       z + static_cast<size_t>(t0) * N, bytes, &full[slot]);
+    const uint32_t bytes = static_cast<uint32_t>(N) * 4u;
+    uint64_t* bar = &full[grp][issued % S];
+    ptx::mbar_arrive_expect_tx(bar, bytes);
+    ptx::bulk_load_g2s(ring + static_cast<size_t>(issued % S) * N,
+                       z + (static_cast<size_t>(pb) * tpb + pr) * N, bytes, bar);
     ++issued;
-    if (++pc * kStreamChunk >= nb) { pc = 0; pb += gridDim.x; }
+    pr += G;
   };
-  if (tid == 0)
-    for (int i = 0; i < kStreamBufs - 1; ++i) issue_next(i);
+  if (leader)
+    for (int i = 0; i < S; ++i) issue_next();
 
-  int ci = 0;   // chunks consumed
-  bool failed = false;
-  for (int b = blockIdx.x; b < nblk && !failed; b += gridDim.x) {
+  const float4* bias4 = reinterpret_cast<const float4*>(s_bias);
+  int ci = 0;   // rows of this group consumed
+  for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
     const int t0b = b * tpb, ntb = min(tpb, T - t0b);
-    float4 acc[VPT];
+    float4 acc[V4];
 #pragma unroll
-    for (int v = 0; v < VPT; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c * kStreamChunk < ntb; ++c, ++ci) {
-      const int slot = ci % kStreamBufs;
-      if (tid == 0) {
-        // the buffer of chunk ci - 1 is free (barrier below): refill it ahead
-        ptx::fence_proxy_async_smem();
-        issue_next((ci + kStreamBufs - 1) % kStreamBufs);
-      }
-      volatile int* ab = &s_abort;
-      const bool ok = ptx::mbar_wait(&full[slot], static_cast<uint32_t>(ci / kStreamBufs) & 1u, ab,
-                                     wait_ns);
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      float* zc = buf + static_cast<size_t>(slot) * kStreamChunk * N;
-      const int nt = min(kStreamChunk, ntb - c * kStreamChunk);
-      const bool active = rw < nt;
-      float4* row = reinterpret_cast<float4*>(zc + static_cast<size_t>(rw) * N);
+    for (int k = 0; k < V4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = grp; r < ntb; r += G, ++ci) {
+      const int slot = ci % S;
+      // after a time-out every wait returns at once (the flag is shared), and
+      // the loop still takes every barrier, so no warp is left waiting
+      if (!ptx::mbar_wait(&full[grp][slot], static_cast<uint32_t>(ci / S) & 1u, ab, wait_ns))
+        *ab = 1;
+      const float4* row = reinterpret_cast<const float4*>(ring + static_cast<size_t>(slot) * N);
       float4 v[V4];
-      float best = -INFINITY, second = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < V4; ++k) {
+        const int q = q_lo + lane + 32 * k;
+        if (q < q_hi) {
+          float4 a = row[q];
+          if (has_bias) {
+            const float4 bb = bias4[q];
+            a = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
+          }
+          v[k] = a;
+        } else {
+          v[k] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+      }
+      float best, second = -INFINITY;
       int bidx = 0x7fffffff, sidx = 0x7fffffff;
-      if (active) {
-        const float4* bias4 = reinterpret_cast<const float4*>(s_bias);
+      if constexpr (TOP2) {
         // chain c holds column 4q + c: ascending columns per chain, so a strict
         // compare keeps each chain's lowest index among equal values
-        float bq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        int iq[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
-        float sq2[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // runner-up (TOP2)
-        int jq[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
-        auto insert = [&](int c4, float val, int col) {
-          if (val > bq[c4]) {
-            if (TOP2) { sq2[c4] = bq[c4]; jq[c4] = iq[c4]; }
-            bq[c4] = val;
-            iq[c4] = col;
-          } else if (TOP2 && val > sq2[c4]) {
-            sq2[c4] = val;
-            jq[c4] = col;
+        float bq[4], sq[4];
+        int iq[4], jq[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          bq[c] = sq[c] = -INFINITY;
+          iq[c] = jq[c] = 0x7fffffff;
+        }
+        auto insert = [&](int c, float val, int col) {
+          if (val > bq[c]) {
+            sq[c] = bq[c];
+            jq[c] = iq[c];
+            bq[c] = val;
+            iq[c] = col;
+          } else if (val > sq[c]) {
+            sq[c] = val;
+            jq[c] = col;
           }
         };
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
           const int q = q_lo + lane + 32 * k;
-          if (q < q_hi) {
-            float4 a = row[q];
-            if (has_bias) {
-              const float4 bb = bias4[q];
-              a = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
-            }
-            v[k] = a;
-          } else {
-            v[k] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-          }
           insert(0, v[k].x, 4 * q);
           insert(1, v[k].y, 4 * q + 1);
           insert(2, v[k].z, 4 * q + 2);
           insert(3, v[k].w, 4 * q + 3);
         }
         best = bq[0];
-        second = sq2[0];
         bidx = iq[0];
+        second = sq[0];
         sidx = jq[0];
 #pragma unroll
-        for (int c4 = 1; c4 < 4; ++c4) {
-          if (TOP2) {
-            top2_merge(best, bidx, second, sidx, bq[c4], iq[c4], sq2[c4], jq[c4]);
-          } else if (rank_before(bq[c4], iq[c4], best, bidx)) {
-            best = bq[c4];
-            bidx = iq[c4];
-          }
-        }
+        for (int c = 1; c < 4; ++c) top2_merge(best, bidx, second, sidx, bq[c], iq[c], sq[c], jq[c]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
           const float ov = __shfl_xor_sync(0xffffffffu, best, off);
           const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-          if (TOP2) {
-            const float os = __shfl_xor_sync(0xffffffffu, second, off);
-            const int oj = __shfl_xor_sync(0xffffffffu, sidx, off);
-            top2_merge(best, bidx, second, sidx, ov, oi, os, oj);
-          } else if (rank_before(ov, oi, best, bidx)) {
-            best = ov;
-            bidx = oi;
+          const float os = __shfl_xor_sync(0xffffffffu, second, off);
+          const int oj = __shfl_xor_sync(0xffffffffu, sidx, off);
+          top2_merge(best, bidx, second, sidx, ov, oi, os, oj);
+        }
+        if (WPR > 1) {
+          if (lane == 0) {
+            x_m[grp][part] = best;
+            x_h[grp][part] = bidx;
+            x_m2[grp][part] = second;
+            x_h2[grp][part] = sidx;
           }
-        }
-        if (lane == 0) {
-          x_b1[rw][half] = best;
-          x_i1[rw][half] = bidx;
-          x_b2[rw][half] = second;
-          x_i2[rw][half] = sidx;
-        }
-      }
-      __syncthreads();
-      if (active) {
-        // both halves of the row: the same merge on both warps, in half order
-        best = x_b1[rw][0];
-        bidx = x_i1[rw][0];
-        second = x_b2[rw][0];
-        sidx = x_i2[rw][0];
+          named_barrier(1 + grp, 32 * WPR);
+          best = x_m[grp][0];
+          bidx = x_h[grp][0];
+          second = x_m2[grp][0];
+          sidx = x_h2[grp][0];
 #pragma unroll
-        for (int h = 1; h < kStreamWPR; ++h) {
-          if (TOP2) {
-            top2_merge(best, bidx, second, sidx, x_b1[rw][h], x_i1[rw][h], x_b2[rw][h],
-                       x_i2[rw][h]);
-          } else if (rank_before(x_b1[rw][h], x_i1[rw][h], best, bidx)) {
-            best = x_b1[rw][h];
-            bidx = x_i1[rw][h];
-          }
+          for (int h = 1; h < WPR; ++h)
+            top2_merge(best, bidx, second, sidx, x_m[grp][h], x_h[grp][h], x_m2[grp][h],
+                       x_h2[grp][h]);
         }
-        const float ml = best * kLog2e;
-        float sq[4] = {0.f, 0.f, 0.f, 0.f};
+      } else {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
-          v[k].x = exp2f(fmaf(v[k].x, kLog2e, -ml));
-          v[k].y = exp2f(fmaf(v[k].y, kLog2e, -ml));
-          v[k].z = exp2f(fmaf(v[k].z, kLog2e, -ml));
-          v[k].w = exp2f(fmaf(v[k].w, kLog2e, -ml));
-          sq[0] += v[k].x;
-          sq[1] += v[k].y;
-          sq[2] += v[k].z;
-          sq[3] += v[k].w;
+          m0 = fmaxf(m0, v[k].x);
+          m1 = fmaxf(m1, v[k].y);
+          m2 = fmaxf(m2, v[k].z);
+          m3 = fmaxf(m3, v[k].w);
         }
-        float ssum = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+        best = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
-        if (lane == 0) x_s[rw][half] = ssum;
+        for (int off = 16; off > 0; off >>= 1)
+          best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+        if (WPR > 1) {
+          if (lane == 0) x_m[grp][part] = best;
+          named_barrier(1 + grp, 32 * WPR);
+          best = x_m[grp][0];
+#pragma unroll
+          for (int h = 1; h < WPR; ++h) best = fmaxf(best, x_m[grp][h]);
+        }
+        // the lowest column of this lane (then of the warp) holding the maximum
+#pragma unroll
+        for (int k = 0; k < V4; ++k) {
+          const float4 a = v[k];
+          if (a.x == best || a.y == best || a.z == best || a.w == best) {
+            const int c = a.x == best ? 0 : a.y == best ? 1 : a.z == best ? 2 : 3;
+            bidx = min(bidx, 4 * (q_lo + lane + 32 * k) + c);
+          }
+        }
+        bidx = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(bidx)));
       }
-      __syncthreads();
-      if (active) {
-        float ssum = x_s[rw][0];
+      __syncwarp();
+      // every warp of the group has its part in registers: the buffer is free
+      if (leader && !*ab) {
+        ptx::fence_proxy_async_smem();
+        issue_next();
+      }
+      const float ml = best * kLog2e;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-        for (int h = 1; h < kStreamWPR; ++h) ssum += x_s[rw][h];
-        const float inv = 1.0f / ssum;
+      for (int k = 0; k < V4; ++k) {
+        v[k].x = ex2_approx(fmaf(v[k].x, kLog2e, -ml));
+        v[k].y = ex2_approx(fmaf(v[k].y, kLog2e, -ml));
+        v[k].z = ex2_approx(fmaf(v[k].z, kLog2e, -ml));
+        v[k].w = ex2_approx(fmaf(v[k].w, kLog2e, -ml));
+        s0 += v[k].x;
+        s1 += v[k].y;
+        s2 += v[k].z;
+        s3 += v[k].w;
+      }
+      float ssum = (s0 + s1) + (s2 + s3);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+      if (WPR > 1) {
+        if (lane == 0) {
+          x_s[grp][part] = ssum;
+          if (!TOP2) x_h[grp][part] = bidx;
+        }
+        named_barrier(1 + grp, 32 * WPR);
+        ssum = x_s[grp][0];
+        if (!TOP2) bidx = x_h[grp][0];
+#pragma unroll
+        for (int h = 1; h < WPR; ++h) {
+          ssum += x_s[grp][h];
+          if (!TOP2) bidx = min(bidx, x_h[grp][h]);
+        }
+      }
+      const float inv = 1.0f / ssum;
+#pragma unroll
+      for (int k = 0; k < V4; ++k) {
+        acc[k].x = fmaf(v[k].x, inv, acc[k].x);
+        acc[k].y = fmaf(v[k].y, inv, acc[k].y);
+        acc[k].z = fmaf(v[k].z, inv, acc[k].z);
+        acc[k].w = fmaf(v[k].w, inv, acc[k].w);
+      }
+      if (leader) {
+        // a non-finite logit (NaN, or an infinite maximum that makes the exp
+        // sum NaN) is flagged; an index with no finite maximum is kept in range
+        bool bad = bidx >= N || !isfinite(best) || !isfinite(ssum);
+        if (bidx >= N) bidx = 0;
+        if (TOP2) {
+          bad = bad || sidx >= N || sidx == bidx;
+          if (sidx >= N || sidx == bidx) sidx = bidx == 0 ? 1 : 0;
+        }
+        if (bad) atomicExch(&hdr->err, kDevNonFiniteLogits);
+        const int t = t0b + r;
+        if (TOP2) {
+          const float e2 = exp2f((second - best) * kLog2e);   // p_e2 / p_e1
+          expert_idx[2 * t] = bidx;
+          expert_idx[2 * t + 1] = sidx;
+          gate[2 * t] = normalize ? 1.0f / (1.0f + e2) : inv;
+          gate[2 * t + 1] = normalize ? e2 / (1.0f + e2) : e2 * inv;
+          eid[0][r] = bidx;
+          eid[K - 1][r] = sidx;
+        } else {
+          expert_idx[t] = bidx;
+          gate[t] = inv;          // p at the expert: 2^0 / s
+          eid[0][r] = bidx;
+        }
+      }
+    }
+    // the block's sums of p: the groups' registers added in group order
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+      __syncthreads();
+      if (grp == g) {
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
           const int q = q_lo + lane + 32 * k;
-          if (q < q_hi)
-            row[q] = make_float4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
-        }
-        if (half == 0) {
-          // a non-finite logit (NaN, or an infinite maximum that makes the exp
-          // sum NaN) is flagged; an index with no finite maximum is kept in range
-          bool bad = bidx >= N || !isfinite(best) || !isfinite(ssum);
-          if (bidx >= N) bidx = 0;
-          if (TOP2) {
-            bad = bad || sidx >= N || sidx == bidx;
-            if (sidx >= N || sidx == bidx) sidx = bidx == 0 ? 1 : 0;
-          }
-          if (bad && lane == 0) atomicExch(&hdr->err, kDevNonFiniteLogits);
-          if (lane == 0) {
-            const int t = t0b + c * kStreamChunk + rw;
-            const int i = c * kStreamChunk + rw;
-            if (TOP2) {
-              const float e2 = exp2f((second - best) * kLog2e);   // p_e2 / p_e1
-              const float g1 = normalize ? 1.0f / (1.0f + e2) : inv;
-              const float g2 = normalize ? e2 / (1.0f + e2) : e2 * inv;
-              expert_idx[2 * t] = bidx;
-              expert_idx[2 * t + 1] = sidx;
-              gate[2 * t] = g1;
-              gate[2 * t + 1] = g2;
-              eid[0][i] = bidx;
-              eid[K - 1][i] = sidx;
+          if (q < q_hi) {
+            float4* d = reinterpret_cast<float4*>(s_psum) + q;
+            if (g == 0) {
+              *d = acc[k];
             } else {
-              expert_idx[t] = bidx;
-              gate[t] = inv;          // p at the argmax: exp(0) / s
-              eid[0][i] = bidx;
+              const float4 o = *d;
+              *d = make_float4(o.x + acc[k].x, o.y + acc[k].y, o.z + acc[k].z, o.w + acc[k].w);
             }
           }
         }
       }
-      __syncthreads();
-      const float4* zc4 = reinterpret_cast<const float4*>(zc);
-#pragma unroll
-      for (int vv = 0; vv < VPT; ++vv) {
-        const int q = tid + kStreamThreads * vv;
-        if (q < NV) {
-          for (int r = 0; r < nt; ++r) {
-            const float4 p = zc4[static_cast<size_t>(r) * NV + q];
-            acc[vv].x += p.x;
-            acc[vv].y += p.y;
-            acc[vv].z += p.z;
-            acc[vv].w += p.w;
-          }
-        }
-      }
-      __syncthreads();   // the chunk buffer is free again
     }
-    if (failed) break;
+    __syncthreads();
     // block bookkeeping: ranks, the block's per-expert counts and sums of p
     if (TOP2) {
       block_ranks_top2(eid[0], eid[K - 1], lead_count, lead_first, ntb, ntb, t0b, local_rank);
@@ -772,15 +815,11 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
     }
     int* cnt_row = blk_count + static_cast<size_t>(b) * N;
     int* cnt1_row = TOP2 ? blk_count1 + static_cast<size_t>(b) * N : nullptr;
-    float* ps_row = blk_psum + static_cast<size_t>(b) * N;
-#pragma unroll
-    for (int vv = 0; vv < VPT; ++vv) {
-      const int q = tid + kStreamThreads * vv;
-      if (q < NV) {
-        reinterpret_cast<float4*>(ps_row)[q] = acc[vv];
-        reinterpret_cast<int4*>(cnt_row)[q] = make_int4(0, 0, 0, 0);
-        if (TOP2) reinterpret_cast<int4*>(cnt1_row)[q] = make_int4(0, 0, 0, 0);
-      }
+    float4* ps_row = reinterpret_cast<float4*>(blk_psum + static_cast<size_t>(b) * N);
+    for (int q = tid; q < NV; q += kStreamThreads) {
+      ps_row[q] = reinterpret_cast<const float4*>(s_psum)[q];
+      reinterpret_cast<int4*>(cnt_row)[q] = make_int4(0, 0, 0, 0);
+      if (TOP2) reinterpret_cast<int4*>(cnt1_row)[q] = make_int4(0, 0, 0, 0);
     }
     __syncthreads();
     for (int i = tid; i < ntb; i += kStreamThreads) {
@@ -792,14 +831,15 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
     }
     __syncthreads();   // eid / lead_count are reused by the next block
   }
-  if (failed) {
-    atomicExch(&hdr->err, kDevPipelineTimeout);
-    // every issued copy must land before the CTA's shared memory goes away
-    if (tid == 0) {
+  __syncthreads();
+  if (*ab) {
+    if (tid == 0) atomicExch(&hdr->err, kDevPipelineTimeout);
+    // every issued copy must land before the CTA's shared memory goes away:
+    // the last one issued into each buffer
+    if (leader) {
       volatile int never = 0;
-      for (int j = ci; j < issued; ++j)
-        ptx::mbar_wait(&full[j % kStreamBufs], static_cast<uint32_t>(j / kStreamBufs) & 1u, &never,
-                       wait_ns);
+      for (int j = max(0, issued - S); j < issued; ++j)
+        ptx::mbar_wait(&full[grp][j % S], static_cast<uint32_t>(j / S) & 1u, &never, wait_ns);
     }
     __syncthreads();
   }
@@ -1332,12 +1372,12 @@ int softmax_variant(const Shape& s) {
   return (s.N + 31) / 32 <= 64 ? kSoftmaxRows : kSoftmaxWide;
 }
 
-template <int V4>
+template <int V4, int WPR>
 cudaError_t launch_stream_t(const Shape& s, const Workspace& ws, const float* b_r,
                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
   const size_t smem = stream_softmax_smem(static_cast<int>(s.N));
-  auto kern = s.topk == 2 ? router_softmax_stream_kernel<V4, true>
-                          : router_softmax_stream_kernel<V4, false>;
+  auto kern = s.topk == 2 ? router_softmax_stream_kernel<V4, WPR, true>
+                          : router_softmax_stream_kernel<V4, WPR, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1358,11 +1398,14 @@ cudaError_t launch_router_softmax(const Shape& s, const Workspace& ws, const flo
   cudaError_t e;
   const int64_t npl = (s.N + 31) / 32;
   if (softmax_variant(s) == kSoftmaxStream) {
-    const int64_t v4 = (s.N / 4 / kStreamWPR + 31) / 32;   // float4 per lane, half a row
-    if (v4 <= 2) e = launch_stream_t<2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
-    else if (v4 <= 4) e = launch_stream_t<4>(s, ws, b_r, expert_idx, gate, local_rank, stream);
-    else if (v4 <= 8) e = launch_stream_t<8>(s, ws, b_r, expert_idx, gate, local_rank, stream);
-    else e = launch_stream_t<8>(s, ws, b_r, expert_idx, gate, local_rank, stream);   // N <= 2048
+    // float4 columns per lane: a row (N <= 1024) or half a row (N <= 2048) per warp
+    const int wpr = stream_wpr(static_cast<int>(s.N));
+    const int64_t v4 = ((s.N / 4 + wpr - 1) / wpr + 31) / 32;
+    if (wpr == 2) e = launch_stream_t<8, 2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else if (v4 <= 1) e = launch_stream_t<1, 1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else if (v4 <= 2) e = launch_stream_t<2, 1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else if (v4 <= 4) e = launch_stream_t<4, 1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
+    else e = launch_stream_t<8, 1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   } else if (npl <= 1) e = launch_softmax_t<1>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 2) e = launch_softmax_t<2>(s, ws, b_r, expert_idx, gate, local_rank, stream);
   else if (npl <= 4) e = launch_softmax_t<4>(s, ws, b_r, expert_idx, gate, local_rank, stream);
