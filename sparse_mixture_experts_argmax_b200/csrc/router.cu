@@ -520,16 +520,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ void named_barrier(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
 // TOP2: the first choice and the runner-up (lowest index on ties for both,
 // two experts per token, see top2_merge), gates p_e1 and p_e2, divided by
 // their sum when `normalize`; outputs are [T, 2] (first choice, then second),
 // the block statistics count both choices (blk_count) and, for the aux loss,
 // first choices alone (blk_count1).
-template <int V4, int WPR, bool TOP2>   // V4: float4 columns per lane, N <= 128 * WPR * V4
+// V4: float4 columns per lane, N <= 128 * WPR * V4; kFull: N == 128 * WPR * V4
+// (every lane's columns exist: no range checks)
+template <int V4, int WPR, bool TOP2, bool kFull>
 __global__ void __launch_bounds__(kStreamThreads, 1)
 router_softmax_stream_kernel(const float* __restrict__ z, const float* __restrict__ b_r, int T,
                              int N, int tpb, int nblk, int* __restrict__ expert_idx,
@@ -612,7 +610,7 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
 #pragma unroll
       for (int k = 0; k < V4; ++k) {
         const int q = q_lo + lane + 32 * k;
-        if (q < q_hi) {
+        if (kFull || q < q_hi) {
           float4 a = row[q];
           if (has_bias) {
             const float4 bb = bias4[q];
@@ -675,7 +673,7 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
             x_m2[grp][part] = second;
             x_h2[grp][part] = sidx;
           }
-          named_barrier(1 + grp, 32 * WPR);
+          ptx::named_bar_sync(1 + grp, 32 * WPR);
           best = x_m[grp][0];
           bidx = x_h[grp][0];
           second = x_m2[grp][0];
@@ -694,24 +692,29 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
           m2 = fmaxf(m2, v[k].z);
           m3 = fmaxf(m3, v[k].w);
         }
-        best = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        const float lane_best = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        best = lane_best;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
           best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
         if (WPR > 1) {
           if (lane == 0) x_m[grp][part] = best;
-          named_barrier(1 + grp, 32 * WPR);
+          ptx::named_bar_sync(1 + grp, 32 * WPR);
           best = x_m[grp][0];
 #pragma unroll
           for (int h = 1; h < WPR; ++h) best = fmaxf(best, x_m[grp][h]);
         }
-        // the lowest column of this lane (then of the warp) holding the maximum
+        // the lowest column holding the maximum: searched only by the lanes
+        // that hold it (columns in descending order, so the last match stands),
+        // then the warp's minimum
+        if (lane_best == best) {
 #pragma unroll
-        for (int k = 0; k < V4; ++k) {
-          const float4 a = v[k];
-          if (a.x == best || a.y == best || a.z == best || a.w == best) {
-            const int c = a.x == best ? 0 : a.y == best ? 1 : a.z == best ? 2 : 3;
-            bidx = min(bidx, 4 * (q_lo + lane + 32 * k) + c);
+          for (int k = V4 - 1; k >= 0; --k) {
+            const int c4 = 4 * (q_lo + lane + 32 * k);
+            if (v[k].w == best) bidx = c4 + 3;
+            if (v[k].z == best) bidx = c4 + 2;
+            if (v[k].y == best) bidx = c4 + 1;
+            if (v[k].x == best) bidx = c4;
           }
         }
         bidx = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(bidx)));
@@ -743,7 +746,7 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
           x_s[grp][part] = ssum;
           if (!TOP2) x_h[grp][part] = bidx;
         }
-        named_barrier(1 + grp, 32 * WPR);
+        ptx::named_bar_sync(1 + grp, 32 * WPR);
         ssum = x_s[grp][0];
         if (!TOP2) bidx = x_h[grp][0];
 #pragma unroll
@@ -794,7 +797,7 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
 #pragma unroll
         for (int k = 0; k < V4; ++k) {
           const int q = q_lo + lane + 32 * k;
-          if (q < q_hi) {
+          if (kFull || q < q_hi) {
             float4* d = reinterpret_cast<float4*>(s_psum) + q;
             if (g == 0) {
               *d = acc[k];
@@ -1279,6 +1282,13 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk) {
   p.tpb = 32;
   for (int tpb = 128; tpb > 32; tpb /= 2)
     if ((T + tpb - 1) / tpb >= 2 * 148) { p.tpb = tpb; break; }
+  if (tensor && N % 4 == 0 && N <= kStreamSoftmaxMaxN) {
+    // the streaming softmax's persistent CTAs (one per SM) take whole blocks:
+    // blocks of up to 128 tokens sized so that every CTA gets the same number
+    const int64_t rounds = (T + 128 * 148 - 1) / (128 * 148);
+    const int64_t tpb = (T + rounds * 148 - 1) / (rounds * 148);
+    p.tpb = static_cast<int>(tpb < 32 ? 32 : tpb);
+  }
   if (tensor) {
     p.path = kRouterTCWide;
     p.ksplit = 1;
@@ -1376,8 +1386,10 @@ template <int V4, int WPR>
 cudaError_t launch_stream_t(const Shape& s, const Workspace& ws, const float* b_r,
                             int* expert_idx, float* gate, int* local_rank, cudaStream_t stream) {
   const size_t smem = stream_softmax_smem(static_cast<int>(s.N));
-  auto kern = s.topk == 2 ? router_softmax_stream_kernel<V4, WPR, true>
-                          : router_softmax_stream_kernel<V4, WPR, false>;
+  const bool full = s.N == 128 * WPR * V4;
+  auto kern = s.topk == 2 ? router_softmax_stream_kernel<V4, WPR, true, false>
+                          : (full ? router_softmax_stream_kernel<V4, WPR, false, true>
+                                  : router_softmax_stream_kernel<V4, WPR, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -127,11 +127,8 @@ router_wsplit_kernel(const float* __restrict__ W_r, __nv_bfloat16* __restrict__ 
   }
 }
 
-// kWide = false: fused routing of N <= NP experts (cluster of S CTAs along z).
-// kWide = true: logits only, CTA (x, y) writes tokens [128y, 128y+128) x experts
-// [NP*x, NP*x + NP) to a.logits (expert tiles fastest, so the CTAs that run
-// together share the x tile in L2); the softmax kernel routes from there.
-template <int NP, bool kWide>
+// Fused routing of N <= NP experts (cluster of S CTAs along z).
+template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const TcArgs a) {
@@ -157,17 +154,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   const int S = static_cast<int>(cluster.num_blocks());
   const int r = static_cast<int>(cluster.block_rank());
   // row stride of the logits tile: NP + 2S (= NP + threads per token in the
-  // routing below, so that a warp's reads fall in distinct banks); NP + 4 for
-  // the logits-only layout
-  const int PS = kWide ? NP + 4 : NP + 2 * S;
+  // routing below, so that a warp's reads fall in distinct banks)
+  const int PS = NP + 2 * S;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   if (blockIdx.x == 0 && blockIdx.y == 0 && r == 0 && threadIdx.x == 0) {
     a.hdr->err = kDevOk;   // per-call device status
     a.hdr->done = 0u;      // arrival counter of the dispatch scan
   }
-  const int m0 = (kWide ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x)) * kBM;
-  const int n0 = kWide ? static_cast<int>(blockIdx.x) * NP : 0;
+  const int m0 = static_cast<int>(blockIdx.x) * kBM;
+  constexpr int n0 = 0;
   const int kb0 = r * a.kb_per;
   const int nk = max(0, min(a.nkb, kb0 + a.kb_per) - kb0);
 
@@ -285,11 +281,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __syncwarp();
   } else if (warp == 3) {
     // bias row for the read-out below (named barrier 1: this warp + warps 4..7)
-    if constexpr (!kWide) {
-      for (int n = lane; n < NP; n += 32)
-        bias_s[n] = n < a.N ? (a.b_r ? a.b_r[n] : 0.f) : -INFINITY;
-      ptx::named_bar_arrive(1, 160);
-    }
+    for (int n = lane; n < NP; n += 32)
+      bias_s[n] = n < a.N ? (a.b_r ? a.b_r[n] : 0.f) : -INFINITY;
+    ptx::named_bar_arrive(1, 160);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ TMEM epilogue
     bool have = false;
@@ -298,9 +292,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       have = __all_sync(0xffffffffu, got);
       if (!have && lane == 0) fail();
     }
-    if constexpr (!kWide) ptx::named_bar_sync(1, 160);
+    ptx::named_bar_sync(1, 160);
     // a lone CTA (S = 1) holds the whole sum: the bias goes in here
-    const bool add_bias = !kWide && S == 1;
+    const bool add_bias = S == 1;
     ptx::tc_fence_after();
     const int q = warp & 3;
     const int row = q * 32 + lane;                 // TMEM lane = token row of the tile
@@ -344,26 +338,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   if (warp == 2) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, C::kTmemCols);
-  }
-  if constexpr (kWide) {
-    // coalesced rows of the logits tile (the bias is added by the softmax kernel)
-    const bool vec = (a.N % 4) == 0;
-    for (int idx = threadIdx.x; idx < kBM * (NP / 4); idx += kThreads) {
-      const int i = idx / (NP / 4), n = (idx % (NP / 4)) * 4;
-      const int t = m0 + i;
-      if (t >= a.T || n0 + n >= a.N) continue;
-      const float4 v = *reinterpret_cast<const float4*>(Ps + i * PS + n);
-      float* dst = a.logits + static_cast<size_t>(t) * a.N + n0 + n;
-      if (vec) {
-        *reinterpret_cast<float4*>(dst) = v;
-      } else {
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (n0 + n + c < a.N) dst[c] = vv[c];
-      }
-    }
-    return;
   }
   // this CTA's rows [r*R, r*R + R), with the bias added and -inf in the padded
   // columns (S > 1: written in place, the peers read only their own rows of
@@ -426,6 +400,238 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   }
 }
 
+// Logits of wide layers (N > 128 experts), persistent: one CTA per SM takes
+// tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... of 128 tokens by 128
+// experts (expert tiles fastest, so the CTAs running together share the x tile
+// in L2; W3 stays in L2), and writes them to a.logits [T, N] fp32 without the
+// bias (the softmax kernel adds it).
+//   warp 0       TMA producer: per k-block the x tile and the three piece tiles
+//                (64 KB) into a ring of kWideStages stages, across tiles
+//   warp 1       MMA issuer: per 16-wide k step x * hi into the tile's first
+//                accumulator, x * mid and x * lo into its second; kWideAcc tile
+//                accumulators in TMEM, so the read-out of one tile runs under
+//                the MMAs of the next
+//   warp 2       TMEM allocator
+//   warps 4..7   read-out (thread = token row): z = D_hi + D_midlo, 32 experts
+//                at a time, transposed through shared memory into row-major
+//                128-byte stores
+constexpr int kWideThreads = 256;
+constexpr int kWideStages = 3;
+constexpr int kWideAcc = 2;          // tile accumulators, [hi | mid+lo] = 256 columns each
+constexpr int kWideNP = 128;         // experts per tile
+constexpr int kWidePitch = 33;       // transpose tile row pitch (floats)
+using WideCfg = TcCfg<kWideNP>;
+constexpr size_t kWideBarOff = static_cast<size_t>(kWideStages) * WideCfg::kStage;
+constexpr size_t kWideStgOff = kWideBarOff + 256;
+constexpr size_t kWideSmem = 1024 + kWideStgOff + 4 * 32 * kWidePitch * sizeof(float);
+
+__global__ void __launch_bounds__(kWideThreads, 1)
+router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
+                          const __grid_constant__ CUtensorMap tmW, const TcArgs a) {
+  // tmW: W3 = [hi; mid; lo] as bf16 [3N, d], box [128 rows, 64 k], 128-byte swizzle
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kWideBarOff);
+  uint64_t* empty_bar = full_bar + kWideStages;
+  uint64_t* tfull = empty_bar + kWideStages;
+  uint64_t* tempty = tfull + kWideAcc;
+  uint64_t* drain_bar = tempty + kWideAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* stg = reinterpret_cast<float*>(smem + kWideStgOff);   // [4 warps][32][kWidePitch]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.hdr->err = kDevOk;   // per-call device status
+    a.hdr->done = 0u;      // arrival counter of the dispatch scan
+  }
+  const int n_tiles = (a.N + kWideNP - 1) / kWideNP;
+  const int total = n_tiles * ((a.T + kBM - 1) / kBM);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWideStages; ++s) {
+      ptx::mbar_init(&full_bar[s], 1);
+      ptx::mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < kWideAcc; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 4);   // one arrive per read-out warp
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmX);
+    ptx::prefetch_tmap(&tmW);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(tmem_slot, 2 * kWideAcc * kWideNP);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicExch(&a.hdr->err, kDevPipelineTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_x = ptx::l2_policy_evict_first();   // x: read by one row of tiles
+      const uint64_t pol_w = ptx::l2_policy_evict_last();    // W3: read by every tile
+      uint32_t issued = 0u, last_par = 0u;
+      pdl_wait();   // W3 comes from the split kernel
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * kWideNP;
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const int s = it % kWideStages;
+          const uint32_t ph = static_cast<uint32_t>(it / kWideStages) & 1u;
+          if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, a.wait_ns)) {
+            fail();
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * WideCfg::kStage;
+          ptx::mbar_arrive_expect_tx(&full_bar[s], WideCfg::kStage);
+          ptx::tma_load_2d(st, &tmX, &full_bar[s], kb * kBK, m0, pol_x);
+#pragma unroll
+          for (int p = 0; p < kPieces; ++p)
+            ptx::tma_load_2d(st + WideCfg::kABytes + p * WideCfg::kPieceBytes, &tmW, &full_bar[s],
+                             kb * kBK, p * a.piece_rows + n0, pol_w);
+          issued |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+        }
+      }
+      // every issued load lands before the stage memory goes away
+      for (int s = 0; s < kWideStages; ++s) {
+        if (issued & (1u << s)) {
+          volatile int never = 0;
+          if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never, a.wait_ns))
+            atomicExch(&a.hdr->err, kDevPipelineTimeout);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = ptx::umma_idesc_bf16_f32(kWideNP);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
+        const int buf = tc % kWideAcc;
+        if (!ptx::mbar_wait(&tempty[buf], (static_cast<uint32_t>(tc / kWideAcc) & 1u) ^ 1u,
+                            abort_flag, a.wait_ns)) {
+          fail();
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_hi = tmem_base + static_cast<uint32_t>(buf * 2 * kWideNP);
+        const uint32_t d_ml = d_hi + kWideNP;
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const int s = it % kWideStages;
+          const uint32_t ph = static_cast<uint32_t>(it / kWideStages) & 1u;
+          if (!ptx::mbar_wait(&full_bar[s], ph, abort_flag, a.wait_ns)) {
+            fail();
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_u32(smem + s * WideCfg::kStage);
+          const uint32_t b_addr = a_addr + WideCfg::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            const uint32_t ko = k * kUmmaK * 2;
+            const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + ko);
+            const uint32_t first = (kb | k) != 0 ? 1u : 0u;
+            ptx::umma_bf16(d_hi, ad, ptx::umma_desc_sw128_kmajor(b_addr + ko), idesc, first);
+            ptx::umma_bf16(d_ml, ad,
+                           ptx::umma_desc_sw128_kmajor(b_addr + WideCfg::kPieceBytes + ko),
+                           idesc, first);
+            ptx::umma_bf16(d_ml, ad,
+                           ptx::umma_desc_sw128_kmajor(b_addr + 2 * WideCfg::kPieceBytes + ko),
+                           idesc, 1u);
+          }
+          ptx::umma_commit(&empty_bar[s]);   // frees the stage once these MMAs are done
+        }
+        if (ok) ptx::umma_commit(&tfull[buf]);
+      }
+      // all MMAs of this thread complete before TMEM is released
+      ptx::umma_commit(drain_bar);
+      volatile int never = 0;
+      if (!ptx::mbar_wait(drain_bar, 0u, &never, a.wait_ns))
+        atomicExch(&a.hdr->err, kDevPipelineTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ read-out
+    const int q = warp & 3;                  // TMEM lanes [32q, 32q + 32): token rows
+    float* st = stg + q * 32 * kWidePitch;
+    const bool vec = (a.N % 4) == 0;
+    int tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const int buf = tc % kWideAcc;
+      const bool got = ptx::mbar_wait(&tfull[buf], static_cast<uint32_t>(tc / kWideAcc) & 1u,
+                                      abort_flag, a.wait_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) fail();
+        break;
+      }
+      ptx::tc_fence_after();
+      const int m0 = (t / n_tiles) * kBM + q * 32, n0 = (t % n_tiles) * kWideNP;
+      const uint32_t ta = tmem_base + static_cast<uint32_t>(buf * 2 * kWideNP) +
+                          (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < kWideNP / 32; ++c) {
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld_32x32b_x32(ta + static_cast<uint32_t>(c * 32), r0);
+        ptx::tmem_ld_32x32b_x32(ta + static_cast<uint32_t>(kWideNP + c * 32), r1);
+        ptx::tmem_ld_wait();
+        if (c == kWideNP / 32 - 1) {
+          // the whole accumulator is in registers: the MMAs of a later tile may reuse it
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          st[lane * kWidePitch + j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
+        __syncwarp();
+        // rows of the 32 x 32 block: 8 lanes per row, 4 rows per store
+        const int col = (lane & 7) * 4;
+        const int n = n0 + c * 32 + col;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = i * 4 + (lane >> 3);
+          const int tok = m0 + row;
+          if (tok >= a.T || n >= a.N) continue;
+          const float* src = st + row * kWidePitch + col;
+          float* dst = a.logits + static_cast<size_t>(tok) * a.N + n;
+          if (vec) {
+            *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
+          } else {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+              if (n + c4 < a.N) dst[c4] = src[c4];
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 2 * kWideAcc * kWideNP);
+  }
+}
+
 template <int NP>
 size_t tc_smem_bytes(int stages) {
   return 1024 + static_cast<size_t>(stages) * TcCfg<NP>::kStage +
@@ -438,15 +644,15 @@ size_t tc_smem_bytes(int stages) {
 // once; each CTA's prologue and routing tail then overlap the other CTA's loads
 // instead of forming a second wave.
 template <int NP>
-int tc_stages(const Shape& s, bool wide, int num_sms) {
+int tc_stages(const Shape& s, int num_sms) {
   int stages = kMaxStages;
   while (stages > 2 && tc_smem_bytes<NP>(stages) > kMaxDynSmem) --stages;
   const int64_t t_tiles = (s.T + kBM - 1) / kBM;
-  if (!wide && s.ksplit_eff == 1 && 3 * NP <= 256 && t_tiles > num_sms) stages = 2;
+  if (s.ksplit_eff == 1 && 3 * NP <= 256 && t_tiles > num_sms) stages = 2;
   return stages;
 }
 
-template <int NP, bool kWide>
+template <int NP>
 cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
                         const CUtensorMap& tmW, const float* b_r, int* expert_idx, float* gate,
                         int* local_rank, const void* pf, size_t pf_bytes, int num_sms,
@@ -469,18 +675,17 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
   a.hdr = ws.hdr;
   a.wait_ns = wait_limit_ns();
   const unsigned t_tiles = static_cast<unsigned>((s.T + kBM - 1) / kBM);
-  const int stages = tc_stages<NP>(s, kWide, num_sms);
+  const int stages = tc_stages<NP>(s, num_sms);
   // the logits tile reuses the stage memory
-  const size_t ps_bytes = static_cast<size_t>(kBM) * (NP + (kWide ? 4 : 2 * s.ksplit_eff)) * 4;
+  const size_t ps_bytes = static_cast<size_t>(kBM) * (NP + 2 * s.ksplit_eff) * 4;
   if (ps_bytes > static_cast<size_t>(stages) * TcCfg<NP>::kStage) return cudaErrorInvalidValue;
   a.stages = stages;
   const size_t smem = tc_smem_bytes<NP>(stages);
-  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NP, kWide>,
+  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<NP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = kWide ? dim3(static_cast<unsigned>((s.N + NP - 1) / NP), t_tiles, 1)
-                      : dim3(t_tiles, 1, static_cast<unsigned>(s.ksplit_eff));
+  cfg.gridDim = dim3(t_tiles, 1, static_cast<unsigned>(s.ksplit_eff));
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -488,12 +693,32 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = kWide ? 1u : static_cast<unsigned>(s.ksplit_eff);
+  attr[0].val.clusterDim.z = static_cast<unsigned>(s.ksplit_eff);
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, router_tc_kernel<NP, kWide>, tmX, tmW, a);
+  return cudaLaunchKernelEx(&cfg, router_tc_kernel<NP>, tmX, tmW, a);
+}
+
+cudaError_t launch_wide(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
+                        const CUtensorMap& tmW, int num_sms, cudaStream_t stream) {
+  TcArgs a = {};
+  a.logits = ws.logits;
+  a.T = static_cast<int>(s.T);
+  a.N = static_cast<int>(s.N);
+  a.piece_rows = static_cast<int>(s.N);
+  a.nkb = static_cast<int>((s.d + kBK - 1) / kBK);
+  a.hdr = ws.hdr;
+  a.wait_ns = wait_limit_ns();
+  const int64_t tiles = ((s.T + kBM - 1) / kBM) * ((s.N + kWideNP - 1) / kWideNP);
+  const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
+  cudaError_t e = cudaFuncSetAttribute(router_logits_wide_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kWideSmem));
+  if (e != cudaSuccess) return e;
+  return launch_dependent(router_logits_wide_kernel, dim3(grid), dim3(kWideThreads), kWideSmem,
+                          stream, tmX, tmW, a);
 }
 
 }  // namespace
@@ -503,12 +728,12 @@ int router_tc_padded_experts(int64_t N) {
 }
 
 int router_tc_stages(const Shape& s, int num_sms) {
-  if (s.router_path == kRouterTCWide) return tc_stages<128>(s, true, num_sms);
+  if (s.router_path == kRouterTCWide) return kWideStages;
   switch (router_tc_padded_experts(s.N)) {
-    case 32: return tc_stages<32>(s, false, num_sms);
-    case 64: return tc_stages<64>(s, false, num_sms);
-    case 96: return tc_stages<96>(s, false, num_sms);
-    case 128: return tc_stages<128>(s, false, num_sms);
+    case 32: return tc_stages<32>(s, num_sms);
+    case 64: return tc_stages<64>(s, num_sms);
+    case 96: return tc_stages<96>(s, num_sms);
+    case 128: return tc_stages<128>(s, num_sms);
     default: return 0;
   }
 }
@@ -529,14 +754,13 @@ cudaError_t launch_router_tc(const Shape& s, const Workspace& ws, const float* W
   count_launch();
   if (e != cudaSuccess) return e;
   if (s.router_path == kRouterTCWide) {
-    e = launch_tc_t<128, true>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch,
-                               l2_prefetch_bytes, num_sms, stream);
+    e = launch_wide(s, ws, tmX, tmW, num_sms, stream);
   } else {
     switch (router_tc_padded_experts(s.N)) {
-      case 32: e = launch_tc_t<32, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
-      case 64: e = launch_tc_t<64, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
-      case 96: e = launch_tc_t<96, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
-      case 128: e = launch_tc_t<128, false>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 32: e = launch_tc_t<32>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 64: e = launch_tc_t<64>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 96: e = launch_tc_t<96>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
+      case 128: e = launch_tc_t<128>(s, ws, tmX, tmW, b_r, expert_idx, gate, local_rank, l2_prefetch, l2_prefetch_bytes, num_sms, stream); break;
       default: e = cudaErrorInvalidValue; break;
     }
   }
