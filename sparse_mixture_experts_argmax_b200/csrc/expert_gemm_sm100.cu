@@ -471,7 +471,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     };
     // publish before blocking on a barrier that is not yet complete (warp-uniform)
     auto publish_if_blocked = [&](uint64_t* bar, uint32_t parity) {
-      if (npending > 0 && __any_sync(0xffffffffu, !ptx::mbar_try_wait(bar, parity))) publish();
+      if (npending > 0 && __any_sync(0xffffffffu, !ptx::mbar_test_wait(bar, parity))) publish();
     };
     int acc = 0;
     uint32_t aph = 0;
