@@ -628,12 +628,13 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
   }
 }
 
-// The split GEMM2 tiles, finished: group blockIdx.x / kReduceParts (an expert's
-// 128 features by one token tile), token columns [part * bn / kReduceParts, ...)
-// of it.  Each thread takes 4 features of a column: the partials added in k
-// order (deterministic), then the bias, the token's gate and the bf16 store to
-// the token's output row.  Launched after the FFN (programmatic dependency).
-constexpr int kReduceParts = 4;
+// The split GEMM2 tiles, finished: one thread per 4 features of one token
+// column of a group (an expert's 128 features by one token tile; a warp covers
+// one column, so each partial is read as 512 contiguous bytes).  Block b takes
+// items [256 * (b % parts), ...) of group b / parts (parts = bn * 32 / 256).  The
+// partials are added in k order (deterministic), then the bias, the token's
+// gate and the bf16 store to the token's output row.  Launched after the FFN
+// (programmatic dependency).
 constexpr int kReduceThreads = 256;
 __global__ void __launch_bounds__(kReduceThreads)
 ffn_split_reduce_kernel(const float* __restrict__ part, const int4* __restrict__ groups,
@@ -643,44 +644,47 @@ ffn_split_reduce_kernel(const float* __restrict__ part, const int4* __restrict__
                         int S, int bn, int M, int T_rows, int* err) {
   pdl_trigger();
   pdl_wait();   // the partial tiles and the group table come from earlier kernels
-  const int grp = blockIdx.x / kReduceParts, quarter = blockIdx.x % kReduceParts;
+  const int parts = bn * (kBM / 4) / kReduceThreads;
+  const int grp = blockIdx.x / parts;
+  const int item = (blockIdx.x % parts) * kReduceThreads + threadIdx.x;
   const int4 gd = groups[grp];
   if (gd.x < 0) return;
   const int e = gd.x, mt = gd.y, nt = gd.z;
+  const int col = item / (kBM / 4);
+  const int f4 = (item % (kBM / 4)) * 4;
+  const int f = mt * kBM + f4;
   const int rows = min(bn, __ldg(exp_rows + e) - nt * bn);
+  if (col >= rows || f >= M) return;
   const int row0 = __ldg(exp_base + e) + nt * bn;
-  const int per = (bn + kReduceParts - 1) / kReduceParts;
-  const int c_lo = quarter * per, c_hi = min(rows, c_lo + per);
+  int dst = __ldg(slot_token + row0 + col);
   const size_t tile = static_cast<size_t>(bn) * kBM;   // floats per partial tile
-  const float* base = part + static_cast<size_t>(grp) * S * tile;
-  for (int item = threadIdx.x; item < (c_hi - c_lo) * (kBM / 4); item += kReduceThreads) {
-    const int col = c_lo + item / (kBM / 4);
-    const int f4 = (item % (kBM / 4)) * 4;
-    const int f = mt * kBM + f4;
-    if (f >= M) continue;
-    const float* src = base + static_cast<size_t>(col) * kBM + f4;
-    float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-    for (int ks = 1; ks < S; ++ks) {   // partials added in k order
-      const float4 w = __ldcg(reinterpret_cast<const float4*>(src + ks * tile));
-      v.x += w.x;
-      v.y += w.y;
-      v.z += w.z;
-      v.w += w.w;
+  const float* src = part + static_cast<size_t>(grp) * S * tile + static_cast<size_t>(col) * kBM + f4;
+  float4 w[kSplitFactor];
+#pragma unroll
+  for (int ks = 0; ks < kSplitFactor; ++ks)   // every partial in flight at once
+    if (ks < S) w[ks] = __ldcg(reinterpret_cast<const float4*>(src + ks * tile));
+  if (!checked_index(dst >= 0 && dst < T_rows, err)) dst = 0;
+  const float g = __ldg(gate + dst);
+  float4 v = w[0];
+#pragma unroll
+  for (int ks = 1; ks < kSplitFactor; ++ks) {   // added in k order
+    if (ks < S) {
+      v.x += w[ks].x;
+      v.y += w[ks].y;
+      v.z += w[ks].z;
+      v.w += w[ks].w;
     }
-    int dst = __ldg(slot_token + row0 + col);
-    if (!checked_index(dst >= 0 && dst < T_rows, err)) dst = 0;
-    const float g = __ldg(gate + dst);
-    const __nv_bfloat16* bb = b2 + static_cast<size_t>(e) * M + f;
-    const float o0 = (v.x + __bfloat162float(bb[0])) * g;
-    const float o1 = (v.y + __bfloat162float(bb[1])) * g;
-    const float o2 = (v.z + __bfloat162float(bb[2])) * g;
-    const float o3 = (v.w + __bfloat162float(bb[3])) * g;
-    __nv_bfloat162 lo2 = __floats2bfloat162_rn(o0, o1), hi2 = __floats2bfloat162_rn(o2, o3);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-    *reinterpret_cast<uint2*>(out + static_cast<size_t>(dst) * M + f) = pk;
   }
+  const __nv_bfloat16* bb = b2 + static_cast<size_t>(e) * M + f;
+  const float o0 = (v.x + __bfloat162float(bb[0])) * g;
+  const float o1 = (v.y + __bfloat162float(bb[1])) * g;
+  const float o2 = (v.z + __bfloat162float(bb[2])) * g;
+  const float o3 = (v.w + __bfloat162float(bb[3])) * g;
+  __nv_bfloat162 lo2 = __floats2bfloat162_rn(o0, o1), hi2 = __floats2bfloat162_rn(o2, o3);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+  pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+  *reinterpret_cast<uint2*>(out + static_cast<size_t>(dst) * M + f) = pk;
 }
 
 size_t ffn_smem_bytes(int bn, int stages, int cached_prefix_ints, int a_tiles = 1) {
@@ -763,7 +767,10 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
                          tmB2, a);
   count_launch();
   if (err != cudaSuccess || a.split <= 1) return err;
-  err = launch_dependent(ffn_split_reduce_kernel, dim3(kSplitMaxGroups * kReduceParts),
+  if (a.split > kSplitFactor || (a.bn * (kBM / 4)) % kReduceThreads != 0)
+    return cudaErrorInvalidValue;
+  const unsigned parts = static_cast<unsigned>(a.bn * (kBM / 4) / kReduceThreads);
+  err = launch_dependent(ffn_split_reduce_kernel, dim3(kSplitMaxGroups * parts),
                          dim3(kReduceThreads), 0, stream, static_cast<const float*>(ws.part),
                          static_cast<const int4*>(static_cast<const void*>(ws.split_grp)),
                          ws.exp_rows, ws.exp_base, ws.slot_token, gate,

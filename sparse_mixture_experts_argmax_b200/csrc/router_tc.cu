@@ -55,6 +55,7 @@ constexpr int kBK = 64;           // k per stage (one 128-byte swizzle row of bf
 constexpr int kUmmaK = 16;
 constexpr int kPieces = 3;        // hi, mid, lo
 constexpr int kMaxStages = 4;
+constexpr int kXAhead = 4;        // x k-blocks requested into L2 beyond the stage ring
 constexpr size_t kMaxDynSmem = 232448 - 8192;   // leave room for the static arrays
 
 template <int NP>
@@ -207,6 +208,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         ptx::tma_load_2d(smem + i * C::kStage, &tmX, &full_bar[i], (kb0 + i) * kBK, m0, pol_x);
         issued |= 1u << i;
       }
+      // x comes from HBM: its next kXAhead k-blocks beyond the stage ring are
+      // requested into L2 ahead of their TMA loads (more bytes in flight than
+      // the stages' shared memory holds)
+      for (int i = first; i < nk && i < first + kXAhead; ++i)
+        ptx::tma_prefetch_2d(&tmX, (kb0 + i) * kBK, m0);
       pdl_wait();   // W3 comes from the split kernel
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
@@ -220,6 +226,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           }
           ptx::mbar_arrive_expect_tx(&full_bar[s], C::kStage);
           ptx::tma_load_2d(st, &tmX, &full_bar[s], kc, m0, pol_x);
+          if (i + kXAhead < nk) ptx::tma_prefetch_2d(&tmX, (kb0 + i + kXAhead) * kBK, m0);
         }
 #pragma unroll
         for (int p = 0; p < kPieces; ++p)

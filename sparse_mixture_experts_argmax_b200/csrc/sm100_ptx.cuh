@@ -142,6 +142,15 @@ __device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, 
       : "memory");
 }
 
+// Bring the box of a 2-D tensor map at (c0, c1) into L2 (no completion, no
+// shared memory: the TMA load of the same box later finds it in L2).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* tmap, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // Bring [addr, addr + bytes) into L2 (no completion; bytes a multiple of 16,
 // addr 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* addr, uint32_t bytes) {
