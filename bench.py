@@ -712,7 +712,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--shape", default=None,
-                    help="ad-hoc bf16 layer T,d,d_ff,N,capacity_factor instead of a named workload")
+                    help="ad-hoc layer T,d,d_ff,N,capacity_factor[,dtype] (dtype bf16, the "
+                         "default, or f32) instead of a named workload")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -725,9 +726,14 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.shape:
-        T, d, d_ff, N, cf = args.shape.split(",")
-        spec = synth.LayerSpec("shape_T%s_d%s_f%s_N%s_cf%s" % (T, d, d_ff, N, cf), int(T), int(d),
-                               int(d_ff), int(N), float(cf), "bf16")
+        fields = args.shape.split(",")
+        T, d, d_ff, N, cf = fields[:5]
+        dt = fields[5] if len(fields) > 5 else "bf16"
+        if dt not in ("bf16", "f32"):
+            raise SystemExit("--shape dtype must be bf16 or f32")
+        spec = synth.LayerSpec("shape_T%s_d%s_f%s_N%s_cf%s%s" % (T, d, d_ff, N, cf,
+                                                                 "" if dt == "bf16" else "_f32"),
+                               int(T), int(d), int(d_ff), int(N), float(cf), dt)
         synth.WORKLOADS[spec.name] = spec
         args.workload = spec.name
     if args.impl == "reference":

@@ -573,41 +573,24 @@ router_softmax_stream_kernel(const float* __restrict__ z, const float* __restric
   __syncthreads();
   pdl_wait();   // the logits come from the logits kernel
 
-  // the leader's cursors over its group's rows, in the consumers' order: the
-  // copies into the ring, and S rows further the L2 prefetches (twice the
-  // ring's rows in flight from HBM)
-  struct Cursor {
-    int pb, pr;
-    // the group's next row (global token index), -1 past the end
-    __device__ int next(int tpb_, int T_, int nblk_, int grp_) {
-      while (pb < nblk_ && pr >= min(tpb_, T_ - pb * tpb_)) {
-        pr = grp_;
-        pb += gridDim.x;
-      }
-      if (pb >= nblk_) return -1;
-      const int row = pb * tpb_ + pr;
-      pr += G;
-      return row;
-    }
-  };
-  Cursor cur{static_cast<int>(blockIdx.x), grp}, pfc{static_cast<int>(blockIdx.x), grp};
+  // the leader's cursor over its group's rows, in the consumers' order
+  int pb = blockIdx.x, pr = grp, issued = 0;
   const uint32_t row_bytes = static_cast<uint32_t>(N) * 4u;
-  int issued = 0;
   auto issue_next = [&]() {
-    const int row = cur.next(tpb, T, nblk, grp);
-    if (row < 0) return;
+    while (pb < nblk && pr >= min(tpb, T - pb * tpb)) {
+      pr = grp;
+      pb += gridDim.x;
+    }
+    if (pb >= nblk) return;
     uint64_t* bar = &full[grp][issued % S];
     ptx::mbar_arrive_expect_tx(bar, row_bytes);
     ptx::bulk_load_g2s(ring + static_cast<size_t>(issued % S) * N,
-                       z + static_cast<size_t>(row) * N, row_bytes, bar);
+                       z + (static_cast<size_t>(pb) * tpb + pr) * N, row_bytes, bar);
     ++issued;
-    const int ahead = pfc.next(tpb, T, nblk, grp);
-    if (ahead >= 0) ptx::prefetch_l2_bulk(z + static_cast<size_t>(ahead) * N, row_bytes);
+    pr += G;
   };
-  if (leader) {
-    for (int i = 0; i < S; ++i) pfc.next(tpb, T, nblk, grp);   // the prefetches run S rows ahead
+  if (leader)
     for (int i = 0; i < S; ++i) issue_next();
-  }
 
   const float4* bias4 = reinterpret_cast<const float4*>(s_bias);
   int ci = 0;   // rows of this group consumed
