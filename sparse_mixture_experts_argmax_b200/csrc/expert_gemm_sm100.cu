@@ -264,11 +264,9 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
 
   if (warp == 3) {
     // ------------------------------------------------------------ tile scheduler
-    // Claims the next tile only once the producer has issued every load of the
-    // previous one (so a CTA holds no second tile while most of its current one
-    // is still ahead, and a CTA that starts early cannot take two of the first
-    // tiles; the stages still in flight cover the claim), decodes it, waits for
-    // its GEMM1 rows when it is a GEMM2 tile, and publishes it in the ring.
+    // Claims the next tile only once the producer has taken the previous one (so
+    // a CTA holds at most one claimed tile it has not started), decodes it, waits
+    // for its GEMM1 rows when it is a GEMM2 tile, and publishes it in the ring.
     // Every tile comes from the counter, so only a running CTA owns a tile: when
     // a GEMM2 tile is claimed, every GEMM1 tile (lower numbers) has already been
     // claimed by a running CTA, whose pipeline finishes it without waiting on
@@ -359,6 +357,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         }
         const TileSlot ts = tile_ring[slot];
         if (ts.t < 0) break;
+        ptx::mbar_arrive(take_bar);   // the scheduler may claim the next tile
         const PhaseArgs& P = args.ph[ts.phase];
         const CUtensorMap* tA = ts.phase == 0 ? &tmA0 : &tmA1;
         const CUtensorMap* tB = ts.phase == 0 ? &tmB0 : &tmB1;
@@ -386,7 +385,6 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
           last_par = (last_par & ~(1u << stage)) | (ph << stage);
           if (++stage == stages) { stage = 0; ph ^= 1u; }
         }
-        if (ok) ptx::mbar_arrive(take_bar);   // the scheduler may claim the next tile
       }
       // drain: every issued load must land before the CTA may exit
       for (int s = 0; s < stages; ++s) {

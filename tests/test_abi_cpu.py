@@ -134,7 +134,7 @@ _PLAN_CASES = [
                                        "dispatch": "two_kernel", "tile_rows": 256,
                                        "accumulators": 2, "gemm2_split": 4}),
     ("many_T65536_d1024_N2048", None, {"router": "tc_wide", "softmax": "stream",
-                                       "dispatch": "two_kernel"}),
+                                       "dispatch": "two_kernel", "tokens_per_block": 111}),
     ("tiny_f32_T64_d32_N4", None, {"router": "ffma_warpsplit", "ffn": "f32", "dispatch": "fused"}),
     # test_kernel_variant_shapes
     ("tc_np96_s4", (1000, 1024, 256, 80, 1.25, "bf16"), {"router": "tc", "ksplit": 4}),
@@ -151,6 +151,11 @@ _PLAN_CASES = [
     ("two_accumulators", (900, 64, 64, 4, 1.0, "bf16"), {"ffn": "sm100", "accumulators": 2}),
     ("gemm2_split_mixed", (12288, 768, 4096, 8, 1.0, "bf16"),
      {"dispatch": "two_kernel", "tile_rows": 256, "gemm2_split": 4}),
+    # streaming softmax: token blocks sized so every persistent CTA takes as many
+    ("stream_full_warp_row", (6600, 128, 64, 1024, 2.0, "bf16"),
+     {"router": "tc_wide", "softmax": "stream", "tokens_per_block": 45}),
+    ("stream_pair_ragged", (5400, 128, 64, 1500, 2.0, "bf16"),
+     {"router": "tc_wide", "softmax": "stream", "tokens_per_block": 37}),
     # test_router_bias_paths
     ("tc_s1_bias_padded", (6000, 128, 64, 50, 1.25, "bf16"),
      {"router": "tc", "ksplit": 1, "router_stages": 4}),

@@ -320,6 +320,10 @@ _VARIANT_SHAPES = [
     ("two_accumulators", 900, 64, 64, 4, 1.0, "bf16"),
     # GEMM2 split over K on the first experts, unsplit tiles on the rest
     ("gemm2_split_mixed", 12288, 768, 4096, 8, 1.0, "bf16"),
+    # streaming softmax: a warp per row at full width (N = 1024), a warp pair per row
+    # with a ragged second half (N = 1500); token blocks of 45 and 37 tokens
+    ("stream_full_warp_row", 6600, 128, 64, 1024, 2.0, "bf16"),
+    ("stream_pair_ragged", 5400, 128, 64, 1500, 2.0, "bf16"),
 ]
 
 
