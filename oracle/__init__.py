@@ -10,5 +10,5 @@ from .switch_layer import (  # noqa: F401
     capacity, router_logits, router_probs, top1, positions, expert_ffn,
     load_balance_stats, aux_loss, switch_forward, switch_forward_sampled,
     logit_gap, capacity_k, top2, positions_top2, switch_forward_top2, gelu, expert_ffn_geglu,
-    switch_backward,
+    switch_backward, positions_ntlb, switch_forward_ntlb,
 )

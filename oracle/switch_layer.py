@@ -71,6 +71,22 @@ the capacity cut are piecewise constant and pass no gradient):
 * dW_r = sum_t dz_t x_t^T (the router's input: x, or x * noise), db_r = sum_t dz_t,
   dx_t += W_r^T dz_t.
 
+No-Token-Left-Behind ([ST-paper] Appendix B, in the capacity-factor discussion
+and the router-design list: tokens that overflow their first expert are sent to
+their second-choice expert, "iteratively", a two-stage process in its Figure 11;
+the paper reports no benefit).  The figure itself is not in the pages; readings:
+
+* two stages: stage 1 is the top-1 layer (first choice, capacity
+  C = ceil(cf T / N), positions in token order); stage 2 takes the tokens that
+  stage 1 dropped, in token order, and offers each to its second choice (the
+  top-2 runner-up), whose free slots are those stage 1 left: the position of an
+  overflow token there is min(count_1(e), C) + (earlier overflow tokens with the
+  same second choice); it is kept iff that position < C, else dropped for good.
+* a kept token's output is p_t,e E_e(x_t) with e the expert that kept it (the
+  gate is that expert's router probability, unnormalised); dropped tokens give 0.
+* f_i counts first choices, as in the top-1 loss formula (the rerouting is not
+  part of the router's decision).
+
 GEGLU experts and router input jitter ([ST-paper] architecture paragraph: "ReLU
 or GEGLU"; Table 11: input jitter, multiplicative noise on the router input,
 a training-time exploration, off at inference).  The pages name both without
@@ -354,6 +370,59 @@ def switch_forward_top2(x, W_r, W1, b1, W2, b2, capacity_factor: float, b_r=None
     f, P = load_balance_stats(e[:, 0], p)
     aux = aux_loss(f, P) if T else 0.0
     return {"out": out, "expert_idx": e, "gate": g, "pos_in_expert": pos, "kept": kept,
+            "capacity": C, "f": f, "P": P, "aux": aux, "probs": p, "logits": z}
+
+
+def positions_ntlb(e: np.ndarray, N: int, C: int) -> np.ndarray:
+    """No-Token-Left-Behind positions, two stages (readings in the module doc).
+    e [T, 2] holds the first and second choices; returns pos [T, 2]: pos[t, 0]
+    the stage-1 position at the first choice (its top-1 position), pos[t, 1]
+    the stage-2 position at the second choice for a token stage 1 dropped
+    (pos[t, 0] >= C), -1 for a token stage 1 kept."""
+    T = e.shape[0]
+    pos = np.full((T, 2), -1, dtype=np.int64)
+    count = [0] * N
+    for t in range(T):                      # stage 1: first choices, token order
+        i = int(e[t, 0])
+        pos[t, 0] = count[i]
+        count[i] += 1
+    filled = [min(c, C) for c in count]     # slots stage 1 took
+    for t in range(T):                      # stage 2: overflow, token order
+        if pos[t, 0] >= C:
+            i = int(e[t, 1])
+            pos[t, 1] = filled[i]
+            filled[i] += 1
+    return pos
+
+
+def switch_forward_ntlb(x, W_r, W1, b1, W2, b2, capacity_factor: float,
+                        b_r=None) -> Dict:
+    """No-Token-Left-Behind layer in float64: out [T, d], expert_idx [T, 2]
+    (first, second choice), gate [T, 2] (their router probabilities),
+    pos_in_expert [T, 2] (``positions_ntlb``), assigned [T] (the expert that
+    processes the token, -1 if dropped), capacity, f, P, aux."""
+    xs = _f64(x)
+    T = xs.shape[0]
+    N = _f64(W_r).shape[0]
+    z = router_logits(xs, W_r, b_r)
+    p = router_probs(z) if T else np.zeros((0, N))
+    e, g = top2(p, normalize=False) if T else (np.zeros((0, 2), np.int64), np.zeros((0, 2)))
+    C = capacity(T, N, capacity_factor)
+    pos = positions_ntlb(e, N, C)
+    stage1 = pos[:, 0] < C
+    stage2 = (~stage1) & (pos[:, 1] >= 0) & (pos[:, 1] < C)
+    assigned = np.where(stage1, e[:, 0], np.where(stage2, e[:, 1], -1))
+    gsel = np.where(stage1, g[:, 0], g[:, 1])
+    out = np.zeros((T, xs.shape[1]))
+    for i in range(N):
+        rows = np.nonzero(assigned == i)[0]
+        if rows.size == 0:
+            continue
+        u = expert_ffn(xs[rows], W1[i], b1[i], W2[i], b2[i])
+        out[rows] = gsel[rows, None] * u
+    f, P = load_balance_stats(e[:, 0], p)
+    aux = aux_loss(f, P) if T else 0.0
+    return {"out": out, "expert_idx": e, "gate": g, "pos_in_expert": pos, "assigned": assigned,
             "capacity": C, "f": f, "P": P, "aux": aux, "probs": p, "logits": z}
 
 

@@ -566,6 +566,90 @@ def pin_backward_dense_ffn():
     assert np.all(gr["dW_r"] == 0) and np.all(gr["db_r"] == 0)
 
 
+# ---------------------------------------------------------------------------
+# No-Token-Left-Behind (two stages; readings in the oracle's module doc)
+# ---------------------------------------------------------------------------
+def pin_ntlb_worked_example():
+    """The hand-derived two-stage examples of the golden fixture: positions and
+    the expert that keeps each token."""
+    for g in _gold("ntlb_worked_example.json")["examples"]:
+        e = np.array(g["choices"], dtype=np.int64)
+        C = g["C"]
+        pos = S.positions_ntlb(e, g["N"], C)
+        assert pos.tolist() == g["positions"]
+        got = [int(e[t, 0]) if pos[t, 0] < C else (int(e[t, 1]) if 0 <= pos[t, 1] < C else -1)
+               for t in range(len(e))]
+        assert got == g["assigned"]
+
+
+def _ntlb_by_sets(e, N, C):
+    """Assignment of a two-stage reroute written with sets: expert i keeps the
+    first C tokens choosing it first; of the tokens it dropped, token order
+    decides which take the slots left at their second choice."""
+    T = e.shape[0]
+    first = {i: [t for t in range(T) if e[t, 0] == i] for i in range(N)}
+    kept1 = {t for i in range(N) for t in first[i][:C]}
+    out = {t: int(e[t, 0]) for t in kept1}
+    for i in range(N):
+        free = C - min(len(first[i]), C)
+        cands = [t for t in range(T) if t not in kept1 and e[t, 1] == i]
+        for t in cands[:free]:
+            out[t] = i
+    return [out.get(t, -1) for t in range(T)]
+
+
+def pin_ntlb_bruteforce():
+    """Every first/second-choice assignment of T <= 5 tokens to N = 3 experts,
+    C in 0..3: the positions give the set-based assignment, stage 1 equals the
+    top-1 positions, and no expert keeps more than C tokens."""
+    pairs = [(a, b) for a in range(3) for b in range(3) if a != b]
+    for T in range(0, 6):
+        for assign in itertools.product(pairs, repeat=T):
+            e = np.array(assign, dtype=np.int64).reshape(T, 2)
+            top1_pos = S.positions(e[:, 0], 3)
+            for C in range(4):
+                pos = S.positions_ntlb(e, 3, C)
+                assert np.array_equal(pos[:, 0], top1_pos)
+                got = [int(e[t, 0]) if pos[t, 0] < C else
+                       (int(e[t, 1]) if 0 <= pos[t, 1] < C else -1) for t in range(T)]
+                assert got == _ntlb_by_sets(e, 3, C)
+                for i in range(3):
+                    assert got.count(i) <= C
+
+
+def pin_ntlb_reduces_and_reroutes():
+    """Without drops in stage 1 the layer is the top-1 layer; otherwise stage-1
+    tokens keep their top-1 rows, rerouted tokens get p_e2 E_e2(x) (torch
+    reference), and the aux loss is the top-1 loss."""
+    rng = np.random.default_rng(21)
+    T, d, d_ff, N = 60, 6, 5, 4
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(N, d)) * 2.0
+    W1, b1, W2, b2 = _rand_ffn(rng, N, d, d_ff)
+    for cf in (float(N), 1.0, 0.75):
+        r = S.switch_forward_ntlb(x, Wr, W1, b1, W2, b2, capacity_factor=cf)
+        t1 = S.switch_forward(x, Wr, W1, b1, W2, b2, capacity_factor=cf)
+        k1 = t1["kept"]
+        assert np.array_equal(r["assigned"][k1], t1["expert_idx"][k1])
+        assert np.allclose(r["out"][k1], t1["out"][k1], rtol=1e-13, atol=1e-13)
+        assert abs(r["aux"] - t1["aux"]) < 1e-13
+        p = torch.softmax(torch.from_numpy(x @ Wr.T), dim=1).numpy()
+        re = np.nonzero((~k1) & (r["assigned"] >= 0))[0]
+        if cf == float(N):
+            assert k1.all() and re.size == 0
+            assert np.allclose(r["out"], t1["out"], rtol=1e-13, atol=1e-13)
+        else:
+            assert re.size > 0
+        for t in re:
+            i = int(r["assigned"][t])
+            assert i == int(np.argsort(-p[t], kind="stable")[1])
+            ref = p[t, i] * _torch_ffn(x[t:t + 1], W1[i], b1[i], W2[i], b2[i])[0]
+            assert np.allclose(r["out"][t], ref, rtol=1e-13, atol=1e-13)
+        dropped = np.nonzero(r["assigned"] < 0)[0]
+        assert not r["out"][dropped].any()
+        assert (r["assigned"] >= 0).sum() >= k1.sum()
+
+
 ALL_PINS = [
     pin_lb_worked_example, pin_even_routing_is_one, pin_collapse_tends_to_N,
     pin_not_a_lower_bound, pin_softmax_rows_and_closed_form, pin_ties_lowest_index,
@@ -574,4 +658,5 @@ ALL_PINS = [
     pin_top2_worked_example, pin_top2_choices_and_capacity, pin_top2_positions_bruteforce,
     pin_top2_closed_forms, pin_top2_drops, pin_gelu, pin_geglu_special_cases, pin_router_jitter,
     pin_backward_finite_differences, pin_backward_dense_ffn,
+    pin_ntlb_worked_example, pin_ntlb_bruteforce, pin_ntlb_reduces_and_reroutes,
 ]

@@ -145,6 +145,50 @@ def _forward_noise_everywhere(x, W_r, W1, b1, W2, b2, capacity_factor, b_r=None,
                          activation=activation)
 
 
+def _ntlb_no_capacity_clip(e, N, C):
+    # mistake: stage 2 counts every stage-1 token as a taken slot (no min with C)
+    T = e.shape[0]
+    pos = np.full((T, 2), -1, dtype=np.int64)
+    count = [0] * N
+    for t in range(T):
+        pos[t, 0] = count[int(e[t, 0])]
+        count[int(e[t, 0])] += 1
+    for t in range(T):
+        if pos[t, 0] >= C:
+            pos[t, 1] = count[int(e[t, 1])]
+            count[int(e[t, 1])] += 1
+    return pos
+
+
+def _ntlb_reverse_order(e, N, C):
+    # mistake: stage 2 serves the overflow tokens last-first
+    T = e.shape[0]
+    pos = _orig_positions_ntlb(e, N, C)
+    filled = [min(int((e[:, 0] == i).sum()), C) for i in range(N)]
+    pos[:, 1] = -1
+    for t in reversed(range(T)):
+        if pos[t, 0] >= C:
+            pos[t, 1] = filled[int(e[t, 1])]
+            filled[int(e[t, 1])] += 1
+    return pos
+
+
+def _ntlb_single_stage(e, N, C):
+    # mistake: no rerouting at all (the top-1 layer)
+    pos = _orig_positions_ntlb(e, N, C)
+    pos[:, 1] = -1
+    return pos
+
+
+def _patched_ntlb(old_line: str, new_line: str):
+    import inspect
+    src = inspect.getsource(_orig_forward_ntlb)
+    assert old_line in src, old_line
+    ns = dict(vars(S))
+    exec(src.replace(old_line, new_line), ns)
+    return ns["switch_forward_ntlb"]
+
+
 def _patched_backward(old_line: str, new_line: str):
     """The oracle's switch_backward with one line replaced (a planted mistake)."""
     import inspect
@@ -178,6 +222,18 @@ MUTATIONS = {
     "geglu_gate_on_value": ("expert_ffn_geglu", _geglu_gate_on_value),
     "jitter_reaches_experts": ("switch_forward", _forward_noise_everywhere),
 }
+
+_orig_positions_ntlb = S.positions_ntlb
+_orig_forward_ntlb = S.switch_forward_ntlb
+MUTATIONS["ntlb_no_capacity_clip"] = ("positions_ntlb", _ntlb_no_capacity_clip)
+MUTATIONS["ntlb_reverse_order"] = ("positions_ntlb", _ntlb_reverse_order)
+MUTATIONS["ntlb_single_stage"] = ("positions_ntlb", _ntlb_single_stage)
+MUTATIONS["ntlb_first_gate_for_rerouted"] = (
+    "switch_forward_ntlb",
+    _patched_ntlb("gsel = np.where(stage1, g[:, 0], g[:, 1])", "gsel = g[:, 0]"))
+MUTATIONS["ntlb_normalised_gates"] = (
+    "switch_forward_ntlb",
+    _patched_ntlb("e, g = top2(p, normalize=False)", "e, g = top2(p, normalize=True)"))
 
 _orig_backward = S.switch_backward
 _BACKWARD_MUTATIONS = {
