@@ -74,6 +74,8 @@ typedef enum swl_dtype { SWL_F32 = 0, SWL_BF16 = 1 } swl_dtype;
 #define SWL_WS_HOST_IO 1
 /* Workspace flag: size for switch_layer_forward_top2 (not combinable with SWL_WS_HOST_IO). */
 #define SWL_WS_TOP2 2
+/* Workspace flag: size for switch_layer_forward_ntlb (not combinable with the others). */
+#define SWL_WS_NTLB 4
 
 /* Number of timed stages and their order (see switch_layer_forward_timed):
  * 0 router (logits; for N <= 128 also softmax/argmax/ranks; bf16 layers include
@@ -90,8 +92,8 @@ typedef enum swl_dtype { SWL_F32 = 0, SWL_BF16 = 1 } swl_dtype;
  * not finite and positive; saturates at INT64_MAX. */
 int64_t switch_layer_capacity(int64_t T, int64_t N, double capacity_factor);
 
-/* Device workspace bytes needed by a forward call of this shape (flags: 0 or
- * SWL_WS_HOST_IO).  The workspace must be 256-byte aligned; its contents need
+/* Device workspace bytes needed by a forward call of this shape (flags: 0,
+ * SWL_WS_HOST_IO, SWL_WS_TOP2 or SWL_WS_NTLB).  The workspace must be 256-byte aligned; its contents need
  * no initialisation.  Returns SWL_ERR_INVALID_ARG / SWL_ERR_UNSUPPORTED for
  * shapes the forward call would reject. */
 swl_status switch_layer_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
@@ -144,6 +146,32 @@ swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t
                                      int32_t* expert_idx, float* gate, int32_t* pos_in_expert,
                                      float* aux_loss, const float* b_r, void* workspace,
                                      size_t workspace_bytes, void* stream);
+
+/* No-Token-Left-Behind variant (paper-graph summary of arXiv 2101.03961,
+ * Appendix B, in the capacity-factor discussion: tokens that overflow their
+ * first expert are rerouted to their second-choice expert, a two-stage process;
+ * the paper reports no benefit from it).  The readings taken:
+ *   e_t,0, e_t,1  first and second choice as in switch_layer_forward_top2;
+ *                 g_t,k = p_t,e_t,k (unnormalised)
+ *   C             = ceil(capacity_factor * T / N), one slot per token (top-1)
+ *   stage 1       pos_t,0 = first choices of e_t,0 by tokens before t (the top-1
+ *                 position); the token is kept there iff pos_t,0 < C
+ *   stage 2       for a token stage 1 dropped, in token order:
+ *                 pos_t,1 = min(c_e, C) + (earlier tokens stage 1 dropped whose
+ *                 second choice is e = e_t,1), c_e = first choices of e;
+ *                 kept at e_t,1 iff pos_t,1 < C; pos_t,1 = -1 for a token stage 1 kept
+ *   out_t         = g_t,k E_e_t,k(x_t) for the stage k that keeps it, else 0
+ *   aux           = N * sum_i f_i P_i with f_i counting first choices
+ * expert_idx, gate and pos_in_expert are [T, 2] (row-major).  Requires
+ * 2 <= N <= 2048, ReLU experts and a workspace sized with SWL_WS_NTLB; other
+ * arguments, layouts and errors as switch_layer_forward. */
+swl_status switch_layer_forward_ntlb(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                     const void* x, const float* W_r, const void* W1,
+                                     const void* b1, const void* W2, const void* b2,
+                                     double capacity_factor, void* out, int32_t* expert_idx,
+                                     float* gate, int32_t* pos_in_expert, float* aux_loss,
+                                     const float* b_r, void* workspace, size_t workspace_bytes,
+                                     void* stream);
 
 /* Backward pass of switch_layer_forward (top-1 routing, ReLU experts): the
  * gradients of L = sum(dout * out) + daux * aux_loss.  The router's gradient

@@ -27,6 +27,7 @@ LIB_PATH = os.path.join(_HERE, "libswitchlayer_checked.so"
 SWL_F32, SWL_BF16 = 0, 1
 SWL_WS_HOST_IO = 1
 SWL_WS_TOP2 = 2
+SWL_WS_NTLB = 4
 SWL_NUM_STAGES = 5
 STATUS = {0: "SWL_OK", 1: "SWL_ERR_INVALID_ARG", 2: "SWL_ERR_UNSUPPORTED",
           3: "SWL_ERR_WORKSPACE", 4: "SWL_ERR_CUDA", 5: "SWL_ERR_DEVICE"}
@@ -41,7 +42,7 @@ EXPORTS = ("switch_layer_capacity", "switch_layer_workspace_size", "switch_layer
            "switch_layer_noalloc_status", "switch_layer_shard_record_bytes",
            "switch_layer_forward_shard_begin", "switch_layer_forward_shard_end",
            "switch_layer_set_wait_limit_ns", "switch_layer_set_stall_test",
-           "switch_layer_forward_top2", "switch_layer_ep_max_recv_rows",
+           "switch_layer_forward_top2", "switch_layer_forward_ntlb", "switch_layer_ep_max_recv_rows",
            "switch_layer_ep_workspace_size", "switch_layer_ep_counts",
            "switch_layer_ep_dispatch", "switch_layer_ep_experts", "switch_layer_ep_combine",
            "switch_layer_variant_workspace_size", "switch_layer_forward_variant",
@@ -150,6 +151,8 @@ def lib() -> ctypes.CDLL:
                                                _FWD_ARGS[18:])
     L.switch_layer_forward_top2.restype = _i32
     L.switch_layer_forward_top2.argtypes = _FWD_ARGS[:12] + [_i32] + _FWD_ARGS[12:]
+    L.switch_layer_forward_ntlb.restype = _i32
+    L.switch_layer_forward_ntlb.argtypes = _FWD_ARGS
     L.switch_layer_set_wait_limit_ns.restype = _i32
     L.switch_layer_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.switch_layer_set_stall_test.restype = _i32
@@ -295,6 +298,32 @@ def switch_layer_forward_top2(x, W_r, W1, b1, W2, b2, capacity_factor, normalize
         _ptr(b2), float(capacity_factor), 1 if normalize else 0, _ptr(out), _ptr(expert_idx),
         _ptr(gate), _ptr(pos_in_expert), _ptr(aux_loss), _ptr(b_r), _ptr(workspace),
         workspace.numel(), _stream_handle(stream)), "forward_top2")
+
+
+def switch_layer_forward_ntlb(x, W_r, W1, b1, W2, b2, capacity_factor, out, expert_idx, gate,
+                              pos_in_expert, aux_loss, b_r=None, workspace=None,
+                              stream=None) -> None:
+    """Enqueue one forward pass of the No-Token-Left-Behind variant (expert_idx,
+    gate, pos_in_expert are [T, 2]; workspace sized with SWL_WS_NTLB)."""
+    T, d, d_ff, N = _shape_of(x, W1, W_r)
+    act = x.dtype
+    for t, n in ((x, "x"), (W1, "W1"), (b1, "b1"), (W2, "W2"), (b2, "b2"), (out, "out")):
+        _require(t, n, act)
+    _require(W_r, "W_r", torch.float32)
+    if b_r is not None:
+        _require(b_r, "b_r", torch.float32)
+    for t, n, dt in ((expert_idx, "expert_idx", torch.int32), (gate, "gate", torch.float32),
+                     (pos_in_expert, "pos_in_expert", torch.int32)):
+        _require(t, n, dt)
+        if t.numel() != 2 * T:
+            raise ValueError("%s must hold [T, 2] values" % n)
+    _require(aux_loss, "aux_loss", torch.float32)
+    _require(workspace, "workspace", torch.uint8)
+    _check(lib().switch_layer_forward_ntlb(
+        T, d, d_ff, N, dtype_code(act), _ptr(x), _ptr(W_r), _ptr(W1), _ptr(b1), _ptr(W2),
+        _ptr(b2), float(capacity_factor), _ptr(out), _ptr(expert_idx), _ptr(gate),
+        _ptr(pos_in_expert), _ptr(aux_loss), _ptr(b_r), _ptr(workspace), workspace.numel(),
+        _stream_handle(stream)), "forward_ntlb")
 
 
 def switch_layer_forward_host_io(x_host, W_r, W1, b1, W2, b2, capacity_factor, out_host,
@@ -474,10 +503,12 @@ def switch_layer_forward_shard_end(x, W1, b1, W2, b2, capacity_factor, T_total, 
 # convenience: allocate outputs + workspace with torch and run
 # ---------------------------------------------------------------------------
 def alloc_workspace(T, d, d_ff, N, act_dtype: torch.dtype, capacity_factor: float,
-                    host_io: bool = False, device="cuda", top2: bool = False) -> torch.Tensor:
+                    host_io: bool = False, device="cuda", top2: bool = False,
+                    ntlb: bool = False) -> torch.Tensor:
     n = switch_layer_workspace_size(T, d, d_ff, N, dtype_code(act_dtype), capacity_factor,
                                     (SWL_WS_HOST_IO if host_io else 0) |
-                                    (SWL_WS_TOP2 if top2 else 0))
+                                    (SWL_WS_TOP2 if top2 else 0) |
+                                    (SWL_WS_NTLB if ntlb else 0))
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
@@ -558,6 +589,31 @@ def forward_top2(inputs: dict, capacity_factor: float, normalize: bool = True,
          "aux_loss": torch.empty(1, dtype=torch.float32, device=x.device)}
     switch_layer_forward_top2(x, inputs["W_r"], W1, inputs["b1"], inputs["W2"], inputs["b2"],
                               capacity_factor, normalize, o["out"], o["expert_idx"], o["gate"],
+                              o["pos_in_expert"], o["aux_loss"], b_r=inputs.get("b_r"),
+                              workspace=workspace, stream=stream)
+    if check:
+        _check(switch_layer_device_status(workspace, stream), "device status")
+    return o
+
+
+def forward_ntlb(inputs: dict, capacity_factor: float,
+                 workspace: Optional[torch.Tensor] = None, stream=None,
+                 check: bool = True) -> dict:
+    """Run the No-Token-Left-Behind variant on ``inputs`` (CUDA tensors); [T, 2]
+    routing outputs."""
+    x, W1 = inputs["x"], inputs["W1"]
+    T, d = x.shape
+    N, d_ff, _ = W1.shape
+    if workspace is None:
+        workspace = alloc_workspace(T, d, d_ff, N, x.dtype, capacity_factor, device=x.device,
+                                    ntlb=True)
+    o = {"out": torch.empty((T, d), dtype=x.dtype, device=x.device),
+         "expert_idx": torch.empty((T, 2), dtype=torch.int32, device=x.device),
+         "gate": torch.empty((T, 2), dtype=torch.float32, device=x.device),
+         "pos_in_expert": torch.empty((T, 2), dtype=torch.int32, device=x.device),
+         "aux_loss": torch.empty(1, dtype=torch.float32, device=x.device)}
+    switch_layer_forward_ntlb(x, inputs["W_r"], W1, inputs["b1"], inputs["W2"], inputs["b2"],
+                              capacity_factor, o["out"], o["expert_idx"], o["gate"],
                               o["pos_in_expert"], o["aux_loss"], b_r=inputs.get("b_r"),
                               workspace=workspace, stream=stream)
     if check:

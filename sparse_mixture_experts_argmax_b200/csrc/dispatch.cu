@@ -779,6 +779,171 @@ ep_combine_kernel(const TA* __restrict__ ret, const int* __restrict__ expert_idx
   }
 }
 
+// ---------------------------------------------------------------- No-Token-Left-Behind
+// Two stages (paper-graph summary of arXiv 2101.03961, Appendix B: tokens that
+// overflow their first expert go to their second choice).  Stage 1 is the top-1
+// dispatch of the first choices (the scan over the router's first-choice block
+// counts gives each block's offsets); stage 2 ranks, in token order, the tokens
+// stage 1 dropped among those with the same second choice, and a second scan
+// gives the blocks' offsets; a token rerouted to expert e takes position
+// min(first-choice count of e, C) + its stage-2 offset and rank.
+constexpr int kNtlbThreads = 256;
+
+// Stage 2 for one token block: each token's stage-1 position (written to
+// pos_in_expert[2t]); the block's overflow tokens' in-block ranks per second
+// choice (rank2) and counts (blk_cnt2 row b, every expert).
+__global__ void __launch_bounds__(kNtlbThreads)
+ntlb_stage2_kernel(const int* __restrict__ expert_idx, const int* __restrict__ blk_off1,
+                   int* __restrict__ pos_in_expert, int* __restrict__ rank2,
+                   int* __restrict__ blk_cnt2, int T, int N, int tpb, int C_cmp, int* err) {
+  __shared__ int e1s[kTokensPerBlock], e2s[kTokensPerBlock], over[kTokensPerBlock];
+  pdl_trigger();
+  pdl_wait();   // the first-choice offsets come from the stage-1 scan
+  const int b = blockIdx.x, t0 = b * tpb, nt = min(tpb, T - t0);
+  int* cnt_row = blk_cnt2 + static_cast<size_t>(b) * N;
+  for (int n = threadIdx.x; n < N; n += kNtlbThreads) cnt_row[n] = 0;
+  for (int i = threadIdx.x; i < nt; i += kNtlbThreads) {
+    int e1 = expert_idx[2 * (t0 + i)], e2 = expert_idx[2 * (t0 + i) + 1];
+    if (!checked_index(e1 >= 0 && e1 < N && e2 >= 0 && e2 < N, err)) e1 = e2 = 0;
+    e1s[i] = e1;
+    e2s[i] = e2;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nt; i += kNtlbThreads) {
+    const int e = e1s[i];
+    int r = 0;
+    for (int j = 0; j < i; ++j) r += (e1s[j] == e);
+    const int p1 = blk_off1[static_cast<size_t>(b) * N + e] + r;
+    pos_in_expert[2 * (t0 + i)] = p1;
+    over[i] = p1 >= C_cmp ? 1 : 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nt; i += kNtlbThreads) {
+    if (!over[i]) continue;
+    const int e = e2s[i];
+    int r = 0;
+    for (int j = 0; j < i; ++j) r += over[j] & (e2s[j] == e);
+    rank2[t0 + i] = r;
+    if (r == 0) {   // the block's first overflow token with this second choice counts them
+      int c = 1;
+      for (int j = i + 1; j < nt; ++j) c += over[j] & (e2s[j] == e);
+      cnt_row[e] = c;
+    }
+  }
+}
+
+// Expert level (one CTA): kept rows per expert (stage-1 rows, then the stage-2
+// rows up to the capacity), packed-row bases, tile prefix, the FFN's per-call
+// state, and the aux loss from the first-choice counts.
+__global__ void __launch_bounds__(kScanThreads)
+ntlb_finish_kernel(const int* __restrict__ tot1, const int* __restrict__ tot2,
+                   const double* __restrict__ psum64, int* __restrict__ exp_rows,
+                   int* __restrict__ exp_base, int* __restrict__ tile_prefix,
+                   int* __restrict__ ready, float* __restrict__ aux_loss, WsHeader* hdr, int N,
+                   int T, int C_cmp, int tile_rows) {
+  __shared__ int s_warp[kScanWarps];
+  __shared__ int s_tot_rows, s_tot_tiles;
+  __shared__ double s_aux[kScanWarps];
+  pdl_trigger();
+  pdl_wait();   // the stage-2 totals come from the second scan
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = (N + kScanThreads - 1) / kScanThreads;
+  const int e0 = threadIdx.x * chunk, e1 = min(N, e0 + chunk);
+  auto rows_of = [&](int i) {
+    const int k1 = min(tot1[i], C_cmp);
+    return k1 + min(tot2[i], C_cmp - k1);
+  };
+  int rows = 0, tiles = 0;
+  double aux = 0.0;
+  for (int i = e0; i < e1; ++i) {
+    const int m = rows_of(i);
+    rows += m;
+    tiles += (m + tile_rows - 1) / tile_rows;
+    aux += static_cast<double>(tot1[i]) * psum64[i];
+  }
+  int base_rows = block_excl_scan(rows, s_warp, &s_tot_rows);
+  int base_tiles = block_excl_scan(tiles, s_warp, &s_tot_tiles);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) aux += __shfl_xor_sync(0xffffffffu, aux, off);
+  if (lane == 0) s_aux[warp] = aux;
+  __syncthreads();
+  for (int i = threadIdx.x; i < s_tot_tiles; i += kScanThreads) ready[i] = 0;
+  if (threadIdx.x == 0) {
+    double a = 0.0;
+    for (int w = 0; w < kScanWarps; ++w) a += s_aux[w];
+    tile_prefix[N] = s_tot_tiles;
+    hdr->next_tile = 0u;
+    *aux_loss = static_cast<float>(static_cast<double>(N) * a /
+                                   (static_cast<double>(T) * static_cast<double>(T)));
+  }
+  for (int i = e0; i < e1; ++i) {
+    const int m = rows_of(i);
+    exp_rows[i] = m;
+    exp_base[i] = base_rows;
+    tile_prefix[i] = base_tiles;
+    base_rows += m;
+    base_tiles += (m + tile_rows - 1) / tile_rows;
+  }
+}
+
+// One warp per token: the expert that keeps it (the first choice in stage 1,
+// else the second in stage 2, else none), its position (pos_in_expert[2t + 1]:
+// the stage-2 position, -1 for a token stage 1 kept), the packed row, the row
+// of x copied there and the keeping expert's router probability; a token
+// neither stage keeps gets a zero output row.
+template <int VEC>
+__global__ void __launch_bounds__(kGatherThreads)
+ntlb_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ expert_idx,
+                   const float* __restrict__ gate, int* __restrict__ pos_in_expert,
+                   const int* __restrict__ rank2, const int* __restrict__ blk_off2,
+                   const int* __restrict__ tot1, const int* __restrict__ exp_base,
+                   int* __restrict__ slot_token, float* __restrict__ gsel,
+                   uint8_t* __restrict__ xbuf, uint8_t* __restrict__ out, int T, int N, int tpb,
+                   int C_cmp, int row_bytes, int* err) {
+  using V = typename std::conditional<VEC == 16, uint4, uint32_t>::type;
+  pdl_trigger();
+  pdl_wait();   // bases come from the finish kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kGatherWarps + warp;
+  if (t >= T) return;
+  int e1 = expert_idx[2 * t], e2 = expert_idx[2 * t + 1];
+  if (!checked_index(e1 >= 0 && e1 < N && e2 >= 0 && e2 < N, err)) e1 = e2 = 0;
+  const int p1 = pos_in_expert[2 * t];
+  int e = -1, pos = 0, p2 = -1;
+  float g = 0.f;
+  if (p1 < C_cmp) {
+    e = e1;
+    pos = p1;
+    g = gate[2 * t];
+  } else {
+    const int b = t / tpb;
+    p2 = min(tot1[e2], C_cmp) + blk_off2[static_cast<size_t>(b) * N + e2] + rank2[t];
+    if (p2 < C_cmp) {
+      e = e2;
+      pos = p2;
+      g = gate[2 * t + 1];
+    }
+  }
+  if (lane == 0) pos_in_expert[2 * t + 1] = p2;
+  const int nv = row_bytes / VEC;
+  if (e >= 0) {
+    const int row = exp_base[e] + pos;
+    if (!checked_index(row >= 0 && row < T, err)) return;
+    if (lane == 0) {
+      slot_token[row] = t;
+      gsel[t] = g;
+    }
+    const V* src = reinterpret_cast<const V*>(x + static_cast<size_t>(t) * row_bytes);
+    V* dst = reinterpret_cast<V*>(xbuf + static_cast<size_t>(row) * row_bytes);
+    for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+  } else {
+    V* dst = reinterpret_cast<V*>(out + static_cast<size_t>(t) * row_bytes);
+    V z;
+    memset(&z, 0, sizeof(V));
+    for (int i = lane; i < nv; i += 32) dst[i] = z;
+  }
+}
+
 }  // namespace
 
 bool dispatch_fused_ok(const Shape& s) {
@@ -926,6 +1091,72 @@ cudaError_t launch_ep_combine(const Shape& s, const Workspace& ws, const void* r
                          static_cast<const int*>(ws.exp_off), static_cast<float*>(out),
                          (int)s.T, (int)s.d, (int)s.C_cmp, ws.hdr);
   }
+  count_launch();
+  return e;
+}
+
+
+// ---------------------------------------------------------------- No-Token-Left-Behind launches
+static cudaError_t launch_scan_totals(const Shape& s, const Workspace& ws, const int* blk_cnt,
+                               int* blk_off, int* exp_cnt, cudaStream_t stream) {
+  // the scan kernel's shard mode: per-block offsets and per-expert totals only
+  // (its expert-level part is left to ntlb_finish_kernel)
+  const int grid = (int)((s.N + 31) / 32);
+  const cudaError_t e = launch_dependent(
+      dispatch_scan_kernel, dim3(grid), dim3(kScanThreads), 0, stream, blk_cnt, ws.blk_psum,
+      blk_off, exp_cnt, ws.psum64, ws.exp_rows, ws.exp_base, ws.tile_prefix, ws.ready,
+      static_cast<float*>(nullptr), ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff,
+      s.tile_rows, static_cast<uint8_t*>(ws.ntlb_rec), (int)shard_record_psum_offset(s.N),
+      static_cast<const int*>(nullptr), static_cast<int*>(nullptr),
+      SplitPlan{1, 1, 0, nullptr, nullptr, nullptr});
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_ntlb_positions(const Shape& s, const Workspace& ws, const int* expert_idx,
+                                  int* pos_in_expert, float* aux_loss, cudaStream_t stream) {
+  cudaError_t e;
+  // stage 1: offsets of the first choices (the router's first-choice block counts)
+  if ((e = launch_scan_totals(s, ws, ws.blk_count1, ws.blk_off, ws.exp_count1, stream)) !=
+      cudaSuccess)
+    return e;
+  e = launch_dependent(ntlb_stage2_kernel, dim3(s.nblk), dim3(kNtlbThreads), 0, stream,
+                       expert_idx, static_cast<const int*>(ws.blk_off), pos_in_expert,
+                       ws.ntlb_rank2, ws.blk_count, (int)s.T, (int)s.N, s.tpb, (int)s.C_cmp,
+                       &ws.hdr->err);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  // stage 2: offsets of the overflow tokens per second choice
+  if ((e = launch_scan_totals(s, ws, ws.blk_count, ws.blk_off, ws.exp_count, stream)) !=
+      cudaSuccess)
+    return e;
+  e = launch_dependent(ntlb_finish_kernel, dim3(1), dim3(kScanThreads), 0, stream,
+                       static_cast<const int*>(ws.exp_count1),
+                       static_cast<const int*>(ws.exp_count),
+                       static_cast<const double*>(ws.psum64), ws.exp_rows, ws.exp_base,
+                       ws.tile_prefix, ws.ready, aux_loss, ws.hdr, (int)s.N, (int)s.T,
+                       (int)s.C_cmp, s.tile_rows);
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_ntlb_gather(const Shape& s, const Workspace& ws, const void* x,
+                               const int* expert_idx, const float* gate, int* pos_in_expert,
+                               void* out, cudaStream_t stream) {
+  const int elem = s.dtype == 1 ? 2 : 4;
+  const int row_bytes = (int)(s.d * elem);
+  const bool vec16 = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(out) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ws.xbuf) & 15) == 0);
+  const int grid = (int)((s.T + kGatherWarps - 1) / kGatherWarps);
+  const cudaError_t e = launch_dependent(vec16 ? ntlb_gather_kernel<16> : ntlb_gather_kernel<4>, dim3(grid),
+                       dim3(kGatherThreads), 0, stream, static_cast<const uint8_t*>(x),
+                       expert_idx, gate, pos_in_expert, static_cast<const int*>(ws.ntlb_rank2),
+                       static_cast<const int*>(ws.blk_off),
+                       static_cast<const int*>(ws.exp_count1),
+                       static_cast<const int*>(ws.exp_base), ws.slot_token, ws.ntlb_gate,
+                       static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T,
+                       (int)s.N, s.tpb, (int)s.C_cmp, row_bytes, &ws.hdr->err);
   count_launch();
   return e;
 }

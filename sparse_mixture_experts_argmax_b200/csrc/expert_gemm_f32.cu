@@ -118,7 +118,7 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
   const int K = static_cast<int>(which == 0 ? s.d : s.d_ff);
   const float* act = static_cast<const float*>(which == 0 ? ws.xbuf : ws.hbuf);
   // upper bound on row tiles: sum_e ceil(m_e / 32) <= A / 32 + N (A = T * topk rows)
-  const int64_t max_tiles = (s.T * s.topk + kTile - 1) / kTile + s.N;
+  const int64_t max_tiles = (packed_rows(s) + kTile - 1) / kTile + s.N;
   dim3 grid(static_cast<unsigned>(max_tiles), (M + kTile - 1) / kTile);
   const bool glu = which == 0 && s.glu;
   const cudaError_t e = launch_dependent(
@@ -128,7 +128,7 @@ cudaError_t launch_expert_gemm_f32(const Shape& s, const Workspace& ws, int whic
       static_cast<const int*>(ws.exp_rows), static_cast<const int*>(ws.exp_base),
       static_cast<const int*>(ws.slot_token), gate, static_cast<float*>(out),
       static_cast<int>(s.N), M, K, which == 1 && gate == nullptr ? 2 : which,
-      static_cast<int>(s.T * s.topk), &ws.hdr->err);
+      static_cast<int>(packed_rows(s)), &ws.hdr->err);
   count_launch();
   return e;
 }

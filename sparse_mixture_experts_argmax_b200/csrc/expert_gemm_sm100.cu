@@ -725,7 +725,7 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.wait_ns = wait_limit_ns();
   a.stall_test = stall_test_enabled() ? 1 : 0;
   a.num_experts = static_cast<int>(s.N);
-  a.T_rows = static_cast<int>(s.T * s.topk);   // packed rows; top-2 writes per assignment
+  a.T_rows = static_cast<int>(packed_rows(s));   // packed rows; top-2 writes per assignment
   a.bn = s.tile_rows;
   a.glu = s.glu ? 1 : 0;
   if (a.glu) {

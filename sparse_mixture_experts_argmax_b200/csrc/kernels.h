@@ -55,6 +55,10 @@ struct Workspace {
   void* xbuf;           // [A, d] packed expert inputs (act dtype), A = T * topk
   void* hbuf;           // [A, d_ff] packed hidden activations (act dtype)
   void* ybuf;           // top-2: [A, d] gated expert output per assignment (act dtype)
+  int* ntlb_rank2;      // No-Token-Left-Behind: [T] in-block rank of an overflow token
+                        // among the block's overflow tokens with the same second choice
+  float* ntlb_gate;     // No-Token-Left-Behind: [T] router probability of the keeping expert
+  void* ntlb_rec;       // No-Token-Left-Behind: per-expert totals scratch of the two scans
   // host-I/O staging (only with SWL_WS_HOST_IO)
   void* x_dev;
   void* out_dev;
@@ -78,6 +82,8 @@ struct Shape {
   int glu;        // 1: GEGLU experts (W1 [N, 2 d_ff, d]: gate rows, then value rows)
   int jitter;     // 1: the router sees x * noise (a jittered fp32 copy of x, FFMA router)
   int normalize;  // top-2: gates divided by their sum
+  int ntlb;       // 1: No-Token-Left-Behind (top-2 router, one slot per token, capacity of
+                  // top-1; tokens stage 1 drops go to their second choice's free slots)
   int router_path;  // RouterPath
   int tpb;        // tokens per block of the softmax / rank / gather stages (<= kTokensPerBlock)
   int nblk;       // ceil(T / tpb)
@@ -106,6 +112,10 @@ struct RouterPlan {
 RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk = 1);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
+
+// Packed expert rows an FFN call may fill: one per assignment (T * topk), one per
+// token for No-Token-Left-Behind.
+inline int64_t packed_rows(const Shape& s) { return s.T * (s.ntlb ? 1 : s.topk); }
 
 // ---- stage launchers (all asynchronous on `stream`; return cudaGetLastError()).
 // N <= kFusedRouterMaxN: one fused kernel (logits + softmax + block statistics);
@@ -159,6 +169,13 @@ struct SplitPlan {
 // exchange record and the expert-level part waits for launch_shard_combine.
 cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux_loss,
                                  void* record, cudaStream_t stream);
+// No-Token-Left-Behind (s.ntlb): the two stages' positions, kept rows and aux
+// loss (after the top-2 router), then the gather of the kept tokens' rows.
+cudaError_t launch_ntlb_positions(const Shape& s, const Workspace& ws, const int* expert_idx,
+                                  int* pos_in_expert, float* aux_loss, cudaStream_t stream);
+cudaError_t launch_ntlb_gather(const Shape& s, const Workspace& ws, const void* x,
+                               const int* expert_idx, const float* gate, int* pos_in_expert,
+                               void* out, cudaStream_t stream);
 // Exchange record of one rank: int32 counts [N], then fp64 sums of p [N] at a
 // 16-byte aligned offset.
 size_t shard_record_psum_offset(int64_t N);

@@ -42,8 +42,8 @@ static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws) {
   const size_t elem = s.dtype == SWL_BF16 ? 2 : 4;
   const size_t T = static_cast<size_t>(s.T), N = static_cast<size_t>(s.N);
-  const size_t A = T * static_cast<size_t>(s.topk);   // expert assignments
-  const bool top2 = s.topk == 2;
+  const size_t A = static_cast<size_t>(packed_rows(s));   // packed expert rows
+  const bool top2 = s.topk == 2;   // the top-2 router's arrays (also No-Token-Left-Behind)
   const size_t nb = static_cast<size_t>(s.nblk);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -83,7 +83,10 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.xj = reinterpret_cast<float*>(take(s.jitter ? T * static_cast<size_t>(s.d) * 4 : 0));
   w.xbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d) * elem));
   w.hbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d_ff) * elem));
-  w.ybuf = reinterpret_cast<void*>(take(top2 ? A * static_cast<size_t>(s.d) * elem : 0));
+  w.ybuf = reinterpret_cast<void*>(take(top2 && !s.ntlb ? A * static_cast<size_t>(s.d) * elem : 0));
+  w.ntlb_rank2 = reinterpret_cast<int*>(take(s.ntlb ? T * 4 : 0));
+  w.ntlb_gate = reinterpret_cast<float*>(take(s.ntlb ? T * 4 : 0));
+  w.ntlb_rec = reinterpret_cast<void*>(take(s.ntlb ? shard_record_bytes(s.N) : 0));
   if (host_io) {
     w.x_dev = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
     w.out_dev = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
@@ -147,8 +150,11 @@ static bool aligned(const void* p, uintptr_t a) {
 // Fills Shape; returns SWL_OK or the validation error.
 static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype, double cf,
                              Shape* s, int topk = 1, int normalize = 1, int glu = 0,
-                             int jitter = 0) {
+                             int jitter = 0, int ntlb = 0) {
   if (T < 0 || d <= 0 || d_ff <= 0 || N <= 0) return SWL_ERR_INVALID_ARG;
+  // No-Token-Left-Behind routes with the top-2 router (first and second choice,
+  // unnormalised gates) and keeps at most one slot per token
+  if (ntlb && (topk != 2 || normalize || glu || jitter)) return SWL_ERR_INVALID_ARG;
   if (topk != 1 && topk != 2) return SWL_ERR_INVALID_ARG;
   if (topk == 2 && N < 2) return SWL_ERR_INVALID_ARG;                    // two experts needed
   if (topk == 2 && N > kStreamSoftmaxMaxN) return SWL_ERR_UNSUPPORTED;
@@ -164,13 +170,15 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->d_ff = d_ff;
   s->N = N;
   s->dtype = dtype;
-  // top-k capacity ceil(k cf T / N) = the formula's value for k T tokens
-  s->C = switch_layer_capacity(T * topk, N, cf);
+  // top-k capacity ceil(k cf T / N) = the formula's value for k T tokens (one
+  // slot per token for No-Token-Left-Behind: the top-1 capacity)
+  s->C = switch_layer_capacity(T * (ntlb ? 1 : topk), N, cf);
   s->C_eff = s->C < T ? s->C : T;   // a token has at most one assignment per expert
   s->T_total = T;
   s->C_cmp = s->C_eff;
   s->sharded = 0;
   s->topk = topk;
+  s->ntlb = ntlb ? 1 : 0;
   s->normalize = normalize ? 1 : 0;
   s->glu = glu ? 1 : 0;
   s->jitter = jitter ? 1 : 0;
@@ -312,9 +320,9 @@ static swl_status run_ffn(const Shape& s, const Workspace& ws, const void* W1, c
     if (sms <= 0) return SWL_ERR_CUDA;
     CUtensorMap a1, b1m, a2, b2m;
     if (!make_tmap_bf16(&a1, W1, s.d, s.N * s.d_ff * (s.glu ? 2 : 1), 128) ||
-        !make_tmap_bf16(&b1m, ws.xbuf, s.d, s.T * s.topk, s.tile_rows) ||
+        !make_tmap_bf16(&b1m, ws.xbuf, s.d, packed_rows(s), s.tile_rows) ||
         !make_tmap_bf16(&a2, W2, s.d_ff, s.N * s.d, 128) ||
-        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, s.T * s.topk, s.tile_rows))
+        !make_tmap_bf16(&b2m, ws.hbuf, s.d_ff, packed_rows(s), s.tile_rows))
       return SWL_ERR_CUDA;
     if (launch_expert_ffn_bf16(s, ws, a1, b1m, a2, b2m, b1, b2, gate, out, sms, stream) !=
         cudaSuccess)
@@ -352,6 +360,22 @@ static swl_status run_forward(const Shape& s, const Workspace& ws, const void* x
   swl_status st = run_routing(s, ws, x, W_r, W1, expert_idx, gate, pos_in_expert, b_r, stream,
                               rec, router_noise);
   if (st != SWL_OK) return st;
+  if (s.ntlb) {
+    // No-Token-Left-Behind: both stages' positions (scan stage), the gather of
+    // the kept tokens, then the top-1 FFN with each token's keeping probability
+    if (launch_ntlb_positions(s, ws, expert_idx, pos_in_expert, aux_loss, stream) !=
+        cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (!rec(3)) return SWL_ERR_CUDA;
+    if (launch_ntlb_gather(s, ws, x, expert_idx, gate, pos_in_expert, out, stream) !=
+        cudaSuccess)
+      return SWL_ERR_CUDA;
+    if (!rec(4)) return SWL_ERR_CUDA;
+    st = run_ffn(s, ws, W1, b1, W2, b2, ws.ntlb_gate, out, stream);
+    if (st != SWL_OK) return st;
+    if (!rec(5)) return SWL_ERR_CUDA;
+    return SWL_OK;
+  }
   if (dispatch_fused_ok(s)) {
     // one launch for scan and gather (timed in the scan stage; the gather stage is empty)
     if (launch_dispatch_fused(s, ws, x, expert_idx, pos_in_expert, out, aux_loss, stream) !=
@@ -404,10 +428,10 @@ static swl_status forward_impl(int64_t T, int64_t d, int64_t d_ff, int64_t N, in
                                const float* b_r, void* workspace, size_t workspace_bytes,
                                void* stream_v, void* const* ev, int topk = 1,
                                int normalize = 1, int glu = 0,
-                               const float* router_noise = nullptr) {
+                               const float* router_noise = nullptr, int ntlb = 0) {
   Shape s;
   swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s, topk, normalize, glu,
-                             router_noise != nullptr ? 1 : 0);
+                             router_noise != nullptr ? 1 : 0, ntlb);
   if (st != SWL_OK) return st;
   st = validate_io(s, x, W_r, W1, b1, W2, b2, out, expert_idx, gate, pos, aux, workspace,
                    workspace_bytes, false);
@@ -488,9 +512,14 @@ int64_t switch_layer_capacity(int64_t T, int64_t N, double cf) {
 swl_status switch_layer_workspace_size(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
                                        double cf, int flags, size_t* bytes) {
   if (!bytes) return SWL_ERR_INVALID_ARG;
-  if ((flags & SWL_WS_TOP2) && (flags & SWL_WS_HOST_IO)) return SWL_ERR_INVALID_ARG;
+  if ((flags & ~(SWL_WS_HOST_IO | SWL_WS_TOP2 | SWL_WS_NTLB)) != 0) return SWL_ERR_INVALID_ARG;
+  if ((flags & (SWL_WS_TOP2 | SWL_WS_NTLB)) && (flags & SWL_WS_HOST_IO)) return SWL_ERR_INVALID_ARG;
+  if ((flags & SWL_WS_TOP2) && (flags & SWL_WS_NTLB)) return SWL_ERR_INVALID_ARG;
   Shape s;
-  const swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s, (flags & SWL_WS_TOP2) ? 2 : 1);
+  const bool ntlb = (flags & SWL_WS_NTLB) != 0;
+  const swl_status st = make_shape(T, d, d_ff, N, dtype, cf, &s,
+                                   (flags & (SWL_WS_TOP2 | SWL_WS_NTLB)) ? 2 : 1, ntlb ? 0 : 1,
+                                   0, 0, ntlb ? 1 : 0);
   if (st != SWL_OK) return st;
   *bytes = workspace_layout(s, (flags & SWL_WS_HOST_IO) != 0, 0, nullptr);
   return SWL_OK;
@@ -552,6 +581,18 @@ swl_status switch_layer_forward_variant(int64_t T, int64_t d, int64_t d_ff, int6
                       expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
                       stream, nullptr, topk, normalize, glu,
                       variant != nullptr ? variant->router_noise : nullptr);
+}
+
+swl_status switch_layer_forward_ntlb(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,
+                                     const void* x, const float* W_r, const void* W1,
+                                     const void* b1, const void* W2, const void* b2,
+                                     double capacity_factor, void* out, int32_t* expert_idx,
+                                     float* gate, int32_t* pos_in_expert, float* aux_loss,
+                                     const float* b_r, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  return forward_impl(T, d, d_ff, N, dtype, x, W_r, W1, b1, W2, b2, capacity_factor, out,
+                      expert_idx, gate, pos_in_expert, aux_loss, b_r, workspace, workspace_bytes,
+                      stream, nullptr, 2, 0, 0, nullptr, 1);
 }
 
 swl_status switch_layer_forward_top2(int64_t T, int64_t d, int64_t d_ff, int64_t N, int dtype,

@@ -230,3 +230,20 @@ def test_top2_workspace_and_validation(L):
     assert L.switch_layer_workspace_size(64, 32, 32, 4, swl.SWL_BF16, 1.0,
                                          swl.SWL_WS_TOP2 | swl.SWL_WS_HOST_IO,
                                          ctypes.byref(n)) == 1
+
+
+def test_ntlb_workspace_and_validation(L):
+    """No-Token-Left-Behind workspaces hold one packed row per token (not two),
+    the top-2 router's block arrays and the stage-2 scratch; the flag combines
+    with no other; one expert is refused."""
+    import ctypes
+    n1 = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25)
+    n2 = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25, swl.SWL_WS_TOP2)
+    nn = swl.switch_layer_workspace_size(4096, 768, 3072, 64, swl.SWL_BF16, 1.25, swl.SWL_WS_NTLB)
+    assert n1 < nn < n2
+    n = ctypes.c_size_t(0)
+    for flags in (swl.SWL_WS_NTLB | swl.SWL_WS_TOP2, swl.SWL_WS_NTLB | swl.SWL_WS_HOST_IO, 8):
+        assert L.switch_layer_workspace_size(64, 32, 32, 4, swl.SWL_BF16, 1.0, flags,
+                                             ctypes.byref(n)) == 1, flags
+    assert L.switch_layer_workspace_size(64, 32, 32, 1, swl.SWL_BF16, 1.0, swl.SWL_WS_NTLB,
+                                         ctypes.byref(n)) == 1
