@@ -429,6 +429,147 @@ def run_gpu(args):
     swl_dist.finalize(swl_dist.rank_info())
 
 
+VARIANTS = ("top2", "ntlb", "geglu", "jitter", "backward")
+
+
+def run_variant(args):
+    """One JSON line for a layer variant on one GPU: the top-2 layer, No-Token-
+    Left-Behind, GEGLU experts, router input jitter (forward passes), or the
+    backward pass of the top-1 layer.  Same method as the default line (graph
+    replay, L2 flushed between steps, device events, clocks sampled), with the
+    variant's own algorithmic bytes (forward) or FLOPs (backward)."""
+    import dataclasses
+    import sparse_mixture_experts_argmax_b200 as swl
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--variant runs on one GPU")
+    dev = torch.device("cuda", 0)
+    base = synth.WORKLOADS[args.workload]
+    v = args.variant
+    spec = dataclasses.replace(base, name=base.name + "_geglu", activation="geglu") \
+        if v == "geglu" else base
+    T, d, d_ff, N, cf = spec.T, spec.d, spec.d_ff, spec.N, spec.cf
+    inputs = synth.make_layer_inputs(spec, device=dev,
+                                     redraws=synth.load_gap_redraws(base.name))
+    act = inputs["x"].dtype
+    elem = 2 if act == torch.bfloat16 else 4
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    noise = synth.router_noise(spec, device=dev) if v == "jitter" else None
+    if v == "top2":
+        ws = swl.alloc_workspace(T, d, d_ff, N, act, cf, device=dev, top2=True)
+        fn = lambda st: swl.forward_top2(inputs, cf, True, workspace=ws, stream=st, check=False)
+    elif v == "ntlb":
+        ws = swl.alloc_workspace(T, d, d_ff, N, act, cf, device=dev, ntlb=True)
+        fn = lambda st: swl.forward_ntlb(inputs, cf, workspace=ws, stream=st, check=False)
+    elif v in ("geglu", "jitter"):
+        var = swl.make_variant(1, True, "geglu" if v == "geglu" else "relu", noise)
+        ws = torch.empty(max(256, swl.switch_layer_variant_workspace_size(
+            T, d, d_ff, N, swl.dtype_code(act), cf, var)), dtype=torch.uint8, device=dev)
+        act_name = "geglu" if v == "geglu" else "relu"
+        fn = lambda st: swl.forward_variant(inputs, cf, 1, True, act_name, noise, workspace=ws,
+                                            stream=st, check=False)
+    else:   # backward of the top-1 layer, after one forward
+        ws = swl.alloc_workspace(T, d, d_ff, N, act, cf, device=dev)
+        fwd = swl.forward(inputs, cf, workspace=ws)
+        dout = synth.draw((0, spec.name, "dout"), (T, d), "normal", 1.0, spec.dtype, dev)
+        fn = lambda st: swl.backward(inputs, cf, fwd, ws, dout, daux=1.0, stream=st, check=False)
+
+    launches = 0
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        c0 = swl.switch_layer_launch_count()
+        out = fn(stream)
+        launches = swl.switch_layer_launch_count() - c0
+    torch.cuda.synchronize()
+    if swl.switch_layer_device_status(ws, stream) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            gout = fn(cap)
+    stream.wait_stream(cap)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        graph.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record(stream)
+        graph.replay()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if swl.switch_layer_device_status(ws, stream) != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    peaks = _peaks()
+    C1 = swl.switch_layer_capacity(T, N, cf)
+    if v == "backward":
+        kept = (fwd["pos_in_expert"].long() < C1)
+        K = int(kept.sum())
+        # dW1, dW2 (K d d_ff each), dh and dx through both matrices (K d d_ff each),
+        # router: dW_r and dx (T d N each), 2 flop per multiply-add
+        flops = 2.0 * (4.0 * K * d * d_ff + 2.0 * T * d * N)
+        peak_fp32 = 2.0 * 128 * torch.cuda.get_device_properties(dev).multi_processor_count * \
+            1.965e9 / 1e12
+        roof = {"kernel": "whole backward", "bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
+                "peak": peak_fp32, "unit": "TFLOP/s",
+                "frac": flops / (ms / 1e3) / 1e12 / peak_fp32, "traffic": None,
+                "algorithmic_flops": flops,
+                "peak_source": "fp32 FMA issue: 148 SMs x 128 lanes x 2 flop x 1965 MHz "
+                               "(SIMT kernels)"}
+        routing = {"kept_tokens": K}
+    else:
+        e = gout["expert_idx"].long().reshape(T, -1)
+        pos = gout["pos_in_expert"].long().reshape(T, -1)
+        if v == "top2":
+            Ck = swl.switch_layer_capacity(2 * T, N, cf)
+            keptm = pos < Ck
+        elif v == "ntlb":
+            keptm = torch.stack([pos[:, 0] < C1, (pos[:, 0] >= C1) & (pos[:, 1] >= 0) &
+                                 (pos[:, 1] < C1)], dim=1)
+        else:
+            keptm = pos < C1
+        K = int(keptm.sum())
+        touched = int(torch.unique(e[keptm]).numel())
+        w_per = (3 if v == "geglu" else 2) * d * d_ff + d + (2 if v == "geglu" else 1) * d_ff
+        ffn_bytes = touched * w_per * elem + K * (2 * d * elem + 8)
+        layer_bytes = (T * d * elem + N * d * 4 + T * d * elem + (4 * T * d if noise is not None
+                                                                   else 0) + ffn_bytes)
+        achieved = layer_bytes / (ms / 1e3) / 1e9
+        roof = {"kernel": "whole layer", "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": None, "algorithmic_bytes": layer_bytes,
+                "peak_source": peaks["source"] + " (burst copy)"}
+        routing = {"experts_touched": touched, "kept_assignments": K}
+    res = {
+        "metric": "Switch-layer %s tokens/sec on 1 B200" % (
+            "backward" if v == "backward" else v + " variant fwd"),
+        "value": T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if act == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded; x ~ N(0,1), T5 truncated-normal init s=0.1)",
+        "config": {"workload": spec.name, "variant": v, "T": T, "d": d, "d_ff": d_ff, "N": N,
+                   "capacity_factor": cf,
+                   "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
+        "roofline": roof, "routing": routing, "gpu_launches": int(launches * args.steps),
+        "clocks": clk,
+    }
+    print(json.dumps(res), flush=True)
+
+
 def run_gpu_sharded(args):
     """N > 1 ranks: ONE global batch of N x T tokens, rank g holding the g-th
     contiguous range of T tokens (rank 0 the workload's own seeded tokens, rank
@@ -720,6 +861,9 @@ def main():
     ap.add_argument("--router", default="tensor", choices=["tensor", "ffma"],
                     help="fp32 router logits of bf16 layers: tensor cores on the exact bf16 "
                          "split of W_r (default) or FFMA on the CUDA cores")
+    ap.add_argument("--variant", default=None, choices=VARIANTS,
+                    help="measure a layer variant instead (one GPU): top2, ntlb "
+                         "(No-Token-Left-Behind), geglu, jitter, or backward")
     ap.add_argument("--global-batch", action="store_true",
                     help="use the multi-rank global-batch path (shard steps and the record "
                          "all-gather) also on a single GPU")
@@ -738,6 +882,8 @@ def main():
         args.workload = spec.name
     if args.impl == "reference":
         run_reference(args)
+    elif args.variant:
+        run_variant(args)
     elif int(os.environ.get("WORLD_SIZE", "1")) > 1 or args.global_batch:
         run_gpu_sharded(args)
     else:
