@@ -27,6 +27,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 
 namespace swl {
@@ -292,6 +294,217 @@ grouped_gemm_kernel(const TAin* __restrict__ A, const TBin* __restrict__ B, TC* 
   }
 }
 
+// bf16 form of grouped_gemm_kernel on the tensor cores: mma.sync m16n8k16 with
+// fp32 accumulation, 128 x 128 outputs per CTA, 8 warps of 64 x 32, K in steps
+// of 32 staged by cp.async into two shared-memory buffers, fragments by
+// ldmatrix (transposed where the contraction runs along a tile's rows).  Same
+// groups, grids (with 128-row tiles) and epilogues as the SIMT kernel.
+//   WGRAD: the contraction runs over the group's rows for both operands, so A
+//     is staged [k][m] and B [k][n] and both are read transposed.
+//   DGRAD: A is staged [r][k] (read as is), W[g] [k][n] (read transposed).
+constexpr int kMT = 128, kMK = 32, kMPad = 8;
+constexpr int kMStride = kMT + kMPad;      // [k][128] tiles: row stride in elements
+constexpr int kMStrideK = kMK + kMPad;     // [128][k] tile: row stride in elements
+constexpr int kMStage = kMK * kMStride > kMT * kMStrideK ? kMK * kMStride : kMT * kMStrideK;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+// 16-byte async copy; a false predicate copies nothing and zero-fills
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(pred ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <bool kWgrad>
+__global__ void __launch_bounds__(256)
+grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
+                        __nv_bfloat16* __restrict__ C, int P, int Q, int K,
+                        const int* __restrict__ base, const int* __restrict__ rows, int rows0,
+                        const int* __restrict__ tile_prefix, int groups, int epi,
+                        const __nv_bfloat16* __restrict__ mask, const int* __restrict__ dst_row,
+                        float* __restrict__ acc_out) {
+  __shared__ __align__(128) __nv_bfloat16 sA[2][kMStage];
+  __shared__ __align__(128) __nv_bfloat16 sB[2][kMK * kMStride];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp >> 2, wn = warp & 3;        // 2 x 4 warps of 64 x 32 outputs
+  const int n0 = blockIdx.x * kMT;
+  int g, r0, nr, m0 = 0, kdim;
+  if (kWgrad) {
+    g = blockIdx.z;
+    r0 = base ? base[g] : 0;
+    nr = rows ? rows[g] : rows0;
+    m0 = blockIdx.y * kMT;
+    kdim = nr;
+    if (nr == 0) {      // an expert with no kept rows has a zero gradient
+      for (int i = tid; i < kMT * kMT; i += 256) {
+        const int mm = m0 + i / kMT, nn = n0 + i % kMT;
+        if (mm < P && nn < Q) C[(static_cast<size_t>(g) * P + mm) * Q + nn] = __float2bfloat16(0.f);
+      }
+      return;
+    }
+  } else {
+    const int tile = blockIdx.y;
+    if (tile_prefix) {
+      if (tile >= tile_prefix[groups]) return;
+      int lo = 0, hi = groups;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tile_prefix[mid] <= tile) lo = mid; else hi = mid;
+      }
+      g = lo;
+      const int nt = tile - tile_prefix[g];
+      r0 = base[g] + nt * kMT;
+      nr = min(kMT, rows[g] - nt * kMT);
+    } else {
+      g = 0;
+      r0 = tile * kMT;
+      nr = min(kMT, rows0 - r0);
+      if (nr <= 0) return;
+    }
+    kdim = K;
+  }
+  const __nv_bfloat16* W = kWgrad ? B : B + static_cast<size_t>(g) * K * Q;
+
+  // stage one K step of 32 into buffer s (every thread: 2 chunks of A, 2 of B)
+  auto load = [&](int s, int k0) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = tid + h * 256;
+      if (kWgrad) {
+        const int k = c >> 4, mc = (c & 15) * 8;   // A[r0 + k0 + k][m0 + mc ...]
+        const bool ok = k0 + k < nr && m0 + mc < P;
+        cp_async16(&sA[s][k * kMStride + mc],
+                   ok ? A + static_cast<size_t>(r0 + k0 + k) * P + m0 + mc : A, ok);
+      } else {
+        const int r = c >> 2, kc = (c & 3) * 8;    // A[r0 + r][k0 + kc ...]
+        const bool ok = r < nr && k0 + kc < K;
+        cp_async16(&sA[s][r * kMStrideK + kc],
+                   ok ? A + static_cast<size_t>(r0 + r) * K + k0 + kc : A, ok);
+      }
+      const int k = c >> 4, nc = (c & 15) * 8;
+      const bool okb = k0 + k < kdim && n0 + nc < Q;
+      const __nv_bfloat16* src =
+          kWgrad ? B + static_cast<size_t>(r0 + k0 + k) * Q + n0 + nc
+                 : W + static_cast<size_t>(k0 + k) * Q + n0 + nc;
+      cp_async16(&sB[s][k * kMStride + nc], okb ? src : B, okb);
+    }
+    cp_async_commit();
+  };
+
+  float acc[4][4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
+
+  const int nk = (kdim + kMK - 1) / kMK;
+  load(0, 0);
+  for (int kt = 0; kt < nk; ++kt) {
+    const int s = kt & 1;
+    if (kt + 1 < nk) {
+      load(s ^ 1, (kt + 1) * kMK);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kMK; kk += 16) {
+      uint32_t af[4][4], bf[4][2];
+      const int jm = lane >> 3, rr = lane & 7;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int mb = wm * 64 + i * 16;
+        if (kWgrad) {   // staged [k][m]: matrices (m, k) blocks at rows k, read transposed
+          ldsm_x4_t(af[i], &sA[s][(kk + rr + (jm >> 1) * 8) * kMStride + mb + (jm & 1) * 8]);
+        } else {        // staged [r][k]
+          ldsm_x4(af[i], &sA[s][(mb + (lane & 15)) * kMStrideK + kk + (lane >> 4) * 8]);
+        }
+      }
+#pragma unroll
+      for (int j2 = 0; j2 < 2; ++j2) {   // two n-fragments of 8 per ldmatrix
+        const int nb = wn * 32 + j2 * 16;
+        uint32_t t4[4];
+        ldsm_x4_t(t4, &sB[s][(kk + rr + (jm & 1) * 8) * kMStride + nb + (jm >> 1) * 8]);
+        bf[2 * j2][0] = t4[0];
+        bf[2 * j2][1] = t4[1];
+        bf[2 * j2 + 1][0] = t4[2];
+        bf[2 * j2 + 1][1] = t4[3];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_bf16(acc[i][j], af[i], bf[j][0], bf[j][1]);
+    }
+    __syncthreads();
+  }
+
+  // epilogue: accumulator (i, j, c) -> row wm*64 + i*16 + lane/4 (+8 for c >= 2),
+  // column wn*32 + j*8 + (lane%4)*2 (+1 for odd c)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int rl = wm * 64 + i * 16 + (lane >> 2) + hh * 8;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int nn = n0 + wn * 32 + j * 8 + (lane & 3) * 2;
+        if (nn >= Q) continue;
+        const float v0 = acc[i][j][2 * hh], v1 = acc[i][j][2 * hh + 1];
+        if (kWgrad) {
+          const int mm = m0 + rl;
+          if (mm < P)
+            *reinterpret_cast<__nv_bfloat162*>(C + (static_cast<size_t>(g) * P + mm) * Q + nn) =
+                __floats2bfloat162_rn(v0, v1);
+        } else {
+          if (rl >= nr) continue;
+          const int r = r0 + rl;
+          const size_t o = static_cast<size_t>(r) * Q + nn;
+          if (epi == 0) {
+            *reinterpret_cast<__nv_bfloat162*>(C + o) = __floats2bfloat162_rn(v0, v1);
+          } else if (epi == 1) {
+            const __nv_bfloat162 mk = *reinterpret_cast<const __nv_bfloat162*>(mask + o);
+            *reinterpret_cast<__nv_bfloat162*>(C + o) = __floats2bfloat162_rn(
+                __bfloat162float(mk.x) > 0.f ? v0 : 0.f, __bfloat162float(mk.y) > 0.f ? v1 : 0.f);
+          } else {
+            const int t = dst_row ? dst_row[r] : r;
+            float* d = acc_out + static_cast<size_t>(t) * Q + nn;
+            d[0] += v0;
+            d[1] += v1;
+          }
+        }
+      }
+    }
+  }
+}
+
 // db[g][m] = sum over the group's rows r of A[r][m]; one thread per (g, m).
 template <typename TA, typename TC>
 __global__ void __launch_bounds__(256)
@@ -306,14 +519,14 @@ bias_grad_kernel(const TA* __restrict__ A, int P, const int* __restrict__ base,
   db[static_cast<size_t>(g) * P + m] = cvt<TC>(s);
 }
 
-// Row tiles of 64 packed rows per expert for the DGRAD grid.
-__global__ void bwd_tile_prefix_kernel(const int* __restrict__ rows, int N,
+// Row tiles of `tile` packed rows per expert for the DGRAD grid.
+__global__ void bwd_tile_prefix_kernel(const int* __restrict__ rows, int N, int tile,
                                        int* __restrict__ prefix) {
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     int acc = 0;
     for (int e = 0; e < N; ++e) {
       prefix[e] = acc;
-      acc += (rows[e] + kGT - 1) / kGT;
+      acc += (rows[e] + tile - 1) / tile;
     }
     prefix[N] = acc;
   }
@@ -358,7 +571,38 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
   ++launches;
   const dim3 blk(256);
   auto tiles = [](int v) { return static_cast<unsigned>((v + kGT - 1) / kGT); };
-  // dW2[e] = du^T h, db2[e] = sum du
+  if constexpr (std::is_same<TA, __nv_bfloat16>::value) {
+    // bf16 layers: the four expert GEMMs on the tensor cores (128 x 128 tiles)
+    auto mt = [](int v) { return static_cast<unsigned>((v + kMT - 1) / kMT); };
+    const __nv_bfloat16* du = static_cast<const __nv_bfloat16*>(bw.du);
+    const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(fw.hbuf);
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(fw.xbuf);
+    __nv_bfloat16* da = static_cast<__nv_bfloat16*>(bw.da);
+    // dW2[e] = du^T h, db2[e] = sum du
+    grouped_gemm_mma_kernel<true><<<dim3(mt(d_ff), mt(d), N), blk, 0, stream>>>(
+        du, hb, static_cast<__nv_bfloat16*>(a.dW2), d, d_ff, 0, fw.exp_base, fw.exp_rows, 0,
+        nullptr, N, 0, nullptr, nullptr, nullptr);
+    bias_grad_kernel<TA, TA><<<dim3((d + 255) / 256, N), blk, 0, stream>>>(
+        static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, static_cast<TA*>(a.db2));
+    // da = (du W2[e]) * [h > 0]
+    bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, kMT, bw.tile_prefix);
+    const unsigned row_tiles = static_cast<unsigned>((T + kMT - 1) / kMT + N);
+    grouped_gemm_mma_kernel<false><<<dim3(mt(d_ff), row_tiles, 1), blk, 0, stream>>>(
+        du, static_cast<const __nv_bfloat16*>(a.W2), da, 0, d_ff, d, fw.exp_base, fw.exp_rows, 0,
+        bw.tile_prefix, N, 1, hb, nullptr, nullptr);
+    // dW1[e] = da^T x, db1[e] = sum da
+    grouped_gemm_mma_kernel<true><<<dim3(mt(d), mt(d_ff), N), blk, 0, stream>>>(
+        da, xb, static_cast<__nv_bfloat16*>(a.dW1), d_ff, d, 0, fw.exp_base, fw.exp_rows, 0,
+        nullptr, N, 0, nullptr, nullptr, nullptr);
+    bias_grad_kernel<TA, TA><<<dim3((d_ff + 255) / 256, N), blk, 0, stream>>>(
+        static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N,
+        static_cast<TA*>(a.db1));
+    // dx (kept tokens) += da W1[e], rows to tokens
+    grouped_gemm_mma_kernel<false><<<dim3(mt(d), row_tiles, 1), blk, 0, stream>>>(
+        da, static_cast<const __nv_bfloat16*>(a.W1), nullptr, 0, d, d_ff, fw.exp_base,
+        fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
+    launches += 7;
+  } else {
   grouped_gemm_kernel<TA, TA, TA, true><<<dim3(tiles(d_ff), tiles(d), N), blk, 0, stream>>>(
       static_cast<const TA*>(bw.du), static_cast<const TA*>(fw.hbuf), static_cast<TA*>(a.dW2), d,
       d_ff, 0, fw.exp_base, fw.exp_rows, 0, nullptr, N, 0, nullptr, nullptr, nullptr);
@@ -366,7 +610,7 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
       static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, static_cast<TA*>(a.db2));
   launches += 2;
   // da = (du W2[e]) * [h > 0]   (W2[e] is [d, d_ff]: K = d, Q = d_ff)
-  bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, bw.tile_prefix);
+  bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, kGT, bw.tile_prefix);
   const unsigned max_row_tiles = static_cast<unsigned>((T + kGT - 1) / kGT + N);
   grouped_gemm_kernel<TA, TA, TA, false><<<dim3(tiles(d_ff), max_row_tiles, 1), blk, 0, stream>>>(
       static_cast<const TA*>(bw.du), static_cast<const TA*>(a.W2), static_cast<TA*>(bw.da), 0,
@@ -386,6 +630,7 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
       static_cast<const TA*>(bw.da), static_cast<const TA*>(a.W1), static_cast<TA*>(nullptr), 0, d,
       d_ff, fw.exp_base, fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
   ++launches;
+  }
   // router: dW_r = dz^T x (one group of T rows), db_r = sum dz, dx += dz W_r
   grouped_gemm_kernel<float, TA, float, true><<<dim3(tiles(d), tiles(N), 1), blk, 0, stream>>>(
       bw.dz, x, a.dW_r, N, d, 0, nullptr, nullptr, T, nullptr, 1, 0, nullptr, nullptr, nullptr);
