@@ -23,7 +23,7 @@
 //                       groups (one group per expert), two forms:
 //                       WGRAD  C[g] = sum over the group's rows of A_r^T B_r
 //                       DGRAD  C_r  = A_r W[g] (+ an epilogue per use)
-//   bias_grad_kernel    db[g] = sum over the group's rows of A_r
+//   colsum_*_kernel     db[g] = sum over the group's rows of A_r (split, then summed)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -156,7 +156,9 @@ bwd_router_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
 // in steps of 16.
 //   WGRAD (kWgrad = true): group g owns rows [base[g], base[g] + rows[g]) of A
 //     [*, P] and B [*, Q]; C[g] [P, Q] = sum over those rows r of A[r]^T B[r]
-//     (C written, not accumulated).  Grid: (Q/64, P/64, groups).
+//     (C written, not accumulated).  Grid: (Q/64, P/64, groups).  With base =
+//     nullptr and groups > 1, group g is the chunk [g K, (g + 1) K) of rows0
+//     rows (partial products of one long sum, added by colsum_finish_kernel).
 //   DGRAD: C[r] [Q] = A[r] [K] x W[g] [K, Q] for the group's rows; the epilogue
 //     by `epi`: 0 store; 1 multiply by [mask[r] > 0] and store (da from dh);
 //     2 add into the fp32 accumulator row dst_row[r] (dx).  Grid: (Q/64,
@@ -179,8 +181,13 @@ grouped_gemm_kernel(const TAin* __restrict__ A, const TBin* __restrict__ B, TC* 
   int m0, n0 = blockIdx.x * kGT;
   if (kWgrad) {
     g = blockIdx.z;
-    r0 = base ? base[g] : 0;
-    nr = rows ? rows[g] : rows0;
+    if (base == nullptr && groups > 1) {   // one group of rows0 rows cut into chunks of K
+      r0 = g * K;
+      nr = max(0, min(K, rows0 - r0));
+    } else {
+      r0 = base ? base[g] : 0;
+      nr = rows ? rows[g] : rows0;
+    }
     m0 = blockIdx.y * kGT;
     if (nr == 0) {      // an expert with no kept rows has a zero gradient
       for (int i = threadIdx.x; i < kGT * kGT; i += 256) {
@@ -505,18 +512,49 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
   }
 }
 
-// db[g][m] = sum over the group's rows r of A[r][m]; one thread per (g, m).
-template <typename TA, typename TC>
+// Column sums per group, in two passes so that long groups spread over many
+// CTAs: partial[s][g][m] = sum of A[r][m] over rows s*R .. s*R + R - 1 of group
+// g (R = kColRows), one CTA per 32 columns, group and split, its 8 warps taking
+// every 8th row and their sums added in warp order; then colsum_finish_kernel
+// adds the splits in order (deterministic).
+constexpr int kColRows = 256;
+constexpr int kRouterChunk = 4096;   // rows per partial product of the router's dW_r
+
+template <typename TA>
 __global__ void __launch_bounds__(256)
-bias_grad_kernel(const TA* __restrict__ A, int P, const int* __restrict__ base,
-                 const int* __restrict__ rows, int rows0, int groups, TC* __restrict__ db) {
-  const int g = blockIdx.y;
-  const int m = blockIdx.x * 256 + threadIdx.x;
-  if (g >= groups || m >= P) return;
+colsum_partial_kernel(const TA* __restrict__ A, int P, const int* __restrict__ base,
+                      const int* __restrict__ rows, int rows0, int groups,
+                      float* __restrict__ partial) {
+  __shared__ float red[8][33];
+  const int g = blockIdx.y, sp = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int m = blockIdx.x * 32 + lane;
   const int r0 = base ? base[g] : 0, nr = rows ? rows[g] : rows0;
-  float s = 0.f;
-  for (int r = 0; r < nr; ++r) s += ld(A + static_cast<size_t>(r0 + r) * P + m);
-  db[static_cast<size_t>(g) * P + m] = cvt<TC>(s);
+  const int lo = sp * kColRows, hi = min(nr, lo + kColRows);
+  float sum = 0.f;
+  if (m < P)
+    for (int r = lo + warp; r < hi; r += 8) sum += ld(A + static_cast<size_t>(r0 + r) * P + m);
+  red[warp][lane] = sum;
+  __syncthreads();
+  if (warp == 0 && m < P) {
+    float t = red[0][lane];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) t += red[w][lane];
+    partial[(static_cast<size_t>(sp) * groups + g) * P + m] = t;
+  }
+}
+
+// out[i] = sum over s < S of partial[s][i], in order; n = groups * P (or the
+// [P, Q] products of a chunked WGRAD).
+template <typename TC>
+__global__ void __launch_bounds__(256)
+colsum_finish_kernel(const float* __restrict__ partial, int S, size_t n, TC* __restrict__ out) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float t = 0.f;
+    for (int sp = 0; sp < S; ++sp) t += partial[static_cast<size_t>(sp) * n + i];
+    out[i] = cvt<TC>(t);
+  }
 }
 
 // Row tiles of `tile` packed rows per expert for the DGRAD grid.
@@ -571,6 +609,21 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
   ++launches;
   const dim3 blk(256);
   auto tiles = [](int v) { return static_cast<unsigned>((v + kGT - 1) / kGT); };
+  // db[g][m] = sum over the group's rows of A[r][m]: split partials, then their sum
+  auto colsum = [&](auto* Ain, int P, const int* gbase, const int* grows, int rows0, int groups,
+                    int max_rows, auto* out) {
+    using TIn = typename std::remove_cv<typename std::remove_pointer<decltype(Ain)>::type>::type;
+    using TOut = typename std::remove_pointer<decltype(out)>::type;
+    const int S = max(1, (max_rows + kColRows - 1) / kColRows);
+    colsum_partial_kernel<TIn><<<dim3((P + 31) / 32, groups, S), blk, 0, stream>>>(
+        Ain, P, gbase, grows, rows0, groups, bw.part);
+    const size_t n = static_cast<size_t>(groups) * P;
+    size_t nb = (n + 255) / 256;
+    if (nb > 8 * 148) nb = 8 * 148;
+    colsum_finish_kernel<TOut><<<static_cast<unsigned>(nb), blk, 0, stream>>>(bw.part, S, n, out);
+    launches += 2;
+  };
+  const int C_rows = static_cast<int>(s.C_eff);
   if constexpr (std::is_same<TA, __nv_bfloat16>::value) {
     // bf16 layers: the four expert GEMMs on the tensor cores (128 x 128 tiles)
     auto mt = [](int v) { return static_cast<unsigned>((v + kMT - 1) / kMT); };
@@ -582,8 +635,8 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
     grouped_gemm_mma_kernel<true><<<dim3(mt(d_ff), mt(d), N), blk, 0, stream>>>(
         du, hb, static_cast<__nv_bfloat16*>(a.dW2), d, d_ff, 0, fw.exp_base, fw.exp_rows, 0,
         nullptr, N, 0, nullptr, nullptr, nullptr);
-    bias_grad_kernel<TA, TA><<<dim3((d + 255) / 256, N), blk, 0, stream>>>(
-        static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, static_cast<TA*>(a.db2));
+    colsum(static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, C_rows,
+           static_cast<TA*>(a.db2));
     // da = (du W2[e]) * [h > 0]
     bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, kMT, bw.tile_prefix);
     const unsigned row_tiles = static_cast<unsigned>((T + kMT - 1) / kMT + N);
@@ -594,21 +647,20 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
     grouped_gemm_mma_kernel<true><<<dim3(mt(d), mt(d_ff), N), blk, 0, stream>>>(
         da, xb, static_cast<__nv_bfloat16*>(a.dW1), d_ff, d, 0, fw.exp_base, fw.exp_rows, 0,
         nullptr, N, 0, nullptr, nullptr, nullptr);
-    bias_grad_kernel<TA, TA><<<dim3((d_ff + 255) / 256, N), blk, 0, stream>>>(
-        static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N,
-        static_cast<TA*>(a.db1));
+    colsum(static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N, C_rows,
+           static_cast<TA*>(a.db1));
     // dx (kept tokens) += da W1[e], rows to tokens
     grouped_gemm_mma_kernel<false><<<dim3(mt(d), row_tiles, 1), blk, 0, stream>>>(
         da, static_cast<const __nv_bfloat16*>(a.W1), nullptr, 0, d, d_ff, fw.exp_base,
         fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
-    launches += 7;
+    launches += 5;
   } else {
   grouped_gemm_kernel<TA, TA, TA, true><<<dim3(tiles(d_ff), tiles(d), N), blk, 0, stream>>>(
       static_cast<const TA*>(bw.du), static_cast<const TA*>(fw.hbuf), static_cast<TA*>(a.dW2), d,
       d_ff, 0, fw.exp_base, fw.exp_rows, 0, nullptr, N, 0, nullptr, nullptr, nullptr);
-  bias_grad_kernel<TA, TA><<<dim3((d + 255) / 256, N), blk, 0, stream>>>(
-      static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, static_cast<TA*>(a.db2));
-  launches += 2;
+  colsum(static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, C_rows,
+         static_cast<TA*>(a.db2));
+  ++launches;
   // da = (du W2[e]) * [h > 0]   (W2[e] is [d, d_ff]: K = d, Q = d_ff)
   bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, kGT, bw.tile_prefix);
   const unsigned max_row_tiles = static_cast<unsigned>((T + kGT - 1) / kGT + N);
@@ -621,25 +673,30 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
   grouped_gemm_kernel<TA, TA, TA, true><<<dim3(tiles(d), tiles(d_ff), N), blk, 0, stream>>>(
       static_cast<const TA*>(bw.da), static_cast<const TA*>(fw.xbuf), static_cast<TA*>(a.dW1),
       d_ff, d, 0, fw.exp_base, fw.exp_rows, 0, nullptr, N, 0, nullptr, nullptr, nullptr);
-  bias_grad_kernel<TA, TA><<<dim3((d_ff + 255) / 256, N), blk, 0, stream>>>(
-      static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N,
-      static_cast<TA*>(a.db1));
-  launches += 2;
+  colsum(static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N, C_rows,
+         static_cast<TA*>(a.db1));
+  ++launches;
   // dx (kept tokens) += da W1[e]   (W1[e] is [d_ff, d]: K = d_ff, Q = d), rows to tokens
   grouped_gemm_kernel<TA, TA, TA, false><<<dim3(tiles(d), max_row_tiles, 1), blk, 0, stream>>>(
       static_cast<const TA*>(bw.da), static_cast<const TA*>(a.W1), static_cast<TA*>(nullptr), 0, d,
       d_ff, fw.exp_base, fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
   ++launches;
   }
-  // router: dW_r = dz^T x (one group of T rows), db_r = sum dz, dx += dz W_r
-  grouped_gemm_kernel<float, TA, float, true><<<dim3(tiles(d), tiles(N), 1), blk, 0, stream>>>(
-      bw.dz, x, a.dW_r, N, d, 0, nullptr, nullptr, T, nullptr, 1, 0, nullptr, nullptr, nullptr);
-  ++launches;
-  if (a.db_r) {
-    bias_grad_kernel<float, float><<<dim3((N + 255) / 256, 1), blk, 0, stream>>>(
-        bw.dz, N, nullptr, nullptr, T, 1, a.db_r);
-    ++launches;
+  // router: dW_r = dz^T x over T rows in chunks of kRouterChunk (partial
+  // products, then their sum in chunk order), db_r = sum dz, dx += dz W_r
+  {
+    const int S = (T + kRouterChunk - 1) / kRouterChunk;
+    grouped_gemm_kernel<float, TA, float, true><<<dim3(tiles(d), tiles(N), S), blk, 0, stream>>>(
+        bw.dz, x, bw.part, N, d, kRouterChunk, nullptr, nullptr, T, nullptr, S, 0, nullptr,
+        nullptr, nullptr);
+    const size_t n = static_cast<size_t>(N) * d;
+    size_t nb = (n + 255) / 256;
+    if (nb > 8 * 148) nb = 8 * 148;
+    colsum_finish_kernel<float><<<static_cast<unsigned>(nb), blk, 0, stream>>>(bw.part, S, n,
+                                                                              a.dW_r);
+    launches += 2;
   }
+  if (a.db_r) colsum(static_cast<const float*>(bw.dz), N, nullptr, nullptr, T, 1, T, a.db_r);
   grouped_gemm_kernel<float, float, float, false><<<dim3(tiles(d), tiles(T), 1), blk, 0, stream>>>(
       bw.dz, a.W_r, static_cast<float*>(nullptr), 0, d, N, nullptr, nullptr, T, nullptr, 1, 2,
       nullptr, nullptr, bw.dx_acc);
@@ -672,6 +729,16 @@ size_t backward_workspace_layout(const Shape& s, uintptr_t base, BwdWorkspace* w
   b.du = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d) * elem));
   b.da = reinterpret_cast<void*>(take(T * static_cast<size_t>(s.d_ff) * elem));
   b.dx_acc = reinterpret_cast<float*>(take(T * static_cast<size_t>(s.d) * 4));
+  // split partials: the column sums (db1, db2, db_r) and the router's dW_r chunks
+  const size_t c_eff = static_cast<size_t>(s.C_eff > 0 ? s.C_eff : 1);
+  const size_t s_exp = (c_eff + kColRows - 1) / kColRows;
+  const size_t s_rt = (T + kColRows - 1) / kColRows;
+  const size_t s_ch = (T + kRouterChunk - 1) / kRouterChunk;
+  const size_t dmax = static_cast<size_t>(s.d > s.d_ff ? s.d : s.d_ff);
+  size_t part = s_exp * N * dmax;
+  if (s_rt * N > part) part = s_rt * N;
+  if (s_ch * N * static_cast<size_t>(s.d) > part) part = s_ch * N * static_cast<size_t>(s.d);
+  b.part = reinterpret_cast<float*>(take(part * 4));
   if (w) *w = b;
   return off;
 }

@@ -244,6 +244,7 @@ struct BwdWorkspace {
   void* du;           // [T, d] packed rows g * dout (act dtype)
   void* da;           // [T, d_ff] packed rows of the gradient of the pre-activations
   float* dx_acc;      // [T, d] fp32 accumulator of dx
+  float* part;        // split partials of the column sums and of the router's dW_r
 };
 struct BwdArgs {
   const void* x;          // [T, d]
