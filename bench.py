@@ -522,14 +522,17 @@ def run_variant(args):
         # dW1, dW2 (K d d_ff each), dh and dx through both matrices (K d d_ff each),
         # router: dW_r and dx (T d N each), 2 flop per multiply-add
         flops = 2.0 * (4.0 * K * d * d_ff + 2.0 * T * d * N)
-        peak_fp32 = 2.0 * 128 * torch.cuda.get_device_properties(dev).multi_processor_count * \
-            1.965e9 / 1e12
-        roof = {"kernel": "whole backward", "bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
-                "peak": peak_fp32, "unit": "TFLOP/s",
-                "frac": flops / (ms / 1e3) / 1e12 / peak_fp32, "traffic": None,
-                "algorithmic_flops": flops,
-                "peak_source": "fp32 FMA issue: 148 SMs x 128 lanes x 2 flop x 1965 MHz "
-                               "(SIMT kernels)"}
+        if act == torch.bfloat16:
+            # the expert GEMMs run on the tensor cores (bf16 operands, fp32 accumulation)
+            peak, bound = peaks["bf16_tflops"], "tensor"
+            src = peaks["source"] + " bf16 (burst); the router's fp32 part runs on the CUDA cores"
+        else:
+            peak = 2.0 * 128 * torch.cuda.get_device_properties(dev).multi_processor_count * \
+                1.965e9 / 1e12
+            bound, src = "alu", "fp32 FMA issue: 148 SMs x 128 lanes x 2 flop x 1965 MHz"
+        roof = {"kernel": "whole backward", "bound": bound, "achieved": flops / (ms / 1e3) / 1e12,
+                "peak": peak, "unit": "TFLOP/s", "frac": flops / (ms / 1e3) / 1e12 / peak,
+                "traffic": None, "algorithmic_flops": flops, "peak_source": src}
         routing = {"kept_tokens": K}
     else:
         e = gout["expert_idx"].long().reshape(T, -1)

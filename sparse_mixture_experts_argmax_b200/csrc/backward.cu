@@ -518,7 +518,17 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
 // every 8th row and their sums added in warp order; then colsum_finish_kernel
 // adds the splits in order (deterministic).
 constexpr int kColRows = 256;
-constexpr int kRouterChunk = 4096;   // rows per partial product of the router's dW_r
+// Rows per partial product of the router's dW_r = dz^T x: enough chunks for ~2048
+// CTAs of 64 x 64 outputs, chunks of at least kColRows rows (a multiple of 16).
+inline int router_chunk_rows(int64_t T, int64_t N, int64_t d) {
+  const int64_t tiles = ((d + 63) / 64) * ((N + 63) / 64);
+  int64_t S = (2048 + tiles - 1) / tiles;
+  const int64_t smax = (T + kColRows - 1) / kColRows;
+  if (S > smax) S = smax;
+  if (S < 1) S = 1;
+  const int64_t chunk = (T + S - 1) / S;
+  return static_cast<int>(chunk < 16 ? 16 : (chunk + 15) / 16 * 16);
+}
 
 template <typename TA>
 __global__ void __launch_bounds__(256)
@@ -682,13 +692,14 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
       d_ff, fw.exp_base, fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
   ++launches;
   }
-  // router: dW_r = dz^T x over T rows in chunks of kRouterChunk (partial
+  // router: dW_r = dz^T x over T rows in chunks (router_chunk_rows; partial
   // products, then their sum in chunk order), db_r = sum dz, dx += dz W_r
   {
-    const int S = (T + kRouterChunk - 1) / kRouterChunk;
+    const int chunk = router_chunk_rows(T, N, d);
+    const int S = (T + chunk - 1) / chunk;
     grouped_gemm_kernel<float, TA, float, true><<<dim3(tiles(d), tiles(N), S), blk, 0, stream>>>(
-        bw.dz, x, bw.part, N, d, kRouterChunk, nullptr, nullptr, T, nullptr, S, 0, nullptr,
-        nullptr, nullptr);
+        bw.dz, x, bw.part, N, d, chunk, nullptr, nullptr, T, nullptr, S, 0, nullptr, nullptr,
+        nullptr);
     const size_t n = static_cast<size_t>(N) * d;
     size_t nb = (n + 255) / 256;
     if (nb > 8 * 148) nb = 8 * 148;
@@ -733,7 +744,8 @@ size_t backward_workspace_layout(const Shape& s, uintptr_t base, BwdWorkspace* w
   const size_t c_eff = static_cast<size_t>(s.C_eff > 0 ? s.C_eff : 1);
   const size_t s_exp = (c_eff + kColRows - 1) / kColRows;
   const size_t s_rt = (T + kColRows - 1) / kColRows;
-  const size_t s_ch = (T + kRouterChunk - 1) / kRouterChunk;
+  const int ch = router_chunk_rows(s.T, s.N, s.d);
+  const size_t s_ch = (T + ch - 1) / ch;
   const size_t dmax = static_cast<size_t>(s.d > s.d_ff ? s.d : s.d_ff);
   size_t part = s_exp * N * dmax;
   if (s_rt * N > part) part = s_rt * N;
