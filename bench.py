@@ -44,6 +44,7 @@ from sparse_mixture_experts_argmax_b200 import dist as swl_dist  # noqa: E402
 DEFAULT_WORKLOAD = "many_T65536_d1024_N2048"
 METRIC = "Switch-layer fwd tokens/sec on 1 B200; expert-GEMM % of bf16 tensor peak"
 L2_FLUSH_BYTES = 256 << 20
+E2E_STREAMS = 3          # end-to-end steps in flight (each on its own stream and workspace)
 
 
 def _peaks():
@@ -278,18 +279,21 @@ def run_gpu(args):
     del graph, graph_timed
 
     # ---- end to end through the host-I/O entry point (pinned host x and outputs).
-    # Two streams, each with its own workspace, take alternate steps, so one
-    # step's copies overlap the other's kernels (host-to-device and
-    # device-to-host run on separate copy engines).  Every step copies its x in
-    # and its outputs back inside the timed region, into host buffers of its own
-    # (up to 32 sets, reused in order), and every step's outputs are compared
+    # E2E_STREAMS streams, each with its own workspace, take the steps in turn:
+    # a step's copy in, forward and copy out are serial on its stream, so with
+    # three steps in flight the host-to-device engine, the SMs and the
+    # device-to-host engine each work on a different step.  Every step copies its
+    # x in and its outputs back inside the timed region, into host buffers of its
+    # own (up to 33 sets, reused in order), and every step's outputs are compared
     # with the device-resident run afterwards.  The expert weights (larger than
     # L2) stream from HBM in every step, so no L2 flush is interposed.
-    e2e_streams = [stream, torch.cuda.Stream(dev)]
+    NS = E2E_STREAMS
+    e2e_streams = [stream] + [torch.cuda.Stream(dev) for _ in range(NS - 1)]
     work_h = [swl.alloc_workspace(T, d, d_ff, N, act, cf, host_io=True, device=dev)
-              for _ in range(2)]
-    xh = [inputs["x"].cpu().pin_memory() for _ in range(2)]
-    n_sets = min(32, args.steps + args.steps % 2)     # even: a set stays on one stream
+              for _ in range(NS)]
+    xh = [inputs["x"].cpu().pin_memory() for _ in range(NS)]
+    # a multiple of NS: each output set stays on one stream
+    n_sets = min(NS * 11, (args.steps + NS - 1) // NS * NS)
 
     def out_set():
         return [torch.empty((T, d), dtype=act).pin_memory(),
@@ -298,37 +302,39 @@ def run_gpu(args):
                 torch.empty(T, dtype=torch.int32).pin_memory(),
                 torch.empty(1, dtype=torch.float32).pin_memory()]
 
-    oh = [out_set() for _ in range(max(2, n_sets))]
+    oh = [out_set() for _ in range(max(NS, n_sets))]
 
     def step_e2e(k):
-        j = k % 2
+        j = k % NS
         swl.switch_layer_forward_host_io(xh[j], inputs["W_r"], inputs["W1"], inputs["b1"],
                                          inputs["W2"], inputs["b2"], cf, *oh[k % len(oh)],
                                          b_r=inputs["b_r"], workspace=work_h[j],
                                          stream=e2e_streams[j])
 
-    for k in range(max(2, args.warmup)):
+    for k in range(max(NS, args.warmup)):
         step_e2e(k)
     torch.cuda.synchronize()
     for o in oh:
         o[0].fill_(0)
         o[1].fill_(-1)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_side = torch.cuda.Event()
     _barrier(ws_n)
     torch.cuda.synchronize()
     e_start.record(e2e_streams[0])
-    e2e_streams[1].wait_event(e_start)
+    for st in e2e_streams[1:]:
+        st.wait_event(e_start)
     for k in range(args.steps):
         step_e2e(k)
-    e_side.record(e2e_streams[1])
-    e2e_streams[0].wait_event(e_side)
+    for st in e2e_streams[1:]:
+        ev_side = torch.cuda.Event()
+        ev_side.record(st)
+        e2e_streams[0].wait_event(ev_side)
     e_end.record(e2e_streams[0])
     e_end.synchronize()             # every step's result is on the host
     _barrier(ws_n)
     e2e_total = _max_over_ranks(ws_n, float(e_start.elapsed_time(e_end)))
     e2e_value = ws_n * T * args.steps / (e2e_total / 1e3)
-    for j in range(2):
+    for j in range(NS):
         if swl.switch_layer_device_status(work_h[j], e2e_streams[j]) != 0:
             raise RuntimeError("device status not OK after the end-to-end steps (stream %d)" % j)
     ref_host = [outs[k].cpu() for k in ("out", "expert_idx", "gate", "pos_in_expert",
@@ -418,7 +424,7 @@ def run_gpu(args):
                 "d2h_bytes_per_step": d2h,
                 "note": "switch_layer_forward_host_io per step (pinned host x in, out / "
                         "expert_idx / gate / pos_in_expert / aux_loss back), alternate steps on "
-                        "two streams so copies overlap the other step's kernels"},
+                        "three streams so copies overlap the other steps' kernels"},
         "gpu_launches": int(launches),
         "clocks": clk,
     }
