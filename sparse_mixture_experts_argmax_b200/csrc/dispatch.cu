@@ -198,6 +198,7 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     for (int w = 0; w < kScanWarps; ++w) a += s_aux[w];
     tile_prefix[N] = s_tot_tiles;
     hdr->next_tile = 0u;
+    hdr->gather_prefetch = 2 * s_tot_rows >= T ? 1 : 0;
     // aux = N * sum_i (count_i / T) * (psum_i / T)
     *aux_loss = (float)((double)N * a / ((double)T * (double)T));
     hdr->done = 0u;   // ready for the next call
@@ -282,9 +283,12 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, const int* __restrict__ ex
   const int nv = row_bytes / VEC;
   const V* src = reinterpret_cast<const V*>(x + (size_t)t * row_bytes);
   V reg[kGatherMaxVecPerLane];
-  // prefetch: the row is requested before its destination is known (x is still
-  // in L2 after the router); otherwise only kept tokens' rows are read
-  const bool in_regs = prefetch && nv <= 32 * kGatherMaxVecPerLane;
+  // prefetch: the row is requested before its destination is known (1: x is
+  // still in L2 after the router; 2: when the scan found at least half of the
+  // tokens kept, so the few dropped rows read for nothing cost less than the
+  // round trip saved); otherwise only kept tokens' rows are read
+  const bool in_regs = (prefetch == 1 || (prefetch == 2 && hdr->gather_prefetch != 0)) &&
+                       nv <= 32 * kGatherMaxVecPerLane;
   if (in_regs) {
 #pragma unroll
     for (int j = 0; j < kGatherMaxVecPerLane; ++j)
@@ -1022,8 +1026,8 @@ cudaError_t launch_dispatch_gather(const Shape& s, const Workspace& ws, const vo
       static_cast<const int*>(ws.blk_off), static_cast<const int*>(ws.exp_base),
       static_cast<const int*>(s.sharded ? ws.exp_off : nullptr), ws.slot_token,
       static_cast<uint8_t*>(ws.xbuf), static_cast<uint8_t*>(out), (int)s.T, (int)s.N,
-      (int)s.C_cmp, row_bytes, s.tpb, s.T * (int64_t)row_bytes <= (int64_t{48} << 20) ? 1 : 0,
-      s.topk, ws.hdr);
+      (int)s.C_cmp, row_bytes, s.tpb,
+      s.T * (int64_t)row_bytes <= (int64_t{48} << 20) ? 1 : (s.sharded ? 0 : 2), s.topk, ws.hdr);
   count_launch();
   return e;
 }

@@ -25,7 +25,9 @@ struct WsHeader {
   int err;                  // DeviceError of the last call
   unsigned int done;        // arrival counter of the dispatch-scan kernel (self-resetting)
   unsigned int next_tile;   // work counter of the expert FFN kernel (zeroed by the scan)
-  int pad[61];
+  int gather_prefetch;      // set by the scan: at least half of the tokens are kept, so
+                            // the gather reads every row before its destination is known
+  int pad[60];
 };
 
 // Device pointers carved out of the caller's workspace.
