@@ -53,7 +53,8 @@ struct Workspace {
   int* split_grp;       // GEMM2 split: [kSplitMaxGroups][4] (expert, m-tile, token tile,
                         // 0) of each group, expert -1 past the last group
   void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
-  float* xj;            // jittered router input x * noise [T, d] fp32 (jitter only)
+  float* xj;            // jittered router input x * noise [T, d] fp32 (jitter on the FFMA router)
+  void* x3;             // jittered router input as three bf16 pieces [3T, d] (xsplit)
   void* xbuf;           // [A, d] packed expert inputs (act dtype), A = T * topk
   void* hbuf;           // [A, d_ff] packed hidden activations (act dtype)
   void* ybuf;           // top-2: [A, d] gated expert output per assignment (act dtype)
@@ -82,7 +83,9 @@ struct Shape {
   int ffn_split;  // GEMM2 split over K of experts with full token tiles (1: none)
   int topk;       // experts per token: 1 (Switch) or 2 (the top-2 variant)
   int glu;        // 1: GEGLU experts (W1 [N, 2 d_ff, d]: gate rows, then value rows)
-  int jitter;     // 1: the router sees x * noise (a jittered fp32 copy of x, FFMA router)
+  int jitter;     // 1: the router sees x * noise (a jittered fp32 copy of x)
+  int xsplit;     // jitter on the tensor-core logits (wide bf16 layers): the fp32 router
+                  // input is split exactly into three bf16 pieces like W_r
   int normalize;  // top-2: gates divided by their sum
   int ntlb;       // 1: No-Token-Left-Behind (top-2 router, one slot per token, capacity of
                   // top-1; tokens stage 1 drops go to their second choice's free slots)

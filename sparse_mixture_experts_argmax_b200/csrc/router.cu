@@ -1320,13 +1320,36 @@ router_jitter_kernel(const TX* __restrict__ x, const float* __restrict__ noise,
     xj[i] = static_cast<float>(x[i]) * noise[i];
 }
 
+// The jittered input for the tensor-core logits: v = x * noise in fp32, split
+// exactly into three bf16 numbers v = hi + mid + lo (each residual is exact in
+// fp32, and 3 x 8 significand bits cover fp32's 24), stored as the pieces
+// [hi; mid; lo] of a bf16 [3T, d] matrix.
+__global__ void __launch_bounds__(256)
+router_jitter_split_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ noise,
+                           __nv_bfloat16* __restrict__ x3, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float v = __bfloat162float(x[i]) * noise[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    x3[i] = h;
+    x3[n + i] = m;
+    x3[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
 cudaError_t launch_router_jitter(const Shape& s, const Workspace& ws, const void* x,
                                  const float* noise, cudaStream_t stream) {
   const size_t n = static_cast<size_t>(s.T) * static_cast<size_t>(s.d);
   size_t blocks = (n + 255) / 256;
   if (blocks > 8 * 148) blocks = 8 * 148;
   if (blocks < 1) blocks = 1;
-  if (s.dtype == 1)
+  if (s.xsplit)
+    router_jitter_split_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), noise, static_cast<__nv_bfloat16*>(ws.x3), n);
+  else if (s.dtype == 1)
     router_jitter_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(x), noise, ws.xj, n);
   else

@@ -423,25 +423,37 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 //                at a time, transposed through shared memory into row-major
 //                128-byte stores
 constexpr int kWideThreads = 256;
-constexpr int kWideStages = 3;
+constexpr int kWideStages = 3;        // 64 KB stages (x tile + three W pieces)
+constexpr int kWideStagesX3 = 2;      // 96 KB stages (three x pieces + three W pieces)
 constexpr int kWideAcc = 2;          // tile accumulators, [hi | mid+lo] = 256 columns each
 constexpr int kWideNP = 128;         // experts per tile
 constexpr int kWidePitch = 33;       // transpose tile row pitch (floats)
 using WideCfg = TcCfg<kWideNP>;
+constexpr uint32_t kWideStageX3 = 3 * WideCfg::kABytes + kPieces * WideCfg::kPieceBytes;
+static_assert(kWideStagesX3 * kWideStageX3 == kWideStages * WideCfg::kStage,
+              "both forms of the wide kernel use the same stage memory");
 constexpr size_t kWideBarOff = static_cast<size_t>(kWideStages) * WideCfg::kStage;
 constexpr size_t kWideStgOff = kWideBarOff + 256;
 constexpr size_t kWideSmem = 1024 + kWideStgOff + 4 * 32 * kWidePitch * sizeof(float);
 
+// kX3: the router input is itself three bf16 pieces (a jittered fp32 input, x3
+// = [xh; xm; xl] [3T, d]); per k step six MMAs keep every product above fp32's
+// resolution: xh wh into the first accumulator, xh wm, xh wl, xm wh, xm wm and
+// xl wh into the second (xm wl, xl wm and xl wl are below 2^-24 of the result).
+template <bool kX3>
 __global__ void __launch_bounds__(kWideThreads, 1)
 router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
                           const __grid_constant__ CUtensorMap tmW, const TcArgs a) {
+  constexpr int kSt = kX3 ? kWideStagesX3 : kWideStages;
+  constexpr uint32_t kStageB = kX3 ? kWideStageX3 : WideCfg::kStage;
+  constexpr uint32_t kXB = (kX3 ? 3 : 1) * WideCfg::kABytes;   // x bytes of a stage
   // tmW: W3 = [hi; mid; lo] as bf16 [3N, d], box [128 rows, 64 k], 128-byte swizzle
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kWideBarOff);
-  uint64_t* empty_bar = full_bar + kWideStages;
-  uint64_t* tfull = empty_bar + kWideStages;
+  uint64_t* empty_bar = full_bar + kSt;
+  uint64_t* tfull = empty_bar + kSt;
   uint64_t* tempty = tfull + kWideAcc;
   uint64_t* drain_bar = tempty + kWideAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -456,7 +468,7 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
   const int n_tiles = (a.N + kWideNP - 1) / kWideNP;
   const int total = n_tiles * ((a.T + kBM - 1) / kBM);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kWideStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       ptx::mbar_init(&full_bar[s], 1);
       ptx::mbar_init(&empty_bar[s], 1);
     }
@@ -496,26 +508,29 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * kWideNP;
         for (int kb = 0; kb < a.nkb; ++kb, ++it) {
-          const int s = it % kWideStages;
-          const uint32_t ph = static_cast<uint32_t>(it / kWideStages) & 1u;
+          const int s = it % kSt;
+          const uint32_t ph = static_cast<uint32_t>(it / kSt) & 1u;
           if (!ptx::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, a.wait_ns)) {
             fail();
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * WideCfg::kStage;
-          ptx::mbar_arrive_expect_tx(&full_bar[s], WideCfg::kStage);
-          ptx::tma_load_2d(st, &tmX, &full_bar[s], kb * kBK, m0, pol_x);
+          uint8_t* st = smem + s * kStageB;
+          ptx::mbar_arrive_expect_tx(&full_bar[s], kStageB);
+#pragma unroll
+          for (int p = 0; p < (kX3 ? kPieces : 1); ++p)
+            ptx::tma_load_2d(st + p * WideCfg::kABytes, &tmX, &full_bar[s], kb * kBK,
+                             p * a.T + m0, pol_x);
 #pragma unroll
           for (int p = 0; p < kPieces; ++p)
-            ptx::tma_load_2d(st + WideCfg::kABytes + p * WideCfg::kPieceBytes, &tmW, &full_bar[s],
-                             kb * kBK, p * a.piece_rows + n0, pol_w);
+            ptx::tma_load_2d(st + kXB + p * WideCfg::kPieceBytes, &tmW, &full_bar[s], kb * kBK,
+                             p * a.piece_rows + n0, pol_w);
           issued |= 1u << s;
           last_par = (last_par & ~(1u << s)) | (ph << s);
         }
       }
       // every issued load lands before the stage memory goes away
-      for (int s = 0; s < kWideStages; ++s) {
+      for (int s = 0; s < kSt; ++s) {
         if (issued & (1u << s)) {
           volatile int never = 0;
           if (!ptx::mbar_wait(&full_bar[s], (last_par >> s) & 1u, &never, a.wait_ns))
@@ -541,28 +556,34 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
         const uint32_t d_hi = tmem_base + static_cast<uint32_t>(buf * 2 * kWideNP);
         const uint32_t d_ml = d_hi + kWideNP;
         for (int kb = 0; kb < a.nkb; ++kb, ++it) {
-          const int s = it % kWideStages;
-          const uint32_t ph = static_cast<uint32_t>(it / kWideStages) & 1u;
+          const int s = it % kSt;
+          const uint32_t ph = static_cast<uint32_t>(it / kSt) & 1u;
           if (!ptx::mbar_wait(&full_bar[s], ph, abort_flag, a.wait_ns)) {
             fail();
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a_addr = ptx::smem_u32(smem + s * WideCfg::kStage);
-          const uint32_t b_addr = a_addr + WideCfg::kABytes;
+          const uint32_t a_addr = ptx::smem_u32(smem + s * kStageB);
+          const uint32_t b_addr = a_addr + kXB;
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             const uint32_t ko = k * kUmmaK * 2;
-            const uint64_t ad = ptx::umma_desc_sw128_kmajor(a_addr + ko);
+            const uint64_t ah = ptx::umma_desc_sw128_kmajor(a_addr + ko);
+            const uint64_t wh = ptx::umma_desc_sw128_kmajor(b_addr + ko);
+            const uint64_t wm = ptx::umma_desc_sw128_kmajor(b_addr + WideCfg::kPieceBytes + ko);
+            const uint64_t wl = ptx::umma_desc_sw128_kmajor(b_addr + 2 * WideCfg::kPieceBytes + ko);
             const uint32_t first = (kb | k) != 0 ? 1u : 0u;
-            ptx::umma_bf16(d_hi, ad, ptx::umma_desc_sw128_kmajor(b_addr + ko), idesc, first);
-            ptx::umma_bf16(d_ml, ad,
-                           ptx::umma_desc_sw128_kmajor(b_addr + WideCfg::kPieceBytes + ko),
-                           idesc, first);
-            ptx::umma_bf16(d_ml, ad,
-                           ptx::umma_desc_sw128_kmajor(b_addr + 2 * WideCfg::kPieceBytes + ko),
-                           idesc, 1u);
+            ptx::umma_bf16(d_hi, ah, wh, idesc, first);
+            ptx::umma_bf16(d_ml, ah, wm, idesc, first);
+            ptx::umma_bf16(d_ml, ah, wl, idesc, 1u);
+            if constexpr (kX3) {
+              const uint64_t am = ptx::umma_desc_sw128_kmajor(a_addr + WideCfg::kABytes + ko);
+              const uint64_t al = ptx::umma_desc_sw128_kmajor(a_addr + 2 * WideCfg::kABytes + ko);
+              ptx::umma_bf16(d_ml, am, wh, idesc, 1u);
+              ptx::umma_bf16(d_ml, am, wm, idesc, 1u);
+              ptx::umma_bf16(d_ml, al, wh, idesc, 1u);
+            }
           }
           ptx::umma_commit(&empty_bar[s]);   // frees the stage once these MMAs are done
         }
@@ -720,11 +741,11 @@ cudaError_t launch_wide(const Shape& s, const Workspace& ws, const CUtensorMap& 
   a.wait_ns = wait_limit_ns();
   const int64_t tiles = ((s.T + kBM - 1) / kBM) * ((s.N + kWideNP - 1) / kWideNP);
   const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
-  cudaError_t e = cudaFuncSetAttribute(router_logits_wide_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = s.xsplit ? router_logits_wide_kernel<true> : router_logits_wide_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kWideSmem));
   if (e != cudaSuccess) return e;
-  return launch_dependent(router_logits_wide_kernel, dim3(grid), dim3(kWideThreads), kWideSmem,
+  return launch_dependent(kern, dim3(grid), dim3(kWideThreads), kWideSmem,
                           stream, tmX, tmW, a);
 }
 
@@ -735,7 +756,7 @@ int router_tc_padded_experts(int64_t N) {
 }
 
 int router_tc_stages(const Shape& s, int num_sms) {
-  if (s.router_path == kRouterTCWide) return kWideStages;
+  if (s.router_path == kRouterTCWide) return s.xsplit ? kWideStagesX3 : kWideStages;
   switch (router_tc_padded_experts(s.N)) {
     case 32: return tc_stages<32>(s, num_sms);
     case 64: return tc_stages<64>(s, num_sms);

@@ -80,7 +80,9 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
       take(s.router_path == kRouterTC || s.router_path == kRouterTCWide
                ? 3 * N * static_cast<size_t>(s.d) * 2
                : 0));
-  w.xj = reinterpret_cast<float*>(take(s.jitter ? T * static_cast<size_t>(s.d) * 4 : 0));
+  w.xj = reinterpret_cast<float*>(
+      take(s.jitter && !s.xsplit ? T * static_cast<size_t>(s.d) * 4 : 0));
+  w.x3 = reinterpret_cast<void*>(take(s.xsplit ? 3 * T * static_cast<size_t>(s.d) * 2 : 0));
   w.xbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d) * elem));
   w.hbuf = reinterpret_cast<void*>(take(A * static_cast<size_t>(s.d_ff) * elem));
   w.ybuf = reinterpret_cast<void*>(take(top2 && !s.ntlb ? A * static_cast<size_t>(s.d) * elem : 0));
@@ -184,11 +186,15 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->jitter = jitter ? 1 : 0;
   if (glu && N * 2 * d_ff > INT32_MAX) return SWL_ERR_UNSUPPORTED;   // TMA row coordinates
   // the tensor-core router serves bf16 layers unless the FFMA router was chosen;
-  // a jittered router input (x * noise, fp32) always takes the FFMA router
-  const bool tensor_router =
-      dtype == SWL_BF16 && !jitter && g_router_mode.load() == SWL_ROUTER_TENSOR;
+  // a jittered router input (x * noise, fp32) takes the tensor-core logits of
+  // the wide path (N > 128 or top-2) with x * noise split into bf16 pieces, and
+  // the FFMA router otherwise
+  const bool wide = N > kFusedRouterMaxN || topk == 2;
+  const bool tensor_router = dtype == SWL_BF16 && (!jitter || wide) &&
+                             g_router_mode.load() == SWL_ROUTER_TENSOR;
   const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0, topk);
   s->router_path = rp.path;
+  s->xsplit = jitter && rp.path == kRouterTCWide ? 1 : 0;
   s->kslice = rp.kslice;
   s->ksplit_eff = rp.ksplit;
   s->tpb = rp.tpb;
@@ -277,13 +283,13 @@ static swl_status run_routing(const Shape& s, const Workspace& ws, const void* x
                               int32_t* pos_in_expert, const float* b_r, cudaStream_t stream,
                               Rec& rec, const float* router_noise = nullptr) {
   if (s.jitter) {
-    // the router sees x * noise (fp32); the experts keep x
+    // the router sees x * noise (fp32, or its three bf16 pieces); the experts keep x
     if (launch_router_jitter(s, ws, x, router_noise, stream) != cudaSuccess) return SWL_ERR_CUDA;
-    x = ws.xj;
+    x = s.xsplit ? ws.x3 : static_cast<const void*>(ws.xj);
   }
   if (s.router_path == kRouterTC || s.router_path == kRouterTCWide) {
     CUtensorMap tx, tw;
-    if (!make_tmap_bf16(&tx, x, s.d, s.T, 128) ||
+    if (!make_tmap_bf16(&tx, x, s.d, (s.xsplit ? 3 : 1) * s.T, 128) ||
         !make_tmap_bf16(&tw, ws.w3, s.d, 3 * s.N,
                         s.router_path == kRouterTCWide ? 128 : router_tc_padded_experts(s.N)))
       return SWL_ERR_CUDA;
