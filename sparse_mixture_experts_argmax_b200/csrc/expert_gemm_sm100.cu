@@ -34,8 +34,13 @@
 // claimed by a CTA that is already running; the token-block count of each
 // expert comes from the device tile prefix written by the dispatch scan.  The
 // scheduler keeps the claim, the decode (dependent loads of the prefix) and the
-// GEMM2 readiness wait off the producer's path.  Every wait is bounded; a
-// stuck pipeline sets the device error word and the CTA drains and exits.
+// GEMM2 readiness wait off the producer's path.  Within an expert the tiles go
+// token block by token block when its weights fit in L2 (the first blocks'
+// GEMM2 can start while GEMM1 of the last ones runs).  Layers with a long GEMM2
+// reduction cut their GEMM2 tiles over K (the kSplit instantiation): each
+// sub-tile stores an fp32 partial and ffn_split_reduce_kernel, launched after,
+// adds them in k order and stores the rows.  Every wait is bounded; a stuck
+// pipeline sets the device error word and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
