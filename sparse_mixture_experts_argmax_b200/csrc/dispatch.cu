@@ -212,11 +212,9 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     base_tiles += (m + tile_rows - 1) / tile_rows;
   }
   if (split.factor > 1) {
-    // GEMM2 split over K for the LAST experts whose groups (an expert's
-    // 128-feature by token-tile GEMM2 tiles) fit the budget: their tiles are
-    // the last ones handed out, so splitting them shortens the FFN's tail.
-    // Written: the split tile prefix, each expert's first group (-1: not
-    // split) and the group table.
+    // GEMM2 split over K, in expert order while the groups (an expert's
+    // 128-feature by token-tile GEMM2 tiles) fit the budget: the split tile
+    // prefix, each expert's first group (-1: not split) and the group table
     __shared__ int s_tot_groups, s_tot_tiles2;
     for (int i = threadIdx.x; i < split.max_groups; i += kScanThreads)
       reinterpret_cast<int4*>(split.groups)[i] = make_int4(-1, 0, 0, 0);
@@ -226,13 +224,12 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
       groups += (m + tile_rows - 1) / tile_rows * split.m_tiles2;
     }
     int g = block_excl_scan(groups, s_warp, &s_tot_groups);
-    const int first_on = max(0, s_tot_groups - split.max_groups);   // first split group
     int tiles2 = 0;
     for (int i = e0; i < e1; ++i) {
       const int m = min(__ldcg(exp_count + i), C_eff);
       const int tl = (m + tile_rows - 1) / tile_rows;
       const int grp = tl * split.m_tiles2;
-      const bool on = grp > 0 && g >= first_on;
+      const bool on = grp > 0 && g + grp <= split.max_groups;
       tiles2 += tl * (on ? split.factor : 1);
       g += grp;
     }
@@ -242,15 +239,14 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
       const int m = min(__ldcg(exp_count + i), C_eff);
       const int tl = (m + tile_rows - 1) / tile_rows;
       const int grp = tl * split.m_tiles2;
-      const bool on = grp > 0 && g >= first_on;
-      const int gb = g - first_on;
+      const bool on = grp > 0 && g + grp <= split.max_groups;
       split.tile_prefix2[i] = base2;
-      split.split_base[i] = on ? gb : -1;
+      split.split_base[i] = on ? g : -1;
       if (on) {
-        // group gb + mt * tl + nt: m-tile mt of token tile nt (the FFN's numbering)
+        // group g + mt * tl + nt: m-tile mt of token tile nt (the FFN's numbering)
         for (int mt = 0; mt < split.m_tiles2; ++mt)
           for (int nt = 0; nt < tl; ++nt)
-            reinterpret_cast<int4*>(split.groups)[gb + mt * tl + nt] = make_int4(i, mt, nt, 0);
+            reinterpret_cast<int4*>(split.groups)[g + mt * tl + nt] = make_int4(i, mt, nt, 0);
       }
       base2 += tl * (on ? split.factor : 1);
       g += grp;

@@ -200,12 +200,11 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   s->tpb = rp.tpb;
   s->nblk = static_cast<int>((T + s->tpb - 1) / s->tpb);
   s->tile_rows = dtype == SWL_BF16 ? bf16_tile_rows(s->C_eff) : kF32TileRows;
-  // GEMM2 split over K: bf16 top-1 ReLU layers with token tiles of at least 128
-  // rows and a long GEMM2 reduction (d_ff >= 4096), whose dispatch is the scan
-  // kernel (the last experts' tiles, up to kSplitMaxGroups groups)
+  // GEMM2 split over K: bf16 top-1 ReLU layers with full 256-row token tiles and
+  // a long GEMM2 reduction (d_ff >= 4096), whose dispatch is the scan kernel
   s->ffn_split = 1;
-  if (dtype == SWL_BF16 && topk == 1 && !glu && !ntlb && s->tile_rows >= 128 &&
-      d_ff >= 4096 && !dispatch_fused_ok(*s))
+  if (dtype == SWL_BF16 && topk == 1 && !glu && s->tile_rows == 256 && d_ff >= 4096 &&
+      !dispatch_fused_ok(*s))
     s->ffn_split = kSplitFactor;
   return SWL_OK;
 }

@@ -129,7 +129,7 @@ _PLAN_CASES = [
                                    "gemm2_split": 1}),
     ("large_T16384_d1024_N128", None, {"router": "tc", "ksplit": 1, "router_stages": 3,
                                        "dispatch": "two_kernel", "tile_rows": 128,
-                                       "accumulators": 4, "gemm2_split": 4}),
+                                       "accumulators": 4}),
     ("skewed_T32768_d2048_N64", None, {"router": "tc", "ksplit": 1, "router_stages": 2,
                                        "dispatch": "two_kernel", "tile_rows": 256,
                                        "accumulators": 2, "gemm2_split": 4}),

@@ -318,7 +318,7 @@ _VARIANT_SHAPES = [
     ("ffma_tile", 25700, 32, 32, 48, 1.0, "f32"),
     ("two_kernel_dispatch", 20000, 256, 32, 8, 1.0, "f32"),
     ("two_accumulators", 900, 64, 64, 4, 1.0, "bf16"),
-    # GEMM2 split over K on the last experts, unsplit tiles on the rest
+    # GEMM2 split over K on the first experts, unsplit tiles on the rest
     ("gemm2_split_mixed", 12288, 768, 4096, 8, 1.0, "bf16"),
     # streaming softmax: a warp per row at full width (N = 1024), a warp pair per row
     # with a ragged second half (N = 1500); token blocks of 45 and 37 tokens
