@@ -408,57 +408,65 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 }
 
 // Logits of wide layers (N > 128 experts), persistent: one CTA per SM takes
-// tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... of 128 tokens by 128
-// experts (expert tiles fastest, so the CTAs running together share the x tile
-// in L2; W3 stays in L2), and writes them to a.logits [T, N] fp32 without the
-// bias (the softmax kernel adds it).
-//   warp 0       TMA producer: per k-block the x tile and the three piece tiles
-//                (64 KB) into a ring of kWideStages stages, across tiles
-//   warp 1       MMA issuer: per 16-wide k step x * hi into the tile's first
-//                accumulator, x * mid and x * lo into its second; kWideAcc tile
-//                accumulators in TMEM, so the read-out of one tile runs under
-//                the MMAs of the next
-//   warp 2       TMEM allocator
-//   warps 4..7   read-out (thread = token row): z = D_hi + D_midlo, 32 experts
-//                at a time, transposed through shared memory into row-major
-//                128-byte stores
-constexpr int kWideThreads = 256;
-constexpr int kWideStages = 3;        // 64 KB stages (x tile + three W pieces)
-constexpr int kWideStagesX3 = 2;      // 96 KB stages (three x pieces + three W pieces)
-constexpr int kWideAcc = 2;          // tile accumulators, [hi | mid+lo] = 256 columns each
-constexpr int kWideNP = 128;         // experts per tile
-constexpr int kWidePitch = 33;       // transpose tile row pitch (floats)
+// units u = blockIdx.x, blockIdx.x + gridDim.x, ... of kTT token tiles of 128
+// tokens by one tile of 128 experts (expert tiles fastest, so the CTAs running
+// together share x tiles in L2; W3 stays in L2), and writes them to a.logits
+// [T, N] fp32 without the bias (the softmax kernel adds it).
+//   warp 0       TMA producer: per k-block the unit's x tiles and the three W
+//                piece tiles into a ring of stages, across units
+//   warp 1       MMA issuer: per 16-wide k step and token tile, x * hi into the
+//                tile's first accumulator and x * mid, x * lo into its second
+//   warp 2       TMEM allocator (512 columns: [hi | mid+lo] = 256 per token tile)
+//   warps 4..    read-out, four warps per token tile (thread = token row):
+//                z = D_hi + D_midlo, 32 experts at a time, transposed through
+//                shared memory into row-major 128-byte stores
+// kTT = 1: two units' accumulators, so a unit's read-out runs under the next
+// unit's MMAs.  kTT = 2: the W pieces of a k-block serve two token tiles (80 KB
+// of operands per two tiles instead of 128), one unit in TMEM at a time.
+// kXP = 3: the router input is itself three bf16 pieces (a jittered fp32
+// input, x3 = [xh; xm; xl] [3T, d]); per k step six MMAs keep every product
+// above fp32's resolution: xh wh into the first accumulator, xh wm, xh wl,
+// xm wh, xm wm and xl wh into the second (xm wl, xl wm and xl wl are below
+// 2^-24 of the result).
+constexpr int kWideNP = 128;          // experts per tile
+constexpr int kWidePitch = 33;        // transpose tile row pitch (floats)
 using WideCfg = TcCfg<kWideNP>;
-constexpr uint32_t kWideStageX3 = 3 * WideCfg::kABytes + kPieces * WideCfg::kPieceBytes;
-static_assert(kWideStagesX3 * kWideStageX3 == kWideStages * WideCfg::kStage,
-              "both forms of the wide kernel use the same stage memory");
-constexpr size_t kWideBarOff = static_cast<size_t>(kWideStages) * WideCfg::kStage;
-constexpr size_t kWideStgOff = kWideBarOff + 256;
-constexpr size_t kWideSmem = 1024 + kWideStgOff + 4 * 32 * kWidePitch * sizeof(float);
 
-// kX3: the router input is itself three bf16 pieces (a jittered fp32 input, x3
-// = [xh; xm; xl] [3T, d]); per k step six MMAs keep every product above fp32's
-// resolution: xh wh into the first accumulator, xh wm, xh wl, xm wh, xm wm and
-// xl wh into the second (xm wl, xl wm and xl wl are below 2^-24 of the result).
-template <bool kX3>
-__global__ void __launch_bounds__(kWideThreads, 1)
+template <int kXP, int kTT>
+struct WideK {
+  static constexpr uint32_t kXB = kTT * kXP * WideCfg::kABytes;      // x bytes of a stage
+  static constexpr uint32_t kStageB = kXB + kPieces * WideCfg::kPieceBytes;
+  static constexpr int kSt = kStageB <= 64 * 1024 ? 3 : 2;
+  static constexpr int kAccCols = kTT * 2 * kWideNP;                 // TMEM columns of a unit
+  static constexpr int kBufs = 512 / kAccCols;
+  static constexpr int kEpiWarps = 4 * kTT;
+  static constexpr int kThreads = 128 + 32 * kEpiWarps;
+  static constexpr size_t kBarOff = static_cast<size_t>(kSt) * kStageB;
+  static constexpr size_t kStgOff = kBarOff + 256;
+  static constexpr size_t kSmem =
+      1024 + kStgOff + static_cast<size_t>(kEpiWarps) * 32 * kWidePitch * sizeof(float);
+  static_assert(kSmem <= 232448, "shared memory of the wide logits kernel");
+};
+constexpr int kWideTT = 2;            // token tiles per unit of the plain (unjittered) input
+
+template <int kXP, int kTT>
+__global__ void __launch_bounds__(WideK<kXP, kTT>::kThreads, 1)
 router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
                           const __grid_constant__ CUtensorMap tmW, const TcArgs a) {
-  constexpr int kSt = kX3 ? kWideStagesX3 : kWideStages;
-  constexpr uint32_t kStageB = kX3 ? kWideStageX3 : WideCfg::kStage;
-  constexpr uint32_t kXB = (kX3 ? 3 : 1) * WideCfg::kABytes;   // x bytes of a stage
+  using K = WideK<kXP, kTT>;
+  constexpr int kSt = K::kSt;
   // tmW: W3 = [hi; mid; lo] as bf16 [3N, d], box [128 rows, 64 k], 128-byte swizzle
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kWideBarOff);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + K::kBarOff);
   uint64_t* empty_bar = full_bar + kSt;
   uint64_t* tfull = empty_bar + kSt;
-  uint64_t* tempty = tfull + kWideAcc;
-  uint64_t* drain_bar = tempty + kWideAcc;
+  uint64_t* tempty = tfull + K::kBufs;
+  uint64_t* drain_bar = tempty + K::kBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* stg = reinterpret_cast<float*>(smem + kWideStgOff);   // [4 warps][32][kWidePitch]
+  float* stg = reinterpret_cast<float*>(smem + K::kStgOff);   // [epilogue warps][32][kWidePitch]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -466,15 +474,16 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
     a.hdr->done = 0u;      // arrival counter of the dispatch scan
   }
   const int n_tiles = (a.N + kWideNP - 1) / kWideNP;
-  const int total = n_tiles * ((a.T + kBM - 1) / kBM);
+  const int t_tiles = (a.T + kBM - 1) / kBM;
+  const int total = n_tiles * ((t_tiles + kTT - 1) / kTT);   // units
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSt; ++s) {
       ptx::mbar_init(&full_bar[s], 1);
       ptx::mbar_init(&empty_bar[s], 1);
     }
-    for (int b = 0; b < kWideAcc; ++b) {
+    for (int b = 0; b < K::kBufs; ++b) {
       ptx::mbar_init(&tfull[b], 1);
-      ptx::mbar_init(&tempty[b], 4);   // one arrive per read-out warp
+      ptx::mbar_init(&tempty[b], K::kEpiWarps);   // one arrive per read-out warp
     }
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -484,7 +493,7 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
     ptx::prefetch_tmap(&tmW);
   }
   if (warp == 2) {
-    ptx::tmem_alloc(tmem_slot, 2 * kWideAcc * kWideNP);
+    ptx::tmem_alloc(tmem_slot, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -499,14 +508,14 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol_x = ptx::l2_policy_evict_first();   // x: read by one row of tiles
-      const uint64_t pol_w = ptx::l2_policy_evict_last();    // W3: read by every tile
+      const uint64_t pol_x = ptx::l2_policy_evict_first();   // x: read by one row of units
+      const uint64_t pol_w = ptx::l2_policy_evict_last();    // W3: read by every unit
       uint32_t issued = 0u, last_par = 0u;
-      pdl_wait();   // W3 comes from the split kernel
+      pdl_wait();   // W3 comes from the split kernel (and x3 from the jitter kernel)
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * kWideNP;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const int m0 = (u / n_tiles) * kTT * kBM, n0 = (u % n_tiles) * kWideNP;
         for (int kb = 0; kb < a.nkb; ++kb, ++it) {
           const int s = it % kSt;
           const uint32_t ph = static_cast<uint32_t>(it / kSt) & 1u;
@@ -515,16 +524,18 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * kStageB;
-          ptx::mbar_arrive_expect_tx(&full_bar[s], kStageB);
+          uint8_t* st = smem + s * K::kStageB;
+          ptx::mbar_arrive_expect_tx(&full_bar[s], K::kStageB);
 #pragma unroll
-          for (int p = 0; p < (kX3 ? kPieces : 1); ++p)
-            ptx::tma_load_2d(st + p * WideCfg::kABytes, &tmX, &full_bar[s], kb * kBK,
-                             p * a.T + m0, pol_x);
+          for (int tt = 0; tt < kTT; ++tt)
+#pragma unroll
+            for (int p = 0; p < kXP; ++p)
+              ptx::tma_load_2d(st + (tt * kXP + p) * WideCfg::kABytes, &tmX, &full_bar[s],
+                               kb * kBK, p * a.T + m0 + tt * kBM, pol_x);
 #pragma unroll
           for (int p = 0; p < kPieces; ++p)
-            ptx::tma_load_2d(st + kXB + p * WideCfg::kPieceBytes, &tmW, &full_bar[s], kb * kBK,
-                             p * a.piece_rows + n0, pol_w);
+            ptx::tma_load_2d(st + K::kXB + p * WideCfg::kPieceBytes, &tmW, &full_bar[s],
+                             kb * kBK, p * a.piece_rows + n0, pol_w);
           issued |= 1u << s;
           last_par = (last_par & ~(1u << s)) | (ph << s);
         }
@@ -543,18 +554,17 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = ptx::umma_idesc_bf16_f32(kWideNP);
-      int it = 0, tc = 0;
+      int it = 0, uc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
-        const int buf = tc % kWideAcc;
-        if (!ptx::mbar_wait(&tempty[buf], (static_cast<uint32_t>(tc / kWideAcc) & 1u) ^ 1u,
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++uc) {
+        const int buf = uc % K::kBufs;
+        if (!ptx::mbar_wait(&tempty[buf], (static_cast<uint32_t>(uc / K::kBufs) & 1u) ^ 1u,
                             abort_flag, a.wait_ns)) {
           fail();
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d_hi = tmem_base + static_cast<uint32_t>(buf * 2 * kWideNP);
-        const uint32_t d_ml = d_hi + kWideNP;
+        const uint32_t d_unit = tmem_base + static_cast<uint32_t>(buf * K::kAccCols);
         for (int kb = 0; kb < a.nkb; ++kb, ++it) {
           const int s = it % kSt;
           const uint32_t ph = static_cast<uint32_t>(it / kSt) & 1u;
@@ -564,25 +574,31 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a_addr = ptx::smem_u32(smem + s * kStageB);
-          const uint32_t b_addr = a_addr + kXB;
+          const uint32_t x_addr = ptx::smem_u32(smem + s * K::kStageB);
+          const uint32_t b_addr = x_addr + K::kXB;
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             const uint32_t ko = k * kUmmaK * 2;
-            const uint64_t ah = ptx::umma_desc_sw128_kmajor(a_addr + ko);
             const uint64_t wh = ptx::umma_desc_sw128_kmajor(b_addr + ko);
             const uint64_t wm = ptx::umma_desc_sw128_kmajor(b_addr + WideCfg::kPieceBytes + ko);
             const uint64_t wl = ptx::umma_desc_sw128_kmajor(b_addr + 2 * WideCfg::kPieceBytes + ko);
             const uint32_t first = (kb | k) != 0 ? 1u : 0u;
-            ptx::umma_bf16(d_hi, ah, wh, idesc, first);
-            ptx::umma_bf16(d_ml, ah, wm, idesc, first);
-            ptx::umma_bf16(d_ml, ah, wl, idesc, 1u);
-            if constexpr (kX3) {
-              const uint64_t am = ptx::umma_desc_sw128_kmajor(a_addr + WideCfg::kABytes + ko);
-              const uint64_t al = ptx::umma_desc_sw128_kmajor(a_addr + 2 * WideCfg::kABytes + ko);
-              ptx::umma_bf16(d_ml, am, wh, idesc, 1u);
-              ptx::umma_bf16(d_ml, am, wm, idesc, 1u);
-              ptx::umma_bf16(d_ml, al, wh, idesc, 1u);
+#pragma unroll
+            for (int tt = 0; tt < kTT; ++tt) {
+              const uint32_t a_t = x_addr + tt * kXP * WideCfg::kABytes;
+              const uint32_t d_hi = d_unit + static_cast<uint32_t>(tt * 2 * kWideNP);
+              const uint32_t d_ml = d_hi + kWideNP;
+              const uint64_t ah = ptx::umma_desc_sw128_kmajor(a_t + ko);
+              ptx::umma_bf16(d_hi, ah, wh, idesc, first);
+              ptx::umma_bf16(d_ml, ah, wm, idesc, first);
+              ptx::umma_bf16(d_ml, ah, wl, idesc, 1u);
+              if constexpr (kXP == 3) {
+                const uint64_t am = ptx::umma_desc_sw128_kmajor(a_t + WideCfg::kABytes + ko);
+                const uint64_t al = ptx::umma_desc_sw128_kmajor(a_t + 2 * WideCfg::kABytes + ko);
+                ptx::umma_bf16(d_ml, am, wh, idesc, 1u);
+                ptx::umma_bf16(d_ml, am, wm, idesc, 1u);
+                ptx::umma_bf16(d_ml, al, wh, idesc, 1u);
+              }
             }
           }
           ptx::umma_commit(&empty_bar[s]);   // frees the stage once these MMAs are done
@@ -599,20 +615,21 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
   } else if (warp >= 4) {
     // ------------------------------------------------------------ read-out
     const int q = warp & 3;                  // TMEM lanes [32q, 32q + 32): token rows
-    float* st = stg + q * 32 * kWidePitch;
+    const int tt = (warp - 4) >> 2;          // token tile of the unit
+    float* st = stg + (warp - 4) * 32 * kWidePitch;
     const bool vec = (a.N % 4) == 0;
-    int tc = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
-      const int buf = tc % kWideAcc;
-      const bool got = ptx::mbar_wait(&tfull[buf], static_cast<uint32_t>(tc / kWideAcc) & 1u,
+    int uc = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++uc) {
+      const int buf = uc % K::kBufs;
+      const bool got = ptx::mbar_wait(&tfull[buf], static_cast<uint32_t>(uc / K::kBufs) & 1u,
                                       abort_flag, a.wait_ns);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) fail();
         break;
       }
       ptx::tc_fence_after();
-      const int m0 = (t / n_tiles) * kBM + q * 32, n0 = (t % n_tiles) * kWideNP;
-      const uint32_t ta = tmem_base + static_cast<uint32_t>(buf * 2 * kWideNP) +
+      const int m0 = ((u / n_tiles) * kTT + tt) * kBM + q * 32, n0 = (u % n_tiles) * kWideNP;
+      const uint32_t ta = tmem_base + static_cast<uint32_t>(buf * K::kAccCols + tt * 2 * kWideNP) +
                           (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < kWideNP / 32; ++c) {
@@ -621,7 +638,7 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
         ptx::tmem_ld_32x32b_x32(ta + static_cast<uint32_t>(kWideNP + c * 32), r1);
         ptx::tmem_ld_wait();
         if (c == kWideNP / 32 - 1) {
-          // the whole accumulator is in registers: the MMAs of a later tile may reuse it
+          // the whole accumulator is in registers: the MMAs of a later unit may reuse it
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
@@ -656,7 +673,7 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
   __syncthreads();
   if (warp == 2) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, 2 * kWideAcc * kWideNP);
+    ptx::tmem_dealloc(tmem_base, 512);
   }
 }
 
@@ -729,6 +746,19 @@ cudaError_t launch_tc_t(const Shape& s, const Workspace& ws, const CUtensorMap& 
   return cudaLaunchKernelEx(&cfg, router_tc_kernel<NP>, tmX, tmW, a);
 }
 
+template <int kXP, int kTT>
+cudaError_t launch_wide_t(const TcArgs& a, const CUtensorMap& tmX, const CUtensorMap& tmW,
+                          int64_t units, int num_sms, cudaStream_t stream) {
+  using K = WideK<kXP, kTT>;
+  const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
+  cudaError_t e = cudaFuncSetAttribute(router_logits_wide_kernel<kXP, kTT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(K::kSmem));
+  if (e != cudaSuccess) return e;
+  return launch_dependent(router_logits_wide_kernel<kXP, kTT>, dim3(grid), dim3(K::kThreads),
+                          K::kSmem, stream, tmX, tmW, a);
+}
+
 cudaError_t launch_wide(const Shape& s, const Workspace& ws, const CUtensorMap& tmX,
                         const CUtensorMap& tmW, int num_sms, cudaStream_t stream) {
   TcArgs a = {};
@@ -739,14 +769,10 @@ cudaError_t launch_wide(const Shape& s, const Workspace& ws, const CUtensorMap& 
   a.nkb = static_cast<int>((s.d + kBK - 1) / kBK);
   a.hdr = ws.hdr;
   a.wait_ns = wait_limit_ns();
-  const int64_t tiles = ((s.T + kBM - 1) / kBM) * ((s.N + kWideNP - 1) / kWideNP);
-  const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
-  auto kern = s.xsplit ? router_logits_wide_kernel<true> : router_logits_wide_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kWideSmem));
-  if (e != cudaSuccess) return e;
-  return launch_dependent(kern, dim3(grid), dim3(kWideThreads), kWideSmem,
-                          stream, tmX, tmW, a);
+  const int64_t t_tiles = (s.T + kBM - 1) / kBM, n_tiles = (s.N + kWideNP - 1) / kWideNP;
+  if (s.xsplit) return launch_wide_t<3, 1>(a, tmX, tmW, t_tiles * n_tiles, num_sms, stream);
+  return launch_wide_t<1, kWideTT>(a, tmX, tmW, (t_tiles + kWideTT - 1) / kWideTT * n_tiles,
+                                   num_sms, stream);
 }
 
 }  // namespace
@@ -756,7 +782,7 @@ int router_tc_padded_experts(int64_t N) {
 }
 
 int router_tc_stages(const Shape& s, int num_sms) {
-  if (s.router_path == kRouterTCWide) return s.xsplit ? kWideStagesX3 : kWideStages;
+  if (s.router_path == kRouterTCWide) return s.xsplit ? WideK<3, 1>::kSt : WideK<1, kWideTT>::kSt;
   switch (router_tc_padded_experts(s.N)) {
     case 32: return tc_stages<32>(s, num_sms);
     case 64: return tc_stages<64>(s, num_sms);
