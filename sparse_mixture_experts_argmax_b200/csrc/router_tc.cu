@@ -414,20 +414,22 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 // [T, N] fp32 without the bias (the softmax kernel adds it).
 //   warp 0       TMA producer: per k-block the unit's x tiles and the three W
 //                piece tiles into a ring of stages, across units
-//   warp 1       MMA issuer: per 16-wide k step and token tile, x * hi into the
-//                tile's first accumulator and x * mid, x * lo into its second
-//   warp 2       TMEM allocator (512 columns: [hi | mid+lo] = 256 per token tile)
-//   warps 4..    read-out, four warps per token tile (thread = token row):
-//                z = D_hi + D_midlo, 32 experts at a time, transposed through
-//                shared memory into row-major 128-byte stores
-// kTT = 1: two units' accumulators, so a unit's read-out runs under the next
-// unit's MMAs.  kTT = 2: the W pieces of a k-block serve two token tiles (80 KB
-// of operands per two tiles instead of 128), one unit in TMEM at a time.
+//   warp 1       MMA issuer: per 16-wide k step and token tile, x * hi, x * mid
+//                and x * lo into the tile's accumulator (128 TMEM columns)
+//   warp 2       TMEM allocator (512 columns: 512 / (128 kTT) unit accumulators)
+//   warps 4..    read-out, four warps per token tile (thread = token row): z,
+//                32 experts at a time, transposed through shared memory into
+//                row-major 128-byte stores
+// Each product x_k * piece_k is exact, and all of them go into one fp32
+// accumulator: 3 x 64 tensor-core accumulation steps of a 1024-wide row
+// against 1024 roundings of an fp32 FFMA loop.  kTT = 2: the W pieces of a
+// k-block serve two token tiles (80 KB of operands per two tiles instead of
+// 128); with one 128-column accumulator per token tile, two units fit in TMEM
+// and a unit's read-out runs under the next unit's MMAs.
 // kXP = 3: the router input is itself three bf16 pieces (a jittered fp32
 // input, x3 = [xh; xm; xl] [3T, d]); per k step six MMAs keep every product
-// above fp32's resolution: xh wh into the first accumulator, xh wm, xh wl,
-// xm wh, xm wm and xl wh into the second (xm wl, xl wm and xl wl are below
-// 2^-24 of the result).
+// above fp32's resolution: xh wh, xh wm, xh wl, xm wh, xm wm and xl wh (xm wl,
+// xl wm and xl wl are below 2^-24 of the result).
 constexpr int kWideNP = 128;          // experts per tile
 constexpr int kWidePitch = 33;        // transpose tile row pitch (floats)
 using WideCfg = TcCfg<kWideNP>;
@@ -437,7 +439,7 @@ struct WideK {
   static constexpr uint32_t kXB = kTT * kXP * WideCfg::kABytes;      // x bytes of a stage
   static constexpr uint32_t kStageB = kXB + kPieces * WideCfg::kPieceBytes;
   static constexpr int kSt = kStageB <= 64 * 1024 ? 3 : 2;
-  static constexpr int kAccCols = kTT * 2 * kWideNP;                 // TMEM columns of a unit
+  static constexpr int kAccCols = kTT * kWideNP;                     // TMEM columns of a unit
   static constexpr int kBufs = 512 / kAccCols;
   static constexpr int kEpiWarps = 4 * kTT;
   static constexpr int kThreads = 128 + 32 * kEpiWarps;
@@ -586,18 +588,17 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
 #pragma unroll
             for (int tt = 0; tt < kTT; ++tt) {
               const uint32_t a_t = x_addr + tt * kXP * WideCfg::kABytes;
-              const uint32_t d_hi = d_unit + static_cast<uint32_t>(tt * 2 * kWideNP);
-              const uint32_t d_ml = d_hi + kWideNP;
+              const uint32_t d_t = d_unit + static_cast<uint32_t>(tt * kWideNP);
               const uint64_t ah = ptx::umma_desc_sw128_kmajor(a_t + ko);
-              ptx::umma_bf16(d_hi, ah, wh, idesc, first);
-              ptx::umma_bf16(d_ml, ah, wm, idesc, first);
-              ptx::umma_bf16(d_ml, ah, wl, idesc, 1u);
+              ptx::umma_bf16(d_t, ah, wh, idesc, first);
+              ptx::umma_bf16(d_t, ah, wm, idesc, 1u);
+              ptx::umma_bf16(d_t, ah, wl, idesc, 1u);
               if constexpr (kXP == 3) {
                 const uint64_t am = ptx::umma_desc_sw128_kmajor(a_t + WideCfg::kABytes + ko);
                 const uint64_t al = ptx::umma_desc_sw128_kmajor(a_t + 2 * WideCfg::kABytes + ko);
-                ptx::umma_bf16(d_ml, am, wh, idesc, 1u);
-                ptx::umma_bf16(d_ml, am, wm, idesc, 1u);
-                ptx::umma_bf16(d_ml, al, wh, idesc, 1u);
+                ptx::umma_bf16(d_t, am, wh, idesc, 1u);
+                ptx::umma_bf16(d_t, am, wm, idesc, 1u);
+                ptx::umma_bf16(d_t, al, wh, idesc, 1u);
               }
             }
           }
@@ -629,13 +630,12 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
       }
       ptx::tc_fence_after();
       const int m0 = ((u / n_tiles) * kTT + tt) * kBM + q * 32, n0 = (u % n_tiles) * kWideNP;
-      const uint32_t ta = tmem_base + static_cast<uint32_t>(buf * K::kAccCols + tt * 2 * kWideNP) +
+      const uint32_t ta = tmem_base + static_cast<uint32_t>(buf * K::kAccCols + tt * kWideNP) +
                           (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < kWideNP / 32; ++c) {
-        uint32_t r0[32], r1[32];
+        uint32_t r0[32];
         ptx::tmem_ld_32x32b_x32(ta + static_cast<uint32_t>(c * 32), r0);
-        ptx::tmem_ld_32x32b_x32(ta + static_cast<uint32_t>(kWideNP + c * 32), r1);
         ptx::tmem_ld_wait();
         if (c == kWideNP / 32 - 1) {
           // the whole accumulator is in registers: the MMAs of a later unit may reuse it
@@ -645,7 +645,7 @@ router_logits_wide_kernel(const __grid_constant__ CUtensorMap tmX,
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          st[lane * kWidePitch + j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
+          st[lane * kWidePitch + j] = __uint_as_float(r0[j]);
         __syncwarp();
         // rows of the 32 x 32 block: 8 lanes per row, 4 rows per store
         const int col = (lane & 7) * 4;

@@ -268,17 +268,19 @@ def test_infinite_router_weight_reports_device_status(dtype, N):
     swl.forward(ig, spec.cf)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_router_decision_needs_float32_weights(dtype):
+@pytest.mark.parametrize("dtype,N", [("bf16", 8), ("f32", 8), ("bf16", 200)])
+def test_router_decision_needs_float32_weights(dtype, N):
     """The router works in float32 (selective precision).  Experts 0 and 1 have
     weights 1 + 2^-9 and 1 + 2^-9 + 2^-17: equal in bfloat16, and equal after
     the first two bf16 pieces of an fp32 split (the 2^-17 lives only in the third
     piece).  Their logits for x = c * ones(64) differ by c * 64 * 2^-17, about 64
     ulps of the logit, far above the worst-case fp32 accumulation error
     (64 * ulp/2), so a float32 router sends every token with c > 0 to expert 1,
-    while any router that drops the low piece ties them and takes expert 0."""
-    T, d, d_ff, N, cf = 256, 64, 64, 8, float(8)
-    spec = synth.LayerSpec("fp32_router_%s" % dtype, T, d, d_ff, N, cf, dtype)
+    while any router that drops the low piece ties them and takes expert 0.
+    N = 200 takes the wide tensor-core logits kernel (all pieces in one
+    accumulator) and the separate softmax."""
+    T, d, d_ff, cf = 256, 64, 64, float(8)
+    spec = synth.LayerSpec("fp32_router_%s_N%d" % (dtype, N), T, d, d_ff, N, cf, dtype)
     ic = synth.make_layer_inputs(spec, device="cpu")
     scale = torch.tensor([0.5, 1.0, 2.0, 4.0, -1.0])[torch.arange(T) % 5]
     ic["x"] = (scale[:, None] * torch.ones(T, d)).to(ic["x"].dtype)
@@ -376,7 +378,7 @@ def test_random_shapes_ffma_router(spec, ffma_router):
 
 
 def test_router_decision_needs_float32_weights_ffma(ffma_router):
-    test_router_decision_needs_float32_weights("bf16")
+    test_router_decision_needs_float32_weights("bf16", 8)
 
 
 # ------------------------------------------------------------------ failure path (bounded waits)
