@@ -218,6 +218,8 @@ dispatch_scan_kernel(const int* __restrict__ blk_count, const float* __restrict_
     __shared__ int s_tot_groups, s_tot_tiles2;
     for (int i = threadIdx.x; i < split.max_groups; i += kScanThreads)
       reinterpret_cast<int4*>(split.groups)[i] = make_int4(-1, 0, 0, 0);
+    for (int i = threadIdx.x; i < split.max_groups * kSplitFactor; i += kScanThreads)
+      split.ready[i] = 0;
     int groups = 0;
     for (int i = e0; i < e1; ++i) {
       const int m = min(__ldcg(exp_count + i), C_eff);
@@ -985,7 +987,7 @@ cudaError_t launch_dispatch_scan(const Shape& s, const Workspace& ws, float* aux
       static_cast<const int*>(s.topk == 2 ? ws.blk_count1 : nullptr),
       s.topk == 2 ? ws.exp_count1 : nullptr,
       SplitPlan{s.ffn_split, (int)((s.d + 127) / 128), kSplitMaxGroups, ws.tile_prefix2,
-                ws.split_base, ws.split_grp});
+                ws.split_base, ws.split_grp, ws.split_ready});
   count_launch();
   return e;
 }
@@ -1112,7 +1114,7 @@ static cudaError_t launch_scan_totals(const Shape& s, const Workspace& ws, const
       static_cast<float*>(nullptr), ws.hdr, s.nblk, (int)s.N, (int)s.T, (int)s.C_eff,
       s.tile_rows, static_cast<uint8_t*>(ws.ntlb_rec), (int)shard_record_psum_offset(s.N),
       static_cast<const int*>(nullptr), static_cast<int*>(nullptr),
-      SplitPlan{1, 1, 0, nullptr, nullptr, nullptr});
+      SplitPlan{1, 1, 0, nullptr, nullptr, nullptr, nullptr});
   count_launch();
   return e;
 }

@@ -105,6 +105,14 @@ struct FfnArgs {
   const int* tile_prefix2;     // [N+1] GEMM2 tile prefix counting split sub-tiles
   const int* split_base;       // [N] first split group of expert e, -1: not split
   float* part;                 // [groups][split][bn][128] fp32 partial tiles
+  // [kSplitMaxGroups][kSplitFactor]: per token tile of a split expert (its
+  // token tiles come first, so g < kSplitMaxGroups) and K chunk of GEMM2, the
+  // GEMM1 epilogue warps of the tiles whose features fall in that chunk that
+  // have stored their rows.  A split sub-tile waits for its own chunk only, and
+  // a split expert's tiles go chunk by chunk (GEMM1: its 128-feature tiles in
+  // `split` runs of consecutive tiles; GEMM2: k-chunk slowest), so the first
+  // chunks' GEMM2 work is ready while the last GEMM1 tiles run.
+  int* split_ready;
   // 1: within an expert, tiles go token tile by token tile (all m-tiles of
   // token tile 0 first), so that GEMM2 of the first token tiles can start
   // while GEMM1 of the last ones runs; 0: m-tile by m-tile (token tiles
@@ -130,6 +138,8 @@ struct TileSlot {
   int kb0, kb1;   // k-blocks [kb0, kb1) of this (sub-)tile
   int ks, nsplit; // GEMM2 split: sub-tile ks of nsplit
   int grp;        // split group (partials and counters), -1: not split
+  int* rdy0;      // GEMM1: the readiness counters its epilogue warps increment
+  int* rdy1;      //        (rdy1: a second K chunk of a split expert, or null)
 };
 
 constexpr int kTileRing = 8;    // decoded tiles handed to the producer, MMA and epilogue
@@ -161,7 +171,29 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const FfnArgs& a, int to
   const int local = tile - q0 * m_tiles;
   c.e = lo;
   c.nsplit = nts2 / nts;
-  if (a.tok_major) {
+  if (kSplit && c.phase == 1 && c.nsplit > 1) {
+    // split GEMM2 tiles: K chunk slowest, then the usual order within a chunk
+    const int per_ks = nts * m_tiles;
+    c.ks = local / per_ks;
+    const int r = local - c.ks * per_ks;
+    if (a.tok_major) {
+      c.nt = r / m_tiles;
+      c.mt = r - c.nt * m_tiles;
+    } else {
+      c.mt = r / nts;
+      c.nt = r - c.mt * nts;
+    }
+  } else if (kSplit && c.phase == 0 && __ldg(a.split_base + lo) >= 0) {
+    // GEMM1 tiles of a split expert: runs of mg consecutive feature tiles (one
+    // run per K chunk of GEMM2), the expert's token tiles within a run
+    const int mg = (m_tiles + a.split - 1) / a.split;
+    const int run = local / (nts * mg);
+    const int r = local - run * nts * mg;
+    const int mg_r = min(mg, m_tiles - run * mg);
+    c.nt = r / mg_r;
+    c.mt = run * mg + (r - c.nt * mg_r);
+    c.ks = 0;
+  } else if (a.tok_major) {
     const int per_nt = m_tiles * c.nsplit;   // the tiles of one token tile
     c.nt = local / per_nt;
     const int r = local - c.nt * per_nt;
@@ -301,6 +333,7 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         ts.kb0 = ts.kb1 = ts.ks = 0;
         ts.nsplit = 1;
         ts.grp = -1;
+        ts.rdy0 = ts.rdy1 = nullptr;
         if (ts.t >= 0) {
           const TileCoord c = decode_tile<kSplit>(ts.t, args, total0, P);
           ts.phase = c.phase;
@@ -323,14 +356,44 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
             ts.kb0 = 0;
             ts.kb1 = kbs;
           }
-          if (c.phase == 1) {
-            // hbuf rows of token tile g: every GEMM1 epilogue warp of g has stored them
-            const int target = kEpiWarps * args.ph[0].m_tiles + (args.stall_test && c.g == 0);
-            bool ready = ld_acquire(args.ready + c.g) >= target;
+          // K chunk of GEMM2 (features of hbuf) for the split experts' counters
+          const int kchunk = kSplit ? (args.ph[1].k_blocks + args.split - 1) / args.split * kBK : kBK;
+          if (c.phase == 0) {
+            ts.rdy0 = args.ready + c.g;
+            if (kSplit && __ldg(args.split_base + c.e) >= 0) {
+              // the chunks this tile's features [f0, f1] fall in
+              const int f0 = c.mt * kBM, f1 = min(args.ph[0].M, f0 + kBM) - 1;
+              const int c0 = f0 / kchunk, c1 = min(args.split - 1, f1 / kchunk);
+              if (!checked_index(c.g >= 0 && c.g < kSplitMaxGroups && c0 <= c1, args.err)) {
+                fail();
+                break;
+              }
+              ts.rdy0 = args.split_ready + c.g * kSplitFactor + c0;
+              ts.rdy1 = c1 != c0 ? args.split_ready + c.g * kSplitFactor + c1 : nullptr;
+            }
+          } else {
+            // hbuf rows of token tile g: every GEMM1 epilogue warp of g has stored
+            // them (of a split sub-tile: every warp of the GEMM1 tiles of its chunk)
+            const int* rp = args.ready + c.g;
+            int target = kEpiWarps * args.ph[0].m_tiles;
+            if (kSplit && c.nsplit > 1) {
+              const int f0 = c.ks * kchunk, f1 = min(args.ph[0].M, f0 + kchunk) - 1;
+              if (!checked_index(c.g >= 0 && c.g < kSplitMaxGroups && f0 <= f1, args.err)) {
+                fail();
+                break;
+              }
+              rp = args.split_ready + c.g * kSplitFactor + c.ks;
+              target = kEpiWarps * (f1 / kBM - f0 / kBM + 1);
+            }
+            target += args.stall_test && c.g == 0;
+            bool ready = ld_acquire(rp) >= target;
             const uint64_t t0 = ptx::globaltimer_ns();
             while (!ready) {
               if (*abort_flag || ptx::globaltimer_ns() - t0 > args.wait_ns) break;
-              ready = ld_acquire(args.ready + c.g) >= target;
+              // the counter lives in one L2 slice that many SMs may poll while
+              // the epilogue warps of the GEMM1 tiles update it: poll sparingly
+              __nanosleep(256);
+              ready = ld_acquire(rp) >= target;
             }
             if (!ready) {
               fail();
@@ -459,7 +522,8 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
     // GEMM1 tiles whose hbuf rows this warp stored but has not yet published:
     // one fence covers up to kMaxPending of them.  The warp publishes before it
     // could block, so a GEMM2 tile never waits on a warp that is itself waiting.
-    int pend0 = 0, pend1 = 0;   // token tiles of the unpublished GEMM1 tiles (warp-uniform)
+    // counters of the unpublished GEMM1 tiles (warp-uniform; b: a second chunk)
+    int *pend0a = nullptr, *pend0b = nullptr, *pend1a = nullptr, *pend1b = nullptr;
     int npending = 0;
     auto publish = [&]() {
       if (npending == 0) return;
@@ -467,8 +531,12 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
       __threadfence();
       __syncwarp();
       if (lane == 0) {
-        atomicAdd(args.ready + pend0, 1);
-        if (npending > 1) atomicAdd(args.ready + pend1, 1);
+        atomicAdd(pend0a, 1);
+        if (pend0b) atomicAdd(pend0b, 1);
+        if (npending > 1) {
+          atomicAdd(pend1a, 1);
+          if (pend1b) atomicAdd(pend1b, 1);
+        }
       }
       npending = 0;
     };
@@ -585,15 +653,20 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         }
         if (!stored) {
           ptx::tmem_ld_wait();
+          const bool relu = P.mode == 0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float v = __uint_as_float(r[j]) + bias;
-            if (P.mode == 0) {
-              v = fmaxf(v, 0.f);
+          for (int j = 0; j < 32; j += 2) {   // two tokens per conversion
+            float v0 = __uint_as_float(r[j]) + bias, v1 = __uint_as_float(r[j + 1]) + bias;
+            if (relu) {
+              v0 = fmaxf(v0, 0.f);
+              v1 = fmaxf(v1, 0.f);
             } else {
-              v *= __shfl_sync(0xffffffffu, g, j);
+              v0 *= __shfl_sync(0xffffffffu, g, j);
+              v1 *= __shfl_sync(0xffffffffu, g, j + 1);
             }
-            st[j * 32 + lane] = __float2bfloat16_rn(v);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+            st[j * 32 + lane] = h2.x;
+            st[(j + 1) * 32 + lane] = h2.y;
           }
         }
         __syncwarp();
@@ -616,7 +689,13 @@ expert_ffn_sm100_kernel(const __grid_constant__ CUtensorMap tmA0,
         ptx::mbar_arrive(&tile_empty[slot]);
       }
       if (ts.phase == 0) {
-        if (npending == 0) pend0 = ts.g; else pend1 = ts.g;
+        if (npending == 0) {
+          pend0a = ts.rdy0;
+          pend0b = ts.rdy1;
+        } else {
+          pend1a = ts.rdy0;
+          pend1b = ts.rdy1;
+        }
         if (++npending == kMaxPending) publish();
       }
       if (++acc == args.num_acc) { acc = 0; aph ^= 1u; }
@@ -725,6 +804,7 @@ cudaError_t launch_expert_ffn_bf16(const Shape& s, const Workspace& ws, const CU
   a.tile_prefix2 = ws.tile_prefix2;
   a.split_base = ws.split_base;
   a.part = ws.part;
+  a.split_ready = ws.split_ready;
   // token-tile order within an expert when its weights sit in L2 anyway
   a.tok_major = s.d * s.d_ff * 2 * (s.glu ? 2 : 1) <= (int64_t{32} << 20) ? 1 : 0;
   a.wait_ns = wait_limit_ns();

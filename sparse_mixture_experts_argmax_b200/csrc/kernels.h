@@ -52,6 +52,8 @@ struct Workspace {
   float* part;          // GEMM2 split: [kSplitMaxGroups][split][tile_rows][128] fp32
   int* split_grp;       // GEMM2 split: [kSplitMaxGroups][4] (expert, m-tile, token tile,
                         // 0) of each group, expert -1 past the last group
+  int* split_ready;     // GEMM2 split: [kSplitMaxGroups][kSplitFactor] per split token tile
+                        // and K chunk: GEMM1 epilogue warps done (zeroed by the scan)
   void* w3;             // tensor-core router: [3N, d] bf16 pieces hi, mid, lo of W_r
   float* xj;            // jittered router input x * noise [T, d] fp32 (jitter on the FFMA router)
   void* x3;             // jittered router input as three bf16 pieces [3T, d] (xsplit)
@@ -169,6 +171,7 @@ struct SplitPlan {
   int* tile_prefix2;
   int* split_base;
   int* groups;       // [max_groups][4]
+  int* ready;        // [max_groups][kSplitFactor] chunk readiness counters, zeroed here
 };
 // record != nullptr: a shard of a global batch; the expert totals go to the
 // exchange record and the expert-level part waits for launch_shard_combine.

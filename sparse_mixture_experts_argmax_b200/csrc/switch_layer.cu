@@ -76,6 +76,8 @@ size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace*
   w.part = reinterpret_cast<float*>(
       take(split ? static_cast<size_t>(kSplitMaxGroups) * s.ffn_split * 128 * s.tile_rows * 4 : 0));
   w.split_grp = reinterpret_cast<int*>(take(split ? static_cast<size_t>(kSplitMaxGroups) * 16 : 0));
+  w.split_ready = reinterpret_cast<int*>(
+      take(split ? static_cast<size_t>(kSplitMaxGroups) * kSplitFactor * 4 : 0));
   w.w3 = reinterpret_cast<void*>(
       take(s.router_path == kRouterTC || s.router_path == kRouterTCWide
                ? 3 * N * static_cast<size_t>(s.d) * 2
