@@ -310,6 +310,7 @@ def test_router_decision_needs_float32_weights(dtype, N):
 #   fp32 N = 48, ~100 big router tiles: FFMA tile router, fused dispatch
 #   fp32 N = 8, x > 16 MiB: warp-split router, two-kernel dispatch (scan + gather)
 #   bf16 N = 4, capacity > 128 rows: two 256-column TMEM accumulators
+#   bf16 x > 48 MiB, cf = 0.25: two-kernel dispatch, most tokens dropped
 _VARIANT_SHAPES = [
     ("tc_np96_s4", 1000, 1024, 256, 80, 1.25, "bf16"),
     ("tc_np128_s2", 2000, 256, 128, 128, 1.25, "bf16"),
@@ -326,6 +327,9 @@ _VARIANT_SHAPES = [
     # with a ragged second half (N = 1500); token blocks of 45 and 37 tokens
     ("stream_full_warp_row", 6600, 128, 64, 1024, 2.0, "bf16"),
     ("stream_pair_ragged", 5400, 128, 64, 1500, 2.0, "bf16"),
+    # x above 48 MiB with most tokens dropped: the gather reads only the kept
+    # tokens' rows (no early row loads) and zeroes the dropped tokens' rows
+    ("gather_mostly_dropped", 25000, 1024, 64, 16, 0.25, "bf16"),
 ]
 
 
