@@ -18,7 +18,8 @@
 //
 // Kernels:
 //   bwd_gate_kernel     per token: dg (fp32), the packed row du = g dout, f counts
-//   bwd_router_kernel   per token: logits, softmax, dz (fp32, [T, N])
+//   bwd_logits_kernel   z = x W_r^T + b_r (fp32, [T, N]): tiles of 128 tokens x 64 experts
+//   bwd_dz_kernel       per token (a warp): softmax of z, dz in place of z
 //   grouped_gemm_kernel SIMT tiles with fp32 accumulation over packed row
 //                       groups (one group per expert), two forms:
 //                       WGRAD  C[g] = sum over the group's rows of A_r^T B_r
@@ -75,80 +76,6 @@ bwd_gate_kernel(const TA* __restrict__ dout, const TA* __restrict__ out,
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) dg[t] = acc / g;
-}
-
-// Router gradient, one CTA per token: z = W_r x_t + b_r (fp32), p = softmax(z),
-// dz_j = kg (delta_{j e} - p_j) + daux (N / T) p_j (f_j - sum_i f_i p_i) with
-// kg = dg_t g_t (0 for a dropped token), f_j = counts_j / T.  Shared scratch: N floats.
-template <typename TA>
-__global__ void __launch_bounds__(kBwdThreads)
-bwd_router_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
-                  const float* __restrict__ b_r, const int* __restrict__ expert_idx,
-                  const float* __restrict__ gate, const float* __restrict__ dg,
-                  const int* __restrict__ counts, int T, int d, int N, float daux,
-                  float* __restrict__ dz) {
-  extern __shared__ float sz[];   // [N] logits, then p
-  __shared__ float red[kBwdWarps];
-  __shared__ float s_bcast;
-  const int t = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const TA* xt = x + static_cast<size_t>(t) * d;
-  // logits: one warp per expert row of W_r
-  for (int n = warp; n < N; n += kBwdWarps) {
-    const float* w = W_r + static_cast<size_t>(n) * d;
-    float acc = 0.f;
-    for (int k = lane; k < d; k += 32) acc = fmaf(ld(xt + k), w[k], acc);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) sz[n] = acc + (b_r ? b_r[n] : 0.f);
-  }
-  __syncthreads();
-  auto block_reduce = [&](float v, bool is_max) -> float {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float o = __shfl_xor_sync(0xffffffffu, v, off);
-      v = is_max ? fmaxf(v, o) : v + o;
-    }
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float r = red[0];
-      for (int w = 1; w < kBwdWarps; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
-      s_bcast = r;
-    }
-    __syncthreads();
-    const float r = s_bcast;
-    __syncthreads();
-    return r;
-  };
-  float m = -INFINITY;
-  for (int n = threadIdx.x; n < N; n += kBwdThreads) m = fmaxf(m, sz[n]);
-  m = block_reduce(m, true);
-  float s = 0.f;
-  for (int n = threadIdx.x; n < N; n += kBwdThreads) {
-    const float e = expf(sz[n] - m);
-    sz[n] = e;
-    s += e;
-  }
-  s = block_reduce(s, false);
-  const float inv = 1.0f / s;
-  const float invT = 1.0f / static_cast<float>(T);
-  float fp = 0.f;   // sum_i f_i p_i
-  for (int n = threadIdx.x; n < N; n += kBwdThreads) {
-    const float p = sz[n] * inv;
-    sz[n] = p;
-    fp += static_cast<float>(counts[n]) * invT * p;
-  }
-  fp = block_reduce(fp, false);
-  const int e = expert_idx[t];
-  const float kg = dg[t] * gate[t];
-  const float ca = daux * static_cast<float>(N) * invT;
-  float* dzt = dz + static_cast<size_t>(t) * N;
-  for (int n = threadIdx.x; n < N; n += kBwdThreads) {
-    const float p = sz[n];
-    const float f = static_cast<float>(counts[n]) * invT;
-    dzt[n] = kg * ((n == e ? 1.f : 0.f) - p) + ca * p * (f - fp);
-  }
 }
 
 // Tiled SIMT GEMM over groups of packed rows, fp32 accumulation.  64 x 64
@@ -301,14 +228,144 @@ grouped_gemm_kernel(const TAin* __restrict__ A, const TBin* __restrict__ B, TC* 
   }
 }
 
-// bf16 form of grouped_gemm_kernel on the tensor cores: mma.sync m16n8k16 with
-// fp32 accumulation, 128 x 128 outputs per CTA, 8 warps of 64 x 32, K in steps
-// of 32 staged by cp.async into two shared-memory buffers, fragments by
-// ldmatrix (transposed where the contraction runs along a tile's rows).  Same
-// groups, grids (with 128-row tiles) and epilogues as the SIMT kernel.
-//   WGRAD: the contraction runs over the group's rows for both operands, so A
-//     is staged [k][m] and B [k][n] and both are read transposed.
-//   DGRAD: A is staged [r][k] (read as is), W[g] [k][n] (read transposed).
+// Router logits for the backward, z = x W_r^T + b_r in fp32 ([T, N], written to
+// dz and turned into dz by bwd_dz_kernel): 128 tokens x 64 experts per CTA,
+// 256 threads with 8 tokens x 4 experts each, K in steps of 16 through shared
+// memory (both tiles k-major, read as 16-byte vectors), so W_r is read once per
+// token tile.  vec: d % 4 == 0 with 16-byte aligned W_r and 4-element aligned x
+// rows, then each thread loads 4 consecutive k of a token row and of an expert
+// row at once; else element by element.
+constexpr int kLT = 128, kLN = 64, kLK = 16;
+template <typename TA>
+__global__ void __launch_bounds__(256)
+bwd_logits_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
+                  const float* __restrict__ b_r, int T, int d, int N, int vec,
+                  float* __restrict__ z) {
+  __shared__ __align__(16) float As[kLK][kLT + 4];   // [k][token]
+  __shared__ __align__(16) float Bs[kLK][kLN + 4];   // [k][expert]
+  const int tid = threadIdx.x;
+  const int tn = tid % 16, tt = tid / 16;           // experts 4 tn.., tokens 8 tt..
+  const int n0 = blockIdx.x * kLN, t0 = blockIdx.y * kLT;
+  float acc[8][4] = {};
+  for (int k0 = 0; k0 < d; k0 += kLK) {
+    if (vec) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {                  // 128 rows x 4 quads of x
+        const int q = tid + h * 256, r = q / 4, kq = (q % 4) * 4;
+        float xa[4] = {0.f, 0.f, 0.f, 0.f};
+        if (t0 + r < T && k0 + kq < d) {
+          const TA* src = x + static_cast<size_t>(t0 + r) * d + k0 + kq;
+          if constexpr (std::is_same<TA, float>::value) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            xa[0] = v.x; xa[1] = v.y; xa[2] = v.z; xa[3] = v.w;
+          } else {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+            xa[0] = __low2float(lo); xa[1] = __high2float(lo);
+            xa[2] = __low2float(hi); xa[3] = __high2float(hi);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) As[kq + c][r] = xa[c];
+      }
+      {                                              // 64 rows x 4 quads of W_r
+        const int r = tid / 4, kq = (tid % 4) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n0 + r < N && k0 + kq < d)
+          v = *reinterpret_cast<const float4*>(W_r + static_cast<size_t>(n0 + r) * d + k0 + kq);
+        Bs[kq][r] = v.x;
+        Bs[kq + 1][r] = v.y;
+        Bs[kq + 2][r] = v.z;
+        Bs[kq + 3][r] = v.w;
+      }
+    } else {
+      for (int i = tid; i < kLK * kLT; i += 256) {
+        const int kk = i % kLK, r = i / kLK;
+        As[kk][r] = (t0 + r < T && k0 + kk < d) ? ld(x + static_cast<size_t>(t0 + r) * d + k0 + kk)
+                                                : 0.f;
+      }
+      for (int i = tid; i < kLK * kLN; i += 256) {
+        const int kk = i % kLK, r = i / kLK;
+        Bs[kk][r] = (n0 + r < N && k0 + kk < d) ? W_r[static_cast<size_t>(n0 + r) * d + k0 + kk]
+                                                : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kLK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][tt * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][tt * 8 + 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tn * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + tt * 8 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tn * 4 + j;
+      if (n < N) z[static_cast<size_t>(t) * N + n] = acc[i][j] + (b_r ? b_r[n] : 0.f);
+    }
+  }
+}
+
+// Router gradient, a warp per token, in place of the logits row z_t:
+// p = softmax(z_t), dz_t,j = kg (delta_{j e} - p_j) + daux (N / T) p_j (f_j -
+// sum_i f_i p_i) with kg = dg_t g_t (0 for a dropped token), f_j = counts_j / T.
+// Three passes over the row: max, then the sums of exp and of f exp, then dz.
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_dz_kernel(const int* __restrict__ expert_idx, const float* __restrict__ gate,
+              const float* __restrict__ dg, const int* __restrict__ counts, int T, int N,
+              float daux, float* __restrict__ dz) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kBwdWarps + warp;
+  if (t >= T) return;
+  float* zt = dz + static_cast<size_t>(t) * N;
+  const float invT = 1.0f / static_cast<float>(T);
+  float m = -INFINITY;
+  for (int n = lane; n < N; n += 32) m = fmaxf(m, zt[n]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float s = 0.f, sf = 0.f;
+  for (int n = lane; n < N; n += 32) {
+    const float e = expf(zt[n] - m);
+    s += e;
+    sf += static_cast<float>(counts[n]) * invT * e;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, off);
+    sf += __shfl_xor_sync(0xffffffffu, sf, off);
+  }
+  const float inv = 1.0f / s;
+  const float fp = sf * inv;   // sum_i f_i p_i
+  const int e = expert_idx[t];
+  const float kg = dg[t] * gate[t];
+  const float ca = daux * static_cast<float>(N) * invT;
+  for (int n = lane; n < N; n += 32) {
+    const float p = expf(zt[n] - m) * inv;
+    const float f = static_cast<float>(counts[n]) * invT;
+    zt[n] = kg * ((n == e ? 1.f : 0.f) - p) + ca * p * (f - fp);
+  }
+}
+
+// bf16 DGRAD form of grouped_gemm_kernel on the tensor cores: mma.sync
+// m16n8k16 with fp32 accumulation, 128 x 128 outputs per CTA, 8 warps of 64 x
+// 32, K in steps of 32 staged by cp.async into two shared-memory buffers,
+// fragments by ldmatrix.  Same row-tile list, grid (with 128-row tiles) and
+// epilogues as the SIMT kernel's DGRAD: A is staged [r][k] (read as is), W[g]
+// [k][n] (read transposed).  The bf16 WGRAD form is grouped_wgrad_mma_kernel
+// below: there the contraction runs over the group's rows for both operands,
+// staged [k][m] and [k][n] and both read transposed.
 constexpr int kMT = 128, kMK = 32, kMPad = 8;
 constexpr int kMStride = kMT + kMPad;      // [k][128] tiles: row stride in elements
 constexpr int kMStrideK = kMK + kMPad;     // [128][k] tile: row stride in elements
@@ -347,10 +404,9 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <bool kWgrad>
 __global__ void __launch_bounds__(256)
 grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
-                        __nv_bfloat16* __restrict__ C, int P, int Q, int K,
+                        __nv_bfloat16* __restrict__ C, int Q, int K,
                         const int* __restrict__ base, const int* __restrict__ rows, int rows0,
                         const int* __restrict__ tile_prefix, int groups, int epi,
                         const __nv_bfloat16* __restrict__ mask, const int* __restrict__ dst_row,
@@ -360,21 +416,8 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp >> 2, wn = warp & 3;        // 2 x 4 warps of 64 x 32 outputs
   const int n0 = blockIdx.x * kMT;
-  int g, r0, nr, m0 = 0, kdim;
-  if (kWgrad) {
-    g = blockIdx.z;
-    r0 = base ? base[g] : 0;
-    nr = rows ? rows[g] : rows0;
-    m0 = blockIdx.y * kMT;
-    kdim = nr;
-    if (nr == 0) {      // an expert with no kept rows has a zero gradient
-      for (int i = tid; i < kMT * kMT; i += 256) {
-        const int mm = m0 + i / kMT, nn = n0 + i % kMT;
-        if (mm < P && nn < Q) C[(static_cast<size_t>(g) * P + mm) * Q + nn] = __float2bfloat16(0.f);
-      }
-      return;
-    }
-  } else {
+  int g, r0, nr;
+  {
     const int tile = blockIdx.y;
     if (tile_prefix) {
       if (tile >= tile_prefix[groups]) return;
@@ -393,32 +436,22 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
       nr = min(kMT, rows0 - r0);
       if (nr <= 0) return;
     }
-    kdim = K;
   }
-  const __nv_bfloat16* W = kWgrad ? B : B + static_cast<size_t>(g) * K * Q;
+  const __nv_bfloat16* W = B + static_cast<size_t>(g) * K * Q;
 
   // stage one K step of 32 into buffer s (every thread: 2 chunks of A, 2 of B)
   auto load = [&](int s, int k0) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c = tid + h * 256;
-      if (kWgrad) {
-        const int k = c >> 4, mc = (c & 15) * 8;   // A[r0 + k0 + k][m0 + mc ...]
-        const bool ok = k0 + k < nr && m0 + mc < P;
-        cp_async16(&sA[s][k * kMStride + mc],
-                   ok ? A + static_cast<size_t>(r0 + k0 + k) * P + m0 + mc : A, ok);
-      } else {
-        const int r = c >> 2, kc = (c & 3) * 8;    // A[r0 + r][k0 + kc ...]
-        const bool ok = r < nr && k0 + kc < K;
-        cp_async16(&sA[s][r * kMStrideK + kc],
-                   ok ? A + static_cast<size_t>(r0 + r) * K + k0 + kc : A, ok);
-      }
-      const int k = c >> 4, nc = (c & 15) * 8;
-      const bool okb = k0 + k < kdim && n0 + nc < Q;
-      const __nv_bfloat16* src =
-          kWgrad ? B + static_cast<size_t>(r0 + k0 + k) * Q + n0 + nc
-                 : W + static_cast<size_t>(k0 + k) * Q + n0 + nc;
-      cp_async16(&sB[s][k * kMStride + nc], okb ? src : B, okb);
+      const int r = c >> 2, kc = (c & 3) * 8;    // A[r0 + r][k0 + kc ...]
+      const bool ok = r < nr && k0 + kc < K;
+      cp_async16(&sA[s][r * kMStrideK + kc],
+                 ok ? A + static_cast<size_t>(r0 + r) * K + k0 + kc : A, ok);
+      const int k = c >> 4, nc = (c & 15) * 8;    // W[g][k0 + k][n0 + nc ...]
+      const bool okb = k0 + k < K && n0 + nc < Q;
+      cp_async16(&sB[s][k * kMStride + nc],
+                 okb ? W + static_cast<size_t>(k0 + k) * Q + n0 + nc : B, okb);
     }
     cp_async_commit();
   };
@@ -431,7 +464,7 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
 
-  const int nk = (kdim + kMK - 1) / kMK;
+  const int nk = (K + kMK - 1) / kMK;
   load(0, 0);
   for (int kt = 0; kt < nk; ++kt) {
     const int s = kt & 1;
@@ -448,12 +481,8 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
       const int jm = lane >> 3, rr = lane & 7;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int mb = wm * 64 + i * 16;
-        if (kWgrad) {   // staged [k][m]: matrices (m, k) blocks at rows k, read transposed
-          ldsm_x4_t(af[i], &sA[s][(kk + rr + (jm >> 1) * 8) * kMStride + mb + (jm & 1) * 8]);
-        } else {        // staged [r][k]
-          ldsm_x4(af[i], &sA[s][(mb + (lane & 15)) * kMStrideK + kk + (lane >> 4) * 8]);
-        }
+        const int mb = wm * 64 + i * 16;   // staged [r][k]
+        ldsm_x4(af[i], &sA[s][(mb + (lane & 15)) * kMStrideK + kk + (lane >> 4) * 8]);
       }
 #pragma unroll
       for (int j2 = 0; j2 < 2; ++j2) {   // two n-fragments of 8 per ldmatrix
@@ -485,30 +514,201 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
         const int nn = n0 + wn * 32 + j * 8 + (lane & 3) * 2;
         if (nn >= Q) continue;
         const float v0 = acc[i][j][2 * hh], v1 = acc[i][j][2 * hh + 1];
-        if (kWgrad) {
-          const int mm = m0 + rl;
-          if (mm < P)
-            *reinterpret_cast<__nv_bfloat162*>(C + (static_cast<size_t>(g) * P + mm) * Q + nn) =
-                __floats2bfloat162_rn(v0, v1);
+        if (rl >= nr) continue;
+        const int r = r0 + rl;
+        const size_t o = static_cast<size_t>(r) * Q + nn;
+        if (epi == 0) {
+          *reinterpret_cast<__nv_bfloat162*>(C + o) = __floats2bfloat162_rn(v0, v1);
+        } else if (epi == 1) {
+          const __nv_bfloat162 mk = *reinterpret_cast<const __nv_bfloat162*>(mask + o);
+          *reinterpret_cast<__nv_bfloat162*>(C + o) = __floats2bfloat162_rn(
+              __bfloat162float(mk.x) > 0.f ? v0 : 0.f, __bfloat162float(mk.y) > 0.f ? v1 : 0.f);
         } else {
-          if (rl >= nr) continue;
-          const int r = r0 + rl;
-          const size_t o = static_cast<size_t>(r) * Q + nn;
-          if (epi == 0) {
-            *reinterpret_cast<__nv_bfloat162*>(C + o) = __floats2bfloat162_rn(v0, v1);
-          } else if (epi == 1) {
-            const __nv_bfloat162 mk = *reinterpret_cast<const __nv_bfloat162*>(mask + o);
-            *reinterpret_cast<__nv_bfloat162*>(C + o) = __floats2bfloat162_rn(
-                __bfloat162float(mk.x) > 0.f ? v0 : 0.f, __bfloat162float(mk.y) > 0.f ? v1 : 0.f);
-          } else {
-            const int t = dst_row ? dst_row[r] : r;
-            float* d = acc_out + static_cast<size_t>(t) * Q + nn;
-            d[0] += v0;
-            d[1] += v1;
-          }
+          const int t = dst_row ? dst_row[r] : r;
+          float* d = acc_out + static_cast<size_t>(t) * Q + nn;
+          d[0] += v0;
+          d[1] += v1;
         }
       }
     }
+  }
+}
+
+// Expert weight gradients on the tensor cores, persistent: C[g] = A[rows of
+// g]^T B[rows of g] ([P, Q] per expert, bf16 inputs, fp32 accumulation, bf16
+// out).  CTA b takes output tiles b, b + gridDim.x, ... of the groups x
+// ceil(P/128) x ceil(Q/128) tiles (group-major, then m-tile, then n-tile, so
+// the CTAs running together share a group's rows in L2, and a group with many
+// rows spreads over every CTA).  A group without rows has a zero gradient: its
+// tiles are plain zero stores.  Per tile the same 8 warps of 64 x 32 outputs
+// as grouped_gemm_mma_kernel, K (the group's rows) in steps of 32 through two
+// cp.async stages; the next tile's first K step is requested before this
+// tile's epilogue, which stages the tile in shared memory and writes whole
+// 16-byte row pieces.
+constexpr int kWgStride = kMT + kMPad;       // epilogue staging row stride (elements)
+constexpr size_t kWgSmem =
+    (4 * static_cast<size_t>(kMK) * kMStride + static_cast<size_t>(kMT) * kWgStride) * 2 + 128;
+
+__global__ void __launch_bounds__(256)
+grouped_wgrad_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
+                         __nv_bfloat16* __restrict__ C, int P, int Q,
+                         const int* __restrict__ base, const int* __restrict__ rows, int groups) {
+  extern __shared__ uint8_t wg_raw[];
+  __nv_bfloat16* smem = reinterpret_cast<__nv_bfloat16*>(
+      (reinterpret_cast<uintptr_t>(wg_raw) + 127) & ~static_cast<uintptr_t>(127));
+  __nv_bfloat16* sA = smem;                              // [2][kMK][kMStride]  A rows [k][m]
+  __nv_bfloat16* sB = sA + 2 * kMK * kMStride;           // [2][kMK][kMStride]  B rows [k][n]
+  __nv_bfloat16* sE = sB + 2 * kMK * kMStride;           // [kMT][kWgStride]    output tile
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp >> 2, wn = warp & 3;
+  const int mtP = (P + kMT - 1) / kMT, mtQ = (Q + kMT - 1) / kMT;
+  const int total = groups * mtP * mtQ;
+  // 16-byte row pieces when every row of C starts 16-byte aligned
+  const bool vec = (Q % 8) == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0;
+  struct Tile { int g, m0, n0, r0, nr; };
+  auto decode = [&](int t) {
+    Tile c;
+    c.g = t / (mtP * mtQ);
+    const int rem = t - c.g * mtP * mtQ;
+    c.m0 = (rem / mtQ) * kMT;
+    c.n0 = (rem % mtQ) * kMT;
+    c.r0 = base[c.g];
+    c.nr = rows[c.g];
+    return c;
+  };
+  // K step k0 of tile c into stage s (every thread: 2 chunks of A, 2 of B)
+  auto load = [&](int s, int k0, const Tile& c) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = tid + h * 256;
+      const int k = i >> 4, col = (i & 15) * 8;
+      const bool oka = k0 + k < c.nr && c.m0 + col < P;
+      cp_async16(&sA[(s * kMK + k) * kMStride + col],
+                 oka ? A + static_cast<size_t>(c.r0 + k0 + k) * P + c.m0 + col : A, oka);
+      const bool okb = k0 + k < c.nr && c.n0 + col < Q;
+      cp_async16(&sB[(s * kMK + k) * kMStride + col],
+                 okb ? B + static_cast<size_t>(c.r0 + k0 + k) * Q + c.n0 + col : B, okb);
+    }
+    cp_async_commit();
+  };
+  int t = blockIdx.x;
+  if (t >= total) return;
+  Tile cur = decode(t);
+  bool pre = false;          // the current tile's first K step is already requested
+  while (true) {
+    __nv_bfloat16* Cg = C + static_cast<size_t>(cur.g) * P * Q;
+    if (cur.nr == 0) {
+      if (vec) {
+        for (int i = tid; i < kMT * (kMT / 8); i += 256) {
+          const int rr = cur.m0 + i / (kMT / 8), cc = cur.n0 + (i % (kMT / 8)) * 8;
+          if (rr < P && cc < Q)
+            *reinterpret_cast<uint4*>(Cg + static_cast<size_t>(rr) * Q + cc) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+      } else {
+        for (int i = tid; i < kMT * kMT; i += 256) {
+          const int rr = cur.m0 + i / kMT, cc = cur.n0 + i % kMT;
+          if (rr < P && cc < Q) Cg[static_cast<size_t>(rr) * Q + cc] = __float2bfloat16(0.f);
+        }
+      }
+      t += gridDim.x;
+      if (t >= total) break;
+      cur = decode(t);
+      pre = false;
+      continue;
+    }
+    if (!pre) load(0, 0, cur);
+    float acc[4][4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
+    const int nk = (cur.nr + kMK - 1) / kMK;
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt & 1;
+      if (kt + 1 < nk) {
+        load(s ^ 1, (kt + 1) * kMK, cur);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const __nv_bfloat16* a_s = sA + s * kMK * kMStride;
+      const __nv_bfloat16* b_s = sB + s * kMK * kMStride;
+#pragma unroll
+      for (int kk = 0; kk < kMK; kk += 16) {
+        uint32_t af[4][4], bf[4][2];
+        const int jm = lane >> 3, rr = lane & 7;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {   // staged [k][m]: (m, k) blocks read transposed
+          const int mb = wm * 64 + i * 16;
+          ldsm_x4_t(af[i], &a_s[(kk + rr + (jm >> 1) * 8) * kMStride + mb + (jm & 1) * 8]);
+        }
+#pragma unroll
+        for (int j2 = 0; j2 < 2; ++j2) {
+          const int nb = wn * 32 + j2 * 16;
+          uint32_t t4[4];
+          ldsm_x4_t(t4, &b_s[(kk + rr + (jm & 1) * 8) * kMStride + nb + (jm >> 1) * 8]);
+          bf[2 * j2][0] = t4[0];
+          bf[2 * j2][1] = t4[1];
+          bf[2 * j2 + 1][0] = t4[2];
+          bf[2 * j2 + 1][1] = t4[3];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma_bf16(acc[i][j], af[i], bf[j][0], bf[j][1]);
+      }
+      __syncthreads();
+    }
+    // every warp is past its last shared-memory read of the stages: the next
+    // tile's first K step goes into stage 0 under this tile's epilogue
+    const int tn = t + static_cast<int>(gridDim.x);
+    Tile nxt = cur;
+    pre = false;
+    if (tn < total) {
+      nxt = decode(tn);
+      if (nxt.nr > 0) {
+        load(0, 0, nxt);
+        pre = true;
+      }
+    }
+    // accumulator (i, j, c) -> row wm*64 + i*16 + lane/4 (+8 for c >= 2), column
+    // wn*32 + j*8 + (lane%4)*2 (+1 for odd c), staged as bf16
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rl = wm * 64 + i * 16 + (lane >> 2) + hh * 8;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int cl = wn * 32 + j * 8 + (lane & 3) * 2;
+          *reinterpret_cast<__nv_bfloat162*>(&sE[rl * kWgStride + cl]) =
+              __floats2bfloat162_rn(acc[i][j][2 * hh], acc[i][j][2 * hh + 1]);
+        }
+      }
+    __syncthreads();
+    if (vec) {
+      for (int i = tid; i < kMT * (kMT / 8); i += 256) {
+        const int rl = i / (kMT / 8), cl = (i % (kMT / 8)) * 8;
+        const int rr = cur.m0 + rl, cc = cur.n0 + cl;
+        if (rr < P && cc < Q)
+          *reinterpret_cast<uint4*>(Cg + static_cast<size_t>(rr) * Q + cc) =
+              *reinterpret_cast<const uint4*>(&sE[rl * kWgStride + cl]);
+      }
+    } else {
+      for (int i = tid; i < kMT * kMT; i += 256) {
+        const int rl = i / kMT, cl = i % kMT;
+        const int rr = cur.m0 + rl, cc = cur.n0 + cl;
+        if (rr < P && cc < Q) Cg[static_cast<size_t>(rr) * Q + cc] = sE[rl * kWgStride + cl];
+      }
+    }
+    __syncthreads();   // sE is free for the next tile
+    if (tn >= total) break;
+    t = tn;
+    cur = nxt;
   }
 }
 
@@ -606,17 +806,18 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
       a.pos_in_expert, fw.exp_base, T, d, static_cast<int>(s.C_cmp), bw.dg,
       static_cast<TA*>(bw.du), bw.counts);
   ++launches;
-  // router: dz [T, N]
-  const size_t rsmem = static_cast<size_t>(N) * 4;
-  if (rsmem > 48 * 1024) {
-    if ((e = cudaFuncSetAttribute(bwd_router_kernel<TA>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(rsmem))) != cudaSuccess)
-      return e;
+  // router: logits z [T, N] into dz, then dz in place
+  {
+    const int vec = (d % 4 == 0 && (reinterpret_cast<uintptr_t>(a.W_r) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(x) & (4 * sizeof(TA) - 1)) == 0)
+                        ? 1
+                        : 0;
+    bwd_logits_kernel<TA><<<dim3((N + kLN - 1) / kLN, (T + kLT - 1) / kLT), kBwdThreads, 0,
+                            stream>>>(x, a.W_r, a.b_r, T, d, N, vec, bw.dz);
+    bwd_dz_kernel<<<(T + kBwdWarps - 1) / kBwdWarps, kBwdThreads, 0, stream>>>(
+        a.expert_idx, a.gate, bw.dg, bw.counts, T, N, a.daux, bw.dz);
+    launches += 2;
   }
-  bwd_router_kernel<TA><<<T, kBwdThreads, rsmem, stream>>>(
-      x, a.W_r, a.b_r, a.expert_idx, a.gate, bw.dg, bw.counts, T, d, N, a.daux, bw.dz);
-  ++launches;
   const dim3 blk(256);
   auto tiles = [](int v) { return static_cast<unsigned>((v + kGT - 1) / kGT); };
   // db[g][m] = sum over the group's rows of A[r][m]: split partials, then their sum
@@ -642,26 +843,37 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(fw.xbuf);
     __nv_bfloat16* da = static_cast<__nv_bfloat16*>(bw.da);
     // dW2[e] = du^T h, db2[e] = sum du
-    grouped_gemm_mma_kernel<true><<<dim3(mt(d_ff), mt(d), N), blk, 0, stream>>>(
-        du, hb, static_cast<__nv_bfloat16*>(a.dW2), d, d_ff, 0, fw.exp_base, fw.exp_rows, 0,
-        nullptr, N, 0, nullptr, nullptr, nullptr);
+    if ((e = cudaFuncSetAttribute(grouped_wgrad_mma_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kWgSmem))) != cudaSuccess)
+      return e;
+    int sms = 0, dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    // persistent: two CTAs per SM (registers), or fewer when the tiles are fewer
+    auto wg_grid = [&](int P, int Q) {
+      const long long tiles = static_cast<long long>(N) * mt(P) * mt(Q);
+      return static_cast<unsigned>(tiles < 2LL * sms ? tiles : 2LL * sms);
+    };
+    grouped_wgrad_mma_kernel<<<wg_grid(d, d_ff), blk, kWgSmem, stream>>>(
+        du, hb, static_cast<__nv_bfloat16*>(a.dW2), d, d_ff, fw.exp_base, fw.exp_rows, N);
     colsum(static_cast<const TA*>(bw.du), d, fw.exp_base, fw.exp_rows, 0, N, C_rows,
            static_cast<TA*>(a.db2));
     // da = (du W2[e]) * [h > 0]
     bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, kMT, bw.tile_prefix);
     const unsigned row_tiles = static_cast<unsigned>((T + kMT - 1) / kMT + N);
-    grouped_gemm_mma_kernel<false><<<dim3(mt(d_ff), row_tiles, 1), blk, 0, stream>>>(
-        du, static_cast<const __nv_bfloat16*>(a.W2), da, 0, d_ff, d, fw.exp_base, fw.exp_rows, 0,
+    grouped_gemm_mma_kernel<<<dim3(mt(d_ff), row_tiles, 1), blk, 0, stream>>>(
+        du, static_cast<const __nv_bfloat16*>(a.W2), da, d_ff, d, fw.exp_base, fw.exp_rows, 0,
         bw.tile_prefix, N, 1, hb, nullptr, nullptr);
     // dW1[e] = da^T x, db1[e] = sum da
-    grouped_gemm_mma_kernel<true><<<dim3(mt(d), mt(d_ff), N), blk, 0, stream>>>(
-        da, xb, static_cast<__nv_bfloat16*>(a.dW1), d_ff, d, 0, fw.exp_base, fw.exp_rows, 0,
-        nullptr, N, 0, nullptr, nullptr, nullptr);
+    grouped_wgrad_mma_kernel<<<wg_grid(d_ff, d), blk, kWgSmem, stream>>>(
+        da, xb, static_cast<__nv_bfloat16*>(a.dW1), d_ff, d, fw.exp_base, fw.exp_rows, N);
     colsum(static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N, C_rows,
            static_cast<TA*>(a.db1));
     // dx (kept tokens) += da W1[e], rows to tokens
-    grouped_gemm_mma_kernel<false><<<dim3(mt(d), row_tiles, 1), blk, 0, stream>>>(
-        da, static_cast<const __nv_bfloat16*>(a.W1), nullptr, 0, d, d_ff, fw.exp_base,
+    grouped_gemm_mma_kernel<<<dim3(mt(d), row_tiles, 1), blk, 0, stream>>>(
+        da, static_cast<const __nv_bfloat16*>(a.W1), nullptr, d, d_ff, fw.exp_base,
         fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
     launches += 5;
   } else {

@@ -116,7 +116,8 @@ struct RouterPlan {
   int ksplit;   // logits slices (CTAs of a cluster on the tile / tensor-core paths)
 };
 // tensor != 0: the tensor-core router (bf16 layers); else the FFMA kernels.
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk = 1);
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk = 1,
+                       int force_wide = 0);
 
 size_t workspace_layout(const Shape& s, bool host_io, uintptr_t base, Workspace* ws);
 

@@ -1241,9 +1241,12 @@ cudaError_t launch_softmax_t(const Shape& s, const Workspace& ws, const float* b
 
 }  // namespace
 
-RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk) {
+RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk, int force_wide) {
   RouterPlan p;
-  if (tensor && N <= kFusedRouterMaxN && topk == 1) {
+  // force_wide (tensor cores only): the logits GEMM and a separate softmax at any
+  // N, for a jittered input, which only that logits kernel takes as bf16 pieces
+  if (!tensor) force_wide = 0;
+  if (tensor && N <= kFusedRouterMaxN && topk == 1 && !force_wide) {
     // tensor cores: 128-token tiles; K split over 2 or 4 CTAs of a cluster while
     // the tiles alone would leave most SMs idle (and each CTA keeps >= 2 k-blocks)
     const int64_t tiles = (T + 127) / 128;
@@ -1257,7 +1260,7 @@ RouterPlan router_plan(int64_t T, int64_t d, int64_t N, int tensor, int topk) {
     p.tpb = (int)(128 / S);
     return p;
   }
-  if (N <= kFusedRouterMaxN && topk == 1) {
+  if (N <= kFusedRouterMaxN && topk == 1 && !force_wide) {
     // one fused kernel; big tiles once there are enough of them to fill the GPU
     const int64_t bm = N <= 64 ? 256 : 128;
     const int64_t tiles = (T + bm - 1) / bm;

@@ -189,12 +189,10 @@ static swl_status make_shape(int64_t T, int64_t d, int64_t d_ff, int64_t N, int 
   if (glu && N * 2 * d_ff > INT32_MAX) return SWL_ERR_UNSUPPORTED;   // TMA row coordinates
   // the tensor-core router serves bf16 layers unless the FFMA router was chosen;
   // a jittered router input (x * noise, fp32) takes the tensor-core logits of
-  // the wide path (N > 128 or top-2) with x * noise split into bf16 pieces, and
-  // the FFMA router otherwise
-  const bool wide = N > kFusedRouterMaxN || topk == 2;
-  const bool tensor_router = dtype == SWL_BF16 && (!jitter || wide) &&
-                             g_router_mode.load() == SWL_ROUTER_TENSOR;
-  const RouterPlan rp = router_plan(T, d, N, tensor_router ? 1 : 0, topk);
+  // the wide path at any N, with x * noise split into bf16 pieces
+  const bool tensor_router = dtype == SWL_BF16 && g_router_mode.load() == SWL_ROUTER_TENSOR;
+  const RouterPlan rp =
+      router_plan(T, d, N, tensor_router ? 1 : 0, topk, jitter && tensor_router ? 1 : 0);
   s->router_path = rp.path;
   s->xsplit = jitter && rp.path == kRouterTCWide ? 1 : 0;
   s->kslice = rp.kslice;

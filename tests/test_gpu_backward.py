@@ -47,6 +47,8 @@ _CASES = [
     ("ragged_f32_bias", synth.LayerSpec("bwd_ragged", 333, 40, 72, 5, 0.8, "f32", bias_std=0.05,
                                         router_bias="zipf0.3")),
     ("wide_bf16", synth.LayerSpec("bwd_wide", 500, 128, 64, 200, 2.0, "bf16", bias_std=0.05)),
+    # d not a multiple of 4: the router logits tiles load element by element
+    ("odd_d_f32", synth.LayerSpec("bwd_odd_d", 150, 19, 23, 3, 1.0, "f32", bias_std=0.05)),
     ("base", synth.WORKLOADS["base_T4096_d768_N64"]),
 ]
 
