@@ -20,6 +20,8 @@
 //   bwd_gate_kernel     per token: dg (fp32), the packed row du = g dout, f counts
 //   bwd_logits_kernel   z = x W_r^T + b_r (fp32, [T, N]): tiles of 128 tokens x 64 experts
 //   bwd_dz_kernel       per token (a warp): softmax of z, dz in place of z
+//   bwd_dwr_kernel      dW_r partials over row chunks (64 experts x 128 columns tiles)
+//   bwd_dx_router_kernel dx = (experts' part) + dz W_r, rounded once to the activation type
 //   grouped_gemm_kernel SIMT tiles with fp32 accumulation over packed row
 //                       groups (one group per expert), two forms:
 //                       WGRAD  C[g] = sum over the group's rows of A_r^T B_r
@@ -237,7 +239,7 @@ grouped_gemm_kernel(const TAin* __restrict__ A, const TBin* __restrict__ B, TC* 
 // row at once; else element by element.
 constexpr int kLT = 128, kLN = 64, kLK = 16;
 template <typename TA>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 bwd_logits_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
                   const float* __restrict__ b_r, int T, int d, int N, int vec,
                   float* __restrict__ z) {
@@ -314,6 +316,169 @@ bwd_logits_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tn * 4 + j;
       if (n < N) z[static_cast<size_t>(t) * N + n] = acc[i][j] + (b_r ? b_r[n] : 0.f);
+    }
+  }
+}
+
+// dW_r partial products over row chunks: part[s][n][c] = sum over the rows r of
+// chunk s (rows [s K, s K + K) of T) of dz[r][n] x[r][c], fp32; 64 experts x 128
+// columns per CTA, 256 threads with 4 experts x 8 columns each, rows in steps of
+// 16 through shared memory (both tiles row-major as read).  vec: N % 4 == 0 and
+// d % 4 == 0 with 16-byte aligned dz and 4-element aligned x.  The chunks are
+// then added in order by colsum_finish_kernel.
+constexpr int kRN = 64, kRC = 128;
+template <typename TA>
+__global__ void __launch_bounds__(256, 2)
+bwd_dwr_kernel(const float* __restrict__ dz, const TA* __restrict__ x, int T, int d, int N,
+               int K, int vec, float* __restrict__ part) {
+  __shared__ __align__(16) float As[kLK][kRN + 4];   // [row][expert]
+  __shared__ __align__(16) float Bs[kLK][kRC + 4];   // [row][column]
+  const int tid = threadIdx.x;
+  const int tn = tid % 16, tc = tid / 16;           // experts 4 tn.., columns 8 tc..
+  const int c0 = blockIdx.x * kRC, n0 = blockIdx.y * kRN, sidx = blockIdx.z;
+  const int r0 = sidx * K, r1 = min(T, r0 + K);
+  float acc[4][8] = {};
+  for (int k0 = r0; k0 < r1; k0 += kLK) {
+    if (vec) {
+      {                                              // 16 rows x 16 quads of dz
+        const int kr = tid / 16, nq = (tid % 16) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k0 + kr < r1 && n0 + nq < N)
+          v = *reinterpret_cast<const float4*>(dz + static_cast<size_t>(k0 + kr) * N + n0 + nq);
+        *reinterpret_cast<float4*>(&As[kr][nq]) = v;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {                  // 16 rows x 32 quads of x
+        const int q = tid + h * 256, kr = q / 32, cq = (q % 32) * 4;
+        float xa[4] = {0.f, 0.f, 0.f, 0.f};
+        if (k0 + kr < r1 && c0 + cq < d) {
+          const TA* src = x + static_cast<size_t>(k0 + kr) * d + c0 + cq;
+          if constexpr (std::is_same<TA, float>::value) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            xa[0] = v.x; xa[1] = v.y; xa[2] = v.z; xa[3] = v.w;
+          } else {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+            xa[0] = __low2float(lo); xa[1] = __high2float(lo);
+            xa[2] = __low2float(hi); xa[3] = __high2float(hi);
+          }
+        }
+        *reinterpret_cast<float4*>(&Bs[kr][cq]) = make_float4(xa[0], xa[1], xa[2], xa[3]);
+      }
+    } else {
+      for (int i = tid; i < kLK * kRN; i += 256) {
+        const int kr = i / kRN, n = i % kRN;
+        As[kr][n] = (k0 + kr < r1 && n0 + n < N) ? dz[static_cast<size_t>(k0 + kr) * N + n0 + n]
+                                                 : 0.f;
+      }
+      for (int i = tid; i < kLK * kRC; i += 256) {
+        const int kr = i / kRC, c = i % kRC;
+        Bs[kr][c] = (k0 + kr < r1 && c0 + c < d) ? ld(x + static_cast<size_t>(k0 + kr) * d + c0 + c)
+                                                 : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kLK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][tn * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tc * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tc * 8 + 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[j][i] = fmaf(av[j], bv[i], acc[j][i]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int n = n0 + tn * 4 + j;
+    if (n >= N) continue;
+    float* dst = part + (static_cast<size_t>(sidx) * N + n) * d;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = c0 + tc * 8 + i;
+      if (c < d) dst[c] = acc[j][i];
+    }
+  }
+}
+
+// dx = dx_acc + dz W_r, rounded once to the activation type: 128 tokens x 64
+// columns per CTA, 256 threads with 8 tokens x 4 columns each, K = N in steps
+// of 16 (dz k-major in shared memory, W_r rows as read).  vec: N % 4 == 0 and d %
+// 4 == 0 with 16-byte aligned dz, W_r and dx_acc.
+template <typename TA>
+__global__ void __launch_bounds__(256, 2)
+bwd_dx_router_kernel(const float* __restrict__ dz, const float* __restrict__ W_r,
+                     const float* __restrict__ dx_acc, int T, int d, int N, int vec,
+                     TA* __restrict__ dx) {
+  __shared__ __align__(16) float As[kLK][kLT + 4];   // [k][token]
+  __shared__ __align__(16) float Bs[kLK][kLN + 4];   // [k][column]
+  const int tid = threadIdx.x;
+  const int tn = tid % 16, tt = tid / 16;           // columns 4 tn.., tokens 8 tt..
+  const int c0 = blockIdx.x * kLN, t0 = blockIdx.y * kLT;
+  float acc[8][4] = {};
+  for (int k0 = 0; k0 < N; k0 += kLK) {
+    if (vec) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {                  // 128 tokens x 4 quads of dz
+        const int q = tid + h * 256, r = q / 4, kq = (q % 4) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t0 + r < T && k0 + kq < N)
+          v = *reinterpret_cast<const float4*>(dz + static_cast<size_t>(t0 + r) * N + k0 + kq);
+        As[kq][r] = v.x;
+        As[kq + 1][r] = v.y;
+        As[kq + 2][r] = v.z;
+        As[kq + 3][r] = v.w;
+      }
+      {                                              // 16 rows x 16 quads of W_r
+        const int kr = tid / 16, cq = (tid % 16) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k0 + kr < N && c0 + cq < d)
+          v = *reinterpret_cast<const float4*>(W_r + static_cast<size_t>(k0 + kr) * d + c0 + cq);
+        *reinterpret_cast<float4*>(&Bs[kr][cq]) = v;
+      }
+    } else {
+      for (int i = tid; i < kLK * kLT; i += 256) {
+        const int kk = i % kLK, r = i / kLK;
+        As[kk][r] = (t0 + r < T && k0 + kk < N) ? dz[static_cast<size_t>(t0 + r) * N + k0 + kk]
+                                                : 0.f;
+      }
+      for (int i = tid; i < kLK * kLN; i += 256) {
+        const int kr = i / kLN, c = i % kLN;
+        Bs[kr][c] = (k0 + kr < N && c0 + c < d) ? W_r[static_cast<size_t>(k0 + kr) * d + c0 + c]
+                                                : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kLK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][tt * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][tt * 8 + 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tn * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + tt * 8 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tn * 4 + j;
+      if (c < d) {
+        const size_t o = static_cast<size_t>(t) * d + c;
+        dx[o] = cvt<TA>(dx_acc[o] + acc[i][j]);
+      }
     }
   }
 }
@@ -781,14 +946,6 @@ __global__ void bwd_tile_prefix_kernel(const int* __restrict__ rows, int N, int 
 }
 
 template <typename TA>
-__global__ void __launch_bounds__(256)
-dx_finish_kernel(const float* __restrict__ acc, TA* __restrict__ dx, size_t n) {
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    dx[i] = cvt<TA>(acc[i]);
-}
-
-template <typename TA>
 cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspace& bw,
                            const BwdArgs& a, cudaStream_t stream) {
   const int T = static_cast<int>(s.T), d = static_cast<int>(s.d), d_ff = static_cast<int>(s.d_ff);
@@ -909,9 +1066,12 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
   {
     const int chunk = router_chunk_rows(T, N, d);
     const int S = (T + chunk - 1) / chunk;
-    grouped_gemm_kernel<float, TA, float, true><<<dim3(tiles(d), tiles(N), S), blk, 0, stream>>>(
-        bw.dz, x, bw.part, N, d, chunk, nullptr, nullptr, T, nullptr, S, 0, nullptr, nullptr,
-        nullptr);
+    const int vec = (N % 4 == 0 && d % 4 == 0 && (reinterpret_cast<uintptr_t>(bw.dz) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(x) & (4 * sizeof(TA) - 1)) == 0)
+                        ? 1
+                        : 0;
+    bwd_dwr_kernel<TA><<<dim3((d + kRC - 1) / kRC, (N + kRN - 1) / kRN, S), blk, 0, stream>>>(
+        bw.dz, x, T, d, N, chunk, vec, bw.part);
     const size_t n = static_cast<size_t>(N) * d;
     size_t nb = (n + 255) / 256;
     if (nb > 8 * 148) nb = 8 * 148;
@@ -920,15 +1080,16 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
     launches += 2;
   }
   if (a.db_r) colsum(static_cast<const float*>(bw.dz), N, nullptr, nullptr, T, 1, T, a.db_r);
-  grouped_gemm_kernel<float, float, float, false><<<dim3(tiles(d), tiles(T), 1), blk, 0, stream>>>(
-      bw.dz, a.W_r, static_cast<float*>(nullptr), 0, d, N, nullptr, nullptr, T, nullptr, 1, 2,
-      nullptr, nullptr, bw.dx_acc);
-  const size_t n = static_cast<size_t>(T) * d;
-  size_t blocks = (n + 255) / 256;
-  if (blocks > 8 * 148) blocks = 8 * 148;
-  dx_finish_kernel<TA><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      bw.dx_acc, static_cast<TA*>(a.dx), n);
-  launches += 2;
+  // dx = dx_acc (the experts' part) + dz W_r, rounded once
+  {
+    const int vec = (N % 4 == 0 && d % 4 == 0 && (reinterpret_cast<uintptr_t>(bw.dz) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.W_r) & 15) == 0)
+                        ? 1
+                        : 0;
+    bwd_dx_router_kernel<TA><<<dim3((d + kLN - 1) / kLN, (T + kLT - 1) / kLT), blk, 0, stream>>>(
+        bw.dz, a.W_r, bw.dx_acc, T, d, N, vec, static_cast<TA*>(a.dx));
+    ++launches;
+  }
   count_launch(launches);
   return cudaGetLastError();
 }
