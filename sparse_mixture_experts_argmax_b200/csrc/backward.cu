@@ -534,7 +534,9 @@ bwd_dz_kernel(const int* __restrict__ expert_idx, const float* __restrict__ gate
 constexpr int kMT = 128, kMK = 32, kMPad = 8;
 constexpr int kMStride = kMT + kMPad;      // [k][128] tiles: row stride in elements
 constexpr int kMStrideK = kMK + kMPad;     // [128][k] tile: row stride in elements
-constexpr int kMStage = kMK * kMStride > kMT * kMStrideK ? kMK * kMStride : kMT * kMStrideK;
+constexpr int kDgStages = 4;               // cp.async ring depth of grouped_gemm_mma_kernel
+constexpr size_t kDgSmem =
+    static_cast<size_t>(kDgStages) * (kMT * kMStrideK + kMK * kMStride) * 2 + 128;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -576,8 +578,11 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
                         const int* __restrict__ tile_prefix, int groups, int epi,
                         const __nv_bfloat16* __restrict__ mask, const int* __restrict__ dst_row,
                         float* __restrict__ acc_out) {
-  __shared__ __align__(128) __nv_bfloat16 sA[2][kMStage];
-  __shared__ __align__(128) __nv_bfloat16 sB[2][kMK * kMStride];
+  extern __shared__ uint8_t dg_raw[];
+  __nv_bfloat16* smem = reinterpret_cast<__nv_bfloat16*>(
+      (reinterpret_cast<uintptr_t>(dg_raw) + 127) & ~static_cast<uintptr_t>(127));
+  __nv_bfloat16* sA = smem;                                // [kDgStages][kMT][kMStrideK]
+  __nv_bfloat16* sB = sA + kDgStages * kMT * kMStrideK;    // [kDgStages][kMK][kMStride]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp >> 2, wn = warp & 3;        // 2 x 4 warps of 64 x 32 outputs
   const int n0 = blockIdx.x * kMT;
@@ -611,14 +616,13 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
       const int c = tid + h * 256;
       const int r = c >> 2, kc = (c & 3) * 8;    // A[r0 + r][k0 + kc ...]
       const bool ok = r < nr && k0 + kc < K;
-      cp_async16(&sA[s][r * kMStrideK + kc],
+      cp_async16(&sA[(s * kMT + r) * kMStrideK + kc],
                  ok ? A + static_cast<size_t>(r0 + r) * K + k0 + kc : A, ok);
       const int k = c >> 4, nc = (c & 15) * 8;    // W[g][k0 + k][n0 + nc ...]
       const bool okb = k0 + k < K && n0 + nc < Q;
-      cp_async16(&sB[s][k * kMStride + nc],
+      cp_async16(&sB[(s * kMK + k) * kMStride + nc],
                  okb ? W + static_cast<size_t>(k0 + k) * Q + n0 + nc : B, okb);
     }
-    cp_async_commit();
   };
 
   float acc[4][4][4];
@@ -629,17 +633,26 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
 
+  // kDgStages-deep ring: K steps kt+1 .. kt+kDgStages-1 are in flight while kt
+  // is computed; one commit group per K step (empty past the end), so that
+  // waiting until kDgStages-2 groups remain leaves step kt landed
   const int nk = (K + kMK - 1) / kMK;
-  load(0, 0);
+#pragma unroll
+  for (int s = 0; s < kDgStages - 1; ++s) {
+    if (s < nk) load(s, s * kMK);
+    cp_async_commit();
+  }
   for (int kt = 0; kt < nk; ++kt) {
-    const int s = kt & 1;
-    if (kt + 1 < nk) {
-      load(s ^ 1, (kt + 1) * kMK);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+    const int s = kt % kDgStages;
+    cp_async_wait<kDgStages - 2>();
+    __syncthreads();   // step kt landed for every thread; step kt-1's stage is free
+    {
+      const int kn = kt + kDgStages - 1;
+      if (kn < nk) load(kn % kDgStages, kn * kMK);
+      cp_async_commit();
     }
-    __syncthreads();
+    const __nv_bfloat16* a_s = sA + s * kMT * kMStrideK;
+    const __nv_bfloat16* b_s = sB + s * kMK * kMStride;
 #pragma unroll
     for (int kk = 0; kk < kMK; kk += 16) {
       uint32_t af[4][4], bf[4][2];
@@ -647,13 +660,13 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int mb = wm * 64 + i * 16;   // staged [r][k]
-        ldsm_x4(af[i], &sA[s][(mb + (lane & 15)) * kMStrideK + kk + (lane >> 4) * 8]);
+        ldsm_x4(af[i], &a_s[(mb + (lane & 15)) * kMStrideK + kk + (lane >> 4) * 8]);
       }
 #pragma unroll
       for (int j2 = 0; j2 < 2; ++j2) {   // two n-fragments of 8 per ldmatrix
         const int nb = wn * 32 + j2 * 16;
         uint32_t t4[4];
-        ldsm_x4_t(t4, &sB[s][(kk + rr + (jm & 1) * 8) * kMStride + nb + (jm >> 1) * 8]);
+        ldsm_x4_t(t4, &b_s[(kk + rr + (jm & 1) * 8) * kMStride + nb + (jm >> 1) * 8]);
         bf[2 * j2][0] = t4[0];
         bf[2 * j2][1] = t4[1];
         bf[2 * j2 + 1][0] = t4[2];
@@ -664,8 +677,8 @@ grouped_gemm_mma_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16
 #pragma unroll
         for (int j = 0; j < 4; ++j) mma_bf16(acc[i][j], af[i], bf[j][0], bf[j][1]);
     }
-    __syncthreads();
   }
+  cp_async_wait<0>();   // the empty trailing groups, before the CTA exits
 
   // epilogue: accumulator (i, j, c) -> row wm*64 + i*16 + lane/4 (+8 for c >= 2),
   // column wn*32 + j*8 + (lane%4)*2 (+1 for odd c)
@@ -1020,7 +1033,11 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
     // da = (du W2[e]) * [h > 0]
     bwd_tile_prefix_kernel<<<1, 32, 0, stream>>>(fw.exp_rows, N, kMT, bw.tile_prefix);
     const unsigned row_tiles = static_cast<unsigned>((T + kMT - 1) / kMT + N);
-    grouped_gemm_mma_kernel<<<dim3(mt(d_ff), row_tiles, 1), blk, 0, stream>>>(
+    if ((e = cudaFuncSetAttribute(grouped_gemm_mma_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kDgSmem))) != cudaSuccess)
+      return e;
+    grouped_gemm_mma_kernel<<<dim3(mt(d_ff), row_tiles, 1), blk, kDgSmem, stream>>>(
         du, static_cast<const __nv_bfloat16*>(a.W2), da, d_ff, d, fw.exp_base, fw.exp_rows, 0,
         bw.tile_prefix, N, 1, hb, nullptr, nullptr);
     // dW1[e] = da^T x, db1[e] = sum da
@@ -1029,7 +1046,7 @@ cudaError_t run_backward_t(const Shape& s, const Workspace& fw, const BwdWorkspa
     colsum(static_cast<const TA*>(bw.da), d_ff, fw.exp_base, fw.exp_rows, 0, N, C_rows,
            static_cast<TA*>(a.db1));
     // dx (kept tokens) += da W1[e], rows to tokens
-    grouped_gemm_mma_kernel<<<dim3(mt(d), row_tiles, 1), blk, 0, stream>>>(
+    grouped_gemm_mma_kernel<<<dim3(mt(d), row_tiles, 1), blk, kDgSmem, stream>>>(
         da, static_cast<const __nv_bfloat16*>(a.W1), nullptr, d, d_ff, fw.exp_base,
         fw.exp_rows, 0, bw.tile_prefix, N, 2, nullptr, fw.slot_token, bw.dx_acc);
     launches += 5;
