@@ -323,6 +323,9 @@ _VARIANT_SHAPES = [
     ("two_accumulators", 900, 64, 64, 4, 1.0, "bf16"),
     # GEMM2 split over K on the first experts, unsplit tiles on the rest
     ("gemm2_split_mixed", 12288, 768, 4096, 8, 1.0, "bf16"),
+    # d_ff = 4160: K chunks of 17 k-blocks (1088 features), so GEMM1 feature tiles
+    # 8 and 25 straddle two chunks and count in both
+    ("gemm2_split_straddle", 12288, 768, 4160, 8, 1.0, "bf16"),
     # streaming softmax: a warp per row at full width (N = 1024), a warp pair per row
     # with a ragged second half (N = 1500); token blocks of 45 and 37 tokens
     ("stream_full_warp_row", 6600, 128, 64, 1024, 2.0, "bf16"),
