@@ -238,75 +238,106 @@ grouped_gemm_kernel(const TAin* __restrict__ A, const TBin* __restrict__ B, TC* 
 // rows, then each thread loads 4 consecutive k of a token row and of an expert
 // row at once; else element by element.
 constexpr int kLT = 128, kLN = 64, kLK = 16;
+
+// A thread's 4 consecutive elements of a row at src (zeros when !ok), as fp32.
+template <typename T>
+__device__ __forceinline__ float4 ld4(const T* src, bool ok) {
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!ok) return r;
+  if constexpr (std::is_same<T, float>::value) {
+    r = *reinterpret_cast<const float4*>(src);
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2*>(src);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+    r = make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+  }
+  return r;
+}
+
+// The three router-gradient products below share one scheme: a 128 x 64 (or 64
+// x 128) output tile per CTA, 8 x 4 (or 4 x 8) outputs per thread, K in steps
+// of 16.  With vec (every row 4-element aligned), two shared-memory buffers: a
+// thread's loads of step k+1 are issued into registers before step k is
+// computed and stored to the other buffer after it, so one barrier per step
+// separates the steps and the loads overlap the FMAs; otherwise one buffer with
+// element-wise loads.
+
+// Router logits for the backward, z = x W_r^T + b_r in fp32 ([T, N], written to
+// dz and turned into dz by bwd_dz_kernel): 128 tokens x 64 experts per CTA,
+// 256 threads with 8 tokens x 4 experts each (both tiles k-major in shared
+// memory, read as 16-byte vectors), so W_r is read once per token tile.  vec:
+// d % 4 == 0 with 16-byte aligned W_r and 4-element aligned x rows.
 template <typename TA>
 __global__ void __launch_bounds__(256, 2)
 bwd_logits_kernel(const TA* __restrict__ x, const float* __restrict__ W_r,
                   const float* __restrict__ b_r, int T, int d, int N, int vec,
                   float* __restrict__ z) {
-  __shared__ __align__(16) float As[kLK][kLT + 4];   // [k][token]
-  __shared__ __align__(16) float Bs[kLK][kLN + 4];   // [k][expert]
+  __shared__ __align__(16) float As[2][kLK][kLT + 4];   // [buffer][k][token]
+  __shared__ __align__(16) float Bs[2][kLK][kLN + 4];   // [buffer][k][expert]
   const int tid = threadIdx.x;
   const int tn = tid % 16, tt = tid / 16;           // experts 4 tn.., tokens 8 tt..
   const int n0 = blockIdx.x * kLN, t0 = blockIdx.y * kLT;
   float acc[8][4] = {};
-  for (int k0 = 0; k0 < d; k0 += kLK) {
-    if (vec) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {                  // 128 rows x 4 quads of x
-        const int q = tid + h * 256, r = q / 4, kq = (q % 4) * 4;
-        float xa[4] = {0.f, 0.f, 0.f, 0.f};
-        if (t0 + r < T && k0 + kq < d) {
-          const TA* src = x + static_cast<size_t>(t0 + r) * d + k0 + kq;
-          if constexpr (std::is_same<TA, float>::value) {
-            const float4 v = *reinterpret_cast<const float4*>(src);
-            xa[0] = v.x; xa[1] = v.y; xa[2] = v.z; xa[3] = v.w;
-          } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(src);
-            const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-            xa[0] = __low2float(lo); xa[1] = __high2float(lo);
-            xa[2] = __low2float(hi); xa[3] = __high2float(hi);
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) As[kq + c][r] = xa[c];
-      }
-      {                                              // 64 rows x 4 quads of W_r
-        const int r = tid / 4, kq = (tid % 4) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n0 + r < N && k0 + kq < d)
-          v = *reinterpret_cast<const float4*>(W_r + static_cast<size_t>(n0 + r) * d + k0 + kq);
-        Bs[kq][r] = v.x;
-        Bs[kq + 1][r] = v.y;
-        Bs[kq + 2][r] = v.z;
-        Bs[kq + 3][r] = v.w;
-      }
-    } else {
-      for (int i = tid; i < kLK * kLT; i += 256) {
-        const int kk = i % kLK, r = i / kLK;
-        As[kk][r] = (t0 + r < T && k0 + kk < d) ? ld(x + static_cast<size_t>(t0 + r) * d + k0 + kk)
-                                                : 0.f;
-      }
-      for (int i = tid; i < kLK * kLN; i += 256) {
-        const int kk = i % kLK, r = i / kLK;
-        Bs[kk][r] = (n0 + r < N && k0 + kk < d) ? W_r[static_cast<size_t>(n0 + r) * d + k0 + kk]
-                                                : 0.f;
-      }
-    }
-    __syncthreads();
+  auto compute = [&](int b) {
 #pragma unroll
     for (int kk = 0; kk < kLK; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][tt * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][tt * 8 + 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tn * 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[b][kk][tt * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[b][kk][tt * 8 + 4]);
+      const float4 w = *reinterpret_cast<const float4*>(&Bs[b][kk][tn * 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bb[4] = {b.x, b.y, b.z, b.w};
+      const float bb[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
     }
+  };
+  if (vec) {
+    // this thread: x rows r = q / 4 (q = tid, tid + 256), W_r row tid / 4, at k quad kq
+    const int kq = (tid % 4) * 4, rx0 = tid / 4, rx1 = rx0 + 64, rw = tid / 4;
+    float4 xa0, xa1, wb;
+    auto fetch = [&](int k0) {
+      const bool kok = k0 + kq < d;
+      xa0 = ld4(x + static_cast<size_t>(t0 + rx0) * d + k0 + kq, kok && t0 + rx0 < T);
+      xa1 = ld4(x + static_cast<size_t>(t0 + rx1) * d + k0 + kq, kok && t0 + rx1 < T);
+      wb = ld4(W_r + static_cast<size_t>(n0 + rw) * d + k0 + kq, kok && n0 + rw < N);
+    };
+    auto stash = [&](int b) {
+      As[b][kq][rx0] = xa0.x; As[b][kq + 1][rx0] = xa0.y;
+      As[b][kq + 2][rx0] = xa0.z; As[b][kq + 3][rx0] = xa0.w;
+      As[b][kq][rx1] = xa1.x; As[b][kq + 1][rx1] = xa1.y;
+      As[b][kq + 2][rx1] = xa1.z; As[b][kq + 3][rx1] = xa1.w;
+      Bs[b][kq][rw] = wb.x; Bs[b][kq + 1][rw] = wb.y;
+      Bs[b][kq + 2][rw] = wb.z; Bs[b][kq + 3][rw] = wb.w;
+    };
+    fetch(0);
+    stash(0);
     __syncthreads();
+    int b = 0;
+    for (int k0 = 0; k0 < d; k0 += kLK, b ^= 1) {
+      const bool more = k0 + kLK < d;
+      if (more) fetch(k0 + kLK);
+      compute(b);
+      if (more) stash(b ^ 1);
+      __syncthreads();
+    }
+  } else {
+    for (int k0 = 0; k0 < d; k0 += kLK) {
+      for (int i = tid; i < kLK * kLT; i += 256) {
+        const int kk = i % kLK, r = i / kLK;
+        As[0][kk][r] = (t0 + r < T && k0 + kk < d) ? ld(x + static_cast<size_t>(t0 + r) * d + k0 + kk)
+                                                   : 0.f;
+      }
+      for (int i = tid; i < kLK * kLN; i += 256) {
+        const int kk = i % kLK, r = i / kLK;
+        Bs[0][kk][r] = (n0 + r < N && k0 + kk < d) ? W_r[static_cast<size_t>(n0 + r) * d + k0 + kk]
+                                                   : 0.f;
+      }
+      __syncthreads();
+      compute(0);
+      __syncthreads();
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -331,59 +362,19 @@ template <typename TA>
 __global__ void __launch_bounds__(256, 2)
 bwd_dwr_kernel(const float* __restrict__ dz, const TA* __restrict__ x, int T, int d, int N,
                int K, int vec, float* __restrict__ part) {
-  __shared__ __align__(16) float As[kLK][kRN + 4];   // [row][expert]
-  __shared__ __align__(16) float Bs[kLK][kRC + 4];   // [row][column]
+  __shared__ __align__(16) float As[2][kLK][kRN + 4];   // [buffer][row][expert]
+  __shared__ __align__(16) float Bs[2][kLK][kRC + 4];   // [buffer][row][column]
   const int tid = threadIdx.x;
   const int tn = tid % 16, tc = tid / 16;           // experts 4 tn.., columns 8 tc..
   const int c0 = blockIdx.x * kRC, n0 = blockIdx.y * kRN, sidx = blockIdx.z;
   const int r0 = sidx * K, r1 = min(T, r0 + K);
   float acc[4][8] = {};
-  for (int k0 = r0; k0 < r1; k0 += kLK) {
-    if (vec) {
-      {                                              // 16 rows x 16 quads of dz
-        const int kr = tid / 16, nq = (tid % 16) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (k0 + kr < r1 && n0 + nq < N)
-          v = *reinterpret_cast<const float4*>(dz + static_cast<size_t>(k0 + kr) * N + n0 + nq);
-        *reinterpret_cast<float4*>(&As[kr][nq]) = v;
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {                  // 16 rows x 32 quads of x
-        const int q = tid + h * 256, kr = q / 32, cq = (q % 32) * 4;
-        float xa[4] = {0.f, 0.f, 0.f, 0.f};
-        if (k0 + kr < r1 && c0 + cq < d) {
-          const TA* src = x + static_cast<size_t>(k0 + kr) * d + c0 + cq;
-          if constexpr (std::is_same<TA, float>::value) {
-            const float4 v = *reinterpret_cast<const float4*>(src);
-            xa[0] = v.x; xa[1] = v.y; xa[2] = v.z; xa[3] = v.w;
-          } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(src);
-            const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-            xa[0] = __low2float(lo); xa[1] = __high2float(lo);
-            xa[2] = __low2float(hi); xa[3] = __high2float(hi);
-          }
-        }
-        *reinterpret_cast<float4*>(&Bs[kr][cq]) = make_float4(xa[0], xa[1], xa[2], xa[3]);
-      }
-    } else {
-      for (int i = tid; i < kLK * kRN; i += 256) {
-        const int kr = i / kRN, n = i % kRN;
-        As[kr][n] = (k0 + kr < r1 && n0 + n < N) ? dz[static_cast<size_t>(k0 + kr) * N + n0 + n]
-                                                 : 0.f;
-      }
-      for (int i = tid; i < kLK * kRC; i += 256) {
-        const int kr = i / kRC, c = i % kRC;
-        Bs[kr][c] = (k0 + kr < r1 && c0 + c < d) ? ld(x + static_cast<size_t>(k0 + kr) * d + c0 + c)
-                                                 : 0.f;
-      }
-    }
-    __syncthreads();
+  auto compute = [&](int b) {
 #pragma unroll
     for (int kk = 0; kk < kLK; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[kk][tn * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tc * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tc * 8 + 4]);
+      const float4 a = *reinterpret_cast<const float4*>(&As[b][kk][tn * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[b][kk][tc * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[b][kk][tc * 8 + 4]);
       const float av[4] = {a.x, a.y, a.z, a.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -391,7 +382,51 @@ bwd_dwr_kernel(const float* __restrict__ dz, const TA* __restrict__ x, int T, in
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[j][i] = fmaf(av[j], bv[i], acc[j][i]);
     }
+  };
+  if (vec) {
+    // this thread: dz row tid / 16 at expert quad nq; x rows q / 32 (q = tid, tid + 256)
+    // at column quad cq
+    const int kr = tid / 16, nq = (tid % 16) * 4;
+    const int xr0 = tid / 32, xr1 = xr0 + 8, cq = (tid % 32) * 4;
+    float4 av, xb0, xb1;
+    auto fetch = [&](int k0) {
+      av = ld4(dz + static_cast<size_t>(k0 + kr) * N + n0 + nq, k0 + kr < r1 && n0 + nq < N);
+      const bool cok = c0 + cq < d;
+      xb0 = ld4(x + static_cast<size_t>(k0 + xr0) * d + c0 + cq, cok && k0 + xr0 < r1);
+      xb1 = ld4(x + static_cast<size_t>(k0 + xr1) * d + c0 + cq, cok && k0 + xr1 < r1);
+    };
+    auto stash = [&](int b) {
+      *reinterpret_cast<float4*>(&As[b][kr][nq]) = av;
+      *reinterpret_cast<float4*>(&Bs[b][xr0][cq]) = xb0;
+      *reinterpret_cast<float4*>(&Bs[b][xr1][cq]) = xb1;
+    };
+    fetch(r0);
+    stash(0);
     __syncthreads();
+    int b = 0;
+    for (int k0 = r0; k0 < r1; k0 += kLK, b ^= 1) {
+      const bool more = k0 + kLK < r1;
+      if (more) fetch(k0 + kLK);
+      compute(b);
+      if (more) stash(b ^ 1);
+      __syncthreads();
+    }
+  } else {
+    for (int k0 = r0; k0 < r1; k0 += kLK) {
+      for (int i = tid; i < kLK * kRN; i += 256) {
+        const int kr = i / kRN, n = i % kRN;
+        As[0][kr][n] = (k0 + kr < r1 && n0 + n < N) ? dz[static_cast<size_t>(k0 + kr) * N + n0 + n]
+                                                    : 0.f;
+      }
+      for (int i = tid; i < kLK * kRC; i += 256) {
+        const int kr = i / kRC, c = i % kRC;
+        Bs[0][kr][c] = (k0 + kr < r1 && c0 + c < d) ? ld(x + static_cast<size_t>(k0 + kr) * d + c0 + c)
+                                                    : 0.f;
+      }
+      __syncthreads();
+      compute(0);
+      __syncthreads();
+    }
   }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -415,58 +450,72 @@ __global__ void __launch_bounds__(256, 2)
 bwd_dx_router_kernel(const float* __restrict__ dz, const float* __restrict__ W_r,
                      const float* __restrict__ dx_acc, int T, int d, int N, int vec,
                      TA* __restrict__ dx) {
-  __shared__ __align__(16) float As[kLK][kLT + 4];   // [k][token]
-  __shared__ __align__(16) float Bs[kLK][kLN + 4];   // [k][column]
+  __shared__ __align__(16) float As[2][kLK][kLT + 4];   // [buffer][k][token]
+  __shared__ __align__(16) float Bs[2][kLK][kLN + 4];   // [buffer][k][column]
   const int tid = threadIdx.x;
   const int tn = tid % 16, tt = tid / 16;           // columns 4 tn.., tokens 8 tt..
   const int c0 = blockIdx.x * kLN, t0 = blockIdx.y * kLT;
   float acc[8][4] = {};
-  for (int k0 = 0; k0 < N; k0 += kLK) {
-    if (vec) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {                  // 128 tokens x 4 quads of dz
-        const int q = tid + h * 256, r = q / 4, kq = (q % 4) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t0 + r < T && k0 + kq < N)
-          v = *reinterpret_cast<const float4*>(dz + static_cast<size_t>(t0 + r) * N + k0 + kq);
-        As[kq][r] = v.x;
-        As[kq + 1][r] = v.y;
-        As[kq + 2][r] = v.z;
-        As[kq + 3][r] = v.w;
-      }
-      {                                              // 16 rows x 16 quads of W_r
-        const int kr = tid / 16, cq = (tid % 16) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (k0 + kr < N && c0 + cq < d)
-          v = *reinterpret_cast<const float4*>(W_r + static_cast<size_t>(k0 + kr) * d + c0 + cq);
-        *reinterpret_cast<float4*>(&Bs[kr][cq]) = v;
-      }
-    } else {
-      for (int i = tid; i < kLK * kLT; i += 256) {
-        const int kk = i % kLK, r = i / kLK;
-        As[kk][r] = (t0 + r < T && k0 + kk < N) ? dz[static_cast<size_t>(t0 + r) * N + k0 + kk]
-                                                : 0.f;
-      }
-      for (int i = tid; i < kLK * kLN; i += 256) {
-        const int kr = i / kLN, c = i % kLN;
-        Bs[kr][c] = (k0 + kr < N && c0 + c < d) ? W_r[static_cast<size_t>(k0 + kr) * d + c0 + c]
-                                                : 0.f;
-      }
-    }
-    __syncthreads();
+  auto compute = [&](int b) {
 #pragma unroll
     for (int kk = 0; kk < kLK; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][tt * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][tt * 8 + 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tn * 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[b][kk][tt * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[b][kk][tt * 8 + 4]);
+      const float4 w = *reinterpret_cast<const float4*>(&Bs[b][kk][tn * 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bb[4] = {b.x, b.y, b.z, b.w};
+      const float bb[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
     }
+  };
+  if (vec) {
+    // this thread: dz rows q / 4 (q = tid, tid + 256) at k quad kq; W_r row tid / 16
+    // at column quad cq
+    const int kq = (tid % 4) * 4, rz0 = tid / 4, rz1 = rz0 + 64;
+    const int kr = tid / 16, cq = (tid % 16) * 4;
+    float4 za0, za1, wb;
+    auto fetch = [&](int k0) {
+      const bool kok = k0 + kq < N;
+      za0 = ld4(dz + static_cast<size_t>(t0 + rz0) * N + k0 + kq, kok && t0 + rz0 < T);
+      za1 = ld4(dz + static_cast<size_t>(t0 + rz1) * N + k0 + kq, kok && t0 + rz1 < T);
+      wb = ld4(W_r + static_cast<size_t>(k0 + kr) * d + c0 + cq, k0 + kr < N && c0 + cq < d);
+    };
+    auto stash = [&](int b) {
+      As[b][kq][rz0] = za0.x; As[b][kq + 1][rz0] = za0.y;
+      As[b][kq + 2][rz0] = za0.z; As[b][kq + 3][rz0] = za0.w;
+      As[b][kq][rz1] = za1.x; As[b][kq + 1][rz1] = za1.y;
+      As[b][kq + 2][rz1] = za1.z; As[b][kq + 3][rz1] = za1.w;
+      *reinterpret_cast<float4*>(&Bs[b][kr][cq]) = wb;
+    };
+    fetch(0);
+    stash(0);
     __syncthreads();
+    int b = 0;
+    for (int k0 = 0; k0 < N; k0 += kLK, b ^= 1) {
+      const bool more = k0 + kLK < N;
+      if (more) fetch(k0 + kLK);
+      compute(b);
+      if (more) stash(b ^ 1);
+      __syncthreads();
+    }
+  } else {
+    for (int k0 = 0; k0 < N; k0 += kLK) {
+      for (int i = tid; i < kLK * kLT; i += 256) {
+        const int kk = i % kLK, r = i / kLK;
+        As[0][kk][r] = (t0 + r < T && k0 + kk < N) ? dz[static_cast<size_t>(t0 + r) * N + k0 + kk]
+                                                   : 0.f;
+      }
+      for (int i = tid; i < kLK * kLN; i += 256) {
+        const int kr = i / kLN, c = i % kLN;
+        Bs[0][kr][c] = (k0 + kr < N && c0 + c < d) ? W_r[static_cast<size_t>(k0 + kr) * d + c0 + c]
+                                                   : 0.f;
+      }
+      __syncthreads();
+      compute(0);
+      __syncthreads();
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
