@@ -220,7 +220,9 @@ swl_status switch_layer_backward(int64_t T, int64_t d, int64_t d_ff, int64_t N, 
  *   router_noise  NULL (inference), or [T, d] fp32 multiplicative noise on the
  *                 router input ("input jitter", Table 11 of the paper-graph
  *                 summary, a training-time exploration): the router sees x * noise
- *                 (fp32, routed with the FFMA router), the experts see x.
+ *                 in fp32 (bf16 layers: split exactly into three bf16 pieces for
+ *                 the tensor-core logits kernel at any N; fp32 layers and
+ *                 SWL_ROUTER_FFMA: the FFMA router), the experts see x.
  * A NULL variant is switch_layer_forward.  The workspace is sized by
  * switch_layer_variant_workspace_size with the same variant (only whether
  * router_noise is NULL matters there).  Invalid fields: SWL_ERR_INVALID_ARG. */
@@ -479,8 +481,9 @@ swl_status switch_layer_set_stall_test(int on);
  * num_sms SMs, under the current router mode, without touching the device
  * (host-only; usable without a GPU).  Writes a NUL-terminated list of
  * comma-separated key=value pairs into the caller's buffer buf of len bytes:
- *   router            tc | tc_wide (tensor-core router, N <= 128 fused / wider
- *                     logits only) | ffma_warpsplit | ffma_tile | ffma_wide
+ *   router            tc | tc_wide (tensor-core router: fused for N <= 128 /
+ *                     logits only for N > 128, top-2 or a jittered input) |
+ *                     ffma_warpsplit | ffma_tile | ffma_wide
  *   ksplit            CTAs per router tile (cluster size) or K slices
  *   router_stages     operand stages per tensor-core router CTA (0: FFMA router)
  *   softmax           fused (in the router, N <= 128) | stream (N > 128, one
